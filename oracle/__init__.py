@@ -1,0 +1,143 @@
+"""fp64 CPU oracle of the Multi-Token Attention forward pass.
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke entry of the package and
+the CPU-baseline leg of the benchmark are the only callers.  The CUDA library
+and its Python binding never import this package.
+
+The arithmetic lives in mta_oracle.c (plain loops in double precision, one
+function per step of the pages' definition); this module only marshals numpy
+arrays through ctypes.  All inputs are widened to float64 before the call.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("d", ctypes.c_int), ("c_q", ctypes.c_int), ("c_k", ctypes.c_int),
+                ("c_h", ctypes.c_int), ("gn_eps", ctypes.c_double)]
+
+
+_lib = None
+
+
+def _configure(lib):
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int)
+    sp = ctypes.POINTER(_Shape)
+    lib.mta_oracle_forward.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_double,
+                                       dp, ctypes.c_int]
+    lib.mta_oracle_rows.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_double,
+                                    ctypes.c_int, ip, ctypes.c_int, dp, ctypes.c_int]
+    lib.mta_oracle_stages.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_double,
+                                      ctypes.c_int, dp, dp, dp, dp, dp]
+    lib.mta_oracle_max_threads.argtypes = []
+    for f in (lib.mta_oracle_forward, lib.mta_oracle_rows, lib.mta_oracle_stages,
+              lib.mta_oracle_max_threads):
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _configure(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+class use_library:
+    """Context manager that routes this module's calls to another build of
+    the oracle source (the mutation tests use it to check that the pins
+    catch planted mistakes)."""
+
+    def __init__(self, path):
+        self._new = _configure(ctypes.CDLL(path))
+
+    def __enter__(self):
+        global _lib
+        self._old = _lib
+        _lib = self._new
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self._old
+        return False
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double)) if a is not None else None
+
+
+def _shape(B, H, T, d, c_q, c_k, c_h, gn_eps):
+    return _Shape(int(B), int(H), int(T), int(d), int(c_q), int(c_k), int(c_h), float(gn_eps))
+
+
+def _unpack(q, w_kq, w_head):
+    B, H, T, d = q.shape
+    _, c_q, c_k = w_kq.shape
+    c_h = w_head.shape[-1]
+    return B, H, T, d, c_q, c_k, c_h
+
+
+def max_threads() -> int:
+    return int(_load().mta_oracle_max_threads())
+
+
+def forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gn_eps=1e-5,
+            nthreads=0):
+    """out[B, T, H*d] for q, k, v [B, H, T, d], w_kq [H, c_q, c_k],
+    w_head [H/c_h, c_h, c_h], gn_weight/gn_bias [H*d]."""
+    q, k, v, w_kq, w_head, gw, gb = map(_f64, (q, k, v, w_kq, w_head, gn_weight, gn_bias))
+    B, H, T, d, c_q, c_k, c_h = _unpack(q, w_kq, w_head)
+    out = np.empty((B, T, H * d), dtype=np.float64)
+    s = _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
+    rc = _load().mta_oracle_forward(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                    _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale),
+                                    _ptr(out), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("mta_oracle_forward failed (%d)" % rc)
+    return out
+
+
+def rows(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, b, row_idx,
+         gn_eps=1e-5, nthreads=0):
+    """out[b, row_idx, :] computed one row at a time: [len(row_idx), H*d]."""
+    q, k, v, w_kq, w_head, gw, gb = map(_f64, (q, k, v, w_kq, w_head, gn_weight, gn_bias))
+    B, H, T, d, c_q, c_k, c_h = _unpack(q, w_kq, w_head)
+    idx = np.ascontiguousarray(np.asarray(row_idx, dtype=np.int32))
+    out = np.empty((idx.size, H * d), dtype=np.float64)
+    s = _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
+    rc = _load().mta_oracle_rows(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                 _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale), int(b),
+                                 idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), int(idx.size),
+                                 _ptr(out), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("mta_oracle_rows failed (%d)" % rc)
+    return out
+
+
+def stages(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, b=0, gn_eps=1e-5):
+    """Intermediates of batch entry b (small T only), as a dict:
+    C [H,T,T] conv logits after both masks (-inf above the diagonal),
+    P [H,T,T] pre-mix softmax, A [H,T,T] post-mix attention,
+    O [H,T,d] pre-normalisation head outputs, out [T, H*d]."""
+    q, k, v, w_kq, w_head, gw, gb = map(_f64, (q, k, v, w_kq, w_head, gn_weight, gn_bias))
+    B, H, T, d, c_q, c_k, c_h = _unpack(q, w_kq, w_head)
+    C = np.empty((H, T, T)); P = np.empty((H, T, T)); A = np.empty((H, T, T))
+    O = np.empty((H, T, d)); out = np.empty((T, H * d))
+    s = _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
+    rc = _load().mta_oracle_stages(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                   _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale), int(b),
+                                   _ptr(C), _ptr(P), _ptr(A), _ptr(O), _ptr(out))
+    if rc != 0:
+        raise RuntimeError("mta_oracle_stages failed (%d)" % rc)
+    return {"C": C, "P": P, "A": A, "O": O, "out": out}

@@ -1,0 +1,81 @@
+"""The pins have teeth: plant one plausible mistake at a time in a copy of the
+oracle source, build it on the CPU, and check that at least one pin fails."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "mta_oracle.c")
+
+# (name, original text, mutated text)
+MUTATIONS = [
+    ("mix matrix transposed", "wg[ho * c_h + hi]", "wg[hi * c_h + ho]"),
+    ("key offset sign flipped", "int c = j - jp;", "int c = j + jp;"),
+    ("query taps reversed", "theta[ip * c_k + (jp - jlo)]",
+     "theta[(c_q - 1 - ip) * c_k + (jp - jlo)]"),
+    ("no Mask_0 before the conv", "for (int c = 0; c <= r; ++c) {",
+     "for (int c = 0; c < T; ++c) {"),
+    ("Mask_-inf replaced by zero", "if (j > i) { C[j] = -INFINITY; continue; }",
+     "if (j > i) { C[j] = 0.0; continue; }"),
+    ("unbiased variance", "        var /= d;\n        double inv",
+     "        var /= (d - 1);\n        double inv"),
+    ("eps outside the square root", "1.0 / sqrt(var + s->gn_eps)",
+     "1.0 / (sqrt(var) + s->gn_eps)"),
+    ("scale 1/d instead of 1/sqrt(d)", "1.0 / sqrt((double)d)", "1.0 / (double)d"),
+    ("value of the input head", "const double *vj = row_of(a->v, s, b, h, j);",
+     "const double *vj = row_of(a->v, s, b, g * c_h + (c_h - 1 - ho), j);"),
+    ("even-c_k window mirrored", "const int jlo = -(c_k / 2);",
+     "const int jlo = -((c_k - 1) / 2);"),
+    ("depth scale dropped", "out_row[chn] = a->depth_scale * y;", "out_row[chn] = y;"),
+]
+
+PIN_CHECKS = [
+    lambda: [pins.test_oracle_matches_library_composition(s) for s in pins.SHAPES],
+    pins.test_identity_kernels_give_causal_softmax_attention,
+    lambda: [pins.test_single_tap_kernel_closed_form(a, b) for a, b in ((6, 11), (3, 4))],
+    pins.test_receptive_field_matches_golden,
+    pins.test_zero_kernel_gives_prefix_mean,
+    pins.test_diff_transformer_special_case,
+    pins.test_causality_future_tokens_do_not_leak,
+    pins.test_row_sums_pre_and_post_mix,
+    pins.test_groupnorm_statistics_and_depth_scale,
+]
+
+
+def _build_mutant(tmp_path, before, after):
+    text = open(SRC).read()
+    assert text.count(before) == 1, before
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(before, after))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(lib), str(src),
+                    "-lm"], check=True)
+    return str(lib)
+
+
+@pytest.mark.parametrize("name,before,after", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_some_pin_catches(tmp_path, name, before, after):
+    lib = _build_mutant(tmp_path, before, after)
+    caught = []
+    with oracle.use_library(lib):
+        for check in PIN_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                caught.append(check)
+    assert caught, "no pin caught the planted mistake: " + name
+
+
+def test_unmutated_source_passes_every_pin(tmp_path):
+    lib = tmp_path / "libsame.so"
+    shutil.copy(SRC, tmp_path / "same.c")
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(lib),
+                    str(tmp_path / "same.c"), "-lm"], check=True)
+    with oracle.use_library(str(lib)):
+        for check in PIN_CHECKS:
+            check()
