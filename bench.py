@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Throughput of the Multi-Token Attention forward on B200.
+
+`python bench.py --gpus N --steps K --warmup W` runs W untimed and K timed
+steps of the MTA forward on the long-context workload (B2 H16 d128 T4096,
+(c_q, c_k, c_h) = (6, 11, 2), bf16) on each of N GPUs (one process per GPU,
+independent replicas: weak scaling), and rank 0 prints one JSON line.
+
+Timing: device time from CUDA events on the stream the library launches on,
+with the L2 cache flushed (a 256 MiB write, untimed) before every timed step;
+barrier + synchronize on both sides of the timed region; max over ranks.
+Per-kernel times come from the library's traced entry point (events recorded
+around each of its launches).  SM clocks and throttle reasons are sampled
+through NVML during the timed region.  `e2e` repeats the measurement through
+the public API with pinned host buffers, copies included.  `cpu_baseline`
+times the fp64 oracle on a bounded sample of the same workload on the host.
+
+`--impl reference` times that oracle (the only reference implementation of
+this method: the pages ship no code) on the host cores instead.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from convolved_logit_attention_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MTA fwd TFLOP/s and tokens/s at T=4096 bf16; % of B200 bf16 tensor peak"
+L2_FLUSH_BYTES = 256 << 20
+# FP32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz.
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["mta", "reference"], default="mta")
+    p.add_argument("--workload", default="longctx_4k", choices=sorted(WORKLOADS))
+    p.add_argument("--path", choices=["forward", "unfused"], default="forward",
+                   help="forward: mta_forward (the fused path where supported); "
+                        "unfused: mta_forward_unfused (materialised maps)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples = []
+        self.reasons = set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self._ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as exc:   # no NVML: report the absence
+            self.error = repr(exc)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons - {"gpu_idle"})}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "mta" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif args.impl == "mta":
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def dist_max(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def device_inputs(x, io, device):
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    d = {n: torch.from_numpy(x[n]).to(device).to(dt) for n in ("q", "k", "v")}
+    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
+        d[n] = torch.from_numpy(x[n]).to(device)
+    return d
+
+
+def kernel_units(name, w):
+    """(bound, algorithmic amount per launch, unit) for each kernel the
+    library launches on workload w.  L = T(T+1)/2 live logits per (b, h)."""
+    logits = w.B * w.H * w.live_logits()
+    io_bytes = 2 if w.io == "bf16" else 4
+    table = {
+        "k_logits": ("alu", logits * 2 * w.d, "FLOP"),
+        "k_conv": ("alu", logits * 2 * w.c_q * w.c_k, "FLOP"),
+        "k_softmax_mix": ("hbm", logits * 8, "B"),            # read C, write A_new (fp32)
+        "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
+        "k_fold_prologue": ("hbm", w.B * w.H * w.T * w.d * io_bytes * (2 + w.c_q + 1), "B"),
+        "k_mta_fused": ("tensor", w.algorithmic_flops(), "FLOP"),
+    }
+    return table.get(name, ("unknown", 0, "FLOP"))
+
+
+def load_traffic():
+    """Per-launch DRAM traffic from committed ncu summaries, valid only while
+    the kernel source they were taken on is unchanged."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    out = {}
+    for name, rec in table.items():
+        src = os.path.join(ROOT, rec.get("source", ""))
+        try:
+            digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        except OSError:
+            continue
+        if digest == rec.get("source_sha256_16"):
+            out[name] = rec
+    return out
+
+
+def roofline(name, w, avg_ms, peaks, peak_src):
+    bound, amount, unit = kernel_units(name, w)
+    secs = avg_ms / 1e3
+    traffic = load_traffic().get(name)
+    tr_bytes = None
+    if traffic is not None and traffic.get("workload") == w.name:
+        tr_bytes = traffic.get("dram_bytes_per_launch")
+    if bound == "hbm":
+        achieved, peak, u = amount / secs / 1e9, peaks["hbm_gbs"], "GB/s"
+        src = peak_src
+    elif bound == "tensor":
+        achieved, peak, u = amount / secs / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        src = peak_src
+    else:
+        achieved, peak, u = amount / secs / 1e12, FP32_ALU_TFLOPS, "TFLOP/s"
+        src = "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"
+    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": u,
+            "frac": achieved / peak, "traffic": tr_bytes, "peak_source": src,
+            "algorithmic_per_launch": amount, "algorithmic_unit": unit,
+            "avg_launch_ms": avg_ms}
+
+
+def time_mta(args, w, d, world, device):
+    import convolved_logit_attention_b200 as mta
+    unfused = args.path == "unfused"
+    shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"], w.gn_eps)
+    nk = mta.mta_kernel_count(shape, unfused)
+    names = [mta.mta_kernel_name(shape, i, unfused) for i in range(nk)]
+    path = "materialised" if (unfused or mta.mta_forward_path(shape) == mta.MTA_PATH_MATERIALISED) \
+        else "fused_tc"
+    ws_bytes = (mta.mta_unfused_workspace_size(shape) if unfused else mta.mta_workspace_size(shape))
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    out = torch.empty((w.B, w.T, w.H * w.d), dtype=d["q"].dtype, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(events):
+        mta.mta_forward_traced(unfused, events, d["q"], d["k"], d["v"], d["w_kq"], d["w_head"],
+                               d["gn_weight"], d["gn_bias"], w.depth_scale, out=out,
+                               workspace=ws, stream=stream, gn_eps=w.gn_eps)
+
+    warm_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(warm_ev)
+    mta.mta_sync_status(stream, device)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)]
+               for _ in range(args.steps)]
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with sampler:
+        for s in range(args.steps):
+            flush.zero_()
+            step_ev[s][0].record(stream)
+            step(kern_ev[s])
+            step_ev[s][1].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world)
+    mta.mta_sync_status(stream, device)
+    total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    per_kernel = {}
+    for s in range(args.steps):
+        for i, name in enumerate(names):
+            per_kernel.setdefault(name, 0.0)
+            per_kernel[name] += kern_ev[s][2 * i].elapsed_time(kern_ev[s][2 * i + 1])
+    return {"total_ms": total_ms, "per_kernel_ms": per_kernel, "names": names,
+            "launches": nk * args.steps, "clocks": sampler.summary(), "path": path}
+
+
+def time_e2e(args, w, x, device):
+    """The public API with host buffers: per step, pinned host -> device copies
+    of every input, mta_forward, device -> host copy of the output."""
+    import convolved_logit_attention_b200 as mta
+    dt = torch.bfloat16 if w.io == "bf16" else torch.float32
+    host = {n: torch.from_numpy(x[n]).to(dt).pin_memory() for n in ("q", "k", "v")}
+    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
+        host[n] = torch.from_numpy(x[n]).pin_memory()
+    dev = {n: torch.empty_like(t, device=device) for n, t in host.items()}
+    out = torch.empty((w.B, w.T, w.H * w.d), dtype=dt, device=device)
+    out_host = torch.empty(out.shape, dtype=dt).pin_memory()
+    shape = mta.shape_of(dev["q"], dev["w_kq"], dev["w_head"], w.gn_eps)
+    ws = torch.empty(max(mta.mta_workspace_size(shape), 1), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out.numel() * out.element_size()
+
+    def step():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        mta.mta_forward(dev["q"], dev["k"], dev["v"], dev["w_kq"], dev["w_head"],
+                        dev["gn_weight"], dev["gn_bias"], w.depth_scale, out=out, workspace=ws,
+                        stream=stream, gn_eps=w.gn_eps)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize(device)
+    return sum(a.elapsed_time(b) for a, b in ev), h2d, d2h
+
+
+def oracle_sample(w, x, n_units):
+    """The first n_units (batch, head-group) units of the workload at full T,
+    as separate B=1, H=c_h problems, with their algorithmic FLOPs."""
+    units = []
+    for u in range(min(n_units, w.B * w.G)):
+        b, g = divmod(u, w.G)
+        hs = slice(g * w.c_h, (g + 1) * w.c_h)
+        cs = slice(g * w.c_h * w.d, (g + 1) * w.c_h * w.d)
+        units.append((x["q"][b:b + 1, hs], x["k"][b:b + 1, hs], x["v"][b:b + 1, hs],
+                      x["w_kq"][hs], x["w_head"][g:g + 1], x["gn_weight"][cs],
+                      x["gn_bias"][cs]))
+    flops = len(units) * w.algorithmic_flops() // (w.B * w.G)
+    return units, flops
+
+
+def run_oracle_units(units, w, nthreads):
+    """Runs the oracle forward on every unit, one unit per host thread (the
+    ctypes call releases the GIL); returns the wall time in seconds."""
+    import concurrent.futures as cf
+    import oracle
+
+    def one(u):
+        return oracle.forward(u[0], u[1], u[2], u[3], u[4], u[5], u[6], w.depth_scale,
+                              gn_eps=w.gn_eps, nthreads=1)
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=nthreads) as ex:
+        list(ex.map(one, units))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, x):
+    cores = os.cpu_count() or 1
+    n_units = min(cores, w.B * w.G)
+    units, flops = oracle_sample(w, x, n_units)
+    secs = run_oracle_units(units, w, n_units)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": n_units, "kind": "oracle",
+            "seconds": secs,
+            "sample": "%d of %d (batch, head-group) units of %s at full T=%d, one unit per "
+                      "host thread" % (len(units), w.B * w.G, w.name, w.T)}
+
+
+def reference_arm(args, w, world, rank):
+    """The fp64 oracle on the host cores, timed like a step: each step is a
+    bounded sample (one unit per host thread, full T) of the workload."""
+    if rank != 0:
+        return None
+    x = make_inputs(w)
+    cores = os.cpu_count() or 1
+    n_units = min(cores, w.B * w.G)
+    units, flops = oracle_sample(w, x, n_units)
+    for _ in range(args.warmup):
+        run_oracle_units(units[:1], w, 1)
+    total = sum(run_oracle_units(units, w, n_units) for _ in range(args.steps))
+    value = flops * args.steps / total / 1e12
+    sample = ("%d of %d (batch, head-group) units of %s at full T=%d per step, one unit per host "
+              "thread" % (len(units), w.B * w.G, w.name, w.T))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, "oracle (host)"),
+            "tokens_per_s": n_units * w.T * args.steps / total,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": n_units, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def workload_config(w, path):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "c_q": w.c_q,
+            "c_k": w.c_k, "c_h": w.c_h, "io": w.io, "path": path,
+            "l2": "flushed before every timed step (256 MiB write, untimed)",
+            "parallelism": "independent replicas, one per GPU"}
+
+
+def mta_arm(args, w, world, rank, local):
+    device = torch.device("cuda", local)
+    from convolved_logit_attention_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    x = make_inputs(w, seed=w.seed + rank)
+    d = device_inputs(x, w.io, device)
+    peaks, peak_src = load_peaks()
+    res = time_mta(args, w, d, world, device)
+    bad = [r for r in res["clocks"]["reasons"] if r in BAD_REASONS]
+    if bad:   # one re-measurement after a throttled run
+        res = time_mta(args, w, d, world, device)
+    total_ms = dist_max(res["total_ms"], world, device)
+    per_step_ms = total_ms / args.steps
+    flops = w.algorithmic_flops()
+    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    kernels = {n: t / args.steps for n, t in res["per_kernel_ms"].items()}
+    dom = max(kernels, key=kernels.get)
+    rl = roofline(dom, w, kernels[dom], peaks, peak_src)
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if (w.io == "bf16" and res["path"] == "fused_tc") else "f32",
+            "data": "synthetic", "config": workload_config(w, res["path"]),
+            "tokens_per_s": world * w.tokens() * args.steps / (total_ms / 1e3),
+            "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
+            "peaks": dict(peaks, source=peak_src),
+            "roofline": {k: rl[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                             "traffic")},
+            "roofline_detail": rl,
+            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src)) for n in res["names"]],
+            "gpu_launches": res["launches"], "clocks": res["clocks"]}
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(args, w, x, device)
+        e2e_ms = dist_max(e2e_ms, world, device)
+        line["e2e"] = {"value": world * flops * args.steps / (e2e_ms / 1e3) / 1e12,
+                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": e2e_ms / args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, x)
+    return line if rank == 0 else None
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_setup(args)
+    w = WORKLOADS[args.workload]
+    try:
+        if args.impl == "reference":
+            line = reference_arm(args, w, world, rank)
+        else:
+            line = mta_arm(args, w, world, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+// C-ABI entry points of libmta.so (declared in include/mta.h): argument
+// validation on the host, workspace queries, and dispatch to the kernels.
+// Nothing is enqueued unless every check passes.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mta.h"
+#include "mta_internal.h"
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool is_pow2_ch(int c) { return c == 1 || c == 2 || c == 4 || c == 8 || c == 16; }
+
+mta_status check_shape(const mta_shape *s)
+{
+    if (!s) return MTA_ERR_INVALID_ARG;
+    if (s->B < 1 || s->H < 1 || s->T < 1 || s->d < 1 || s->c_q < 1 || s->c_k < 1 || s->c_h < 1)
+        return MTA_ERR_INVALID_ARG;
+    if (s->H % s->c_h != 0) return MTA_ERR_INVALID_ARG;
+    if (!(s->gn_eps > 0.f)) return MTA_ERR_INVALID_ARG;
+    if (s->io != MTA_F32 && s->io != MTA_BF16) return MTA_ERR_INVALID_ARG;
+    if (s->d < 8 || s->d > 128 || s->d % 8 != 0) return MTA_ERR_UNSUPPORTED;
+    if (s->c_q > 8 || s->c_k > 15 || !is_pow2_ch(s->c_h)) return MTA_ERR_UNSUPPORTED;
+    // grid dimensions of the materialised kernels and 32-bit row counts
+    if ((long long)s->B * s->H > 65535 || s->T > 65535 * 32) return MTA_ERR_UNSUPPORTED;
+    return MTA_OK;
+}
+
+mta_status check_tensors(const void *q, const void *k, const void *v, const float *w_kq,
+                         const float *w_head, const float *gn_weight, const float *gn_bias,
+                         const void *out)
+{
+    const void *ptrs[] = {q, k, v, w_kq, w_head, gn_weight, gn_bias, out};
+    for (const void *p : ptrs)
+        if (!p) return MTA_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return MTA_ERR_ALIGNMENT;
+    return MTA_OK;
+}
+
+mta_status check_workspace(const void *ws, size_t have, size_t need)
+{
+    if (need == 0) return MTA_OK;
+    if (!ws) return MTA_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return MTA_ERR_ALIGNMENT;
+    if (have < need) return MTA_ERR_WORKSPACE;
+    return MTA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mta_version(void) { return 100; }
+
+const char *mta_status_string(mta_status st)
+{
+    switch (st) {
+        case MTA_OK: return "ok";
+        case MTA_ERR_INVALID_ARG: return "invalid argument";
+        case MTA_ERR_UNSUPPORTED: return "unsupported shape";
+        case MTA_ERR_ALIGNMENT: return "misaligned pointer";
+        case MTA_ERR_WORKSPACE: return "workspace too small";
+        case MTA_ERR_CUDA: return "CUDA runtime error";
+        case MTA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+mta_path mta_forward_path(const mta_shape *s)
+{
+    if (check_shape(s) != MTA_OK) return MTA_PATH_MATERIALISED;
+    return mta::fused_supported(*s) ? MTA_PATH_FUSED_TC : MTA_PATH_MATERIALISED;
+}
+
+size_t mta_workspace_size(const mta_shape *s)
+{
+    if (check_shape(s) != MTA_OK) return 0;
+    return mta::fused_supported(*s) ? mta::fused_workspace_bytes(*s)
+                                    : mta::unfused_workspace_bytes(*s);
+}
+
+size_t mta_unfused_workspace_size(const mta_shape *s)
+{
+    if (check_shape(s) != MTA_OK) return 0;
+    return mta::unfused_workspace_bytes(*s);
+}
+
+mta_status mta_forward_traced(int unfused, const mta_shape *s, const void *q, const void *k,
+                              const void *v, const float *w_kq, const float *w_head,
+                              const float *gn_weight, const float *gn_bias, float depth_scale,
+                              void *out, void *workspace, size_t workspace_bytes, void *stream,
+                              void *const *events, int n_events)
+{
+    mta_status rc = check_shape(s);
+    if (rc == MTA_OK) rc = check_tensors(q, k, v, w_kq, w_head, gn_weight, gn_bias, out);
+    if (rc != MTA_OK) return rc;
+    if (n_events < 0 || (n_events > 0 && !events)) return MTA_ERR_INVALID_ARG;
+    const bool fused = !unfused && mta::fused_supported(*s);
+    const size_t need = fused ? mta::fused_workspace_bytes(*s) : mta::unfused_workspace_bytes(*s);
+    rc = check_workspace(workspace, workspace_bytes, need);
+    if (rc != MTA_OK) return rc;
+    mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out};
+    mta::Trace tr;
+    tr.events = events;
+    tr.n = n_events;
+    cudaStream_t st = (cudaStream_t)stream;
+    return fused ? mta::launch_fused(*s, a, workspace, st, tr)
+                 : mta::launch_unfused(*s, a, workspace, st, tr);
+}
+
+mta_status mta_forward(const mta_shape *s, const void *q, const void *k, const void *v,
+                       const float *w_kq, const float *w_head, const float *gn_weight,
+                       const float *gn_bias, float depth_scale, void *out, void *workspace,
+                       size_t workspace_bytes, void *stream)
+{
+    return mta_forward_traced(0, s, q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out,
+                              workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+mta_status mta_forward_unfused(const mta_shape *s, const void *q, const void *k, const void *v,
+                               const float *w_kq, const float *w_head, const float *gn_weight,
+                               const float *gn_bias, float depth_scale, void *out,
+                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    return mta_forward_traced(1, s, q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out,
+                              workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+int mta_kernel_count(const mta_shape *s, int unfused)
+{
+    if (check_shape(s) != MTA_OK) return 0;
+    if (!unfused && mta::fused_supported(*s)) return mta::fused_kernel_count(*s);
+    return mta::kUnfusedKernels;
+}
+
+const char *mta_kernel_name(const mta_shape *s, int unfused, int index)
+{
+    if (check_shape(s) != MTA_OK || index < 0 || index >= mta_kernel_count(s, unfused))
+        return nullptr;
+    if (!unfused && mta::fused_supported(*s)) return mta::fused_kernel_name(*s, index);
+    return mta::kUnfusedKernelNames[index];
+}
+
+mta_status mta_debug_attention(const mta_shape *s, const void *q, const void *k,
+                               const float *w_kq, const float *w_head, float *attn, int stage,
+                               void *workspace, size_t workspace_bytes, void *stream)
+{
+    mta_status rc = check_shape(s);
+    if (rc != MTA_OK) return rc;
+    if (stage != 0 && stage != 1) return MTA_ERR_INVALID_ARG;
+    if (s->T > 2048) return MTA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {q, k, w_kq, w_head, attn};
+    for (const void *p : ptrs)
+        if (!p) return MTA_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return MTA_ERR_ALIGNMENT;
+    rc = check_workspace(workspace, workspace_bytes, mta::unfused_workspace_bytes(*s));
+    if (rc != MTA_OK) return rc;
+    return mta::launch_debug_attention(*s, q, k, w_kq, w_head, attn, stage, workspace,
+                                       (cudaStream_t)stream);
+}
+
+mta_status mta_sync_status(void *stream)
+{
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MTA_ERR_CUDA;
+    if (mta::fused_take_error() != 0) return MTA_ERR_DEVICE_TIMEOUT;
+    return MTA_OK;
+}
+
+}  // extern "C"

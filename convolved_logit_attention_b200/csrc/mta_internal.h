@@ -1,0 +1,56 @@
+// Internal interfaces between the C-ABI layer (api.cu) and the kernel
+// translation units.  Not installed; the public ABI is include/mta.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "mta.h"
+
+namespace mta {
+
+// Tensor arguments of one forward call, all device pointers.
+struct ForwardArgs {
+    const void *q, *k, *v;
+    const float *w_kq, *w_head, *gn_weight, *gn_bias;
+    float depth_scale;
+    void *out;
+};
+
+// Optional CUDA events recorded around the kernel launches of one call.
+struct Trace {
+    void *const *events = nullptr;
+    int n = 0;
+    void before(int launch, cudaStream_t st) const {
+        if (2 * launch + 1 < n) cudaEventRecord((cudaEvent_t)events[2 * launch], st);
+    }
+    void after(int launch, cudaStream_t st) const {
+        if (2 * launch + 1 < n) cudaEventRecord((cudaEvent_t)events[2 * launch + 1], st);
+    }
+};
+
+inline size_t bh_tt(const mta_shape &s) {
+    return (size_t)s.B * s.H * (size_t)s.T * (size_t)s.T;
+}
+
+// Materialised chain (unfused.cu).
+size_t unfused_workspace_bytes(const mta_shape &s);
+constexpr int kUnfusedKernels = 4;
+extern const char *const kUnfusedKernelNames[kUnfusedKernels];
+mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
+                          const Trace &tr);
+mta_status launch_debug_attention(const mta_shape &s, const void *q, const void *k,
+                                  const float *w_kq, const float *w_head, float *attn, int stage,
+                                  void *ws, cudaStream_t st);
+
+// Fused tcgen05 path (fused_tc.cu).
+bool fused_supported(const mta_shape &s);
+size_t fused_workspace_bytes(const mta_shape &s);
+int fused_kernel_count(const mta_shape &s);
+const char *fused_kernel_name(const mta_shape &s, int index);
+mta_status launch_fused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
+                        const Trace &tr);
+// Reads and clears the fused kernels' device error word on the current device.
+unsigned int fused_take_error();
+
+}  // namespace mta

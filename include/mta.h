@@ -1,0 +1,169 @@
+/*
+ * mta.h -- C ABI of the Multi-Token Attention (MTA) forward library for
+ * NVIDIA B200 (sm_100a).  Library: convolved_logit_attention_b200/libmta.so.
+ *
+ * What is computed (per batch entry b, head h, query i, key j, following
+ * "Multi-Token Attention -- Paper Graph", section 3.4):
+ *   S1  A^[i][j]  = q_i . k_j / sqrt(d)                ("Standard Multi-Head
+ *                                                        Attention")
+ *   S2  A0        = Mask_0(A^): zero where j > i       ("Key-Query Convolution",
+ *                                                        Eq. (5), first mask)
+ *   S3  C[i][j]   = sum_{i'=0}^{c_q-1} sum_{j'=-floor(c_k/2)}^{ceil(c_k/2)-1}
+ *                   theta_h[i'][j'] A0[i-i'][j-j']     (Eq. (4) index ranges;
+ *                   taps outside [0,T)^2 read zero)
+ *   S4  C[i][j]   = -inf where j > i                   (Eq. (5), second mask)
+ *   S5  P^h       = softmax over j of C                ("Standard MHA")
+ *   S6  A^h_new   = sum_{h' in group(h)} w_g[h][h'] P^h'
+ *                   (groups of c_h consecutive heads; "Head Mixing
+ *                   Convolution", Eq. (7), applied after the softmax)
+ *   S7  O^h       = A^h_new V^h
+ *   S8  y         = GroupNorm over each head's d values (biased variance,
+ *                   eps inside the root) with per-channel gamma, beta
+ *                   ("Group Normalization with Sigmoid Gating"; one group
+ *                   per head)
+ *   S9  out       = depth_scale * y                    ("Article Overview:
+ *                   Multi-Token Attention", section 2, "Group Normalization
+ *                   with Depth Scaling")
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is DEVICE memory owned by the caller; the library
+ *     never allocates, frees or keeps a pointer after the call returns.
+ *   - Tensors are dense and contiguous, row-major, with these layouts:
+ *       q, k, v    [B][H][T][d]       dtype shape->io (fp32 or bf16)
+ *       w_kq       [H][c_q][c_k]      fp32; tap (i', j') at [h][i'][j'+floor(c_k/2)]
+ *       w_head     [H/c_h][c_h][c_h]  fp32; [group][output head][input head]
+ *       gn_weight  [H*d], gn_bias [H*d]   fp32, channel h*d + e
+ *       out        [B][T][H*d]        dtype shape->io (the head concatenation)
+ *   - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as a
+ *     plain pointer; NULL means the legacy default stream).  Argument errors
+ *     are detected on the host before anything is enqueued, and nothing is
+ *     enqueued when a call returns an error.
+ *   - Errors are returned as mta_status codes; the library never aborts,
+ *     throws or prints.  A device-side wait that runs out of its bound makes
+ *     the kernel return early and raises a flag that mta_sync_status()
+ *     reports as MTA_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef MTA_H
+#define MTA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of the ABI are exported; everything else in the library is hidden. */
+#if defined(__GNUC__)
+#define MTA_API __attribute__((visibility("default")))
+#else
+#define MTA_API
+#endif
+
+typedef enum {
+    MTA_OK = 0,
+    MTA_ERR_INVALID_ARG = -1,    /* null pointer, non-positive size, H % c_h != 0 */
+    MTA_ERR_UNSUPPORTED = -2,    /* shape outside the supported ranges below */
+    MTA_ERR_ALIGNMENT = -3,      /* pointer not 16-byte (workspace: 256-byte) aligned */
+    MTA_ERR_WORKSPACE = -4,      /* workspace smaller than the *_workspace_size query */
+    MTA_ERR_CUDA = -5,           /* a CUDA runtime call failed */
+    MTA_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait expired */
+} mta_status;
+
+typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
+
+/* Problem description.  Supported ranges: B, H, T >= 1 with B*H <= 65535;
+ * 8 <= d <= 128 with d % 8 == 0; 1 <= c_q <= 8; 1 <= c_k <= 15;
+ * c_h in {1, 2, 4, 8, 16} with H % c_h == 0; gn_eps > 0 (1e-5 is the usual
+ * GroupNorm default; the pages do not state one).  Violations of the
+ * arithmetic constraints (non-positive sizes, H % c_h, gn_eps) are
+ * MTA_ERR_INVALID_ARG; sizes outside the supported ranges are
+ * MTA_ERR_UNSUPPORTED. */
+typedef struct {
+    int B, H, T, d, c_q, c_k, c_h;
+    mta_dtype io;
+    float gn_eps;
+} mta_shape;
+
+/* Which device path mta_forward takes for a shape. */
+typedef enum {
+    MTA_PATH_FUSED_TC = 0,       /* fused tcgen05 kernel: no T x T map in HBM */
+    MTA_PATH_MATERIALISED = 1    /* the S1..S9 chain of mta_forward_unfused */
+} mta_path;
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+MTA_API int mta_version(void);
+
+/* Static text for a status code; never NULL. */
+MTA_API const char *mta_status_string(mta_status status);
+
+/* The path mta_forward uses for *shape (an invalid shape reports
+ * MTA_PATH_MATERIALISED; validation happens in the call itself). */
+MTA_API mta_path mta_forward_path(const mta_shape *shape);
+
+/* Bytes of device workspace mta_forward needs for *shape (0 on an invalid
+ * shape).  Sized for the path mta_forward_path() names. */
+MTA_API size_t mta_workspace_size(const mta_shape *shape);
+
+/* Bytes of device workspace mta_forward_unfused and mta_debug_attention need:
+ * two fp32 [B][H][T][T] maps. */
+MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
+
+/* The MTA forward S1..S9 above, out = depth_scale * GN(...), written to out.
+ * The bf16 fused path computes the folded logits and P V on tensor cores with
+ * bf16 operands and fp32 accumulation; the materialised path computes in fp32.
+ * The workspace is scratch owned by the caller for the duration of the
+ * enqueued work; its contents on entry are ignored. */
+MTA_API mta_status mta_forward(const mta_shape *shape, const void *q, const void *k, const void *v,
+                       const float *w_kq, const float *w_head, const float *gn_weight,
+                       const float *gn_bias, float depth_scale, void *out,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* The same forward computed step by step with the T x T maps materialised in
+ * the workspace (S1+S2 logits, S3+S4 conv, S5+S6 softmax and mix, S7..S9
+ * PV with the GroupNorm epilogue), all arithmetic in fp32.  Same arguments
+ * and contract as mta_forward. */
+MTA_API mta_status mta_forward_unfused(const mta_shape *shape, const void *q, const void *k,
+                               const void *v, const float *w_kq, const float *w_head,
+                               const float *gn_weight, const float *gn_bias, float depth_scale,
+                               void *out, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Debug view of the attention maps for small problems (T <= 2048):
+ * attn [B][H][T][T] fp32 receives the pre-mix softmax P (stage 0) or the
+ * post-mix A_new (stage 1), with zeros above the diagonal.  Workspace as for
+ * mta_forward_unfused.  Any other stage is MTA_ERR_INVALID_ARG; T > 2048 is
+ * MTA_ERR_UNSUPPORTED. */
+MTA_API mta_status mta_debug_attention(const mta_shape *shape, const void *q, const void *k,
+                               const float *w_kq, const float *w_head, float *attn, int stage,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Kernel launches one mta_forward (unfused == 0) or mta_forward_unfused
+ * (unfused != 0) call makes for *shape, and the name of launch `index`
+ * (NULL when out of range or the shape is invalid).  For tracing. */
+MTA_API int mta_kernel_count(const mta_shape *shape, int unfused);
+MTA_API const char *mta_kernel_name(const mta_shape *shape, int unfused, int index);
+
+/* mta_forward (unfused == 0) or mta_forward_unfused (unfused != 0) that also
+ * records caller-created CUDA events (cudaEvent_t handles passed as plain
+ * pointers) on `stream` around its kernel launches: events[2*i] just before
+ * and events[2*i+1] just after launch i, for i < n_events / 2.  The events
+ * stay owned by the caller.  Same contract as the untraced call otherwise;
+ * a NULL `events` with n_events == 0 records nothing. */
+MTA_API mta_status mta_forward_traced(int unfused, const mta_shape *shape, const void *q,
+                                      const void *k, const void *v, const float *w_kq,
+                                      const float *w_head, const float *gn_weight,
+                                      const float *gn_bias, float depth_scale, void *out,
+                                      void *workspace, size_t workspace_bytes, void *stream,
+                                      void *const *events, int n_events);
+
+/* Synchronises `stream`, then reports (and clears) the device error flag set
+ * by a kernel whose bounded wait expired: MTA_ERR_DEVICE_TIMEOUT in that case,
+ * MTA_ERR_CUDA if the synchronisation itself failed, MTA_OK otherwise. */
+MTA_API mta_status mta_sync_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MTA_H */

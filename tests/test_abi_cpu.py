@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/mta.h declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import convolved_logit_attention_b200 as mta
+from convolved_logit_attention_b200 import _binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from convolved_logit_attention_b200 import build
+    build.build()
+    return mta.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "mta.h")).read()
+    return sorted(set(re.findall(r"MTA_API\s+[\w\s\*]*?\b(mta_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert header_functions() == sorted(_binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in header_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(L):
+    assert mta.mta_version() == 100
+    for code in _binding.STATUS:
+        assert mta.mta_status_string(code)
+    assert mta.mta_status_string(123) == "unknown status"
+
+
+GOOD = dict(B=2, H=4, T=64, d=32, c_q=6, c_k=11, c_h=2)
+
+
+def shape(**kw):
+    args = dict(GOOD)
+    args.update(kw)
+    io = args.pop("io", "bf16")
+    return mta.make_shape(io=io, **args)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), -1), (dict(T=0), -1), (dict(H=3), -1), (dict(c_q=0), -1),
+    (dict(d=12), -2), (dict(d=136), -2), (dict(c_q=9), -2), (dict(c_k=16), -2),
+    (dict(H=6, c_h=3), -2),
+])
+def test_forward_rejects_bad_shapes_before_launch(L, kw, status):
+    s = shape(**kw)
+    p = ctypes.c_void_p(1 << 20)    # aligned fake pointers: the call must not launch
+    rc = L.mta_forward(ctypes.byref(s), p, p, p, p, p, p, p, 0.8, p, p, 1 << 40, None)
+    assert rc == status
+    assert mta.mta_workspace_size(s) == 0
+
+
+def test_forward_rejects_null_misaligned_and_small_workspace(L):
+    s = shape()
+    a = ctypes.c_void_p(1 << 20)
+    z = ctypes.c_void_p(0)
+    bad = ctypes.c_void_p((1 << 20) + 4)
+    need = mta.mta_workspace_size(s)
+    assert need > 0
+    args = [a] * 7
+    assert L.mta_forward(ctypes.byref(s), z, *args[1:], 0.8, a, a, need, None) == -1
+    assert L.mta_forward(ctypes.byref(s), bad, *args[1:], 0.8, a, a, need, None) == -3
+    assert L.mta_forward(ctypes.byref(s), *args, 0.8, a, ctypes.c_void_p((1 << 20) + 16),
+                         need, None) == -3
+    assert L.mta_forward(ctypes.byref(s), *args, 0.8, a, a, need - 1, None) == -4
+    assert L.mta_forward(ctypes.byref(s), *args, 0.8, a, z, need, None) == -1
+    assert L.mta_forward_unfused(ctypes.byref(s), *args, 0.8, a, a,
+                                 mta.mta_unfused_workspace_size(s) - 1, None) == -4
+
+
+def test_debug_attention_argument_checks(L):
+    s = shape()
+    a = ctypes.c_void_p(1 << 20)
+    ws = mta.mta_unfused_workspace_size(s)
+    assert L.mta_debug_attention(ctypes.byref(s), a, a, a, a, a, 2, a, ws, None) == -1
+    big = shape(T=4096)
+    assert L.mta_debug_attention(ctypes.byref(big), a, a, a, a, a, 0, a, 1 << 60, None) == -2
+
+
+def test_unfused_workspace_is_two_fp32_maps(L):
+    s = shape()
+    assert mta.mta_unfused_workspace_size(s) == 2 * 4 * 2 * 4 * 64 * 64

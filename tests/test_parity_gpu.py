@@ -1,0 +1,182 @@
+"""Parity of the CUDA path (called through the C ABI) with the fp64 oracle.
+
+Tolerances: fp32 I/O max-abs <= 1e-4; bf16 I/O max-abs <= 2e-2 and
+relative L2 <= 5e-3 (fp32 accumulation), measured on `out` against the oracle
+run on the same rounded inputs.  Small problems are compared element by
+element; full-size workloads (in the launch configuration the benchmark
+times) on sampled rows that the oracle computes one at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import convolved_logit_attention_b200 as mta
+from convolved_logit_attention_b200.workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32_MAXABS = 1e-4
+TOL_BF16_MAXABS = 2e-2
+TOL_BF16_RELL2 = 5e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from convolved_logit_attention_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def to_device(x, io):
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    dev = torch.device("cuda", 0)
+    d = {n: torch.from_numpy(np.ascontiguousarray(x[n])).to(dev).to(dt) for n in ("q", "k", "v")}
+    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
+        d[n] = torch.from_numpy(np.ascontiguousarray(x[n])).to(dev)
+    return d
+
+
+def run(fn, d, x, **kw):
+    out = fn(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"], d["gn_bias"],
+             x["depth_scale"], gn_eps=x["gn_eps"], **kw)
+    mta.mta_sync_status()
+    return out.float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(got, ref, io, what=""):
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), what + ": non-finite output"
+    maxabs = float(err.max())
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    if io == "f32":
+        assert maxabs <= TOL_F32_MAXABS, "%s: max-abs %.3g" % (what, maxabs)
+    else:
+        assert maxabs <= TOL_BF16_MAXABS and rel <= TOL_BF16_RELL2, \
+            "%s: max-abs %.3g rel-L2 %.3g" % (what, maxabs, rel)
+    return maxabs, rel
+
+
+def oracle_full(x):
+    return oracle.forward(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                          x["gn_bias"], x["depth_scale"], gn_eps=x["gn_eps"])
+
+
+FNS = {"forward": mta.mta_forward, "unfused": mta.mta_forward_unfused}
+
+
+@pytest.mark.parametrize("fn", sorted(FNS))
+@pytest.mark.parametrize("name", ["tiny_f32", "toy_letters"])
+def test_small_workloads_elementwise(name, fn):
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    ref = oracle_full(x)
+    got = run(FNS[fn], to_device(x, w.io), x)
+    assert_close(got, ref, w.io, name + "/" + fn)
+
+
+RAGGED = [
+    # B, H, T, d, c_q, c_k, c_h, io
+    (1, 2, 1, 32, 6, 11, 2, "bf16"),        # a single token
+    (1, 2, 7, 64, 6, 11, 2, "f32"),
+    (2, 4, 65, 32, 3, 4, 4, "bf16"),        # even c_k, ragged T
+    (1, 4, 200, 64, 6, 11, 2, "bf16"),
+    (1, 2, 300, 128, 8, 15, 2, "bf16"),
+    (1, 2, 257, 128, 2, 3, 1, "f32"),
+    (1, 8, 130, 16, 1, 1, 8, "bf16"),
+    (1, 4, 129, 128, 6, 11, 4, "bf16"),
+    (2, 2, 384, 128, 6, 11, 2, "bf16"),     # several full tiles
+    (1, 2, 511, 64, 4, 15, 2, "bf16"),
+]
+
+
+@pytest.mark.parametrize("fn", sorted(FNS))
+@pytest.mark.parametrize("shape", RAGGED, ids=[str(s) for s in RAGGED])
+def test_ragged_shapes_elementwise(shape, fn):
+    B, H, T, d, c_q, c_k, c_h, io = shape
+    w = Workload("ragged", B, H, T, d, c_q, c_k, c_h, io, seed=hash(shape) % 1000)
+    x = make_inputs(w)
+    ref = oracle_full(x)
+    got = run(FNS[fn], to_device(x, io), x)
+    assert_close(got, ref, io, str(shape) + "/" + fn)
+
+
+@pytest.mark.parametrize("fn", sorted(FNS))
+def test_identity_kernels_and_strong_kernels(fn):
+    # identity kernels (standard attention) and kernels far from identity
+    w = Workload("kern", 1, 4, 192, 64, 6, 11, 2, "bf16", seed=7)
+    x = make_inputs(w)
+    x["w_kq"][:] = 0
+    x["w_kq"][:, 0, 5] = 1
+    x["w_head"][:] = np.eye(2, dtype=np.float32)
+    assert_close(run(FNS[fn], to_device(x, "bf16"), x), oracle_full(x), "bf16", "identity")
+    rng = np.random.default_rng(8)
+    x["w_kq"] = rng.standard_normal(x["w_kq"].shape).astype(np.float32) * 0.4
+    x["w_head"] = rng.standard_normal(x["w_head"].shape).astype(np.float32)
+    assert_close(run(FNS[fn], to_device(x, "bf16"), x), oracle_full(x), "bf16", "strong")
+
+
+@pytest.mark.parametrize("stage", [0, 1])
+def test_debug_attention_maps(stage):
+    w = Workload("dbg", 1, 4, 96, 32, 6, 11, 2, "f32", seed=9)
+    x = make_inputs(w)
+    d = to_device(x, "f32")
+    attn = mta.mta_debug_attention(d["q"], d["k"], d["w_kq"], d["w_head"], stage)
+    mta.mta_sync_status()
+    st = oracle.stages(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                       x["gn_bias"], x["depth_scale"], b=0)
+    ref = st["P"] if stage == 0 else st["A"]
+    got = attn[0].cpu().numpy()
+    assert np.abs(got - ref).max() < 1e-5
+    assert np.all(np.triu(got, 1) == 0)
+
+
+def sample_rows(T, rng, n=12):
+    fixed = [0, 1, 2, 5, 63, 64, 127, 128, 129, 255, 256, T // 2, T - 2, T - 1]
+    rows = {r for r in fixed if 0 <= r < T}
+    rows |= set(int(r) for r in rng.integers(0, T, size=n))
+    return sorted(rows)
+
+
+FULL = ["pretrain_2k", "longctx_4k"] + sorted(n for n in WORKLOADS if n.startswith("long16k"))
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_rows(name):
+    """The benchmark's call (mta_forward on the full workload); rows sampled
+    per batch entry, including tile boundaries and both ends."""
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    d = to_device(x, w.io)
+    got = run(mta.mta_forward, d, x)
+    del d
+    torch.cuda.empty_cache()
+    rng = np.random.default_rng(11)
+    for b in range(w.B):
+        rows = sample_rows(w.T, rng)
+        ref = oracle.rows(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                          x["gn_bias"], x["depth_scale"], b, rows, gn_eps=x["gn_eps"])
+        assert_close(got[b, rows], ref, w.io, "%s b=%d" % (name, b))
+
+
+def test_full_size_output_properties():
+    """Properties that hold at any size: with unit gamma and zero bias each
+    (t, h) slice of out/depth_scale has mean 0 and variance <= 1."""
+    w = WORKLOADS["longctx_4k"]
+    x = make_inputs(w)
+    got = run(mta.mta_forward, to_device(x, w.io), x).reshape(w.B, w.T, w.H, w.d) / 0.8
+    assert np.abs(got.mean(-1)).max() < 2e-2
+    assert got.var(-1).max() < 1.0 + 2e-2
+
+
+def test_workspace_and_stream_reuse_gives_identical_results():
+    w = WORKLOADS["toy_letters"]
+    x = make_inputs(w)
+    d = to_device(x, w.io)
+    shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"])
+    ws = torch.empty(mta.mta_workspace_size(shape), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = run(mta.mta_forward, d, x, workspace=ws, stream=s)
+        b = run(mta.mta_forward, d, x, workspace=ws, stream=s)
+    assert np.array_equal(a, b)
