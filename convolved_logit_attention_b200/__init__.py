@@ -9,6 +9,7 @@ from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
                        MTA_PATH_MATERIALISED, MtaError, MtaShape, lib, make_shape,
                        mta_debug_attention, mta_forward, mta_forward_path, mta_forward_traced,
                        mta_forward_unfused, mta_kernel_count, mta_kernel_name,
+                       mta_selftest_wait_timeout,
                        mta_status_string, mta_sync_status, mta_unfused_workspace_size,
                        mta_version, mta_workspace_size, shape_of)
 
@@ -16,5 +17,6 @@ __all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC",
            "MTA_PATH_MATERIALISED", "MtaError", "MtaShape", "lib", "make_shape",
            "mta_debug_attention", "mta_forward", "mta_forward_path", "mta_forward_traced",
            "mta_forward_unfused", "mta_kernel_count", "mta_kernel_name",
+           "mta_selftest_wait_timeout",
            "mta_status_string", "mta_sync_status", "mta_unfused_workspace_size", "mta_version",
            "mta_workspace_size", "shape_of"]

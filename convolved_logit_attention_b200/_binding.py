@@ -19,13 +19,13 @@ MTA_F32, MTA_BF16 = 0, 1
 MTA_PATH_FUSED_TC, MTA_PATH_MATERIALISED = 0, 1
 STATUS = {0: "MTA_OK", -1: "MTA_ERR_INVALID_ARG", -2: "MTA_ERR_UNSUPPORTED",
           -3: "MTA_ERR_ALIGNMENT", -4: "MTA_ERR_WORKSPACE", -5: "MTA_ERR_CUDA",
-          -6: "MTA_ERR_DEVICE_TIMEOUT"}
+          -6: "MTA_ERR_DEVICE_TIMEOUT", -7: "MTA_ERR_RANGE"}
 
 # Every function include/mta.h declares.
 EXPORTS = ("mta_version", "mta_status_string", "mta_forward_path", "mta_workspace_size",
            "mta_unfused_workspace_size", "mta_forward", "mta_forward_unfused",
            "mta_debug_attention", "mta_kernel_count", "mta_kernel_name", "mta_forward_traced",
-           "mta_sync_status")
+           "mta_selftest_wait_timeout", "mta_sync_status")
 
 
 class MtaShape(ctypes.Structure):
@@ -77,6 +77,8 @@ def lib():
         L.mta_forward_traced.argtypes = [ctypes.c_int] + fwd + [ctypes.POINTER(ctypes.c_void_p),
                                                                ctypes.c_int]
         L.mta_forward_traced.restype = ctypes.c_int
+        L.mta_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+        L.mta_selftest_wait_timeout.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -238,6 +240,14 @@ def mta_debug_attention(q, k, w_kq, w_head, stage, attn=None, workspace=None, st
                                        _stream_ptr(stream, q.device))
     _check("mta_debug_attention", status)
     return attn
+
+
+def mta_selftest_wait_timeout(budget_cycles=1 << 20, stream=None, device=None):
+    """Enqueues the timeout-path diagnostic kernel (see include/mta.h)."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    _check("mta_selftest_wait_timeout",
+           lib().mta_selftest_wait_timeout(int(budget_cycles), _stream_ptr(stream, device)))
 
 
 def mta_sync_status(stream=None, device=None):

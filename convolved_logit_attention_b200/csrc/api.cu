@@ -65,6 +65,7 @@ const char *mta_status_string(mta_status st)
         case MTA_ERR_WORKSPACE: return "workspace too small";
         case MTA_ERR_CUDA: return "CUDA runtime error";
         case MTA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case MTA_ERR_RANGE: return "value outside the fp16 range of the fused path";
     }
     return "unknown status";
 }
@@ -163,10 +164,18 @@ mta_status mta_debug_attention(const mta_shape *s, const void *q, const void *k,
                                        (cudaStream_t)stream);
 }
 
+mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stream)
+{
+    if (budget_cycles <= 0 || budget_cycles >= (1ll << 31)) return MTA_ERR_INVALID_ARG;
+    return mta::launch_selftest_wait_timeout(budget_cycles, (cudaStream_t)stream);
+}
+
 mta_status mta_sync_status(void *stream)
 {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MTA_ERR_CUDA;
-    if (mta::fused_take_error() != 0) return MTA_ERR_DEVICE_TIMEOUT;
+    const unsigned int err = mta::fused_take_error();
+    if (err & 1u) return MTA_ERR_DEVICE_TIMEOUT;
+    if (err & 2u) return MTA_ERR_RANGE;
     return MTA_OK;
 }
 

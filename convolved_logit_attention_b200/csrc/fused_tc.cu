@@ -1,17 +1,727 @@
-// Fused tcgen05 MTA forward (placeholder until the kernel lands).
+// Fused MTA forward on sm_100a tensor cores (bf16 operands, fp32 accumulate).
+//
+// The key-query convolution of "Multi-Token Attention -- Paper Graph",
+// section 3.4, Eq. (4)/(5), is linear in the logits, so away from the
+// diagonal it folds into the contraction:
+//     C[i][j] = sum_{i'} q_{i-i'} . Kf^{(i')}_j,
+//     Kf^{(i')}_j = sum_{j'} theta[i'][j'] k_{j-j'} / sqrt(d)
+// (q rows before the sequence and k rows outside it are zero).  The first
+// mask of Eq. (5) zeroes logits of future keys before the convolution; the
+// fold includes those terms for pairs (i, j) within D_m = c_q - 1 +
+// floor(c_k/2) diagonals of the main one, and a per-row correction table
+// subtracts them there.
+//
+// Three kernels:
+//   k_fold_prologue  per (b, h, 128-row block): Kf^{(i')} for every i'
+//                    (fp16, scaled by log2(e)/sqrt(d) so that the softmax
+//                    runs on exp2), the query rows of the block (fp16) in the
+//                    permuted order the main kernel's shifted operand needs,
+//                    and the correction table corr[i][e] for key j = i - e.
+//                    fp16 carries three more mantissa bits than bf16 for the
+//                    folded logits; values outside its range raise an error.
+//   k_mta_fused      per (b, source head h', 128 query rows): for every key
+//                    tile, S = sum_{i'} Q_{shift i'} Kf^{(i')T} on tcgen05
+//                    (TMEM accumulator), correction + causal mask + online
+//                    softmax on CUDA cores, then U^{h,h'} += P~ V^h for every
+//                    head h of the group (post-softmax head mixing, Eq. (7),
+//                    with per-source-head normalisation deferred to the end).
+//                    Writes (w[h][h'] / l^{h'}) U^{h,h'} per row.
+//   k_mix_groupnorm  per (b, query row): O^h = sum_{h'} of those partials,
+//                    per-head GroupNorm with warp-shuffle reductions, depth
+//                    scale, bf16 store.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
 #include "mta_internal.h"
+#include "tc_util.cuh"
+#include "tmap.h"
 
 namespace mta {
+namespace {
 
-bool fused_supported(const mta_shape &) { return false; }
-size_t fused_workspace_bytes(const mta_shape &) { return 0; }
-int fused_kernel_count(const mta_shape &) { return 0; }
-const char *fused_kernel_name(const mta_shape &, int) { return nullptr; }
-mta_status launch_fused(const mta_shape &, const ForwardArgs &, void *, cudaStream_t,
-                        const Trace &)
+constexpr int kBM = 128;          // query rows per CTA (TMEM lanes)
+constexpr int kBN = 128;          // keys per tile
+constexpr int kCorrW = 16;        // correction entries stored per row (D_m <= 14)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr long long kWaitBudget = 1ll << 30;   // ~0.55 s at 1.965 GHz per wait
+
+// Device error word: bit 0 a bounded wait expired, bit 1 a folded operand
+// fell outside the fp16 range.
+__device__ unsigned int g_fused_error;
+constexpr unsigned int kErrTimeout = 1u, kErrRange = 2u;
+
+// Rows of the permuted query block: NA atoms of 8 rows; atom a, row s holds
+// query i0 - (c_q - 1) + a + 16 s.
+__host__ __device__ inline int q_atoms(int c_q) { return 16 + c_q - 1; }
+__host__ __device__ inline int d_m(int c_q, int c_k) { return c_q - 1 + c_k / 2; }
+
+// ------------------------------------------------------------ prologue
+
+constexpr int kProRows = 128;
+constexpr int kProKLo = 8;        // k rows loaded before the block
+constexpr int kProKHi = 15;       // k rows loaded after it
+constexpr int kProQLo = 7;        // q rows loaded before the block
+
+// One CTA per (128-row block, b*H + h).  Shared memory holds the block's k
+// rows with a halo ([j0-8, j0+143)) and q rows ([j0-7, j0+128)) as fp32.
+template <int D>
+__global__ void __launch_bounds__(256)
+k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                const float *__restrict__ w_kq, __half *__restrict__ kf,
+                __half *__restrict__ qp, float *__restrict__ corr, int T, int Tp, int H,
+                int c_q, int c_k, float scale)
 {
+    extern __shared__ __align__(16) float psm[];
+    constexpr int KR = kProKLo + kProRows + kProKHi;
+    constexpr int QR = kProQLo + kProRows;
+    float *ks = psm;                       // [KR][D]
+    float *qs = ks + KR * D;               // [QR][D]
+    float *fs = qs + QR * D;               // [QR][kCorrW] future logits q_r . k_{r+delta}
+    float *th = fs + QR * kCorrW;          // [c_q][c_k]
+    const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
+    const int j0 = blk * kProRows;
+    const int tid = threadIdx.x;
+    const size_t head_off = (size_t)bh * T * D;
+    for (int idx = tid; idx < KR * D; idx += 256) {
+        int r = idx / D, e = idx % D, j = j0 - kProKLo + r;
+        ks[idx] = (j >= 0 && j < T) ? __bfloat162float(k[head_off + (size_t)j * D + e]) : 0.f;
+    }
+    for (int idx = tid; idx < QR * D; idx += 256) {
+        int r = idx / D, e = idx % D, i = j0 - kProQLo + r;
+        qs[idx] = (i >= 0 && i < T) ? __bfloat162float(q[head_off + (size_t)i * D + e]) : 0.f;
+    }
+    for (int idx = tid; idx < c_q * c_k; idx += 256) th[idx] = w_kq[(size_t)h * c_q * c_k + idx];
+    __syncthreads();
+
+    // (a) Kf^{(i')}_j = scale * sum_jj theta[i'][jj] k_{j - (jj - floor(c_k/2))}
+    {
+        const int R = c_k / 2;
+        constexpr int EP = D / 2;                 // element pairs per row
+        const int ep = tid % EP, jg = tid / EP;   // 256 / EP row groups
+        constexpr int NG = 256 / EP;
+        bool range_ok = true;
+        for (int ip = 0; ip < c_q; ++ip) {
+            __half *dst = kf + (((size_t)bh * c_q + ip) * Tp + j0) * D;
+            for (int jr = jg; jr < kProRows; jr += NG) {
+                float a0 = 0.f, a1 = 0.f;
+                for (int jj = 0; jj < c_k; ++jj) {
+                    const float t = th[ip * c_k + jj];
+                    const float *kr = ks + (kProKLo + jr - (jj - R)) * D + 2 * ep;
+                    a0 = fmaf(t, kr[0], a0);
+                    a1 = fmaf(t, kr[1], a1);
+                }
+                a0 *= scale;
+                a1 *= scale;
+                range_ok &= fabsf(a0) <= 65504.f && fabsf(a1) <= 65504.f;
+                *(__half2 *)(dst + (size_t)jr * D + 2 * ep) = __floats2half2_rn(a0, a1);
+            }
+        }
+        if (!range_ok) atomicOr(&g_fused_error, kErrRange);
+    }
+    // (b) permuted query rows of this block: atom a, row s <- q_{j0-(c_q-1)+a+16s}
+    {
+        const int NA = q_atoms(c_q);
+        __half *dst = qp + ((size_t)bh * (Tp / kBM) + blk) * (size_t)NA * 8 * D;
+        bool range_ok = true;
+        for (int idx = tid; idx < NA * 8 * D; idx += 256) {
+            int row = idx / D, e = idx % D;
+            int a = row / 8, s = row % 8;
+            int i = j0 - (c_q - 1) + a + 16 * s;       // in [j0 - 7, j0 + 127]
+            const float x = qs[(i - (j0 - kProQLo)) * D + e];
+            range_ok &= fabsf(x) <= 65504.f;
+            dst[idx] = __float2half_rn(x);
+        }
+        if (!range_ok) atomicOr(&g_fused_error, kErrRange);
+    }
+    // (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in [1, D_m],
+    //     zero when r + delta >= T (those keys are zero padding in Kf too)
+    const int Dm = d_m(c_q, c_k);
+    for (int idx = tid; idx < QR * Dm; idx += 256) {
+        int rr = idx / Dm, dl = idx % Dm + 1;
+        int r = j0 - kProQLo + rr, c = r + dl;
+        float acc = 0.f;
+        if (r >= 0 && c < T) {
+            const float *qr = qs + rr * D;
+            const float *kc = ks + (c - (j0 - kProKLo)) * D;
+#pragma unroll 8
+            for (int e = 0; e < D; ++e) acc = fmaf(qr[e], kc[e], acc);
+        }
+        fs[rr * kCorrW + dl - 1] = acc * scale;
+    }
+    __syncthreads();
+    // (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
+    //     r = i - i' >= 0 of theta[i'][j'] F[r][delta]
+    for (int idx = tid; idx < kProRows * kCorrW; idx += 256) {
+        int ir = idx / kCorrW, e = idx % kCorrW;
+        int i = j0 + ir;
+        float acc = 0.f;
+        if (e < Dm) {
+            for (int ip = 0; ip < c_q; ++ip) {
+                int r = i - ip;
+                if (r < 0) continue;
+                for (int jj = 0; jj < c_k; ++jj) {
+                    int jp = jj - c_k / 2;
+                    int dl = ip - jp - e;
+                    if (dl < 1) continue;
+                    acc = fmaf(th[ip * c_k + jj], fs[(r - (j0 - kProQLo)) * kCorrW + dl - 1], acc);
+                }
+            }
+        }
+        corr[((size_t)bh * Tp + i) * kCorrW + e] = acc;
+    }
+}
+
+size_t prologue_smem_bytes(int D)
+{
+    return sizeof(float) * ((size_t)(kProKLo + kProRows + kProKHi) * D +
+                            (size_t)(kProQLo + kProRows) * D + (kProQLo + kProRows) * kCorrW +
+                            8 * 15);
+}
+
+// ------------------------------------------------------------ main kernel
+
+template <int D>
+struct FusedCfg {
+    static constexpr int kChunks = D / 64;                  // 64-element (128-B) column chunks
+    static constexpr int kStageBytes = kBN * D * 2;         // one Kf or V tile
+    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kMaxAtoms = 23;                    // q_atoms(8)
+    static constexpr int kQChunkBytes = kMaxAtoms * 1024;
+    static constexpr int kOffRing = kChunks * kQChunkBytes;
+    static constexpr int kOffP = kOffRing + kStages * kStageBytes;
+    static constexpr int kOffCorr = kOffP + kBM * kBN * 2;
+    static constexpr int kOffBar = kOffCorr + kBM * kCorrW * 4;
+    static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Bounded wait: false when the budget ran out (the CTA's abort flag and the
+// device error word are then set) or another role already aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         long long budget = kWaitBudget)
+{
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > budget) {
+            *abort_flag = 1;
+            atomicOr(&g_fused_error, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Grid (query blocks, H, B); block 192 threads = warp 0 TMA producer,
+// warp 1 MMA issuer (and TMEM owner), warps 2..5 softmax / epilogue (one TMEM
+// lane, i.e. one query row, per thread).  TMEM columns: S double buffer at
+// 0 and 128, U^{h,h'} for the c_h output heads from 256.
+template <int D, int CH>
+__global__ void __launch_bounds__(192, 1)
+k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+            const __grid_constant__ CUtensorMap mapV, const float *__restrict__ corr,
+            const float *__restrict__ w_head, float *__restrict__ part, int T, int Tp, int H,
+            int c_q, int nqb)
+{
+    using C = FusedCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sQ = base;
+    uint8_t *ring = base + C::kOffRing;
+    uint8_t *sP = base + C::kOffP;
+    float *sCorr = (float *)(base + C::kOffCorr);
+    uint64_t *bar_q = (uint64_t *)(base + C::kOffBar);
+    uint64_t *full = bar_q + 1;
+    uint64_t *empty = full + C::kStages;
+    uint64_t *s_full = empty + C::kStages;
+    uint64_t *s_free = s_full + 2;
+    uint64_t *p_full = s_free + 2;
+    uint64_t *pv_done = p_full + 1;
+    uint64_t *mma_drain = pv_done + 1;
+    uint64_t *scr_bar = mma_drain + 1;
+    uint32_t *tmem_slot = (uint32_t *)(scr_bar + 1);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int qb = nqb - 1 - (int)blockIdx.x;     // longest rows first
+    const int hs = blockIdx.y, b = blockIdx.z;
+    const int g = hs / CH, hl = hs % CH;
+    const int bh = b * H + hs;
+    const int i0 = qb * kBM;
+    const int ntiles = qb + 1;
+    const int NA = q_atoms(c_q);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar_q, 1);
+        for (int s = 0; s < C::kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
+        tc::mbar_init(&s_full[0], 1); tc::mbar_init(&s_full[1], 1);
+        tc::mbar_init(&s_free[0], 4); tc::mbar_init(&s_free[1], 4);
+        tc::mbar_init(p_full, 4);
+        tc::mbar_init(pv_done, 1);
+        tc::mbar_init(mma_drain, 1);
+        tc::mbar_init(scr_bar, 4);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) { tc::tmem_alloc(tmem_slot, 512); tc::tmem_relinquish(); }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            tc::prefetch_tmap(&mapQ); tc::prefetch_tmap(&mapK); tc::prefetch_tmap(&mapV);
+            tc::mbar_arrive_expect_tx(bar_q, C::kChunks * NA * 8 * 128);
+            for (int c = 0; c < C::kChunks; ++c)
+                tc::tma_load_3d(sQ + c * C::kQChunkBytes, &mapQ, bar_q, 64 * c, qb * NA * 8, bh);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_phase[C::kStages];
+            bool issued[C::kStages];
+            for (int s = 0; s < C::kStages; ++s) issued[s] = false;
+            bool ok = true;
+            auto load = [&](const CUtensorMap *map, int y, int z) -> bool {
+                if (!wait_bar(&empty[stage], phase ^ 1, abort_flag)) return false;
+                tc::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+                for (int c = 0; c < C::kChunks; ++c)
+                    tc::tma_load_3d(ring + stage * C::kStageBytes + c * (kBN * 128), map, &full[stage],
+                                    64 * c, y, z);
+                issued[stage] = true;
+                issued_phase[stage] = phase;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                return true;
+            };
+            auto load_v = [&](int u) -> bool {
+                for (int hh = 0; hh < CH && ok; ++hh) ok = load(&mapV, u * kBN, b * H + g * CH + hh);
+                return ok;
+            };
+            for (int t = 0; t < ntiles && ok; ++t) {
+                for (int ip = 0; ip < c_q && ok; ++ip) ok = load(&mapK, t * kBN, bh * c_q + ip);
+                if (ok && t > 0) load_v(t - 1);
+            }
+            if (ok) load_v(ntiles - 1);
+            // every copy this thread started lands before the CTA may exit
+            tc::mbar_wait(bar_q, 0, kWaitBudget);
+            for (int s = 0; s < C::kStages; ++s)
+                if (issued[s]) tc::mbar_wait(&full[s], issued_phase[s], kWaitBudget);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            const uint32_t idq = tc::idesc_f16(kBM, kBN, false, false);
+            const uint32_t idv = tc::idesc_bf16(kBM, D, false, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = wait_bar(bar_q, 0, abort_flag);
+            tc::tc_fence_after();
+            auto issue_pv = [&](int u) -> bool {
+                if (!wait_bar(p_full, u & 1, abort_flag)) return false;
+                tc::tc_fence_after();
+                for (int hh = 0; hh < CH; ++hh) {
+                    if (!wait_bar(&full[stage], phase, abort_flag)) return false;
+                    tc::tc_fence_after();
+                    const uint8_t *vt = ring + stage * C::kStageBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32), 16, 1024);
+                        uint64_t bd = tc::sdesc_sw128(tc::smem_u32(vt + kk * 2048), kBN * 128, 1024);
+                        tc::mma_bf16(tm + 256 + hh * D, ad, bd, idv, (u > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&empty[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                }
+                tc::mma_commit(pv_done);
+                return true;
+            };
+            for (int t = 0; t < ntiles && ok; ++t) {
+                const int sb = t & 1;
+                if (t >= 2) {
+                    ok = wait_bar(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag);
+                    tc::tc_fence_after();
+                }
+                for (int ip = 0; ip < c_q && ok; ++ip) {
+                    ok = wait_bar(&full[stage], phase, abort_flag);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    const uint32_t aoff = (uint32_t)(c_q - 1 - ip) * 1024u;
+                    const uint8_t *kt = ring + stage * C::kStageBytes;
+#pragma unroll
+                    for (int c = 0; c < C::kChunks; ++c)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sQ + c * C::kQChunkBytes + aoff + kk * 32), 16, 1024);
+                            uint64_t bd = tc::sdesc_sw128(tc::smem_u32(kt + c * (kBN * 128) + kk * 32), 16, 1024);
+                            tc::mma_bf16(tm + sb * kBN, ad, bd, idq, (ip | c | kk) ? 1u : 0u);
+                        }
+                    tc::mma_commit(&empty[stage]);
+                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc::mma_commit(&s_full[sb]);
+                if (t > 0) ok = issue_pv(t - 1);
+            }
+            if (ok) issue_pv(ntiles - 1);
+            // all MMAs this thread issued complete before TMEM is released
+            tc::mma_commit(mma_drain);
+            tc::mbar_wait(mma_drain, 0, kWaitBudget);
+        }
+    } else {
+        // ---------------- softmax and epilogue: thread = TMEM lane = one query row
+        const int q4 = warp & 3;                       // lane quarter this warp may access
+        const int r = q4 * 32 + lane;
+        const int i_row = i0 + 16 * (r & 7) + (r >> 3);   // permuted row order of the Q operand
+        const uint32_t lane_base = tm + ((uint32_t)(q4 * 32) << 16);
+        float *crow = sCorr + r * kCorrW;
+        {
+            const float4 *src = (const float4 *)(corr + ((size_t)bh * Tp + i_row) * kCorrW);
+#pragma unroll
+            for (int u = 0; u < kCorrW / 4; ++u) ((float4 *)crow)[u] = src[u];
+        }
+        float m_run = -INFINITY, l = 0.f;
+        bool ok = true;
+        int band_tiles = 0;
+        for (int t = 0; t < ntiles; ++t) {
+            const int sb = t & 1;
+            ok = __all_sync(0xffffffffu, wait_bar(&s_full[sb], (t >> 1) & 1, abort_flag));
+            if (!ok) break;
+            tc::tc_fence_after();
+            float s[kBN];
+#pragma unroll
+            for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&s_free[sb]);
+            const int j0 = t * kBN;
+            // Band tiles (the diagonal tile and the one before it): causal -inf
+            // mask, and the Mask_0 correction of the D_m (< kCorrW) diagonals
+            // below the main one.  The correction column depends on the row, so
+            // the chunks it touches go through a per-thread scratch row in the
+            // P~ buffer, idle once PV(t-1) has completed.
+            bool pv_waited = false;
+            if (t >= ntiles - 2) {
+                const int bse = i_row - j0;        // column of key i_row (>= 128 before the diagonal)
+                if (t == ntiles - 1) {
+#pragma unroll
+                    for (int c = 0; c < kBN; ++c) s[c] = (c > bse) ? -INFINITY : s[c];
+                }
+                if (t > 0) {
+                    ok = __all_sync(0xffffffffu, wait_bar(pv_done, (t - 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    pv_waited = true;
+                }
+                float *scr = (float *)sP + r * 33;
+#pragma unroll
+                for (int k = 0; k < kBN / 32; ++k) {
+                    if (32 * k <= bse && 32 * k + 31 >= bse - (kCorrW - 1)) {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) scr[x] = s[32 * k + x];
+#pragma unroll
+                        for (int e = 0; e < kCorrW; ++e) {
+                            const int col = bse - e - 32 * k;
+                            if (col >= 0 && col < 32) scr[col] -= crow[e];
+                        }
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) s[32 * k + x] = scr[x];
+                    }
+                }
+                // every softmax warp is done with its scratch rows before any
+                // P~ row overwrites them (bounded wait, like every other)
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(scr_bar);
+                ok = __all_sync(0xffffffffu, wait_bar(scr_bar, band_tiles & 1, abort_flag));
+                ++band_tiles;
+                if (!ok) break;
+            }
+            float mt = s[0];
+#pragma unroll
+            for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+            // the running max moves only when it grows by more than 2^8 in scale
+            const bool need = mt > m_run + 8.f;
+            const float m_new = need ? mt : m_run;
+            const float alpha = ex2(m_run - m_new);
+            if (t > 0) {
+                if (!pv_waited) {
+                    ok = __all_sync(0xffffffffu, wait_bar(pv_done, (t - 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                }
+                if (__any_sync(0xffffffffu, need)) {
+                    const float f = need ? alpha : 1.f;
+#pragma unroll
+                    for (int hh = 0; hh < CH; ++hh)
+#pragma unroll
+                        for (int j = 0; j < D / 32; ++j) {
+                            uint32_t u[32];
+                            const uint32_t a = lane_base + 256 + hh * D + 32 * j;
+                            tc::tmem_ld32(a, u);
+                            tc::tmem_ld_wait();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
+                            tc::tmem_st32(a, u);
+                        }
+                    tc::tmem_st_wait();
+                }
+            }
+            l *= alpha;
+            m_run = m_new;
+#pragma unroll
+            for (int c0 = 0; c0 < kBN; c0 += 8) {
+                float p[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) { p[x] = ex2(s[c0 + x] - m_run); l += p[x]; }
+                uint4 pk = make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
+                                      pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+                *(uint4 *)(sP + (c0 >> 6) * (kBM * 128) + tc::sw128_offset(r, c0 & 63)) = pk;
+            }
+            tc::fence_async_shared();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(p_full);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, wait_bar(pv_done, (ntiles - 1) & 1, abort_flag));
+        if (ok) {
+            tc::tc_fence_after();
+            const float inv_l = 1.f / l;
+#pragma unroll
+            for (int hh = 0; hh < CH; ++hh) {
+                const float coef = w_head[((size_t)g * CH + hh) * CH + hl] * inv_l;
+                float *dst = part + (((size_t)b * T + i_row) * H + (g * CH + hh)) * (size_t)(CH * D) + hl * D;
+#pragma unroll
+                for (int j = 0; j < D / 32; ++j) {
+                    uint32_t u[32];
+                    tc::tmem_ld32(lane_base + 256 + hh * D + 32 * j, u);
+                    tc::tmem_ld_wait();
+                    if (i_row < T) {
+#pragma unroll
+                        for (int x = 0; x < 32; x += 4)
+                            *(float4 *)(dst + 32 * j + x) = make_float4(
+                                __uint_as_float(u[x]) * coef, __uint_as_float(u[x + 1]) * coef,
+                                __uint_as_float(u[x + 2]) * coef, __uint_as_float(u[x + 3]) * coef);
+                    }
+                }
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tm, 512);
+    }
+}
+
+// One thread waits, with the fused kernels' bounded wait, on a barrier that
+// expects an arrival nobody makes; the wait gives up after `budget` cycles.
+__global__ void k_selftest_wait_timeout(long long budget)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    tc::mbar_init(&bar, 1);
+    abort_flag = 0;
+    tc::fence_barrier_init();
+    wait_bar(&bar, 0, &abort_flag, budget);
+}
+
+// ------------------------------------------------------------ mix + GroupNorm
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// One CTA per (query row i, batch b); warp w handles heads w, w+4, ...:
+// O^h = sum_{h'} part[b][i][h][h'], then GroupNorm over the head's d values
+// (mean and biased variance by warp shuffles), affine, depth scale.
+template <int D, int CH>
+__global__ void __launch_bounds__(128)
+k_mix_groupnorm(const float *__restrict__ part, const float *__restrict__ gn_weight,
+                const float *__restrict__ gn_bias, float depth_scale, float eps,
+                __nv_bfloat16 *__restrict__ out, int T, int H)
+{
+    const int i = blockIdx.x, b = blockIdx.y;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    constexpr int PER = D / 32;
+    for (int h = warp; h < H; h += 4) {
+        const float *src = part + (((size_t)b * T + i) * H + h) * (size_t)(CH * D);
+        float o[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            float acc = 0.f;
+#pragma unroll
+            for (int hs = 0; hs < CH; ++hs) acc += src[hs * D + lane + 32 * u];
+            o[u] = acc;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) sum += o[u];
+        const float mean = warp_sum(sum) / D;
+        float sq = 0.f;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) sq += (o[u] - mean) * (o[u] - mean);
+        const float inv = 1.f / sqrtf(warp_sum(sq) / D + eps);
+        __nv_bfloat16 *dst = out + ((size_t)b * T + i) * ((size_t)H * D) + (size_t)h * D;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int e = lane + 32 * u, ch = h * D + e;
+            dst[e] = __float2bfloat16_rn(depth_scale * ((o[u] - mean) * inv * gn_weight[ch] + gn_bias[ch]));
+        }
+    }
+}
+
+// ------------------------------------------------------------ host side
+
+struct FusedLayout {
+    int Tp, nqb, NA;
+    size_t off_kf, off_qp, off_corr, off_part, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+FusedLayout fused_layout(const mta_shape &s)
+{
+    FusedLayout L;
+    L.Tp = (s.T + kBM - 1) / kBM * kBM;
+    L.nqb = L.Tp / kBM;
+    L.NA = q_atoms(s.c_q);
+    const size_t BH = (size_t)s.B * s.H;
+    size_t off = 0;
+    L.off_kf = off;   off += align256(BH * s.c_q * L.Tp * s.d * 2);
+    L.off_qp = off;   off += align256(BH * L.nqb * L.NA * 8 * s.d * 2);
+    L.off_corr = off; off += align256(BH * L.Tp * kCorrW * 4);
+    L.off_part = off; off += align256((size_t)s.B * s.T * s.H * s.c_h * s.d * 4);
+    L.total = off;
+    return L;
+}
+
+const char *const kFusedNames[3] = {"k_fold_prologue", "k_mta_fused", "k_mix_groupnorm"};
+
+template <int D, int CH>
+mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
+                          const Trace &tr)
+{
+    using C = FusedCfg<D>;
+    const FusedLayout L = fused_layout(s);
+    uint8_t *w = (uint8_t *)ws;
+    __half *kf = (__half *)(w + L.off_kf);
+    __half *qp = (__half *)(w + L.off_qp);
+    float *corr = (float *)(w + L.off_corr);
+    float *part = (float *)(w + L.off_part);
+    const uint64_t BH = (uint64_t)s.B * s.H;
+    CUtensorMap mQ, mK, mV;
+    {
+        uint64_t dims[3] = {(uint64_t)D, (uint64_t)L.nqb * L.NA * 8, BH};
+        uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)L.nqb * L.NA * 8 * D * 2};
+        uint32_t box[3] = {64, (uint32_t)(L.NA * 8), 1};
+        if (!make_tmap_f16(&mQ, qp, 3, dims, strides, box)) return MTA_ERR_CUDA;
+    }
+    {
+        uint64_t dims[3] = {(uint64_t)D, (uint64_t)L.Tp, BH * s.c_q};
+        uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)L.Tp * D * 2};
+        uint32_t box[3] = {64, (uint32_t)kBN, 1};
+        if (!make_tmap_f16(&mK, kf, 3, dims, strides, box)) return MTA_ERR_CUDA;
+    }
+    {
+        uint64_t dims[3] = {(uint64_t)D, (uint64_t)s.T, BH};
+        uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)s.T * D * 2};
+        uint32_t box[3] = {64, (uint32_t)kBN, 1};
+        if (!make_tmap_bf16(&mV, a.v, 3, dims, strides, box)) return MTA_ERR_CUDA;
+    }
+    const size_t pro_smem = prologue_smem_bytes(D);
+    if (cudaFuncSetAttribute(k_fold_prologue<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)pro_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(k_mta_fused<D, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+        return MTA_ERR_CUDA;
+    const float scale = kLog2e / sqrtf((float)D);
+    tr.before(0, st);
+    k_fold_prologue<D><<<dim3(L.nqb, (unsigned)BH), 256, pro_smem, st>>>(
+        (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, kf, qp, corr, s.T, L.Tp,
+        s.H, s.c_q, s.c_k, scale);
+    tr.after(0, st);
+    tr.before(1, st);
+    k_mta_fused<D, CH><<<dim3(L.nqb, s.H, s.B), 192, C::kSmemBytes, st>>>(
+        mQ, mK, mV, corr, a.w_head, part, s.T, L.Tp, s.H, s.c_q, L.nqb);
+    tr.after(1, st);
+    tr.before(2, st);
+    k_mix_groupnorm<D, CH><<<dim3(s.T, s.B), 128, 0, st>>>(part, a.gn_weight, a.gn_bias,
+                                                         a.depth_scale, s.gn_eps,
+                                                         (__nv_bfloat16 *)a.out, s.T, s.H);
+    tr.after(2, st);
+    return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+}
+
+}  // namespace
+
+bool fused_supported(const mta_shape &s)
+{
+    if (s.io != MTA_BF16) return false;
+    if (s.d != 64 && s.d != 128) return false;
+    if (!(s.c_h == 1 || s.c_h == 2 || s.c_h == 4) || s.c_h * s.d > 256) return false;
+    if (s.c_q > 8 || s.c_k > 15 || d_m(s.c_q, s.c_k) > kCorrW) return false;
+    return true;
+}
+
+size_t fused_workspace_bytes(const mta_shape &s) { return fused_layout(s).total; }
+
+int fused_kernel_count(const mta_shape &) { return 3; }
+
+const char *fused_kernel_name(const mta_shape &, int index)
+{
+    return (index >= 0 && index < 3) ? kFusedNames[index] : nullptr;
+}
+
+mta_status launch_fused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
+                        const Trace &tr)
+{
+    if (s.d == 128) {
+        if (s.c_h == 1) return launch_fused_t<128, 1>(s, a, ws, st, tr);
+        if (s.c_h == 2) return launch_fused_t<128, 2>(s, a, ws, st, tr);
+    } else {
+        if (s.c_h == 1) return launch_fused_t<64, 1>(s, a, ws, st, tr);
+        if (s.c_h == 2) return launch_fused_t<64, 2>(s, a, ws, st, tr);
+        if (s.c_h == 4) return launch_fused_t<64, 4>(s, a, ws, st, tr);
+    }
     return MTA_ERR_UNSUPPORTED;
 }
-unsigned int fused_take_error() { return 0; }
+
+mta_status launch_selftest_wait_timeout(long long budget_cycles, cudaStream_t st)
+{
+    k_selftest_wait_timeout<<<1, 1, 0, st>>>(budget_cycles);
+    return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+}
+
+unsigned int fused_take_error()
+{
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fused_error, sizeof(v)) != cudaSuccess) return 0;
+    if (v) {
+        unsigned int z = 0;
+        cudaMemcpyToSymbol(g_fused_error, &z, sizeof(z));
+    }
+    return v;
+}
 
 }  // namespace mta

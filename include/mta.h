@@ -67,7 +67,8 @@ typedef enum {
     MTA_ERR_ALIGNMENT = -3,      /* pointer not 16-byte (workspace: 256-byte) aligned */
     MTA_ERR_WORKSPACE = -4,      /* workspace smaller than the *_workspace_size query */
     MTA_ERR_CUDA = -5,           /* a CUDA runtime call failed */
-    MTA_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait expired */
+    MTA_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
+    MTA_ERR_RANGE = -7           /* the fused path met q or folded-key values beyond fp16 range */
 } mta_status;
 
 typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
@@ -110,8 +111,10 @@ MTA_API size_t mta_workspace_size(const mta_shape *shape);
 MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
 
 /* The MTA forward S1..S9 above, out = depth_scale * GN(...), written to out.
- * The bf16 fused path computes the folded logits and P V on tensor cores with
- * bf16 operands and fp32 accumulation; the materialised path computes in fp32.
+ * The fused path computes the folded logits on tensor cores with fp16
+ * operands (q and the folded keys, |x| <= 65504, else the call's next
+ * mta_sync_status() reports MTA_ERR_RANGE) and P V with bf16 operands, both
+ * with fp32 accumulation; the materialised path computes in fp32.
  * The workspace is scratch owned by the caller for the duration of the
  * enqueued work; its contents on entry are ignored. */
 MTA_API mta_status mta_forward(const mta_shape *shape, const void *q, const void *k, const void *v,
@@ -157,9 +160,19 @@ MTA_API mta_status mta_forward_traced(int unfused, const mta_shape *shape, const
                                       void *workspace, size_t workspace_bytes, void *stream,
                                       void *const *events, int n_events);
 
-/* Synchronises `stream`, then reports (and clears) the device error flag set
- * by a kernel whose bounded wait expired: MTA_ERR_DEVICE_TIMEOUT in that case,
- * MTA_ERR_CUDA if the synchronisation itself failed, MTA_OK otherwise. */
+/* Diagnostic for the timeout path: enqueues one single-thread kernel that
+ * waits on a shared-memory barrier nothing ever completes, with the same
+ * bounded wait the fused kernels use, cut off after `budget_cycles` SM clock
+ * cycles (must be in (0, 2^31)).  The kernel then raises the device error
+ * flag and returns, so the next mta_sync_status() reports
+ * MTA_ERR_DEVICE_TIMEOUT (and clears the flag) while the CUDA context stays
+ * usable. */
+MTA_API mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stream);
+
+/* Synchronises `stream`, then reports (and clears) the device error flags:
+ * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
+ * the fused path met a value outside fp16 range, MTA_ERR_CUDA if the
+ * synchronisation itself failed, MTA_OK otherwise. */
 MTA_API mta_status mta_sync_status(void *stream);
 
 #ifdef __cplusplus

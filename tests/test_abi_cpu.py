@@ -95,3 +95,26 @@ def test_debug_attention_argument_checks(L):
 def test_unfused_workspace_is_two_fp32_maps(L):
     s = shape()
     assert mta.mta_unfused_workspace_size(s) == 2 * 4 * 2 * 4 * 64 * 64
+
+
+@pytest.mark.parametrize("kw,path", [
+    (dict(B=2, H=16, T=4096, d=128, c_q=6, c_k=11, c_h=2), 0),     # the benchmark workload
+    (dict(B=1, H=16, T=16384, d=128, c_q=8, c_k=15, c_h=2), 0),
+    (dict(B=8, H=4, T=256, d=64, c_q=4, c_k=15, c_h=2), 0),
+    (dict(B=1, H=16, T=64, d=64, c_q=2, c_k=3, c_h=4), 0),
+    (dict(B=1, H=16, T=16384, d=128, c_q=6, c_k=11, c_h=4), 1),    # c_h * d > 256
+    (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2), 1),        # d not 64 or 128
+    (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2, io="f32"), 1),
+    (dict(B=1, H=4, T=128, d=128, c_q=6, c_k=11, c_h=2, io="f32"), 1),
+])
+def test_forward_path_selection(L, kw, path):
+    s = shape(**kw)
+    assert mta.mta_forward_path(s) == path
+    assert mta.mta_kernel_count(s) == (3 if path == 0 else 4)
+    names = [mta.mta_kernel_name(s, i) for i in range(mta.mta_kernel_count(s))]
+    assert ("k_mta_fused" in names) == (path == 0)
+
+
+def test_selftest_rejects_bad_budget(L):
+    assert L.mta_selftest_wait_timeout(0, None) == -1
+    assert L.mta_selftest_wait_timeout(1 << 31, None) == -1
