@@ -25,7 +25,7 @@ STATUS = {0: "MTA_OK", -1: "MTA_ERR_INVALID_ARG", -2: "MTA_ERR_UNSUPPORTED",
 EXPORTS = ("mta_version", "mta_status_string", "mta_forward_path", "mta_workspace_size",
            "mta_unfused_workspace_size", "mta_forward", "mta_forward_unfused",
            "mta_debug_attention", "mta_kernel_count", "mta_kernel_name", "mta_forward_traced",
-           "mta_selftest_wait_timeout", "mta_sync_status")
+           "mta_selftest_wait_timeout", "mta_forward_noalloc", "mta_sync_status")
 
 
 class MtaShape(ctypes.Structure):
@@ -79,6 +79,8 @@ def lib():
         L.mta_forward_traced.restype = ctypes.c_int
         L.mta_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
         L.mta_selftest_wait_timeout.restype = ctypes.c_int
+        L.mta_forward_noalloc.argtypes = [sp, vp, vp, vp, fp, fp, fp, fp, ctypes.c_float, vp, vp]
+        L.mta_forward_noalloc.restype = ctypes.c_int
         _lib = L
     return _lib
 

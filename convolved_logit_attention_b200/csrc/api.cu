@@ -130,6 +130,23 @@ mta_status mta_forward_unfused(const mta_shape *s, const void *q, const void *k,
                               workspace, workspace_bytes, stream, nullptr, 0);
 }
 
+mta_status mta_forward_noalloc(const mta_shape *s, const void *q, const void *k, const void *v,
+                               const float *w_kq, const float *w_head, const float *gn_weight,
+                               const float *gn_bias, float depth_scale, void *out, void *stream)
+{
+    mta_status rc = check_shape(s);
+    if (rc == MTA_OK) rc = check_tensors(q, k, v, w_kq, w_head, gn_weight, gn_bias, out);
+    if (rc != MTA_OK) return rc;
+    if (!mta::fused_supported(*s)) return MTA_ERR_UNSUPPORTED;
+    if (mta::fused_workspace_bytes(*s) > (size_t)MTA_NOALLOC_SCRATCH_BYTES) return MTA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    rc = mta::noalloc_scratch(&scratch);
+    if (rc != MTA_OK) return rc;
+    mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out};
+    const mta::Trace none;
+    return mta::launch_fused(*s, a, scratch, (cudaStream_t)stream, none);
+}
+
 int mta_kernel_count(const mta_shape *s, int unfused)
 {
     if (check_shape(s) != MTA_OK) return 0;

@@ -36,6 +36,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "mta_internal.h"
 #include "tc_util.cuh"
 #include "tmap.h"
@@ -711,6 +713,28 @@ mta_status launch_selftest_wait_timeout(long long budget_cycles, cudaStream_t st
 {
     k_selftest_wait_timeout<<<1, 1, 0, st>>>(budget_cycles);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+}
+
+// Scratch of mta_forward_noalloc: a file-scope device array, one per device
+// that loads the library.  Host code sees only a stand-in symbol; its device
+// address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MTA_NOALLOC_SCRATCH_BYTES];
+
+mta_status noalloc_scratch(void **ptr)
+{
+    constexpr int kMaxDevices = 64;
+    static void *addr[kMaxDevices] = {};
+    static std::mutex lock;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTA_ERR_CUDA;
+    std::lock_guard<std::mutex> guard(lock);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MTA_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return MTA_OK;
 }
 
 unsigned int fused_take_error()

@@ -169,6 +169,35 @@ MTA_API mta_status mta_forward_traced(int unfused, const mta_shape *shape, const
  * usable. */
 MTA_API mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stream);
 
+/* Bytes of the static device scratch mta_forward_noalloc works in. */
+#define MTA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* mta_forward for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is a convenience of the interface, not of the
+ * method.  Some callers are handed only their input and output buffers and
+ * have no way to obtain scratch, for example a plugin whose host framework
+ * owns every device allocation, or an application that reserves all of its
+ * device memory up front and forbids allocations afterwards.  This entry
+ * takes the same arguments as mta_forward minus the workspace and runs the
+ * same fused kernels in a scratch area that lives inside the library: a
+ * MTA_NOALLOC_SCRATCH_BYTES (32 MiB) device array that every GPU which loads
+ * the library keeps until the process exits.  It allocates nothing and frees
+ * nothing.
+ *   - Shapes whose fused-path scratch (mta_workspace_size) exceeds
+ *     MTA_NOALLOC_SCRATCH_BYTES return MTA_ERR_WORKSPACE; shapes that do not
+ *     take the fused path (mta_forward_path) return MTA_ERR_UNSUPPORTED.
+ *     Nothing is enqueued in either case.
+ *   - The first call on a device looks up the scratch's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one scratch area and leave their data
+ *     in it.  Every byte a call reads there it has written first, so stale
+ *     contents do no harm, but calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on it: serialise them. */
+MTA_API mta_status mta_forward_noalloc(const mta_shape *shape, const void *q, const void *k,
+                                       const void *v, const float *w_kq, const float *w_head,
+                                       const float *gn_weight, const float *gn_bias,
+                                       float depth_scale, void *out, void *stream);
+
 /* Synchronises `stream`, then reports (and clears) the device error flags:
  * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
  * the fused path met a value outside fp16 range, MTA_ERR_CUDA if the

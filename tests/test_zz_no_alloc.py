@@ -1,0 +1,82 @@
+"""mta_forward_noalloc: the forward for callers that cannot allocate device
+memory (a plugin handed only its input and output buffers, an application
+that reserves all device memory up front).  It works in a fixed scratch area
+inside the library instead of a caller workspace.  Called here through the C
+ABI and compared with mta_forward, the entry that takes a workspace.
+
+This file is collected last on purpose, and it must also pass when run alone
+in a fresh process (the first call on a device sets up the scratch address).
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import convolved_logit_attention_b200 as mta
+from convolved_logit_attention_b200.workloads import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAXABS, TOL_RELL2 = 2e-2, 5e-3   # the bf16 tolerance of the parity tests
+
+
+def _device_inputs(w, seed):
+    x = make_inputs(w, seed=seed)
+    dev = torch.device("cuda", 0)
+    d = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v")}
+    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
+        d[n] = torch.from_numpy(x[n]).to(dev)
+    return x, d
+
+
+def _noalloc(d, x, out):
+    L = mta.lib()
+    shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"], x["gn_eps"])
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return L.mta_forward_noalloc(ctypes.byref(shape), p(d["q"]), p(d["k"]), p(d["v"]),
+                                 p(d["w_kq"]), p(d["w_head"]), p(d["gn_weight"]),
+                                 p(d["gn_bias"]), ctypes.c_float(x["depth_scale"]), p(out),
+                                 stream)
+
+
+def test_noalloc_matches_forward_on_two_calls_in_a_row():
+    from convolved_logit_attention_b200 import build
+    build.build()
+    w = Workload("noalloc", 4, 4, 384, 128, 6, 11, 2, "bf16", seed=0)
+    shape = mta.make_shape(w.B, w.H, w.T, w.d, w.c_q, w.c_k, w.c_h)
+    assert mta.mta_forward_path(shape) == mta.MTA_PATH_FUSED_TC
+    assert mta.mta_workspace_size(shape) <= 32 << 20
+    for seed in (21, 22):    # the second call runs over the first call's leftovers
+        x, d = _device_inputs(w, seed)
+        ref = mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                              d["gn_bias"], x["depth_scale"], gn_eps=x["gn_eps"])
+        out = torch.full_like(ref, float("nan"))
+        assert _noalloc(d, x, out) == 0
+        mta.mta_sync_status()
+        got = out.float().cpu().numpy().astype(np.float64)
+        want = ref.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all()
+        err = np.abs(got - want)
+        assert err.max() <= TOL_MAXABS
+        assert np.linalg.norm(got - want) / np.linalg.norm(want) <= TOL_RELL2
+
+
+def test_noalloc_rejects_what_it_cannot_hold():
+    # scratch needed beyond the 32 MiB array: MTA_ERR_WORKSPACE
+    big = Workload("big", 4, 16, 2048, 128, 6, 11, 2, "bf16", seed=0)
+    shape = mta.make_shape(big.B, big.H, big.T, big.d, big.c_q, big.c_k, big.c_h)
+    assert mta.mta_workspace_size(shape) > 32 << 20
+    x, d = _device_inputs(Workload("small", 1, 2, 64, 128, 6, 11, 2, "bf16", seed=1), 1)
+    L = mta.lib()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    args = [p(d[n]) for n in ("q", "k", "v", "w_kq", "w_head", "gn_weight", "gn_bias")]
+    out = torch.empty((1, 64, 256), dtype=torch.bfloat16, device="cuda")
+    assert L.mta_forward_noalloc(ctypes.byref(shape), *args, ctypes.c_float(0.8), p(out),
+                                 None) == -4
+    # a shape the fused path does not take (fp32 I/O): MTA_ERR_UNSUPPORTED
+    f32 = mta.make_shape(1, 2, 64, 128, 6, 11, 2, io="f32")
+    assert L.mta_forward_noalloc(ctypes.byref(f32), *args, ctypes.c_float(0.8), p(out),
+                                 None) == -2
+    mta.mta_sync_status()
