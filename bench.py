@@ -54,6 +54,8 @@ def parse_args(argv=None):
     p.add_argument("--path", choices=["forward", "unfused"], default="forward",
                    help="forward: mta_forward (the fused path where supported); "
                         "unfused: mta_forward_unfused (materialised maps)")
+    p.add_argument("--batch", type=int, default=None,
+                   help="override the workload's batch size (smaller cases for profiler captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -436,6 +438,9 @@ def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_setup(args)
     w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        from dataclasses import replace
+        w = replace(w, B=args.batch, name="%s_b%d" % (w.name, args.batch))
     try:
         if args.impl == "reference":
             line = reference_arm(args, w, world, rank)

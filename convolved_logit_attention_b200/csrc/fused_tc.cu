@@ -63,134 +63,198 @@ __host__ __device__ inline int d_m(int c_q, int c_k) { return c_q - 1 + c_k / 2;
 
 // ------------------------------------------------------------ prologue
 
-constexpr int kProRows = 128;
-constexpr int kProKLo = 8;        // k rows loaded before the block
-constexpr int kProKHi = 15;       // k rows loaded after it
-constexpr int kProQLo = 7;        // q rows loaded before the block
+constexpr int kProRows = 128;     // rows (keys and queries) per prologue CTA
+constexpr int kProQLo = 7;        // query rows before the block whose future logits are needed
 
-// One CTA per (128-row block, b*H + h).  Shared memory holds the block's k
-// rows with a halo ([j0-8, j0+143)) and q rows ([j0-7, j0+128)) as fp32.
-template <int D>
-__global__ void __launch_bounds__(256)
+// One CTA per (128-row block, b*H + h), 256 threads, four sections:
+//  (a) Kf^{(i')}_j for the block's keys: thread = one column pair x a run of
+//      RPG consecutive keys.  The k rows the taps reach are loaded once into
+//      registers; theta is zero-padded to CK taps centred like the real
+//      kernel (CK = c_k for the common sizes, 15 otherwise), so every tap
+//      index is a compile-time constant.
+//  (b) the block's query rows in the permuted atom order, converted to fp16.
+//  (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in
+//      [1, D_m], for r in [j0 - 7, j0 + 128), from shared-memory copies of
+//      the rows involved.
+//  (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
+//      r = i - i' >= 0 of theta[i'][j'] F[r][delta].
+template <int D, int CK>
+__global__ void __launch_bounds__(256, 2)
 k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                 const float *__restrict__ w_kq, __half *__restrict__ kf,
                 __half *__restrict__ qp, float *__restrict__ corr, int T, int Tp, int H,
                 int c_q, int c_k, float scale)
 {
-    extern __shared__ __align__(16) float psm[];
-    constexpr int KR = kProKLo + kProRows + kProKHi;
+    constexpr int EP = D / 2;                  // column pairs
+    constexpr int RG = 256 / EP;               // key runs per block
+    constexpr int RPG = kProRows / RG;         // keys per run
+    constexpr int RT = CK / 2, LT = CK - 1 - RT;
     constexpr int QR = kProQLo + kProRows;
-    float *ks = psm;                       // [KR][D]
-    float *qs = ks + KR * D;               // [QR][D]
-    float *fs = qs + QR * D;               // [QR][kCorrW] future logits q_r . k_{r+delta}
-    float *th = fs + QR * kCorrW;          // [c_q][c_k]
+    __shared__ float th[8 * CK];               // zero-padded taps
+    __shared__ float fs[QR * kCorrW];
+    extern __shared__ __align__(16) __nv_bfloat16 qk_sm[];   // section (c) row copies
     const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
     const int j0 = blk * kProRows;
     const int tid = threadIdx.x;
     const size_t head_off = (size_t)bh * T * D;
-    for (int idx = tid; idx < KR * D; idx += 256) {
-        int r = idx / D, e = idx % D, j = j0 - kProKLo + r;
-        ks[idx] = (j >= 0 && j < T) ? __bfloat162float(k[head_off + (size_t)j * D + e]) : 0.f;
+    const int R = c_k / 2, shift = RT - R;     // real tap jj sits at padded index jj + shift
+    for (int idx = tid; idx < 8 * CK; idx += 256) {
+        const int ip = idx / CK, jp = idx % CK - shift;
+        th[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] : 0.f;
     }
-    for (int idx = tid; idx < QR * D; idx += 256) {
-        int r = idx / D, e = idx % D, i = j0 - kProQLo + r;
-        qs[idx] = (i >= 0 && i < T) ? __bfloat162float(q[head_off + (size_t)i * D + e]) : 0.f;
-    }
-    for (int idx = tid; idx < c_q * c_k; idx += 256) th[idx] = w_kq[(size_t)h * c_q * c_k + idx];
     __syncthreads();
 
-    // (a) Kf^{(i')}_j = scale * sum_jj theta[i'][jj] k_{j - (jj - floor(c_k/2))}
+    // (a) folded keys, in windows of SUB consecutive keys
     {
-        const int R = c_k / 2;
-        constexpr int EP = D / 2;                 // element pairs per row
-        const int ep = tid % EP, jg = tid / EP;   // 256 / EP row groups
-        constexpr int NG = 256 / EP;
+        constexpr int SUB = 16;
+        constexpr int WS = SUB + CK - 1;           // window rows
+        const int ep = tid % EP, rg = tid / EP;
         bool range_ok = true;
-        for (int ip = 0; ip < c_q; ++ip) {
-            __half *dst = kf + (((size_t)bh * c_q + ip) * Tp + j0) * D;
-            for (int jr = jg; jr < kProRows; jr += NG) {
-                float a0 = 0.f, a1 = 0.f;
-                for (int jj = 0; jj < c_k; ++jj) {
-                    const float t = th[ip * c_k + jj];
-                    const float *kr = ks + (kProKLo + jr - (jj - R)) * D + 2 * ep;
-                    a0 = fmaf(t, kr[0], a0);
-                    a1 = fmaf(t, kr[1], a1);
+#pragma unroll 1
+        for (int sub = 0; sub < RPG / SUB; ++sub) {
+            const int jr0 = j0 + rg * RPG + sub * SUB;     // first key of the window
+            float2 win[WS];
+#pragma unroll
+            for (int w = 0; w < WS; ++w) {
+                const int row = jr0 - LT + w;
+                float2 v = make_float2(0.f, 0.f);
+                if (row >= 0 && row < T)
+                    v = __bfloat1622float2(*(const __nv_bfloat162 *)(k + head_off + (size_t)row * D + 2 * ep));
+                win[w] = v;
+            }
+            for (int ip = 0; ip < c_q; ++ip) {
+                float t[CK];
+#pragma unroll
+                for (int jj = 0; jj < CK; ++jj) t[jj] = th[ip * CK + jj];
+                __half *dst = kf + (((size_t)bh * c_q + ip) * Tp + jr0) * D + 2 * ep;
+#pragma unroll
+                for (int r = 0; r < SUB; ++r) {
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < CK; ++jj) {
+                        a0 = fmaf(t[jj], win[r + CK - 1 - jj].x, a0);
+                        a1 = fmaf(t[jj], win[r + CK - 1 - jj].y, a1);
+                    }
+                    a0 *= scale;
+                    a1 *= scale;
+                    range_ok &= fabsf(a0) <= 65504.f && fabsf(a1) <= 65504.f;
+                    *(__half2 *)(dst + (size_t)r * D) = __floats2half2_rn(a0, a1);
                 }
-                a0 *= scale;
-                a1 *= scale;
-                range_ok &= fabsf(a0) <= 65504.f && fabsf(a1) <= 65504.f;
-                *(__half2 *)(dst + (size_t)jr * D + 2 * ep) = __floats2half2_rn(a0, a1);
             }
         }
         if (!range_ok) atomicOr(&g_fused_error, kErrRange);
     }
-    // (b) permuted query rows of this block: atom a, row s <- q_{j0-(c_q-1)+a+16s}
+    // (b) permuted query rows: atom a, row s <- q_{j0-(c_q-1)+a+16s}; 8 elements per thread
     {
         const int NA = q_atoms(c_q);
         __half *dst = qp + ((size_t)bh * (Tp / kBM) + blk) * (size_t)NA * 8 * D;
+        constexpr int CPR = D / 8;             // 16-byte chunks per row
         bool range_ok = true;
-        for (int idx = tid; idx < NA * 8 * D; idx += 256) {
-            int row = idx / D, e = idx % D;
-            int a = row / 8, s = row % 8;
-            int i = j0 - (c_q - 1) + a + 16 * s;       // in [j0 - 7, j0 + 127]
-            const float x = qs[(i - (j0 - kProQLo)) * D + e];
-            range_ok &= fabsf(x) <= 65504.f;
-            dst[idx] = __float2half_rn(x);
+        for (int idx = tid; idx < NA * 8 * CPR; idx += 256) {
+            const int row = idx / CPR, c8 = idx % CPR;
+            const int i = j0 - (c_q - 1) + row / 8 + 16 * (row % 8);
+            uint4 outv = make_uint4(0, 0, 0, 0);
+            if (i >= 0 && i < T) {
+                const uint4 in = *(const uint4 *)(q + head_off + (size_t)i * D + 8 * c8);
+                const __nv_bfloat162 *bp = (const __nv_bfloat162 *)&in;
+                __half2 *hp = (__half2 *)&outv;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(bp[u]);
+                    range_ok &= fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
+                    hp[u] = __floats2half2_rn(f.x, f.y);
+                }
+            }
+            *(uint4 *)(dst + (size_t)row * D + 8 * c8) = outv;
         }
         if (!range_ok) atomicOr(&g_fused_error, kErrRange);
     }
-    // (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in [1, D_m],
-    //     zero when r + delta >= T (those keys are zero padding in Kf too)
+    // (c) future logits from shared-memory copies of the rows they need
+    //     (q rows [j0-7, j0+128), k rows [j0-6, j0+142)), one dot product of
+    //     length d per thread at a time; rows are padded by 16 bytes so that
+    //     threads on different rows hit different banks.
     const int Dm = d_m(c_q, c_k);
-    for (int idx = tid; idx < QR * Dm; idx += 256) {
-        int rr = idx / Dm, dl = idx % Dm + 1;
-        int r = j0 - kProQLo + rr, c = r + dl;
-        float acc = 0.f;
-        if (r >= 0 && c < T) {
-            const float *qr = qs + rr * D;
-            const float *kc = ks + (c - (j0 - kProKLo)) * D;
-#pragma unroll 8
-            for (int e = 0; e < D; ++e) acc = fmaf(qr[e], kc[e], acc);
+    {
+        constexpr int RS = D + 8;              // padded row stride in bf16 elements
+        constexpr int KR = QR + kCorrW - 3;    // k rows j0-6 .. j0+141 (r + delta <= j0+127+14)
+        __nv_bfloat16 *qsm = qk_sm;            // [QR][RS]
+        __nv_bfloat16 *ksm = qk_sm + QR * RS;  // [KR][RS]
+        constexpr int CPR = D / 8;
+        for (int idx = tid; idx < (QR + KR) * CPR; idx += 256) {
+            const int row = idx / CPR, c8 = idx % CPR;
+            const bool isq = row < QR;
+            const int g = isq ? j0 - kProQLo + row : j0 - (kProQLo - 1) + (row - QR);
+            const __nv_bfloat16 *src = isq ? q : k;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (g >= 0 && g < T) v = *(const uint4 *)(src + head_off + (size_t)g * D + 8 * c8);
+            *(uint4 *)((isq ? qsm + row * RS : ksm + (row - QR) * RS) + 8 * c8) = v;
         }
-        fs[rr * kCorrW + dl - 1] = acc * scale;
+        __syncthreads();
+        for (int idx = tid; idx < QR * Dm; idx += 256) {
+            const int rr = idx / Dm, dl = idx % Dm + 1;
+            const int r = j0 - kProQLo + rr, c = r + dl;
+            float acc = 0.f;
+            if (r >= 0 && c < T) {
+                const __nv_bfloat16 *qr = qsm + rr * RS;
+                const __nv_bfloat16 *kc = ksm + (rr + dl - 1) * RS;   // k row c = j0-6+(rr+dl-1)
+#pragma unroll 4
+                for (int c8 = 0; c8 < CPR; ++c8) {
+                    const uint4 a4 = *(const uint4 *)(qr + 8 * c8);
+                    const uint4 b4 = *(const uint4 *)(kc + 8 * c8);
+                    const __nv_bfloat162 *a2 = (const __nv_bfloat162 *)&a4;
+                    const __nv_bfloat162 *b2 = (const __nv_bfloat162 *)&b4;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 x = __bfloat1622float2(a2[u]), y = __bfloat1622float2(b2[u]);
+                        acc = fmaf(x.x, y.x, acc);
+                        acc = fmaf(x.y, y.y, acc);
+                    }
+                }
+            }
+            fs[rr * kCorrW + dl - 1] = acc * scale;
+        }
     }
     __syncthreads();
-    // (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
-    //     r = i - i' >= 0 of theta[i'][j'] F[r][delta]
+    // (d) correction table
     for (int idx = tid; idx < kProRows * kCorrW; idx += 256) {
-        int ir = idx / kCorrW, e = idx % kCorrW;
-        int i = j0 + ir;
+        const int ir = idx / kCorrW, e = idx % kCorrW;
+        const int i = j0 + ir;
         float acc = 0.f;
         if (e < Dm) {
             for (int ip = 0; ip < c_q; ++ip) {
-                int r = i - ip;
+                const int r = i - ip;
                 if (r < 0) continue;
-                for (int jj = 0; jj < c_k; ++jj) {
-                    int jp = jj - c_k / 2;
-                    int dl = ip - jp - e;
-                    if (dl < 1) continue;
-                    acc = fmaf(th[ip * c_k + jj], fs[(r - (j0 - kProQLo)) * kCorrW + dl - 1], acc);
-                }
+                // taps with delta = ip - (jj - R) - e >= 1, i.e. jj <= ip + R - e - 1
+                const int jmax = min(c_k - 1, ip + R - e - 1);
+                const float *frow = fs + (r - (j0 - kProQLo)) * kCorrW;
+                const float *trow = th + ip * CK + shift;
+                for (int jj = 0; jj <= jmax; ++jj)
+                    acc = fmaf(trow[jj], frow[ip + R - e - jj - 1], acc);
             }
         }
         corr[((size_t)bh * Tp + i) * kCorrW + e] = acc;
     }
 }
 
+// Dynamic shared memory of the prologue: section (c)'s bf16 copies of
+// 135 query rows and 148 key rows, each padded by 8 elements.
 size_t prologue_smem_bytes(int D)
 {
-    return sizeof(float) * ((size_t)(kProKLo + kProRows + kProKHi) * D +
-                            (size_t)(kProQLo + kProRows) * D + (kProQLo + kProRows) * kCorrW +
-                            8 * 15);
+    const int QR = kProQLo + kProRows;
+    return (size_t)(QR + QR + kCorrW - 3) * (D + 8) * sizeof(__nv_bfloat16);
 }
 
 // ------------------------------------------------------------ main kernel
 
-template <int D>
+// PAIR: two CTAs (consecutive 128-row query blocks of one head) share every
+// MMA as one M = 256 tcgen05 operation; each CTA then loads only half of
+// every key tile (64 keys of Kf, 64 of the d columns of V).
+template <int D, bool PAIR>
 struct FusedCfg {
     static constexpr int kChunks = D / 64;                  // 64-element (128-B) column chunks
-    static constexpr int kStageBytes = kBN * D * 2;         // one Kf or V tile
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kKfRows = PAIR ? kBN / 2 : kBN;    // keys of a Kf tile held by this CTA
+    static constexpr int kStageBytes = PAIR ? kBN * 64 * 2 : kBN * D * 2;
+    static constexpr int kStages = (kStageBytes <= 16384) ? 8 : 4;
     static constexpr int kMaxAtoms = 23;                    // q_atoms(8)
     static constexpr int kQChunkBytes = kMaxAtoms * 1024;
     static constexpr int kOffRing = kChunks * kQChunkBytes;
@@ -231,18 +295,51 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Bounded wait used by every role; in pair mode barriers that the other CTA
+// arrives on are waited on with cluster-scope acquire.
+template <bool PAIR>
+__device__ __forceinline__ bool wait_role(uint64_t *bar, uint32_t parity, volatile int *abort_flag)
+{
+    if constexpr (!PAIR) {
+        return wait_bar(bar, parity, abort_flag);
+    } else {
+        if (tc::mbar_try_wait_cluster(bar, parity)) return true;
+        const long long t0 = clock64();
+        while (true) {
+            if (tc::mbar_try_wait_cluster(bar, parity)) return true;
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitBudget) {
+                *abort_flag = 1;
+                atomicOr(&g_fused_error, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Arrival on a barrier of the MMA-issuing CTA (rank 0 of a pair, or self).
+template <bool PAIR>
+__device__ __forceinline__ void arrive_leader(uint64_t *bar)
+{
+    if constexpr (PAIR) tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(bar), 0));
+    else tc::mbar_arrive(bar);
+}
+
 // Grid (query blocks, H, B); block 192 threads = warp 0 TMA producer,
 // warp 1 MMA issuer (and TMEM owner), warps 2..5 softmax / epilogue (one TMEM
 // lane, i.e. one query row, per thread).  TMEM columns: S double buffer at
 // 0 and 128, U^{h,h'} for the c_h output heads from 256.
-template <int D, int CH>
+// PAIR (d = 128): clusters of two CTAs own query blocks 2p and 2p+1 of one
+// head; rank 0 issues the M = 256 MMAs for both and every completion is
+// multicast to both CTAs' barriers.
+template <int D, int CH, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
 k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
             const __grid_constant__ CUtensorMap mapV, const float *__restrict__ corr,
             const float *__restrict__ w_head, float *__restrict__ part, int T, int Tp, int H,
             int c_q, int nqb)
 {
-    using C = FusedCfg<D>;
+    using C = FusedCfg<D, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sQ = base;
@@ -261,30 +358,44 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     uint32_t *tmem_slot = (uint32_t *)(scr_bar + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
-    const int qb = nqb - 1 - (int)blockIdx.x;     // longest rows first
+    const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    int qb, ntiles;
+    if constexpr (PAIR) {
+        const int pair = nqb / 2 - 1 - (int)(blockIdx.x >> 1);   // longest rows first
+        qb = 2 * pair + (int)rank;
+        ntiles = 2 * pair + 2;        // both CTAs run to the diagonal of block 2p+1
+    } else {
+        qb = nqb - 1 - (int)blockIdx.x;
+        ntiles = qb + 1;
+    }
     const int hs = blockIdx.y, b = blockIdx.z;
     const int g = hs / CH, hl = hs % CH;
     const int bh = b * H + hs;
     const int i0 = qb * kBM;
-    const int ntiles = qb + 1;
     const int NA = q_atoms(c_q);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int consumers = PAIR ? 8 : 4;   // softmax warps that release S and publish P~
 
     if (threadIdx.x == 0) {
         tc::mbar_init(bar_q, 1);
         for (int s = 0; s < C::kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
         tc::mbar_init(&s_full[0], 1); tc::mbar_init(&s_full[1], 1);
-        tc::mbar_init(&s_free[0], 4); tc::mbar_init(&s_free[1], 4);
-        tc::mbar_init(p_full, 4);
+        tc::mbar_init(&s_free[0], consumers); tc::mbar_init(&s_free[1], consumers);
+        tc::mbar_init(p_full, consumers);
         tc::mbar_init(pv_done, 1);
         tc::mbar_init(mma_drain, 1);
         tc::mbar_init(scr_bar, 4);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
-    if (warp == 1) { tc::tmem_alloc(tmem_slot, 512); tc::tmem_relinquish(); }
+    if (warp == 1) {
+        if constexpr (PAIR) { tc::tmem_alloc_pair(tmem_slot, 512); tc::tmem_relinquish_pair(); }
+        else { tc::tmem_alloc(tmem_slot, 512); tc::tmem_relinquish(); }
+    }
     tc::tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) tc::cluster_sync();   // the peer's barriers exist before any remote use
     tc::tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
@@ -292,76 +403,109 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         if (lane == 0) {
             // ---------------- TMA producer
             tc::prefetch_tmap(&mapQ); tc::prefetch_tmap(&mapK); tc::prefetch_tmap(&mapV);
-            tc::mbar_arrive_expect_tx(bar_q, C::kChunks * NA * 8 * 128);
-            for (int c = 0; c < C::kChunks; ++c)
-                tc::tma_load_3d(sQ + c * C::kQChunkBytes, &mapQ, bar_q, 64 * c, qb * NA * 8, bh);
+            const uint32_t q_bytes = C::kChunks * NA * 8 * 128;
+            const uint32_t bq = tc::mapa_shared(tc::smem_u32(bar_q), 0);
+            if (leader) tc::mbar_arrive_expect_tx(bar_q, PAIR ? 2 * q_bytes : q_bytes);
+            for (int c = 0; c < C::kChunks; ++c) {
+                if constexpr (PAIR) tc::tma_load_3d_pair(sQ + c * C::kQChunkBytes, &mapQ, bq, 64 * c, qb * NA * 8, bh);
+                else tc::tma_load_3d(sQ + c * C::kQChunkBytes, &mapQ, bar_q, 64 * c, qb * NA * 8, bh);
+            }
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_phase[C::kStages];
             bool issued[C::kStages];
             for (int s = 0; s < C::kStages; ++s) issued[s] = false;
             bool ok = true;
-            auto load = [&](const CUtensorMap *map, int y, int z) -> bool {
-                if (!wait_bar(&empty[stage], phase ^ 1, abort_flag)) return false;
-                tc::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-                for (int c = 0; c < C::kChunks; ++c)
-                    tc::tma_load_3d(ring + stage * C::kStageBytes + c * (kBN * 128), map, &full[stage],
-                                    64 * c, y, z);
+            // one stage: a Kf tile (kKfRows keys x d) or this CTA's d chunks of a V tile
+            auto load = [&](bool is_k, int y, int z) -> bool {
+                if (!wait_role<PAIR>(&empty[stage], phase ^ 1, abort_flag)) return false;
+                uint8_t *dst = ring + stage * C::kStageBytes;
+                if constexpr (PAIR) {
+                    const uint32_t bf = tc::mapa_shared(tc::smem_u32(&full[stage]), 0);
+                    if (leader) tc::mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+                    if (is_k) {
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tc::tma_load_3d_pair(dst + c * (C::kKfRows * 128), &mapK, bf, 64 * c,
+                                                 y + (int)rank * C::kKfRows, z);
+                    } else {
+                        tc::tma_load_3d_pair(dst, &mapV, bf, 64 * (int)rank, y, z);
+                    }
+                } else {
+                    tc::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tc::tma_load_3d(dst + c * (kBN * 128), is_k ? &mapK : &mapV, &full[stage],
+                                        64 * c, y, z);
+                }
                 issued[stage] = true;
                 issued_phase[stage] = phase;
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
                 return true;
             };
             auto load_v = [&](int u) -> bool {
-                for (int hh = 0; hh < CH && ok; ++hh) ok = load(&mapV, u * kBN, b * H + g * CH + hh);
+                for (int hh = 0; hh < CH && ok; ++hh) ok = load(false, u * kBN, b * H + g * CH + hh);
                 return ok;
             };
             for (int t = 0; t < ntiles && ok; ++t) {
-                for (int ip = 0; ip < c_q && ok; ++ip) ok = load(&mapK, t * kBN, bh * c_q + ip);
+                for (int ip = 0; ip < c_q && ok; ++ip) ok = load(true, t * kBN, bh * c_q + ip);
                 if (ok && t > 0) load_v(t - 1);
             }
             if (ok) load_v(ntiles - 1);
-            // every copy this thread started lands before the CTA may exit
-            tc::mbar_wait(bar_q, 0, kWaitBudget);
-            for (int s = 0; s < C::kStages; ++s)
-                if (issued[s]) tc::mbar_wait(&full[s], issued_phase[s], kWaitBudget);
+            // copies this thread started land before the CTA may exit; in a pair
+            // their completion is counted in the leader, so the peer waits a while
+            if (leader) {
+                tc::mbar_wait(bar_q, 0, kWaitBudget);
+                for (int s = 0; s < C::kStages; ++s)
+                    if (issued[s]) tc::mbar_wait(&full[s], issued_phase[s], kWaitBudget);
+            } else if (!ok) {
+                const long long t0 = clock64();
+                while (clock64() - t0 < (1ll << 22)) { }
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // ---------------- MMA issuer
-            const uint32_t idq = tc::idesc_f16(kBM, kBN, false, false);
-            const uint32_t idv = tc::idesc_bf16(kBM, D, false, true);
+            constexpr int M = PAIR ? 2 * kBM : kBM;
+            const uint32_t idq = tc::idesc_f16(M, kBN, false, false);
+            const uint32_t idv = tc::idesc_bf16(M, D, false, true);
+            auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
+                if constexpr (PAIR) tc::mma_pair(d, ad, bd, id, acc);
+                else tc::mma_bf16(d, ad, bd, id, acc);
+            };
+            auto commit = [&](uint64_t *bar) {
+                if constexpr (PAIR) tc::mma_commit_pair_multicast(bar, 0x3);
+                else tc::mma_commit(bar);
+            };
             int stage = 0;
             uint32_t phase = 0;
-            bool ok = wait_bar(bar_q, 0, abort_flag);
+            bool ok = wait_role<PAIR>(bar_q, 0, abort_flag);
             tc::tc_fence_after();
             auto issue_pv = [&](int u) -> bool {
-                if (!wait_bar(p_full, u & 1, abort_flag)) return false;
+                if (!wait_role<PAIR>(p_full, u & 1, abort_flag)) return false;
                 tc::tc_fence_after();
                 for (int hh = 0; hh < CH; ++hh) {
-                    if (!wait_bar(&full[stage], phase, abort_flag)) return false;
+                    if (!wait_role<PAIR>(&full[stage], phase, abort_flag)) return false;
                     tc::tc_fence_after();
                     const uint8_t *vt = ring + stage * C::kStageBytes;
 #pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk) {
                         uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32), 16, 1024);
                         uint64_t bd = tc::sdesc_sw128(tc::smem_u32(vt + kk * 2048), kBN * 128, 1024);
-                        tc::mma_bf16(tm + 256 + hh * D, ad, bd, idv, (u > 0 || kk > 0) ? 1u : 0u);
+                        mma(tm + 256 + hh * D, ad, bd, idv, (u > 0 || kk > 0) ? 1u : 0u);
                     }
-                    tc::mma_commit(&empty[stage]);
+                    commit(&empty[stage]);
                     if (++stage == C::kStages) { stage = 0; phase ^= 1; }
                 }
-                tc::mma_commit(pv_done);
+                commit(pv_done);
                 return true;
             };
             for (int t = 0; t < ntiles && ok; ++t) {
                 const int sb = t & 1;
                 if (t >= 2) {
-                    ok = wait_bar(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag);
+                    ok = wait_role<PAIR>(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag);
                     tc::tc_fence_after();
                 }
                 for (int ip = 0; ip < c_q && ok; ++ip) {
-                    ok = wait_bar(&full[stage], phase, abort_flag);
+                    ok = wait_role<PAIR>(&full[stage], phase, abort_flag);
                     if (!ok) break;
                     tc::tc_fence_after();
                     const uint32_t aoff = (uint32_t)(c_q - 1 - ip) * 1024u;
@@ -371,19 +515,20 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sQ + c * C::kQChunkBytes + aoff + kk * 32), 16, 1024);
-                            uint64_t bd = tc::sdesc_sw128(tc::smem_u32(kt + c * (kBN * 128) + kk * 32), 16, 1024);
-                            tc::mma_bf16(tm + sb * kBN, ad, bd, idq, (ip | c | kk) ? 1u : 0u);
+                            uint64_t bd = tc::sdesc_sw128(tc::smem_u32(kt + c * (C::kKfRows * 128) + kk * 32), 16, 1024);
+                            mma(tm + sb * kBN, ad, bd, idq, (ip | c | kk) ? 1u : 0u);
                         }
-                    tc::mma_commit(&empty[stage]);
+                    commit(&empty[stage]);
                     if (++stage == C::kStages) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                tc::mma_commit(&s_full[sb]);
+                commit(&s_full[sb]);
                 if (t > 0) ok = issue_pv(t - 1);
             }
             if (ok) issue_pv(ntiles - 1);
             // all MMAs this thread issued complete before TMEM is released
-            tc::mma_commit(mma_drain);
+            if constexpr (PAIR) tc::mma_commit_pair_multicast(mma_drain, 0x1);
+            else tc::mma_commit(mma_drain);
             tc::mbar_wait(mma_drain, 0, kWaitBudget);
         }
     } else {
@@ -403,7 +548,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         int band_tiles = 0;
         for (int t = 0; t < ntiles; ++t) {
             const int sb = t & 1;
-            ok = __all_sync(0xffffffffu, wait_bar(&s_full[sb], (t >> 1) & 1, abort_flag));
+            ok = __all_sync(0xffffffffu, wait_role<PAIR>(&s_full[sb], (t >> 1) & 1, abort_flag));
             if (!ok) break;
             tc::tc_fence_after();
             float s[kBN];
@@ -412,22 +557,24 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             tc::tmem_ld_wait();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&s_free[sb]);
+            if (lane == 0) arrive_leader<PAIR>(&s_free[sb]);
             const int j0 = t * kBN;
-            // Band tiles (the diagonal tile and the one before it): causal -inf
-            // mask, and the Mask_0 correction of the D_m (< kCorrW) diagonals
-            // below the main one.  The correction column depends on the row, so
-            // the chunks it touches go through a per-thread scratch row in the
-            // P~ buffer, idle once PV(t-1) has completed.
+            // Band tiles (this block's diagonal tile and the one before it):
+            // causal -inf mask, and the Mask_0 correction of the D_m (< kCorrW)
+            // diagonals below the main one.  Tiles past the diagonal (the
+            // first block of a pair runs one) are masked entirely.  The
+            // correction column depends on the row, so the chunks it touches go
+            // through a per-thread scratch row in the P~ buffer, idle once
+            // PV(t-1) has completed.
             bool pv_waited = false;
-            if (t >= ntiles - 2) {
+            if (t >= qb - 1) {
                 const int bse = i_row - j0;        // column of key i_row (>= 128 before the diagonal)
-                if (t == ntiles - 1) {
+                if (t >= qb) {
 #pragma unroll
                     for (int c = 0; c < kBN; ++c) s[c] = (c > bse) ? -INFINITY : s[c];
                 }
                 if (t > 0) {
-                    ok = __all_sync(0xffffffffu, wait_bar(pv_done, (t - 1) & 1, abort_flag));
+                    ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
                     if (!ok) break;
                     tc::tc_fence_after();
                     pv_waited = true;
@@ -451,7 +598,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 // P~ row overwrites them (bounded wait, like every other)
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(scr_bar);
-                ok = __all_sync(0xffffffffu, wait_bar(scr_bar, band_tiles & 1, abort_flag));
+                ok = __all_sync(0xffffffffu, wait_role<PAIR>(scr_bar, band_tiles & 1, abort_flag));
                 ++band_tiles;
                 if (!ok) break;
             }
@@ -464,7 +611,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             const float alpha = ex2(m_run - m_new);
             if (t > 0) {
                 if (!pv_waited) {
-                    ok = __all_sync(0xffffffffu, wait_bar(pv_done, (t - 1) & 1, abort_flag));
+                    ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
                     if (!ok) break;
                     tc::tc_fence_after();
                 }
@@ -499,9 +646,9 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             tc::fence_async_shared();
             tc::tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(p_full);
+            if (lane == 0) arrive_leader<PAIR>(p_full);
         }
-        if (ok) ok = __all_sync(0xffffffffu, wait_bar(pv_done, (ntiles - 1) & 1, abort_flag));
+        if (ok) ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (ntiles - 1) & 1, abort_flag));
         if (ok) {
             tc::tc_fence_after();
             const float inv_l = 1.f / l;
@@ -527,9 +674,12 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     }
     tc::tc_fence_before();
     __syncthreads();
+    // in a pair, the leader's MMAs touch both CTAs' TMEM and shared memory
+    if constexpr (PAIR) tc::cluster_sync();
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tm, 512);
+        if constexpr (PAIR) tc::tmem_dealloc_pair(tm, 512);
+        else tc::tmem_dealloc(tm, 512);
     }
 }
 
@@ -605,7 +755,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 FusedLayout fused_layout(const mta_shape &s)
 {
     FusedLayout L;
-    L.Tp = (s.T + kBM - 1) / kBM * kBM;
+    L.Tp = (s.T + 2 * kBM - 1) / (2 * kBM) * (2 * kBM);   // an even number of query blocks
     L.nqb = L.Tp / kBM;
     L.NA = q_atoms(s.c_q);
     const size_t BH = (size_t)s.B * s.H;
@@ -624,7 +774,8 @@ template <int D, int CH>
 mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr)
 {
-    using C = FusedCfg<D>;
+    constexpr bool PAIR = (D == 128);
+    using C = FusedCfg<D, PAIR>;
     const FusedLayout L = fused_layout(s);
     uint8_t *w = (uint8_t *)ws;
     __half *kf = (__half *)(w + L.off_kf);
@@ -642,7 +793,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     {
         uint64_t dims[3] = {(uint64_t)D, (uint64_t)L.Tp, BH * s.c_q};
         uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)L.Tp * D * 2};
-        uint32_t box[3] = {64, (uint32_t)kBN, 1};
+        uint32_t box[3] = {64, (uint32_t)C::kKfRows, 1};
         if (!make_tmap_f16(&mK, kf, 3, dims, strides, box)) return MTA_ERR_CUDA;
     }
     {
@@ -651,21 +802,40 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         uint32_t box[3] = {64, (uint32_t)kBN, 1};
         if (!make_tmap_bf16(&mV, a.v, 3, dims, strides, box)) return MTA_ERR_CUDA;
     }
-    const size_t pro_smem = prologue_smem_bytes(D);
-    if (cudaFuncSetAttribute(k_fold_prologue<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)pro_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(k_mta_fused<D, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
+    auto main_kernel = k_mta_fused<D, CH, PAIR>;
+    auto prologue = s.c_k == 11 ? k_fold_prologue<D, 11>
+                  : s.c_k == 3  ? k_fold_prologue<D, 3>
+                                : k_fold_prologue<D, 15>;
+    const int pro_smem = (int)prologue_smem_bytes(D);
+    if (cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, pro_smem) !=
+            cudaSuccess)
         return MTA_ERR_CUDA;
     const float scale = kLog2e / sqrtf((float)D);
     tr.before(0, st);
-    k_fold_prologue<D><<<dim3(L.nqb, (unsigned)BH), 256, pro_smem, st>>>(
+    prologue<<<dim3(L.nqb, (unsigned)BH), 256, pro_smem, st>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, kf, qp, corr, s.T, L.Tp,
         s.H, s.c_q, s.c_k, scale);
     tr.after(0, st);
     tr.before(1, st);
-    k_mta_fused<D, CH><<<dim3(L.nqb, s.H, s.B), 192, C::kSmemBytes, st>>>(
-        mQ, mK, mV, corr, a.w_head, part, s.T, L.Tp, s.H, s.c_q, L.nqb);
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(L.nqb, s.H, s.B);
+        cfg.blockDim = dim3(192, 1, 1);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, main_kernel, mQ, mK, mV, (const float *)corr, a.w_head, part,
+                               s.T, L.Tp, s.H, s.c_q, L.nqb) != cudaSuccess)
+            return MTA_ERR_CUDA;
+    }
     tr.after(1, st);
     tr.before(2, st);
     k_mix_groupnorm<D, CH><<<dim3(s.T, s.B), 128, 0, st>>>(part, a.gn_weight, a.gn_bias,
@@ -682,7 +852,7 @@ bool fused_supported(const mta_shape &s)
     if (s.io != MTA_BF16) return false;
     if (s.d != 64 && s.d != 128) return false;
     if (!(s.c_h == 1 || s.c_h == 2 || s.c_h == 4) || s.c_h * s.d > 256) return false;
-    if (s.c_q > 8 || s.c_k > 15 || d_m(s.c_q, s.c_k) > kCorrW) return false;
+    if (s.c_q > 8 || s.c_k > 15 || d_m(s.c_q, s.c_k) > kCorrW - 2) return false;
     return true;
 }
 
