@@ -102,6 +102,8 @@ k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
         const int ip = idx / CK, jp = idx % CK - shift;
         th[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] : 0.f;
     }
+    __shared__ float ths[8 * CK];              // the same taps times the logit scale
+    for (int idx = tid; idx < 8 * CK; idx += 256) ths[idx] = th[idx] * scale;
     __syncthreads();
 
     // (a) folded keys, in windows of SUB consecutive keys
@@ -109,7 +111,7 @@ k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
         constexpr int SUB = 16;
         constexpr int WS = SUB + CK - 1;           // window rows
         const int ep = tid % EP, rg = tid / EP;
-        bool range_ok = true;
+        float amax = 0.f;                          // largest |Kf| written by this thread
 #pragma unroll 1
         for (int sub = 0; sub < RPG / SUB; ++sub) {
             const int jr0 = j0 + rg * RPG + sub * SUB;     // first key of the window
@@ -125,7 +127,7 @@ k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
             for (int ip = 0; ip < c_q; ++ip) {
                 float t[CK];
 #pragma unroll
-                for (int jj = 0; jj < CK; ++jj) t[jj] = th[ip * CK + jj];
+                for (int jj = 0; jj < CK; ++jj) t[jj] = ths[ip * CK + jj];
                 __half *dst = kf + (((size_t)bh * c_q + ip) * Tp + jr0) * D + 2 * ep;
 #pragma unroll
                 for (int r = 0; r < SUB; ++r) {
@@ -135,14 +137,12 @@ k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
                         a0 = fmaf(t[jj], win[r + CK - 1 - jj].x, a0);
                         a1 = fmaf(t[jj], win[r + CK - 1 - jj].y, a1);
                     }
-                    a0 *= scale;
-                    a1 *= scale;
-                    range_ok &= fabsf(a0) <= 65504.f && fabsf(a1) <= 65504.f;
+                    amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
                     *(__half2 *)(dst + (size_t)r * D) = __floats2half2_rn(a0, a1);
                 }
             }
         }
-        if (!range_ok) atomicOr(&g_fused_error, kErrRange);
+        if (amax > 65504.f) atomicOr(&g_fused_error, kErrRange);   // NaN inputs propagate as NaN
     }
     // (b) permuted query rows: atom a, row s <- q_{j0-(c_q-1)+a+16s}; 8 elements per thread
     {
@@ -258,8 +258,8 @@ struct FusedCfg {
     static constexpr int kMaxAtoms = 23;                    // q_atoms(8)
     static constexpr int kQChunkBytes = kMaxAtoms * 1024;
     static constexpr int kOffRing = kChunks * kQChunkBytes;
-    static constexpr int kOffP = kOffRing + kStages * kStageBytes;
-    static constexpr int kOffCorr = kOffP + kBM * kBN * 2;
+    static constexpr int kOffScr = kOffRing + kStages * kStageBytes;   // band-tile scratch rows
+    static constexpr int kOffCorr = kOffScr + ((kBM * 33 * 4 + 1023) / 1024) * 1024;
     static constexpr int kOffBar = kOffCorr + kBM * kCorrW * 4;
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 };
@@ -325,7 +325,7 @@ __device__ __forceinline__ void arrive_leader(uint64_t *bar)
     else tc::mbar_arrive(bar);
 }
 
-// Grid (query blocks, H, B); block 192 threads = warp 0 TMA producer,
+// Block 192 threads = warp 0 TMA producer,
 // warp 1 MMA issuer (and TMEM owner), warps 2..5 softmax / epilogue (one TMEM
 // lane, i.e. one query row, per thread).  TMEM columns: S double buffer at
 // 0 and 128, U^{h,h'} for the c_h output heads from 256.
@@ -344,48 +344,47 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sQ = base;
     uint8_t *ring = base + C::kOffRing;
-    uint8_t *sP = base + C::kOffP;
+    float *sScr = (float *)(base + C::kOffScr);
     float *sCorr = (float *)(base + C::kOffCorr);
     uint64_t *bar_q = (uint64_t *)(base + C::kOffBar);
     uint64_t *full = bar_q + 1;
     uint64_t *empty = full + C::kStages;
     uint64_t *s_full = empty + C::kStages;
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
+    uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 1;
     uint64_t *mma_drain = pv_done + 1;
-    uint64_t *scr_bar = mma_drain + 1;
-    uint32_t *tmem_slot = (uint32_t *)(scr_bar + 1);
+    uint32_t *tmem_slot = (uint32_t *)(mma_drain + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
+    // Grid: x = (batch, head) [x2 CTAs per pair], y = query block (pair) in
+    // reverse order, so the longest blocks of every head start first.
     const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
     const bool leader = rank == 0;
     int qb, ntiles;
+    const int bhx = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
     if constexpr (PAIR) {
-        const int pair = nqb / 2 - 1 - (int)(blockIdx.x >> 1);   // longest rows first
+        const int pair = nqb / 2 - 1 - (int)blockIdx.y;
         qb = 2 * pair + (int)rank;
         ntiles = 2 * pair + 2;        // both CTAs run to the diagonal of block 2p+1
     } else {
-        qb = nqb - 1 - (int)blockIdx.x;
+        qb = nqb - 1 - (int)blockIdx.y;
         ntiles = qb + 1;
     }
-    const int hs = blockIdx.y, b = blockIdx.z;
+    const int hs = bhx % H, b = bhx / H;
     const int g = hs / CH, hl = hs % CH;
     const int bh = b * H + hs;
     const int i0 = qb * kBM;
     const int NA = q_atoms(c_q);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int consumers = PAIR ? 8 : 4;   // softmax warps that release S and publish P~
+    const int consumers = PAIR ? 8 : 4;   // softmax warps that publish P~
 
     if (threadIdx.x == 0) {
         tc::mbar_init(bar_q, 1);
         for (int s = 0; s < C::kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
         tc::mbar_init(&s_full[0], 1); tc::mbar_init(&s_full[1], 1);
-        tc::mbar_init(&s_free[0], consumers); tc::mbar_init(&s_free[1], consumers);
         tc::mbar_init(p_full, consumers);
         tc::mbar_init(pv_done, 1);
         tc::mbar_init(mma_drain, 1);
-        tc::mbar_init(scr_bar, 4);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -445,7 +444,23 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 for (int hh = 0; hh < CH && ok; ++hh) ok = load(false, u * kBN, b * H + g * CH + hh);
                 return ok;
             };
+            // L2 prefetch of the tiles kPrefetch key tiles ahead, so that the
+            // loads into the ring find them in L2
+            constexpr int kPrefetch = 2;
+            auto prefetch = [&](int u) {
+                if (u >= ntiles) return;
+                for (int ip = 0; ip < c_q; ++ip)
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tc::tma_prefetch_3d(&mapK, 64 * c, u * kBN + (PAIR ? (int)rank * C::kKfRows : 0),
+                                            bh * c_q + ip);
+                for (int hh = 0; hh < CH; ++hh)
+                    for (int c = 0; c < (PAIR ? 1 : C::kChunks); ++c)
+                        tc::tma_prefetch_3d(&mapV, 64 * (PAIR ? (int)rank : c), u * kBN,
+                                            b * H + g * CH + hh);
+            };
+            for (int u = 0; u < kPrefetch; ++u) prefetch(u);
             for (int t = 0; t < ntiles && ok; ++t) {
+                prefetch(t + kPrefetch);
                 for (int ip = 0; ip < c_q && ok; ++ip) ok = load(true, t * kBN, bh * c_q + ip);
                 if (ok && t > 0) load_v(t - 1);
             }
@@ -464,12 +479,21 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------- MMA issuer
+            // Descriptors are built once; the start-address field holds
+            // address >> 4, so every tile, stage and K step below is one add.
             constexpr int M = PAIR ? 2 * kBM : kBM;
             const uint32_t idq = tc::idesc_f16(M, kBN, false, false);
             const uint32_t idv = tc::idesc_bf16(M, D, false, true);
+            const uint64_t dq0 = tc::sdesc_sw128(tc::smem_u32(sQ), 16, 1024);
+            const uint64_t dk0 = tc::sdesc_sw128(tc::smem_u32(ring), 16, 1024);
+            const uint64_t dv0 = tc::sdesc_sw128(tc::smem_u32(ring), kBN * 128, 1024);
             auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
                 if constexpr (PAIR) tc::mma_pair(d, ad, bd, id, acc);
                 else tc::mma_bf16(d, ad, bd, id, acc);
+            };
+            auto mma_t = [&](uint32_t d, uint32_t at, uint64_t bd, uint32_t id, uint32_t acc) {
+                if constexpr (PAIR) tc::mma_pair_ts(d, at, bd, id, acc);
+                else tc::mma_ts(d, at, bd, id, acc);
             };
             auto commit = [&](uint64_t *bar) {
                 if constexpr (PAIR) tc::mma_commit_pair_multicast(bar, 0x3);
@@ -477,20 +501,35 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             };
             int stage = 0;
             uint32_t phase = 0;
+            // While a stage's MMAs are queued, test (without blocking) whether
+            // the next ring stage has landed; if it has, its turn starts with
+            // no wait, so the tensor pipe sees no gap between stages.
+            bool next_ready = false;
+            auto look_ahead = [&]() {
+                const int ns = (stage + 1 == C::kStages) ? 0 : stage + 1;
+                const uint32_t np = (stage + 1 == C::kStages) ? phase ^ 1 : phase;
+                next_ready = PAIR ? tc::mbar_try_wait_cluster(&full[ns], np) : tc::mbar_try_wait(&full[ns], np);
+            };
+            auto acquire = [&]() -> bool {
+                if (next_ready) { next_ready = false; return true; }
+                return wait_role<PAIR>(&full[stage], phase, abort_flag);
+            };
             bool ok = wait_role<PAIR>(bar_q, 0, abort_flag);
-            tc::tc_fence_after();
+            // The TMA data behind a full barrier needs no tcgen05 fence; P~ (in
+            // TMEM over the first half of its S buffer) and the rescaled U behind
+            // p_full do.  S(t+2) overwrites the buffer only after PV(t), which
+            // reads P~(t), has been issued: the pipe executes in issue order.
             auto issue_pv = [&](int u) -> bool {
                 if (!wait_role<PAIR>(p_full, u & 1, abort_flag)) return false;
                 tc::tc_fence_after();
                 for (int hh = 0; hh < CH; ++hh) {
-                    if (!wait_role<PAIR>(&full[stage], phase, abort_flag)) return false;
-                    tc::tc_fence_after();
-                    const uint8_t *vt = ring + stage * C::kStageBytes;
+                    if (!acquire()) return false;
+                    const uint64_t bv = dv0 + (uint64_t)((stage * C::kStageBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk) {
-                        uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sP + (kk >> 2) * (kBM * 128) + (kk & 3) * 32), 16, 1024);
-                        uint64_t bd = tc::sdesc_sw128(tc::smem_u32(vt + kk * 2048), kBN * 128, 1024);
-                        mma(tm + 256 + hh * D, ad, bd, idv, (u > 0 || kk > 0) ? 1u : 0u);
+                        mma_t(tm + 256 + hh * D, tm + (u & 1) * kBN + kk * 8,
+                              bv + (uint64_t)((kk * 2048) >> 4), idv, (u > 0 || kk > 0) ? 1u : 0u);
+                        if (kk == 1) look_ahead();
                     }
                     commit(&empty[stage]);
                     if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -500,23 +539,19 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             };
             for (int t = 0; t < ntiles && ok; ++t) {
                 const int sb = t & 1;
-                if (t >= 2) {
-                    ok = wait_role<PAIR>(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag);
-                    tc::tc_fence_after();
-                }
                 for (int ip = 0; ip < c_q && ok; ++ip) {
-                    ok = wait_role<PAIR>(&full[stage], phase, abort_flag);
+                    ok = acquire();
                     if (!ok) break;
-                    tc::tc_fence_after();
-                    const uint32_t aoff = (uint32_t)(c_q - 1 - ip) * 1024u;
-                    const uint8_t *kt = ring + stage * C::kStageBytes;
+                    const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
+                    const uint64_t bk = dk0 + (uint64_t)((stage * C::kStageBytes) >> 4);
 #pragma unroll
                     for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            uint64_t ad = tc::sdesc_sw128(tc::smem_u32(sQ + c * C::kQChunkBytes + aoff + kk * 32), 16, 1024);
-                            uint64_t bd = tc::sdesc_sw128(tc::smem_u32(kt + c * (C::kKfRows * 128) + kk * 32), 16, 1024);
-                            mma(tm + sb * kBN, ad, bd, idq, (ip | c | kk) ? 1u : 0u);
+                            mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
+                                bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
+                                (ip | c | kk) ? 1u : 0u);
+                            if (c == 0 && kk == 1) look_ahead();
                         }
                     commit(&empty[stage]);
                     if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -545,7 +580,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         }
         float m_run = -INFINITY, l = 0.f;
         bool ok = true;
-        int band_tiles = 0;
+        float *scr = sScr + r * 33;        // this thread's scratch row (band tiles)
         for (int t = 0; t < ntiles; ++t) {
             const int sb = t & 1;
             ok = __all_sync(0xffffffffu, wait_role<PAIR>(&s_full[sb], (t >> 1) & 1, abort_flag));
@@ -555,31 +590,19 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
 #pragma unroll
             for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
             tc::tmem_ld_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive_leader<PAIR>(&s_free[sb]);
             const int j0 = t * kBN;
             // Band tiles (this block's diagonal tile and the one before it):
             // causal -inf mask, and the Mask_0 correction of the D_m (< kCorrW)
             // diagonals below the main one.  Tiles past the diagonal (the
             // first block of a pair runs one) are masked entirely.  The
             // correction column depends on the row, so the chunks it touches go
-            // through a per-thread scratch row in the P~ buffer, idle once
-            // PV(t-1) has completed.
-            bool pv_waited = false;
+            // through the thread's scratch row in shared memory.
             if (t >= qb - 1) {
                 const int bse = i_row - j0;        // column of key i_row (>= 128 before the diagonal)
                 if (t >= qb) {
 #pragma unroll
                     for (int c = 0; c < kBN; ++c) s[c] = (c > bse) ? -INFINITY : s[c];
                 }
-                if (t > 0) {
-                    ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
-                    if (!ok) break;
-                    tc::tc_fence_after();
-                    pv_waited = true;
-                }
-                float *scr = (float *)sP + r * 33;
 #pragma unroll
                 for (int k = 0; k < kBN / 32; ++k) {
                     if (32 * k <= bse && 32 * k + 31 >= bse - (kCorrW - 1)) {
@@ -594,56 +617,56 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                         for (int x = 0; x < 32; ++x) s[32 * k + x] = scr[x];
                     }
                 }
-                // every softmax warp is done with its scratch rows before any
-                // P~ row overwrites them (bounded wait, like every other)
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(scr_bar);
-                ok = __all_sync(0xffffffffu, wait_role<PAIR>(scr_bar, band_tiles & 1, abort_flag));
-                ++band_tiles;
-                if (!ok) break;
             }
-            float mt = s[0];
+            // row max as 8 independent partial maxima
+            float mp[8];
 #pragma unroll
-            for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+            for (int x = 0; x < 8; ++x) mp[x] = s[x];
+#pragma unroll
+            for (int c = 8; c < kBN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+            const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
             // the running max moves only when it grows by more than 2^8 in scale
             const bool need = mt > m_run + 8.f;
             const float m_new = need ? mt : m_run;
             const float alpha = ex2(m_run - m_new);
-            if (t > 0) {
-                if (!pv_waited) {
-                    ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
-                    if (!ok) break;
-                    tc::tc_fence_after();
-                }
-                if (__any_sync(0xffffffffu, need)) {
-                    const float f = need ? alpha : 1.f;
+            // P~ = exp2(S - m), packed to bf16 pairs
+            uint32_t pk[kBN / 2];
+            float lp[8];
 #pragma unroll
-                    for (int hh = 0; hh < CH; ++hh)
+            for (int x = 0; x < 8; ++x) lp[x] = 0.f;
 #pragma unroll
-                        for (int j = 0; j < D / 32; ++j) {
-                            uint32_t u[32];
-                            const uint32_t a = lane_base + 256 + hh * D + 32 * j;
-                            tc::tmem_ld32(a, u);
-                            tc::tmem_ld_wait();
-#pragma unroll
-                            for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
-                            tc::tmem_st32(a, u);
-                        }
-                    tc::tmem_st_wait();
-                }
+            for (int c = 0; c < kBN; c += 2) {
+                const float p0 = ex2(s[c] - m_new), p1 = ex2(s[c + 1] - m_new);
+                lp[(c >> 1) & 7] += p0 + p1;
+                pk[c >> 1] = pack_bf16(p0, p1);
             }
-            l *= alpha;
+            // U is rescaled (rarely) once PV(t-1) has finished adding into it
+            if (t > 0 && __any_sync(0xffffffffu, need)) {
+                ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
+                if (!ok) break;
+                tc::tc_fence_after();
+                const float f = need ? alpha : 1.f;
+#pragma unroll
+                for (int hh = 0; hh < CH; ++hh)
+#pragma unroll
+                    for (int j = 0; j < D / 32; ++j) {
+                        uint32_t u[32];
+                        const uint32_t a = lane_base + 256 + hh * D + 32 * j;
+                        tc::tmem_ld32(a, u);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
+                        tc::tmem_st32(a, u);
+                    }
+            }
+            l = l * alpha + (((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7])));
             m_run = m_new;
-#pragma unroll
-            for (int c0 = 0; c0 < kBN; c0 += 8) {
-                float p[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) { p[x] = ex2(s[c0 + x] - m_run); l += p[x]; }
-                uint4 pk = make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                                      pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-                *(uint4 *)(sP + (c0 >> 6) * (kBM * 128) + tc::sw128_offset(r, c0 & 63)) = pk;
-            }
-            tc::fence_async_shared();
+            // P~(t) goes to TMEM over the first kBN/2 columns of its S buffer,
+            // where PV(t) reads it as the A operand
+            tc::tmem_st32(lane_base + sb * kBN, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+            tc::tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+            tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_leader<PAIR>(p_full);
@@ -821,7 +844,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     tr.before(1, st);
     {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(L.nqb, s.H, s.B);
+        cfg.gridDim = PAIR ? dim3(2 * s.B * s.H, L.nqb / 2, 1) : dim3(s.B * s.H, L.nqb, 1);
         cfg.blockDim = dim3(192, 1, 1);
         cfg.dynamicSmemBytes = C::kSmemBytes;
         cfg.stream = st;
