@@ -49,6 +49,8 @@ constexpr int kBM = 128;          // query rows per CTA (TMEM lanes)
 constexpr int kBN = 128;          // keys per tile
 constexpr int kCorrW = 16;        // correction entries stored per row (D_m <= 14)
 constexpr float kLog2e = 1.4426950408889634f;
+// named barrier at which the MMA issuer and its gate warp meet once per step
+constexpr int kGateBar = 1;
 constexpr long long kWaitBudget = 1ll << 30;   // ~0.55 s at 1.965 GHz per wait
 
 // Device error word: bit 0 a bounded wait expired, bit 1 a folded operand
@@ -325,15 +327,15 @@ __device__ __forceinline__ void arrive_leader(uint64_t *bar)
     else tc::mbar_arrive(bar);
 }
 
-// Block 192 threads = warp 0 TMA producer,
+// Block 224 threads = warp 0 TMA producer,
 // warp 1 MMA issuer (and TMEM owner), warps 2..5 softmax / epilogue (one TMEM
-// lane, i.e. one query row, per thread).  TMEM columns: S double buffer at
+// lane, i.e. one query row, per thread), warp 6 gate of the issuer.  TMEM columns: S double buffer at
 // 0 and 128, U^{h,h'} for the c_h output heads from 256.
 // PAIR (d = 128): clusters of two CTAs own query blocks 2p and 2p+1 of one
 // head; rank 0 issues the M = 256 MMAs for both and every completion is
 // multicast to both CTAs' barriers.
 template <int D, int CH, bool PAIR>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
 k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
             const __grid_constant__ CUtensorMap mapV, const float *__restrict__ corr,
             const float *__restrict__ w_head, float *__restrict__ part, int T, int Tp, int H,
@@ -477,8 +479,11 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && leader) {
-            // ---------------- MMA issuer
+        if (leader) {
+            // ---------------- MMA issuer: lane 0 issues, the whole warp meets
+            // the gate warp at one named barrier per step, so no shared-memory
+            // access sits in the issue stream.
+            const bool issuer = lane == 0;
             // Descriptors are built once; the start-address field holds
             // address >> 4, so every tile, stage and K step below is one add.
             constexpr int M = PAIR ? 2 * kBM : kBM;
@@ -499,75 +504,96 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 if constexpr (PAIR) tc::mma_commit_pair_multicast(bar, 0x3);
                 else tc::mma_commit(bar);
             };
+            auto gate = [&](int id) {
+                __syncwarp();
+                tc::named_bar_sync(id, 64);
+            };
             int stage = 0;
-            uint32_t phase = 0;
-            // While a stage's MMAs are queued, test (without blocking) whether
-            // the next ring stage has landed; if it has, its turn starts with
-            // no wait, so the tensor pipe sees no gap between stages.
-            bool next_ready = false;
-            auto look_ahead = [&]() {
-                const int ns = (stage + 1 == C::kStages) ? 0 : stage + 1;
-                const uint32_t np = (stage + 1 == C::kStages) ? phase ^ 1 : phase;
-                next_ready = PAIR ? tc::mbar_try_wait_cluster(&full[ns], np) : tc::mbar_try_wait(&full[ns], np);
-            };
-            auto acquire = [&]() -> bool {
-                if (next_ready) { next_ready = false; return true; }
-                return wait_role<PAIR>(&full[stage], phase, abort_flag);
-            };
-            bool ok = wait_role<PAIR>(bar_q, 0, abort_flag);
+            gate(kGateBar);
             // The TMA data behind a full barrier needs no tcgen05 fence; P~ (in
             // TMEM over the first half of its S buffer) and the rescaled U behind
             // p_full do.  S(t+2) overwrites the buffer only after PV(t), which
             // reads P~(t), has been issued: the pipe executes in issue order.
-            auto issue_pv = [&](int u) -> bool {
-                if (!wait_role<PAIR>(p_full, u & 1, abort_flag)) return false;
+            auto issue_pv = [&](int u) {
+                gate(kGateBar);
                 tc::tc_fence_after();
                 for (int hh = 0; hh < CH; ++hh) {
-                    if (!acquire()) return false;
-                    const uint64_t bv = dv0 + (uint64_t)((stage * C::kStageBytes) >> 4);
+                    gate(kGateBar);
+                    if (issuer) {
+                        const uint64_t bv = dv0 + (uint64_t)((stage * C::kStageBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        mma_t(tm + 256 + hh * D, tm + (u & 1) * kBN + kk * 8,
-                              bv + (uint64_t)((kk * 2048) >> 4), idv, (u > 0 || kk > 0) ? 1u : 0u);
-                        if (kk == 1) look_ahead();
+                        for (int kk = 0; kk < kBN / 16; ++kk)
+                            mma_t(tm + 256 + hh * D, tm + (u & 1) * kBN + kk * 8,
+                                  bv + (uint64_t)((kk * 2048) >> 4), idv, (u > 0 || kk > 0) ? 1u : 0u);
+                        commit(&empty[stage]);
                     }
-                    commit(&empty[stage]);
-                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                    if (++stage == C::kStages) stage = 0;
                 }
-                commit(pv_done);
-                return true;
+                if (issuer) commit(pv_done);
             };
-            for (int t = 0; t < ntiles && ok; ++t) {
+            for (int t = 0; t < ntiles; ++t) {
                 const int sb = t & 1;
-                for (int ip = 0; ip < c_q && ok; ++ip) {
-                    ok = acquire();
-                    if (!ok) break;
-                    const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
-                    const uint64_t bk = dk0 + (uint64_t)((stage * C::kStageBytes) >> 4);
+                for (int ip = 0; ip < c_q; ++ip) {
+                    gate(kGateBar);
+                    if (issuer) {
+                        const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
+                        const uint64_t bk = dk0 + (uint64_t)((stage * C::kStageBytes) >> 4);
 #pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
+                        for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
-                                bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
-                                (ip | c | kk) ? 1u : 0u);
-                            if (c == 0 && kk == 1) look_ahead();
-                        }
-                    commit(&empty[stage]);
-                    if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
+                                    bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
+                                    (ip | c | kk) ? 1u : 0u);
+                        commit(&empty[stage]);
+                    }
+                    if (++stage == C::kStages) stage = 0;
                 }
-                if (!ok) break;
-                commit(&s_full[sb]);
-                if (t > 0) ok = issue_pv(t - 1);
+                if (issuer) commit(&s_full[sb]);
+                if (t > 0) issue_pv(t - 1);
             }
-            if (ok) issue_pv(ntiles - 1);
-            // all MMAs this thread issued complete before TMEM is released
-            if constexpr (PAIR) tc::mma_commit_pair_multicast(mma_drain, 0x1);
-            else tc::mma_commit(mma_drain);
-            tc::mbar_wait(mma_drain, 0, kWaitBudget);
+            issue_pv(ntiles - 1);
+            // all MMAs this warp issued complete before TMEM is released
+            if (issuer) {
+                if constexpr (PAIR) tc::mma_commit_pair_multicast(mma_drain, 0x1);
+                else tc::mma_commit(mma_drain);
+                tc::mbar_wait(mma_drain, 0, kWaitBudget);
+            }
+        }
+    } else if (warp == 6) {
+        if (leader) {
+            // ---------------- gate: waits, in the issuer's order, for each
+            // barrier the next MMA step depends on, then meets the issuer at the
+            // step's named barrier.  Both sides use bar.sync, so they move in
+            // lockstep and a barrier id never holds two generations at once.
+            // After a timeout or abort the waits are skipped but every meeting
+            // still happens, so the issuer runs to its end and drains.
+            bool ok = true;
+            int stage = 0;
+            uint32_t phase = 0;
+            auto pass = [&](uint64_t *bar, uint32_t parity, int id) {
+                int r = 1;
+                if (lane == 0 && ok) r = wait_role<PAIR>(bar, parity, abort_flag) ? 1 : 0;
+                ok = ok && __shfl_sync(0xffffffffu, r, 0) != 0;
+                tc::named_bar_sync(id, 64);
+            };
+            auto pass_stage = [&]() {
+                pass(&full[stage], phase, kGateBar);
+                if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            };
+            pass(bar_q, 0, kGateBar);
+            auto pass_pv = [&](int u) {
+                pass(p_full, u & 1, kGateBar);
+                for (int hh = 0; hh < CH; ++hh) pass_stage();
+            };
+            for (int t = 0; t < ntiles; ++t) {
+                for (int ip = 0; ip < c_q; ++ip) pass_stage();
+                if (t > 0) pass_pv(t - 1);
+            }
+            pass_pv(ntiles - 1);
         }
     } else {
-        // ---------------- softmax and epilogue: thread = TMEM lane = one query row
+        // ---------------- softmax and epilogue (warps 2..5): thread = TMEM lane = one query row
         const int q4 = warp & 3;                       // lane quarter this warp may access
         const int r = q4 * 32 + lane;
         const int i_row = i0 + 16 * (r & 7) + (r >> 3);   // permuted row order of the Q operand
@@ -845,7 +871,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = PAIR ? dim3(2 * s.B * s.H, L.nqb / 2, 1) : dim3(s.B * s.H, L.nqb, 1);
-        cfg.blockDim = dim3(192, 1, 1);
+        cfg.blockDim = dim3(224, 1, 1);
         cfg.dynamicSmemBytes = C::kSmemBytes;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];

@@ -68,6 +68,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     return true;
 }
 
+// Named CTA barriers (ids 1..15; 0 is __syncthreads).  `count` threads, a
+// multiple of 32, take part; whole warps execute these.  They need no
+// shared-memory access, so a warp that issues tcgen05.mma can wait on one
+// without a load that queues behind its MMAs.
+__device__ __forceinline__ void named_bar_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads (tensor-core operands).
 __device__ __forceinline__ void fence_async_shared()
