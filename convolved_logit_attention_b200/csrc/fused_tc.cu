@@ -667,11 +667,18 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 lp[(c >> 1) & 7] += p0 + p1;
                 pk[c >> 1] = pack_bf16(p0, p1);
             }
-            // U is rescaled (rarely) once PV(t-1) has finished adding into it
-            if (t > 0 && __any_sync(0xffffffffu, need)) {
+            // Every warp waits for PV(t-1) to complete before it publishes
+            // P~(t).  p_full counts arrivals from all softmax warps (of both
+            // CTAs in a pair); without this wait a warp that ran a tile ahead
+            // could complete phase t for a warp still working on tile t.  The
+            // wait also orders the (rare) rescale of U after PV(t-1) added
+            // into it.
+            if (t > 0) {
                 ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
                 if (!ok) break;
                 tc::tc_fence_after();
+            }
+            if (t > 0 && __any_sync(0xffffffffu, need)) {
                 const float f = need ? alpha : 1.f;
 #pragma unroll
                 for (int hh = 0; hh < CH; ++hh)

@@ -68,13 +68,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     return true;
 }
 
-// Named CTA barriers (ids 1..15; 0 is __syncthreads).  `count` threads, a
-// multiple of 32, take part; whole warps execute these.  They need no
-// shared-memory access, so a warp that issues tcgen05.mma can wait on one
-// without a load that queues behind its MMAs.
+// Named CTA barriers (ids 1..15; 0 is __syncthreads); `count` is a multiple
+// of 32.  The non-aligned form first gathers all non-exited lanes of the
+// executing warp and then counts the warp once, so a warp whose lanes reach
+// it on different paths (one lane issuing MMAs, the others not) still
+// arrives exactly once.  (The aligned bar.sync would count each divergent
+// group as a whole warp.)  No shared-memory access is involved, so a warp
+// that issues tcgen05.mma can wait on it without a load queued behind its
+// MMAs.
 __device__ __forceinline__ void named_bar_sync(int id, int count)
 {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Orders this thread's generic-proxy shared-memory writes before later
