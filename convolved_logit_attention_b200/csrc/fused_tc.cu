@@ -49,8 +49,10 @@ constexpr int kBM = 128;          // query rows per CTA (TMEM lanes)
 constexpr int kBN = 128;          // keys per tile
 constexpr int kCorrW = 16;        // correction entries stored per row (D_m <= 14)
 constexpr float kLog2e = 1.4426950408889634f;
-// named barrier at which the MMA issuer and its gate warp meet once per step
-constexpr int kGateBar = 1;
+// Named barriers at which the MMA issuer meets its gate warp: one per ring
+// slot and one for the Q tile.
+constexpr int kGateStage0 = 1;     // ids 1 .. kStages (at most 8)
+constexpr int kGateQ = 9;
 constexpr long long kWaitBudget = 1ll << 30;   // ~0.55 s at 1.965 GHz per wait
 
 // Device error word: bit 0 a bounded wait expired, bit 1 a folded operand
@@ -248,22 +250,36 @@ size_t prologue_smem_bytes(int D)
 
 // ------------------------------------------------------------ main kernel
 
-// PAIR: two CTAs (consecutive 128-row query blocks of one head) share every
-// MMA as one M = 256 tcgen05 operation; each CTA then loads only half of
-// every key tile (64 keys of Kf, 64 of the d columns of V).
-template <int D, bool PAIR>
+// PAIR (d = 128): two CTAs (consecutive 128-row query blocks of one head)
+// share every MMA as one M = 256 tcgen05 operation; each CTA then loads only
+// half of every Kf tile (64 keys) and half of the V columns.  Without PAIR
+// (d = 64) a CTA loads whole tiles.
+//
+// Ring slots are 32 KB.  A Kf slot holds two shifts i' (16 KB each: 64 keys
+// x 128 d, or 128 keys x 64 d); a V slot holds the V tiles of kVHeads output
+// heads, whose PV products then run as one MMA chain of N = kVHeads * d
+// (in a pair each CTA holds one head's tile, or one half of the single
+// head's columns).  The issuer meets its gate once per slot.
+template <int D, int CH, bool PAIR>
 struct FusedCfg {
+    static_assert(PAIR == (D == 128), "pairs serve d = 128, single CTAs d = 64");
     static constexpr int kChunks = D / 64;                  // 64-element (128-B) column chunks
     static constexpr int kKfRows = PAIR ? kBN / 2 : kBN;    // keys of a Kf tile held by this CTA
-    static constexpr int kStageBytes = PAIR ? kBN * 64 * 2 : kBN * D * 2;
-    static constexpr int kStages = (kStageBytes <= 16384) ? 8 : 4;
+    static constexpr int kShiftBytes = kKfRows * D * 2;     // one shift of one Kf tile
+    static constexpr int kSlotBytes = 2 * kShiftBytes;
+    static constexpr int kStages = 4;
+    static constexpr int kVHeads = CH < 2 ? CH : 2;         // output heads per V slot
+    static constexpr int kVSlots = CH / kVHeads;            // V slots per key tile
+    static constexpr int kVN = kVHeads * D;                 // N of one PV MMA chain
+    static constexpr int kVBytes = kVHeads * 16384;         // bytes of a V slot this CTA loads
     static constexpr int kMaxAtoms = 23;                    // q_atoms(8)
     static constexpr int kQChunkBytes = kMaxAtoms * 1024;
     static constexpr int kOffRing = kChunks * kQChunkBytes;
-    static constexpr int kOffScr = kOffRing + kStages * kStageBytes;   // band-tile scratch rows
+    static constexpr int kOffScr = kOffRing + kStages * kSlotBytes;   // band-tile scratch rows
     static constexpr int kOffCorr = kOffScr + ((kBM * 33 * 4 + 1023) / 1024) * 1024;
     static constexpr int kOffBar = kOffCorr + kBM * kCorrW * 4;
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+    static_assert(kShiftBytes == 16384 && kVN <= 256, "slot layout");
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -341,7 +357,8 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             const float *__restrict__ w_head, float *__restrict__ part, int T, int Tp, int H,
             int c_q, int nqb)
 {
-    using C = FusedCfg<D, PAIR>;
+    using C = FusedCfg<D, CH, PAIR>;
+    static_assert(C::kStages <= kGateQ - kGateStage0, "one gate barrier id per ring slot");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sQ = base;
@@ -417,34 +434,54 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             bool issued[C::kStages];
             for (int s = 0; s < C::kStages; ++s) issued[s] = false;
             bool ok = true;
-            // one stage: a Kf tile (kKfRows keys x d) or this CTA's d chunks of a V tile
-            auto load = [&](bool is_k, int y, int z) -> bool {
-                if (!wait_role<PAIR>(&empty[stage], phase ^ 1, abort_flag)) return false;
-                uint8_t *dst = ring + stage * C::kStageBytes;
-                if constexpr (PAIR) {
-                    const uint32_t bf = tc::mapa_shared(tc::smem_u32(&full[stage]), 0);
-                    if (leader) tc::mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-                    if (is_k) {
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tc::tma_load_3d_pair(dst + c * (C::kKfRows * 128), &mapK, bf, 64 * c,
-                                                 y + (int)rank * C::kKfRows, z);
-                    } else {
-                        tc::tma_load_3d_pair(dst, &mapV, bf, 64 * (int)rank, y, z);
-                    }
-                } else {
-                    tc::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tc::tma_load_3d(dst + c * (kBN * 128), is_k ? &mapK : &mapV, &full[stage],
-                                        64 * c, y, z);
-                }
+            // Claims the next ring slot and counts `bytes` (this CTA's part) on
+            // its full barrier; the leader of a pair expects both CTAs' parts.
+            auto claim = [&](uint32_t bytes) -> uint8_t * {
+                if (!wait_role<PAIR>(&empty[stage], phase ^ 1, abort_flag)) return nullptr;
+                if (leader) tc::mbar_arrive_expect_tx(&full[stage], PAIR ? 2 * bytes : bytes);
+                return ring + stage * C::kSlotBytes;
+            };
+            auto advance = [&]() {
                 issued[stage] = true;
                 issued_phase[stage] = phase;
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+            };
+            auto tile_load = [&](uint8_t *dst, const CUtensorMap *map, int x, int y, int z) {
+                if constexpr (PAIR)
+                    tc::tma_load_3d_pair(dst, map, tc::mapa_shared(tc::smem_u32(&full[stage]), 0), x, y, z);
+                else
+                    tc::tma_load_3d(dst, map, &full[stage], x, y, z);
+            };
+            // Kf slot m of key tile t: shifts 2m and 2m+1 (when below c_q)
+            auto load_kf = [&](int t, int m) -> bool {
+                const int n = (2 * m + 1 < c_q) ? 2 : 1;
+                uint8_t *dst = claim(n * C::kShiftBytes);
+                if (dst == nullptr) return false;
+                for (int h = 0; h < n; ++h)
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tile_load(dst + h * C::kShiftBytes + c * (C::kKfRows * 128), &mapK, 64 * c,
+                                  t * kBN + (PAIR ? (int)rank * C::kKfRows : 0), bh * c_q + 2 * m + h);
+                advance();
                 return true;
             };
-            auto load_v = [&](int u) -> bool {
-                for (int hh = 0; hh < CH && ok; ++hh) ok = load(false, u * kBN, b * H + g * CH + hh);
-                return ok;
+            // V slot vs of key tile u: heads vs*kVHeads ...; in a pair with two
+            // heads CTA r loads head r whole, with one head it loads column half r
+            auto load_v = [&](int u, int vs) -> bool {
+                uint8_t *dst = claim(C::kVBytes);
+                if (dst == nullptr) return false;
+                const int z0 = b * H + g * CH + vs * C::kVHeads;
+                if constexpr (PAIR) {
+                    if (C::kVHeads == 2) {
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tile_load(dst + c * 16384, &mapV, 64 * c, u * kBN, z0 + (int)rank);
+                    } else {
+                        tile_load(dst, &mapV, 64 * (int)rank, u * kBN, z0);
+                    }
+                } else {
+                    for (int j = 0; j < C::kVHeads; ++j) tile_load(dst + j * 16384, &mapV, 0, u * kBN, z0 + j);
+                }
+                advance();
+                return true;
             };
             // L2 prefetch of the tiles kPrefetch key tiles ahead, so that the
             // loads into the ring find them in L2
@@ -455,18 +492,26 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                     for (int c = 0; c < C::kChunks; ++c)
                         tc::tma_prefetch_3d(&mapK, 64 * c, u * kBN + (PAIR ? (int)rank * C::kKfRows : 0),
                                             bh * c_q + ip);
-                for (int hh = 0; hh < CH; ++hh)
-                    for (int c = 0; c < (PAIR ? 1 : C::kChunks); ++c)
-                        tc::tma_prefetch_3d(&mapV, 64 * (PAIR ? (int)rank : c), u * kBN,
-                                            b * H + g * CH + hh);
+                for (int vs = 0; vs < C::kVSlots; ++vs) {
+                    const int z0 = b * H + g * CH + vs * C::kVHeads;
+                    if (PAIR && C::kVHeads == 2) {
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tc::tma_prefetch_3d(&mapV, 64 * c, u * kBN, z0 + (int)rank);
+                    } else if (PAIR) {
+                        tc::tma_prefetch_3d(&mapV, 64 * (int)rank, u * kBN, z0);
+                    } else {
+                        for (int j = 0; j < C::kVHeads; ++j) tc::tma_prefetch_3d(&mapV, 0, u * kBN, z0 + j);
+                    }
+                }
             };
+            const int kf_slots = (c_q + 1) / 2;
             for (int u = 0; u < kPrefetch; ++u) prefetch(u);
             for (int t = 0; t < ntiles && ok; ++t) {
                 prefetch(t + kPrefetch);
-                for (int ip = 0; ip < c_q && ok; ++ip) ok = load(true, t * kBN, bh * c_q + ip);
-                if (ok && t > 0) load_v(t - 1);
+                for (int m = 0; m < kf_slots && ok; ++m) ok = load_kf(t, m);
+                for (int vs = 0; vs < C::kVSlots && ok && t > 0; ++vs) ok = load_v(t - 1, vs);
             }
-            if (ok) load_v(ntiles - 1);
+            for (int vs = 0; vs < C::kVSlots && ok; ++vs) ok = load_v(ntiles - 1, vs);
             // copies this thread started land before the CTA may exit; in a pair
             // their completion is counted in the leader, so the peer waits a while
             if (leader) {
@@ -488,10 +533,11 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             // address >> 4, so every tile, stage and K step below is one add.
             constexpr int M = PAIR ? 2 * kBM : kBM;
             const uint32_t idq = tc::idesc_f16(M, kBN, false, false);
-            const uint32_t idv = tc::idesc_bf16(M, D, false, true);
+            const uint32_t idv = tc::idesc_bf16(M, C::kVN, false, true);
             const uint64_t dq0 = tc::sdesc_sw128(tc::smem_u32(sQ), 16, 1024);
             const uint64_t dk0 = tc::sdesc_sw128(tc::smem_u32(ring), 16, 1024);
-            const uint64_t dv0 = tc::sdesc_sw128(tc::smem_u32(ring), kBN * 128, 1024);
+            // V is MN-major: 64-column chunks of one slot lie 16 KB apart
+            const uint64_t dv0 = tc::sdesc_sw128(tc::smem_u32(ring), 16384, 1024);
             auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t id, uint32_t acc) {
                 if constexpr (PAIR) tc::mma_pair(d, ad, bd, id, acc);
                 else tc::mma_bf16(d, ad, bd, id, acc);
@@ -509,21 +555,22 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 tc::named_bar_sync(id, 64);
             };
             int stage = 0;
-            gate(kGateBar);
+            const int kf_slots = (c_q + 1) / 2;
+            gate(kGateQ);
             // The TMA data behind a full barrier needs no tcgen05 fence; P~ (in
-            // TMEM over the first half of its S buffer) and the rescaled U behind
-            // p_full do.  S(t+2) overwrites the buffer only after PV(t), which
-            // reads P~(t), has been issued: the pipe executes in issue order.
+            // TMEM over the first half of its S buffer) and the rescaled U,
+            // which the gate also waited for before the first V slot, do.
+            // S(t+2) overwrites the buffer only after PV(t), which reads P~(t),
+            // has been issued: the pipe executes in issue order.
             auto issue_pv = [&](int u) {
-                gate(kGateBar);
-                tc::tc_fence_after();
-                for (int hh = 0; hh < CH; ++hh) {
-                    gate(kGateBar);
+                for (int vs = 0; vs < C::kVSlots; ++vs) {
+                    gate(kGateStage0 + stage);
+                    if (vs == 0) tc::tc_fence_after();
                     if (issuer) {
-                        const uint64_t bv = dv0 + (uint64_t)((stage * C::kStageBytes) >> 4);
+                        const uint64_t bv = dv0 + (uint64_t)((stage * C::kSlotBytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_t(tm + 256 + hh * D, tm + (u & 1) * kBN + kk * 8,
+                            mma_t(tm + 256 + vs * C::kVN, tm + (u & 1) * kBN + kk * 8,
                                   bv + (uint64_t)((kk * 2048) >> 4), idv, (u > 0 || kk > 0) ? 1u : 0u);
                         commit(&empty[stage]);
                     }
@@ -533,18 +580,23 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             };
             for (int t = 0; t < ntiles; ++t) {
                 const int sb = t & 1;
-                for (int ip = 0; ip < c_q; ++ip) {
-                    gate(kGateBar);
+                for (int m = 0; m < kf_slots; ++m) {
+                    gate(kGateStage0 + stage);
                     if (issuer) {
-                        const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
-                        const uint64_t bk = dk0 + (uint64_t)((stage * C::kStageBytes) >> 4);
+                        const uint64_t bs = dk0 + (uint64_t)((stage * C::kSlotBytes) >> 4);
+                        for (int h = 0; h < 2; ++h) {
+                            const int ip = 2 * m + h;
+                            if (ip >= c_q) break;
+                            const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
+                            const uint64_t bk = bs + (uint64_t)((h * C::kShiftBytes) >> 4);
 #pragma unroll
-                        for (int c = 0; c < C::kChunks; ++c)
+                            for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
-                                    bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
-                                    (ip | c | kk) ? 1u : 0u);
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
+                                        bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
+                                        (ip | c | kk) ? 1u : 0u);
+                        }
                         commit(&empty[stage]);
                     }
                     if (++stage == C::kStages) stage = 0;
@@ -563,34 +615,43 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     } else if (warp == 6) {
         if (leader) {
             // ---------------- gate: waits, in the issuer's order, for each
-            // barrier the next MMA step depends on, then meets the issuer at the
-            // step's named barrier.  Both sides use bar.sync, so they move in
-            // lockstep and a barrier id never holds two generations at once.
-            // After a timeout or abort the waits are skipped but every meeting
-            // still happens, so the issuer runs to its end and drains.
+            // barrier the next MMA step depends on and arrives (without
+            // blocking) at that ring slot's named barrier, so it runs ahead of
+            // the issuer.  A slot's barrier never receives a second arrival
+            // before the issuer has consumed the first: the slot is refilled
+            // only after the issuer's commit for its previous use.  The first
+            // V slot of PV(u) also waits for P~(u) (p_full).  After a timeout
+            // or abort the gate stops waiting on data but still arrives at
+            // every meeting, each time after the issuer's commit for the
+            // slot's previous use, so the issuer runs to its end and drains.
             bool ok = true;
             int stage = 0;
             uint32_t phase = 0;
-            auto pass = [&](uint64_t *bar, uint32_t parity, int id) {
+            auto meet = [&](bool with_p, int u) {
                 int r = 1;
-                if (lane == 0 && ok) r = wait_role<PAIR>(bar, parity, abort_flag) ? 1 : 0;
+                if (lane == 0) {
+                    if (ok && with_p) r = wait_role<PAIR>(p_full, u & 1, abort_flag) ? 1 : 0;
+                    if (ok && r) r = wait_role<PAIR>(&full[stage], phase, abort_flag) ? 1 : 0;
+                    if (!ok || !r) tc::mbar_wait(&empty[stage], phase ^ 1, kWaitBudget);
+                }
                 ok = ok && __shfl_sync(0xffffffffu, r, 0) != 0;
-                tc::named_bar_sync(id, 64);
-            };
-            auto pass_stage = [&]() {
-                pass(&full[stage], phase, kGateBar);
+                __syncwarp();
+                tc::named_bar_arrive(kGateStage0 + stage, 64);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
             };
-            pass(bar_q, 0, kGateBar);
-            auto pass_pv = [&](int u) {
-                pass(p_full, u & 1, kGateBar);
-                for (int hh = 0; hh < CH; ++hh) pass_stage();
-            };
-            for (int t = 0; t < ntiles; ++t) {
-                for (int ip = 0; ip < c_q; ++ip) pass_stage();
-                if (t > 0) pass_pv(t - 1);
+            {
+                int r = 1;
+                if (lane == 0) r = wait_role<PAIR>(bar_q, 0, abort_flag) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+                __syncwarp();
+                tc::named_bar_arrive(kGateQ, 64);
             }
-            pass_pv(ntiles - 1);
+            const int kf_slots = (c_q + 1) / 2;
+            for (int t = 0; t < ntiles; ++t) {
+                for (int m = 0; m < kf_slots; ++m) meet(false, 0);
+                for (int vs = 0; vs < C::kVSlots && t > 0; ++vs) meet(vs == 0, t - 1);
+            }
+            for (int vs = 0; vs < C::kVSlots; ++vs) meet(vs == 0, ntiles - 1);
         }
     } else {
         // ---------------- softmax and epilogue (warps 2..5): thread = TMEM lane = one query row
@@ -831,7 +892,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
                           const Trace &tr)
 {
     constexpr bool PAIR = (D == 128);
-    using C = FusedCfg<D, PAIR>;
+    using C = FusedCfg<D, CH, PAIR>;
     const FusedLayout L = fused_layout(s);
     uint8_t *w = (uint8_t *)ws;
     __half *kf = (__half *)(w + L.off_kf);

@@ -81,6 +81,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int count)
     asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrival without waiting (non-aligned form, counted once per warp).
+__device__ __forceinline__ void named_bar_arrive(int id, int count)
+{
+    asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads (tensor-core operands).
 __device__ __forceinline__ void fence_async_shared()
