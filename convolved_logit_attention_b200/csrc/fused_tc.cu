@@ -48,6 +48,8 @@ namespace {
 constexpr int kBM = 128;          // query rows per CTA (TMEM lanes)
 constexpr int kBN = 128;          // keys per tile
 constexpr int kCorrW = 16;        // correction entries stored per row (D_m <= 14)
+constexpr int kCorrStride = 17;   // shared-memory row stride of that table (conflict-free reads)
+constexpr int kScrStride = 36;    // floats per scratch row: 16-B aligned, conflict-free by float4
 constexpr float kLog2e = 1.4426950408889634f;
 // Named barriers at which the MMA issuer meets its gate warp: one per ring
 // slot and one for the Q tile.
@@ -276,8 +278,8 @@ struct FusedCfg {
     static constexpr int kQChunkBytes = kMaxAtoms * 1024;
     static constexpr int kOffRing = kChunks * kQChunkBytes;
     static constexpr int kOffScr = kOffRing + kStages * kSlotBytes;   // band-tile scratch rows
-    static constexpr int kOffCorr = kOffScr + ((kBM * 33 * 4 + 1023) / 1024) * 1024;
-    static constexpr int kOffBar = kOffCorr + kBM * kCorrW * 4;
+    static constexpr int kOffCorr = kOffScr + ((kBM * kScrStride * 4 + 1023) / 1024) * 1024;
+    static constexpr int kOffBar = kOffCorr + kBM * kCorrStride * 4;
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
     static_assert(kShiftBytes == 16384 && kVN <= 256, "slot layout");
 };
@@ -505,10 +507,10 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 }
             };
             const int kf_slots = (c_q + 1) / 2;
-            for (int u = 0; u < kPrefetch; ++u) prefetch(u);
             for (int t = 0; t < ntiles && ok; ++t) {
-                prefetch(t + kPrefetch);
                 for (int m = 0; m < kf_slots && ok; ++m) ok = load_kf(t, m);
+                // tile 0 is loaded first, then the prefetches start
+                for (int u = (t == 0 ? 1 : t + kPrefetch); u <= t + kPrefetch; ++u) prefetch(u);
                 for (int vs = 0; vs < C::kVSlots && ok && t > 0; ++vs) ok = load_v(t - 1, vs);
             }
             for (int vs = 0; vs < C::kVSlots && ok; ++vs) ok = load_v(ntiles - 1, vs);
@@ -659,34 +661,46 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         const int r = q4 * 32 + lane;
         const int i_row = i0 + 16 * (r & 7) + (r >> 3);   // permuted row order of the Q operand
         const uint32_t lane_base = tm + ((uint32_t)(q4 * 32) << 16);
-        float *crow = sCorr + r * kCorrW;
+        float *crow = sCorr + r * kCorrStride;
         {
             const float4 *src = (const float4 *)(corr + ((size_t)bh * Tp + i_row) * kCorrW);
 #pragma unroll
-            for (int u = 0; u < kCorrW / 4; ++u) ((float4 *)crow)[u] = src[u];
+            for (int u = 0; u < kCorrW / 4; ++u) {
+                const float4 v = src[u];
+                crow[4 * u] = v.x; crow[4 * u + 1] = v.y; crow[4 * u + 2] = v.z; crow[4 * u + 3] = v.w;
+            }
         }
         float m_run = -INFINITY, l = 0.f;
         bool ok = true;
-        float *scr = sScr + r * 33;        // this thread's scratch row (band tiles)
+        float *scr = sScr + r * kScrStride;   // this thread's scratch row (band tiles, epilogue)
         for (int t = 0; t < ntiles; ++t) {
             const int sb = t & 1;
             ok = __all_sync(0xffffffffu, wait_role<PAIR>(&s_full[sb], (t >> 1) & 1, abort_flag));
             if (!ok) break;
             tc::tc_fence_after();
+            // The first block of a pair runs one tile past its diagonal: every
+            // key there is in the future, so P~ is zero and the row state stays.
+            const bool live = t <= qb;
+            uint32_t pk[kBN / 2];
+            float lp[8];
+            bool need = false;
+            float m_new = m_run, alpha = 1.f;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) lp[x] = 0.f;
+            if (live) {
             float s[kBN];
 #pragma unroll
             for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
             tc::tmem_ld_wait();
             const int j0 = t * kBN;
             // Band tiles (this block's diagonal tile and the one before it):
-            // causal -inf mask, and the Mask_0 correction of the D_m (< kCorrW)
-            // diagonals below the main one.  Tiles past the diagonal (the
-            // first block of a pair runs one) are masked entirely.  The
+            // causal -inf mask on the diagonal tile, and the Mask_0 correction
+            // of the D_m (< kCorrW) diagonals below the main one.  The
             // correction column depends on the row, so the chunks it touches go
             // through the thread's scratch row in shared memory.
             if (t >= qb - 1) {
                 const int bse = i_row - j0;        // column of key i_row (>= 128 before the diagonal)
-                if (t >= qb) {
+                if (t == qb) {
 #pragma unroll
                     for (int c = 0; c < kBN; ++c) s[c] = (c > bse) ? -INFINITY : s[c];
                 }
@@ -714,19 +728,19 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                                    fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
             // the running max moves only when it grows by more than 2^8 in scale
-            const bool need = mt > m_run + 8.f;
-            const float m_new = need ? mt : m_run;
-            const float alpha = ex2(m_run - m_new);
+            need = mt > m_run + 8.f;
+            m_new = need ? mt : m_run;
+            alpha = ex2(m_run - m_new);
             // P~ = exp2(S - m), packed to bf16 pairs
-            uint32_t pk[kBN / 2];
-            float lp[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) lp[x] = 0.f;
 #pragma unroll
             for (int c = 0; c < kBN; c += 2) {
                 const float p0 = ex2(s[c] - m_new), p1 = ex2(s[c + 1] - m_new);
                 lp[(c >> 1) & 7] += p0 + p1;
                 pk[c >> 1] = pack_bf16(p0, p1);
+            }
+            } else {
+#pragma unroll
+                for (int x = 0; x < kBN / 2; ++x) pk[x] = 0u;
             }
             // Every warp waits for PV(t-1) to complete before it publishes
             // P~(t).  p_full counts arrivals from all softmax warps (of both
@@ -767,23 +781,34 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         }
         if (ok) ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (ntiles - 1) & 1, abort_flag));
         if (ok) {
+            // (w_head / l) U, 32 columns at a time: each thread puts its row's
+            // 32 values into its scratch row, then every 16-B store of the
+            // warp covers, with 8 lanes, the 128-B segment of one of 4 rows
             tc::tc_fence_after();
             const float inv_l = 1.f / l;
+            const size_t row_stride = (size_t)H * CH * D;
 #pragma unroll
             for (int hh = 0; hh < CH; ++hh) {
                 const float coef = w_head[((size_t)g * CH + hh) * CH + hl] * inv_l;
-                float *dst = part + (((size_t)b * T + i_row) * H + (g * CH + hh)) * (size_t)(CH * D) + hl * D;
+                float *dst = part + (size_t)b * T * row_stride + (size_t)(g * CH + hh) * (CH * D) + hl * D;
 #pragma unroll
                 for (int j = 0; j < D / 32; ++j) {
                     uint32_t u[32];
                     tc::tmem_ld32(lane_base + 256 + hh * D + 32 * j, u);
                     tc::tmem_ld_wait();
-                    if (i_row < T) {
+                    __syncwarp();
 #pragma unroll
-                        for (int x = 0; x < 32; x += 4)
-                            *(float4 *)(dst + 32 * j + x) = make_float4(
-                                __uint_as_float(u[x]) * coef, __uint_as_float(u[x + 1]) * coef,
-                                __uint_as_float(u[x + 2]) * coef, __uint_as_float(u[x + 3]) * coef);
+                    for (int x = 0; x < 32; x += 4)
+                        *(float4 *)(scr + x) = make_float4(
+                            __uint_as_float(u[x]) * coef, __uint_as_float(u[x + 1]) * coef,
+                            __uint_as_float(u[x + 2]) * coef, __uint_as_float(u[x + 3]) * coef);
+                    __syncwarp();
+#pragma unroll
+                    for (int rho = 0; rho < 8; ++rho) {
+                        const int rr = q4 * 32 + 4 * rho + (lane >> 3);
+                        const int ir = i0 + 16 * (rr & 7) + (rr >> 3);
+                        const float4 v = *(const float4 *)(sScr + rr * kScrStride + 4 * (lane & 7));
+                        if (ir < T) *(float4 *)(dst + (size_t)ir * row_stride + 32 * j + 4 * (lane & 7)) = v;
                     }
                 }
             }
