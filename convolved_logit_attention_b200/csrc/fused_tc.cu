@@ -47,7 +47,8 @@ namespace {
 
 constexpr int kBM = 128;          // query rows per CTA (TMEM lanes)
 constexpr int kBN = 128;          // keys per tile
-constexpr int kCorrW = 16;        // correction entries stored per row (D_m <= 14)
+constexpr int kCorrW = 16;        // correction entries stored per row (D_m <= 14); must be 16
+static_assert(kCorrW == 16, "band tiles index the table modulo 16");
 constexpr int kCorrStride = 17;   // shared-memory row stride of that table (conflict-free reads)
 constexpr int kScrStride = 36;    // floats per scratch row: 16-B aligned, conflict-free by float4
 constexpr float kLog2e = 1.4426950408889634f;
@@ -692,31 +693,40 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
 #pragma unroll
             for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
             tc::tmem_ld_wait();
-            const int j0 = t * kBN;
             // Band tiles (this block's diagonal tile and the one before it):
-            // causal -inf mask on the diagonal tile, and the Mask_0 correction
-            // of the D_m (< kCorrW) diagonals below the main one.  The
-            // correction column depends on the row, so the chunks it touches go
-            // through the thread's scratch row in shared memory.
+            // for key j0 + c the diagonal offset is e = i_row - j0 - c; keys
+            // with e < 0 are in the future (-inf), and the Mask_0 correction
+            // corr[i][e] (nonzero for e < D_m < kCorrW = 16) is subtracted.
+            // With the permuted row order i_row - i0 = 16 a + beta (a = lane & 7,
+            // beta = 4 q4 + lane / 8) and c = 16 a' + gamma, the diagonal tile
+            // has e = 16 (a - a') + beta - gamma: e lies in [0, 16) only for
+            // a' = a, gamma <= beta, or a' = a - 1, gamma > beta, and then
+            // corr[e] = corr[(beta - gamma) mod 16].  So 16 table reads per
+            // row serve the whole tile and the rest is register selects.  The
+            // tile before the diagonal has e >= 1, and e < 16 only in the rows
+            // with a = 0, at columns c = 112 + gamma with gamma > beta.
             if (t >= qb - 1) {
-                const int bse = i_row - j0;        // column of key i_row (>= 128 before the diagonal)
+                const int a = lane & 7, beta = 4 * q4 + (lane >> 3);
+                float w[kCorrW];
+#pragma unroll
+                for (int gm = 0; gm < kCorrW; ++gm) w[gm] = crow[(beta - gm) & (kCorrW - 1)];
                 if (t == qb) {
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c) s[c] = (c > bse) ? -INFINITY : s[c];
-                }
+                    for (int a2 = 0; a2 < kBN / 16; ++a2) {
+                        const bool same = a2 == a, prev = a2 == a - 1, later = a2 > a;
 #pragma unroll
-                for (int k = 0; k < kBN / 32; ++k) {
-                    if (32 * k <= bse && 32 * k + 31 >= bse - (kCorrW - 1)) {
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) scr[x] = s[32 * k + x];
-#pragma unroll
-                        for (int e = 0; e < kCorrW; ++e) {
-                            const int col = bse - e - 32 * k;
-                            if (col >= 0 && col < 32) scr[col] -= crow[e];
+                        for (int gm = 0; gm < 16; ++gm) {
+                            const int c = 16 * a2 + gm;
+                            const bool band = (gm <= beta) ? same : prev;
+                            const bool future = later || (same && gm > beta);
+                            const float v = s[c] - (band ? w[gm] : 0.f);
+                            s[c] = future ? -INFINITY : v;
                         }
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) s[32 * k + x] = scr[x];
                     }
+                } else if (a == 0) {
+#pragma unroll
+                    for (int gm = 0; gm < 16; ++gm)
+                        if (gm > beta) s[kBN - 16 + gm] -= w[gm];
                 }
             }
             // row max as 8 independent partial maxima
