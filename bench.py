@@ -178,6 +178,8 @@ def kernel_units(name, w):
         "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
         "k_fold_prologue": ("hbm", w.B * w.H * w.T * w.d * io_bytes * (2 + w.c_q + 1), "B"),
         "k_mta_fused": ("tensor", w.algorithmic_flops(), "FLOP"),
+        # read the fp32 partial outputs (c_h per output head), write out
+        "k_mix_groupnorm": ("hbm", w.B * w.T * w.H * w.d * (4 * w.c_h + io_bytes), "B"),
     }
     return table.get(name, ("unknown", 0, "FLOP"))
 
