@@ -176,7 +176,10 @@ def kernel_units(name, w):
         "k_conv": ("alu", logits * 2 * w.c_q * w.c_k, "FLOP"),
         "k_softmax_mix": ("hbm", logits * 8, "B"),            # read C, write A_new (fp32)
         "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
-        "k_fold_prologue": ("hbm", w.B * w.H * w.T * w.d * io_bytes * (2 + w.c_q + 1), "B"),
+        # read k, write the c_q folded-key copies (fp16)
+        "k_fold_keys": ("hbm", w.B * w.H * w.T * w.d * 2 * (1 + w.c_q), "B"),
+        # read q and k, write the permuted q (fp16) and the 16-entry correction rows
+        "k_fold_aux": ("hbm", w.B * w.H * w.T * (w.d * 2 * 3 + 64), "B"),
         "k_mta_fused": ("tensor", w.algorithmic_flops(), "FLOP"),
         # read the fp32 partial outputs (c_h per output head), write out
         "k_mix_groupnorm": ("hbm", w.B * w.T * w.H * w.d * (4 * w.c_h + io_bytes), "B"),

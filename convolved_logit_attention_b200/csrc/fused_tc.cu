@@ -11,14 +11,16 @@
 // floor(c_k/2) diagonals of the main one, and a per-row correction table
 // subtracts them there.
 //
-// Three kernels:
-//   k_fold_prologue  per (b, h, 128-row block): Kf^{(i')} for every i'
-//                    (fp16, scaled by log2(e)/sqrt(d) so that the softmax
-//                    runs on exp2), the query rows of the block (fp16) in the
-//                    permuted order the main kernel's shifted operand needs,
-//                    and the correction table corr[i][e] for key j = i - e.
-//                    fp16 carries three more mantissa bits than bf16 for the
-//                    folded logits; values outside its range raise an error.
+// Four kernels:
+//   k_fold_keys      per (b, h, 128-key block): Kf^{(i')} for every i' (fp16,
+//                    scaled by log2(e)/sqrt(d) so that the softmax runs on
+//                    exp2).  fp16 carries three more mantissa bits than bf16
+//                    for the folded logits; values outside its range raise an
+//                    error.
+//   k_fold_aux       per (b, h, 128-row block): the query rows of the block
+//                    (fp16) in the permuted order the main kernel's shifted
+//                    operand needs, and the correction table corr[i][e] for
+//                    key j = i - e.
 //   k_mta_fused      per (b, source head h', 128 query rows): for every key
 //                    tile, S = sum_{i'} Q_{shift i'} Kf^{(i')T} on tcgen05
 //                    (TMEM accumulator), correction + causal mask + online
@@ -73,84 +75,128 @@ __host__ __device__ inline int d_m(int c_q, int c_k) { return c_q - 1 + c_k / 2;
 constexpr int kProRows = 128;     // rows (keys and queries) per prologue CTA
 constexpr int kProQLo = 7;        // query rows before the block whose future logits are needed
 
-// One CTA per (128-row block, b*H + h), 256 threads, four sections:
-//  (a) Kf^{(i')}_j for the block's keys: thread = one column pair x a run of
-//      RPG consecutive keys.  The k rows the taps reach are loaded once into
-//      registers; theta is zero-padded to CK taps centred like the real
-//      kernel (CK = c_k for the common sizes, 15 otherwise), so every tap
-//      index is a compile-time constant.
+// Packed fp32 pairs (Blackwell's f32x2 arithmetic): one instruction does two
+// fp32 FMAs, each rounded once, exactly as fmaf would.
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long v)
+{
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// A bf16 pair as a packed fp32 pair (widening is exact).
+__device__ __forceinline__ unsigned long long bf2_to_f2(uint32_t v)
+{
+    return f2_pack(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+// Folded keys: one CTA per (128-key block, b*H + h), 256 threads; thread =
+// one column pair x a run of RPG consecutive keys, in windows of SUB keys.
+// Kf^{(i')}_j = sum_jj ths[i'][jj] k_{j + RT - jj}, with the taps zero-padded
+// to CK (CK = c_k for the common sizes, 15 otherwise) and centred like the
+// real kernel, so every tap index is a compile-time constant.  The two
+// columns of a pair share every tap: one packed f32x2 FMA per tap.
+template <int D, int CK>
+__global__ void __launch_bounds__(256, 3)
+k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
+            __half *__restrict__ kf, int T, int Tp, int H, int c_q, int c_k, float scale)
+{
+    constexpr int EP = D / 2;                  // column pairs
+    constexpr int RG = 256 / EP;               // key runs per block
+    constexpr int RPG = kProRows / RG;         // keys per run
+    constexpr int RT = CK / 2, LT = CK - 1 - RT;
+    constexpr int SUB = 16;
+    constexpr int WS = SUB + CK - 1;           // window rows
+    __shared__ float ths[8 * CK];              // zero-padded taps times the logit scale
+    const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
+    const int j0 = blk * kProRows;
+    const int tid = threadIdx.x;
+    const int R = c_k / 2, shift = RT - R;     // real tap jj sits at padded index jj + shift
+    for (int idx = tid; idx < 8 * CK; idx += 256) {
+        const int ip = idx / CK, jp = idx % CK - shift;
+        ths[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] * scale
+                                                     : 0.f;
+    }
+    __syncthreads();
+    const int ep = tid % EP, rg = tid / EP;
+    const __nv_bfloat16 *kh = k + (size_t)bh * T * D + 2 * ep;
+    __half2 amax = __floats2half2_rn(0.f, 0.f);   // largest |Kf| this thread wrote, per column
+#pragma unroll 1
+    for (int sub = 0; sub < RPG / SUB; ++sub) {
+        const int jr0 = j0 + rg * RPG + sub * SUB;     // first key of the window
+        unsigned long long win[WS];
+#pragma unroll
+        for (int w = 0; w < WS; ++w) {
+            const int row = jr0 - LT + w;
+            const uint32_t v = (row >= 0 && row < T) ? *(const uint32_t *)(kh + (size_t)row * D) : 0u;
+            win[w] = bf2_to_f2(v);
+        }
+        for (int ip = 0; ip < c_q; ++ip) {
+            unsigned long long tt[CK];
+#pragma unroll
+            for (int jj = 0; jj < CK; ++jj) {
+                const float t = ths[ip * CK + jj];
+                tt[jj] = f2_pack(t, t);
+            }
+            __half *dst = kf + (((size_t)bh * c_q + ip) * Tp + jr0) * D + 2 * ep;
+#pragma unroll
+            for (int r = 0; r < SUB; ++r) {
+                unsigned long long acc = 0ull;
+#pragma unroll
+                for (int jj = 0; jj < CK; ++jj) acc = f2_fma(tt[jj], win[r + CK - 1 - jj], acc);
+                const float2 a = f2_unpack(acc);
+                const __half2 hv = __floats2half2_rn(a.x, a.y);
+                amax = __hmax2(amax, __habs2(hv));
+                *(__half2 *)(dst + (size_t)r * D) = hv;
+            }
+        }
+    }
+    // a folded key beyond the fp16 range became infinite (NaN inputs stay NaN)
+    const float2 am = __half22float2(amax);
+    if (am.x > 65504.f || am.y > 65504.f) atomicOr(&g_fused_error, kErrRange);
+}
+
+// The rest of the prologue: one CTA per (128-row block, b*H + h), 256
+// threads, three sections:
 //  (b) the block's query rows in the permuted atom order, converted to fp16.
 //  (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in
 //      [1, D_m], for r in [j0 - 7, j0 + 128), from shared-memory copies of
 //      the rows involved.
 //  (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
 //      r = i - i' >= 0 of theta[i'][j'] F[r][delta].
-template <int D, int CK>
+template <int D>
 __global__ void __launch_bounds__(256, 2)
-k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                const float *__restrict__ w_kq, __half *__restrict__ kf,
-                __half *__restrict__ qp, float *__restrict__ corr, int T, int Tp, int H,
-                int c_q, int c_k, float scale)
+k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+           const float *__restrict__ w_kq, __half *__restrict__ qp, float *__restrict__ corr, int T,
+           int Tp, int H, int c_q, int c_k, float scale)
 {
-    constexpr int EP = D / 2;                  // column pairs
-    constexpr int RG = 256 / EP;               // key runs per block
-    constexpr int RPG = kProRows / RG;         // keys per run
-    constexpr int RT = CK / 2, LT = CK - 1 - RT;
     constexpr int QR = kProQLo + kProRows;
-    __shared__ float th[8 * CK];               // zero-padded taps
+    constexpr int TW = 16;                     // tap row stride (c_k <= 15)
+    __shared__ float th[8 * TW];
     __shared__ float fs[QR * kCorrW];
     extern __shared__ __align__(16) __nv_bfloat16 qk_sm[];   // section (c) row copies
     const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
     const int j0 = blk * kProRows;
     const int tid = threadIdx.x;
     const size_t head_off = (size_t)bh * T * D;
-    const int R = c_k / 2, shift = RT - R;     // real tap jj sits at padded index jj + shift
-    for (int idx = tid; idx < 8 * CK; idx += 256) {
-        const int ip = idx / CK, jp = idx % CK - shift;
-        th[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] : 0.f;
+    const int R = c_k / 2;
+    for (int idx = tid; idx < 8 * TW; idx += 256) {
+        const int ip = idx / TW, jj = idx % TW;
+        th[idx] = (ip < c_q && jj < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jj] : 0.f;
     }
-    __shared__ float ths[8 * CK];              // the same taps times the logit scale
-    for (int idx = tid; idx < 8 * CK; idx += 256) ths[idx] = th[idx] * scale;
     __syncthreads();
-
-    // (a) folded keys, in windows of SUB consecutive keys
-    {
-        constexpr int SUB = 16;
-        constexpr int WS = SUB + CK - 1;           // window rows
-        const int ep = tid % EP, rg = tid / EP;
-        float amax = 0.f;                          // largest |Kf| written by this thread
-#pragma unroll 1
-        for (int sub = 0; sub < RPG / SUB; ++sub) {
-            const int jr0 = j0 + rg * RPG + sub * SUB;     // first key of the window
-            float2 win[WS];
-#pragma unroll
-            for (int w = 0; w < WS; ++w) {
-                const int row = jr0 - LT + w;
-                float2 v = make_float2(0.f, 0.f);
-                if (row >= 0 && row < T)
-                    v = __bfloat1622float2(*(const __nv_bfloat162 *)(k + head_off + (size_t)row * D + 2 * ep));
-                win[w] = v;
-            }
-            for (int ip = 0; ip < c_q; ++ip) {
-                float t[CK];
-#pragma unroll
-                for (int jj = 0; jj < CK; ++jj) t[jj] = ths[ip * CK + jj];
-                __half *dst = kf + (((size_t)bh * c_q + ip) * Tp + jr0) * D + 2 * ep;
-#pragma unroll
-                for (int r = 0; r < SUB; ++r) {
-                    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-                    for (int jj = 0; jj < CK; ++jj) {
-                        a0 = fmaf(t[jj], win[r + CK - 1 - jj].x, a0);
-                        a1 = fmaf(t[jj], win[r + CK - 1 - jj].y, a1);
-                    }
-                    amax = fmaxf(amax, fmaxf(fabsf(a0), fabsf(a1)));
-                    *(__half2 *)(dst + (size_t)r * D) = __floats2half2_rn(a0, a1);
-                }
-            }
-        }
-        if (amax > 65504.f) atomicOr(&g_fused_error, kErrRange);   // NaN inputs propagate as NaN
-    }
     // (b) permuted query rows: atom a, row s <- q_{j0-(c_q-1)+a+16s}; 8 elements per thread
     {
         const int NA = q_atoms(c_q);
@@ -197,49 +243,74 @@ k_fold_prologue(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
             *(uint4 *)((isq ? qsm + row * RS : ksm + (row - QR) * RS) + 8 * c8) = v;
         }
         __syncthreads();
-        for (int idx = tid; idx < QR * Dm; idx += 256) {
-            const int rr = idx / Dm, dl = idx % Dm + 1;
-            const int r = j0 - kProQLo + rr, c = r + dl;
-            float acc = 0.f;
-            if (r >= 0 && c < T) {
+        // work item = (row rr, half of the diagonals): 7 independent packed
+        // accumulator chains share each loaded chunk of q_r
+        constexpr int DH = (kCorrW - 2) / 2;   // diagonals per half (delta <= 14)
+        for (int w = tid; w < 2 * QR; w += 256) {
+            const int rr = w >> 1, d0 = 1 + (w & 1) * DH;
+            const int r = j0 - kProQLo + rr;
+            unsigned long long acc[DH];
+#pragma unroll
+            for (int x = 0; x < DH; ++x) acc[x] = 0ull;
+            if (r >= 0) {
                 const __nv_bfloat16 *qr = qsm + rr * RS;
-                const __nv_bfloat16 *kc = ksm + (rr + dl - 1) * RS;   // k row c = j0-6+(rr+dl-1)
-#pragma unroll 4
+                const __nv_bfloat16 *kc = ksm + (rr + d0 - 1) * RS;   // k row r + d0
+#pragma unroll 2
                 for (int c8 = 0; c8 < CPR; ++c8) {
                     const uint4 a4 = *(const uint4 *)(qr + 8 * c8);
-                    const uint4 b4 = *(const uint4 *)(kc + 8 * c8);
-                    const __nv_bfloat162 *a2 = (const __nv_bfloat162 *)&a4;
-                    const __nv_bfloat162 *b2 = (const __nv_bfloat162 *)&b4;
+                    const unsigned long long qa0 = bf2_to_f2(a4.x), qa1 = bf2_to_f2(a4.y),
+                                             qa2 = bf2_to_f2(a4.z), qa3 = bf2_to_f2(a4.w);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 x = __bfloat1622float2(a2[u]), y = __bfloat1622float2(b2[u]);
-                        acc = fmaf(x.x, y.x, acc);
-                        acc = fmaf(x.y, y.y, acc);
+                    for (int x = 0; x < DH; ++x) {
+                        const uint4 b4 = *(const uint4 *)(kc + x * RS + 8 * c8);
+                        acc[x] = f2_fma(qa0, bf2_to_f2(b4.x), acc[x]);
+                        acc[x] = f2_fma(qa1, bf2_to_f2(b4.y), acc[x]);
+                        acc[x] = f2_fma(qa2, bf2_to_f2(b4.z), acc[x]);
+                        acc[x] = f2_fma(qa3, bf2_to_f2(b4.w), acc[x]);
                     }
                 }
             }
-            fs[rr * kCorrW + dl - 1] = acc * scale;
-        }
-    }
-    __syncthreads();
-    // (d) correction table
-    for (int idx = tid; idx < kProRows * kCorrW; idx += 256) {
-        const int ir = idx / kCorrW, e = idx % kCorrW;
-        const int i = j0 + ir;
-        float acc = 0.f;
-        if (e < Dm) {
-            for (int ip = 0; ip < c_q; ++ip) {
-                const int r = i - ip;
-                if (r < 0) continue;
-                // taps with delta = ip - (jj - R) - e >= 1, i.e. jj <= ip + R - e - 1
-                const int jmax = min(c_k - 1, ip + R - e - 1);
-                const float *frow = fs + (r - (j0 - kProQLo)) * kCorrW;
-                const float *trow = th + ip * CK + shift;
-                for (int jj = 0; jj <= jmax; ++jj)
-                    acc = fmaf(trow[jj], frow[ip + R - e - jj - 1], acc);
+#pragma unroll
+            for (int x = 0; x < DH; ++x) {
+                const int dl = d0 + x;
+                const float2 a2 = f2_unpack(acc[x]);
+                fs[rr * kCorrW + dl - 1] = (r >= 0 && dl <= Dm && r + dl < T) ? (a2.x + a2.y) * scale : 0.f;
             }
         }
-        corr[((size_t)bh * Tp + i) * kCorrW + e] = acc;
+    }
+    // taps indexed by s = e + delta: ts[i'][s] = theta[i'][i' + R - s]
+    __shared__ float ts[8 * 32];
+    for (int idx = tid; idx < 8 * 32; idx += 256) {
+        const int ip = idx / 32, jj = ip + R - idx % 32;
+        ts[idx] = (ip < c_q && jj >= 0 && jj < c_k) ? th[ip * TW + jj] : 0.f;
+    }
+    __syncthreads();
+    // (d) correction table: thread = one row i, all 16 entries e.
+    //     corr[i][e] = sum_{i'} sum_{delta} ts[i'][e + delta] F[i - i'][delta];
+    //     taps with delta < 1 or jj outside [0, c_k) are zero in ts, F rows
+    //     before the sequence are zero, so e >= D_m comes out zero too.
+    if (tid < kProRows) {
+        const int ir = tid, i = j0 + ir;
+        float acc[kCorrW];
+#pragma unroll
+        for (int e = 0; e < kCorrW; ++e) acc[e] = 0.f;
+        for (int ip = 0; ip < c_q; ++ip) {
+            const float *frow = fs + (ir + kProQLo - ip) * kCorrW;   // F row i - i'
+            const float *trow = ts + ip * 32;
+            float f[kCorrW - 2], t[2 * kCorrW - 2];
+#pragma unroll
+            for (int x = 0; x < kCorrW - 2; ++x) f[x] = frow[x];
+#pragma unroll
+            for (int x = 1; x < 2 * kCorrW - 2; ++x) t[x] = trow[x];
+#pragma unroll
+            for (int e = 0; e < kCorrW; ++e)
+#pragma unroll
+                for (int dl = 1; dl <= kCorrW - 2; ++dl) acc[e] = fmaf(t[e + dl], f[dl - 1], acc[e]);
+        }
+        float4 *dst = (float4 *)(corr + ((size_t)bh * Tp + i) * kCorrW);
+#pragma unroll
+        for (int u = 0; u < kCorrW / 4; ++u)
+            dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
     }
 }
 
@@ -920,7 +991,7 @@ FusedLayout fused_layout(const mta_shape &s)
     return L;
 }
 
-const char *const kFusedNames[3] = {"k_fold_prologue", "k_mta_fused", "k_mix_groupnorm"};
+const char *const kFusedNames[4] = {"k_fold_keys", "k_fold_aux", "k_mta_fused", "k_mix_groupnorm"};
 
 template <int D, int CH>
 mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
@@ -955,22 +1026,26 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         if (!make_tmap_bf16(&mV, a.v, 3, dims, strides, box)) return MTA_ERR_CUDA;
     }
     auto main_kernel = k_mta_fused<D, CH, PAIR>;
-    auto prologue = s.c_k == 11 ? k_fold_prologue<D, 11>
-                  : s.c_k == 3  ? k_fold_prologue<D, 3>
-                                : k_fold_prologue<D, 15>;
-    const int pro_smem = (int)prologue_smem_bytes(D);
+    auto fold_keys = s.c_k == 11 ? k_fold_keys<D, 11>
+                   : s.c_k == 3  ? k_fold_keys<D, 3>
+                                 : k_fold_keys<D, 15>;
+    const int aux_smem = (int)prologue_smem_bytes(D);
     if (cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, pro_smem) !=
+        cudaFuncSetAttribute(k_fold_aux<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, aux_smem) !=
             cudaSuccess)
         return MTA_ERR_CUDA;
     const float scale = kLog2e / sqrtf((float)D);
     tr.before(0, st);
-    prologue<<<dim3(L.nqb, (unsigned)BH), 256, pro_smem, st>>>(
-        (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, kf, qp, corr, s.T, L.Tp,
-        s.H, s.c_q, s.c_k, scale);
+    fold_keys<<<dim3(L.nqb, (unsigned)BH), 256, 0, st>>>((const __nv_bfloat16 *)a.k, a.w_kq, kf, s.T,
+                                                         L.Tp, s.H, s.c_q, s.c_k, scale);
     tr.after(0, st);
     tr.before(1, st);
+    k_fold_aux<D><<<dim3(L.nqb, (unsigned)BH), 256, aux_smem, st>>>(
+        (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, qp, corr, s.T, L.Tp, s.H,
+        s.c_q, s.c_k, scale);
+    tr.after(1, st);
+    tr.before(2, st);
     {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = PAIR ? dim3(2 * s.B * s.H, L.nqb / 2, 1) : dim3(s.B * s.H, L.nqb, 1);
@@ -988,12 +1063,12 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
                                s.T, L.Tp, s.H, s.c_q, L.nqb) != cudaSuccess)
             return MTA_ERR_CUDA;
     }
-    tr.after(1, st);
-    tr.before(2, st);
+    tr.after(2, st);
+    tr.before(3, st);
     k_mix_groupnorm<D, CH><<<dim3(s.T, s.B), 128, 0, st>>>(part, a.gn_weight, a.gn_bias,
                                                          a.depth_scale, s.gn_eps,
                                                          (__nv_bfloat16 *)a.out, s.T, s.H);
-    tr.after(2, st);
+    tr.after(3, st);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
@@ -1010,11 +1085,11 @@ bool fused_supported(const mta_shape &s)
 
 size_t fused_workspace_bytes(const mta_shape &s) { return fused_layout(s).total; }
 
-int fused_kernel_count(const mta_shape &) { return 3; }
+int fused_kernel_count(const mta_shape &) { return 4; }
 
 const char *fused_kernel_name(const mta_shape &, int index)
 {
-    return (index >= 0 && index < 3) ? kFusedNames[index] : nullptr;
+    return (index >= 0 && index < 4) ? kFusedNames[index] : nullptr;
 }
 
 mta_status launch_fused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
