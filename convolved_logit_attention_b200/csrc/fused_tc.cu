@@ -197,51 +197,50 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
         th[idx] = (ip < c_q && jj < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jj] : 0.f;
     }
     __syncthreads();
-    // (b) permuted query rows: atom a, row s <- q_{j0-(c_q-1)+a+16s}; 8 elements per thread
+    // Row copies in shared memory, all in flight at once (cp.async): q rows
+    // [j0-7, j0+128) and k rows [j0-6, j0+142), zero outside [0, T); rows are
+    // padded by 16 bytes so that threads on different rows hit different banks.
+    constexpr int RS = D + 8;                  // padded row stride in bf16 elements
+    constexpr int KR = QR + kCorrW - 3;        // k rows j0-6 .. j0+141 (r + delta <= j0+127+14)
+    constexpr int CPR = D / 8;                 // 16-byte chunks per row
+    __nv_bfloat16 *qsm = qk_sm;                // [QR][RS]
+    __nv_bfloat16 *ksm = qk_sm + QR * RS;      // [KR][RS]
+    for (int idx = tid; idx < (QR + KR) * CPR; idx += 256) {
+        const int row = idx / CPR, c8 = idx % CPR;
+        const bool isq = row < QR;
+        const int g = isq ? j0 - kProQLo + row : j0 - (kProQLo - 1) + (row - QR);
+        const bool in = g >= 0 && g < T;
+        const __nv_bfloat16 *src = (isq ? q : k) + head_off + (size_t)(in ? g : 0) * D + 8 * c8;
+        tc::cp_async16((isq ? qsm + row * RS : ksm + (row - QR) * RS) + 8 * c8, src, in);
+    }
+    tc::cp_async_wait_all();
+    __syncthreads();
+    // (b) permuted query rows: atom a, row s <- q_{j0-(c_q-1)+a+16s}, from the
+    //     copy (those rows lie in [j0-7, j0+128) since c_q <= 8); 8 elements per thread
     {
         const int NA = q_atoms(c_q);
         __half *dst = qp + ((size_t)bh * (Tp / kBM) + blk) * (size_t)NA * 8 * D;
-        constexpr int CPR = D / 8;             // 16-byte chunks per row
         bool range_ok = true;
         for (int idx = tid; idx < NA * 8 * CPR; idx += 256) {
             const int row = idx / CPR, c8 = idx % CPR;
-            const int i = j0 - (c_q - 1) + row / 8 + 16 * (row % 8);
-            uint4 outv = make_uint4(0, 0, 0, 0);
-            if (i >= 0 && i < T) {
-                const uint4 in = *(const uint4 *)(q + head_off + (size_t)i * D + 8 * c8);
-                const __nv_bfloat162 *bp = (const __nv_bfloat162 *)&in;
-                __half2 *hp = (__half2 *)&outv;
+            const int rq = kProQLo - (c_q - 1) + row / 8 + 16 * (row % 8);   // copy row of q_i
+            const uint4 in = *(const uint4 *)(qsm + rq * RS + 8 * c8);
+            const __nv_bfloat162 *bp = (const __nv_bfloat162 *)&in;
+            uint4 outv;
+            __half2 *hp = (__half2 *)&outv;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float2 f = __bfloat1622float2(bp[u]);
-                    range_ok &= fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
-                    hp[u] = __floats2half2_rn(f.x, f.y);
-                }
+            for (int u = 0; u < 4; ++u) {
+                const float2 f = __bfloat1622float2(bp[u]);
+                range_ok &= fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
+                hp[u] = __floats2half2_rn(f.x, f.y);
             }
             *(uint4 *)(dst + (size_t)row * D + 8 * c8) = outv;
         }
         if (!range_ok) atomicOr(&g_fused_error, kErrRange);
     }
-    // (c) future logits from shared-memory copies of the rows they need
-    //     (q rows [j0-7, j0+128), k rows [j0-6, j0+142)), one dot product of
-    //     length d per thread at a time; rows are padded by 16 bytes so that
-    //     threads on different rows hit different banks.
+    // (c) future logits F[r][delta] = scale * q_r . k_{r+delta} from the copies
     const int Dm = d_m(c_q, c_k);
     {
-        constexpr int RS = D + 8;              // padded row stride in bf16 elements
-        constexpr int KR = QR + kCorrW - 3;    // k rows j0-6 .. j0+141 (r + delta <= j0+127+14)
-        __nv_bfloat16 *qsm = qk_sm;            // [QR][RS]
-        __nv_bfloat16 *ksm = qk_sm + QR * RS;  // [KR][RS]
-        constexpr int CPR = D / 8;
-        for (int idx = tid; idx < (QR + KR) * CPR; idx += 256) {
-            const int row = idx / CPR, c8 = idx % CPR;
-            const bool isq = row < QR;
-            const int g = isq ? j0 - kProQLo + row : j0 - (kProQLo - 1) + (row - QR);
-            const __nv_bfloat16 *src = isq ? q : k;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (g >= 0 && g < T) v = *(const uint4 *)(src + head_off + (size_t)g * D + 8 * c8);
-            *(uint4 *)((isq ? qsm + row * RS : ksm + (row - QR) * RS) + 8 * c8) = v;
-        }
         __syncthreads();
         // work item = (row rr, half of the diagonals): 7 independent packed
         // accumulator chains share each loaded chunk of q_r

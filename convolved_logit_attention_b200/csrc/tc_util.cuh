@@ -87,6 +87,19 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count)
     asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (cp.async); with `valid` false
+// nothing is read and the 16 bytes are zero-filled.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy reads (tensor-core operands).
 __device__ __forceinline__ void fence_async_shared()
