@@ -74,6 +74,7 @@ __host__ __device__ inline int d_m(int c_q, int c_k) { return c_q - 1 + c_k / 2;
 
 constexpr int kProRows = 128;     // rows (keys and queries) per prologue CTA
 constexpr int kProQLo = 7;        // query rows before the block whose future logits are needed
+constexpr int kAuxThreads = 288;  // aux prologue: one future-logit work item per thread
 
 // Packed fp32 pairs (Blackwell's f32x2 arithmetic): one instruction does two
 // fp32 FMAs, each rounded once, exactly as fmaf would.
@@ -168,7 +169,7 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
     if (am.x > 65504.f || am.y > 65504.f) atomicOr(&g_fused_error, kErrRange);
 }
 
-// The rest of the prologue: one CTA per (128-row block, b*H + h), 256
+// The rest of the prologue: one CTA per (128-row block, b*H + h), 288
 // threads, three sections:
 //  (b) the block's query rows in the permuted atom order, converted to fp16.
 //  (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in
@@ -177,7 +178,7 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
 //  (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
 //      r = i - i' >= 0 of theta[i'][j'] F[r][delta].
 template <int D>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(kAuxThreads, 2)
 k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
            const float *__restrict__ w_kq, __half *__restrict__ qp, float *__restrict__ corr, int T,
            int Tp, int H, int c_q, int c_k, float scale)
@@ -192,7 +193,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     const int tid = threadIdx.x;
     const size_t head_off = (size_t)bh * T * D;
     const int R = c_k / 2;
-    for (int idx = tid; idx < 8 * TW; idx += 256) {
+    for (int idx = tid; idx < 8 * TW; idx += kAuxThreads) {
         const int ip = idx / TW, jj = idx % TW;
         th[idx] = (ip < c_q && jj < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jj] : 0.f;
     }
@@ -205,7 +206,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     constexpr int CPR = D / 8;                 // 16-byte chunks per row
     __nv_bfloat16 *qsm = qk_sm;                // [QR][RS]
     __nv_bfloat16 *ksm = qk_sm + QR * RS;      // [KR][RS]
-    for (int idx = tid; idx < (QR + KR) * CPR; idx += 256) {
+    for (int idx = tid; idx < (QR + KR) * CPR; idx += kAuxThreads) {
         const int row = idx / CPR, c8 = idx % CPR;
         const bool isq = row < QR;
         const int g = isq ? j0 - kProQLo + row : j0 - (kProQLo - 1) + (row - QR);
@@ -221,7 +222,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
         const int NA = q_atoms(c_q);
         __half *dst = qp + ((size_t)bh * (Tp / kBM) + blk) * (size_t)NA * 8 * D;
         bool range_ok = true;
-        for (int idx = tid; idx < NA * 8 * CPR; idx += 256) {
+        for (int idx = tid; idx < NA * 8 * CPR; idx += kAuxThreads) {
             const int row = idx / CPR, c8 = idx % CPR;
             const int rq = kProQLo - (c_q - 1) + row / 8 + 16 * (row % 8);   // copy row of q_i
             const uint4 in = *(const uint4 *)(qsm + rq * RS + 8 * c8);
@@ -245,7 +246,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
         // work item = (row rr, half of the diagonals): 7 independent packed
         // accumulator chains share each loaded chunk of q_r
         constexpr int DH = (kCorrW - 2) / 2;   // diagonals per half (delta <= 14)
-        for (int w = tid; w < 2 * QR; w += 256) {
+        for (int w = tid; w < 2 * QR; w += kAuxThreads) {
             const int rr = w >> 1, d0 = 1 + (w & 1) * DH;
             const int r = j0 - kProQLo + rr;
             unsigned long long acc[DH];
@@ -279,36 +280,37 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
     // taps indexed by s = e + delta: ts[i'][s] = theta[i'][i' + R - s]
     __shared__ float ts[8 * 32];
-    for (int idx = tid; idx < 8 * 32; idx += 256) {
+    for (int idx = tid; idx < 8 * 32; idx += kAuxThreads) {
         const int ip = idx / 32, jj = ip + R - idx % 32;
         ts[idx] = (ip < c_q && jj >= 0 && jj < c_k) ? th[ip * TW + jj] : 0.f;
     }
     __syncthreads();
-    // (d) correction table: thread = one row i, all 16 entries e.
+    // (d) correction table: thread = one row i and 8 of its 16 entries e.
     //     corr[i][e] = sum_{i'} sum_{delta} ts[i'][e + delta] F[i - i'][delta];
     //     taps with delta < 1 or jj outside [0, c_k) are zero in ts, F rows
     //     before the sequence are zero, so e >= D_m comes out zero too.
-    if (tid < kProRows) {
-        const int ir = tid, i = j0 + ir;
-        float acc[kCorrW];
+    if (tid < 2 * kProRows) {
+        constexpr int EH = kCorrW / 2;
+        const int ir = tid >> 1, e0 = (tid & 1) * EH, i = j0 + ir;
+        float acc[EH];
 #pragma unroll
-        for (int e = 0; e < kCorrW; ++e) acc[e] = 0.f;
+        for (int e = 0; e < EH; ++e) acc[e] = 0.f;
         for (int ip = 0; ip < c_q; ++ip) {
             const float *frow = fs + (ir + kProQLo - ip) * kCorrW;   // F row i - i'
-            const float *trow = ts + ip * 32;
-            float f[kCorrW - 2], t[2 * kCorrW - 2];
+            const float *trow = ts + ip * 32 + e0;
+            float f[kCorrW - 2], t[EH + kCorrW - 2];
 #pragma unroll
             for (int x = 0; x < kCorrW - 2; ++x) f[x] = frow[x];
 #pragma unroll
-            for (int x = 1; x < 2 * kCorrW - 2; ++x) t[x] = trow[x];
+            for (int x = 1; x < EH + kCorrW - 2; ++x) t[x] = trow[x];
 #pragma unroll
-            for (int e = 0; e < kCorrW; ++e)
+            for (int e = 0; e < EH; ++e)
 #pragma unroll
                 for (int dl = 1; dl <= kCorrW - 2; ++dl) acc[e] = fmaf(t[e + dl], f[dl - 1], acc[e]);
         }
-        float4 *dst = (float4 *)(corr + ((size_t)bh * Tp + i) * kCorrW);
+        float4 *dst = (float4 *)(corr + ((size_t)bh * Tp + i) * kCorrW + e0);
 #pragma unroll
-        for (int u = 0; u < kCorrW / 4; ++u)
+        for (int u = 0; u < EH / 4; ++u)
             dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
     }
 }
@@ -992,6 +994,36 @@ FusedLayout fused_layout(const mta_shape &s)
 
 const char *const kFusedNames[4] = {"k_fold_keys", "k_fold_aux", "k_mta_fused", "k_mix_groupnorm"};
 
+// The two prologue kernels are independent and bound by different units
+// (FMA issue vs load latency), so k_fold_aux runs on a side stream of the
+// library while k_fold_keys runs on the caller's stream; the caller's stream
+// forks to the side stream and joins back before the main kernel.  One side
+// stream and event pair per device; the fork/join sequence is enqueued under
+// a lock so that concurrent callers cannot interleave their event records.
+// The pattern is also legal under stream capture.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_lock;
+
+mta_status side_stream(SideStream *out)
+{
+    constexpr int kMaxDevices = 64;
+    static SideStream tab[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTA_ERR_CUDA;
+    SideStream &ss = tab[dev];
+    if (!ss.s) {
+        if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess)
+            return MTA_ERR_CUDA;
+    }
+    *out = ss;
+    return MTA_OK;
+}
+
 template <int D, int CH>
 mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr)
@@ -1035,15 +1067,26 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
             cudaSuccess)
         return MTA_ERR_CUDA;
     const float scale = kLog2e / sqrtf((float)D);
-    tr.before(0, st);
-    fold_keys<<<dim3(L.nqb, (unsigned)BH), 256, 0, st>>>((const __nv_bfloat16 *)a.k, a.w_kq, kf, s.T,
-                                                         L.Tp, s.H, s.c_q, s.c_k, scale);
-    tr.after(0, st);
-    tr.before(1, st);
-    k_fold_aux<D><<<dim3(L.nqb, (unsigned)BH), 256, aux_smem, st>>>(
-        (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, qp, corr, s.T, L.Tp, s.H,
-        s.c_q, s.c_k, scale);
-    tr.after(1, st);
+    {
+        std::lock_guard<std::mutex> guard(g_side_lock);
+        SideStream side;
+        if (side_stream(&side) != MTA_OK) return MTA_ERR_CUDA;
+        if (cudaEventRecord(side.fork, st) != cudaSuccess ||
+            cudaStreamWaitEvent(side.s, side.fork, 0) != cudaSuccess)
+            return MTA_ERR_CUDA;
+        tr.before(1, side.s);
+        k_fold_aux<D><<<dim3(L.nqb, (unsigned)BH), kAuxThreads, aux_smem, side.s>>>(
+            (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, qp, corr, s.T, L.Tp, s.H,
+            s.c_q, s.c_k, scale);
+        tr.after(1, side.s);
+        tr.before(0, st);
+        fold_keys<<<dim3(L.nqb, (unsigned)BH), 256, 0, st>>>((const __nv_bfloat16 *)a.k, a.w_kq, kf,
+                                                             s.T, L.Tp, s.H, s.c_q, s.c_k, scale);
+        tr.after(0, st);
+        if (cudaEventRecord(side.join, side.s) != cudaSuccess ||
+            cudaStreamWaitEvent(st, side.join, 0) != cudaSuccess)
+            return MTA_ERR_CUDA;
+    }
     tr.before(2, st);
     {
         cudaLaunchConfig_t cfg = {};
