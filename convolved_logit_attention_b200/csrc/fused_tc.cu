@@ -27,7 +27,7 @@
 //                    softmax on CUDA cores, then U^{h,h'} += P~ V^h for every
 //                    head h of the group (post-softmax head mixing, Eq. (7),
 //                    with per-source-head normalisation deferred to the end).
-//                    Writes (w[h][h'] / l^{h'}) U^{h,h'} per row.
+//                    Writes (w[h][h'] / l^{h'}) U^{h,h'} per row, in fp16.
 //   k_mix_groupnorm  per (b, query row): O^h = sum_{h'} of those partials,
 //                    per-head GroupNorm with warp-shuffle reductions, depth
 //                    scale, bf16 store.
@@ -382,6 +382,12 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
 }
 
+__device__ __forceinline__ uint32_t pack_h2(float a, float b)
+{
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -418,6 +424,40 @@ __device__ __forceinline__ void arrive_leader(uint64_t *bar)
     else tc::mbar_arrive(bar);
 }
 
+// Work items of the persistent main kernel: (b, h, query block) without
+// pairs, (b, h, pair of blocks) with them.  The list is ordered by decreasing
+// length (key tiles), and cluster cl takes one item per round, snaking across
+// the clusters (left to right in even rounds, right to left in odd ones), so
+// every role derives the same sequence with no communication.
+struct WorkItem {
+    int bh, b, g, hl, qb, i0, ntiles;
+};
+
+template <bool PAIR>
+__device__ __forceinline__ bool work_item(int k, int cl, int ncl, int BH, int H, int CH, int nqb,
+                                          uint32_t rank, WorkItem &it)
+{
+    const int per_head = PAIR ? nqb / 2 : nqb;
+    const int pos = k * ncl + ((k & 1) ? ncl - 1 - cl : cl);
+    if (pos >= per_head * BH) return false;
+    const int cls = pos / BH, bhx = pos % BH;
+    const int hs = bhx % H;
+    it.bh = bhx;
+    it.b = bhx / H;
+    it.g = hs / CH;
+    it.hl = hs % CH;
+    if (PAIR) {
+        const int pair = per_head - 1 - cls;
+        it.qb = 2 * pair + (int)rank;
+        it.ntiles = 2 * pair + 2;     // both CTAs run to the diagonal of block 2p+1
+    } else {
+        it.qb = nqb - 1 - cls;
+        it.ntiles = it.qb + 1;
+    }
+    it.i0 = it.qb * kBM;
+    return true;
+}
+
 // Block 224 threads = warp 0 TMA producer,
 // warp 1 MMA issuer (and TMEM owner), warps 2..5 softmax / epilogue (one TMEM
 // lane, i.e. one query row, per thread), warp 6 gate of the issuer.  TMEM columns: S double buffer at
@@ -429,8 +469,8 @@ template <int D, int CH, bool PAIR>
 __global__ void __launch_bounds__(224, 1)
 k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
             const __grid_constant__ CUtensorMap mapV, const float *__restrict__ corr,
-            const float *__restrict__ w_head, float *__restrict__ part, int T, int Tp, int H,
-            int c_q, int nqb)
+            const float *__restrict__ w_head, __half *__restrict__ part, int T, int Tp, int H,
+            int c_q, int nqb, int nbh)
 {
     using C = FusedCfg<D, CH, PAIR>;
     static_assert(C::kStages <= kGateQ - kGateStage0, "one gate barrier id per ring slot");
@@ -447,30 +487,24 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 1;
     uint64_t *mma_drain = pv_done + 1;
-    uint32_t *tmem_slot = (uint32_t *)(mma_drain + 1);
+
+    uint64_t *q_free = mma_drain + 1;
+    uint32_t *tmem_slot = (uint32_t *)(q_free + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
-    // Grid: x = (batch, head) [x2 CTAs per pair], y = query block (pair) in
-    // reverse order, so the longest blocks of every head start first.
+    // Persistent grid: cluster cl of ncl walks its work items (work_item);
+    // every role keeps its ring slot, barrier phases and the global key-tile
+    // counter gt running across items.
     const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
     const bool leader = rank == 0;
-    int qb, ntiles;
-    const int bhx = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    if constexpr (PAIR) {
-        const int pair = nqb / 2 - 1 - (int)blockIdx.y;
-        qb = 2 * pair + (int)rank;
-        ntiles = 2 * pair + 2;        // both CTAs run to the diagonal of block 2p+1
-    } else {
-        qb = nqb - 1 - (int)blockIdx.y;
-        ntiles = qb + 1;
-    }
-    const int hs = bhx % H, b = bhx / H;
-    const int g = hs / CH, hl = hs % CH;
-    const int bh = b * H + hs;
-    const int i0 = qb * kBM;
+    const int ncl = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+    const int cl = PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+    const int BH = nbh;
     const int NA = q_atoms(c_q);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int consumers = PAIR ? 8 : 4;   // softmax warps that publish P~
+    const int kf_slots = (c_q + 1) / 2;
+    auto item = [&](int k, WorkItem &it) { return work_item<PAIR>(k, cl, ncl, BH, H, CH, nqb, rank, it); };
 
     if (threadIdx.x == 0) {
         tc::mbar_init(bar_q, 1);
@@ -479,6 +513,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
         tc::mbar_init(p_full, consumers);
         tc::mbar_init(pv_done, 1);
         tc::mbar_init(mma_drain, 1);
+        tc::mbar_init(q_free, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -497,18 +532,13 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             // ---------------- TMA producer
             tc::prefetch_tmap(&mapQ); tc::prefetch_tmap(&mapK); tc::prefetch_tmap(&mapV);
             const uint32_t q_bytes = C::kChunks * NA * 8 * 128;
-            const uint32_t bq = tc::mapa_shared(tc::smem_u32(bar_q), 0);
-            if (leader) tc::mbar_arrive_expect_tx(bar_q, PAIR ? 2 * q_bytes : q_bytes);
-            for (int c = 0; c < C::kChunks; ++c) {
-                if constexpr (PAIR) tc::tma_load_3d_pair(sQ + c * C::kQChunkBytes, &mapQ, bq, 64 * c, qb * NA * 8, bh);
-                else tc::tma_load_3d(sQ + c * C::kQChunkBytes, &mapQ, bar_q, 64 * c, qb * NA * 8, bh);
-            }
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_phase[C::kStages];
             bool issued[C::kStages];
             for (int s = 0; s < C::kStages; ++s) issued[s] = false;
             bool ok = true;
+            int q_loads = 0;
             // Claims the next ring slot and counts `bytes` (this CTA's part) on
             // its full barrier; the leader of a pair expects both CTAs' parts.
             auto claim = [&](uint32_t bytes) -> uint8_t * {
@@ -527,24 +557,37 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 else
                     tc::tma_load_3d(dst, map, &full[stage], x, y, z);
             };
+            // the permuted Q block of an item, once the previous item's last
+            // QK MMAs have finished reading the buffer
+            auto load_q = [&](const WorkItem &it) -> bool {
+                if (q_loads > 0 && !wait_role<PAIR>(q_free, (q_loads - 1) & 1, abort_flag)) return false;
+                if (leader) tc::mbar_arrive_expect_tx(bar_q, PAIR ? 2 * q_bytes : q_bytes);
+                const uint32_t bq = tc::mapa_shared(tc::smem_u32(bar_q), 0);
+                for (int c = 0; c < C::kChunks; ++c) {
+                    if constexpr (PAIR) tc::tma_load_3d_pair(sQ + c * C::kQChunkBytes, &mapQ, bq, 64 * c, it.qb * NA * 8, it.bh);
+                    else tc::tma_load_3d(sQ + c * C::kQChunkBytes, &mapQ, bar_q, 64 * c, it.qb * NA * 8, it.bh);
+                }
+                ++q_loads;
+                return true;
+            };
             // Kf slot m of key tile t: shifts 2m and 2m+1 (when below c_q)
-            auto load_kf = [&](int t, int m) -> bool {
+            auto load_kf = [&](const WorkItem &it, int t, int m) -> bool {
                 const int n = (2 * m + 1 < c_q) ? 2 : 1;
                 uint8_t *dst = claim(n * C::kShiftBytes);
                 if (dst == nullptr) return false;
                 for (int h = 0; h < n; ++h)
                     for (int c = 0; c < C::kChunks; ++c)
                         tile_load(dst + h * C::kShiftBytes + c * (C::kKfRows * 128), &mapK, 64 * c,
-                                  t * kBN + (PAIR ? (int)rank * C::kKfRows : 0), bh * c_q + 2 * m + h);
+                                  t * kBN + (PAIR ? (int)rank * C::kKfRows : 0), it.bh * c_q + 2 * m + h);
                 advance();
                 return true;
             };
             // V slot vs of key tile u: heads vs*kVHeads ...; in a pair with two
             // heads CTA r loads head r whole, with one head it loads column half r
-            auto load_v = [&](int u, int vs) -> bool {
+            auto load_v = [&](const WorkItem &it, int u, int vs) -> bool {
                 uint8_t *dst = claim(C::kVBytes);
                 if (dst == nullptr) return false;
-                const int z0 = b * H + g * CH + vs * C::kVHeads;
+                const int z0 = it.b * H + it.g * CH + vs * C::kVHeads;
                 if constexpr (PAIR) {
                     if (C::kVHeads == 2) {
                         for (int c = 0; c < C::kChunks; ++c)
@@ -558,17 +601,16 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 advance();
                 return true;
             };
-            // L2 prefetch of the tiles kPrefetch key tiles ahead, so that the
-            // loads into the ring find them in L2
-            constexpr int kPrefetch = 2;
-            auto prefetch = [&](int u) {
-                if (u >= ntiles) return;
+            // L2 prefetch of key tile u of an item, so that the ring loads
+            // find it in L2
+            auto prefetch = [&](const WorkItem &it, int u) {
+                if (u >= it.ntiles) return;
                 for (int ip = 0; ip < c_q; ++ip)
                     for (int c = 0; c < C::kChunks; ++c)
                         tc::tma_prefetch_3d(&mapK, 64 * c, u * kBN + (PAIR ? (int)rank * C::kKfRows : 0),
-                                            bh * c_q + ip);
+                                            it.bh * c_q + ip);
                 for (int vs = 0; vs < C::kVSlots; ++vs) {
-                    const int z0 = b * H + g * CH + vs * C::kVHeads;
+                    const int z0 = it.b * H + it.g * CH + vs * C::kVHeads;
                     if (PAIR && C::kVHeads == 2) {
                         for (int c = 0; c < C::kChunks; ++c)
                             tc::tma_prefetch_3d(&mapV, 64 * c, u * kBN, z0 + (int)rank);
@@ -579,18 +621,36 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                     }
                 }
             };
-            const int kf_slots = (c_q + 1) / 2;
-            for (int t = 0; t < ntiles && ok; ++t) {
-                for (int m = 0; m < kf_slots && ok; ++m) ok = load_kf(t, m);
-                // tile 0 is loaded first, then the prefetches start
-                for (int u = (t == 0 ? 1 : t + kPrefetch); u <= t + kPrefetch; ++u) prefetch(u);
-                for (int vs = 0; vs < C::kVSlots && ok && t > 0; ++vs) ok = load_v(t - 1, vs);
+            constexpr int kPrefetch = 2;     // key tiles prefetched ahead
+            WorkItem it, nx, prev;
+            bool have = item(0, it);
+            int prev_t = -1;
+            for (int k = 0; have && ok; ++k) {
+                const bool have_next = item(k + 1, nx);
+                for (int t = 0; t < it.ntiles && ok; ++t) {
+                    for (int m = 0; m < kf_slots && ok; ++m) ok = load_kf(it, t, m);
+                    if (ok && t == 0) ok = load_q(it);
+                    // prefetch: the item's tiles kPrefetch ahead, then the next
+                    // item's Q block and first tiles
+                    for (int u = (t == 0 ? 1 : t + kPrefetch); u <= t + kPrefetch; ++u) prefetch(it, u);
+                    if (have_next && t == it.ntiles - 1) {
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tc::tma_prefetch_3d(&mapQ, 64 * c, nx.qb * NA * 8, nx.bh);
+                        prefetch(nx, 0);
+                        prefetch(nx, 1);
+                    }
+                    for (int vs = 0; vs < C::kVSlots && ok && prev_t >= 0; ++vs) ok = load_v(prev, prev_t, vs);
+                    prev = it;
+                    prev_t = t;
+                }
+                it = nx;
+                have = have_next;
             }
-            for (int vs = 0; vs < C::kVSlots && ok; ++vs) ok = load_v(ntiles - 1, vs);
+            for (int vs = 0; vs < C::kVSlots && ok && prev_t >= 0; ++vs) ok = load_v(prev, prev_t, vs);
             // copies this thread started land before the CTA may exit; in a pair
             // their completion is counted in the leader, so the peer waits a while
             if (leader) {
-                tc::mbar_wait(bar_q, 0, kWaitBudget);
+                if (q_loads > 0) tc::mbar_wait(bar_q, (q_loads - 1) & 1, kWaitBudget);
                 for (int s = 0; s < C::kStages; ++s)
                     if (issued[s]) tc::mbar_wait(&full[s], issued_phase[s], kWaitBudget);
             } else if (!ok) {
@@ -630,14 +690,14 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 tc::named_bar_sync(id, 64);
             };
             int stage = 0;
-            const int kf_slots = (c_q + 1) / 2;
-            gate(kGateQ);
             // The TMA data behind a full barrier needs no tcgen05 fence; P~ (in
             // TMEM over the first half of its S buffer) and the rescaled U,
             // which the gate also waited for before the first V slot, do.
-            // S(t+2) overwrites the buffer only after PV(t), which reads P~(t),
-            // has been issued: the pipe executes in issue order.
-            auto issue_pv = [&](int u) {
+            // S(g+2) overwrites the buffer only after PV(g), which reads P~(g),
+            // has been issued: the pipe executes in issue order.  PV of an
+            // item's first tile overwrites U (the softmax warps read the
+            // previous item's U before they publish that tile's P~).
+            auto issue_pv = [&](int gprev, int tprev) {
                 for (int vs = 0; vs < C::kVSlots; ++vs) {
                     gate(kGateStage0 + stage);
                     if (vs == 0) tc::tc_fence_after();
@@ -645,41 +705,50 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                         const uint64_t bv = dv0 + (uint64_t)((stage * C::kSlotBytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < kBN / 16; ++kk)
-                            mma_t(tm + 256 + vs * C::kVN, tm + (u & 1) * kBN + kk * 8,
-                                  bv + (uint64_t)((kk * 2048) >> 4), idv, (u > 0 || kk > 0) ? 1u : 0u);
+                            mma_t(tm + 256 + vs * C::kVN, tm + (gprev & 1) * kBN + kk * 8,
+                                  bv + (uint64_t)((kk * 2048) >> 4), idv, (tprev > 0 || kk > 0) ? 1u : 0u);
                         commit(&empty[stage]);
                     }
                     if (++stage == C::kStages) stage = 0;
                 }
                 if (issuer) commit(pv_done);
             };
-            for (int t = 0; t < ntiles; ++t) {
-                const int sb = t & 1;
-                for (int m = 0; m < kf_slots; ++m) {
-                    gate(kGateStage0 + stage);
-                    if (issuer) {
-                        const uint64_t bs = dk0 + (uint64_t)((stage * C::kSlotBytes) >> 4);
-                        for (int h = 0; h < 2; ++h) {
-                            const int ip = 2 * m + h;
-                            if (ip >= c_q) break;
-                            const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
-                            const uint64_t bk = bs + (uint64_t)((h * C::kShiftBytes) >> 4);
+            int gt = 0, prev_t = -1;
+            WorkItem it;
+            for (int k = 0; item(k, it); ++k) {
+                gate(kGateQ);                  // this item's Q block has landed
+                for (int t = 0; t < it.ntiles; ++t, ++gt) {
+                    const int sb = gt & 1;
+                    for (int m = 0; m < kf_slots; ++m) {
+                        gate(kGateStage0 + stage);
+                        if (issuer) {
+                            const uint64_t bs = dk0 + (uint64_t)((stage * C::kSlotBytes) >> 4);
+                            for (int h = 0; h < 2; ++h) {
+                                const int ip = 2 * m + h;
+                                if (ip >= c_q) break;
+                                const uint64_t aq = dq0 + (uint64_t)(((c_q - 1 - ip) * 1024) >> 4);
+                                const uint64_t bk = bs + (uint64_t)((h * C::kShiftBytes) >> 4);
 #pragma unroll
-                            for (int c = 0; c < C::kChunks; ++c)
+                                for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
-                                        bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
-                                        (ip | c | kk) ? 1u : 0u);
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        mma(tm + sb * kBN, aq + (uint64_t)((c * C::kQChunkBytes + kk * 32) >> 4),
+                                            bk + (uint64_t)((c * (C::kKfRows * 128) + kk * 32) >> 4), idq,
+                                            (ip | c | kk) ? 1u : 0u);
+                            }
+                            commit(&empty[stage]);
                         }
-                        commit(&empty[stage]);
+                        if (++stage == C::kStages) stage = 0;
                     }
-                    if (++stage == C::kStages) stage = 0;
+                    if (issuer) {
+                        commit(&s_full[sb]);
+                        if (t == it.ntiles - 1) commit(q_free);   // the Q block may be replaced
+                    }
+                    if (gt > 0) issue_pv(gt - 1, prev_t);
+                    prev_t = t;
                 }
-                if (issuer) commit(&s_full[sb]);
-                if (t > 0) issue_pv(t - 1);
             }
-            issue_pv(ntiles - 1);
+            if (gt > 0) issue_pv(gt - 1, prev_t);
             // all MMAs this warp issued complete before TMEM is released
             if (issuer) {
                 if constexpr (PAIR) tc::mma_commit_pair_multicast(mma_drain, 0x1);
@@ -714,186 +783,225 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 tc::named_bar_arrive(kGateStage0 + stage, 64);
                 if (++stage == C::kStages) { stage = 0; phase ^= 1; }
             };
-            {
+            // Q block of item k; after an abort, only once the issuer's commit
+            // after the previous item's last QK shows it consumed the last meeting
+            auto meet_q = [&](int k) {
                 int r = 1;
-                if (lane == 0) r = wait_role<PAIR>(bar_q, 0, abort_flag) ? 1 : 0;
-                ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+                if (lane == 0) {
+                    if (ok) r = wait_role<PAIR>(bar_q, k & 1, abort_flag) ? 1 : 0;
+                    if ((!ok || !r) && k > 0) tc::mbar_wait(q_free, (k - 1) & 1, kWaitBudget);
+                }
+                ok = ok && __shfl_sync(0xffffffffu, r, 0) != 0;
                 __syncwarp();
                 tc::named_bar_arrive(kGateQ, 64);
+            };
+            int gt = 0;
+            WorkItem it;
+            for (int k = 0; item(k, it); ++k) {
+                meet_q(k);
+                for (int t = 0; t < it.ntiles; ++t, ++gt) {
+                    for (int m = 0; m < kf_slots; ++m) meet(false, 0);
+                    for (int vs = 0; vs < C::kVSlots && gt > 0; ++vs) meet(vs == 0, gt - 1);
+                }
             }
-            const int kf_slots = (c_q + 1) / 2;
-            for (int t = 0; t < ntiles; ++t) {
-                for (int m = 0; m < kf_slots; ++m) meet(false, 0);
-                for (int vs = 0; vs < C::kVSlots && t > 0; ++vs) meet(vs == 0, t - 1);
-            }
-            for (int vs = 0; vs < C::kVSlots; ++vs) meet(vs == 0, ntiles - 1);
+            for (int vs = 0; vs < C::kVSlots && gt > 0; ++vs) meet(vs == 0, gt - 1);
         }
     } else {
         // ---------------- softmax and epilogue (warps 2..5): thread = TMEM lane = one query row
         const int q4 = warp & 3;                       // lane quarter this warp may access
         const int r = q4 * 32 + lane;
-        const int i_row = i0 + 16 * (r & 7) + (r >> 3);   // permuted row order of the Q operand
         const uint32_t lane_base = tm + ((uint32_t)(q4 * 32) << 16);
         float *crow = sCorr + r * kCorrStride;
-        {
-            const float4 *src = (const float4 *)(corr + ((size_t)bh * Tp + i_row) * kCorrW);
+        float *scr = sScr + r * kScrStride;   // this thread's scratch row (band tiles, epilogue)
+        bool ok = true;
+        int gt = 0;
+        WorkItem it, nx;
+        // this row's correction entries of an item (read an item ahead, so
+        // that the load overlaps the previous item's epilogue)
+        float4 cnext[kCorrW / 4];
+        auto fetch_corr = [&](const WorkItem &w) {
+            const int ir = w.i0 + 16 * (r & 7) + (r >> 3);
+            const float4 *src = (const float4 *)(corr + ((size_t)w.bh * Tp + ir) * kCorrW);
+#pragma unroll
+            for (int u = 0; u < kCorrW / 4; ++u) cnext[u] = src[u];
+        };
+        bool have = item(0, it);
+        if (have) fetch_corr(it);
+        for (int k = 0; ok && have; ++k) {
+            const int qb = it.qb, i0 = it.i0, b = it.b, g = it.g, hl = it.hl;
 #pragma unroll
             for (int u = 0; u < kCorrW / 4; ++u) {
-                const float4 v = src[u];
-                crow[4 * u] = v.x; crow[4 * u + 1] = v.y; crow[4 * u + 2] = v.z; crow[4 * u + 3] = v.w;
+                crow[4 * u] = cnext[u].x; crow[4 * u + 1] = cnext[u].y;
+                crow[4 * u + 2] = cnext[u].z; crow[4 * u + 3] = cnext[u].w;
             }
-        }
-        float m_run = -INFINITY, l = 0.f;
-        bool ok = true;
-        float *scr = sScr + r * kScrStride;   // this thread's scratch row (band tiles, epilogue)
-        for (int t = 0; t < ntiles; ++t) {
-            const int sb = t & 1;
-            ok = __all_sync(0xffffffffu, wait_role<PAIR>(&s_full[sb], (t >> 1) & 1, abort_flag));
-            if (!ok) break;
-            tc::tc_fence_after();
-            // The first block of a pair runs one tile past its diagonal: every
-            // key there is in the future, so P~ is zero and the row state stays.
-            const bool live = t <= qb;
-            uint32_t pk[kBN / 2];
-            float lp[8];
-            bool need = false;
-            float m_new = m_run, alpha = 1.f;
-#pragma unroll
-            for (int x = 0; x < 8; ++x) lp[x] = 0.f;
-            if (live) {
-            float s[kBN];
-#pragma unroll
-            for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
-            tc::tmem_ld_wait();
-            // Band tiles (this block's diagonal tile and the one before it):
-            // for key j0 + c the diagonal offset is e = i_row - j0 - c; keys
-            // with e < 0 are in the future (-inf), and the Mask_0 correction
-            // corr[i][e] (nonzero for e < D_m < kCorrW = 16) is subtracted.
-            // With the permuted row order i_row - i0 = 16 a + beta (a = lane & 7,
-            // beta = 4 q4 + lane / 8) and c = 16 a' + gamma, the diagonal tile
-            // has e = 16 (a - a') + beta - gamma: e lies in [0, 16) only for
-            // a' = a, gamma <= beta, or a' = a - 1, gamma > beta, and then
-            // corr[e] = corr[(beta - gamma) mod 16].  So 16 table reads per
-            // row serve the whole tile and the rest is register selects.  The
-            // tile before the diagonal has e >= 1, and e < 16 only in the rows
-            // with a = 0, at columns c = 112 + gamma with gamma > beta.
-            if (t >= qb - 1) {
-                const int a = lane & 7, beta = 4 * q4 + (lane >> 3);
-                float w[kCorrW];
-#pragma unroll
-                for (int gm = 0; gm < kCorrW; ++gm) w[gm] = crow[(beta - gm) & (kCorrW - 1)];
-                if (t == qb) {
-#pragma unroll
-                    for (int a2 = 0; a2 < kBN / 16; ++a2) {
-                        const bool same = a2 == a, prev = a2 == a - 1, later = a2 > a;
-#pragma unroll
-                        for (int gm = 0; gm < 16; ++gm) {
-                            const int c = 16 * a2 + gm;
-                            const bool band = (gm <= beta) ? same : prev;
-                            const bool future = later || (same && gm > beta);
-                            const float v = s[c] - (band ? w[gm] : 0.f);
-                            s[c] = future ? -INFINITY : v;
-                        }
-                    }
-                } else if (a == 0) {
-#pragma unroll
-                    for (int gm = 0; gm < 16; ++gm)
-                        if (gm > beta) s[kBN - 16 + gm] -= w[gm];
-                }
-            }
-            // row max as 8 independent partial maxima
-            float mp[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) mp[x] = s[x];
-#pragma unroll
-            for (int c = 8; c < kBN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-            const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-            // the running max moves only when it grows by more than 2^8 in scale
-            need = mt > m_run + 8.f;
-            m_new = need ? mt : m_run;
-            alpha = ex2(m_run - m_new);
-            // P~ = exp2(S - m), packed to bf16 pairs
-#pragma unroll
-            for (int c = 0; c < kBN; c += 2) {
-                const float p0 = ex2(s[c] - m_new), p1 = ex2(s[c + 1] - m_new);
-                lp[(c >> 1) & 7] += p0 + p1;
-                pk[c >> 1] = pack_bf16(p0, p1);
-            }
-            } else {
-#pragma unroll
-                for (int x = 0; x < kBN / 2; ++x) pk[x] = 0u;
-            }
-            // Every warp waits for PV(t-1) to complete before it publishes
-            // P~(t).  p_full counts arrivals from all softmax warps (of both
-            // CTAs in a pair); without this wait a warp that ran a tile ahead
-            // could complete phase t for a warp still working on tile t.  The
-            // wait also orders the (rare) rescale of U after PV(t-1) added
-            // into it.
-            if (t > 0) {
-                ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (t - 1) & 1, abort_flag));
+            const bool have_next = item(k + 1, nx);
+            float m_run = -INFINITY, l = 0.f;
+            for (int t = 0; t < it.ntiles; ++t, ++gt) {
+                const int sb = gt & 1;
+                ok = __all_sync(0xffffffffu, wait_role<PAIR>(&s_full[sb], (gt >> 1) & 1, abort_flag));
                 if (!ok) break;
                 tc::tc_fence_after();
-            }
-            if (t > 0 && __any_sync(0xffffffffu, need)) {
-                const float f = need ? alpha : 1.f;
+                // The first block of a pair runs one tile past its diagonal: every
+                // key there is in the future, so P~ is zero and the row state stays.
+                const bool live = t <= qb;
+                uint32_t pk[kBN / 2];
+                float lp[8];
+                bool need = false;
+                float m_new = m_run, alpha = 1.f;
 #pragma unroll
-                for (int hh = 0; hh < CH; ++hh)
+                for (int x = 0; x < 8; ++x) lp[x] = 0.f;
+                if (live) {
+                float s[kBN];
 #pragma unroll
-                    for (int j = 0; j < D / 32; ++j) {
-                        uint32_t u[32];
-                        const uint32_t a = lane_base + 256 + hh * D + 32 * j;
-                        tc::tmem_ld32(a, u);
-                        tc::tmem_ld_wait();
+                for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
+                tc::tmem_ld_wait();
+                // Band tiles (this block's diagonal tile and the one before it):
+                // for key j0 + c the diagonal offset is e = i_row - j0 - c; keys
+                // with e < 0 are in the future (-inf), and the Mask_0 correction
+                // corr[i][e] (nonzero for e < D_m < kCorrW = 16) is subtracted.
+                // With the permuted row order i_row - i0 = 16 a + beta (a = lane & 7,
+                // beta = 4 q4 + lane / 8) and c = 16 a' + gamma, the diagonal tile
+                // has e = 16 (a - a') + beta - gamma: e lies in [0, 16) only for
+                // a' = a, gamma <= beta, or a' = a - 1, gamma > beta, and then
+                // corr[e] = corr[(beta - gamma) mod 16].  So 16 table reads per
+                // row serve the whole tile and the rest is register selects.  The
+                // tile before the diagonal has e >= 1, and e < 16 only in the rows
+                // with a = 0, at columns c = 112 + gamma with gamma > beta.
+                if (t >= qb - 1) {
+                    const int a = lane & 7, beta = 4 * q4 + (lane >> 3);
+                    float w[kCorrW];
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
-                        tc::tmem_st32(a, u);
+                    for (int gm = 0; gm < kCorrW; ++gm) w[gm] = crow[(beta - gm) & (kCorrW - 1)];
+                    if (t == qb) {
+#pragma unroll
+                        for (int a2 = 0; a2 < kBN / 16; ++a2) {
+                            const bool same = a2 == a, prev = a2 == a - 1, later = a2 > a;
+#pragma unroll
+                            for (int gm = 0; gm < 16; ++gm) {
+                                const int c = 16 * a2 + gm;
+                                const bool band = (gm <= beta) ? same : prev;
+                                const bool future = later || (same && gm > beta);
+                                const float v = s[c] - (band ? w[gm] : 0.f);
+                                s[c] = future ? -INFINITY : v;
+                            }
+                        }
+                    } else if (a == 0) {
+#pragma unroll
+                        for (int gm = 0; gm < 16; ++gm)
+                            if (gm > beta) s[kBN - 16 + gm] -= w[gm];
                     }
+                }
+                // row max as 8 independent partial maxima
+                float mp[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) mp[x] = s[x];
+#pragma unroll
+                for (int c = 8; c < kBN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+                const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+                // the running max moves only when it grows by more than 2^8 in scale
+                need = mt > m_run + 8.f;
+                m_new = need ? mt : m_run;
+                alpha = ex2(m_run - m_new);
+                // P~ = exp2(S - m), packed to bf16 pairs
+#pragma unroll
+                for (int c = 0; c < kBN; c += 2) {
+                    const float p0 = ex2(s[c] - m_new), p1 = ex2(s[c + 1] - m_new);
+                    lp[(c >> 1) & 7] += p0 + p1;
+                    pk[c >> 1] = pack_bf16(p0, p1);
+                }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < kBN / 2; ++x) pk[x] = 0u;
+                }
+                // Every warp waits for PV(t-1) to complete before it publishes
+                // P~(t).  p_full counts arrivals from all softmax warps (of both
+                // CTAs in a pair); without this wait a warp that ran a tile ahead
+                // could complete phase t for a warp still working on tile t.  The
+                // wait also orders the (rare) rescale of U after PV(t-1) added
+                // into it.
+                if (gt > 0) {
+                    ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (gt - 1) & 1, abort_flag));
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                }
+                if (t > 0 && __any_sync(0xffffffffu, need)) {
+                    const float f = need ? alpha : 1.f;
+#pragma unroll
+                    for (int hh = 0; hh < CH; ++hh)
+#pragma unroll
+                        for (int j = 0; j < D / 32; ++j) {
+                            uint32_t u[32];
+                            const uint32_t a = lane_base + 256 + hh * D + 32 * j;
+                            tc::tmem_ld32(a, u);
+                            tc::tmem_ld_wait();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) u[x] = __float_as_uint(__uint_as_float(u[x]) * f);
+                            tc::tmem_st32(a, u);
+                        }
+                }
+                l = l * alpha + (((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7])));
+                m_run = m_new;
+                // P~(t) goes to TMEM over the first kBN/2 columns of its S buffer,
+                // where PV(t) reads it as the A operand
+                tc::tmem_st32(lane_base + sb * kBN, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+                tc::tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_leader<PAIR>(p_full);
             }
-            l = l * alpha + (((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7])));
-            m_run = m_new;
-            // P~(t) goes to TMEM over the first kBN/2 columns of its S buffer,
-            // where PV(t) reads it as the A operand
-            tc::tmem_st32(lane_base + sb * kBN, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-            tc::tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
-            tc::tmem_st_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) arrive_leader<PAIR>(p_full);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (ntiles - 1) & 1, abort_flag));
-        if (ok) {
-            // (w_head / l) U, 32 columns at a time: each thread puts its row's
-            // 32 values into its scratch row, then every 16-B store of the
-            // warp covers, with 8 lanes, the 128-B segment of one of 4 rows
-            tc::tc_fence_after();
-            const float inv_l = 1.f / l;
-            const size_t row_stride = (size_t)H * CH * D;
+            if (!ok) break;
+            if (have_next) fetch_corr(nx);
+            float coef[CH];
 #pragma unroll
-            for (int hh = 0; hh < CH; ++hh) {
-                const float coef = w_head[((size_t)g * CH + hh) * CH + hl] * inv_l;
-                float *dst = part + (size_t)b * T * row_stride + (size_t)(g * CH + hh) * (CH * D) + hl * D;
+            for (int hh = 0; hh < CH; ++hh) coef[hh] = w_head[((size_t)g * CH + hh) * CH + hl];
+            // the item's last PV has completed: write its partial outputs
+            ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (gt - 1) & 1, abort_flag));
+            if (ok) {
+                // (w_head / l) U in fp16, one head's d columns loaded from TMEM at
+                // once, written 64 columns (128 B) at a time: each thread puts its
+                // row's 64 values into its scratch row, then every 16-B store of
+                // the warp covers, with 8 lanes, the 128-B segment of one of 4 rows
+                tc::tc_fence_after();
+                const float inv_l = 1.f / l;
+                const size_t row_stride = (size_t)H * CH * D;
+#pragma unroll 1
+                for (int hh = 0; hh < CH; ++hh) {
+                    const float cf = coef[hh] * inv_l;
+                    __half *dst = part + (size_t)b * T * row_stride + (size_t)(g * CH + hh) * (CH * D) + hl * D;
+                    uint32_t u[D];
 #pragma unroll
-                for (int j = 0; j < D / 32; ++j) {
-                    uint32_t u[32];
-                    tc::tmem_ld32(lane_base + 256 + hh * D + 32 * j, u);
+                    for (int j = 0; j < D / 32; ++j)
+                        tc::tmem_ld32(lane_base + 256 + hh * D + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * j));
                     tc::tmem_ld_wait();
-                    __syncwarp();
+                    uint32_t *srow = reinterpret_cast<uint32_t *>(scr);
 #pragma unroll
-                    for (int x = 0; x < 32; x += 4)
-                        *(float4 *)(scr + x) = make_float4(
-                            __uint_as_float(u[x]) * coef, __uint_as_float(u[x + 1]) * coef,
-                            __uint_as_float(u[x + 2]) * coef, __uint_as_float(u[x + 3]) * coef);
-                    __syncwarp();
+                    for (int j = 0; j < D / 64; ++j) {
+                        __syncwarp();
 #pragma unroll
-                    for (int rho = 0; rho < 8; ++rho) {
-                        const int rr = q4 * 32 + 4 * rho + (lane >> 3);
-                        const int ir = i0 + 16 * (rr & 7) + (rr >> 3);
-                        const float4 v = *(const float4 *)(sScr + rr * kScrStride + 4 * (lane & 7));
-                        if (ir < T) *(float4 *)(dst + (size_t)ir * row_stride + 32 * j + 4 * (lane & 7)) = v;
+                        for (int x = 0; x < 32; x += 4) {
+                            uint4 w4;
+                            const int c = 64 * j + 2 * x;
+                            w4.x = pack_h2(__uint_as_float(u[c]) * cf, __uint_as_float(u[c + 1]) * cf);
+                            w4.y = pack_h2(__uint_as_float(u[c + 2]) * cf, __uint_as_float(u[c + 3]) * cf);
+                            w4.z = pack_h2(__uint_as_float(u[c + 4]) * cf, __uint_as_float(u[c + 5]) * cf);
+                            w4.w = pack_h2(__uint_as_float(u[c + 6]) * cf, __uint_as_float(u[c + 7]) * cf);
+                            *(uint4 *)(srow + x) = w4;
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int rho = 0; rho < 8; ++rho) {
+                            const int rr = q4 * 32 + 4 * rho + (lane >> 3);
+                            const int ir = i0 + 16 * (rr & 7) + (rr >> 3);
+                            const uint4 v = *(const uint4 *)(sScr + rr * kScrStride + 4 * (lane & 7));
+                            if (ir < T) *(uint4 *)(dst + (size_t)ir * row_stride + 64 * j + 8 * (lane & 7)) = v;
+                        }
                     }
                 }
             }
+            it = nx;
+            have = have_next;
         }
     }
     tc::tc_fence_before();
@@ -929,40 +1037,48 @@ __device__ __forceinline__ float warp_sum(float x)
 }
 
 // One CTA per (query row i, batch b); warp w handles heads w, w+4, ...:
-// O^h = sum_{h'} part[b][i][h][h'], then GroupNorm over the head's d values
-// (mean and biased variance by warp shuffles), affine, depth scale.
+// O^h = sum_{h'} part[b][i][h][h'] (fp16 partials, summed in fp32), then
+// GroupNorm over the head's d values (mean and biased variance by warp
+// shuffles), affine, depth scale.
 template <int D, int CH>
 __global__ void __launch_bounds__(128)
-k_mix_groupnorm(const float *__restrict__ part, const float *__restrict__ gn_weight,
+k_mix_groupnorm(const __half *__restrict__ part, const float *__restrict__ gn_weight,
                 const float *__restrict__ gn_bias, float depth_scale, float eps,
                 __nv_bfloat16 *__restrict__ out, int T, int H)
 {
     const int i = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    constexpr int PER = D / 32;
+    constexpr int PER = D / 64;                // column pairs per lane
     for (int h = warp; h < H; h += 4) {
-        const float *src = part + (((size_t)b * T + i) * H + h) * (size_t)(CH * D);
-        float o[PER];
+        const __half2 *src = (const __half2 *)(part + (((size_t)b * T + i) * H + h) * (size_t)(CH * D));
+        float2 o[PER];
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
-            float acc = 0.f;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int hs = 0; hs < CH; ++hs) acc += src[hs * D + lane + 32 * u];
+            for (int hs = 0; hs < CH; ++hs) {
+                const float2 f = __half22float2(src[hs * (D / 2) + lane + 32 * u]);
+                acc.x += f.x;
+                acc.y += f.y;
+            }
             o[u] = acc;
         }
         float sum = 0.f;
 #pragma unroll
-        for (int u = 0; u < PER; ++u) sum += o[u];
+        for (int u = 0; u < PER; ++u) sum += o[u].x + o[u].y;
         const float mean = warp_sum(sum) / D;
         float sq = 0.f;
 #pragma unroll
-        for (int u = 0; u < PER; ++u) sq += (o[u] - mean) * (o[u] - mean);
+        for (int u = 0; u < PER; ++u)
+            sq += (o[u].x - mean) * (o[u].x - mean) + (o[u].y - mean) * (o[u].y - mean);
         const float inv = 1.f / sqrtf(warp_sum(sq) / D + eps);
-        __nv_bfloat16 *dst = out + ((size_t)b * T + i) * ((size_t)H * D) + (size_t)h * D;
+        __nv_bfloat162 *dst = (__nv_bfloat162 *)(out + ((size_t)b * T + i) * ((size_t)H * D) + (size_t)h * D);
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
-            const int e = lane + 32 * u, ch = h * D + e;
-            dst[e] = __float2bfloat16_rn(depth_scale * ((o[u] - mean) * inv * gn_weight[ch] + gn_bias[ch]));
+            const int e = 2 * (lane + 32 * u), ch = h * D + e;
+            dst[lane + 32 * u] = __floats2bfloat162_rn(
+                depth_scale * ((o[u].x - mean) * inv * gn_weight[ch] + gn_bias[ch]),
+                depth_scale * ((o[u].y - mean) * inv * gn_weight[ch + 1] + gn_bias[ch + 1]));
         }
     }
 }
@@ -987,7 +1103,7 @@ FusedLayout fused_layout(const mta_shape &s)
     L.off_kf = off;   off += align256(BH * s.c_q * L.Tp * s.d * 2);
     L.off_qp = off;   off += align256(BH * L.nqb * L.NA * 8 * s.d * 2);
     L.off_corr = off; off += align256(BH * L.Tp * kCorrW * 4);
-    L.off_part = off; off += align256((size_t)s.B * s.T * s.H * s.c_h * s.d * 4);
+    L.off_part = off; off += align256((size_t)s.B * s.T * s.H * s.c_h * s.d * 2);
     L.total = off;
     return L;
 }
@@ -1024,6 +1140,41 @@ mta_status side_stream(SideStream *out)
     return MTA_OK;
 }
 
+// Clusters of the main kernel that fit on the device at once (one CTA per SM
+// at this shared-memory size), cached per kernel instantiation and device.
+template <int D, int CH>
+mta_status max_resident_clusters(const cudaLaunchConfig_t &cfg, int *out)
+{
+    constexpr bool PAIR = (D == 128);
+    constexpr int cluster = PAIR ? 2 : 1;
+    auto kernel = k_mta_fused<D, CH, PAIR>;
+    constexpr int kMaxDevices = 64;
+    static int cached[kMaxDevices] = {};
+    static std::mutex lock;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTA_ERR_CUDA;
+    std::lock_guard<std::mutex> guard(lock);
+    if (!cached[dev]) {
+        int n = 0;
+        if (cluster > 1) {
+            cudaLaunchConfig_t c = cfg;
+            c.gridDim = dim3((unsigned)cluster, 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&n, (void *)kernel, &c) != cudaSuccess) return MTA_ERR_CUDA;
+        } else {
+            int per_sm = 0, sms = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (int)cfg.blockDim.x,
+                                                              cfg.dynamicSmemBytes) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return MTA_ERR_CUDA;
+            n = per_sm * sms;
+        }
+        if (n < 1) return MTA_ERR_CUDA;
+        cached[dev] = n;
+    }
+    *out = cached[dev];
+    return MTA_OK;
+}
+
 template <int D, int CH>
 mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr)
@@ -1035,7 +1186,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     __half *kf = (__half *)(w + L.off_kf);
     __half *qp = (__half *)(w + L.off_qp);
     float *corr = (float *)(w + L.off_corr);
-    float *part = (float *)(w + L.off_part);
+    __half *part = (__half *)(w + L.off_part);
     const uint64_t BH = (uint64_t)s.B * s.H;
     CUtensorMap mQ, mK, mV;
     {
@@ -1089,8 +1240,9 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     }
     tr.before(2, st);
     {
+        // persistent: as many clusters as can be resident at once, each
+        // walking its share of the work items
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = PAIR ? dim3(2 * s.B * s.H, L.nqb / 2, 1) : dim3(s.B * s.H, L.nqb, 1);
         cfg.blockDim = dim3(224, 1, 1);
         cfg.dynamicSmemBytes = C::kSmemBytes;
         cfg.stream = st;
@@ -1101,8 +1253,14 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
+        const int n_items = (int)BH * (PAIR ? L.nqb / 2 : L.nqb);
+        int resident = 0;
+        if (max_resident_clusters<D, CH>(cfg, &resident) != MTA_OK)
+            return MTA_ERR_CUDA;
+        const int ncl = resident < n_items ? resident : n_items;
+        cfg.gridDim = dim3((unsigned)(ncl * (PAIR ? 2 : 1)), 1, 1);
         if (cudaLaunchKernelEx(&cfg, main_kernel, mQ, mK, mV, (const float *)corr, a.w_head, part,
-                               s.T, L.Tp, s.H, s.c_q, L.nqb) != cudaSuccess)
+                               s.T, L.Tp, s.H, s.c_q, L.nqb, (int)BH) != cudaSuccess)
             return MTA_ERR_CUDA;
     }
     tr.after(2, st);
