@@ -181,8 +181,8 @@ def kernel_units(name, w):
         # read q and k, write the permuted q (fp16) and the 16-entry correction rows
         "k_fold_aux": ("hbm", w.B * w.H * w.T * (w.d * 2 * 3 + 64), "B"),
         "k_mta_fused": ("tensor", w.algorithmic_flops(), "FLOP"),
-        # read the fp32 partial outputs (c_h per output head), write out
-        "k_mix_groupnorm": ("hbm", w.B * w.T * w.H * w.d * (4 * w.c_h + io_bytes), "B"),
+        # read the fp16 partial outputs (c_h per output head), write out
+        "k_mix_groupnorm": ("hbm", w.B * w.T * w.H * w.d * (2 * w.c_h + io_bytes), "B"),
     }
     return table.get(name, ("unknown", 0, "FLOP"))
 
