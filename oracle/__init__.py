@@ -35,8 +35,12 @@ def _configure(lib):
                                     ctypes.c_int, ip, ctypes.c_int, dp, ctypes.c_int]
     lib.mta_oracle_stages.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_double,
                                       ctypes.c_int, dp, dp, dp, dp, dp]
+    lib.mta_oracle_forward_gated.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+    lib.mta_oracle_rows_gated.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ip,
+                                          ctypes.c_int, dp, ctypes.c_int]
     lib.mta_oracle_max_threads.argtypes = []
     for f in (lib.mta_oracle_forward, lib.mta_oracle_rows, lib.mta_oracle_stages,
+              lib.mta_oracle_forward_gated, lib.mta_oracle_rows_gated,
               lib.mta_oracle_max_threads):
         f.restype = ctypes.c_int
     return lib
@@ -93,33 +97,50 @@ def max_threads() -> int:
 
 
 def forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gn_eps=1e-5,
-            nthreads=0):
+            nthreads=0, gate=None):
     """out[B, T, H*d] for q, k, v [B, H, T, d], w_kq [H, c_q, c_k],
-    w_head [H/c_h, c_h, c_h], gn_weight/gn_bias [H*d]."""
+    w_head [H/c_h, c_h, c_h], gn_weight/gn_bias [H*d].  With gate [H] given,
+    head h's GroupNorm output is scaled by sigmoid(gate[h]) instead of
+    depth_scale (which is then ignored)."""
     q, k, v, w_kq, w_head, gw, gb = map(_f64, (q, k, v, w_kq, w_head, gn_weight, gn_bias))
     B, H, T, d, c_q, c_k, c_h = _unpack(q, w_kq, w_head)
     out = np.empty((B, T, H * d), dtype=np.float64)
     s = _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
-    rc = _load().mta_oracle_forward(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
-                                    _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale),
-                                    _ptr(out), int(nthreads))
+    if gate is not None:
+        g = _f64(gate)
+        assert g.shape == (H,)
+        rc = _load().mta_oracle_forward_gated(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(w_kq), _ptr(w_head), _ptr(gw), _ptr(gb),
+                                              _ptr(g), _ptr(out), int(nthreads))
+    else:
+        rc = _load().mta_oracle_forward(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                        _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale),
+                                        _ptr(out), int(nthreads))
     if rc != 0:
         raise RuntimeError("mta_oracle_forward failed (%d)" % rc)
     return out
 
 
 def rows(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, b, row_idx,
-         gn_eps=1e-5, nthreads=0):
-    """out[b, row_idx, :] computed one row at a time: [len(row_idx), H*d]."""
+         gn_eps=1e-5, nthreads=0, gate=None):
+    """out[b, row_idx, :] computed one row at a time: [len(row_idx), H*d]
+    (gate as in forward)."""
     q, k, v, w_kq, w_head, gw, gb = map(_f64, (q, k, v, w_kq, w_head, gn_weight, gn_bias))
     B, H, T, d, c_q, c_k, c_h = _unpack(q, w_kq, w_head)
     idx = np.ascontiguousarray(np.asarray(row_idx, dtype=np.int32))
     out = np.empty((idx.size, H * d), dtype=np.float64)
     s = _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
-    rc = _load().mta_oracle_rows(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
-                                 _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale), int(b),
-                                 idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), int(idx.size),
-                                 _ptr(out), int(nthreads))
+    ip = idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    if gate is not None:
+        g = _f64(gate)
+        assert g.shape == (H,)
+        rc = _load().mta_oracle_rows_gated(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                           _ptr(w_head), _ptr(gw), _ptr(gb), _ptr(g), int(b), ip,
+                                           int(idx.size), _ptr(out), int(nthreads))
+    else:
+        rc = _load().mta_oracle_rows(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                     _ptr(w_head), _ptr(gw), _ptr(gb), float(depth_scale), int(b),
+                                     ip, int(idx.size), _ptr(out), int(nthreads))
     if rc != 0:
         raise RuntimeError("mta_oracle_rows failed (%d)" % rc)
     return out

@@ -26,13 +26,18 @@
  *          head's d-vector is normalised on its own);
  *          "Article Overview: Multi-Token Attention", section 2, "Group
  *          Normalization with Depth Scaling": the scale is a depth scaling.
+ *   [GATE] "Multi-Token Attention -- Paper Graph", "Group Normalization with
+ *          Sigmoid Gating": the pages' default scale, one learned scalar g_h
+ *          per head, output = GroupNorm(concat) * sigmoid(g_h) on head h.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - taps that fall outside [0,T) x [0,T) read zero (zero padding);
  *   - w_head is stored [group][out head][in head];
  *   - GroupNorm uses the biased variance and eps inside the square root,
  *     with a per-channel affine (gamma, beta) over the H*d concatenation;
- *   - depth scaling is a caller-supplied scalar multiplying the GN output.
+ *   - depth scaling is a caller-supplied scalar multiplying the GN output;
+ *   - the sigmoid gate multiplies the GN output (after its affine) in place
+ *     of the depth scale.
  *
  * Layouts: q, k, v are [B][H][T][d]; w_kq is [H][c_q][c_k] with the tap
  * (i', j') at [h][i'][j' + floor(c_k/2)]; w_head is [H/c_h][c_h][c_h];
@@ -53,6 +58,7 @@ typedef struct {
 typedef struct {
     const double *q, *k, *v, *w_kq, *w_head, *gn_weight, *gn_bias;
     double depth_scale;
+    const double *gate;   /* [H] gate logits g_h, or NULL for the depth scale */
 } mta_oracle_args;
 
 static int shape_ok(const mta_oracle_shape *s)
@@ -202,10 +208,12 @@ static void group_row(const mta_oracle_shape *s, const mta_oracle_args *a,
         for (int e = 0; e < d; ++e) var += (u->O[e] - mean) * (u->O[e] - mean);
         var /= d;
         double inv = 1.0 / sqrt(var + s->gn_eps);
+        /* [GATE] sigmoid(g_h), or the depth scale */
+        double scale = a->gate ? 1.0 / (1.0 + exp(-a->gate[h])) : a->depth_scale;
         for (int e = 0; e < d; ++e) {
             size_t chn = (size_t)h * d + e;
             double y = (u->O[e] - mean) * inv * a->gn_weight[chn] + a->gn_bias[chn];
-            out_row[chn] = a->depth_scale * y;   /* depth scaling */
+            out_row[chn] = scale * y;
         }
     }
 }
@@ -229,14 +237,13 @@ static void fresh_rows(const mta_oracle_shape *s, const mta_oracle_args *a, int 
 /* Full forward: out[B][T][H*d].  Units (b, g) are independent and spread over
  * threads; inside a unit the query rows run in order, keeping the last c_q
  * masked logit rows of each head in a ring.  Returns 0 on success. */
-int mta_oracle_forward(const mta_oracle_shape *s, const double *q, const double *k,
-                       const double *v, const double *w_kq, const double *w_head,
-                       const double *gn_weight, const double *gn_bias,
-                       double depth_scale, double *out, int nthreads)
+static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, double *out,
+                        int nthreads)
 {
-    if (!shape_ok(s) || !q || !k || !v || !w_kq || !w_head || !gn_weight || !gn_bias || !out)
+    if (!shape_ok(s) || !pa->q || !pa->k || !pa->v || !pa->w_kq || !pa->w_head ||
+        !pa->gn_weight || !pa->gn_bias || !out)
         return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale};
+    const mta_oracle_args a = *pa;
     const int G = s->H / s->c_h;
     const int units = s->B * G;
     const size_t HD = (size_t)s->H * s->d;
@@ -276,18 +283,16 @@ int mta_oracle_forward(const mta_oracle_shape *s, const double *q, const double 
 /* Output rows of one batch entry, each computed from scratch: for every
  * requested query row rows_idx[n], out_rows[n][H*d] receives out[b][i][*].
  * Used to check large problems at sampled positions. */
-int mta_oracle_rows(const mta_oracle_shape *s, const double *q, const double *k,
-                    const double *v, const double *w_kq, const double *w_head,
-                    const double *gn_weight, const double *gn_bias,
-                    double depth_scale, int b, const int *rows_idx, int nrows,
-                    double *out_rows, int nthreads)
+static int rows_args(const mta_oracle_shape *s, const mta_oracle_args *pa, int b,
+                     const int *rows_idx, int nrows, double *out_rows, int nthreads)
 {
-    if (!shape_ok(s) || !q || !k || !v || !w_kq || !w_head || !gn_weight || !gn_bias ||
-        !out_rows || !rows_idx || b < 0 || b >= s->B || nrows < 0)
+    if (!shape_ok(s) || !pa->q || !pa->k || !pa->v || !pa->w_kq || !pa->w_head ||
+        !pa->gn_weight || !pa->gn_bias || !out_rows || !rows_idx || b < 0 || b >= s->B ||
+        nrows < 0)
         return -1;
     for (int n = 0; n < nrows; ++n)
         if (rows_idx[n] < 0 || rows_idx[n] >= s->T) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale};
+    const mta_oracle_args a = *pa;
     const int G = s->H / s->c_h;
     const size_t HD = (size_t)s->H * s->d;
     const int tasks = nrows * G;
@@ -313,6 +318,48 @@ int mta_oracle_rows(const mta_oracle_shape *s, const double *q, const double *k,
     return failed ? -2 : 0;
 }
 
+int mta_oracle_forward(const mta_oracle_shape *s, const double *q, const double *k,
+                       const double *v, const double *w_kq, const double *w_head,
+                       const double *gn_weight, const double *gn_bias,
+                       double depth_scale, double *out, int nthreads)
+{
+    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL};
+    return forward_args(s, &a, out, nthreads);
+}
+
+/* The same forward with the [GATE] scale: out head h is multiplied by
+ * sigmoid(gate[h]) instead of a depth scale. */
+int mta_oracle_forward_gated(const mta_oracle_shape *s, const double *q, const double *k,
+                             const double *v, const double *w_kq, const double *w_head,
+                             const double *gn_weight, const double *gn_bias,
+                             const double *gate, double *out, int nthreads)
+{
+    if (!gate) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.0, gate};
+    return forward_args(s, &a, out, nthreads);
+}
+
+int mta_oracle_rows(const mta_oracle_shape *s, const double *q, const double *k,
+                    const double *v, const double *w_kq, const double *w_head,
+                    const double *gn_weight, const double *gn_bias,
+                    double depth_scale, int b, const int *rows_idx, int nrows,
+                    double *out_rows, int nthreads)
+{
+    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL};
+    return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
+}
+
+int mta_oracle_rows_gated(const mta_oracle_shape *s, const double *q, const double *k,
+                          const double *v, const double *w_kq, const double *w_head,
+                          const double *gn_weight, const double *gn_bias,
+                          const double *gate, int b, const int *rows_idx, int nrows,
+                          double *out_rows, int nthreads)
+{
+    if (!gate) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.0, gate};
+    return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
+}
+
 /* Intermediates of one batch entry for small T; any output may be NULL:
  *   C   [H][T][T]  conv logits after both masks of [KQ5] (-inf above the diagonal)
  *   P   [H][T][T]  pre-mix softmax probabilities
@@ -328,7 +375,7 @@ int mta_oracle_stages(const mta_oracle_shape *s, const double *q, const double *
     if (!shape_ok(s) || !q || !k || !v || !w_kq || !w_head || !gn_weight || !gn_bias ||
         b < 0 || b >= s->B)
         return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale};
+    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL};
     const int T = s->T, d = s->d, c_h = s->c_h, c_q = s->c_q, H = s->H;
     const int G = H / c_h;
     const size_t HD = (size_t)H * d;

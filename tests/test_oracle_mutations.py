@@ -31,7 +31,10 @@ MUTATIONS = [
      "const double *vj = row_of(a->v, s, b, g * c_h + (c_h - 1 - ho), j);"),
     ("even-c_k window mirrored", "const int jlo = -(c_k / 2);",
      "const int jlo = -((c_k - 1) / 2);"),
-    ("depth scale dropped", "out_row[chn] = a->depth_scale * y;", "out_row[chn] = y;"),
+    ("depth scale dropped", ": a->depth_scale;", ": 1.0;"),
+    ("gate sign flipped", "exp(-a->gate[h])", "exp(a->gate[h])"),
+    ("gate applied before the affine bias", "out_row[chn] = scale * y;",
+     "out_row[chn] = scale * (y - a->gn_bias[chn]) + a->gn_bias[chn];"),
 ]
 
 PIN_CHECKS = [
@@ -44,6 +47,7 @@ PIN_CHECKS = [
     pins.test_causality_future_tokens_do_not_leak,
     pins.test_row_sums_pre_and_post_mix,
     pins.test_groupnorm_statistics_and_depth_scale,
+    pins.test_sigmoid_gate_scales_each_head_after_the_affine,
 ]
 
 

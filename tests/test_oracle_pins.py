@@ -246,6 +246,30 @@ def test_groupnorm_statistics_and_depth_scale():
     np.testing.assert_allclose(y.var(-1), s2 / (s2 + eps), rtol=1e-11, atol=0)
 
 
+def test_sigmoid_gate_scales_each_head_after_the_affine():
+    # "Group Normalization with Sigmoid Gating": output = GroupNorm(concat)
+    # * sigmoid(g_h) on head h, the gate taking the place of the depth scale.
+    # Against the depth-scaled output with scale 1 (pinned above), head h must
+    # come out multiplied by 1 / (1 + e^-g_h), computed here with numpy; a
+    # nonzero bias makes a gate applied before the affine visible.
+    rng = np.random.default_rng(10)
+    B, H, T, d, c_q, c_k, c_h = 2, 4, 14, 8, 3, 5, 2
+    q, k, v, th, w, gw, gb = rand_inputs(rng, B, H, T, d, c_q, c_k, c_h)
+    gb = rng.standard_normal(H * d)
+    g = np.array([-2.5, -0.3, 0.7, 3.0])
+    plain = oracle.forward(q, k, v, th, w, gw, gb, 1.0).reshape(B, T, H, d)
+    gated = oracle.forward(q, k, v, th, w, gw, gb, 0.0, gate=g).reshape(B, T, H, d)
+    sig = 1.0 / (1.0 + np.exp(-g))
+    np.testing.assert_allclose(gated, plain * sig[None, None, :, None], rtol=1e-13, atol=1e-14)
+    # the sampled-row entry point agrees, and saturated gates turn heads off / fully on
+    r = oracle.rows(q, k, v, th, w, gw, gb, 0.0, 1, [0, 5, 13], gate=g)
+    np.testing.assert_array_equal(r, gated[1, [0, 5, 13]].reshape(3, H * d))
+    off = oracle.forward(q, k, v, th, w, gw, gb, 0.0, gate=np.array([-800.0, 800.0, 0.0, 0.0]))
+    off = off.reshape(B, T, H, d)
+    assert np.all(off[:, :, 0] == 0.0)
+    np.testing.assert_array_equal(off[:, :, 1], plain[:, :, 1])
+
+
 def test_head_outputs_linear_in_mixing_weights():
     # Eq. (7) is linear in w, and so is the pre-normalisation output; summed
     # over a group it equals sum_h' P^h' (sum_h w[h][h'] V^h) (the rank
