@@ -7,7 +7,8 @@ tests and the benchmark (``convolved_logit_attention_b200.workloads``).
 """
 from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
                        MTA_PATH_MATERIALISED, MtaError, MtaShape, lib, make_shape,
-                       mta_debug_attention, mta_forward, mta_forward_path, mta_forward_traced,
+                       mta_debug_attention, mta_forward, mta_forward_gated, mta_forward_path,
+                       mta_forward_traced,
                        mta_forward_unfused, mta_kernel_count, mta_kernel_name,
                        mta_selftest_wait_timeout,
                        mta_status_string, mta_sync_status, mta_unfused_workspace_size,
@@ -15,7 +16,8 @@ from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
 
 __all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC",
            "MTA_PATH_MATERIALISED", "MtaError", "MtaShape", "lib", "make_shape",
-           "mta_debug_attention", "mta_forward", "mta_forward_path", "mta_forward_traced",
+           "mta_debug_attention", "mta_forward", "mta_forward_gated", "mta_forward_path",
+           "mta_forward_traced",
            "mta_forward_unfused", "mta_kernel_count", "mta_kernel_name",
            "mta_selftest_wait_timeout",
            "mta_status_string", "mta_sync_status", "mta_unfused_workspace_size", "mta_version",

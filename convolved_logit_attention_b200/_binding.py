@@ -25,7 +25,8 @@ STATUS = {0: "MTA_OK", -1: "MTA_ERR_INVALID_ARG", -2: "MTA_ERR_UNSUPPORTED",
 EXPORTS = ("mta_version", "mta_status_string", "mta_forward_path", "mta_workspace_size",
            "mta_unfused_workspace_size", "mta_forward", "mta_forward_unfused",
            "mta_debug_attention", "mta_kernel_count", "mta_kernel_name", "mta_forward_traced",
-           "mta_selftest_wait_timeout", "mta_forward_noalloc", "mta_sync_status")
+           "mta_selftest_wait_timeout", "mta_forward_noalloc", "mta_sync_status",
+           "mta_forward_gated")
 
 
 class MtaShape(ctypes.Structure):
@@ -81,6 +82,9 @@ def lib():
         L.mta_selftest_wait_timeout.restype = ctypes.c_int
         L.mta_forward_noalloc.argtypes = [sp, vp, vp, vp, fp, fp, fp, fp, ctypes.c_float, vp, vp]
         L.mta_forward_noalloc.restype = ctypes.c_int
+        L.mta_forward_gated.argtypes = [sp, vp, vp, vp, fp, fp, fp, fp, fp, vp, vp,
+                                        ctypes.c_size_t, vp]
+        L.mta_forward_gated.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -206,6 +210,30 @@ def mta_forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out=None
     """MTA forward on the path mta_forward_path() names; returns out [B, T, H*d]."""
     return _forward("mta_forward", mta_workspace_size, q, k, v, w_kq, w_head, gn_weight,
                     gn_bias, depth_scale, out, workspace, stream, gn_eps)
+
+
+def mta_forward_gated(q, k, v, w_kq, w_head, gn_weight, gn_bias, gate, out=None,
+                      workspace=None, stream=None, gn_eps=1e-5):
+    """MTA forward with the sigmoid-gated output: head h of GroupNorm times
+    sigmoid(gate[h]) (gate: float32 [H] on the device); returns out [B, T, H*d]."""
+    _check_inputs(q, k, v, w_kq, w_head, gn_weight, gn_bias)
+    B, H, T, d = q.shape
+    if gate.dtype != torch.float32 or gate.shape != (H,) or gate.device != q.device \
+            or not gate.is_contiguous():
+        raise ValueError("gate must be a contiguous float32 [H] tensor on q's device")
+    if out is None:
+        out = torch.empty((B, T, H * d), dtype=q.dtype, device=q.device)
+    elif (out.shape != (B, T, H * d) or out.dtype != q.dtype or out.device != q.device
+          or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous [B, T, H*d] tensor like q")
+    shape = shape_of(q, w_kq, w_head, gn_eps)
+    ws = _workspace(mta_workspace_size(shape), q.device, workspace)
+    status = lib().mta_forward_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq),
+                                     _ptr(w_head), _ptr(gn_weight), _ptr(gn_bias), _ptr(gate),
+                                     _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream_ptr(stream, q.device))
+    _check("mta_forward_gated", status)
+    return out
 
 
 def mta_forward_unfused(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out=None,

@@ -89,11 +89,13 @@ size_t mta_unfused_workspace_size(const mta_shape *s)
     return mta::unfused_workspace_bytes(*s);
 }
 
-mta_status mta_forward_traced(int unfused, const mta_shape *s, const void *q, const void *k,
-                              const void *v, const float *w_kq, const float *w_head,
-                              const float *gn_weight, const float *gn_bias, float depth_scale,
-                              void *out, void *workspace, size_t workspace_bytes, void *stream,
-                              void *const *events, int n_events)
+namespace {
+
+mta_status forward_impl(int unfused, const mta_shape *s, const void *q, const void *k,
+                        const void *v, const float *w_kq, const float *w_head,
+                        const float *gn_weight, const float *gn_bias, float depth_scale,
+                        const float *gate, void *out, void *workspace, size_t workspace_bytes,
+                        void *stream, void *const *events, int n_events)
 {
     mta_status rc = check_shape(s);
     if (rc == MTA_OK) rc = check_tensors(q, k, v, w_kq, w_head, gn_weight, gn_bias, out);
@@ -103,13 +105,36 @@ mta_status mta_forward_traced(int unfused, const mta_shape *s, const void *q, co
     const size_t need = fused ? mta::fused_workspace_bytes(*s) : mta::unfused_workspace_bytes(*s);
     rc = check_workspace(workspace, workspace_bytes, need);
     if (rc != MTA_OK) return rc;
-    mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out};
+    mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out, gate};
     mta::Trace tr;
     tr.events = events;
     tr.n = n_events;
     cudaStream_t st = (cudaStream_t)stream;
     return fused ? mta::launch_fused(*s, a, workspace, st, tr)
                  : mta::launch_unfused(*s, a, workspace, st, tr);
+}
+
+}  // namespace
+
+mta_status mta_forward_traced(int unfused, const mta_shape *s, const void *q, const void *k,
+                              const void *v, const float *w_kq, const float *w_head,
+                              const float *gn_weight, const float *gn_bias, float depth_scale,
+                              void *out, void *workspace, size_t workspace_bytes, void *stream,
+                              void *const *events, int n_events)
+{
+    return forward_impl(unfused, s, q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale,
+                        nullptr, out, workspace, workspace_bytes, stream, events, n_events);
+}
+
+mta_status mta_forward_gated(const mta_shape *s, const void *q, const void *k, const void *v,
+                             const float *w_kq, const float *w_head, const float *gn_weight,
+                             const float *gn_bias, const float *gate, void *out, void *workspace,
+                             size_t workspace_bytes, void *stream)
+{
+    if (!gate) return MTA_ERR_INVALID_ARG;
+    if (((uintptr_t)gate & 3u) != 0) return MTA_ERR_ALIGNMENT;
+    return forward_impl(0, s, q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.f, gate, out,
+                        workspace, workspace_bytes, stream, nullptr, 0);
 }
 
 mta_status mta_forward(const mta_shape *s, const void *q, const void *k, const void *v,

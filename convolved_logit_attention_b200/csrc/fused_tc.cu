@@ -1039,12 +1039,14 @@ __device__ __forceinline__ float warp_sum(float x)
 // One CTA per (query row i, batch b); warp w handles heads w, w+4, ...:
 // O^h = sum_{h'} part[b][i][h][h'] (fp16 partials, summed in fp32), then
 // GroupNorm over the head's d values (mean and biased variance by warp
-// shuffles), affine, depth scale.
+// shuffles), affine, and the head's scale: the depth scale, or sigmoid(g_h)
+// ("Group Normalization with Sigmoid Gating").
 template <int D, int CH>
 __global__ void __launch_bounds__(128)
 k_mix_groupnorm(const __half *__restrict__ part, const float *__restrict__ gn_weight,
-                const float *__restrict__ gn_bias, float depth_scale, float eps,
-                __nv_bfloat16 *__restrict__ out, int T, int H)
+                const float *__restrict__ gn_bias, float depth_scale,
+                const float *__restrict__ gate, float eps, __nv_bfloat16 *__restrict__ out,
+                int T, int H)
 {
     const int i = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -1072,13 +1074,15 @@ k_mix_groupnorm(const __half *__restrict__ part, const float *__restrict__ gn_we
         for (int u = 0; u < PER; ++u)
             sq += (o[u].x - mean) * (o[u].x - mean) + (o[u].y - mean) * (o[u].y - mean);
         const float inv = 1.f / sqrtf(warp_sum(sq) / D + eps);
+        // the head's output scale: sigmoid(g_h), or the depth scale
+        const float scale = gate ? 1.f / (1.f + expf(-gate[h])) : depth_scale;
         __nv_bfloat162 *dst = (__nv_bfloat162 *)(out + ((size_t)b * T + i) * ((size_t)H * D) + (size_t)h * D);
 #pragma unroll
         for (int u = 0; u < PER; ++u) {
             const int e = 2 * (lane + 32 * u), ch = h * D + e;
             dst[lane + 32 * u] = __floats2bfloat162_rn(
-                depth_scale * ((o[u].x - mean) * inv * gn_weight[ch] + gn_bias[ch]),
-                depth_scale * ((o[u].y - mean) * inv * gn_weight[ch + 1] + gn_bias[ch + 1]));
+                scale * ((o[u].x - mean) * inv * gn_weight[ch] + gn_bias[ch]),
+                scale * ((o[u].y - mean) * inv * gn_weight[ch + 1] + gn_bias[ch + 1]));
         }
     }
 }
@@ -1266,7 +1270,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     tr.after(2, st);
     tr.before(3, st);
     k_mix_groupnorm<D, CH><<<dim3(s.T, s.B), 128, 0, st>>>(part, a.gn_weight, a.gn_bias,
-                                                         a.depth_scale, s.gn_eps,
+                                                         a.depth_scale, a.gate, s.gn_eps,
                                                          (__nv_bfloat16 *)a.out, s.T, s.H);
     tr.after(3, st);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;

@@ -15,6 +15,7 @@ struct ForwardArgs {
     const float *w_kq, *w_head, *gn_weight, *gn_bias;
     float depth_scale;
     void *out;
+    const float *gate = nullptr;   // [H] sigmoid-gate logits; null: depth scale
 };
 
 // Optional CUDA events recorded around the kernel launches of one call.

@@ -212,12 +212,15 @@ k_softmax_mix(const float *__restrict__ map1, float *__restrict__ dst,
 
 // S7..S9: O = A_new V for 32 query rows of one (b, h) and all d columns,
 // then per row: mean and biased variance over d (warp-shuffle reductions),
-// out = depth_scale * ((O - mean) / sqrt(var + eps) * gamma + beta).
+// out = scale_h * ((O - mean) / sqrt(var + eps) * gamma + beta), with scale_h
+// the depth scale or, with a gate, sigmoid(g_h) ("Group Normalization with
+// Sigmoid Gating").
 template <typename TIO>
 __global__ void __launch_bounds__(256)
 k_pv_groupnorm(const float *__restrict__ amap, const TIO *__restrict__ v,
                const float *__restrict__ gn_weight, const float *__restrict__ gn_bias,
-               float depth_scale, float eps, TIO *__restrict__ out, int T, int H, int d)
+               float depth_scale, const float *__restrict__ gate, float eps,
+               TIO *__restrict__ out, int T, int H, int d)
 {
     const int i0 = blockIdx.x * kPvRows;
     const size_t bh = blockIdx.y;
@@ -277,10 +280,11 @@ k_pv_groupnorm(const float *__restrict__ amap, const TIO *__restrict__ v,
         for (int e = lane; e < d; e += 32) { float t = os[r][e] - mean; s2 += t * t; }
         const float var = warp_sum(s2) / d;
         const float inv = 1.f / sqrtf(var + eps);
+        const float scale = gate ? 1.f / (1.f + expf(-gate[h])) : depth_scale;
         TIO *dst = out + ((size_t)b * T + i) * ((size_t)H * d) + (size_t)h * d;
         for (int e = lane; e < d; e += 32) {
             const size_t ch = (size_t)h * d + e;
-            dst[e] = from_f32<TIO>(depth_scale * ((os[r][e] - mean) * inv * gn_weight[ch] + gn_bias[ch]));
+            dst[e] = from_f32<TIO>(scale * ((os[r][e] - mean) * inv * gn_weight[ch] + gn_bias[ch]));
         }
     }
 }
@@ -347,11 +351,11 @@ mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     tr.before(3, st);
     if (s.io == MTA_BF16)
         k_pv_groupnorm<__nv_bfloat16><<<g4, 256, 0, st>>>(
-            map0, (const __nv_bfloat16 *)a.v, a.gn_weight, a.gn_bias, a.depth_scale, s.gn_eps,
-            (__nv_bfloat16 *)a.out, s.T, s.H, s.d);
+            map0, (const __nv_bfloat16 *)a.v, a.gn_weight, a.gn_bias, a.depth_scale, a.gate,
+            s.gn_eps, (__nv_bfloat16 *)a.out, s.T, s.H, s.d);
     else
         k_pv_groupnorm<float><<<g4, 256, 0, st>>>(map0, (const float *)a.v, a.gn_weight,
-                                                  a.gn_bias, a.depth_scale, s.gn_eps,
+                                                  a.gn_bias, a.depth_scale, a.gate, s.gn_eps,
                                                   (float *)a.out, s.T, s.H, s.d);
     tr.after(3, st);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;

@@ -122,6 +122,17 @@ MTA_API mta_status mta_forward(const mta_shape *shape, const void *q, const void
                        const float *gn_bias, float depth_scale, void *out,
                        void *workspace, size_t workspace_bytes, void *stream);
 
+/* The forward with the pages' default output scale ("Multi-Token Attention
+ * -- Paper Graph", "Group Normalization with Sigmoid Gating"): head h of the
+ * GroupNorm output (after its affine) is multiplied by sigmoid(gate[h]),
+ * out = GN(...) * sigmoid(g), in place of a depth scale.  gate is a caller-
+ * owned device array of H floats (4-byte aligned); NULL is MTA_ERR_INVALID_ARG.
+ * Path, workspace and every other argument as for mta_forward. */
+MTA_API mta_status mta_forward_gated(const mta_shape *shape, const void *q, const void *k,
+                             const void *v, const float *w_kq, const float *w_head,
+                             const float *gn_weight, const float *gn_bias, const float *gate,
+                             void *out, void *workspace, size_t workspace_bytes, void *stream);
+
 /* The same forward computed step by step with the T x T maps materialised in
  * the workspace (S1+S2 logits, S3+S4 conv, S5+S6 softmax and mix, S7..S9
  * PV with the GroupNorm epilogue), all arithmetic in fp32.  Same arguments

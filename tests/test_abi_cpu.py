@@ -83,6 +83,21 @@ def test_forward_rejects_null_misaligned_and_small_workspace(L):
                                  mta.mta_unfused_workspace_size(s) - 1, None) == -4
 
 
+def test_gated_forward_argument_checks(L):
+    # the gate is required and 4-byte aligned; the other checks are mta_forward's
+    s = shape()
+    a = ctypes.c_void_p(1 << 20)
+    z = ctypes.c_void_p(0)
+    need = mta.mta_workspace_size(s)
+    args = [a] * 7
+    assert L.mta_forward_gated(ctypes.byref(s), *args, z, a, a, need, None) == -1
+    assert L.mta_forward_gated(ctypes.byref(s), *args, ctypes.c_void_p((1 << 20) + 2), a, a,
+                               need, None) == -3
+    assert L.mta_forward_gated(ctypes.byref(s), *args, a, a, a, need - 1, None) == -4
+    bad = shape(c_h=3)
+    assert L.mta_forward_gated(ctypes.byref(bad), *args, a, a, a, 1 << 40, None) == -1
+
+
 def test_debug_attention_argument_checks(L):
     s = shape()
     a = ctypes.c_void_p(1 << 20)

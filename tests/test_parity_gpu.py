@@ -197,3 +197,42 @@ def test_full_size_every_row_repeatable_and_matches_materialised_path():
     err = np.abs(runs[0] - ref)
     assert float(err.max()) <= 2 * TOL_BF16_MAXABS
     assert float(np.linalg.norm(runs[0] - ref) / np.linalg.norm(ref)) <= 2 * TOL_BF16_RELL2
+
+
+GATE = np.array([-2.0, -0.5, 0.25, 1.5, 3.0, -1.0, 0.0, 0.75] * 4, dtype=np.float32)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "toy_letters"])
+def test_gated_output_elementwise(name):
+    """Sigmoid-gated output ("Group Normalization with Sigmoid Gating") on
+    both paths: tiny_f32 takes the materialised path, toy_letters the fused
+    one; the gate values are exactly representable, and the oracle widens the
+    same float32 values."""
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    d = to_device(x, w.io)
+    gate = GATE[:w.H].copy()
+    out = mta.mta_forward_gated(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                                d["gn_bias"], torch.from_numpy(gate).cuda(), gn_eps=x["gn_eps"])
+    mta.mta_sync_status()
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = oracle.forward(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                         x["gn_bias"], 0.0, gn_eps=x["gn_eps"], gate=gate)
+    assert_close(got, ref, w.io, name + " gated")
+
+
+def test_gated_output_full_size_sampled_rows():
+    """The T = 4096 workload on the fused path with the gate, on sampled rows."""
+    w = WORKLOADS["longctx_4k"]
+    x = make_inputs(w)
+    d = to_device(x, w.io)
+    gate = GATE[:w.H].copy()
+    got = mta.mta_forward_gated(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                                d["gn_bias"], torch.from_numpy(gate).cuda(), gn_eps=x["gn_eps"])
+    mta.mta_sync_status()
+    got = got.float().cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(12)
+    rows = sample_rows(w.T, rng, n=6)
+    ref = oracle.rows(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                      x["gn_bias"], 0.0, 1, rows, gn_eps=x["gn_eps"], gate=gate)
+    assert_close(got[1, rows], ref, w.io, "longctx_4k gated")
