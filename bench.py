@@ -56,6 +56,9 @@ def parse_args(argv=None):
                         "unfused: mta_forward_unfused (materialised maps)")
     p.add_argument("--batch", type=int, default=None,
                    help="override the workload's batch size (smaller cases for profiler captures)")
+    p.add_argument("--gate", action="store_true",
+                   help="time mta_forward_gated (sigmoid-gated output, fixed gate values) "
+                        "instead of mta_forward; reported on the whole step")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -245,7 +248,14 @@ def time_mta(args, w, d, world, device):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
+    gate = torch.linspace(-2.0, 2.0, w.H, dtype=torch.float32, device=device)
+
     def step(events):
+        if args.gate:
+            mta.mta_forward_gated(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                                  d["gn_bias"], gate, out=out, workspace=ws, stream=stream,
+                                  gn_eps=w.gn_eps)
+            return
         mta.mta_forward_traced(unfused, events, d["q"], d["k"], d["v"], d["w_kq"], d["w_head"],
                                d["gn_weight"], d["gn_bias"], w.depth_scale, out=out,
                                workspace=ws, stream=stream, gn_eps=w.gn_eps)
@@ -273,7 +283,7 @@ def time_mta(args, w, d, world, device):
     mta.mta_sync_status(stream, device)
     total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
     per_kernel = {}
-    for s in range(args.steps):
+    for s in range(args.steps if not args.gate else 0):
         for i, name in enumerate(names):
             per_kernel.setdefault(name, 0.0)
             per_kernel[name] += kern_ev[s][2 * i].elapsed_time(kern_ev[s][2 * i + 1])
@@ -413,22 +423,29 @@ def mta_arm(args, w, world, rank, local):
     flops = w.algorithmic_flops()
     value = world * flops * args.steps / (total_ms / 1e3) / 1e12
     kernels = {n: t / args.steps for n, t in res["per_kernel_ms"].items()}
-    dom = max(kernels, key=kernels.get)
-    rl = roofline(dom, w, kernels[dom], peaks, peak_src)
+    if kernels:
+        dom = max(kernels, key=kernels.get)
+        rl = roofline(dom, w, kernels[dom], peaks, peak_src)
+    else:   # --gate: no per-launch events; the whole step against the tensor peak
+        rl = dict(roofline("k_mta_fused", w, per_step_ms, peaks, peak_src), traffic=None,
+                  kernel="whole step (mta_forward_gated)")
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if (w.io == "bf16" and res["path"] == "fused_tc") else "f32",
-            "data": "synthetic", "config": workload_config(w, res["path"]),
+            "data": "synthetic",
+            "config": dict(workload_config(w, res["path"]),
+                           output_scale="sigmoid gate" if args.gate else "depth scale"),
             "tokens_per_s": world * w.tokens() * args.steps / (total_ms / 1e3),
             "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
             "peaks": dict(peaks, source=peak_src),
             "roofline": {k: rl[k] for k in ("bound", "achieved", "peak", "unit", "frac",
                                              "traffic")},
             "roofline_detail": rl,
-            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src)) for n in res["names"]],
+            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src)) for n in res["names"]
+                        if n in kernels],
             "gpu_launches": res["launches"], "clocks": res["clocks"]}
-    if not args.no_e2e:
+    if not args.no_e2e and not args.gate:
         e2e_ms, h2d, d2h = time_e2e(args, w, x, device)
         e2e_ms = dist_max(e2e_ms, world, device)
         line["e2e"] = {"value": world * flops * args.steps / (e2e_ms / 1e3) / 1e12,
