@@ -343,8 +343,13 @@ struct FusedCfg {
     static constexpr int kShiftBytes = kKfRows * D * 2;     // one shift of one Kf tile
     static constexpr int kSlotBytes = 2 * kShiftBytes;
     static constexpr int kStages = 4;
-    static constexpr int kVHeads = CH < 2 ? CH : 2;         // output heads per V slot
-    static constexpr int kVSlots = CH / kVHeads;            // V slots per key tile
+    // output heads per work item: their U accumulators take at most 256 TMEM
+    // columns; a larger group is split into kSplits items that repeat the
+    // QK^T and softmax work for their share of the output heads
+    static constexpr int kCHU = CH * D <= 256 ? CH : 256 / D;
+    static constexpr int kSplits = CH / kCHU;
+    static constexpr int kVHeads = kCHU < 2 ? kCHU : 2;     // output heads per V slot
+    static constexpr int kVSlots = kCHU / kVHeads;          // V slots per key tile
     static constexpr int kVN = kVHeads * D;                 // N of one PV MMA chain
     static constexpr int kVBytes = kVHeads * 16384;         // bytes of a V slot this CTA loads
     static constexpr int kMaxAtoms = 23;                    // q_atoms(8)
@@ -430,17 +435,20 @@ __device__ __forceinline__ void arrive_leader(uint64_t *bar)
 // the clusters (left to right in even rounds, right to left in odd ones), so
 // every role derives the same sequence with no communication.
 struct WorkItem {
-    int bh, b, g, hl, qb, i0, ntiles;
+    int bh, b, g, hl, hh0, qb, i0, ntiles;
 };
 
 template <bool PAIR>
-__device__ __forceinline__ bool work_item(int k, int cl, int ncl, int BH, int H, int CH, int nqb,
-                                          uint32_t rank, WorkItem &it)
+__device__ __forceinline__ bool work_item(int k, int cl, int ncl, int BH, int H, int CH,
+                                          int chu, int nqb, uint32_t rank, WorkItem &it)
 {
     const int per_head = PAIR ? nqb / 2 : nqb;
+    const int splits = CH / chu;
     const int pos = k * ncl + ((k & 1) ? ncl - 1 - cl : cl);
-    if (pos >= per_head * BH) return false;
-    const int cls = pos / BH, bhx = pos % BH;
+    if (pos >= per_head * BH * splits) return false;
+    const int cls = pos / (BH * splits), rem = pos % (BH * splits);
+    const int bhx = rem / splits;
+    it.hh0 = (rem % splits) * chu;            // first output head of the item
     const int hs = bhx % H;
     it.bh = bhx;
     it.b = bhx / H;
@@ -504,7 +512,9 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int consumers = PAIR ? 8 : 4;   // softmax warps that publish P~
     const int kf_slots = (c_q + 1) / 2;
-    auto item = [&](int k, WorkItem &it) { return work_item<PAIR>(k, cl, ncl, BH, H, CH, nqb, rank, it); };
+    auto item = [&](int k, WorkItem &it) {
+        return work_item<PAIR>(k, cl, ncl, BH, H, CH, C::kCHU, nqb, rank, it);
+    };
 
     if (threadIdx.x == 0) {
         tc::mbar_init(bar_q, 1);
@@ -587,7 +597,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             auto load_v = [&](const WorkItem &it, int u, int vs) -> bool {
                 uint8_t *dst = claim(C::kVBytes);
                 if (dst == nullptr) return false;
-                const int z0 = it.b * H + it.g * CH + vs * C::kVHeads;
+                const int z0 = it.b * H + it.g * CH + it.hh0 + vs * C::kVHeads;
                 if constexpr (PAIR) {
                     if (C::kVHeads == 2) {
                         for (int c = 0; c < C::kChunks; ++c)
@@ -610,7 +620,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                         tc::tma_prefetch_3d(&mapK, 64 * c, u * kBN + (PAIR ? (int)rank * C::kKfRows : 0),
                                             it.bh * c_q + ip);
                 for (int vs = 0; vs < C::kVSlots; ++vs) {
-                    const int z0 = it.b * H + it.g * CH + vs * C::kVHeads;
+                    const int z0 = it.b * H + it.g * CH + it.hh0 + vs * C::kVHeads;
                     if (PAIR && C::kVHeads == 2) {
                         for (int c = 0; c < C::kChunks; ++c)
                             tc::tma_prefetch_3d(&mapV, 64 * c, u * kBN, z0 + (int)rank);
@@ -928,7 +938,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 if (t > 0 && __any_sync(0xffffffffu, need)) {
                     const float f = need ? alpha : 1.f;
 #pragma unroll
-                    for (int hh = 0; hh < CH; ++hh)
+                    for (int hh = 0; hh < C::kCHU; ++hh)
 #pragma unroll
                         for (int j = 0; j < D / 32; ++j) {
                             uint32_t u[32];
@@ -953,9 +963,10 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             }
             if (!ok) break;
             if (have_next) fetch_corr(nx);
-            float coef[CH];
+            const int hh0 = it.hh0;
+            float coef[C::kCHU];
 #pragma unroll
-            for (int hh = 0; hh < CH; ++hh) coef[hh] = w_head[((size_t)g * CH + hh) * CH + hl];
+            for (int hh = 0; hh < C::kCHU; ++hh) coef[hh] = w_head[((size_t)g * CH + hh0 + hh) * CH + hl];
             // the item's last PV has completed: write its partial outputs
             ok = __all_sync(0xffffffffu, wait_role<PAIR>(pv_done, (gt - 1) & 1, abort_flag));
             if (ok) {
@@ -967,9 +978,9 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 const float inv_l = 1.f / l;
                 const size_t row_stride = (size_t)H * CH * D;
 #pragma unroll 1
-                for (int hh = 0; hh < CH; ++hh) {
+                for (int hh = 0; hh < C::kCHU; ++hh) {
                     const float cf = coef[hh] * inv_l;
-                    __half *dst = part + (size_t)b * T * row_stride + (size_t)(g * CH + hh) * (CH * D) + hl * D;
+                    __half *dst = part + (size_t)b * T * row_stride + (size_t)(g * CH + hh0 + hh) * (CH * D) + hl * D;
                     uint32_t u[D];
 #pragma unroll
                     for (int j = 0; j < D / 32; ++j)
@@ -1257,7 +1268,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const int n_items = (int)BH * (PAIR ? L.nqb / 2 : L.nqb);
+        const int n_items = (int)BH * (PAIR ? L.nqb / 2 : L.nqb) * C::kSplits;
         int resident = 0;
         if (max_resident_clusters<D, CH>(cfg, &resident) != MTA_OK)
             return MTA_ERR_CUDA;
@@ -1282,7 +1293,8 @@ bool fused_supported(const mta_shape &s)
 {
     if (s.io != MTA_BF16) return false;
     if (s.d != 64 && s.d != 128) return false;
-    if (!(s.c_h == 1 || s.c_h == 2 || s.c_h == 4) || s.c_h * s.d > 256) return false;
+    // up to 256 / d output heads per work item; larger groups split in two
+    if (!(s.c_h == 1 || s.c_h == 2 || s.c_h == 4 || s.c_h == 8) || s.c_h * s.d > 512) return false;
     if (s.c_q > 8 || s.c_k > 15 || d_m(s.c_q, s.c_k) > kCorrW - 2) return false;
     return true;
 }
@@ -1302,10 +1314,12 @@ mta_status launch_fused(const mta_shape &s, const ForwardArgs &a, void *ws, cuda
     if (s.d == 128) {
         if (s.c_h == 1) return launch_fused_t<128, 1>(s, a, ws, st, tr);
         if (s.c_h == 2) return launch_fused_t<128, 2>(s, a, ws, st, tr);
+        if (s.c_h == 4) return launch_fused_t<128, 4>(s, a, ws, st, tr);
     } else {
         if (s.c_h == 1) return launch_fused_t<64, 1>(s, a, ws, st, tr);
         if (s.c_h == 2) return launch_fused_t<64, 2>(s, a, ws, st, tr);
         if (s.c_h == 4) return launch_fused_t<64, 4>(s, a, ws, st, tr);
+        if (s.c_h == 8) return launch_fused_t<64, 8>(s, a, ws, st, tr);
     }
     return MTA_ERR_UNSUPPORTED;
 }

@@ -117,7 +117,8 @@ def test_unfused_workspace_is_two_fp32_maps(L):
     (dict(B=1, H=16, T=16384, d=128, c_q=8, c_k=15, c_h=2), 0),
     (dict(B=8, H=4, T=256, d=64, c_q=4, c_k=15, c_h=2), 0),
     (dict(B=1, H=16, T=64, d=64, c_q=2, c_k=3, c_h=4), 0),
-    (dict(B=1, H=16, T=16384, d=128, c_q=6, c_k=11, c_h=4), 1),    # c_h * d > 256
+    (dict(B=1, H=16, T=16384, d=128, c_q=6, c_k=11, c_h=4), 0),    # split output heads
+    (dict(B=1, H=16, T=256, d=128, c_q=6, c_k=11, c_h=8), 1),      # c_h * d > 512
     (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2), 1),        # d not 64 or 128
     (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2, io="f32"), 1),
     (dict(B=1, H=4, T=128, d=128, c_q=6, c_k=11, c_h=2, io="f32"), 1),

@@ -87,6 +87,8 @@ RAGGED = [
     (1, 4, 129, 128, 6, 11, 4, "bf16"),
     (2, 2, 384, 128, 6, 11, 2, "bf16"),     # several full tiles
     (1, 2, 511, 64, 4, 15, 2, "bf16"),
+    (2, 4, 384, 128, 6, 11, 4, "bf16"),     # output heads split over two work items
+    (1, 8, 200, 64, 3, 5, 8, "bf16"),
 ]
 
 
