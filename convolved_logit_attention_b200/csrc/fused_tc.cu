@@ -74,7 +74,8 @@ __host__ __device__ inline int d_m(int c_q, int c_k) { return c_q - 1 + c_k / 2;
 
 constexpr int kProRows = 128;     // rows (keys and queries) per prologue CTA
 constexpr int kProQLo = 7;        // query rows before the block whose future logits are needed
-constexpr int kAuxThreads = 288;  // aux prologue: one future-logit work item per thread
+constexpr int kAuxRows = 64;      // query rows per aux prologue CTA
+constexpr int kAuxThreads = 160;  // aux prologue: one future-logit work item per thread
 
 // Packed fp32 pairs (Blackwell's f32x2 arithmetic): one instruction does two
 // fp32 FMAs, each rounded once, exactly as fmaf would.
@@ -169,27 +170,29 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
     if (am.x > 65504.f || am.y > 65504.f) atomicOr(&g_fused_error, kErrRange);
 }
 
-// The rest of the prologue: one CTA per (128-row block, b*H + h), 288
+// The rest of the prologue: one CTA per (64-row block, b*H + h), 160
 // threads, three sections:
 //  (b) the block's query rows in the permuted atom order, converted to fp16.
 //  (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in
-//      [1, D_m], for r in [j0 - 7, j0 + 128), from shared-memory copies of
+//      [1, D_m], for r in [j0 - 7, j0 + 64), from shared-memory copies of
 //      the rows involved.
 //  (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
 //      r = i - i' >= 0 of theta[i'][j'] F[r][delta].
 template <int D>
-__global__ void __launch_bounds__(kAuxThreads, 2)
+__global__ void __launch_bounds__(kAuxThreads, 4)
 k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
            const float *__restrict__ w_kq, __half *__restrict__ qp, float *__restrict__ corr, int T,
            int Tp, int H, int c_q, int c_k, float scale)
 {
-    constexpr int QR = kProQLo + kProRows;
+    constexpr int QR = kProQLo + kAuxRows;
     constexpr int TW = 16;                     // tap row stride (c_k <= 15)
     __shared__ float th[8 * TW];
     __shared__ float fs[QR * kCorrW];
     extern __shared__ __align__(16) __nv_bfloat16 qk_sm[];   // section (c) row copies
     const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
-    const int j0 = blk * kProRows;
+    const int j0 = blk * kAuxRows;
+    // the 128-row query block whose permuted rows this CTA writes one half of
+    const int qblk = j0 / kProRows, half = (j0 % kProRows) / kAuxRows;
     const int tid = threadIdx.x;
     const size_t head_off = (size_t)bh * T * D;
     const int R = c_k / 2;
@@ -199,10 +202,10 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
     __syncthreads();
     // Row copies in shared memory, all in flight at once (cp.async): q rows
-    // [j0-7, j0+128) and k rows [j0-6, j0+142), zero outside [0, T); rows are
+    // [j0-7, j0+64) and k rows [j0-6, j0+78), zero outside [0, T); rows are
     // padded by 16 bytes so that threads on different rows hit different banks.
     constexpr int RS = D + 8;                  // padded row stride in bf16 elements
-    constexpr int KR = QR + kCorrW - 3;        // k rows j0-6 .. j0+141 (r + delta <= j0+127+14)
+    constexpr int KR = QR + kCorrW - 3;        // k rows j0-6 .. j0+77 (r + delta <= j0+63+14)
     constexpr int CPR = D / 8;                 // 16-byte chunks per row
     __nv_bfloat16 *qsm = qk_sm;                // [QR][RS]
     __nv_bfloat16 *ksm = qk_sm + QR * RS;      // [KR][RS]
@@ -216,15 +219,19 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
     tc::cp_async_wait_all();
     __syncthreads();
-    // (b) permuted query rows: atom a, row s <- q_{j0-(c_q-1)+a+16s}, from the
-    //     copy (those rows lie in [j0-7, j0+128) since c_q <= 8); 8 elements per thread
+    // (b) permuted query rows of the 128-row block jb0 = j0 - 64*half: atom a,
+    //     row s <- q_{jb0-(c_q-1)+a+16s}; this CTA writes rows s in
+    //     [4*half, 4*half+4), which lie in its copy [j0-7, j0+64) since
+    //     c_q <= 8; 8 elements per thread
     {
         const int NA = q_atoms(c_q);
-        __half *dst = qp + ((size_t)bh * (Tp / kBM) + blk) * (size_t)NA * 8 * D;
+        __half *dst = qp + ((size_t)bh * (Tp / kBM) + qblk) * (size_t)NA * 8 * D;
         bool range_ok = true;
-        for (int idx = tid; idx < NA * 8 * CPR; idx += kAuxThreads) {
-            const int row = idx / CPR, c8 = idx % CPR;
-            const int rq = kProQLo - (c_q - 1) + row / 8 + 16 * (row % 8);   // copy row of q_i
+        for (int idx = tid; idx < NA * 4 * CPR; idx += kAuxThreads) {
+            const int rowh = idx / CPR, c8 = idx % CPR;
+            const int a = rowh / 4, sr = rowh % 4;                // atom, row within this half
+            const int row = 8 * a + 4 * half + sr;                // row of the block's atom layout
+            const int rq = kProQLo - (c_q - 1) + a + 16 * sr;    // copy row of q_i
             const uint4 in = *(const uint4 *)(qsm + rq * RS + 8 * c8);
             const __nv_bfloat162 *bp = (const __nv_bfloat162 *)&in;
             uint4 outv;
@@ -289,7 +296,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     //     corr[i][e] = sum_{i'} sum_{delta} ts[i'][e + delta] F[i - i'][delta];
     //     taps with delta < 1 or jj outside [0, c_k) are zero in ts, F rows
     //     before the sequence are zero, so e >= D_m comes out zero too.
-    if (tid < 2 * kProRows) {
+    if (tid < 2 * kAuxRows) {
         constexpr int EH = kCorrW / 2;
         const int ir = tid >> 1, e0 = (tid & 1) * EH, i = j0 + ir;
         float acc[EH];
@@ -315,11 +322,11 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
 }
 
-// Dynamic shared memory of the prologue: section (c)'s bf16 copies of
-// 135 query rows and 148 key rows, each padded by 8 elements.
+// Dynamic shared memory of the aux prologue: bf16 copies of 71 query rows
+// and 84 key rows, each padded by 8 elements.
 size_t prologue_smem_bytes(int D)
 {
-    const int QR = kProQLo + kProRows;
+    const int QR = kProQLo + kAuxRows;
     return (size_t)(QR + QR + kCorrW - 3) * (D + 8) * sizeof(__nv_bfloat16);
 }
 
@@ -1241,7 +1248,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
             cudaStreamWaitEvent(side.s, side.fork, 0) != cudaSuccess)
             return MTA_ERR_CUDA;
         tr.before(1, side.s);
-        k_fold_aux<D><<<dim3(L.nqb, (unsigned)BH), kAuxThreads, aux_smem, side.s>>>(
+        k_fold_aux<D><<<dim3(L.Tp / kAuxRows, (unsigned)BH), kAuxThreads, aux_smem, side.s>>>(
             (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, qp, corr, s.T, L.Tp, s.H,
             s.c_q, s.c_k, scale);
         tr.after(1, side.s);
