@@ -639,9 +639,10 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 }
             };
             constexpr int kPrefetch = 2;     // key tiles prefetched ahead
-            WorkItem it, nx, prev;
+            // slot order = the issuer's: per item, Kf(t) then V(t-1) for each
+            // tile, and the item's last V right after its last Kf
+            WorkItem it, nx;
             bool have = item(0, it);
-            int prev_t = -1;
             for (int k = 0; have && ok; ++k) {
                 const bool have_next = item(k + 1, nx);
                 for (int t = 0; t < it.ntiles && ok; ++t) {
@@ -656,14 +657,12 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                         prefetch(nx, 0);
                         prefetch(nx, 1);
                     }
-                    for (int vs = 0; vs < C::kVSlots && ok && prev_t >= 0; ++vs) ok = load_v(prev, prev_t, vs);
-                    prev = it;
-                    prev_t = t;
+                    for (int vs = 0; vs < C::kVSlots && ok && t > 0; ++vs) ok = load_v(it, t - 1, vs);
                 }
+                for (int vs = 0; vs < C::kVSlots && ok; ++vs) ok = load_v(it, it.ntiles - 1, vs);
                 it = nx;
                 have = have_next;
             }
-            for (int vs = 0; vs < C::kVSlots && ok && prev_t >= 0; ++vs) ok = load_v(prev, prev_t, vs);
             // copies this thread started land before the CTA may exit; in a pair
             // their completion is counted in the leader, so the peer waits a while
             if (leader) {
@@ -730,7 +729,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 }
                 if (issuer) commit(pv_done);
             };
-            int gt = 0, prev_t = -1;
+            int gt = 0;
             WorkItem it;
             for (int k = 0; item(k, it); ++k) {
                 gate(kGateQ);                  // this item's Q block has landed
@@ -761,11 +760,12 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                         commit(&s_full[sb]);
                         if (t == it.ntiles - 1) commit(q_free);   // the Q block may be replaced
                     }
-                    if (gt > 0) issue_pv(gt - 1, prev_t);
-                    prev_t = t;
+                    if (t > 0) issue_pv(gt - 1, t - 1);
                 }
+                // the item's last PV before the next item's first QK: its
+                // partial outputs can be written while that QK runs
+                issue_pv(gt - 1, it.ntiles - 1);
             }
-            if (gt > 0) issue_pv(gt - 1, prev_t);
             // all MMAs this warp issued complete before TMEM is released
             if (issuer) {
                 if constexpr (PAIR) tc::mma_commit_pair_multicast(mma_drain, 0x1);
@@ -818,10 +818,10 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 meet_q(k);
                 for (int t = 0; t < it.ntiles; ++t, ++gt) {
                     for (int m = 0; m < kf_slots; ++m) meet(false, 0);
-                    for (int vs = 0; vs < C::kVSlots && gt > 0; ++vs) meet(vs == 0, gt - 1);
+                    for (int vs = 0; vs < C::kVSlots && t > 0; ++vs) meet(vs == 0, gt - 1);
                 }
+                for (int vs = 0; vs < C::kVSlots; ++vs) meet(vs == 0, gt - 1);
             }
-            for (int vs = 0; vs < C::kVSlots && gt > 0; ++vs) meet(vs == 0, gt - 1);
         }
     } else {
         // ---------------- softmax and epilogue (warps 2..5): thread = TMEM lane = one query row
