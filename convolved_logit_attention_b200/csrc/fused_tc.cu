@@ -104,6 +104,29 @@ __device__ __forceinline__ unsigned long long bf2_to_f2(uint32_t v)
     return f2_pack(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
+// Warp-level bf16 MMA (m16n8k16, fp32 accumulate) and its shared-memory
+// fragment loads, for the small banded product of the aux prologue.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(tc::smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void *p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(tc::smem_u32(p)));
+}
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4],
+                                               const uint32_t (&b)[2])
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+                 "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // Folded keys: one CTA per (128-key block, b*H + h), 256 threads; thread =
 // one column pair x a run of RPG consecutive keys, in windows of SUB keys.
 // Kf^{(i')}_j = sum_jj ths[i'][jj] k_{j + RT - jj}, with the taps zero-padded
@@ -203,19 +226,23 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     __syncthreads();
     // Row copies in shared memory, all in flight at once (cp.async): q rows
     // [j0-7, j0+64) and k rows [j0-6, j0+78), zero outside [0, T); rows are
-    // padded by 16 bytes so that threads on different rows hit different banks.
+    // padded by 16 bytes so that threads on different rows hit different banks,
+    // and both copies are padded with zero rows to whole MMA tiles (QRP, KRP).
     constexpr int RS = D + 8;                  // padded row stride in bf16 elements
     constexpr int KR = QR + kCorrW - 3;        // k rows j0-6 .. j0+77 (r + delta <= j0+63+14)
+    constexpr int QRP = (QR + 15) / 16 * 16;   // 80 q rows: five 16-row MMA tiles
+    constexpr int KRP = QRP + 16;              // 96 k rows: each tile reaches 32 rows on
     constexpr int CPR = D / 8;                 // 16-byte chunks per row
-    __nv_bfloat16 *qsm = qk_sm;                // [QR][RS]
-    __nv_bfloat16 *ksm = qk_sm + QR * RS;      // [KR][RS]
-    for (int idx = tid; idx < (QR + KR) * CPR; idx += kAuxThreads) {
+    __nv_bfloat16 *qsm = qk_sm;                // [QRP][RS]
+    __nv_bfloat16 *ksm = qk_sm + QRP * RS;     // [KRP][RS]
+    for (int idx = tid; idx < (QRP + KRP) * CPR; idx += kAuxThreads) {
         const int row = idx / CPR, c8 = idx % CPR;
-        const bool isq = row < QR;
-        const int g = isq ? j0 - kProQLo + row : j0 - (kProQLo - 1) + (row - QR);
-        const bool in = g >= 0 && g < T;
+        const bool isq = row < QRP;
+        const int lr = isq ? row : row - QRP;
+        const int g = isq ? j0 - kProQLo + lr : j0 - (kProQLo - 1) + lr;
+        const bool in = (isq ? lr < QR : lr < KR) && g >= 0 && g < T;
         const __nv_bfloat16 *src = (isq ? q : k) + head_off + (size_t)(in ? g : 0) * D + 8 * c8;
-        tc::cp_async16((isq ? qsm + row * RS : ksm + (row - QR) * RS) + 8 * c8, src, in);
+        tc::cp_async16((isq ? qsm : ksm) + lr * RS + 8 * c8, src, in);
     }
     tc::cp_async_wait_all();
     __syncthreads();
@@ -246,45 +273,49 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
         }
         if (!range_ok) atomicOr(&g_fused_error, kErrRange);
     }
-    // (c) future logits F[r][delta] = scale * q_r . k_{r+delta} from the copies
+    // (c) future logits F[r][delta] = scale * q_r . k_{r+delta} from the copies,
+    //     on tensor cores (mma.sync m16n8k16, bf16 products summed in fp32): warp
+    //     w takes q rows rr in [16w, 16w+16) against k rows kr in [16w, 16w+32),
+    //     which hold every band entry delta = kr - rr + 1 in [1, 14] of its rows;
+    //     each (rr, delta) lands in exactly one accumulator element.
     const int Dm = d_m(c_q, c_k);
     {
-        __syncthreads();
-        // work item = (row rr, half of the diagonals): 7 independent packed
-        // accumulator chains share each loaded chunk of q_r
-        constexpr int DH = (kCorrW - 2) / 2;   // diagonals per half (delta <= 14)
-        for (int w = tid; w < 2 * QR; w += kAuxThreads) {
-            const int rr = w >> 1, d0 = 1 + (w & 1) * DH;
-            const int r = j0 - kProQLo + rr;
-            unsigned long long acc[DH];
+        const int wp = tid / 32, l = tid % 32;
+        if (wp < QRP / 16) {
+            const int m0 = 16 * wp;
+            float acc[4][4];
 #pragma unroll
-            for (int x = 0; x < DH; ++x) acc[x] = 0ull;
-            if (r >= 0) {
-                const __nv_bfloat16 *qr = qsm + rr * RS;
-                const __nv_bfloat16 *kc = ksm + (rr + d0 - 1) * RS;   // k row r + d0
-#pragma unroll 2
-                for (int c8 = 0; c8 < CPR; ++c8) {
-                    const uint4 a4 = *(const uint4 *)(qr + 8 * c8);
-                    const unsigned long long qa0 = bf2_to_f2(a4.x), qa1 = bf2_to_f2(a4.y),
-                                             qa2 = bf2_to_f2(a4.z), qa3 = bf2_to_f2(a4.w);
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
-                    for (int x = 0; x < DH; ++x) {
-                        const uint4 b4 = *(const uint4 *)(kc + x * RS + 8 * c8);
-                        acc[x] = f2_fma(qa0, bf2_to_f2(b4.x), acc[x]);
-                        acc[x] = f2_fma(qa1, bf2_to_f2(b4.y), acc[x]);
-                        acc[x] = f2_fma(qa2, bf2_to_f2(b4.z), acc[x]);
-                        acc[x] = f2_fma(qa3, bf2_to_f2(b4.w), acc[x]);
-                    }
+                for (int x = 0; x < 4; ++x) acc[j][x] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(af, qsm + (m0 + (l & 15)) * RS + 16 * ks + 8 * (l >> 4));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t bf[2];
+                    ldsm_x2(bf, ksm + (m0 + 8 * j + (l & 7)) * RS + 16 * ks + 8 * ((l >> 3) & 1));
+                    mma_16816_bf16(acc[j], af, bf);
                 }
             }
+            const int gq = l >> 2, tq = l & 3;
 #pragma unroll
-            for (int x = 0; x < DH; ++x) {
-                const int dl = d0 + x;
-                const float2 a2 = f2_unpack(acc[x]);
-                fs[rr * kCorrW + dl - 1] = (r >= 0 && dl <= Dm && r + dl < T) ? (a2.x + a2.y) * scale : 0.f;
-            }
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int rr = m0 + gq + 8 * (x >> 1);
+                    const int kr = m0 + 8 * j + 2 * tq + (x & 1);
+                    const int dl = kr - rr + 1;
+                    if (rr < QR && dl >= 1 && dl <= kCorrW - 2) {
+                        const int r = j0 - kProQLo + rr;
+                        fs[rr * kCorrW + dl - 1] =
+                            (r >= 0 && dl <= Dm && r + dl < T) ? acc[j][x] * scale : 0.f;
+                    }
+                }
         }
     }
+    __syncthreads();
     // taps indexed by s = e + delta: ts[i'][s] = theta[i'][i' + R - s]
     __shared__ float ts[8 * 32];
     for (int idx = tid; idx < 8 * 32; idx += kAuxThreads) {
@@ -322,12 +353,12 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
 }
 
-// Dynamic shared memory of the aux prologue: bf16 copies of 71 query rows
-// and 84 key rows, each padded by 8 elements.
+// Dynamic shared memory of the aux prologue: bf16 copies of 80 query rows
+// and 96 key rows (71 and 84 used, the rest zero), each padded by 8 elements.
 size_t prologue_smem_bytes(int D)
 {
-    const int QR = kProQLo + kAuxRows;
-    return (size_t)(QR + QR + kCorrW - 3) * (D + 8) * sizeof(__nv_bfloat16);
+    const int QRP = (kProQLo + kAuxRows + 15) / 16 * 16;
+    return (size_t)(QRP + QRP + 16) * (D + 8) * sizeof(__nv_bfloat16);
 }
 
 // ------------------------------------------------------------ main kernel
