@@ -330,26 +330,31 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     if (tid < 2 * kAuxRows) {
         constexpr int EH = kCorrW / 2;
         const int ir = tid >> 1, e0 = (tid & 1) * EH, i = j0 + ir;
-        float acc[EH];
+        // entries e, e+1 share F[.][delta]: one packed f32x2 FMA for both
+        unsigned long long acc[EH / 2];
 #pragma unroll
-        for (int e = 0; e < EH; ++e) acc[e] = 0.f;
+        for (int p = 0; p < EH / 2; ++p) acc[p] = 0ull;
         for (int ip = 0; ip < c_q; ++ip) {
             const float *frow = fs + (ir + kProQLo - ip) * kCorrW;   // F row i - i'
             const float *trow = ts + ip * 32 + e0;
-            float f[kCorrW - 2], t[EH + kCorrW - 2];
+            float t[EH + kCorrW - 1];
 #pragma unroll
-            for (int x = 0; x < kCorrW - 2; ++x) f[x] = frow[x];
+            for (int x = 1; x < EH + kCorrW - 1; ++x) t[x] = trow[x];
 #pragma unroll
-            for (int x = 1; x < EH + kCorrW - 2; ++x) t[x] = trow[x];
+            for (int dl = 1; dl <= kCorrW - 2; ++dl) {
+                const float f = frow[dl - 1];
+                const unsigned long long ff = f2_pack(f, f);
 #pragma unroll
-            for (int e = 0; e < EH; ++e)
-#pragma unroll
-                for (int dl = 1; dl <= kCorrW - 2; ++dl) acc[e] = fmaf(t[e + dl], f[dl - 1], acc[e]);
+                for (int p = 0; p < EH / 2; ++p)
+                    acc[p] = f2_fma(f2_pack(t[2 * p + dl], t[2 * p + 1 + dl]), ff, acc[p]);
+            }
         }
         float4 *dst = (float4 *)(corr + ((size_t)bh * Tp + i) * kCorrW + e0);
 #pragma unroll
-        for (int u = 0; u < EH / 4; ++u)
-            dst[u] = make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
+        for (int u = 0; u < EH / 4; ++u) {
+            const float2 lo = f2_unpack(acc[2 * u]), hi = f2_unpack(acc[2 * u + 1]);
+            dst[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        }
     }
 }
 
