@@ -155,6 +155,12 @@ def dist_max(x, world, device):
     return float(t.item())
 
 
+def replica_tflops(world, flops_per_step, steps, max_total_ms):
+    """Whole-job throughput of `world` independent replicas, each doing
+    `steps` steps of `flops_per_step`, timed by the slowest rank."""
+    return world * flops_per_step * steps / (max_total_ms / 1e3) / 1e12
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -435,7 +441,7 @@ def mta_arm(args, w, world, rank, local):
     total_ms = dist_max(res["total_ms"], world, device)
     per_step_ms = total_ms / args.steps
     flops = w.algorithmic_flops()
-    value = world * flops * args.steps / (total_ms / 1e3) / 1e12
+    value = replica_tflops(world, flops, args.steps, total_ms)
     kernels = dict(res["per_kernel_ms"])   # average ms per launch, traced pass
     dom = max(kernels, key=kernels.get)
     rl = roofline(dom, w, kernels[dom], peaks, peak_src)
