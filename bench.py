@@ -312,41 +312,69 @@ def time_mta(args, w, d, world, device):
 
 
 def time_e2e(args, w, x, device):
-    """The public API with host buffers: per step, pinned host -> device copies
-    of every input, mta_forward, device -> host copy of the output."""
+    """The public API with host buffers: every step copies all of its inputs
+    from pinned host memory to the device, calls mta_forward and copies the
+    output back to pinned host memory.  Steps are pipelined the way a serving
+    loop would drive the library: two device buffer sets, with step s+1's
+    input copy (copy-in stream) overlapping step s's compute (compute stream)
+    and step s-1's output copy (copy-out stream).  The time runs from the
+    first input copy of the timed steps to the end of their last output copy."""
     import convolved_logit_attention_b200 as mta
     dt = torch.bfloat16 if w.io == "bf16" else torch.float32
+    names = ("q", "k", "v", "w_kq", "w_head", "gn_weight", "gn_bias")
     host = {n: torch.from_numpy(x[n]).to(dt).pin_memory() for n in ("q", "k", "v")}
     for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
         host[n] = torch.from_numpy(x[n]).pin_memory()
-    dev = {n: torch.empty_like(t, device=device) for n, t in host.items()}
-    out = torch.empty((w.B, w.T, w.H * w.d), dtype=dt, device=device)
-    out_host = torch.empty(out.shape, dtype=dt).pin_memory()
-    shape = mta.shape_of(dev["q"], dev["w_kq"], dev["w_head"], w.gn_eps)
+    nbuf = 2
+    dev = [{n: torch.empty_like(host[n], device=device) for n in names} for _ in range(nbuf)]
+    out = [torch.empty((w.B, w.T, w.H * w.d), dtype=dt, device=device) for _ in range(nbuf)]
+    out_host = [torch.empty(out[0].shape, dtype=dt).pin_memory() for _ in range(nbuf)]
+    shape = mta.shape_of(dev[0]["q"], dev[0]["w_kq"], dev[0]["w_head"], w.gn_eps)
     ws = torch.empty(max(mta.mta_workspace_size(shape), 1), dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream(device)
+    s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out.numel() * out.element_size()
+    d2h = out[0].numel() * out[0].element_size()
 
-    def step():
-        for n in host:
-            dev[n].copy_(host[n], non_blocking=True)
-        mta.mta_forward(dev["q"], dev["k"], dev["v"], dev["w_kq"], dev["w_head"],
-                        dev["gn_weight"], dev["gn_bias"], w.depth_scale, out=out, workspace=ws,
-                        stream=stream, gn_eps=w.gn_eps)
-        out_host.copy_(out, non_blocking=True)
+    def run(n_steps, first=None, last=None):
+        copied = [None] * n_steps
+        computed = [None] * n_steps
+        drained = [None] * n_steps
+        for st in range(n_steps):
+            bi = st % nbuf
+            with torch.cuda.stream(s_in):
+                if st >= nbuf:
+                    s_in.wait_event(computed[st - nbuf])      # buffer set free again
+                if st == 0 and first is not None:
+                    first.record(s_in)
+                for n in names:
+                    dev[bi][n].copy_(host[n], non_blocking=True)
+                copied[st] = torch.cuda.Event()
+                copied[st].record(s_in)
+            s_comp.wait_event(copied[st])
+            if st >= nbuf:
+                s_comp.wait_event(drained[st - nbuf])         # output buffer read back
+            d = dev[bi]
+            mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                            d["gn_bias"], w.depth_scale, out=out[bi], workspace=ws, stream=s_comp,
+                            gn_eps=w.gn_eps)
+            computed[st] = torch.cuda.Event()
+            computed[st].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[st])
+                out_host[bi].copy_(out[bi], non_blocking=True)
+                drained[st] = torch.cuda.Event()
+                drained[st].record(s_out)
+        if last is not None:
+            s_out.wait_event(drained[n_steps - 1])
+            last.record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        step()
+    run(max(1, args.warmup))
     torch.cuda.synchronize(device)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    for s in range(args.steps):
-        ev[s][0].record(stream)
-        step()
-        ev[s][1].record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    run(args.steps, t0, t1)
     torch.cuda.synchronize(device)
-    return sum(a.elapsed_time(b) for a, b in ev), h2d, d2h
+    mta.mta_sync_status(s_comp, device)
+    return t0.elapsed_time(t1), h2d, d2h
 
 
 def oracle_sample(w, x, n_units):
