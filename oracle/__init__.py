@@ -38,10 +38,19 @@ def _configure(lib):
     lib.mta_oracle_forward_gated.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
     lib.mta_oracle_rows_gated.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ip,
                                           ctypes.c_int, dp, ctypes.c_int]
+    lib.mta_oracle_forward_composed.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                                ctypes.c_double, dp, dp, ctypes.c_int]
+    lib.mta_oracle_rows_composed.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                             ctypes.c_double, dp, ctypes.c_int, ip, ctypes.c_int,
+                                             dp, ctypes.c_int]
+    lib.mta_oracle_stages_composed.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                               ctypes.c_double, dp, ctypes.c_int, dp, dp, dp, dp,
+                                               dp, dp]
     lib.mta_oracle_max_threads.argtypes = []
     for f in (lib.mta_oracle_forward, lib.mta_oracle_rows, lib.mta_oracle_stages,
               lib.mta_oracle_forward_gated, lib.mta_oracle_rows_gated,
-              lib.mta_oracle_max_threads):
+              lib.mta_oracle_forward_composed, lib.mta_oracle_rows_composed,
+              lib.mta_oracle_stages_composed, lib.mta_oracle_max_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -162,3 +171,81 @@ def stages(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, b=0, gn_eps=1
     if rc != 0:
         raise RuntimeError("mta_oracle_stages failed (%d)" % rc)
     return {"C": C, "P": P, "A": A, "O": O, "out": out}
+
+
+def _composed(q, w_kq, w_head, w_kq_post, w_head_post, gn_eps):
+    """Shape of a composition: (c_q, c_k) from the key-query kernels (both
+    [H, c_q, c_k] when both are given), c_h from the head mixes (1 when
+    there is none)."""
+    B, H, T, d = q.shape
+    kq = [w for w in (w_kq, w_kq_post) if w is not None]
+    hm = [w for w in (w_head, w_head_post) if w is not None]
+    c_q, c_k = kq[0].shape[1:] if kq else (1, 1)
+    c_h = hm[0].shape[-1] if hm else 1
+    for w in kq:
+        assert w.shape == (H, c_q, c_k), w.shape
+    for w in hm:
+        assert w.shape == (H // c_h, c_h, c_h), w.shape
+    return _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
+
+
+def forward_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
+                     depth_scale, gn_eps=1e-5, nthreads=0, gate=None):
+    """out[B, T, H*d] of a composition of "Putting Everything Together": the
+    steps Mask_0, [key-query conv w_kq], Mask_-inf, softmax, [head mix
+    w_head], [key-query conv w_kq_post on the probabilities, Mask_0],
+    [head mix w_head_post], A V, GroupNorm, scale; a bracketed step whose
+    weights are None is left out.  gate as in forward."""
+    q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
+    ws = [None if w is None else _f64(w) for w in (w_kq, w_head, w_kq_post, w_head_post)]
+    s = _composed(q, *ws, gn_eps)
+    g = None if gate is None else _f64(gate)
+    out = np.empty((s.B, s.T, s.H * s.d), dtype=np.float64)
+    rc = _load().mta_oracle_forward_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
+                                             *map(_ptr, ws), _ptr(gw), _ptr(gb),
+                                             float(depth_scale), _ptr(g), _ptr(out),
+                                             int(nthreads))
+    if rc != 0:
+        raise RuntimeError("mta_oracle_forward_composed failed (%d)" % rc)
+    return out
+
+
+def rows_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
+                  depth_scale, b, row_idx, gn_eps=1e-5, nthreads=0, gate=None):
+    """out[b, row_idx, :] of forward_composed, one row at a time."""
+    q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
+    ws = [None if w is None else _f64(w) for w in (w_kq, w_head, w_kq_post, w_head_post)]
+    s = _composed(q, *ws, gn_eps)
+    g = None if gate is None else _f64(gate)
+    idx = np.ascontiguousarray(np.asarray(row_idx, dtype=np.int32))
+    out = np.empty((idx.size, s.H * s.d), dtype=np.float64)
+    rc = _load().mta_oracle_rows_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
+                                          *map(_ptr, ws), _ptr(gw), _ptr(gb),
+                                          float(depth_scale), _ptr(g), int(b),
+                                          idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                          int(idx.size), _ptr(out), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("mta_oracle_rows_composed failed (%d)" % rc)
+    return out
+
+
+def stages_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
+                    depth_scale, b=0, gn_eps=1e-5, gate=None):
+    """Intermediates of forward_composed for batch entry b (small T only):
+    C [H,T,T] softmax input after both masks, P [H,T,T] softmax, A1 [H,T,T]
+    after the first head mix, A [H,T,T] the attention that meets V,
+    O [H,T,d] pre-normalisation head outputs, out [T, H*d]."""
+    q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
+    ws = [None if w is None else _f64(w) for w in (w_kq, w_head, w_kq_post, w_head_post)]
+    s = _composed(q, *ws, gn_eps)
+    g = None if gate is None else _f64(gate)
+    H, T, d = s.H, s.T, s.d
+    C, P, A1, A = (np.empty((H, T, T)) for _ in range(4))
+    O = np.empty((H, T, d)); out = np.empty((T, H * d))
+    rc = _load().mta_oracle_stages_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
+                                            *map(_ptr, ws), _ptr(gw), _ptr(gb),
+                                            float(depth_scale), _ptr(g), int(b), _ptr(C),
+                                            _ptr(P), _ptr(A1), _ptr(A), _ptr(O), _ptr(out))
+    if rc != 0:
+        raise RuntimeError("mta_oracle_stages_composed failed (%d)" % rc)
+    return {"C": C, "P": P, "A1": A1, "A": A, "O": O, "out": out}

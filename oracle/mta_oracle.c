@@ -29,6 +29,13 @@
  *   [GATE] "Multi-Token Attention -- Paper Graph", "Group Normalization with
  *          Sigmoid Gating": the pages' default scale, one learned scalar g_h
  *          per head, output = GroupNorm(concat) * sigmoid(g_h) on head h.
+ *   [POST] "Multi-Token Attention -- Paper Graph", "Key-Query Convolution",
+ *          the post-softmax variant: Mask_0(Conv2d_theta(Softmax(
+ *          Mask_-inf(A^)))), the same convolution (index ranges of Eq. (4))
+ *          applied to the attention probabilities, future entries zeroed.
+ *   [FULL] same page, "Putting Everything Together: The Full MTA Module":
+ *          the compositions of the two convolutions around the softmax and
+ *          the repeat of the MTA convolution (key-query, then head) after it.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - taps that fall outside [0,T) x [0,T) read zero (zero padding);
@@ -38,6 +45,11 @@
  *   - depth scaling is a caller-supplied scalar multiplying the GN output;
  *   - the sigmoid gate multiplies the GN output (after its affine) in place
  *     of the depth scale.
+ *   - a composition runs the steps in one fixed order, each bracketed step
+ *     optional: Mask_0 -> [key-query conv] -> Mask_-inf -> softmax ->
+ *     [head mix] -> [key-query conv -> Mask_0] -> [head mix] -> A V -> GN;
+ *     the pages' default has the first two, the repeat all four, and "both
+ *     post-softmax" the last two; both key-query kernels are c_q x c_k.
  *
  * Layouts: q, k, v are [B][H][T][d]; w_kq is [H][c_q][c_k] with the tap
  * (i', j') at [h][i'][j' + floor(c_k/2)]; w_head is [H/c_h][c_h][c_h];
@@ -56,7 +68,12 @@ typedef struct {
 } mta_oracle_shape;
 
 typedef struct {
-    const double *q, *k, *v, *w_kq, *w_head, *gn_weight, *gn_bias;
+    const double *q, *k, *v;
+    const double *w_kq;        /* key-query kernel before the softmax, or NULL */
+    const double *w_head;      /* head mix right after the softmax, or NULL */
+    const double *w_kq_post;   /* key-query kernel on the probabilities, or NULL */
+    const double *w_head_post; /* head mix after w_kq_post, or NULL */
+    const double *gn_weight, *gn_bias;
     double depth_scale;
     const double *gate;   /* [H] gate logits g_h, or NULL for the depth scale */
 } mta_oracle_args;
@@ -95,18 +112,18 @@ static void masked0_logit_row(const mta_oracle_shape *s, const mta_oracle_args *
     }
 }
 
-/* [KQ4]/[KQ5]: C[i][j] = sum_{i'} sum_{j'} theta[i'][j'] A0[i-i'][j-j'] for
- * j in [0, i]; then the second mask of [KQ5] sets C[i][j] = -inf for j > i.
- * rows[i'] holds the masked logit row A0[i - i'][*]. */
-static void conv_row(const mta_oracle_shape *s, const mta_oracle_args *a, int h,
-                     int i, double *const *rows, double *C)
+/* [KQ4]: out[j] = sum_{i'} sum_{j'} theta[i'][j'] X[i-i'][j-j'] for j in
+ * [0, i], and out[j] = fill for j > i: -inf is the second mask of [KQ5]
+ * (ahead of a softmax), 0 the Mask_0 of [POST] (after one).  rows[i'] holds
+ * the row X[i - i'][*]; X is zero outside [0,T) x [0,T) (zero padding). */
+static void conv2d_row(const mta_oracle_shape *s, const double *theta, int i,
+                       double *const *rows, double fill, double *out)
 {
     const int T = s->T, c_q = s->c_q, c_k = s->c_k;
     const int jlo = -(c_k / 2);               /* -floor(c_k/2)    */
     const int jhi = (c_k + 1) / 2 - 1;        /*  ceil(c_k/2) - 1 */
-    const double *theta = a->w_kq + (size_t)h * c_q * c_k;
     for (int j = 0; j < T; ++j) {
-        if (j > i) { C[j] = -INFINITY; continue; }
+        if (j > i) { out[j] = fill; continue; }
         double acc = 0.0;
         for (int ip = 0; ip < c_q; ++ip) {
             if (i - ip < 0) continue;          /* zero row above the sequence */
@@ -116,7 +133,7 @@ static void conv_row(const mta_oracle_shape *s, const mta_oracle_args *a, int h,
                 acc += theta[ip * c_k + (jp - jlo)] * rows[ip][c];
             }
         }
-        C[j] = acc;
+        out[j] = acc;
     }
 }
 
@@ -133,116 +150,205 @@ static void softmax_row(int T, const double *C, double *P)
     for (int j = 0; j < T; ++j) P[j] /= sum;
 }
 
+/* [HM7] over the c_h heads of one group: out[ho][j] = sum_{hi} wg[ho][hi]
+ * in[hi][j], in and out [c_h][T]; wg == NULL means no mixing (a copy). */
+static void head_mix(int c_h, int T, const double *wg, const double *in, double *out)
+{
+    for (int ho = 0; ho < c_h; ++ho)
+        for (int j = 0; j < T; ++j) {
+            if (!wg) { out[(size_t)ho * T + j] = in[(size_t)ho * T + j]; continue; }
+            double acc = 0.0;
+            for (int hi = 0; hi < c_h; ++hi) acc += wg[ho * c_h + hi] * in[(size_t)hi * T + j];
+            out[(size_t)ho * T + j] = acc;
+        }
+}
+
+/* [MHA] O = A V over the keys j <= i of head h (A is zero on later keys),
+ * then [GN] on O with the [GATE] or depth scale into out_row[h*d ..
+ * h*d + d) when out_row != NULL. */
+static void pv_groupnorm_row(const mta_oracle_shape *s, const mta_oracle_args *a, int b,
+                             int h, int i, const double *A, double *O, double *out_row)
+{
+    const int d = s->d;
+    for (int e = 0; e < d; ++e) O[e] = 0.0;
+    for (int j = 0; j <= i; ++j) {
+        const double *vj = row_of(a->v, s, b, h, j);
+        for (int e = 0; e < d; ++e) O[e] += A[j] * vj[e];
+    }
+    if (!out_row) return;
+    /* [GN]: the head's d-vector is one group; biased variance. */
+    double mean = 0.0;
+    for (int e = 0; e < d; ++e) mean += O[e];
+    mean /= d;
+    double var = 0.0;
+    for (int e = 0; e < d; ++e) var += (O[e] - mean) * (O[e] - mean);
+    var /= d;
+    double inv = 1.0 / sqrt(var + s->gn_eps);
+    /* [GATE] sigmoid(g_h), or the depth scale */
+    double scale = a->gate ? 1.0 / (1.0 + exp(-a->gate[h])) : a->depth_scale;
+    for (int e = 0; e < d; ++e) {
+        size_t chn = (size_t)h * d + e;
+        double y = (O[e] - mean) * inv * a->gn_weight[chn] + a->gn_bias[chn];
+        out_row[chn] = scale * y;
+    }
+}
+
 /* Work buffers for one (batch, head group) unit. */
 typedef struct {
-    double *ring;   /* [c_h][c_q][T] masked logit rows, ring over the query index */
+    double *ring0;  /* [c_h][c_q][T] masked logit rows A0, a ring over the query index */
+    double *ring1;  /* [c_h][c_q][T] first-stage attention rows A1, the same ring */
     double *C;      /* [T] */
-    double *P;      /* [c_h][T] pre-mix probabilities of the group's heads */
-    double *A;      /* [T] mixed attention row of one output head */
+    double *P;      /* [c_h][T] softmax rows of the group's heads */
+    double *A1;     /* [c_h][T] first-stage rows (after the first head mix) */
+    double *A2;     /* [c_h][T] after the post-softmax key-query conv */
+    double *A3;     /* [c_h][T] after the second head mix: the rows that meet V */
     double *O;      /* [d] */
+    double *zero;   /* [T] the zero row above the sequence */
+    double **rows0; /* [c_h * c_q] row pointers into ring0 */
+    double **rows1; /* [c_h * c_q] row pointers into ring1 */
 } unit_buffers;
 
 static int alloc_unit(const mta_oracle_shape *s, unit_buffers *u)
 {
-    size_t T = (size_t)s->T;
-    u->ring = (double *)calloc((size_t)s->c_h * s->c_q * T, sizeof(double));
+    size_t T = (size_t)s->T, hq = (size_t)s->c_h * s->c_q, hT = (size_t)s->c_h * T;
+    u->ring0 = (double *)calloc(hq * T, sizeof(double));
+    u->ring1 = (double *)calloc(hq * T, sizeof(double));
     u->C = (double *)malloc(T * sizeof(double));
-    u->P = (double *)malloc((size_t)s->c_h * T * sizeof(double));
-    u->A = (double *)malloc(T * sizeof(double));
+    u->P = (double *)malloc(hT * sizeof(double));
+    u->A1 = (double *)malloc(hT * sizeof(double));
+    u->A2 = (double *)malloc(hT * sizeof(double));
+    u->A3 = (double *)malloc(hT * sizeof(double));
     u->O = (double *)malloc((size_t)s->d * sizeof(double));
-    return u->ring && u->C && u->P && u->A && u->O;
+    u->zero = (double *)calloc(T, sizeof(double));
+    u->rows0 = (double **)malloc(hq * sizeof(double *));
+    u->rows1 = (double **)malloc(hq * sizeof(double *));
+    return u->ring0 && u->ring1 && u->C && u->P && u->A1 && u->A2 && u->A3 && u->O &&
+           u->zero && u->rows0 && u->rows1;
 }
 
 static void free_unit(unit_buffers *u)
 {
-    free(u->ring); free(u->C); free(u->P); free(u->A); free(u->O);
+    free(u->ring0); free(u->ring1); free(u->C); free(u->P); free(u->A1); free(u->A2);
+    free(u->A3); free(u->O); free(u->zero); free(u->rows0); free(u->rows1);
 }
 
-/* Optional per-row intermediates (each [c_h][T] or [c_h][d]); any may be NULL. */
+/* Optional per-row intermediates of one group (each [c_h][T] or [c_h][d]);
+ * any may be NULL. */
 typedef struct {
-    double *C;      /* conv logits after both masks, per head of the group */
-    double *P;      /* pre-mix softmax rows */
-    double *A;      /* post-mix attention rows */
+    double *C;      /* logits that enter the softmax, both masks applied */
+    double *P;      /* softmax rows */
+    double *A1;     /* first-stage rows, after the first head mix */
+    double *A;      /* the attention rows that meet V */
     double *O;      /* pre-normalisation head outputs A^h V^h, [c_h][d] */
 } row_taps;
 
-/* One query row i of one (batch b, group g), given the masked logit rows:
- * rows_per_head[hh * c_q + ip] is A0[i - ip] of head g*c_h + hh.
- * Writes out_row[h*d + e] (the [H*d] output row of (b, i)) for the group's
- * heads when out_row != NULL, and the intermediates asked for in taps. */
-static void group_row(const mta_oracle_shape *s, const mta_oracle_args *a,
-                      int b, int g, int i, unit_buffers *u,
-                      double *const *rows_per_head, double *out_row, row_taps *taps)
+/* Query row r of group g up to the first head mix.  rows0[hh*c_q + ip] is
+ * A0[r - ip] of head g*c_h + hh.  [KQ5] per head: the key-query conv with
+ * w_kq when given (else A0[r] itself), Mask_-inf, softmax; then [HM7] with
+ * w_head when given.  Leaves the group's rows in u->A1. */
+static void first_stage(const mta_oracle_shape *s, const mta_oracle_args *a, int g, int r,
+                        unit_buffers *u, double *const *rows0, row_taps *taps)
 {
-    const int T = s->T, d = s->d, c_h = s->c_h;
-    /* [KQ5] per head: conv, masks, softmax. */
+    const int T = s->T, c_h = s->c_h, c_q = s->c_q, c_k = s->c_k;
     for (int hh = 0; hh < c_h; ++hh) {
         int h = g * c_h + hh;
-        conv_row(s, a, h, i, rows_per_head + (size_t)hh * s->c_q, u->C);
-        if (taps && taps->C) memcpy(taps->C + (size_t)hh * T, u->C, T * sizeof(double));
+        double *const *rows = rows0 + (size_t)hh * c_q;
+        if (a->w_kq)
+            conv2d_row(s, a->w_kq + (size_t)h * c_q * c_k, r, rows, -INFINITY, u->C);
+        else
+            for (int j = 0; j < T; ++j) u->C[j] = (j <= r) ? rows[0][j] : -INFINITY;
         softmax_row(T, u->C, u->P + (size_t)hh * T);
-        if (taps && taps->P) memcpy(taps->P + (size_t)hh * T, u->P + (size_t)hh * T, T * sizeof(double));
+        if (taps && taps->C) memcpy(taps->C + (size_t)hh * T, u->C, T * sizeof(double));
     }
-    /* [HM7] post-softmax head mixing, then A^h V^h of the output head [MHA]. */
-    const double *wg = a->w_head + (size_t)g * c_h * c_h;
+    head_mix(c_h, T, a->w_head ? a->w_head + (size_t)g * c_h * c_h : NULL, u->P, u->A1);
+    if (taps && taps->P) memcpy(taps->P, u->P, (size_t)c_h * T * sizeof(double));
+    if (taps && taps->A1) memcpy(taps->A1, u->A1, (size_t)c_h * T * sizeof(double));
+}
+
+/* Query row i of group g of batch entry b from the first-stage rows on:
+ * rows1[hh*c_q + ip] is A1[i - ip] of head g*c_h + hh.  [POST] per head:
+ * the key-query conv with w_kq_post when given, future keys zero (else
+ * A1[i] itself); [HM7] with w_head_post when given; then per output head
+ * A V and [GN] into out_row (the [H*d] output row of (b, i)) when given. */
+static void second_stage(const mta_oracle_shape *s, const mta_oracle_args *a, int b, int g,
+                         int i, unit_buffers *u, double *const *rows1, double *out_row,
+                         row_taps *taps)
+{
+    const int T = s->T, d = s->d, c_h = s->c_h, c_q = s->c_q, c_k = s->c_k;
+    for (int hh = 0; hh < c_h; ++hh) {
+        int h = g * c_h + hh;
+        double *const *rows = rows1 + (size_t)hh * c_q;
+        if (a->w_kq_post)
+            conv2d_row(s, a->w_kq_post + (size_t)h * c_q * c_k, i, rows, 0.0,
+                       u->A2 + (size_t)hh * T);
+        else
+            memcpy(u->A2 + (size_t)hh * T, rows[0], T * sizeof(double));
+    }
+    head_mix(c_h, T, a->w_head_post ? a->w_head_post + (size_t)g * c_h * c_h : NULL, u->A2,
+             u->A3);
     for (int ho = 0; ho < c_h; ++ho) {
         int h = g * c_h + ho;
-        for (int j = 0; j < T; ++j) {
-            double acc = 0.0;
-            for (int hi = 0; hi < c_h; ++hi) acc += wg[ho * c_h + hi] * u->P[(size_t)hi * T + j];
-            u->A[j] = acc;
-        }
-        if (taps && taps->A) memcpy(taps->A + (size_t)ho * T, u->A, T * sizeof(double));
-        for (int e = 0; e < d; ++e) u->O[e] = 0.0;
-        for (int j = 0; j <= i; ++j) {
-            const double *vj = row_of(a->v, s, b, h, j);
-            for (int e = 0; e < d; ++e) u->O[e] += u->A[j] * vj[e];
-        }
+        pv_groupnorm_row(s, a, b, h, i, u->A3 + (size_t)ho * T, u->O, out_row);
+        if (taps && taps->A) memcpy(taps->A + (size_t)ho * T, u->A3 + (size_t)ho * T, T * sizeof(double));
         if (taps && taps->O) memcpy(taps->O + (size_t)ho * d, u->O, d * sizeof(double));
-        if (!out_row) continue;
-        /* [GN]: the head's d-vector is one group; biased variance. */
-        double mean = 0.0;
-        for (int e = 0; e < d; ++e) mean += u->O[e];
-        mean /= d;
-        double var = 0.0;
-        for (int e = 0; e < d; ++e) var += (u->O[e] - mean) * (u->O[e] - mean);
-        var /= d;
-        double inv = 1.0 / sqrt(var + s->gn_eps);
-        /* [GATE] sigmoid(g_h), or the depth scale */
-        double scale = a->gate ? 1.0 / (1.0 + exp(-a->gate[h])) : a->depth_scale;
-        for (int e = 0; e < d; ++e) {
-            size_t chn = (size_t)h * d + e;
-            double y = (u->O[e] - mean) * inv * a->gn_weight[chn] + a->gn_bias[chn];
-            out_row[chn] = scale * y;
-        }
     }
 }
 
-/* Points rows[hh*c_q + ip] at A0[i - ip] of each head of group g, computing
- * every row afresh into the unit's buffer (rows above the sequence are the
- * zero row). */
-static void fresh_rows(const mta_oracle_shape *s, const mta_oracle_args *a, int b, int g,
-                       int i, unit_buffers *u, const double *zero_row, double **rows)
+/* rows[hh*c_q + ip] = row i - ip of head hh in a [c_h][c_q][T] ring indexed
+ * by the row number modulo c_q, or the zero row above the sequence. */
+static void point_rows(const mta_oracle_shape *s, double *ring, int i, double *zero,
+                       double **rows)
 {
-    for (int hh = 0; hh < s->c_h; ++hh) {
-        double *base = u->ring + (size_t)hh * s->c_q * s->T;
+    for (int hh = 0; hh < s->c_h; ++hh)
         for (int ip = 0; ip < s->c_q; ++ip) {
-            if (i - ip < 0) { rows[(size_t)hh * s->c_q + ip] = (double *)zero_row; continue; }
-            masked0_logit_row(s, a, b, g * s->c_h + hh, i - ip, base + (size_t)ip * s->T);
-            rows[(size_t)hh * s->c_q + ip] = base + (size_t)ip * s->T;
+            int r = i - ip;
+            rows[(size_t)hh * s->c_q + ip] =
+                (r < 0) ? zero : ring + ((size_t)hh * s->c_q + (r % s->c_q)) * s->T;
+        }
+}
+
+/* Query row i of (b, g) from scratch: the first-stage rows A1[i - ip] for
+ * ip < c_q (only ip = 0 without a post-softmax conv), each from freshly
+ * computed masked logit rows; then the second stage.  Taps are those of
+ * row i. */
+static void fresh_row(const mta_oracle_shape *s, const mta_oracle_args *a, int b, int g, int i,
+                      unit_buffers *u, double *out_row, row_taps *taps)
+{
+    const int T = s->T, c_h = s->c_h, c_q = s->c_q;
+    const int needed = a->w_kq_post ? c_q : 1;
+    for (int ip = 0; ip < c_q; ++ip) {
+        const int r = i - ip;
+        for (int hh = 0; hh < c_h; ++hh) u->rows1[(size_t)hh * c_q + ip] = u->zero;
+        if (ip >= needed || r < 0) continue;
+        for (int hh = 0; hh < c_h; ++hh)
+            for (int ip2 = 0; ip2 < c_q; ++ip2) {
+                double *slot = u->ring0 + ((size_t)hh * c_q + ip2) * T;
+                masked0_logit_row(s, a, b, g * c_h + hh, r - ip2, slot);
+                u->rows0[(size_t)hh * c_q + ip2] = slot;
+            }
+        first_stage(s, a, g, r, u, u->rows0, ip == 0 ? taps : NULL);
+        for (int hh = 0; hh < c_h; ++hh) {
+            double *slot = u->ring1 + ((size_t)hh * c_q + ip) * T;
+            memcpy(slot, u->A1 + (size_t)hh * T, T * sizeof(double));
+            u->rows1[(size_t)hh * c_q + ip] = slot;
         }
     }
+    second_stage(s, a, b, g, i, u, u->rows1, out_row, taps);
+}
+
+static int args_ok(const mta_oracle_shape *s, const mta_oracle_args *a)
+{
+    return shape_ok(s) && a->q && a->k && a->v && a->gn_weight && a->gn_bias;
 }
 
 /* Full forward: out[B][T][H*d].  Units (b, g) are independent and spread over
  * threads; inside a unit the query rows run in order, keeping the last c_q
- * masked logit rows of each head in a ring.  Returns 0 on success. */
+ * masked logit rows and first-stage rows of each head in rings.  Returns 0
+ * on success. */
 static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, double *out,
                         int nthreads)
 {
-    if (!shape_ok(s) || !pa->q || !pa->k || !pa->v || !pa->w_kq || !pa->w_head ||
-        !pa->gn_weight || !pa->gn_bias || !out)
-        return -1;
+    if (!args_ok(s, pa) || !out) return -1;
     const mta_oracle_args a = *pa;
     const int G = s->H / s->c_h;
     const int units = s->B * G;
@@ -255,27 +361,23 @@ static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, do
     for (int un = 0; un < units; ++un) {
         int b = un / G, g = un % G;
         unit_buffers u;
-        double **rows = (double **)malloc((size_t)s->c_h * s->c_q * sizeof(double *));
-        double *zero_row = (double *)calloc((size_t)s->T, sizeof(double));
-        if (!alloc_unit(s, &u) || !rows || !zero_row) {
-            failed |= 1; free_unit(&u); free(rows); free(zero_row); continue;
-        }
+        if (!alloc_unit(s, &u)) { failed |= 1; free_unit(&u); continue; }
+        const size_t T = (size_t)s->T;
         for (int i = 0; i < s->T; ++i) {
-            for (int hh = 0; hh < s->c_h; ++hh) {
-                double *base = u.ring + (size_t)hh * s->c_q * s->T;
-                /* the new row i takes the ring slot of row i - c_q */
-                masked0_logit_row(s, &a, b, g * s->c_h + hh, i, base + (size_t)(i % s->c_q) * s->T);
-                for (int ip = 0; ip < s->c_q; ++ip) {
-                    int r = i - ip;
-                    rows[(size_t)hh * s->c_q + ip] =
-                        (r < 0) ? zero_row : base + (size_t)(r % s->c_q) * s->T;
-                }
-            }
-            group_row(s, &a, b, g, i, &u, rows, out + ((size_t)b * s->T + i) * HD, NULL);
+            /* the new rows i take the ring slots of rows i - c_q */
+            const size_t slot = (size_t)(i % s->c_q);
+            for (int hh = 0; hh < s->c_h; ++hh)
+                masked0_logit_row(s, &a, b, g * s->c_h + hh, i,
+                                  u.ring0 + ((size_t)hh * s->c_q + slot) * T);
+            point_rows(s, u.ring0, i, u.zero, u.rows0);
+            first_stage(s, &a, g, i, &u, u.rows0, NULL);
+            for (int hh = 0; hh < s->c_h; ++hh)
+                memcpy(u.ring1 + ((size_t)hh * s->c_q + slot) * T, u.A1 + (size_t)hh * T,
+                       T * sizeof(double));
+            point_rows(s, u.ring1, i, u.zero, u.rows1);
+            second_stage(s, &a, b, g, i, &u, u.rows1, out + ((size_t)b * s->T + i) * HD, NULL);
         }
         free_unit(&u);
-        free(rows);
-        free(zero_row);
     }
     return failed ? -2 : 0;
 }
@@ -286,9 +388,7 @@ static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, do
 static int rows_args(const mta_oracle_shape *s, const mta_oracle_args *pa, int b,
                      const int *rows_idx, int nrows, double *out_rows, int nthreads)
 {
-    if (!shape_ok(s) || !pa->q || !pa->k || !pa->v || !pa->w_kq || !pa->w_head ||
-        !pa->gn_weight || !pa->gn_bias || !out_rows || !rows_idx || b < 0 || b >= s->B ||
-        nrows < 0)
+    if (!args_ok(s, pa) || !out_rows || !rows_idx || b < 0 || b >= s->B || nrows < 0)
         return -1;
     for (int n = 0; n < nrows; ++n)
         if (rows_idx[n] < 0 || rows_idx[n] >= s->T) return -1;
@@ -304,26 +404,58 @@ static int rows_args(const mta_oracle_shape *s, const mta_oracle_args *pa, int b
     for (int t = 0; t < tasks; ++t) {
         int n = t / G, g = t % G;
         unit_buffers u;
-        double **rows = (double **)malloc((size_t)s->c_h * s->c_q * sizeof(double *));
-        double *zero_row = (double *)calloc((size_t)s->T, sizeof(double));
-        if (!alloc_unit(s, &u) || !rows || !zero_row) {
-            failed |= 1; free_unit(&u); free(rows); free(zero_row); continue;
-        }
-        fresh_rows(s, &a, b, g, rows_idx[n], &u, zero_row, rows);
-        group_row(s, &a, b, g, rows_idx[n], &u, rows, out_rows + (size_t)n * HD, NULL);
+        if (!alloc_unit(s, &u)) { failed |= 1; free_unit(&u); continue; }
+        fresh_row(s, &a, b, g, rows_idx[n], &u, out_rows + (size_t)n * HD, NULL);
         free_unit(&u);
-        free(rows);
-        free(zero_row);
     }
     return failed ? -2 : 0;
 }
 
+/* Intermediates of batch entry b (small T), any output may be NULL; each
+ * map is [H][T][T], O is [H][T][d], out is [T][H*d] (see row_taps). */
+static int stages_args(const mta_oracle_shape *s, const mta_oracle_args *pa, int b, double *C,
+                       double *P, double *A1, double *A, double *O, double *out)
+{
+    if (!args_ok(s, pa) || b < 0 || b >= s->B) return -1;
+    const int T = s->T, d = s->d, c_h = s->c_h, H = s->H;
+    const int G = H / c_h;
+    const size_t HD = (size_t)H * d;
+    unit_buffers u;
+    double *tC = (double *)malloc((size_t)c_h * T * sizeof(double));
+    double *tP = (double *)malloc((size_t)c_h * T * sizeof(double));
+    double *tA1 = (double *)malloc((size_t)c_h * T * sizeof(double));
+    double *tA = (double *)malloc((size_t)c_h * T * sizeof(double));
+    double *tO = (double *)malloc((size_t)c_h * d * sizeof(double));
+    int ok = alloc_unit(s, &u) && tC && tP && tA1 && tA && tO;
+    if (ok) {
+        for (int g = 0; g < G; ++g) {
+            for (int i = 0; i < T; ++i) {
+                row_taps taps = {tC, tP, tA1, tA, tO};
+                fresh_row(s, pa, b, g, i, &u, out ? out + (size_t)i * HD : NULL, &taps);
+                for (int hh = 0; hh < c_h; ++hh) {
+                    int h = g * c_h + hh;
+                    size_t off = ((size_t)h * T + i) * T, src = (size_t)hh * T;
+                    if (C) memcpy(C + off, tC + src, T * sizeof(double));
+                    if (P) memcpy(P + off, tP + src, T * sizeof(double));
+                    if (A1) memcpy(A1 + off, tA1 + src, T * sizeof(double));
+                    if (A) memcpy(A + off, tA + src, T * sizeof(double));
+                    if (O) memcpy(O + ((size_t)h * T + i) * d, tO + (size_t)hh * d, d * sizeof(double));
+                }
+            }
+        }
+    }
+    free_unit(&u); free(tC); free(tP); free(tA1); free(tA); free(tO);
+    return ok ? 0 : -2;
+}
+
+/* The pages' default composition ([KQ5] then [HM7]) with the depth scale. */
 int mta_oracle_forward(const mta_oracle_shape *s, const double *q, const double *k,
                        const double *v, const double *w_kq, const double *w_head,
                        const double *gn_weight, const double *gn_bias,
                        double depth_scale, double *out, int nthreads)
 {
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL};
+    if (!w_kq || !w_head) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, depth_scale, NULL};
     return forward_args(s, &a, out, nthreads);
 }
 
@@ -334,8 +466,22 @@ int mta_oracle_forward_gated(const mta_oracle_shape *s, const double *q, const d
                              const double *gn_weight, const double *gn_bias,
                              const double *gate, double *out, int nthreads)
 {
-    if (!gate) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.0, gate};
+    if (!w_kq || !w_head || !gate) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, 0.0, gate};
+    return forward_args(s, &a, out, nthreads);
+}
+
+/* [FULL]: any composition.  Each of w_kq, w_head, w_kq_post, w_head_post
+ * may be NULL (that step is left out); gate may be NULL (depth scale). */
+int mta_oracle_forward_composed(const mta_oracle_shape *s, const double *q, const double *k,
+                                const double *v, const double *w_kq, const double *w_head,
+                                const double *w_kq_post, const double *w_head_post,
+                                const double *gn_weight, const double *gn_bias,
+                                double depth_scale, const double *gate, double *out,
+                                int nthreads)
+{
+    mta_oracle_args a = {q, k, v, w_kq, w_head, w_kq_post, w_head_post,
+                         gn_weight, gn_bias, depth_scale, gate};
     return forward_args(s, &a, out, nthreads);
 }
 
@@ -345,7 +491,8 @@ int mta_oracle_rows(const mta_oracle_shape *s, const double *q, const double *k,
                     double depth_scale, int b, const int *rows_idx, int nrows,
                     double *out_rows, int nthreads)
 {
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL};
+    if (!w_kq || !w_head) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, depth_scale, NULL};
     return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
 }
 
@@ -355,12 +502,25 @@ int mta_oracle_rows_gated(const mta_oracle_shape *s, const double *q, const doub
                           const double *gate, int b, const int *rows_idx, int nrows,
                           double *out_rows, int nthreads)
 {
-    if (!gate) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.0, gate};
+    if (!w_kq || !w_head || !gate) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, 0.0, gate};
     return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
 }
 
-/* Intermediates of one batch entry for small T; any output may be NULL:
+int mta_oracle_rows_composed(const mta_oracle_shape *s, const double *q, const double *k,
+                             const double *v, const double *w_kq, const double *w_head,
+                             const double *w_kq_post, const double *w_head_post,
+                             const double *gn_weight, const double *gn_bias,
+                             double depth_scale, const double *gate, int b,
+                             const int *rows_idx, int nrows, double *out_rows, int nthreads)
+{
+    mta_oracle_args a = {q, k, v, w_kq, w_head, w_kq_post, w_head_post,
+                         gn_weight, gn_bias, depth_scale, gate};
+    return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
+}
+
+/* Intermediates of one batch entry of the default composition for small T;
+ * any output may be NULL:
  *   C   [H][T][T]  conv logits after both masks of [KQ5] (-inf above the diagonal)
  *   P   [H][T][T]  pre-mix softmax probabilities
  *   A   [H][T][T]  post-mix attention [HM7]
@@ -372,40 +532,24 @@ int mta_oracle_stages(const mta_oracle_shape *s, const double *q, const double *
                       double depth_scale, int b, double *C, double *P, double *A,
                       double *O, double *out)
 {
-    if (!shape_ok(s) || !q || !k || !v || !w_kq || !w_head || !gn_weight || !gn_bias ||
-        b < 0 || b >= s->B)
-        return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL};
-    const int T = s->T, d = s->d, c_h = s->c_h, c_q = s->c_q, H = s->H;
-    const int G = H / c_h;
-    const size_t HD = (size_t)H * d;
-    unit_buffers u;
-    double **rows = (double **)malloc((size_t)c_h * c_q * sizeof(double *));
-    double *zero_row = (double *)calloc((size_t)T, sizeof(double));
-    double *tC = (double *)malloc((size_t)c_h * T * sizeof(double));
-    double *tP = (double *)malloc((size_t)c_h * T * sizeof(double));
-    double *tA = (double *)malloc((size_t)c_h * T * sizeof(double));
-    double *tO = (double *)malloc((size_t)c_h * d * sizeof(double));
-    int ok = alloc_unit(s, &u) && rows && zero_row && tC && tP && tA && tO;
-    if (ok) {
-        for (int g = 0; g < G; ++g) {
-            for (int i = 0; i < T; ++i) {
-                fresh_rows(s, &a, b, g, i, &u, zero_row, rows);
-                row_taps taps = {tC, tP, tA, tO};
-                group_row(s, &a, b, g, i, &u, rows, out ? out + (size_t)i * HD : NULL, &taps);
-                for (int hh = 0; hh < c_h; ++hh) {
-                    int h = g * c_h + hh;
-                    size_t off = ((size_t)h * T + i) * T;
-                    if (C) memcpy(C + off, tC + (size_t)hh * T, T * sizeof(double));
-                    if (P) memcpy(P + off, tP + (size_t)hh * T, T * sizeof(double));
-                    if (A) memcpy(A + off, tA + (size_t)hh * T, T * sizeof(double));
-                    if (O) memcpy(O + ((size_t)h * T + i) * d, tO + (size_t)hh * d, d * sizeof(double));
-                }
-            }
-        }
-    }
-    free_unit(&u); free(rows); free(zero_row); free(tC); free(tP); free(tA); free(tO);
-    return ok ? 0 : -2;
+    if (!w_kq || !w_head) return -1;
+    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, depth_scale, NULL};
+    return stages_args(s, &a, b, C, P, NULL, A, O, out);
+}
+
+/* Intermediates of one batch entry of any composition (small T): as
+ * mta_oracle_stages, plus A1 [H][T][T] (the rows after the first head mix);
+ * A is then the attention that meets V. */
+int mta_oracle_stages_composed(const mta_oracle_shape *s, const double *q, const double *k,
+                               const double *v, const double *w_kq, const double *w_head,
+                               const double *w_kq_post, const double *w_head_post,
+                               const double *gn_weight, const double *gn_bias,
+                               double depth_scale, const double *gate, int b, double *C,
+                               double *P, double *A1, double *A, double *O, double *out)
+{
+    mta_oracle_args a = {q, k, v, w_kq, w_head, w_kq_post, w_head_post,
+                         gn_weight, gn_bias, depth_scale, gate};
+    return stages_args(s, &a, b, C, P, A1, A, O, out);
 }
 
 int mta_oracle_max_threads(void)

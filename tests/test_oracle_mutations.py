@@ -7,6 +7,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_composed_pins as cpins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -20,21 +21,35 @@ MUTATIONS = [
      "theta[(c_q - 1 - ip) * c_k + (jp - jlo)]"),
     ("no Mask_0 before the conv", "for (int c = 0; c <= r; ++c) {",
      "for (int c = 0; c < T; ++c) {"),
-    ("Mask_-inf replaced by zero", "if (j > i) { C[j] = -INFINITY; continue; }",
-     "if (j > i) { C[j] = 0.0; continue; }"),
-    ("unbiased variance", "        var /= d;\n        double inv",
-     "        var /= (d - 1);\n        double inv"),
+    ("Mask_-inf replaced by zero", "rows, -INFINITY, u->C);", "rows, 0.0, u->C);"),
+    ("unbiased variance", "    var /= d;\n    double inv", "    var /= (d - 1);\n    double inv"),
     ("eps outside the square root", "1.0 / sqrt(var + s->gn_eps)",
      "1.0 / (sqrt(var) + s->gn_eps)"),
     ("scale 1/d instead of 1/sqrt(d)", "1.0 / sqrt((double)d)", "1.0 / (double)d"),
     ("value of the input head", "const double *vj = row_of(a->v, s, b, h, j);",
-     "const double *vj = row_of(a->v, s, b, g * c_h + (c_h - 1 - ho), j);"),
+     "const double *vj = row_of(a->v, s, b, (h / s->c_h) * s->c_h + (s->c_h - 1 - h % s->c_h), j);"),
     ("even-c_k window mirrored", "const int jlo = -(c_k / 2);",
      "const int jlo = -((c_k - 1) / 2);"),
     ("depth scale dropped", ": a->depth_scale;", ": 1.0;"),
     ("gate sign flipped", "exp(-a->gate[h])", "exp(a->gate[h])"),
     ("gate applied before the affine bias", "out_row[chn] = scale * y;",
      "out_row[chn] = scale * (y - a->gn_bias[chn]) + a->gn_bias[chn];"),
+    # compositions of "Putting Everything Together"
+    ("post-softmax conv keeps future keys", "rows, 0.0,", "rows, 1.0,"),
+    ("second head mix skipped", "a->w_head_post ? a->w_head_post + (size_t)g * c_h * c_h : NULL",
+     "NULL"),
+    ("post-softmax conv fed unmixed rows", "u.A1 + (size_t)hh * T,", "u.P + (size_t)hh * T,"),
+    ("fresh first-stage rows fed unmixed rows", "memcpy(slot, u->A1 + (size_t)hh * T,",
+     "memcpy(slot, u->P + (size_t)hh * T,"),
+    ("fresh first-stage rows from the wrong logits",
+     "masked0_logit_row(s, a, b, g * c_h + hh, r - ip2, slot);",
+     "masked0_logit_row(s, a, b, g * c_h + hh, i - ip2, slot);"),
+    ("no Mask_-inf without a key-query conv", "u->C[j] = (j <= r) ? rows[0][j] : -INFINITY;",
+     "u->C[j] = rows[0][j];"),
+    ("post-softmax conv reads the current row only",
+     "point_rows(s, u.ring1, i, u.zero, u.rows1);",
+     "point_rows(s, u.ring1, i, u.zero, u.rows1);\n"
+     "            for (int z = 0; z < s->c_h * s->c_q; ++z) u.rows1[z] = u.rows1[z - z % s->c_q];"),
 ]
 
 PIN_CHECKS = [
@@ -48,6 +63,11 @@ PIN_CHECKS = [
     pins.test_row_sums_pre_and_post_mix,
     pins.test_groupnorm_statistics_and_depth_scale,
     pins.test_sigmoid_gate_scales_each_head_after_the_affine,
+    lambda: [cpins.test_composition_matches_library_brute_force(s, n)
+             for s in cpins.SHAPES[:2] for n in ("repeat", "post_kq_only", "plain_attention")],
+    lambda: cpins.test_post_conv_single_tap_closed_form(3, 5),
+    cpins.test_plain_composition_is_causal_attention,
+    lambda: [cpins.test_composed_rows_and_forward_agree(n) for n in ("repeat", "both_post")],
 ]
 
 
