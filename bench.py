@@ -15,10 +15,16 @@ through NVML during the timed region.  `e2e` repeats the measurement through
 the public API with pinned host buffers, copies included.  `cpu_baseline`
 times the fp64 oracle on a bounded sample of the same workload on the host.
 
+`--compose NAME` times one composition of "Putting Everything Together: The
+Full MTA Module" (e.g. `repeat`: the MTA convolution repeated after the
+softmax) through mta_forward_composed, with FLOPs counted for the steps it
+has.
+
 `--impl reference` times that oracle (the only reference implementation of
 this method: the pages ship no code) on the host cores instead.
 """
 import argparse
+import ctypes
 import datetime
 import json
 import os
@@ -34,7 +40,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from convolved_logit_attention_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+from convolved_logit_attention_b200.workloads import (COMPOSITIONS, WORKLOADS,  # noqa: E402
+                                                      composed_inputs, make_inputs)
 
 METRIC = "MTA fwd TFLOP/s and tokens/s at T=4096 bf16; % of B200 bf16 tensor peak"
 L2_FLUSH_BYTES = 256 << 20
@@ -59,6 +66,8 @@ def parse_args(argv=None):
     p.add_argument("--gate", action="store_true",
                    help="time mta_forward_gated (sigmoid-gated output, fixed gate values) "
                         "instead of mta_forward")
+    p.add_argument("--compose", choices=sorted(COMPOSITIONS), default=None,
+                   help="time mta_forward_composed on this composition of the module")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -167,12 +176,20 @@ def barrier(world):
         dist.barrier()
 
 
+WEIGHTS = ("w_kq", "w_head", "w_kq_post", "w_head_post")
+
+
 def device_inputs(x, io, device):
     dt = torch.bfloat16 if io == "bf16" else torch.float32
     d = {n: torch.from_numpy(x[n]).to(device).to(dt) for n in ("q", "k", "v")}
-    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
-        d[n] = torch.from_numpy(x[n]).to(device)
+    for n in WEIGHTS + ("gn_weight", "gn_bias"):
+        d[n] = torch.from_numpy(x[n]).to(device) if x.get(n) is not None else None
     return d
+
+
+def step_flops(args, w):
+    return w.composition_flops(COMPOSITIONS[args.compose]) if args.compose \
+        else w.algorithmic_flops()
 
 
 def kernel_units(name, w):
@@ -184,6 +201,7 @@ def kernel_units(name, w):
         "k_logits": ("alu", logits * 2 * w.d, "FLOP"),
         "k_conv": ("alu", logits * 2 * w.c_q * w.c_k, "FLOP"),
         "k_softmax_mix": ("hbm", logits * 8, "B"),            # read C, write A_new (fp32)
+        "k_head_mix": ("hbm", logits * 8, "B"),               # read and write one fp32 map
         "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
         # read k, write the c_q folded-key copies (fp16)
         "k_fold_keys": ("hbm", w.B * w.H * w.T * w.d * 2 * (1 + w.c_q), "B"),
@@ -243,12 +261,21 @@ def roofline(name, w, avg_ms, peaks, peak_src):
 def time_mta(args, w, d, world, device):
     import convolved_logit_attention_b200 as mta
     unfused = args.path == "unfused"
-    shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"], w.gn_eps)
-    nk = mta.mta_kernel_count(shape, unfused)
-    names = [mta.mta_kernel_name(shape, i, unfused) for i in range(nk)]
-    path = "materialised" if (unfused or mta.mta_forward_path(shape) == mta.MTA_PATH_MATERIALISED) \
-        else "fused_tc"
-    ws_bytes = (mta.mta_unfused_workspace_size(shape) if unfused else mta.mta_workspace_size(shape))
+    if args.compose:
+        shape = mta.composed_shape(d["q"], *(d[n] for n in WEIGHTS), gn_eps=w.gn_eps)
+        comp = mta.composition(*(d[n] for n in WEIGHTS))
+        names = mta.mta_composed_kernel_names(shape, comp)
+        nk = len(names)
+        fused = "k_mta_fused" in names
+        ws_bytes = mta.lib().mta_composed_workspace_size(ctypes.byref(shape), ctypes.byref(comp))
+    else:
+        shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"], w.gn_eps)
+        nk = mta.mta_kernel_count(shape, unfused)
+        names = [mta.mta_kernel_name(shape, i, unfused) for i in range(nk)]
+        fused = not unfused and mta.mta_forward_path(shape) == mta.MTA_PATH_FUSED_TC
+        ws_bytes = (mta.mta_unfused_workspace_size(shape) if unfused
+                    else mta.mta_workspace_size(shape))
+    path = "fused_tc" if fused else "materialised"
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
     out = torch.empty((w.B, w.T, w.H * w.d), dtype=d["q"].dtype, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -260,8 +287,17 @@ def time_mta(args, w, d, world, device):
     # mta_forward_gated): events recorded between the kernels would add their
     # own cost to the step.  A separate traced pass afterwards gives each
     # kernel's time for the roofline.
+    def composed(events=None):
+        mta.mta_forward_composed(d["q"], d["k"], d["v"], *(d[n] for n in WEIGHTS),
+                                 gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
+                                 depth_scale=w.depth_scale, gate=gate if args.gate else None,
+                                 out=out, workspace=ws, stream=stream, gn_eps=w.gn_eps,
+                                 events=events)
+
     def step():
-        if args.gate:
+        if args.compose:
+            composed()
+        elif args.gate:
             mta.mta_forward_gated(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
                                   d["gn_bias"], gate, out=out, workspace=ws, stream=stream,
                                   gn_eps=w.gn_eps)
@@ -271,6 +307,9 @@ def time_mta(args, w, d, world, device):
                w.depth_scale, out=out, workspace=ws, stream=stream, gn_eps=w.gn_eps)
 
     def traced_step(events):
+        if args.compose:
+            composed(events)
+            return
         mta.mta_forward_traced(unfused, events, d["q"], d["k"], d["v"], d["w_kq"], d["w_head"],
                                d["gn_weight"], d["gn_bias"], w.depth_scale, out=out,
                                workspace=ws, stream=stream, gn_eps=w.gn_eps)
@@ -302,11 +341,12 @@ def time_mta(args, w, d, world, device):
         traced_step(kern_ev[s])
     torch.cuda.synchronize(device)
     mta.mta_sync_status(stream, device)
-    per_kernel = {}
-    for s in range(n_tr):
-        for i, name in enumerate(names):
-            per_kernel.setdefault(name, 0.0)
-            per_kernel[name] += kern_ev[s][2 * i].elapsed_time(kern_ev[s][2 * i + 1]) / n_tr
+    per_kernel = {}          # average ms per launch (a name may launch twice per step)
+    for i, name in enumerate(names):
+        per_kernel[name] = per_kernel.get(name, 0.0) + sum(
+            kern_ev[s][2 * i].elapsed_time(kern_ev[s][2 * i + 1]) for s in range(n_tr)) / n_tr
+    for name in per_kernel:
+        per_kernel[name] /= names.count(name)
     return {"total_ms": total_ms, "per_kernel_ms": per_kernel, "names": names,
             "launches": nk * args.steps, "clocks": sampler.summary(), "path": path}
 
@@ -321,16 +361,24 @@ def time_e2e(args, w, x, device):
     first input copy of the timed steps to the end of their last output copy."""
     import convolved_logit_attention_b200 as mta
     dt = torch.bfloat16 if w.io == "bf16" else torch.float32
-    names = ("q", "k", "v", "w_kq", "w_head", "gn_weight", "gn_bias")
+    names = tuple(n for n in ("q", "k", "v") + WEIGHTS + ("gn_weight", "gn_bias")
+                  if x.get(n) is not None)
     host = {n: torch.from_numpy(x[n]).to(dt).pin_memory() for n in ("q", "k", "v")}
-    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
+    for n in names[3:]:
         host[n] = torch.from_numpy(x[n]).pin_memory()
     nbuf = 2
     dev = [{n: torch.empty_like(host[n], device=device) for n in names} for _ in range(nbuf)]
     out = [torch.empty((w.B, w.T, w.H * w.d), dtype=dt, device=device) for _ in range(nbuf)]
     out_host = [torch.empty(out[0].shape, dtype=dt).pin_memory() for _ in range(nbuf)]
-    shape = mta.shape_of(dev[0]["q"], dev[0]["w_kq"], dev[0]["w_head"], w.gn_eps)
-    ws = torch.empty(max(mta.mta_workspace_size(shape), 1), dtype=torch.uint8, device=device)
+    if args.compose:
+        wts = [dev[0].get(n) for n in WEIGHTS]
+        shape = mta.composed_shape(dev[0]["q"], *wts, gn_eps=w.gn_eps)
+        ws_bytes = mta.lib().mta_composed_workspace_size(ctypes.byref(shape),
+                                                         ctypes.byref(mta.composition(*wts)))
+    else:
+        shape = mta.shape_of(dev[0]["q"], dev[0]["w_kq"], dev[0]["w_head"], w.gn_eps)
+        ws_bytes = mta.mta_workspace_size(shape)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
     s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out[0].numel() * out[0].element_size()
@@ -354,9 +402,15 @@ def time_e2e(args, w, x, device):
             if st >= nbuf:
                 s_comp.wait_event(drained[st - nbuf])         # output buffer read back
             d = dev[bi]
-            mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
-                            d["gn_bias"], w.depth_scale, out=out[bi], workspace=ws, stream=s_comp,
-                            gn_eps=w.gn_eps)
+            if args.compose:
+                mta.mta_forward_composed(d["q"], d["k"], d["v"], *(d.get(n) for n in WEIGHTS),
+                                         gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
+                                         depth_scale=w.depth_scale, out=out[bi], workspace=ws,
+                                         stream=s_comp, gn_eps=w.gn_eps)
+            else:
+                mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                                d["gn_bias"], w.depth_scale, out=out[bi], workspace=ws,
+                                stream=s_comp, gn_eps=w.gn_eps)
             computed[st] = torch.cuda.Event()
             computed[st].record(s_comp)
             with torch.cuda.stream(s_out):
@@ -377,18 +431,22 @@ def time_e2e(args, w, x, device):
     return t0.elapsed_time(t1), h2d, d2h
 
 
-def oracle_sample(w, x, n_units):
+def oracle_sample(w, x, n_units, flops_per_step):
     """The first n_units (batch, head-group) units of the workload at full T,
-    as separate B=1, H=c_h problems, with their algorithmic FLOPs."""
+    as separate B=1, H=c_h problems (weights a composition leaves out stay
+    None), with their algorithmic FLOPs."""
+    def part(name, sl):
+        return x[name][sl] if x.get(name) is not None else None
     units = []
     for u in range(min(n_units, w.B * w.G)):
         b, g = divmod(u, w.G)
         hs = slice(g * w.c_h, (g + 1) * w.c_h)
         cs = slice(g * w.c_h * w.d, (g + 1) * w.c_h * w.d)
+        gs = slice(g, g + 1)
         units.append((x["q"][b:b + 1, hs], x["k"][b:b + 1, hs], x["v"][b:b + 1, hs],
-                      x["w_kq"][hs], x["w_head"][g:g + 1], x["gn_weight"][cs],
-                      x["gn_bias"][cs]))
-    flops = len(units) * w.algorithmic_flops() // (w.B * w.G)
+                      part("w_kq", hs), part("w_head", gs), part("w_kq_post", hs),
+                      part("w_head_post", gs), x["gn_weight"][cs], x["gn_bias"][cs]))
+    flops = len(units) * flops_per_step // (w.B * w.G)
     return units, flops
 
 
@@ -399,8 +457,11 @@ def run_oracle_units(units, w, nthreads):
     import oracle
 
     def one(u):
-        return oracle.forward(u[0], u[1], u[2], u[3], u[4], u[5], u[6], w.depth_scale,
-                              gn_eps=w.gn_eps, nthreads=1)
+        if u[5] is None and u[6] is None:
+            return oracle.forward(u[0], u[1], u[2], u[3], u[4], u[7], u[8], w.depth_scale,
+                                  gn_eps=w.gn_eps, nthreads=1)
+        return oracle.forward_composed(*u[:7], u[7], u[8], w.depth_scale, gn_eps=w.gn_eps,
+                                       nthreads=1)
 
     t0 = time.perf_counter()
     with cf.ThreadPoolExecutor(max_workers=nthreads) as ex:
@@ -408,10 +469,10 @@ def run_oracle_units(units, w, nthreads):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, x):
+def cpu_baseline(w, x, flops_per_step):
     cores = os.cpu_count() or 1
     n_units = min(cores, w.B * w.G)
-    units, flops = oracle_sample(w, x, n_units)
+    units, flops = oracle_sample(w, x, n_units, flops_per_step)
     secs = run_oracle_units(units, w, n_units)
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": n_units, "kind": "oracle",
             "seconds": secs,
@@ -424,10 +485,10 @@ def reference_arm(args, w, world, rank):
     bounded sample (one unit per host thread, full T) of the workload."""
     if rank != 0:
         return None
-    x = make_inputs(w)
+    x = composed_inputs(w, args.compose) if args.compose else make_inputs(w)
     cores = os.cpu_count() or 1
     n_units = min(cores, w.B * w.G)
-    units, flops = oracle_sample(w, x, n_units)
+    units, flops = oracle_sample(w, x, n_units, step_flops(args, w))
     for _ in range(args.warmup):
         run_oracle_units(units[:1], w, 1)
     total = sum(run_oracle_units(units, w, n_units) for _ in range(args.steps))
@@ -438,7 +499,8 @@ def reference_arm(args, w, world, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, "oracle (host)"),
+            "config": dict(workload_config(w, "oracle (host)"),
+                           composition=args.compose or "default"),
             "tokens_per_s": n_units * w.T * args.steps / total,
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": n_units, "kind": "oracle",
                              "sample": sample},
@@ -459,7 +521,8 @@ def mta_arm(args, w, world, rank, local):
     if rank == 0 or world == 1:
         build.build()
     barrier(world)
-    x = make_inputs(w, seed=w.seed + rank)
+    x = (composed_inputs(w, args.compose, seed=w.seed + rank) if args.compose
+         else make_inputs(w, seed=w.seed + rank))
     d = device_inputs(x, w.io, device)
     peaks, peak_src = load_peaks()
     res = time_mta(args, w, d, world, device)
@@ -468,7 +531,7 @@ def mta_arm(args, w, world, rank, local):
         res = time_mta(args, w, d, world, device)
     total_ms = dist_max(res["total_ms"], world, device)
     per_step_ms = total_ms / args.steps
-    flops = w.algorithmic_flops()
+    flops = step_flops(args, w)
     value = replica_tflops(world, flops, args.steps, total_ms)
     kernels = dict(res["per_kernel_ms"])   # average ms per launch, traced pass
     dom = max(kernels, key=kernels.get)
@@ -479,23 +542,26 @@ def mta_arm(args, w, world, rank, local):
             "dtype": "bf16" if (w.io == "bf16" and res["path"] == "fused_tc") else "f32",
             "data": "synthetic",
             "config": dict(workload_config(w, res["path"]),
-                           output_scale="sigmoid gate" if args.gate else "depth scale"),
+                           output_scale="sigmoid gate" if args.gate else "depth scale",
+                           composition=args.compose or "default"),
             "tokens_per_s": world * w.tokens() * args.steps / (total_ms / 1e3),
             "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
             "peaks": dict(peaks, source=peak_src),
             "roofline": {k: rl[k] for k in ("bound", "achieved", "peak", "unit", "frac",
                                              "traffic")},
             "roofline_detail": rl,
-            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src)) for n in res["names"]],
+            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src),
+                             launches_per_step=res["names"].count(n))
+                        for n in dict.fromkeys(res["names"])],
             "gpu_launches": res["launches"], "clocks": res["clocks"]}
-    if not args.no_e2e and not args.gate:
+    if not args.no_e2e and not args.gate:     # e2e follows --compose when given
         e2e_ms, h2d, d2h = time_e2e(args, w, x, device)
         e2e_ms = dist_max(e2e_ms, world, device)
         line["e2e"] = {"value": world * flops * args.steps / (e2e_ms / 1e3) / 1e12,
                        "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": e2e_ms / args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, x)
+        line["cpu_baseline"] = cpu_baseline(w, x, flops)
     return line if rank == 0 else None
 
 

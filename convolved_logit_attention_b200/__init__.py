@@ -6,8 +6,9 @@ names as the C entry points, plus the seeded synthetic workloads used by the
 tests and the benchmark (``convolved_logit_attention_b200.workloads``).
 """
 from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
-                       MTA_PATH_MATERIALISED, MtaError, MtaShape, lib, make_shape,
-                       mta_debug_attention, mta_forward, mta_forward_gated, mta_forward_path,
+                       MTA_PATH_MATERIALISED, MtaComposition, MtaError, MtaShape, lib,
+                       make_shape, composed_shape, composition, mta_composed_kernel_names,
+                       mta_debug_attention, mta_forward_composed, mta_forward, mta_forward_gated, mta_forward_path,
                        mta_forward_traced,
                        mta_forward_unfused, mta_kernel_count, mta_kernel_name,
                        mta_selftest_wait_timeout,
@@ -15,8 +16,9 @@ from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
                        mta_version, mta_workspace_size, shape_of)
 
 __all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC",
-           "MTA_PATH_MATERIALISED", "MtaError", "MtaShape", "lib", "make_shape",
-           "mta_debug_attention", "mta_forward", "mta_forward_gated", "mta_forward_path",
+           "MTA_PATH_MATERIALISED", "MtaComposition", "MtaError", "MtaShape", "lib",
+           "make_shape", "composed_shape", "composition", "mta_composed_kernel_names",
+           "mta_debug_attention", "mta_forward_composed", "mta_forward", "mta_forward_gated", "mta_forward_path",
            "mta_forward_traced",
            "mta_forward_unfused", "mta_kernel_count", "mta_kernel_name",
            "mta_selftest_wait_timeout",

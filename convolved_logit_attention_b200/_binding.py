@@ -26,7 +26,8 @@ EXPORTS = ("mta_version", "mta_status_string", "mta_forward_path", "mta_workspac
            "mta_unfused_workspace_size", "mta_forward", "mta_forward_unfused",
            "mta_debug_attention", "mta_kernel_count", "mta_kernel_name", "mta_forward_traced",
            "mta_selftest_wait_timeout", "mta_forward_noalloc", "mta_sync_status",
-           "mta_forward_gated")
+           "mta_forward_gated", "mta_composed_workspace_size", "mta_forward_composed",
+           "mta_forward_composed_traced", "mta_composed_kernel_count", "mta_composed_kernel_name")
 
 
 class MtaShape(ctypes.Structure):
@@ -38,6 +39,11 @@ class MtaShape(ctypes.Structure):
         return "MtaShape(B=%d, H=%d, T=%d, d=%d, c_q=%d, c_k=%d, c_h=%d, io=%s, gn_eps=%g)" % (
             self.B, self.H, self.T, self.d, self.c_q, self.c_k, self.c_h,
             "bf16" if self.io == MTA_BF16 else "f32", self.gn_eps)
+
+
+class MtaComposition(ctypes.Structure):
+    _fields_ = [("w_kq", ctypes.c_void_p), ("w_head", ctypes.c_void_p),
+                ("w_kq_post", ctypes.c_void_p), ("w_head_post", ctypes.c_void_p)]
 
 
 class MtaError(RuntimeError):
@@ -85,6 +91,18 @@ def lib():
         L.mta_forward_gated.argtypes = [sp, vp, vp, vp, fp, fp, fp, fp, fp, vp, vp,
                                         ctypes.c_size_t, vp]
         L.mta_forward_gated.restype = ctypes.c_int
+        cp = ctypes.POINTER(MtaComposition)
+        L.mta_composed_workspace_size.argtypes = [sp, cp]
+        L.mta_composed_workspace_size.restype = ctypes.c_size_t
+        comp = [sp, vp, vp, vp, cp, fp, fp, ctypes.c_float, fp, vp, vp, ctypes.c_size_t, vp]
+        L.mta_forward_composed.argtypes, L.mta_forward_composed.restype = comp, ctypes.c_int
+        L.mta_forward_composed_traced.argtypes = comp + [ctypes.POINTER(ctypes.c_void_p),
+                                                         ctypes.c_int]
+        L.mta_forward_composed_traced.restype = ctypes.c_int
+        L.mta_composed_kernel_count.argtypes = [sp, cp]
+        L.mta_composed_kernel_count.restype = ctypes.c_int
+        L.mta_composed_kernel_name.argtypes = [sp, cp, ctypes.c_int]
+        L.mta_composed_kernel_name.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -285,3 +303,83 @@ def mta_sync_status(stream=None, device=None):
     if device is None:
         device = torch.device("cuda", torch.cuda.current_device())
     _check("mta_sync_status", lib().mta_sync_status(_stream_ptr(stream, device)))
+
+
+def composition(w_kq=None, w_head=None, w_kq_post=None, w_head_post=None) -> MtaComposition:
+    """The C struct of a composition; the tensors must outlive its use."""
+    return MtaComposition(*[t.data_ptr() if t is not None else None
+                            for t in (w_kq, w_head, w_kq_post, w_head_post)])
+
+
+def composed_shape(q, w_kq=None, w_head=None, w_kq_post=None, w_head_post=None,
+                   gn_eps=1e-5) -> MtaShape:
+    """Shape of a composition: (c_q, c_k) from the key-query kernels (equal
+    when both are given), c_h from the head mixes (1 when there is none)."""
+    B, H, T, d = q.shape
+    kq = [w for w in (w_kq, w_kq_post) if w is not None]
+    hm = [w for w in (w_head, w_head_post) if w is not None]
+    c_q, c_k = tuple(kq[0].shape[1:]) if kq else (1, 1)
+    c_h = hm[0].shape[-1] if hm else 1
+    for w in kq:
+        if w.dim() != 3 or tuple(w.shape) != (H, c_q, c_k):
+            raise ValueError("key-query kernels must both be [H, c_q, c_k]")
+    for w in hm:
+        if w.dim() != 3 or c_h < 1 or H % c_h or tuple(w.shape) != (H // c_h, c_h, c_h):
+            raise ValueError("head mixes must both be [H/c_h, c_h, c_h]")
+    return make_shape(B, H, T, d, c_q, c_k, c_h, q.dtype, gn_eps)
+
+
+def mta_composed_kernel_names(shape: MtaShape, comp: MtaComposition):
+    n = lib().mta_composed_kernel_count(ctypes.byref(shape), ctypes.byref(comp))
+    return [lib().mta_composed_kernel_name(ctypes.byref(shape), ctypes.byref(comp), i).decode()
+            for i in range(n)]
+
+
+def mta_forward_composed(q, k, v, w_kq=None, w_head=None, w_kq_post=None, w_head_post=None,
+                         gn_weight=None, gn_bias=None, depth_scale=1.0, gate=None, out=None,
+                         workspace=None, stream=None, gn_eps=1e-5, events=None):
+    """Forward of one composition of the module (see mta_composition in
+    include/mta.h): weights left as None are steps left out.  gate (float32
+    [H]) replaces the depth scale by sigmoid(gate[h]).  With events (a list
+    of torch.cuda.Event, two per launch) the traced entry records them
+    around the launches.  Returns out [B, T, H*d]."""
+    ws_ = [w_kq, w_head, w_kq_post, w_head_post]
+    if q.device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    for name, t in (("k", k), ("v", v)):
+        if t.device != q.device or t.dtype != q.dtype or t.shape != q.shape or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous tensor like q" % name)
+    if q.dtype not in (torch.float32, torch.bfloat16) or not q.is_contiguous():
+        raise ValueError("q must be a contiguous float32 or bfloat16 tensor")
+    B, H, T, d = q.shape
+    for t in ws_ + [gn_weight, gn_bias, gate]:
+        if t is not None and (t.device != q.device or t.dtype != torch.float32
+                              or not t.is_contiguous()):
+            raise ValueError("weights must be contiguous float32 tensors on q's device")
+    if gn_weight is None or gn_bias is None or gn_weight.numel() != H * d \
+            or gn_bias.numel() != H * d:
+        raise ValueError("gn_weight and gn_bias must have H*d elements")
+    if gate is not None and gate.shape != (H,):
+        raise ValueError("gate must be [H]")
+    shape = composed_shape(q, *ws_, gn_eps=gn_eps)
+    comp = composition(*ws_)
+    if out is None:
+        out = torch.empty((B, T, H * d), dtype=q.dtype, device=q.device)
+    elif (out.shape != (B, T, H * d) or out.dtype != q.dtype or out.device != q.device
+          or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous [B, T, H*d] tensor like q")
+    need = lib().mta_composed_workspace_size(ctypes.byref(shape), ctypes.byref(comp))
+    ws = _workspace(need, q.device, workspace)
+    args = [ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(comp), _ptr(gn_weight),
+            _ptr(gn_bias), float(depth_scale), _ptr(gate), _ptr(out), _ptr(ws),
+            ws.numel() * ws.element_size(), _stream_ptr(stream, q.device)]
+    if events is None:
+        _check("mta_forward_composed", lib().mta_forward_composed(*args))
+    else:
+        for e in events:
+            if not e.cuda_event:
+                e.record()
+        handles = (ctypes.c_void_p * max(len(events), 1))(*[e.cuda_event for e in events])
+        _check("mta_forward_composed_traced",
+               lib().mta_forward_composed_traced(*args, handles, len(events)))
+    return out

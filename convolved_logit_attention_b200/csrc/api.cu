@@ -137,6 +137,99 @@ mta_status mta_forward_gated(const mta_shape *s, const void *q, const void *k, c
                         workspace, workspace_bytes, stream, nullptr, 0);
 }
 
+namespace {
+
+bool is_default_composition(const mta_composition *c)
+{
+    return c->w_kq && c->w_head && !c->w_kq_post && !c->w_head_post;
+}
+
+mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const void *v,
+                         const mta_composition *c, const float *gn_weight, const float *gn_bias,
+                         float depth_scale, const float *gate, void *out, void *workspace,
+                         size_t workspace_bytes, void *stream, void *const *events, int n_events)
+{
+    if (!c) return MTA_ERR_INVALID_ARG;
+    if (gate && ((uintptr_t)gate & 3u) != 0) return MTA_ERR_ALIGNMENT;
+    if (is_default_composition(c))
+        return forward_impl(0, s, q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias, depth_scale,
+                            gate, out, workspace, workspace_bytes, stream, events, n_events);
+    mta_status rc = check_shape(s);
+    if (rc != MTA_OK) return rc;
+    const void *need[] = {q, k, v, gn_weight, gn_bias, out};
+    for (const void *p : need)
+        if (!p) return MTA_ERR_INVALID_ARG;
+    for (const void *p : need)
+        if (!aligned(p, 16)) return MTA_ERR_ALIGNMENT;
+    const void *opt[] = {c->w_kq, c->w_head, c->w_kq_post, c->w_head_post};
+    for (const void *p : opt)
+        if (p && !aligned(p, 16)) return MTA_ERR_ALIGNMENT;
+    if (n_events < 0 || (n_events > 0 && !events)) return MTA_ERR_INVALID_ARG;
+    rc = check_workspace(workspace, workspace_bytes, mta::unfused_workspace_bytes(*s));
+    if (rc != MTA_OK) return rc;
+    mta::ForwardArgs a{q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias, depth_scale, out, gate,
+                       c->w_kq_post, c->w_head_post};
+    mta::Trace tr;
+    tr.events = events;
+    tr.n = n_events;
+    return mta::launch_unfused(*s, a, workspace, (cudaStream_t)stream, tr);
+}
+
+mta::ForwardArgs chain_args(const mta_composition *c)
+{
+    mta::ForwardArgs a{};
+    a.w_kq = c->w_kq;
+    a.w_head = c->w_head;
+    a.w_kq_post = c->w_kq_post;
+    a.w_head_post = c->w_head_post;
+    return a;
+}
+
+}  // namespace
+
+size_t mta_composed_workspace_size(const mta_shape *s, const mta_composition *c)
+{
+    if (!c || check_shape(s) != MTA_OK) return 0;
+    return is_default_composition(c) ? mta_workspace_size(s) : mta::unfused_workspace_bytes(*s);
+}
+
+mta_status mta_forward_composed(const mta_shape *s, const void *q, const void *k, const void *v,
+                                const mta_composition *c, const float *gn_weight,
+                                const float *gn_bias, float depth_scale, const float *gate,
+                                void *out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return composed_impl(s, q, k, v, c, gn_weight, gn_bias, depth_scale, gate, out, workspace,
+                         workspace_bytes, stream, nullptr, 0);
+}
+
+mta_status mta_forward_composed_traced(const mta_shape *s, const void *q, const void *k,
+                                       const void *v, const mta_composition *c,
+                                       const float *gn_weight, const float *gn_bias,
+                                       float depth_scale, const float *gate, void *out,
+                                       void *workspace, size_t workspace_bytes, void *stream,
+                                       void *const *events, int n_events)
+{
+    return composed_impl(s, q, k, v, c, gn_weight, gn_bias, depth_scale, gate, out, workspace,
+                         workspace_bytes, stream, events, n_events);
+}
+
+int mta_composed_kernel_count(const mta_shape *s, const mta_composition *c)
+{
+    if (!c || check_shape(s) != MTA_OK) return 0;
+    if (is_default_composition(c)) return mta_kernel_count(s, 0);
+    const char *names[mta::kMaxChainKernels];
+    return mta::unfused_chain(chain_args(c), names);
+}
+
+const char *mta_composed_kernel_name(const mta_shape *s, const mta_composition *c, int index)
+{
+    if (!c || check_shape(s) != MTA_OK || index < 0) return nullptr;
+    if (is_default_composition(c)) return mta_kernel_name(s, 0, index);
+    const char *names[mta::kMaxChainKernels];
+    const int n = mta::unfused_chain(chain_args(c), names);
+    return index < n ? names[index] : nullptr;
+}
+
 mta_status mta_forward(const mta_shape *s, const void *q, const void *k, const void *v,
                        const float *w_kq, const float *w_head, const float *gn_weight,
                        const float *gn_bias, float depth_scale, void *out, void *workspace,

@@ -16,6 +16,10 @@ struct ForwardArgs {
     float depth_scale;
     void *out;
     const float *gate = nullptr;   // [H] sigmoid-gate logits; null: depth scale
+    // Steps after the first head mix (materialised path only): a key-query
+    // kernel on the probabilities and a second head mix; null: left out.
+    // On that path w_kq and w_head may be null too (the step is left out).
+    const float *w_kq_post = nullptr, *w_head_post = nullptr;
 };
 
 // Optional CUDA events recorded around the kernel launches of one call.
@@ -38,6 +42,10 @@ inline size_t bh_tt(const mta_shape &s) {
 size_t unfused_workspace_bytes(const mta_shape &s);
 constexpr int kUnfusedKernels = 4;
 extern const char *const kUnfusedKernelNames[kUnfusedKernels];
+// Launch sequence of launch_unfused for the steps a names (at most
+// kMaxChainKernels); fills names[] in launch order and returns the count.
+constexpr int kMaxChainKernels = 6;
+int unfused_chain(const ForwardArgs &a, const char **names);
 mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr);
 mta_status launch_debug_attention(const mta_shape &s, const void *q, const void *k,

@@ -1,13 +1,18 @@
 // Materialised MTA forward: the T x T maps of one call live in the workspace.
 //
-// Four kernels, one per group of steps of "Multi-Token Attention -- Paper
-// Graph", section 3.4, all arithmetic in fp32 on CUDA cores:
+// One kernel per group of steps of "Multi-Token Attention -- Paper Graph",
+// section 3.4, all arithmetic in fp32 on CUDA cores:
 //   k_logits        S1 + S2   A0 = Mask_0(Q K^T / sqrt(d))      -> map0
 //   k_conv          S3 (+S4)  C = Conv2d_theta(A0), Eq. (4)/(5) -> map1
 //   k_softmax_mix   S5 + S6   softmax rows, post-softmax head mix (Eq. (7))
 //                             -> map0 (A0 is dead by then)
 //   k_pv_groupnorm  S7..S9    A_new V, per-head GroupNorm with warp-shuffle
 //                             reductions, depth scale -> out
+// The compositions of "Putting Everything Together: The Full MTA Module"
+// reuse the chain: k_conv with a second kernel on the probabilities (the
+// post-softmax variant of "Key-Query Convolution", its Mask_0 being the
+// j <= i rule below) and k_head_mix, a second head mix without a softmax.
+// Steps a composition leaves out are skipped; the maps alternate.
 // Only entries with key j <= query i are written or read; the maps hold
 // garbage above the diagonal.  This path is the measured stepping stone and
 // the general fallback (fp32 I/O, shapes the fused kernel does not take).
@@ -21,19 +26,26 @@
 namespace mta {
 namespace {
 
-constexpr int kLogitTile = 64;   // k_logits: 64 x 64 output tile
-constexpr int kLogitDk = 32;     // contraction chunk
+constexpr int kLogitTile = 128;  // k_logits: 128 x 128 output tile
+constexpr int kLogitDk = 16;     // contraction chunk
+constexpr int kLogitStride = kLogitTile + 4;
 constexpr int kConvRows = 32;    // k_conv: 32 x 64 output tile
 constexpr int kConvCols = 64;
+constexpr int kConvStride = 100; // k_conv halo row stride (floats), 4 (mod 32)
 constexpr int kMaxCq = 8;
 constexpr int kMaxCk = 15;
-constexpr int kPvRows = 32;      // k_pv_groupnorm: 32 query rows x d
+constexpr int kPvRows = 64;      // k_pv_groupnorm: 64 query rows x d
 constexpr int kPvKeys = 32;
+constexpr int kPvAStride = kPvRows + 4;   // transposed attention chunk: key-major rows
 constexpr int kMaxD = 128;
 
 // S1 + S2: map0[bh][i][j] = (j <= i) ? q_i . k_j * scale : 0 on tiles that
 // touch the causal triangle.  Grid (col tiles, row tiles, B*H), 256 threads,
-// each thread a 4 x 4 block of the 64 x 64 tile.
+// 128 x 128 tiles.  Thread (tx, ty) = (tid % 16, tid / 16) owns rows
+// {ty*4 .. ty*4+3} and {64+ty*4 .. 64+ty*4+3} and the same pattern of
+// columns with tx, so that its operands for one contraction index are four
+// 16-byte shared loads (eight lanes of a warp read 128 contiguous bytes) for
+// 64 FMAs.  Chunks of 16 contraction indices are staged transposed.
 template <typename TIO>
 __global__ void __launch_bounds__(256)
 k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict__ map0,
@@ -43,86 +55,136 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
     if (ct > rt) return;                     // the whole tile lies above the diagonal
     const size_t bh = blockIdx.z;
     const int i0 = rt * kLogitTile, j0 = ct * kLogitTile;
-    __shared__ float qs[kLogitDk][kLogitTile + 1];
-    __shared__ float ks[kLogitDk][kLogitTile + 1];
+    __shared__ __align__(16) float qs[kLogitDk * kLogitStride];
+    __shared__ __align__(16) float ks[kLogitDk * kLogitStride];
     const int tid = threadIdx.x;
     const int tx = tid % 16, ty = tid / 16;
-    float acc[4][4] = {};
+    float acc[8][8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc[u][w] = 0.f;
     const TIO *qb = q + bh * (size_t)T * d;
     const TIO *kb = k + bh * (size_t)T * d;
     for (int e0 = 0; e0 < d; e0 += kLogitDk) {
         for (int idx = tid; idx < kLogitTile * kLogitDk; idx += 256) {
-            int r = idx / kLogitDk, e = idx % kLogitDk;
-            int gi = i0 + r, gj = j0 + r, ge = e0 + e;
-            qs[e][r] = (gi < T && ge < d) ? to_f32(qb[(size_t)gi * d + ge]) : 0.f;
-            ks[e][r] = (gj < T && ge < d) ? to_f32(kb[(size_t)gj * d + ge]) : 0.f;
+            const int r = idx / kLogitDk, e = idx % kLogitDk;
+            const int gi = i0 + r, gj = j0 + r, ge = e0 + e;
+            qs[e * kLogitStride + r] = (gi < T && ge < d) ? to_f32(qb[(size_t)gi * d + ge]) : 0.f;
+            ks[e * kLogitStride + r] = (gj < T && ge < d) ? to_f32(kb[(size_t)gj * d + ge]) : 0.f;
         }
         __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
         for (int e = 0; e < kLogitDk; ++e) {
-            float a[4], b[4];
+            const float *qe = qs + e * kLogitStride, *ke = ks + e * kLogitStride;
+            const float4 a0 = *reinterpret_cast<const float4 *>(qe + ty * 4);
+            const float4 a1 = *reinterpret_cast<const float4 *>(qe + 64 + ty * 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(ke + tx * 4);
+            const float4 b1 = *reinterpret_cast<const float4 *>(ke + 64 + tx * 4);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) { a[u] = qs[e][ty * 4 + u]; b[u] = ks[e][tx * 4 + u]; }
+            for (int u = 0; u < 8; ++u)
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+                for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], bb[w], acc[u][w]);
         }
         __syncthreads();
     }
     float *mb = map0 + bh * (size_t)T * T;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        int i = i0 + ty * 4 + u;
+    for (int u = 0; u < 8; ++u) {
+        const int i = i0 + (u < 4 ? ty * 4 + u : 64 + ty * 4 + u - 4);
         if (i >= T) continue;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            int j = j0 + tx * 4 + w;
-            if (j >= T) continue;
-            mb[(size_t)i * T + j] = (j <= i) ? acc[u][w] * scale : 0.f;
+        for (int half = 0; half < 2; ++half) {
+            const int jb = j0 + half * 64 + tx * 4;
+            float x[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) x[w] = (jb + w <= i) ? acc[u][half * 4 + w] * scale : 0.f;
+            if ((T & 3) == 0) {
+                if (jb < T)
+                    *reinterpret_cast<float4 *>(mb + (size_t)i * T + jb) =
+                        make_float4(x[0], x[1], x[2], x[3]);
+            } else {
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    if (jb + w < T) mb[(size_t)i * T + jb + w] = x[w];
+            }
         }
     }
 }
 
-// S3 (+S4): map1[bh][i][j] = sum_{i',j'} theta[i'][j'] A0[i-i'][j-j'] for
-// j <= i.  The 32 x 64 output tile reads a (32 + c_q - 1) x (64 + c_k - 1)
-// halo of A0 into shared memory; reads outside [0,T) or above the diagonal
-// (c > r) are the zeros of Mask_0 and of the zero padding.
+// S3 (+S4): dst[bh][i][j] = sum_{i',j'} theta[i'][j'] src[i-i'][j-j'] for
+// j <= i (also the post-softmax conv of the probabilities).  The 32 x 64
+// output tile reads a (32 + c_q - 1)-row halo of src into shared memory;
+// reads outside [0,T) or above the diagonal (c > r) are the zeros of Mask_0
+// and of the zero padding.  Thread (warp w, lane l) owns output row l and
+// the 8 columns 8w .. 8w+7: per query tap i' it loads the row segment those
+// columns reach (8 + c_k - 1 values, 16-byte shared loads) into registers and
+// applies the c_k key taps from there, so that shared-memory loads stay far
+// below the FMA count.  The halo rows are kConvStride floats apart, 4 (mod 32)
+// banks, so the 16-byte loads of 8 consecutive rows hit distinct banks.  The
+// taps accumulate in the order i' then j' for every output.
+template <int CK>
 __global__ void __launch_bounds__(256)
-k_conv(const float *__restrict__ map0, float *__restrict__ map1, const float *__restrict__ w_kq,
-       int T, int H, int c_q, int c_k)
+k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__restrict__ w_kq,
+       int T, int H, int c_q)
 {
+    constexpr int NV = (CK + 7 + 3) / 4;          // float4 loads per row segment
+    constexpr int kLoadCols = 7 * 8 + 4 * NV;     // halo columns any thread reads
+    static_assert(kLoadCols <= kConvStride && kLoadCols >= kConvCols + CK - 1, "halo width");
+    constexpr int L = (CK + 1) / 2 - 1;           // keys reached to the left
     const int i0 = blockIdx.y * kConvRows, j0 = blockIdx.x * kConvCols;
-    if (j0 > i0 + kConvRows - 1) return;     // tile entirely above the diagonal
+    if (j0 > i0 + kConvRows - 1) return;          // tile entirely above the diagonal
     const size_t bh = blockIdx.z;
     const int h = (int)(bh % H);
-    __shared__ float tile[kConvRows + kMaxCq - 1][kConvCols + kMaxCk - 1 + 1];
+    __shared__ __align__(16) float tile[(kConvRows + kMaxCq - 1) * kConvStride];
     __shared__ float th[kMaxCq * kMaxCk];
     const int tid = threadIdx.x;
-    const int L = (c_k + 1) / 2 - 1;         // keys reached to the left
-    const int rows = kConvRows + c_q - 1, cols = kConvCols + c_k - 1;
-    const float *mb = map0 + bh * (size_t)T * T;
-    for (int idx = tid; idx < rows * cols; idx += 256) {
-        int rr = idx / cols, cc = idx % cols;
-        int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
-        tile[rr][cc] = (r >= 0 && r < T && c >= 0 && c <= r) ? mb[(size_t)r * T + c] : 0.f;
+    const int rows = kConvRows + c_q - 1;
+    const float *mb = src + bh * (size_t)T * T;
+    const int cc = tid % 128;
+    for (int rr = tid / 128; rr < rows; rr += 2) {
+        if (cc >= kLoadCols) break;
+        const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
+        tile[rr * kConvStride + cc] =
+            (r >= 0 && r < T && c >= 0 && c <= r) ? mb[(size_t)r * T + c] : 0.f;
     }
-    for (int idx = tid; idx < c_q * c_k; idx += 256) th[idx] = w_kq[(size_t)h * c_q * c_k + idx];
+    for (int idx = tid; idx < c_q * CK; idx += 256) th[idx] = w_kq[(size_t)h * c_q * CK + idx];
     __syncthreads();
-    const int col = tid % kConvCols;
-    const int rbase = (tid / kConvCols) * (kConvRows / 4);
-    float *cb = map1 + bh * (size_t)T * T;
-    const int j = j0 + col;
-    for (int ro = rbase; ro < rbase + kConvRows / 4; ++ro) {
-        const int i = i0 + ro;
-        if (i >= T || j >= T || j > i) continue;
-        float acc = 0.f;
-        for (int ip = 0; ip < c_q; ++ip) {
-            const float *trow = &tile[ro + c_q - 1 - ip][col + c_k - 1];
-            const float *trow_th = &th[ip * c_k];
-            for (int jj = 0; jj < c_k; ++jj) acc = fmaf(trow_th[jj], trow[-jj], acc);
+    const int ro = tid % 32;                      // output row within the tile
+    const int c0 = (tid / 32) * 8;                // first of the thread's 8 output columns
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+    for (int ip = 0; ip < c_q; ++ip) {
+        const float4 *seg4 =
+            reinterpret_cast<const float4 *>(&tile[(ro + c_q - 1 - ip) * kConvStride + c0]);
+        float seg[4 * NV];
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            const float4 t = seg4[v];
+            seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
         }
-        cb[(size_t)i * T + j] = acc;
+        const float *tr = &th[ip * CK];
+#pragma unroll
+        for (int jj = 0; jj < CK; ++jj) {
+            const float t = tr[jj];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = fmaf(t, seg[CK - 1 - jj + u], acc[u]);
+        }
+    }
+    const int i = i0 + ro;
+    if (i >= T) return;
+    const int jb = j0 + c0;
+    float *row = dst + bh * (size_t)T * T + (size_t)i * T;
+    if ((T & 3) == 0 && jb + 7 <= i && jb + 7 < T) {
+        reinterpret_cast<float4 *>(row + jb)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        reinterpret_cast<float4 *>(row + jb)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (jb + u < T && jb + u <= i) row[jb + u] = acc[u];
     }
 }
 
@@ -151,7 +213,8 @@ __device__ float block_reduce(float x, float *red) {
 }
 
 // S5 + S6 for one (batch, group, query row i): softmax of each head's conv
-// row over j <= i, then A^h_new = sum_h' w_g[h][h'] P^h'.  mode 0 writes
+// row over j <= i, then A^h_new = sum_h' w_g[h][h'] P^h' (w_head null: the
+// identity, no mixing).  mode 0 writes
 // A_new for j <= i into dst (the forward); mode 1 writes P (pre-mix) and
 // mode 2 writes A_new, both with zeros for i < j < T (the debug view).
 template <int CH>
@@ -165,7 +228,8 @@ k_softmax_mix(const float *__restrict__ map1, float *__restrict__ dst,
     const int b = bg / G, g = bg % G;
     __shared__ float red[8];
     __shared__ float wsm[CH * CH];
-    for (int idx = threadIdx.x; idx < CH * CH; idx += 256) wsm[idx] = w_head[(size_t)g * CH * CH + idx];
+    for (int idx = threadIdx.x; idx < CH * CH; idx += 256)
+        wsm[idx] = w_head ? w_head[(size_t)g * CH * CH + idx] : (idx / CH == idx % CH ? 1.f : 0.f);
     float m[CH], inv_l[CH];
     const float *rowp[CH];
     float *dstp[CH];
@@ -210,11 +274,46 @@ k_softmax_mix(const float *__restrict__ map1, float *__restrict__ dst,
     }
 }
 
-// S7..S9: O = A_new V for 32 query rows of one (b, h) and all d columns,
+// Eq. (7) without a softmax, for one (batch, group, query row i):
+// dst^h[i][j] = sum_h' w_g[h][h'] src^h'[i][j] for j <= i.  The second head
+// mix of a repeated MTA convolution, applied to probabilities that the
+// post-softmax key-query conv has already filtered.
+template <int CH>
+__global__ void __launch_bounds__(256)
+k_head_mix(const float *__restrict__ src, float *__restrict__ dst,
+           const float *__restrict__ w_head, int T, int H)
+{
+    const int i = blockIdx.x;
+    const int bg = blockIdx.y;
+    const int G = H / CH;
+    const int b = bg / G, g = bg % G;
+    __shared__ float wsm[CH * CH];
+    for (int idx = threadIdx.x; idx < CH * CH; idx += 256) wsm[idx] = w_head[(size_t)g * CH * CH + idx];
+    __syncthreads();
+    const size_t bh0 = (size_t)b * H + (size_t)g * CH;
+    for (int j = threadIdx.x; j <= i; j += 256) {
+        float x[CH];
+#pragma unroll
+        for (int hh = 0; hh < CH; ++hh) x[hh] = src[((bh0 + hh) * T + i) * (size_t)T + j];
+#pragma unroll
+        for (int ho = 0; ho < CH; ++ho) {
+            float a = 0.f;
+#pragma unroll
+            for (int hi = 0; hi < CH; ++hi) a = fmaf(wsm[ho * CH + hi], x[hi], a);
+            dst[((bh0 + ho) * T + i) * (size_t)T + j] = a;
+        }
+    }
+}
+
+// S7..S9: O = A_new V for 64 query rows of one (b, h) and all d columns,
 // then per row: mean and biased variance over d (warp-shuffle reductions),
 // out = scale_h * ((O - mean) / sqrt(var + eps) * gamma + beta), with scale_h
 // the depth scale or, with a gate, sigmoid(g_h) ("Group Normalization with
-// Sigmoid Gating").
+// Sigmoid Gating").  Thread (warp w, lane l) accumulates rows 8w .. 8w+7 and
+// columns 4l .. 4l+3.  Each 32-key chunk of the attention rows is stored
+// transposed (key-major), so that the 8 values a thread needs for one key
+// are two 16-byte broadcast loads and its V values one 16-byte load: three
+// shared loads per 32 FMAs.  Keys accumulate in increasing order.
 template <typename TIO>
 __global__ void __launch_bounds__(256)
 k_pv_groupnorm(const float *__restrict__ amap, const TIO *__restrict__ v,
@@ -225,66 +324,78 @@ k_pv_groupnorm(const float *__restrict__ amap, const TIO *__restrict__ v,
     const int i0 = blockIdx.x * kPvRows;
     const size_t bh = blockIdx.y;
     const int b = (int)(bh / H), h = (int)(bh % H);
-    __shared__ float as[kPvRows][kPvKeys + 1];
-    __shared__ float vs[kPvKeys][kMaxD];
-    __shared__ float os[kPvRows][kMaxD + 1];
+    // the key loop's chunks, then (aliased) the finished O rows
+    __shared__ __align__(16) float smem[kPvRows * (kMaxD + 1)];
+    static_assert(kPvKeys * (kPvAStride + kMaxD) <= kPvRows * (kMaxD + 1), "smem carve");
+    float *asT = smem;                             // [kPvKeys][kPvAStride]
+    float *vs = smem + kPvKeys * kPvAStride;       // [kPvKeys][kMaxD]
+    float *os = smem;                              // [kPvRows][kMaxD + 1]
     const int tid = threadIdx.x;
-    const int rg = tid / 32;                 // rows rg*4 .. rg*4+3
-    const int cg = (tid % 32) * 4;           // columns cg .. cg+3
-    float acc[4][4] = {};
+    const int rg = tid / 32;                       // rows rg*8 .. rg*8+7
+    const int cg = (tid % 32) * 4;                 // columns cg .. cg+3
+    float acc[8][4];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = 0.f;
     const float *ab = amap + bh * (size_t)T * T;
     const TIO *vb = v + bh * (size_t)T * d;
-    const int jend = min(T, i0 + kPvRows);   // keys beyond the last row are masked
+    const int jend = min(T, i0 + kPvRows);        // keys beyond the last row are masked
     for (int j0 = 0; j0 < jend; j0 += kPvKeys) {
         for (int idx = tid; idx < kPvRows * kPvKeys; idx += 256) {
-            int r = idx / kPvKeys, c = idx % kPvKeys;
-            int i = i0 + r, j = j0 + c;
-            as[r][c] = (i < T && j <= i) ? ab[(size_t)i * T + j] : 0.f;
+            const int r = idx / kPvKeys, c = idx % kPvKeys;
+            const int i = i0 + r, j = j0 + c;
+            asT[c * kPvAStride + r] = (i < T && j <= i) ? ab[(size_t)i * T + j] : 0.f;
         }
         for (int idx = tid; idx < kPvKeys * d; idx += 256) {
-            int r = idx / d, e = idx % d;
-            int j = j0 + r;
-            vs[r][e] = (j < T) ? to_f32(vb[(size_t)j * d + e]) : 0.f;
+            const int r = idx / d, e = idx % d;
+            const int j = j0 + r;
+            vs[r * kMaxD + e] = (j < T) ? to_f32(vb[(size_t)j * d + e]) : 0.f;
         }
         __syncthreads();
         if (cg < d) {
 #pragma unroll 4
             for (int c = 0; c < kPvKeys; ++c) {
-                float x[4], y[4];
+                const float4 xa = *reinterpret_cast<const float4 *>(&asT[c * kPvAStride + rg * 8]);
+                const float4 xb =
+                    *reinterpret_cast<const float4 *>(&asT[c * kPvAStride + rg * 8 + 4]);
+                const float4 y = *reinterpret_cast<const float4 *>(&vs[c * kMaxD + cg]);
+                const float x[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                const float yy[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-                for (int u = 0; u < 4; ++u) { x[u] = as[rg * 4 + u][c]; y[u] = vs[c][cg + u]; }
+                for (int u = 0; u < 8; ++u)
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(x[u], y[w], acc[u][w]);
+                    for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(x[u], yy[w], acc[u][w]);
             }
         }
         __syncthreads();
     }
+    // every thread has passed the loop's last barrier: os may reuse the chunks
     if (cg < d) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 8; ++u)
 #pragma unroll
-            for (int w = 0; w < 4; ++w) os[rg * 4 + u][cg + w] = acc[u][w];
+            for (int w = 0; w < 4; ++w) os[(rg * 8 + u) * (kMaxD + 1) + cg + w] = acc[u][w];
     }
     __syncthreads();
-    // one warp per row: warp rg owns rows rg*4 .. rg*4+3
+    // one warp per row: warp rg owns rows rg*8 .. rg*8+7
     const int lane = tid % 32;
-    for (int u = 0; u < 4; ++u) {
-        const int r = rg * 4 + u, i = i0 + r;
+    const float scale = gate ? 1.f / (1.f + expf(-gate[h])) : depth_scale;
+    for (int u = 0; u < 8; ++u) {
+        const int r = rg * 8 + u, i = i0 + r;
         if (i >= T) continue;
+        const float *orow = os + r * (kMaxD + 1);
         float s = 0.f;
-        for (int e = lane; e < d; e += 32) s += os[r][e];
+        for (int e = lane; e < d; e += 32) s += orow[e];
         const float mean = warp_sum(s) / d;
         float s2 = 0.f;
-        for (int e = lane; e < d; e += 32) { float t = os[r][e] - mean; s2 += t * t; }
+        for (int e = lane; e < d; e += 32) { float t = orow[e] - mean; s2 += t * t; }
         const float var = warp_sum(s2) / d;
         const float inv = 1.f / sqrtf(var + eps);
-        const float scale = gate ? 1.f / (1.f + expf(-gate[h])) : depth_scale;
         TIO *dst = out + ((size_t)b * T + i) * ((size_t)H * d) + (size_t)h * d;
         for (int e = lane; e < d; e += 32) {
             const size_t ch = (size_t)h * d + e;
-            dst[e] = from_f32<TIO>(scale * ((os[r][e] - mean) * inv * gn_weight[ch] + gn_bias[ch]));
+            dst[e] = from_f32<TIO>(scale * ((orow[e] - mean) * inv * gn_weight[ch] + gn_bias[ch]));
         }
     }
 }
@@ -311,20 +422,71 @@ mta_status softmax_mix(const mta_shape &s, const float *map1, float *dst, const 
     return MTA_OK;
 }
 
+template <int CH>
+void launch_head_mix(const mta_shape &s, const float *src, float *dst, const float *w_head,
+                     cudaStream_t st)
+{
+    dim3 grid(s.T, s.B * (s.H / CH));
+    k_head_mix<CH><<<grid, 256, 0, st>>>(src, dst, w_head, s.T, s.H);
+}
+
+mta_status head_mix(const mta_shape &s, const float *src, float *dst, const float *w_head,
+                    cudaStream_t st)
+{
+    switch (s.c_h) {
+        case 1: launch_head_mix<1>(s, src, dst, w_head, st); break;
+        case 2: launch_head_mix<2>(s, src, dst, w_head, st); break;
+        case 4: launch_head_mix<4>(s, src, dst, w_head, st); break;
+        case 8: launch_head_mix<8>(s, src, dst, w_head, st); break;
+        case 16: launch_head_mix<16>(s, src, dst, w_head, st); break;
+        default: return MTA_ERR_UNSUPPORTED;
+    }
+    return MTA_OK;
+}
+
 template <typename TIO>
-void logits_and_conv(const mta_shape &s, const void *q, const void *k, const float *w_kq,
-                     float *map0, float *map1, cudaStream_t st, const Trace &tr)
+void launch_logits(const mta_shape &s, const void *q, const void *k, float *map0, cudaStream_t st)
 {
     const int nt = (s.T + kLogitTile - 1) / kLogitTile;
     dim3 g1(nt, nt, s.B * s.H);
-    tr.before(0, st);
     k_logits<TIO><<<g1, 256, 0, st>>>((const TIO *)q, (const TIO *)k, map0, s.T, s.d,
                                       1.0f / sqrtf((float)s.d));
-    tr.after(0, st);
+}
+
+void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq,
+                 cudaStream_t st)
+{
     dim3 g2((s.T + kConvCols - 1) / kConvCols, (s.T + kConvRows - 1) / kConvRows, s.B * s.H);
-    tr.before(1, st);
-    k_conv<<<g2, 256, 0, st>>>(map0, map1, w_kq, s.T, s.H, s.c_q, s.c_k);
-    tr.after(1, st);
+    switch (s.c_k) {
+#define MTA_CONV_CASE(n) \
+        case n: k_conv<n><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q); break;
+        MTA_CONV_CASE(1) MTA_CONV_CASE(2) MTA_CONV_CASE(3) MTA_CONV_CASE(4) MTA_CONV_CASE(5)
+        MTA_CONV_CASE(6) MTA_CONV_CASE(7) MTA_CONV_CASE(8) MTA_CONV_CASE(9) MTA_CONV_CASE(10)
+        MTA_CONV_CASE(11) MTA_CONV_CASE(12) MTA_CONV_CASE(13) MTA_CONV_CASE(14) MTA_CONV_CASE(15)
+#undef MTA_CONV_CASE
+        default: break;   // c_k <= 15 is checked before any launch
+    }
+}
+
+void logits(const mta_shape &s, const void *q, const void *k, float *map0, cudaStream_t st)
+{
+    if (s.io == MTA_BF16)
+        launch_logits<__nv_bfloat16>(s, q, k, map0, st);
+    else
+        launch_logits<float>(s, q, k, map0, st);
+}
+
+void pv_groupnorm(const mta_shape &s, const float *amap, const ForwardArgs &a, cudaStream_t st)
+{
+    dim3 g4((s.T + kPvRows - 1) / kPvRows, s.B * s.H);
+    if (s.io == MTA_BF16)
+        k_pv_groupnorm<__nv_bfloat16><<<g4, 256, 0, st>>>(
+            amap, (const __nv_bfloat16 *)a.v, a.gn_weight, a.gn_bias, a.depth_scale, a.gate,
+            s.gn_eps, (__nv_bfloat16 *)a.out, s.T, s.H, s.d);
+    else
+        k_pv_groupnorm<float><<<g4, 256, 0, st>>>(amap, (const float *)a.v, a.gn_weight,
+                                                  a.gn_bias, a.depth_scale, a.gate, s.gn_eps,
+                                                  (float *)a.out, s.T, s.H, s.d);
 }
 
 }  // namespace
@@ -334,30 +496,56 @@ const char *const kUnfusedKernelNames[kUnfusedKernels] = {"k_logits", "k_conv",
 
 size_t unfused_workspace_bytes(const mta_shape &s) { return 2 * bh_tt(s) * sizeof(float); }
 
+int unfused_chain(const ForwardArgs &a, const char **names)
+{
+    int n = 0;
+    names[n++] = "k_logits";
+    if (a.w_kq) names[n++] = "k_conv";
+    names[n++] = "k_softmax_mix";
+    if (a.w_kq_post) names[n++] = "k_conv";
+    if (a.w_head_post) names[n++] = "k_head_mix";
+    names[n++] = "k_pv_groupnorm";
+    return n;
+}
+
+// The launches follow unfused_chain(); each step reads maps[cur] and writes
+// maps[cur ^ 1].  For the default composition that is logits -> map0,
+// conv -> map1, softmax + mix -> map0, PV + GroupNorm from map0.
 mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr)
 {
-    float *map0 = (float *)ws;
-    float *map1 = map0 + bh_tt(s);
-    if (s.io == MTA_BF16)
-        logits_and_conv<__nv_bfloat16>(s, a.q, a.k, a.w_kq, map0, map1, st, tr);
-    else
-        logits_and_conv<float>(s, a.q, a.k, a.w_kq, map0, map1, st, tr);
-    tr.before(2, st);
-    mta_status rc = softmax_mix(s, map1, map0, a.w_head, 0, st);
-    tr.after(2, st);
+    float *maps[2] = {(float *)ws, (float *)ws + bh_tt(s)};
+    int cur = 0, launch = 0;
+    tr.before(launch, st);
+    logits(s, a.q, a.k, maps[0], st);
+    tr.after(launch++, st);
+    if (a.w_kq) {
+        tr.before(launch, st);
+        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq, st);
+        tr.after(launch++, st);
+        cur ^= 1;
+    }
+    tr.before(launch, st);
+    mta_status rc = softmax_mix(s, maps[cur], maps[cur ^ 1], a.w_head, 0, st);
+    tr.after(launch++, st);
     if (rc != MTA_OK) return rc;
-    dim3 g4((s.T + kPvRows - 1) / kPvRows, s.B * s.H);
-    tr.before(3, st);
-    if (s.io == MTA_BF16)
-        k_pv_groupnorm<__nv_bfloat16><<<g4, 256, 0, st>>>(
-            map0, (const __nv_bfloat16 *)a.v, a.gn_weight, a.gn_bias, a.depth_scale, a.gate,
-            s.gn_eps, (__nv_bfloat16 *)a.out, s.T, s.H, s.d);
-    else
-        k_pv_groupnorm<float><<<g4, 256, 0, st>>>(map0, (const float *)a.v, a.gn_weight,
-                                                  a.gn_bias, a.depth_scale, a.gate, s.gn_eps,
-                                                  (float *)a.out, s.T, s.H, s.d);
-    tr.after(3, st);
+    cur ^= 1;
+    if (a.w_kq_post) {
+        tr.before(launch, st);
+        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq_post, st);
+        tr.after(launch++, st);
+        cur ^= 1;
+    }
+    if (a.w_head_post) {
+        tr.before(launch, st);
+        rc = head_mix(s, maps[cur], maps[cur ^ 1], a.w_head_post, st);
+        tr.after(launch++, st);
+        if (rc != MTA_OK) return rc;
+        cur ^= 1;
+    }
+    tr.before(launch, st);
+    pv_groupnorm(s, maps[cur], a, st);
+    tr.after(launch, st);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
@@ -367,11 +555,8 @@ mta_status launch_debug_attention(const mta_shape &s, const void *q, const void 
 {
     float *map0 = (float *)ws;
     float *map1 = map0 + bh_tt(s);
-    const Trace none;
-    if (s.io == MTA_BF16)
-        logits_and_conv<__nv_bfloat16>(s, q, k, w_kq, map0, map1, st, none);
-    else
-        logits_and_conv<float>(s, q, k, w_kq, map0, map1, st, none);
+    logits(s, q, k, map0, st);
+    launch_conv(s, map0, map1, w_kq, st);
     mta_status rc = softmax_mix(s, map1, attn, w_head, stage == 0 ? 1 : 2, st);
     if (rc != MTA_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;

@@ -34,6 +34,10 @@ Recipes:
   longctx_4k      per (b, h) six distinct key positions p ~ U[0, T-1) each
                   paired with a query position t ~ U(p, T); the key at p is
                   replaced by q_t + N(0, 0.1^2).
+  w_kq_post,      the second key-query kernel and head mix of the
+  w_head_post     compositions of "Putting Everything Together: The Full MTA
+                  Module", drawn like w_kq and w_head from their own stream
+                  (seed + 7919), so that the default inputs stay unchanged.
 """
 from dataclasses import dataclass, replace
 
@@ -74,6 +78,27 @@ class Workload:
 
     def tokens(self) -> int:
         return self.B * self.T
+
+    def composition_flops(self, use) -> int:
+        """algorithmic_flops for a composition: use = which of (w_kq,
+        w_head, w_kq_post, w_head_post) it has; every key-query conv costs
+        c_q c_k MACs per live logit and every head mix c_h."""
+        n_kq = int(bool(use[0])) + int(bool(use[2]))
+        n_mix = int(bool(use[1])) + int(bool(use[3]))
+        per_logit = 4 * self.d + 2 * n_kq * self.c_q * self.c_k + 2 * n_mix * self.c_h
+        return self.B * self.H * self.live_logits() * per_logit
+
+
+# Which of (w_kq, w_head, w_kq_post, w_head_post) each composition uses.
+COMPOSITIONS = {
+    "default": (1, 1, 0, 0),            # key-query pre-softmax, head post-softmax
+    "repeat": (1, 1, 1, 1),             # the MTA convolution repeated after the softmax
+    "both_post": (0, 0, 1, 1),          # both convolutions after the softmax
+    "post_kq": (0, 0, 1, 0),            # the post-softmax key-query variant alone
+    "mix_then_post_kq": (0, 1, 1, 0),
+    "pre_and_post_kq": (1, 0, 1, 0),
+    "plain_attention": (0, 0, 0, 0),
+}
 
 
 WORKLOADS = {
@@ -140,6 +165,29 @@ def make_inputs(w: Workload, seed: int = None) -> dict:
     return {"q": q, "k": k, "v": v, "w_kq": w_kq, "w_head": w_head.astype(np.float32),
             "gn_weight": gn_weight, "gn_bias": gn_bias,
             "depth_scale": float(w.depth_scale), "gn_eps": float(w.gn_eps)}
+
+
+def post_weights(w: Workload, seed: int = None) -> dict:
+    """w_kq_post [H,c_q,c_k] and w_head_post [G,c_h,c_h] (float32), drawn
+    like w_kq and w_head: identity plus N(0, 0.05^2)."""
+    rng = np.random.default_rng((w.seed if seed is None else seed) + 7919)
+    w_kq_post = np.float32(0.05) * rng.standard_normal((w.H, w.c_q, w.c_k), dtype=np.float32)
+    w_kq_post[:, 0, w.c_k // 2] += np.float32(1.0)
+    w_head_post = np.eye(w.c_h, dtype=np.float32)[None] + \
+        np.float32(0.05) * rng.standard_normal((w.G, w.c_h, w.c_h), dtype=np.float32)
+    return {"w_kq_post": w_kq_post, "w_head_post": w_head_post.astype(np.float32)}
+
+
+def composed_inputs(w: Workload, composition: str, seed: int = None) -> dict:
+    """make_inputs plus post_weights, with the weights a composition leaves
+    out set to None."""
+    x = make_inputs(w, seed)
+    x.update(post_weights(w, seed))
+    for name, used in zip(("w_kq", "w_head", "w_kq_post", "w_head_post"),
+                          COMPOSITIONS[composition]):
+        if not used:
+            x[name] = None
+    return x
 
 
 def small_variant(w: Workload, **changes) -> Workload:

@@ -209,6 +209,63 @@ MTA_API mta_status mta_forward_noalloc(const mta_shape *shape, const void *q, co
                                        const float *gn_weight, const float *gn_bias,
                                        float depth_scale, void *out, void *stream);
 
+/* One composition of the module ("Multi-Token Attention -- Paper Graph",
+ * "Putting Everything Together: The Full MTA Module").  The steps run in
+ * this fixed order, each bracketed one only when its weights are given:
+ *   S1+S2, [S3 with w_kq], S4, S5, [S6 with w_head],
+ *   [P1: conv of the probabilities with w_kq_post, zero where j > i],
+ *   [P2: Eq. (7) head mix with w_head_post], S7..S9
+ * P1 is the post-softmax variant of "Key-Query Convolution":
+ * A1 -> Mask_0(Conv2d_theta(A1)), with the index ranges and zero padding of
+ * S3.  The pages' default is {w_kq, w_head}; the repeated MTA convolution
+ * ("repeat this operation") is all four; "both post-softmax" is
+ * {w_kq_post, w_head_post}.  Both key-query kernels are [H][c_q][c_k] and
+ * both head mixes [H/c_h][c_h][c_h], laid out as w_kq and w_head above;
+ * pointers are device memory, 16-byte aligned, NULL for a step left out. */
+typedef struct {
+    const float *w_kq;         /* S3 before the softmax, or NULL */
+    const float *w_head;       /* S6 right after the softmax, or NULL */
+    const float *w_kq_post;    /* P1 on the probabilities, or NULL */
+    const float *w_head_post;  /* P2 after P1, or NULL */
+} mta_composition;
+
+/* Bytes of device workspace mta_forward_composed needs (0 on an invalid
+ * shape or a NULL composition): mta_workspace_size() for the default
+ * composition, two fp32 [B][H][T][T] maps for every other one. */
+MTA_API size_t mta_composed_workspace_size(const mta_shape *shape, const mta_composition *comp);
+
+/* The forward of the composition *comp, written to out.  The default
+ * composition takes mta_forward's path (fused where mta_forward_path says
+ * so); every other composition runs on the materialised chain, in fp32, with
+ * P1 as a second conv launch and P2 as a mix-only launch.  gate is NULL for
+ * out = depth_scale * GN(...), or a device array of H floats (4-byte
+ * aligned) for the sigmoid gate of mta_forward_gated, depth_scale then
+ * ignored.  A NULL comp is MTA_ERR_INVALID_ARG; every other argument and the
+ * contract are as for mta_forward. */
+MTA_API mta_status mta_forward_composed(const mta_shape *shape, const void *q, const void *k,
+                                        const void *v, const mta_composition *comp,
+                                        const float *gn_weight, const float *gn_bias,
+                                        float depth_scale, const float *gate, void *out,
+                                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* mta_forward_composed that records events around its launches, as
+ * mta_forward_traced does; the launches are those mta_composed_kernel_name
+ * lists, in order. */
+MTA_API mta_status mta_forward_composed_traced(const mta_shape *shape, const void *q,
+                                               const void *k, const void *v,
+                                               const mta_composition *comp,
+                                               const float *gn_weight, const float *gn_bias,
+                                               float depth_scale, const float *gate, void *out,
+                                               void *workspace, size_t workspace_bytes,
+                                               void *stream, void *const *events, int n_events);
+
+/* Kernel launches of one mta_forward_composed call and the name of launch
+ * `index` (0 / NULL for an invalid shape, a NULL comp or an index out of
+ * range). */
+MTA_API int mta_composed_kernel_count(const mta_shape *shape, const mta_composition *comp);
+MTA_API const char *mta_composed_kernel_name(const mta_shape *shape, const mta_composition *comp,
+                                             int index);
+
 /* Synchronises `stream`, then reports (and clears) the device error flags:
  * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
  * the fused path met a value outside fp16 range, MTA_ERR_CUDA if the

@@ -134,3 +134,61 @@ def test_forward_path_selection(L, kw, path):
 def test_selftest_rejects_bad_budget(L):
     assert L.mta_selftest_wait_timeout(0, None) == -1
     assert L.mta_selftest_wait_timeout(1 << 31, None) == -1
+
+
+def test_composed_launch_sequences_and_workspace(L):
+    # "Putting Everything Together": each composition's launch list on the
+    # materialised chain, and the default one on mta_forward's path.
+    a = 1 << 20
+    C = _binding.MtaComposition
+    s = shape()
+    seqs = {
+        (a, a, a, a): ["k_logits", "k_conv", "k_softmax_mix", "k_conv", "k_head_mix",
+                       "k_pv_groupnorm"],
+        (None, None, a, None): ["k_logits", "k_softmax_mix", "k_conv", "k_pv_groupnorm"],
+        (None, None, a, a): ["k_logits", "k_softmax_mix", "k_conv", "k_head_mix",
+                             "k_pv_groupnorm"],
+        (None, None, None, None): ["k_logits", "k_softmax_mix", "k_pv_groupnorm"],
+        (a, None, a, None): ["k_logits", "k_conv", "k_softmax_mix", "k_conv", "k_pv_groupnorm"],
+    }
+    for ptrs, names in seqs.items():
+        comp = C(*ptrs)
+        assert mta.mta_composed_kernel_names(s, comp) == names
+        assert L.mta_composed_workspace_size(ctypes.byref(s), ctypes.byref(comp)) == \
+            mta.mta_unfused_workspace_size(s)
+    fused = shape(B=2, H=16, T=4096, d=128, c_q=6, c_k=11, c_h=2)
+    default = C(a, a, None, None)
+    assert mta.mta_composed_kernel_names(fused, default) == \
+        [mta.mta_kernel_name(fused, i) for i in range(mta.mta_kernel_count(fused))]
+    assert L.mta_composed_workspace_size(ctypes.byref(fused), ctypes.byref(default)) == \
+        mta.mta_workspace_size(fused)
+    assert L.mta_composed_workspace_size(ctypes.byref(fused), None) == 0
+    assert L.mta_composed_kernel_name(ctypes.byref(s), ctypes.byref(C(a, a, a, a)), 6) is None
+
+
+def test_composed_argument_checks(L):
+    s = shape()
+    a = ctypes.c_void_p(1 << 20)
+    z = ctypes.c_void_p(0)
+    C = _binding.MtaComposition
+    rep = C(1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    need = mta.mta_unfused_workspace_size(s)
+
+    def call(sh, comp, gw=a, gate=z, ws=a, nbytes=need, q=a):
+        return L.mta_forward_composed(ctypes.byref(sh), q, a, a,
+                                      ctypes.byref(comp) if comp is not None else None, gw, a,
+                                      0.8, gate, a, ws, nbytes, None)
+
+    assert call(s, None) == -1
+    assert call(s, rep, gw=z) == -1
+    assert call(s, rep, q=z) == -1
+    assert call(s, C(1 << 20, 1 << 20, (1 << 20) + 8, None)) == -3
+    assert call(s, rep, gate=ctypes.c_void_p((1 << 20) + 2)) == -3
+    assert call(s, rep, nbytes=need - 1) == -4
+    assert call(s, rep, ws=z) == -1
+    assert call(shape(H=3), rep) == -1
+    assert call(shape(c_q=9), rep) == -2
+    # the default composition keeps mta_forward's checks (its workspace size)
+    fused = shape(B=2, H=16, T=4096, d=128, c_q=6, c_k=11, c_h=2)
+    fneed = mta.mta_workspace_size(fused)
+    assert call(fused, C(1 << 20, 1 << 20, None, None), nbytes=fneed - 1) == -4

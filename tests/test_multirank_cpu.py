@@ -70,3 +70,31 @@ def test_reference_arm_under_the_launcher_two_ranks():
     assert len(lines) == 1                      # rank 0 alone prints
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["n_gpus"] == 2
+
+
+def test_reference_arm_times_a_composition():
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny_f32",
+           "--compose", "repeat", "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([l for l in r.stdout.splitlines() if l.startswith("{")][0])
+    assert d["config"]["composition"] == "repeat" and d["value"] > 0
+
+
+def test_oracle_units_are_slices_of_the_composed_forward():
+    # The CPU-baseline sample cuts (batch, head-group) units out of the
+    # workload, post-softmax weights included; each unit's oracle output
+    # is the matching slice of the whole problem's.
+    import oracle
+    from convolved_logit_attention_b200.workloads import COMPOSITIONS, composed_inputs
+    w = WORKLOADS["tiny_f32"]
+    x = composed_inputs(w, "repeat")
+    flops = w.composition_flops(COMPOSITIONS["repeat"])
+    units, f = bench.oracle_sample(w, x, 2, flops)
+    assert f == 2 * flops // (w.B * w.G)
+    full = oracle.forward_composed(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["w_kq_post"],
+                                   x["w_head_post"], x["gn_weight"], x["gn_bias"], w.depth_scale)
+    for g, u in enumerate(units):
+        part = oracle.forward_composed(*u[:7], u[7], u[8], w.depth_scale)
+        cs = slice(g * w.c_h * w.d, (g + 1) * w.c_h * w.d)
+        np.testing.assert_array_equal(part[0], full[0, :, cs])

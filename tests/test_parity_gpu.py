@@ -6,6 +6,8 @@ run on the same rounded inputs.  Small problems are compared element by
 element; full-size workloads (in the launch configuration the benchmark
 times) on sampled rows that the oracle computes one at a time.
 """
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -96,7 +98,8 @@ RAGGED = [
 @pytest.mark.parametrize("shape", RAGGED, ids=[str(s) for s in RAGGED])
 def test_ragged_shapes_elementwise(shape, fn):
     B, H, T, d, c_q, c_k, c_h, io = shape
-    w = Workload("ragged", B, H, T, d, c_q, c_k, c_h, io, seed=hash(shape) % 1000)
+    w = Workload("ragged", B, H, T, d, c_q, c_k, c_h, io,
+                 seed=zlib.crc32(repr(shape).encode()) % 1000)
     x = make_inputs(w)
     ref = oracle_full(x)
     got = run(FNS[fn], to_device(x, io), x)
