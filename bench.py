@@ -534,7 +534,8 @@ def mta_arm(args, w, world, rank, local):
     flops = step_flops(args, w)
     value = replica_tflops(world, flops, args.steps, total_ms)
     kernels = dict(res["per_kernel_ms"])   # average ms per launch, traced pass
-    dom = max(kernels, key=kernels.get)
+    # the dominant kernel by device time per step (a name may launch twice)
+    dom = max(kernels, key=lambda n: kernels[n] * res["names"].count(n))
     rl = roofline(dom, w, kernels[dom], peaks, peak_src)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,

@@ -29,9 +29,9 @@ namespace {
 constexpr int kLogitTile = 128;  // k_logits: 128 x 128 output tile
 constexpr int kLogitDk = 16;     // contraction chunk
 constexpr int kLogitStride = kLogitTile + 4;
-constexpr int kConvRows = 32;    // k_conv: 32 x 64 output tile
-constexpr int kConvCols = 64;
-constexpr int kConvStride = 100; // k_conv halo row stride (floats), 4 (mod 32)
+constexpr int kConvRows = 32;    // k_conv: 32 x 128 output tile
+constexpr int kConvCols = 128;
+constexpr int kConvStride = 164; // k_conv halo row stride (floats), 4 (mod 32)
 constexpr int kMaxCq = 8;
 constexpr int kMaxCk = 15;
 constexpr int kPvRows = 64;      // k_pv_groupnorm: 64 query rows x d
@@ -115,23 +115,26 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
 }
 
 // S3 (+S4): dst[bh][i][j] = sum_{i',j'} theta[i'][j'] src[i-i'][j-j'] for
-// j <= i (also the post-softmax conv of the probabilities).  The 32 x 64
+// j <= i (also the post-softmax conv of the probabilities).  The 32 x 128
 // output tile reads a (32 + c_q - 1)-row halo of src into shared memory;
 // reads outside [0,T) or above the diagonal (c > r) are the zeros of Mask_0
 // and of the zero padding.  Thread (warp w, lane l) owns output row l and
-// the 8 columns 8w .. 8w+7: per query tap i' it loads the row segment those
-// columns reach (8 + c_k - 1 values, 16-byte shared loads) into registers and
-// applies the c_k key taps from there, so that shared-memory loads stay far
-// below the FMA count.  The halo rows are kConvStride floats apart, 4 (mod 32)
-// banks, so the 16-byte loads of 8 consecutive rows hit distinct banks.  The
-// taps accumulate in the order i' then j' for every output.
+// the 16 columns 16w .. 16w+15: per query tap i' it loads the row segment
+// those columns reach (16 + c_k - 1 values) and the tap row theta[i'][*]
+// with 16-byte shared loads into registers and applies the c_k key taps from
+// there (c_k is a template parameter), so that shared loads stay far below
+// the FMA count.  Halo rows are kConvStride floats apart, 4 (mod 32) banks,
+// so the 16-byte loads of 8 consecutive rows hit distinct banks.  The taps
+// accumulate in the order i' then j' for every output.
 template <int CK>
 __global__ void __launch_bounds__(256)
 k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__restrict__ w_kq,
        int T, int H, int c_q)
 {
-    constexpr int NV = (CK + 7 + 3) / 4;          // float4 loads per row segment
-    constexpr int kLoadCols = 7 * 8 + 4 * NV;     // halo columns any thread reads
+    constexpr int NC = kConvCols / 8;             // output columns per thread
+    constexpr int NV = (CK + NC - 1 + 3) / 4;     // float4 loads per row segment
+    constexpr int CKP = (CK + 3) / 4 * 4;         // padded tap row
+    constexpr int kLoadCols = 7 * NC + 4 * NV;    // halo columns any thread reads
     static_assert(kLoadCols <= kConvStride && kLoadCols >= kConvCols + CK - 1, "halo width");
     constexpr int L = (CK + 1) / 2 - 1;           // keys reached to the left
     const int i0 = blockIdx.y * kConvRows, j0 = blockIdx.x * kConvCols;
@@ -139,24 +142,27 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
     const size_t bh = blockIdx.z;
     const int h = (int)(bh % H);
     __shared__ __align__(16) float tile[(kConvRows + kMaxCq - 1) * kConvStride];
-    __shared__ float th[kMaxCq * kMaxCk];
+    static_assert(kMaxCk <= 16, "tap rows are padded to 16 floats");
+    __shared__ __align__(16) float th[kMaxCq * 16];
     const int tid = threadIdx.x;
     const int rows = kConvRows + c_q - 1;
     const float *mb = src + bh * (size_t)T * T;
-    const int cc = tid % 128;
-    for (int rr = tid / 128; rr < rows; rr += 2) {
-        if (cc >= kLoadCols) break;
+    for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
+        const int rr = idx / kLoadCols, cc = idx % kLoadCols;
         const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
         tile[rr * kConvStride + cc] =
             (r >= 0 && r < T && c >= 0 && c <= r) ? mb[(size_t)r * T + c] : 0.f;
     }
-    for (int idx = tid; idx < c_q * CK; idx += 256) th[idx] = w_kq[(size_t)h * c_q * CK + idx];
+    for (int idx = tid; idx < c_q * CKP; idx += 256) {
+        const int ip = idx / CKP, jj = idx % CKP;
+        th[idx] = jj < CK ? w_kq[((size_t)h * c_q + ip) * CK + jj] : 0.f;
+    }
     __syncthreads();
     const int ro = tid % 32;                      // output row within the tile
-    const int c0 = (tid / 32) * 8;                // first of the thread's 8 output columns
-    float acc[8];
+    const int c0 = (tid / 32) * NC;               // first of the thread's output columns
+    float acc[NC];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+    for (int u = 0; u < NC; ++u) acc[u] = 0.f;
     for (int ip = 0; ip < c_q; ++ip) {
         const float4 *seg4 =
             reinterpret_cast<const float4 *>(&tile[(ro + c_q - 1 - ip) * kConvStride + c0]);
@@ -166,25 +172,32 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
             const float4 t = seg4[v];
             seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
         }
-        const float *tr = &th[ip * CK];
+        const float4 *tr4 = reinterpret_cast<const float4 *>(&th[ip * CKP]);
+        float tr[CKP];
 #pragma unroll
-        for (int jj = 0; jj < CK; ++jj) {
-            const float t = tr[jj];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) acc[u] = fmaf(t, seg[CK - 1 - jj + u], acc[u]);
+        for (int v = 0; v < CKP / 4; ++v) {
+            const float4 t = tr4[v];
+            tr[4 * v] = t.x; tr[4 * v + 1] = t.y; tr[4 * v + 2] = t.z; tr[4 * v + 3] = t.w;
         }
+#pragma unroll
+        for (int jj = 0; jj < CK; ++jj)
+#pragma unroll
+            for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[CK - 1 - jj + u], acc[u]);
     }
     const int i = i0 + ro;
     if (i >= T) return;
-    const int jb = j0 + c0;
     float *row = dst + bh * (size_t)T * T + (size_t)i * T;
-    if ((T & 3) == 0 && jb + 7 <= i && jb + 7 < T) {
-        reinterpret_cast<float4 *>(row + jb)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        reinterpret_cast<float4 *>(row + jb)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    } else {
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (jb + u < T && jb + u <= i) row[jb + u] = acc[u];
+    for (int g = 0; g < NC / 4; ++g) {
+        const int jb = j0 + c0 + 4 * g;
+        if ((T & 3) == 0 && jb + 3 <= i && jb < T) {
+            *reinterpret_cast<float4 *>(row + jb) =
+                make_float4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (jb + u < T && jb + u <= i) row[jb + u] = acc[4 * g + u];
+        }
     }
 }
 
@@ -340,17 +353,36 @@ k_pv_groupnorm(const float *__restrict__ amap, const TIO *__restrict__ v,
         for (int w = 0; w < 4; ++w) acc[u][w] = 0.f;
     const float *ab = amap + bh * (size_t)T * T;
     const TIO *vb = v + bh * (size_t)T * d;
+    const bool vec4 = (T & 3) == 0;               // attention rows 16-byte aligned
     const int jend = min(T, i0 + kPvRows);        // keys beyond the last row are masked
     for (int j0 = 0; j0 < jend; j0 += kPvKeys) {
-        for (int idx = tid; idx < kPvRows * kPvKeys; idx += 256) {
-            const int r = idx / kPvKeys, c = idx % kPvKeys;
+        // attention chunk: thread (row r, keys 4q .. 4q+3), transposed into asT
+        for (int idx = tid; idx < kPvRows * (kPvKeys / 4); idx += 256) {
+            const int r = idx / (kPvKeys / 4), c = (idx % (kPvKeys / 4)) * 4;
             const int i = i0 + r, j = j0 + c;
-            asT[c * kPvAStride + r] = (i < T && j <= i) ? ab[(size_t)i * T + j] : 0.f;
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
+            if (i < T) {
+                const float *src = ab + (size_t)i * T + j;
+                if (vec4 && j + 3 <= i) {
+                    const float4 t = *reinterpret_cast<const float4 *>(src);
+                    x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) x[u] = (j + u <= i) ? src[u] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) asT[(c + u) * kPvAStride + r] = x[u];
         }
-        for (int idx = tid; idx < kPvKeys * d; idx += 256) {
-            const int r = idx / d, e = idx % d;
+        // V chunk: thread (key r, columns 4q .. 4q+3); d is a multiple of 8
+        for (int r = tid / 32; r < kPvKeys; r += 8) {
             const int j = j0 + r;
-            vs[r * kMaxD + e] = (j < T) ? to_f32(vb[(size_t)j * d + e]) : 0.f;
+            for (int e = (tid % 32) * 4; e < d; e += 128) {
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
+                if (j < T) load4_f32(vb + (size_t)j * d + e, y);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) vs[r * kMaxD + e + u] = y[u];
+            }
         }
         __syncthreads();
         if (cg < d) {
