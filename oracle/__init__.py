@@ -22,6 +22,12 @@ class _Shape(ctypes.Structure):
                 ("c_h", ctypes.c_int), ("gn_eps", ctypes.c_double)]
 
 
+class _Composition(ctypes.Structure):
+    _fields_ = [("w_kq", ctypes.c_void_p), ("w_head_pre", ctypes.c_void_p),
+                ("w_head", ctypes.c_void_p), ("w_kq_post", ctypes.c_void_p),
+                ("w_head_post", ctypes.c_void_p), ("exact_mask", ctypes.c_int)]
+
+
 _lib = None
 
 
@@ -38,14 +44,13 @@ def _configure(lib):
     lib.mta_oracle_forward_gated.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
     lib.mta_oracle_rows_gated.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ip,
                                           ctypes.c_int, dp, ctypes.c_int]
-    lib.mta_oracle_forward_composed.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
-                                                ctypes.c_double, dp, dp, ctypes.c_int]
-    lib.mta_oracle_rows_composed.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
-                                             ctypes.c_double, dp, ctypes.c_int, ip, ctypes.c_int,
-                                             dp, ctypes.c_int]
-    lib.mta_oracle_stages_composed.argtypes = [sp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
-                                               ctypes.c_double, dp, ctypes.c_int, dp, dp, dp, dp,
-                                               dp, dp]
+    cp = ctypes.POINTER(_Composition)
+    lib.mta_oracle_forward_composed.argtypes = [sp, dp, dp, dp, cp, dp, dp, ctypes.c_double, dp,
+                                                dp, ctypes.c_int]
+    lib.mta_oracle_rows_composed.argtypes = [sp, dp, dp, dp, cp, dp, dp, ctypes.c_double, dp,
+                                             ctypes.c_int, ip, ctypes.c_int, dp, ctypes.c_int]
+    lib.mta_oracle_stages_composed.argtypes = [sp, dp, dp, dp, cp, dp, dp, ctypes.c_double, dp,
+                                               ctypes.c_int, dp, dp, dp, dp, dp, dp]
     lib.mta_oracle_max_threads.argtypes = []
     for f in (lib.mta_oracle_forward, lib.mta_oracle_rows, lib.mta_oracle_stages,
               lib.mta_oracle_forward_gated, lib.mta_oracle_rows_gated,
@@ -173,36 +178,47 @@ def stages(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, b=0, gn_eps=1
     return {"C": C, "P": P, "A": A, "O": O, "out": out}
 
 
-def _composed(q, w_kq, w_head, w_kq_post, w_head_post, gn_eps):
-    """Shape of a composition: (c_q, c_k) from the key-query kernels (both
-    [H, c_q, c_k] when both are given), c_h from the head mixes (1 when
-    there is none)."""
+def _composed(q, ws, exact_mask, gn_eps):
+    """Shape and C struct of a composition.  ws = (w_kq, w_head_pre, w_head,
+    w_kq_post, w_head_post), float64 arrays or None: (c_q, c_k) from the
+    key-query kernels (both [H, c_q, c_k] when both are given), c_h from the
+    head mixes (1 when there is none)."""
     B, H, T, d = q.shape
-    kq = [w for w in (w_kq, w_kq_post) if w is not None]
-    hm = [w for w in (w_head, w_head_post) if w is not None]
+    kq = [w for w in (ws[0], ws[3]) if w is not None]
+    hm = [w for w in (ws[1], ws[2], ws[4]) if w is not None]
     c_q, c_k = kq[0].shape[1:] if kq else (1, 1)
     c_h = hm[0].shape[-1] if hm else 1
     for w in kq:
         assert w.shape == (H, c_q, c_k), w.shape
     for w in hm:
         assert w.shape == (H // c_h, c_h, c_h), w.shape
-    return _shape(B, H, T, d, c_q, c_k, c_h, gn_eps)
+    comp = _Composition(*[None if w is None else w.ctypes.data for w in ws],
+                        int(bool(exact_mask)))
+    return _shape(B, H, T, d, c_q, c_k, c_h, gn_eps), comp
+
+
+def _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post):
+    return [None if w is None else _f64(w)
+            for w in (w_kq, w_head_pre, w_head, w_kq_post, w_head_post)]
 
 
 def forward_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
-                     depth_scale, gn_eps=1e-5, nthreads=0, gate=None):
+                     depth_scale, gn_eps=1e-5, nthreads=0, gate=None, w_head_pre=None,
+                     exact_mask=False):
     """out[B, T, H*d] of a composition of "Putting Everything Together": the
-    steps Mask_0, [key-query conv w_kq], Mask_-inf, softmax, [head mix
-    w_head], [key-query conv w_kq_post on the probabilities, Mask_0],
-    [head mix w_head_post], A V, GroupNorm, scale; a bracketed step whose
-    weights are None is left out.  gate as in forward."""
+    steps Mask_0, [key-query conv w_kq], [head mix of the logits
+    w_head_pre], Mask_-inf, softmax, [head mix w_head], [key-query conv
+    w_kq_post on the probabilities, Mask_0], [head mix w_head_post], A V,
+    GroupNorm, scale; a bracketed step whose weights are None is left out.
+    exact_mask: the w_kq conv uses Eq. (4)'s indicator instead of Mask_0.
+    gate as in forward."""
     q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
-    ws = [None if w is None else _f64(w) for w in (w_kq, w_head, w_kq_post, w_head_post)]
-    s = _composed(q, *ws, gn_eps)
+    ws = _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post)
+    s, comp = _composed(q, ws, exact_mask, gn_eps)
     g = None if gate is None else _f64(gate)
     out = np.empty((s.B, s.T, s.H * s.d), dtype=np.float64)
     rc = _load().mta_oracle_forward_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
-                                             *map(_ptr, ws), _ptr(gw), _ptr(gb),
+                                             ctypes.byref(comp), _ptr(gw), _ptr(gb),
                                              float(depth_scale), _ptr(g), _ptr(out),
                                              int(nthreads))
     if rc != 0:
@@ -211,16 +227,17 @@ def forward_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, g
 
 
 def rows_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
-                  depth_scale, b, row_idx, gn_eps=1e-5, nthreads=0, gate=None):
+                  depth_scale, b, row_idx, gn_eps=1e-5, nthreads=0, gate=None,
+                  w_head_pre=None, exact_mask=False):
     """out[b, row_idx, :] of forward_composed, one row at a time."""
     q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
-    ws = [None if w is None else _f64(w) for w in (w_kq, w_head, w_kq_post, w_head_post)]
-    s = _composed(q, *ws, gn_eps)
+    ws = _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post)
+    s, comp = _composed(q, ws, exact_mask, gn_eps)
     g = None if gate is None else _f64(gate)
     idx = np.ascontiguousarray(np.asarray(row_idx, dtype=np.int32))
     out = np.empty((idx.size, s.H * s.d), dtype=np.float64)
     rc = _load().mta_oracle_rows_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
-                                          *map(_ptr, ws), _ptr(gw), _ptr(gb),
+                                          ctypes.byref(comp), _ptr(gw), _ptr(gb),
                                           float(depth_scale), _ptr(g), int(b),
                                           idx.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
                                           int(idx.size), _ptr(out), int(nthreads))
@@ -230,20 +247,21 @@ def rows_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_b
 
 
 def stages_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
-                    depth_scale, b=0, gn_eps=1e-5, gate=None):
+                    depth_scale, b=0, gn_eps=1e-5, gate=None, w_head_pre=None,
+                    exact_mask=False):
     """Intermediates of forward_composed for batch entry b (small T only):
-    C [H,T,T] softmax input after both masks, P [H,T,T] softmax, A1 [H,T,T]
-    after the first head mix, A [H,T,T] the attention that meets V,
-    O [H,T,d] pre-normalisation head outputs, out [T, H*d]."""
+    C [H,T,T] softmax input (after both masks and the logit mix), P [H,T,T]
+    softmax, A1 [H,T,T] after the first head mix, A [H,T,T] the attention
+    that meets V, O [H,T,d] pre-normalisation head outputs, out [T, H*d]."""
     q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
-    ws = [None if w is None else _f64(w) for w in (w_kq, w_head, w_kq_post, w_head_post)]
-    s = _composed(q, *ws, gn_eps)
+    ws = _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post)
+    s, comp = _composed(q, ws, exact_mask, gn_eps)
     g = None if gate is None else _f64(gate)
     H, T, d = s.H, s.T, s.d
     C, P, A1, A = (np.empty((H, T, T)) for _ in range(4))
     O = np.empty((H, T, d)); out = np.empty((T, H * d))
     rc = _load().mta_oracle_stages_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
-                                            *map(_ptr, ws), _ptr(gw), _ptr(gb),
+                                            ctypes.byref(comp), _ptr(gw), _ptr(gb),
                                             float(depth_scale), _ptr(g), int(b), _ptr(C),
                                             _ptr(P), _ptr(A1), _ptr(A), _ptr(O), _ptr(out))
     if rc != 0:

@@ -35,7 +35,15 @@
  *          applied to the attention probabilities, future entries zeroed.
  *   [FULL] same page, "Putting Everything Together: The Full MTA Module":
  *          the compositions of the two convolutions around the softmax and
- *          the repeat of the MTA convolution (key-query, then head) after it.
+ *          the repeat of the MTA convolution (key-query, then head) after it;
+ *          "both pre-softmax" is the key-query conv followed by [HMPRE], the
+ *          separable case of the 3-D convolution over (query, key, head).
+ *   [HMPRE] same page, "Head Mixing Convolution", pre-softmax version: the
+ *          logits of a group's heads are mixed, A^h_new = sum_h' w A^h'.
+ *   [EXACT] same page, Eq. (4): the tap (i', j') of output (i, j) adds
+ *          theta q_{i-i'} k_{j-j'}^T / sqrt(d) whenever key j - j' <= i (the
+ *          indicator 1_{i >= j-j'}), which Eq. (5)'s two-pass masking
+ *          narrows to j - j' <= i - i'.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - taps that fall outside [0,T) x [0,T) read zero (zero padding);
@@ -46,8 +54,10 @@
  *   - the sigmoid gate multiplies the GN output (after its affine) in place
  *     of the depth scale.
  *   - a composition runs the steps in one fixed order, each bracketed step
- *     optional: Mask_0 -> [key-query conv] -> Mask_-inf -> softmax ->
- *     [head mix] -> [key-query conv -> Mask_0] -> [head mix] -> A V -> GN;
+ *     optional: Mask_0 -> [key-query conv] -> [head mix of the logits] ->
+ *     Mask_-inf -> softmax -> [head mix] -> [key-query conv -> Mask_0] ->
+ *     [head mix] -> A V -> GN; with [EXACT] the first conv reads the
+ *     unmasked logits under the indicator instead of Mask_0's zeros;
  *     the pages' default has the first two, the repeat all four, and "both
  *     post-softmax" the last two; both key-query kernels are c_q x c_k.
  *
@@ -70,6 +80,8 @@ typedef struct {
 typedef struct {
     const double *q, *k, *v;
     const double *w_kq;        /* key-query kernel before the softmax, or NULL */
+    const double *w_head_pre;  /* head mix of the logits before the softmax, or NULL */
+    int exact;                 /* [EXACT] masking of the first conv instead of [KQ5] */
     const double *w_head;      /* head mix right after the softmax, or NULL */
     const double *w_kq_post;   /* key-query kernel on the probabilities, or NULL */
     const double *w_head_post; /* head mix after w_kq_post, or NULL */
@@ -95,7 +107,10 @@ static const double *row_of(const double *x, const mta_oracle_shape *s,
 
 /* [MHA] then the first mask of [KQ5]: the scaled logit q_r . k_c / sqrt(d)
  * when key c is not in the future of query r, zero otherwise; rows or
- * columns outside [0,T) are zero padding.  Fills out[0..T). */
+ * columns outside [0,T) are zero padding.  Fills out[0..T).  Under [EXACT]
+ * the row also keeps the logits of the c_q - 1 keys after r, which the taps
+ * of the next queries may use (every later key is left out by the
+ * indicator). */
 static void masked0_logit_row(const mta_oracle_shape *s, const mta_oracle_args *a,
                               int b, int h, int r, double *out)
 {
@@ -104,7 +119,8 @@ static void masked0_logit_row(const mta_oracle_shape *s, const mta_oracle_args *
     for (int c = 0; c < T; ++c) out[c] = 0.0;
     if (r < 0 || r >= T) return;
     const double *qr = row_of(a->q, s, b, h, r);
-    for (int c = 0; c <= r; ++c) {
+    const int last = a->exact ? r + s->c_q - 1 : r;
+    for (int c = 0; c <= last && c < T; ++c) {
         const double *kc = row_of(a->k, s, b, h, c);
         double dot = 0.0;
         for (int e = 0; e < d; ++e) dot += qr[e] * kc[e];
@@ -115,9 +131,10 @@ static void masked0_logit_row(const mta_oracle_shape *s, const mta_oracle_args *
 /* [KQ4]: out[j] = sum_{i'} sum_{j'} theta[i'][j'] X[i-i'][j-j'] for j in
  * [0, i], and out[j] = fill for j > i: -inf is the second mask of [KQ5]
  * (ahead of a softmax), 0 the Mask_0 of [POST] (after one).  rows[i'] holds
- * the row X[i - i'][*]; X is zero outside [0,T) x [0,T) (zero padding). */
+ * the row X[i - i'][*]; X is zero outside [0,T) x [0,T) (zero padding).
+ * With exact != 0 a tap reading key c > i is left out ([EXACT]). */
 static void conv2d_row(const mta_oracle_shape *s, const double *theta, int i,
-                       double *const *rows, double fill, double *out)
+                       double *const *rows, int exact, double fill, double *out)
 {
     const int T = s->T, c_q = s->c_q, c_k = s->c_k;
     const int jlo = -(c_k / 2);               /* -floor(c_k/2)    */
@@ -130,6 +147,7 @@ static void conv2d_row(const mta_oracle_shape *s, const double *theta, int i,
             for (int jp = jlo; jp <= jhi; ++jp) {
                 int c = j - jp;
                 if (c < 0 || c >= T) continue; /* zero padding */
+                if (exact && c > i) continue;  /* the indicator 1_{i >= j - j'} */
                 acc += theta[ip * c_k + (jp - jlo)] * rows[ip][c];
             }
         }
@@ -161,6 +179,22 @@ static void head_mix(int c_h, int T, const double *wg, const double *in, double 
             for (int hi = 0; hi < c_h; ++hi) acc += wg[ho * c_h + hi] * in[(size_t)hi * T + j];
             out[(size_t)ho * T + j] = acc;
         }
+}
+
+/* [HMPRE] on the logits of query row r: out[ho][j] = sum_{hi} wg[ho][hi]
+ * in[hi][j] for the keys j <= r; later keys stay -inf (the second mask of
+ * [KQ5]).  in and out are [c_h][T]. */
+static void logit_mix(int c_h, int T, int r, const double *wg, const double *in, double *out)
+{
+    for (int ho = 0; ho < c_h; ++ho) {
+        const double *wrow = wg + (size_t)ho * c_h;   /* output head ho's weights */
+        for (int j = 0; j < T; ++j) {
+            if (j > r) { out[(size_t)ho * T + j] = -INFINITY; continue; }
+            double acc = 0.0;
+            for (int hi = 0; hi < c_h; ++hi) acc += wrow[hi] * in[(size_t)hi * T + j];
+            out[(size_t)ho * T + j] = acc;
+        }
+    }
 }
 
 /* [MHA] O = A V over the keys j <= i of head h (A is zero on later keys),
@@ -197,7 +231,8 @@ static void pv_groupnorm_row(const mta_oracle_shape *s, const mta_oracle_args *a
 typedef struct {
     double *ring0;  /* [c_h][c_q][T] masked logit rows A0, a ring over the query index */
     double *ring1;  /* [c_h][c_q][T] first-stage attention rows A1, the same ring */
-    double *C;      /* [T] */
+    double *C;      /* [c_h][T] softmax inputs before the logit mix */
+    double *Cm;     /* [c_h][T] after the logit mix [HMPRE] */
     double *P;      /* [c_h][T] softmax rows of the group's heads */
     double *A1;     /* [c_h][T] first-stage rows (after the first head mix) */
     double *A2;     /* [c_h][T] after the post-softmax key-query conv */
@@ -213,7 +248,8 @@ static int alloc_unit(const mta_oracle_shape *s, unit_buffers *u)
     size_t T = (size_t)s->T, hq = (size_t)s->c_h * s->c_q, hT = (size_t)s->c_h * T;
     u->ring0 = (double *)calloc(hq * T, sizeof(double));
     u->ring1 = (double *)calloc(hq * T, sizeof(double));
-    u->C = (double *)malloc(T * sizeof(double));
+    u->C = (double *)malloc(hT * sizeof(double));
+    u->Cm = (double *)malloc(hT * sizeof(double));
     u->P = (double *)malloc(hT * sizeof(double));
     u->A1 = (double *)malloc(hT * sizeof(double));
     u->A2 = (double *)malloc(hT * sizeof(double));
@@ -222,13 +258,13 @@ static int alloc_unit(const mta_oracle_shape *s, unit_buffers *u)
     u->zero = (double *)calloc(T, sizeof(double));
     u->rows0 = (double **)malloc(hq * sizeof(double *));
     u->rows1 = (double **)malloc(hq * sizeof(double *));
-    return u->ring0 && u->ring1 && u->C && u->P && u->A1 && u->A2 && u->A3 && u->O &&
+    return u->ring0 && u->ring1 && u->C && u->Cm && u->P && u->A1 && u->A2 && u->A3 && u->O &&
            u->zero && u->rows0 && u->rows1;
 }
 
 static void free_unit(unit_buffers *u)
 {
-    free(u->ring0); free(u->ring1); free(u->C); free(u->P); free(u->A1); free(u->A2);
+    free(u->ring0); free(u->ring1); free(u->C); free(u->Cm); free(u->P); free(u->A1); free(u->A2);
     free(u->A3); free(u->O); free(u->zero); free(u->rows0); free(u->rows1);
 }
 
@@ -244,8 +280,9 @@ typedef struct {
 
 /* Query row r of group g up to the first head mix.  rows0[hh*c_q + ip] is
  * A0[r - ip] of head g*c_h + hh.  [KQ5] per head: the key-query conv with
- * w_kq when given (else A0[r] itself), Mask_-inf, softmax; then [HM7] with
- * w_head when given.  Leaves the group's rows in u->A1. */
+ * w_kq when given (else A0[r] itself) and Mask_-inf; [HMPRE] with
+ * w_head_pre when given; softmax; then [HM7] with w_head when given.
+ * Leaves the group's rows in u->A1. */
 static void first_stage(const mta_oracle_shape *s, const mta_oracle_args *a, int g, int r,
                         unit_buffers *u, double *const *rows0, row_taps *taps)
 {
@@ -253,13 +290,20 @@ static void first_stage(const mta_oracle_shape *s, const mta_oracle_args *a, int
     for (int hh = 0; hh < c_h; ++hh) {
         int h = g * c_h + hh;
         double *const *rows = rows0 + (size_t)hh * c_q;
+        double *C = u->C + (size_t)hh * T;
         if (a->w_kq)
-            conv2d_row(s, a->w_kq + (size_t)h * c_q * c_k, r, rows, -INFINITY, u->C);
+            conv2d_row(s, a->w_kq + (size_t)h * c_q * c_k, r, rows, a->exact, -INFINITY, C);
         else
-            for (int j = 0; j < T; ++j) u->C[j] = (j <= r) ? rows[0][j] : -INFINITY;
-        softmax_row(T, u->C, u->P + (size_t)hh * T);
-        if (taps && taps->C) memcpy(taps->C + (size_t)hh * T, u->C, T * sizeof(double));
+            for (int j = 0; j < T; ++j) C[j] = (j <= r) ? rows[0][j] : -INFINITY;
     }
+    const double *logits = u->C;
+    if (a->w_head_pre) {
+        logit_mix(c_h, T, r, a->w_head_pre + (size_t)g * c_h * c_h, u->C, u->Cm);
+        logits = u->Cm;
+    }
+    for (int hh = 0; hh < c_h; ++hh)
+        softmax_row(T, logits + (size_t)hh * T, u->P + (size_t)hh * T);
+    if (taps && taps->C) memcpy(taps->C, logits, (size_t)c_h * T * sizeof(double));
     head_mix(c_h, T, a->w_head ? a->w_head + (size_t)g * c_h * c_h : NULL, u->P, u->A1);
     if (taps && taps->P) memcpy(taps->P, u->P, (size_t)c_h * T * sizeof(double));
     if (taps && taps->A1) memcpy(taps->A1, u->A1, (size_t)c_h * T * sizeof(double));
@@ -279,7 +323,7 @@ static void second_stage(const mta_oracle_shape *s, const mta_oracle_args *a, in
         int h = g * c_h + hh;
         double *const *rows = rows1 + (size_t)hh * c_q;
         if (a->w_kq_post)
-            conv2d_row(s, a->w_kq_post + (size_t)h * c_q * c_k, i, rows, 0.0,
+            conv2d_row(s, a->w_kq_post + (size_t)h * c_q * c_k, i, rows, 0, 0.0,
                        u->A2 + (size_t)hh * T);
         else
             memcpy(u->A2 + (size_t)hh * T, rows[0], T * sizeof(double));
@@ -448,14 +492,49 @@ static int stages_args(const mta_oracle_shape *s, const mta_oracle_args *pa, int
     return ok ? 0 : -2;
 }
 
-/* The pages' default composition ([KQ5] then [HM7]) with the depth scale. */
+/* The pages' default composition ([KQ5] then [HM7]). */
+static mta_oracle_args default_args(const double *q, const double *k, const double *v,
+                                    const double *w_kq, const double *w_head,
+                                    const double *gn_weight, const double *gn_bias,
+                                    double depth_scale, const double *gate)
+{
+    mta_oracle_args a = {0};
+    a.q = q; a.k = k; a.v = v; a.w_kq = w_kq; a.w_head = w_head;
+    a.gn_weight = gn_weight; a.gn_bias = gn_bias; a.depth_scale = depth_scale; a.gate = gate;
+    return a;
+}
+
+/* A composition of [FULL]: each weight may be NULL (that step is left out). */
+typedef struct {
+    const double *w_kq;        /* [H][c_q][c_k] key-query conv before the softmax */
+    const double *w_head_pre;  /* [H/c_h][c_h][c_h] [HMPRE] mix of the logits */
+    const double *w_head;      /* [H/c_h][c_h][c_h] [HM7] mix after the softmax */
+    const double *w_kq_post;   /* [H][c_q][c_k] [POST] conv of the probabilities */
+    const double *w_head_post; /* [H/c_h][c_h][c_h] [HM7] mix after w_kq_post */
+    int exact_mask;            /* nonzero: [EXACT] masking of the w_kq conv */
+} mta_oracle_composition;
+
+static mta_oracle_args composed_args(const double *q, const double *k, const double *v,
+                                     const mta_oracle_composition *c,
+                                     const double *gn_weight, const double *gn_bias,
+                                     double depth_scale, const double *gate)
+{
+    mta_oracle_args a = default_args(q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias,
+                                     depth_scale, gate);
+    a.w_head_pre = c->w_head_pre;
+    a.exact = c->exact_mask != 0;
+    a.w_kq_post = c->w_kq_post;
+    a.w_head_post = c->w_head_post;
+    return a;
+}
+
 int mta_oracle_forward(const mta_oracle_shape *s, const double *q, const double *k,
                        const double *v, const double *w_kq, const double *w_head,
                        const double *gn_weight, const double *gn_bias,
                        double depth_scale, double *out, int nthreads)
 {
     if (!w_kq || !w_head) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, depth_scale, NULL};
+    mta_oracle_args a = default_args(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL);
     return forward_args(s, &a, out, nthreads);
 }
 
@@ -467,21 +546,19 @@ int mta_oracle_forward_gated(const mta_oracle_shape *s, const double *q, const d
                              const double *gate, double *out, int nthreads)
 {
     if (!w_kq || !w_head || !gate) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, 0.0, gate};
+    mta_oracle_args a = default_args(q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.0, gate);
     return forward_args(s, &a, out, nthreads);
 }
 
-/* [FULL]: any composition.  Each of w_kq, w_head, w_kq_post, w_head_post
- * may be NULL (that step is left out); gate may be NULL (depth scale). */
+/* [FULL]: the composition *c; gate may be NULL (depth scale). */
 int mta_oracle_forward_composed(const mta_oracle_shape *s, const double *q, const double *k,
-                                const double *v, const double *w_kq, const double *w_head,
-                                const double *w_kq_post, const double *w_head_post,
+                                const double *v, const mta_oracle_composition *c,
                                 const double *gn_weight, const double *gn_bias,
                                 double depth_scale, const double *gate, double *out,
                                 int nthreads)
 {
-    mta_oracle_args a = {q, k, v, w_kq, w_head, w_kq_post, w_head_post,
-                         gn_weight, gn_bias, depth_scale, gate};
+    if (!c) return -1;
+    mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return forward_args(s, &a, out, nthreads);
 }
 
@@ -492,7 +569,7 @@ int mta_oracle_rows(const mta_oracle_shape *s, const double *q, const double *k,
                     double *out_rows, int nthreads)
 {
     if (!w_kq || !w_head) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, depth_scale, NULL};
+    mta_oracle_args a = default_args(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL);
     return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
 }
 
@@ -503,19 +580,18 @@ int mta_oracle_rows_gated(const mta_oracle_shape *s, const double *q, const doub
                           double *out_rows, int nthreads)
 {
     if (!w_kq || !w_head || !gate) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, 0.0, gate};
+    mta_oracle_args a = default_args(q, k, v, w_kq, w_head, gn_weight, gn_bias, 0.0, gate);
     return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
 }
 
 int mta_oracle_rows_composed(const mta_oracle_shape *s, const double *q, const double *k,
-                             const double *v, const double *w_kq, const double *w_head,
-                             const double *w_kq_post, const double *w_head_post,
+                             const double *v, const mta_oracle_composition *c,
                              const double *gn_weight, const double *gn_bias,
                              double depth_scale, const double *gate, int b,
                              const int *rows_idx, int nrows, double *out_rows, int nthreads)
 {
-    mta_oracle_args a = {q, k, v, w_kq, w_head, w_kq_post, w_head_post,
-                         gn_weight, gn_bias, depth_scale, gate};
+    if (!c) return -1;
+    mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
 }
 
@@ -533,22 +609,22 @@ int mta_oracle_stages(const mta_oracle_shape *s, const double *q, const double *
                       double *O, double *out)
 {
     if (!w_kq || !w_head) return -1;
-    mta_oracle_args a = {q, k, v, w_kq, w_head, NULL, NULL, gn_weight, gn_bias, depth_scale, NULL};
+    mta_oracle_args a = default_args(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, NULL);
     return stages_args(s, &a, b, C, P, NULL, A, O, out);
 }
 
 /* Intermediates of one batch entry of any composition (small T): as
- * mta_oracle_stages, plus A1 [H][T][T] (the rows after the first head mix);
- * A is then the attention that meets V. */
+ * mta_oracle_stages (C is the softmax input, after the logit mix), plus A1
+ * [H][T][T] (the rows after the first head mix); A is then the attention
+ * that meets V. */
 int mta_oracle_stages_composed(const mta_oracle_shape *s, const double *q, const double *k,
-                               const double *v, const double *w_kq, const double *w_head,
-                               const double *w_kq_post, const double *w_head_post,
+                               const double *v, const mta_oracle_composition *c,
                                const double *gn_weight, const double *gn_bias,
                                double depth_scale, const double *gate, int b, double *C,
                                double *P, double *A1, double *A, double *O, double *out)
 {
-    mta_oracle_args a = {q, k, v, w_kq, w_head, w_kq_post, w_head_post,
-                         gn_weight, gn_bias, depth_scale, gate};
+    if (!c) return -1;
+    mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return stages_args(s, &a, b, C, P, A1, A, O, out);
 }
 

@@ -1,11 +1,14 @@
 """Pins of the oracle's compositions of the two MTA convolutions around the
 softmax ("Multi-Token Attention -- Paper Graph", "Key-Query Convolution",
-post-softmax variant; "Putting Everything Together: The Full MTA Module").
+post-softmax variant and Eq. (4); "Head Mixing Convolution", pre-softmax
+version; "Putting Everything Together: The Full MTA Module").
 
-A composition runs, in this order, Mask_0, [key-query conv w_kq], Mask_-inf,
-softmax, [head mix w_head], [key-query conv w_kq_post, Mask_0],
-[head mix w_head_post], A V, GroupNorm, scale; a bracketed step with no
-weights is left out.  The pins here do not come from the oracle: a brute force
+A composition runs, in this order, Mask_0, [key-query conv w_kq],
+[head mix of the logits w_head_pre], Mask_-inf, softmax, [head mix w_head],
+[key-query conv w_kq_post, Mask_0], [head mix w_head_post], A V, GroupNorm,
+scale; a bracketed step with no weights is left out.  With exact_mask the
+w_kq conv reads the unmasked logits under Eq. (4)'s indicator 1_{i >= j-j'}
+instead of Mask_0's zeros.  The pins here do not come from the oracle: a brute force
 built from scipy's true 2-D convolution and numpy on materialised maps, a
 closed form for a single-tap kernel on the probabilities, reductions to
 torch's causal attention, and invariants.
@@ -37,6 +40,24 @@ def true_conv2d(X, th):
     return Y
 
 
+def indicator_conv(Afull, th):
+    """Eq. (4) taken literally: C[b,h,i,j] = sum over taps (a, jj), with
+    jp = jj - c_k//2, of th[h,a,jj] Afull[b,h,i-a,j-jp] where i-a >= 0,
+    0 <= j-jp < T and j-jp <= i; Afull holds the unmasked logits."""
+    B, H, T, _ = Afull.shape
+    c_q, c_k = th.shape[1:]
+    I = np.arange(T)[:, None]
+    J = np.arange(T)[None, :]
+    C = np.zeros_like(Afull)
+    for a in range(c_q):
+        for jj in range(c_k):
+            r, c = I - a, J - (jj - c_k // 2)
+            ok = (r >= 0) & (c >= 0) & (c < T) & (c <= I)
+            shifted = Afull[:, :, np.clip(r, 0, T - 1), np.clip(c, 0, T - 1)]
+            C += th[:, a, jj][None, :, None, None] * np.where(ok, shifted, 0.0)
+    return C
+
+
 def mix(Aw, w):
     B, H, T, _ = Aw.shape
     c_h = w.shape[-1]
@@ -44,11 +65,18 @@ def mix(Aw, w):
     return np.einsum("goi,bgitj->bgotj", w, Aw.reshape(B, G, c_h, T, T)).reshape(B, H, T, T)
 
 
-def brute_force_composed(q, k, v, th, w, th_post, w_post, gw, gb, depth, gate=None, eps=1e-5):
+def brute_force_composed(q, k, v, th, w, th_post, w_post, gw, gb, depth, gate=None, eps=1e-5,
+                         w_pre=None, exact=False):
     B, H, T, d = q.shape
     causal = np.tril(np.ones((T, T), dtype=bool))
-    A0 = np.where(causal, np.einsum("bhie,bhje->bhij", q, k) / np.sqrt(d), 0.0)
-    C = true_conv2d(A0, th) if th is not None else A0
+    Afull = np.einsum("bhie,bhje->bhij", q, k) / np.sqrt(d)
+    A0 = np.where(causal, Afull, 0.0)
+    if th is None:
+        C = A0
+    else:
+        C = indicator_conv(Afull, th) if exact else true_conv2d(A0, th)
+    if w_pre is not None:
+        C = mix(C, w_pre)          # logits mixed before the second mask
     C = np.where(causal, C, -np.inf)
     P = scipy.special.softmax(C, axis=-1)
     A1 = mix(P, w) if w is not None else P
@@ -233,4 +261,141 @@ def test_composed_rows_and_forward_agree(name):
     idx = [0, 1, 4, 5, 6, 11, 20, 39]
     for b in range(shape[0]):
         r = oracle.rows_composed(q, k, v, *ws, gw, gb, 0.8, b, idx)
+        np.testing.assert_allclose(r, out[b, idx], rtol=0, atol=1e-13)
+
+
+
+# (w_kq, w_head_pre, w_head, w_kq_post, w_head_post, exact_mask)
+PRE_COMPOSITIONS = {
+    "both_pre": (1, 1, 0, 0, 0, 0),
+    "logit_mix_only": (0, 1, 0, 0, 0, 0),
+    "pre_mix_and_post_mix": (1, 1, 1, 0, 0, 0),
+    "exact_default": (1, 0, 1, 0, 0, 1),
+    "exact_both_pre": (1, 1, 0, 0, 0, 1),
+    "exact_everything": (1, 1, 1, 1, 1, 1),
+}
+
+
+def pre_inputs(rng, shape, use):
+    q, k, v, th, w, gw, gb = rand_inputs(rng, *shape)
+    w_pre = rng.standard_normal(w.shape)
+    th_post = 0.5 * rng.standard_normal(th.shape)
+    w_post = rng.standard_normal(w.shape)
+    picked = [x if u else None for x, u in zip((th, w_pre, w, th_post, w_post), use[:5])]
+    return q, k, v, picked, bool(use[5]), gw, gb
+
+
+def call_pre(fn, q, k, v, ws, exact, gw, gb, depth, **kw):
+    th, w_pre, w, th_post, w_post = ws
+    return fn(q, k, v, th, w, th_post, w_post, gw, gb, depth, w_head_pre=w_pre,
+              exact_mask=exact, **kw)
+
+
+@pytest.mark.parametrize("name", sorted(PRE_COMPOSITIONS))
+@pytest.mark.parametrize("shape", SHAPES)
+def test_pre_softmax_compositions_match_brute_force(shape, name):
+    rng = np.random.default_rng(zlib.crc32(repr((shape, name, "pre")).encode()))
+    q, k, v, ws, exact, gw, gb = pre_inputs(rng, shape, PRE_COMPOSITIONS[name])
+    th, w_pre, w, th_post, w_post = ws
+    ref = brute_force_composed(q, k, v, th, w, th_post, w_post, gw, gb, 0.7, w_pre=w_pre,
+                               exact=exact)
+    out = call_pre(oracle.forward_composed, q, k, v, ws, exact, gw, gb, 0.7)
+    np.testing.assert_allclose(out, ref["out"], rtol=0, atol=1e-11)
+    for b in range(shape[0]):
+        st = call_pre(oracle.stages_composed, q, k, v, ws, exact, gw, gb, 0.7, b=b)
+        for key in ("P", "A1", "A", "O"):
+            np.testing.assert_allclose(st[key], ref[key][b], rtol=0, atol=1e-11, err_msg=key)
+        live = np.isfinite(ref["C"][b])
+        assert np.array_equal(live, np.isfinite(st["C"]))
+        np.testing.assert_allclose(st["C"][live], ref["C"][b][live], rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("c_q,c_k", [(3, 5), (4, 4)])
+def test_exact_indicator_single_tap_closed_form(c_q, c_k):
+    # Eq. (4) with one non-zero tap (i', j'): C[i][j] = q_{i-i'} . k_{j-j'} /
+    # sqrt(d) when i-i' >= 0, 0 <= j-j' < T and j-j' <= i (the indicator), 0
+    # otherwise, -inf for j > i.  Unlike Eq. (5)'s Mask_0 this keeps pairs
+    # with i-i' < j-j' <= i, whose logits lie above the diagonal.
+    rng = np.random.default_rng(40)
+    H, T, d = 1, 13, 5
+    q, k, v = (rng.standard_normal((1, H, T, d)) for _ in range(3))
+    gw = np.ones(H * d); gb = np.zeros(H * d)
+    kept_above = 0
+    for ip in range(c_q):
+        for jj in range(c_k):
+            jp = jj - c_k // 2
+            th = np.zeros((H, c_q, c_k)); th[0, ip, jj] = 1.0
+            C = oracle.stages_composed(q, k, v, th, None, None, None, gw, gb, 1.0,
+                                       exact_mask=True)["C"][0]
+            for i in range(T):
+                for j in range(T):
+                    if j > i:
+                        assert C[i, j] == -np.inf
+                        continue
+                    r, c = i - ip, j - jp
+                    if r >= 0 and 0 <= c < T and c <= i:
+                        want = float(q[0, 0, r] @ k[0, 0, c]) / np.sqrt(d)
+                        kept_above += c > r
+                    else:
+                        want = 0.0
+                    assert abs(C[i, j] - want) < 1e-12, (ip, jp, i, j)
+    assert kept_above > 0
+
+
+def test_exact_indicator_equals_two_pass_masking_for_one_query_tap():
+    # With c_q = 1 the indicator 1_{i >= j-j'} and Mask_0 (j-j' <= i-0) agree.
+    rng = np.random.default_rng(41)
+    q, k, v, th, w, gw, gb = rand_inputs(rng, 2, 4, 23, 8, 1, 7, 2)
+    a = oracle.forward_composed(q, k, v, th, w, None, None, gw, gb, 0.8)
+    b = oracle.forward_composed(q, k, v, th, w, None, None, gw, gb, 0.8, exact_mask=True)
+    assert np.array_equal(a, b)
+    c = oracle.forward_composed(q, k, v, np.tile(th, (1, 3, 1)) / 3, w, None, None, gw, gb, 0.8,
+                                exact_mask=True)
+    assert not np.allclose(c, oracle.forward_composed(q, k, v, np.tile(th, (1, 3, 1)) / 3, w,
+                                                      None, None, gw, gb, 0.8))
+
+
+def test_logit_mix_is_softmax_of_mixed_logits():
+    # "Head Mixing Convolution", pre-softmax version: with no key-query conv
+    # the attention of head h is softmax(causal(sum_h' w[h][h'] q_h' k_h'^T /
+    # sqrt(d))), computed here with torch.
+    rng = np.random.default_rng(42)
+    B, H, T, d, c_h = 1, 4, 19, 8, 2
+    q, k, v = (rng.standard_normal((B, H, T, d)) for _ in range(3))
+    w = rng.standard_normal((H // c_h, c_h, c_h))
+    tq, tk = torch.as_tensor(q[0]), torch.as_tensor(k[0])
+    logits = tq @ tk.transpose(-1, -2) / np.sqrt(d)                  # [H,T,T]
+    mixed = torch.einsum("goi,gitj->gotj", torch.as_tensor(w),
+                         logits.reshape(H // c_h, c_h, T, T)).reshape(H, T, T)
+    P = torch.softmax(mixed.masked_fill(~torch.ones(T, T, dtype=torch.bool).tril(),
+                                        float("-inf")), dim=-1)
+    st = oracle.stages_composed(q, k, v, None, None, None, None, np.ones(H * d), np.zeros(H * d),
+                                1.0, w_head_pre=w)
+    np.testing.assert_allclose(st["P"], P.numpy(), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(st["O"], (P @ torch.as_tensor(v[0])).numpy(), rtol=0, atol=1e-12)
+
+
+def test_exact_and_logit_mix_causality():
+    rng = np.random.default_rng(43)
+    shape = (1, 4, 28, 8, 6, 11, 2)
+    q, k, v, ws, exact, gw, gb = pre_inputs(rng, shape, PRE_COMPOSITIONS["exact_everything"])
+    out = call_pre(oracle.forward_composed, q, k, v, ws, exact, gw, gb, 0.8)
+    for t in (0, 3, 16, 26):
+        q2, k2, v2 = q.copy(), k.copy(), v.copy()
+        for x in (q2, k2, v2):
+            x[:, :, t + 1:] += rng.standard_normal(x[:, :, t + 1:].shape)
+        out2 = call_pre(oracle.forward_composed, q2, k2, v2, ws, exact, gw, gb, 0.8)
+        assert np.array_equal(out[:, : t + 1], out2[:, : t + 1])
+        assert not np.allclose(out[:, t + 1:], out2[:, t + 1:])
+
+
+@pytest.mark.parametrize("name", ["exact_everything", "both_pre"])
+def test_pre_softmax_rows_and_forward_agree(name):
+    rng = np.random.default_rng(44)
+    shape = (2, 4, 40, 8, 6, 11, 2)
+    q, k, v, ws, exact, gw, gb = pre_inputs(rng, shape, PRE_COMPOSITIONS[name])
+    out = call_pre(oracle.forward_composed, q, k, v, ws, exact, gw, gb, 0.8)
+    idx = [0, 1, 4, 5, 6, 11, 20, 39]
+    for b in range(shape[0]):
+        r = call_pre(oracle.rows_composed, q, k, v, ws, exact, gw, gb, 0.8, b=b, row_idx=idx)
         np.testing.assert_allclose(r, out[b, idx], rtol=0, atol=1e-13)

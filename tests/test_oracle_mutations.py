@@ -19,9 +19,9 @@ MUTATIONS = [
     ("key offset sign flipped", "int c = j - jp;", "int c = j + jp;"),
     ("query taps reversed", "theta[ip * c_k + (jp - jlo)]",
      "theta[(c_q - 1 - ip) * c_k + (jp - jlo)]"),
-    ("no Mask_0 before the conv", "for (int c = 0; c <= r; ++c) {",
-     "for (int c = 0; c < T; ++c) {"),
-    ("Mask_-inf replaced by zero", "rows, -INFINITY, u->C);", "rows, 0.0, u->C);"),
+    ("no Mask_0 before the conv", "const int last = a->exact ? r + s->c_q - 1 : r;",
+     "const int last = T - 1;"),
+    ("Mask_-inf replaced by zero", "rows, a->exact, -INFINITY, C);", "rows, a->exact, 0.0, C);"),
     ("unbiased variance", "    var /= d;\n    double inv", "    var /= (d - 1);\n    double inv"),
     ("eps outside the square root", "1.0 / sqrt(var + s->gn_eps)",
      "1.0 / (sqrt(var) + s->gn_eps)"),
@@ -35,7 +35,7 @@ MUTATIONS = [
     ("gate applied before the affine bias", "out_row[chn] = scale * y;",
      "out_row[chn] = scale * (y - a->gn_bias[chn]) + a->gn_bias[chn];"),
     # compositions of "Putting Everything Together"
-    ("post-softmax conv keeps future keys", "rows, 0.0,", "rows, 1.0,"),
+    ("post-softmax conv keeps future keys", "rows, 0, 0.0,", "rows, 0, 1.0,"),
     ("second head mix skipped", "a->w_head_post ? a->w_head_post + (size_t)g * c_h * c_h : NULL",
      "NULL"),
     ("post-softmax conv fed unmixed rows", "u.A1 + (size_t)hh * T,", "u.P + (size_t)hh * T,"),
@@ -44,12 +44,22 @@ MUTATIONS = [
     ("fresh first-stage rows from the wrong logits",
      "masked0_logit_row(s, a, b, g * c_h + hh, r - ip2, slot);",
      "masked0_logit_row(s, a, b, g * c_h + hh, i - ip2, slot);"),
-    ("no Mask_-inf without a key-query conv", "u->C[j] = (j <= r) ? rows[0][j] : -INFINITY;",
-     "u->C[j] = rows[0][j];"),
+    ("no Mask_-inf without a key-query conv", "C[j] = (j <= r) ? rows[0][j] : -INFINITY;",
+     "C[j] = rows[0][j];"),
     ("post-softmax conv reads the current row only",
      "point_rows(s, u.ring1, i, u.zero, u.rows1);",
      "point_rows(s, u.ring1, i, u.zero, u.rows1);\n"
      "            for (int z = 0; z < s->c_h * s->c_q; ++z) u.rows1[z] = u.rows1[z - z % s->c_q];"),
+    # pre-softmax head mix and the exact indicator of Eq. (4)
+    ("logit mix transposed", "acc += wrow[hi] *", "acc += wg[(size_t)hi * c_h + ho] *"),
+    ("logit mix fills future keys with zero",
+     "if (j > r) { out[(size_t)ho * T + j] = -INFINITY; continue; }",
+     "if (j > r) { out[(size_t)ho * T + j] = 0.0; continue; }"),
+    ("logit mix skipped", "    if (a->w_head_pre) {", "    if (0) {"),
+    ("exact indicator tested against the shifted query", "if (exact && c > i) continue;",
+     "if (exact && c > i - ip) continue;"),
+    ("exact rows without the keys past the query", "const int last = a->exact ? r + s->c_q - 1 : r;",
+     "const int last = a->exact ? r + s->c_q - 2 : r;"),
 ]
 
 PIN_CHECKS = [
@@ -68,6 +78,11 @@ PIN_CHECKS = [
     lambda: cpins.test_post_conv_single_tap_closed_form(3, 5),
     cpins.test_plain_composition_is_causal_attention,
     lambda: [cpins.test_composed_rows_and_forward_agree(n) for n in ("repeat", "both_post")],
+    lambda: [cpins.test_pre_softmax_compositions_match_brute_force(cpins.SHAPES[1], n)
+             for n in ("both_pre", "exact_everything")],
+    lambda: cpins.test_exact_indicator_single_tap_closed_form(3, 5),
+    cpins.test_logit_mix_is_softmax_of_mixed_logits,
+    lambda: cpins.test_pre_softmax_rows_and_forward_agree("exact_everything"),
 ]
 
 
