@@ -176,13 +176,20 @@ def barrier(world):
         dist.barrier()
 
 
-WEIGHTS = ("w_kq", "w_head", "w_kq_post", "w_head_post")
+WEIGHTS = ("w_kq", "w_head", "w_kq_post", "w_head_post")   # positional order of the call
+
+
+def compose_kw(args, d):
+    """Keyword arguments of mta_forward_composed beyond the four positional
+    weights: the logit mix and the exact-mask flag of the composition."""
+    return {"w_head_pre": d.get("w_head_pre"),
+            "exact_mask": bool(COMPOSITIONS[args.compose].get("exact_mask"))}
 
 
 def device_inputs(x, io, device):
     dt = torch.bfloat16 if io == "bf16" else torch.float32
     d = {n: torch.from_numpy(x[n]).to(device).to(dt) for n in ("q", "k", "v")}
-    for n in WEIGHTS + ("gn_weight", "gn_bias"):
+    for n in WEIGHTS + ("w_head_pre", "gn_weight", "gn_bias"):
         d[n] = torch.from_numpy(x[n]).to(device) if x.get(n) is not None else None
     return d
 
@@ -262,8 +269,10 @@ def time_mta(args, w, d, world, device):
     import convolved_logit_attention_b200 as mta
     unfused = args.path == "unfused"
     if args.compose:
-        shape = mta.composed_shape(d["q"], *(d[n] for n in WEIGHTS), gn_eps=w.gn_eps)
-        comp = mta.composition(*(d[n] for n in WEIGHTS))
+        kw = compose_kw(args, d)
+        shape = mta.composed_shape(d["q"], *(d[n] for n in WEIGHTS), gn_eps=w.gn_eps,
+                                   w_head_pre=kw["w_head_pre"])
+        comp = mta.composition(*(d[n] for n in WEIGHTS), **kw)
         names = mta.mta_composed_kernel_names(shape, comp)
         nk = len(names)
         fused = "k_mta_fused" in names
@@ -292,7 +301,7 @@ def time_mta(args, w, d, world, device):
                                  gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
                                  depth_scale=w.depth_scale, gate=gate if args.gate else None,
                                  out=out, workspace=ws, stream=stream, gn_eps=w.gn_eps,
-                                 events=events)
+                                 events=events, **compose_kw(args, d))
 
     def step():
         if args.compose:
@@ -361,7 +370,7 @@ def time_e2e(args, w, x, device):
     first input copy of the timed steps to the end of their last output copy."""
     import convolved_logit_attention_b200 as mta
     dt = torch.bfloat16 if w.io == "bf16" else torch.float32
-    names = tuple(n for n in ("q", "k", "v") + WEIGHTS + ("gn_weight", "gn_bias")
+    names = tuple(n for n in ("q", "k", "v") + WEIGHTS + ("w_head_pre", "gn_weight", "gn_bias")
                   if x.get(n) is not None)
     host = {n: torch.from_numpy(x[n]).to(dt).pin_memory() for n in ("q", "k", "v")}
     for n in names[3:]:
@@ -372,9 +381,10 @@ def time_e2e(args, w, x, device):
     out_host = [torch.empty(out[0].shape, dtype=dt).pin_memory() for _ in range(nbuf)]
     if args.compose:
         wts = [dev[0].get(n) for n in WEIGHTS]
-        shape = mta.composed_shape(dev[0]["q"], *wts, gn_eps=w.gn_eps)
-        ws_bytes = mta.lib().mta_composed_workspace_size(ctypes.byref(shape),
-                                                         ctypes.byref(mta.composition(*wts)))
+        kw = compose_kw(args, dev[0])
+        shape = mta.composed_shape(dev[0]["q"], *wts, gn_eps=w.gn_eps, w_head_pre=kw["w_head_pre"])
+        ws_bytes = mta.lib().mta_composed_workspace_size(
+            ctypes.byref(shape), ctypes.byref(mta.composition(*wts, **kw)))
     else:
         shape = mta.shape_of(dev[0]["q"], dev[0]["w_kq"], dev[0]["w_head"], w.gn_eps)
         ws_bytes = mta.mta_workspace_size(shape)
@@ -406,7 +416,7 @@ def time_e2e(args, w, x, device):
                 mta.mta_forward_composed(d["q"], d["k"], d["v"], *(d.get(n) for n in WEIGHTS),
                                          gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
                                          depth_scale=w.depth_scale, out=out[bi], workspace=ws,
-                                         stream=s_comp, gn_eps=w.gn_eps)
+                                         stream=s_comp, gn_eps=w.gn_eps, **compose_kw(args, d))
             else:
                 mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
                                 d["gn_bias"], w.depth_scale, out=out[bi], workspace=ws,
@@ -433,8 +443,8 @@ def time_e2e(args, w, x, device):
 
 def oracle_sample(w, x, n_units, flops_per_step):
     """The first n_units (batch, head-group) units of the workload at full T,
-    as separate B=1, H=c_h problems (weights a composition leaves out stay
-    None), with their algorithmic FLOPs."""
+    as separate B=1, H=c_h problems (dicts of arrays; weights a composition
+    leaves out stay None), with their algorithmic FLOPs."""
     def part(name, sl):
         return x[name][sl] if x.get(name) is not None else None
     units = []
@@ -443,29 +453,37 @@ def oracle_sample(w, x, n_units, flops_per_step):
         hs = slice(g * w.c_h, (g + 1) * w.c_h)
         cs = slice(g * w.c_h * w.d, (g + 1) * w.c_h * w.d)
         gs = slice(g, g + 1)
-        units.append((x["q"][b:b + 1, hs], x["k"][b:b + 1, hs], x["v"][b:b + 1, hs],
-                      part("w_kq", hs), part("w_head", gs), part("w_kq_post", hs),
-                      part("w_head_post", gs), x["gn_weight"][cs], x["gn_bias"][cs]))
+        units.append({"q": x["q"][b:b + 1, hs], "k": x["k"][b:b + 1, hs],
+                      "v": x["v"][b:b + 1, hs], "w_kq": part("w_kq", hs),
+                      "w_head_pre": part("w_head_pre", gs), "w_head": part("w_head", gs),
+                      "w_kq_post": part("w_kq_post", hs), "w_head_post": part("w_head_post", gs),
+                      "gn_weight": x["gn_weight"][cs], "gn_bias": x["gn_bias"][cs],
+                      "exact_mask": bool(x.get("exact_mask"))})
     flops = len(units) * flops_per_step // (w.B * w.G)
     return units, flops
+
+
+def run_oracle_unit(u, w, nthreads=1):
+    import oracle
+    default = (u["w_kq"] is not None and u["w_head"] is not None and u["w_head_pre"] is None
+               and u["w_kq_post"] is None and u["w_head_post"] is None and not u["exact_mask"])
+    if default:
+        return oracle.forward(u["q"], u["k"], u["v"], u["w_kq"], u["w_head"], u["gn_weight"],
+                              u["gn_bias"], w.depth_scale, gn_eps=w.gn_eps, nthreads=nthreads)
+    return oracle.forward_composed(u["q"], u["k"], u["v"], u["w_kq"], u["w_head"], u["w_kq_post"],
+                                   u["w_head_post"], u["gn_weight"], u["gn_bias"], w.depth_scale,
+                                   gn_eps=w.gn_eps, nthreads=nthreads,
+                                   w_head_pre=u["w_head_pre"], exact_mask=u["exact_mask"])
 
 
 def run_oracle_units(units, w, nthreads):
     """Runs the oracle forward on every unit, one unit per host thread (the
     ctypes call releases the GIL); returns the wall time in seconds."""
     import concurrent.futures as cf
-    import oracle
-
-    def one(u):
-        if u[5] is None and u[6] is None:
-            return oracle.forward(u[0], u[1], u[2], u[3], u[4], u[7], u[8], w.depth_scale,
-                                  gn_eps=w.gn_eps, nthreads=1)
-        return oracle.forward_composed(*u[:7], u[7], u[8], w.depth_scale, gn_eps=w.gn_eps,
-                                       nthreads=1)
 
     t0 = time.perf_counter()
     with cf.ThreadPoolExecutor(max_workers=nthreads) as ex:
-        list(ex.map(one, units))
+        list(ex.map(lambda u: run_oracle_unit(u, w), units))
     return time.perf_counter() - t0
 
 

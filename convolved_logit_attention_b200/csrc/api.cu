@@ -141,7 +141,8 @@ namespace {
 
 bool is_default_composition(const mta_composition *c)
 {
-    return c->w_kq && c->w_head && !c->w_kq_post && !c->w_head_post;
+    return c->w_kq && c->w_head && !c->w_kq_post && !c->w_head_post && !c->w_head_pre &&
+           !c->exact_mask;
 }
 
 mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const void *v,
@@ -161,14 +162,14 @@ mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const
         if (!p) return MTA_ERR_INVALID_ARG;
     for (const void *p : need)
         if (!aligned(p, 16)) return MTA_ERR_ALIGNMENT;
-    const void *opt[] = {c->w_kq, c->w_head, c->w_kq_post, c->w_head_post};
+    const void *opt[] = {c->w_kq, c->w_head, c->w_kq_post, c->w_head_post, c->w_head_pre};
     for (const void *p : opt)
         if (p && !aligned(p, 16)) return MTA_ERR_ALIGNMENT;
     if (n_events < 0 || (n_events > 0 && !events)) return MTA_ERR_INVALID_ARG;
     rc = check_workspace(workspace, workspace_bytes, mta::unfused_workspace_bytes(*s));
     if (rc != MTA_OK) return rc;
     mta::ForwardArgs a{q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias, depth_scale, out, gate,
-                       c->w_kq_post, c->w_head_post};
+                       c->w_kq_post, c->w_head_post, c->w_head_pre, c->exact_mask != 0};
     mta::Trace tr;
     tr.events = events;
     tr.n = n_events;
@@ -182,6 +183,8 @@ mta::ForwardArgs chain_args(const mta_composition *c)
     a.w_head = c->w_head;
     a.w_kq_post = c->w_kq_post;
     a.w_head_post = c->w_head_post;
+    a.w_head_pre = c->w_head_pre;
+    a.exact_mask = c->exact_mask != 0;
     return a;
 }
 

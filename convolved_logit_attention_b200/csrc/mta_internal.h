@@ -20,6 +20,10 @@ struct ForwardArgs {
     // kernel on the probabilities and a second head mix; null: left out.
     // On that path w_kq and w_head may be null too (the step is left out).
     const float *w_kq_post = nullptr, *w_head_post = nullptr;
+    // Before the softmax: a mix of the logits after the w_kq conv, and the
+    // exact indicator of Eq. (4) for that conv instead of Mask_0.
+    const float *w_head_pre = nullptr;
+    int exact_mask = 0;
 };
 
 // Optional CUDA events recorded around the kernel launches of one call.
@@ -44,7 +48,7 @@ constexpr int kUnfusedKernels = 4;
 extern const char *const kUnfusedKernelNames[kUnfusedKernels];
 // Launch sequence of launch_unfused for the steps a names (at most
 // kMaxChainKernels); fills names[] in launch order and returns the count.
-constexpr int kMaxChainKernels = 6;
+constexpr int kMaxChainKernels = 7;
 int unfused_chain(const ForwardArgs &a, const char **names);
 mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr);

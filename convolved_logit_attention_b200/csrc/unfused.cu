@@ -39,8 +39,10 @@ constexpr int kPvKeys = 32;
 constexpr int kPvAStride = kPvRows + 4;   // transposed attention chunk: key-major rows
 constexpr int kMaxD = 128;
 
-// S1 + S2: map0[bh][i][j] = (j <= i) ? q_i . k_j * scale : 0 on tiles that
-// touch the causal triangle.  Grid (col tiles, row tiles, B*H), 256 threads,
+// S1 + S2: map0[bh][i][j] = (j <= i + band) ? q_i . k_j * scale : 0 on tiles
+// that touch the causal triangle widened by `band` keys: band = 0 is Mask_0;
+// the exact indicator of Eq. (4) needs the c_q - 1 keys past each query
+// (band = c_q - 1), which the convolution's taps of later queries may read.  Grid (col tiles, row tiles, B*H), 256 threads,
 // 128 x 128 tiles.  Thread (tx, ty) = (tid % 16, tid / 16) owns rows
 // {ty*4 .. ty*4+3} and {64+ty*4 .. 64+ty*4+3} and the same pattern of
 // columns with tx, so that its operands for one contraction index are four
@@ -49,12 +51,12 @@ constexpr int kMaxD = 128;
 template <typename TIO>
 __global__ void __launch_bounds__(256)
 k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict__ map0,
-         int T, int d, float scale)
+         int T, int d, float scale, int band)
 {
     const int ct = blockIdx.x, rt = blockIdx.y;
-    if (ct > rt) return;                     // the whole tile lies above the diagonal
-    const size_t bh = blockIdx.z;
     const int i0 = rt * kLogitTile, j0 = ct * kLogitTile;
+    if (j0 > i0 + kLogitTile - 1 + band) return;   // the whole tile lies past the band
+    const size_t bh = blockIdx.z;
     __shared__ __align__(16) float qs[kLogitDk * kLogitStride];
     __shared__ __align__(16) float ks[kLogitDk * kLogitStride];
     const int tid = threadIdx.x;
@@ -100,7 +102,8 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
             const int jb = j0 + half * 64 + tx * 4;
             float x[4];
 #pragma unroll
-            for (int w = 0; w < 4; ++w) x[w] = (jb + w <= i) ? acc[u][half * 4 + w] * scale : 0.f;
+            for (int w = 0; w < 4; ++w)
+                x[w] = (jb + w <= i + band) ? acc[u][half * 4 + w] * scale : 0.f;
             if ((T & 3) == 0) {
                 if (jb < T)
                     *reinterpret_cast<float4 *>(mb + (size_t)i * T + jb) =
@@ -118,7 +121,10 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
 // j <= i (also the post-softmax conv of the probabilities).  The 32 x 128
 // output tile reads a (32 + c_q - 1)-row halo of src into shared memory;
 // reads outside [0,T) or above the diagonal (c > r) are the zeros of Mask_0
-// and of the zero padding.  Thread (warp w, lane l) owns output row l and
+// and of the zero padding.  With kExact (the exact indicator of Eq. (4))
+// the halo keeps src[r][c] for c <= r + band, and each output row i zeroes
+// the keys c > i of the segments it reads: a tap (i', j') then adds
+// src[i-i'][j-j'] exactly when j - j' <= i.  Thread (warp w, lane l) owns output row l and
 // the 16 columns 16w .. 16w+15: per query tap i' it loads the row segment
 // those columns reach (16 + c_k - 1 values) and the tap row theta[i'][*]
 // with 16-byte shared loads into registers and applies the c_k key taps from
@@ -126,10 +132,10 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
 // the FMA count.  Halo rows are kConvStride floats apart, 4 (mod 32) banks,
 // so the 16-byte loads of 8 consecutive rows hit distinct banks.  The taps
 // accumulate in the order i' then j' for every output.
-template <int CK>
+template <int CK, bool kExact>
 __global__ void __launch_bounds__(256)
 k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__restrict__ w_kq,
-       int T, int H, int c_q)
+       int T, int H, int c_q, int band)
 {
     constexpr int NC = kConvCols / 8;             // output columns per thread
     constexpr int NV = (CK + NC - 1 + 3) / 4;     // float4 loads per row segment
@@ -151,7 +157,7 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
         const int rr = idx / kLoadCols, cc = idx % kLoadCols;
         const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
         tile[rr * kConvStride + cc] =
-            (r >= 0 && r < T && c >= 0 && c <= r) ? mb[(size_t)r * T + c] : 0.f;
+            (r >= 0 && r < T && c >= 0 && c < T && c <= r + band) ? mb[(size_t)r * T + c] : 0.f;
     }
     for (int idx = tid; idx < c_q * CKP; idx += 256) {
         const int ip = idx / CKP, jj = idx % CKP;
@@ -171,6 +177,12 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
         for (int v = 0; v < NV; ++v) {
             const float4 t = seg4[v];
             seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
+        }
+        if (kExact) {                             // the indicator: keys past query i read 0
+            const int kfirst = j0 - L + c0;       // key of seg[0]
+#pragma unroll
+            for (int v = 0; v < 4 * NV; ++v)
+                if (kfirst + v > i0 + ro) seg[v] = 0.f;
         }
         const float4 *tr4 = reinterpret_cast<const float4 *>(&th[ip * CKP]);
         float tr[CKP];
@@ -477,21 +489,27 @@ mta_status head_mix(const mta_shape &s, const float *src, float *dst, const floa
 }
 
 template <typename TIO>
-void launch_logits(const mta_shape &s, const void *q, const void *k, float *map0, cudaStream_t st)
+void launch_logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
+                   cudaStream_t st)
 {
     const int nt = (s.T + kLogitTile - 1) / kLogitTile;
     dim3 g1(nt, nt, s.B * s.H);
     k_logits<TIO><<<g1, 256, 0, st>>>((const TIO *)q, (const TIO *)k, map0, s.T, s.d,
-                                      1.0f / sqrtf((float)s.d));
+                                      1.0f / sqrtf((float)s.d), band);
 }
 
-void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq,
+void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq, int band,
                  cudaStream_t st)
 {
     dim3 g2((s.T + kConvCols - 1) / kConvCols, (s.T + kConvRows - 1) / kConvRows, s.B * s.H);
     switch (s.c_k) {
 #define MTA_CONV_CASE(n) \
-        case n: k_conv<n><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q); break;
+        case n:                                                                          \
+            if (band > 0)                                                                \
+                k_conv<n, true><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q, band);  \
+            else                                                                         \
+                k_conv<n, false><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q, 0);    \
+            break;
         MTA_CONV_CASE(1) MTA_CONV_CASE(2) MTA_CONV_CASE(3) MTA_CONV_CASE(4) MTA_CONV_CASE(5)
         MTA_CONV_CASE(6) MTA_CONV_CASE(7) MTA_CONV_CASE(8) MTA_CONV_CASE(9) MTA_CONV_CASE(10)
         MTA_CONV_CASE(11) MTA_CONV_CASE(12) MTA_CONV_CASE(13) MTA_CONV_CASE(14) MTA_CONV_CASE(15)
@@ -500,12 +518,13 @@ void launch_conv(const mta_shape &s, const float *src, float *dst, const float *
     }
 }
 
-void logits(const mta_shape &s, const void *q, const void *k, float *map0, cudaStream_t st)
+void logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
+            cudaStream_t st)
 {
     if (s.io == MTA_BF16)
-        launch_logits<__nv_bfloat16>(s, q, k, map0, st);
+        launch_logits<__nv_bfloat16>(s, q, k, map0, band, st);
     else
-        launch_logits<float>(s, q, k, map0, st);
+        launch_logits<float>(s, q, k, map0, band, st);
 }
 
 void pv_groupnorm(const mta_shape &s, const float *amap, const ForwardArgs &a, cudaStream_t st)
@@ -533,6 +552,7 @@ int unfused_chain(const ForwardArgs &a, const char **names)
     int n = 0;
     names[n++] = "k_logits";
     if (a.w_kq) names[n++] = "k_conv";
+    if (a.w_head_pre) names[n++] = "k_head_mix";
     names[n++] = "k_softmax_mix";
     if (a.w_kq_post) names[n++] = "k_conv";
     if (a.w_head_post) names[n++] = "k_head_mix";
@@ -542,29 +562,39 @@ int unfused_chain(const ForwardArgs &a, const char **names)
 
 // The launches follow unfused_chain(); each step reads maps[cur] and writes
 // maps[cur ^ 1].  For the default composition that is logits -> map0,
-// conv -> map1, softmax + mix -> map0, PV + GroupNorm from map0.
+// conv -> map1, softmax + mix -> map0, PV + GroupNorm from map0.  The exact
+// indicator widens the logits and the first conv's halo by c_q - 1 keys.
 mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr)
 {
     float *maps[2] = {(float *)ws, (float *)ws + bh_tt(s)};
+    const int band = (a.exact_mask && a.w_kq) ? s.c_q - 1 : 0;
     int cur = 0, launch = 0;
+    mta_status rc = MTA_OK;
     tr.before(launch, st);
-    logits(s, a.q, a.k, maps[0], st);
+    logits(s, a.q, a.k, maps[0], band, st);
     tr.after(launch++, st);
     if (a.w_kq) {
         tr.before(launch, st);
-        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq, st);
+        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq, band, st);
         tr.after(launch++, st);
         cur ^= 1;
     }
+    if (a.w_head_pre) {                           // mix of the logits, before the softmax
+        tr.before(launch, st);
+        rc = head_mix(s, maps[cur], maps[cur ^ 1], a.w_head_pre, st);
+        tr.after(launch++, st);
+        if (rc != MTA_OK) return rc;
+        cur ^= 1;
+    }
     tr.before(launch, st);
-    mta_status rc = softmax_mix(s, maps[cur], maps[cur ^ 1], a.w_head, 0, st);
+    rc = softmax_mix(s, maps[cur], maps[cur ^ 1], a.w_head, 0, st);
     tr.after(launch++, st);
     if (rc != MTA_OK) return rc;
     cur ^= 1;
     if (a.w_kq_post) {
         tr.before(launch, st);
-        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq_post, st);
+        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq_post, 0, st);
         tr.after(launch++, st);
         cur ^= 1;
     }
@@ -587,8 +617,8 @@ mta_status launch_debug_attention(const mta_shape &s, const void *q, const void 
 {
     float *map0 = (float *)ws;
     float *map1 = map0 + bh_tt(s);
-    logits(s, q, k, map0, st);
-    launch_conv(s, map0, map1, w_kq, st);
+    logits(s, q, k, map0, 0, st);
+    launch_conv(s, map0, map1, w_kq, 0, st);
     mta_status rc = softmax_mix(s, map1, attn, w_head, stage == 0 ? 1 : 2, st);
     if (rc != MTA_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;

@@ -35,9 +35,10 @@ Recipes:
                   paired with a query position t ~ U(p, T); the key at p is
                   replaced by q_t + N(0, 0.1^2).
   w_kq_post,      the second key-query kernel and head mix of the
-  w_head_post     compositions of "Putting Everything Together: The Full MTA
-                  Module", drawn like w_kq and w_head from their own stream
-                  (seed + 7919), so that the default inputs stay unchanged.
+  w_head_post,    compositions of "Putting Everything Together: The Full MTA
+  w_head_pre      Module" and the pre-softmax head mix of the logits, drawn
+                  like w_kq and w_head from their own stream (seed + 7919), so
+                  that the default inputs stay unchanged.
 """
 from dataclasses import dataclass, replace
 
@@ -79,25 +80,33 @@ class Workload:
     def tokens(self) -> int:
         return self.B * self.T
 
-    def composition_flops(self, use) -> int:
-        """algorithmic_flops for a composition: use = which of (w_kq,
-        w_head, w_kq_post, w_head_post) it has; every key-query conv costs
-        c_q c_k MACs per live logit and every head mix c_h."""
-        n_kq = int(bool(use[0])) + int(bool(use[2]))
-        n_mix = int(bool(use[1])) + int(bool(use[3]))
+    def composition_flops(self, comp: dict) -> int:
+        """algorithmic_flops for a composition (an entry of COMPOSITIONS):
+        every key-query conv costs c_q c_k MACs per live logit and every
+        head mix c_h."""
+        n_kq = sum(bool(comp.get(n)) for n in ("w_kq", "w_kq_post"))
+        n_mix = sum(bool(comp.get(n)) for n in ("w_head_pre", "w_head", "w_head_post"))
         per_logit = 4 * self.d + 2 * n_kq * self.c_q * self.c_k + 2 * n_mix * self.c_h
         return self.B * self.H * self.live_logits() * per_logit
 
 
-# Which of (w_kq, w_head, w_kq_post, w_head_post) each composition uses.
+WEIGHT_NAMES = ("w_kq", "w_head_pre", "w_head", "w_kq_post", "w_head_post")
+
+# The steps of each composition: the weights it has (the others are None)
+# and whether its first key-query conv uses the exact indicator of Eq. (4).
 COMPOSITIONS = {
-    "default": (1, 1, 0, 0),            # key-query pre-softmax, head post-softmax
-    "repeat": (1, 1, 1, 1),             # the MTA convolution repeated after the softmax
-    "both_post": (0, 0, 1, 1),          # both convolutions after the softmax
-    "post_kq": (0, 0, 1, 0),            # the post-softmax key-query variant alone
-    "mix_then_post_kq": (0, 1, 1, 0),
-    "pre_and_post_kq": (1, 0, 1, 0),
-    "plain_attention": (0, 0, 0, 0),
+    "default": dict(w_kq=1, w_head=1),     # key-query pre-softmax, head post-softmax
+    "repeat": dict(w_kq=1, w_head=1, w_kq_post=1, w_head_post=1),
+    "both_post": dict(w_kq_post=1, w_head_post=1),
+    "post_kq": dict(w_kq_post=1),          # the post-softmax key-query variant alone
+    "mix_then_post_kq": dict(w_head=1, w_kq_post=1),
+    "pre_and_post_kq": dict(w_kq=1, w_kq_post=1),
+    "plain_attention": dict(),
+    "both_pre": dict(w_kq=1, w_head_pre=1),  # the separable 3-D conv of the logits
+    "logit_mix": dict(w_head_pre=1),       # the pre-softmax head mix alone
+    "exact": dict(w_kq=1, w_head=1, exact_mask=1),
+    "exact_both_pre": dict(w_kq=1, w_head_pre=1, exact_mask=1),
+    "exact_repeat": dict(w_kq=1, w_head=1, w_kq_post=1, w_head_post=1, exact_mask=1),
 }
 
 
@@ -175,18 +184,22 @@ def post_weights(w: Workload, seed: int = None) -> dict:
     w_kq_post[:, 0, w.c_k // 2] += np.float32(1.0)
     w_head_post = np.eye(w.c_h, dtype=np.float32)[None] + \
         np.float32(0.05) * rng.standard_normal((w.G, w.c_h, w.c_h), dtype=np.float32)
-    return {"w_kq_post": w_kq_post, "w_head_post": w_head_post.astype(np.float32)}
+    w_head_pre = np.eye(w.c_h, dtype=np.float32)[None] + \
+        np.float32(0.05) * rng.standard_normal((w.G, w.c_h, w.c_h), dtype=np.float32)
+    return {"w_kq_post": w_kq_post, "w_head_post": w_head_post.astype(np.float32),
+            "w_head_pre": w_head_pre.astype(np.float32)}
 
 
 def composed_inputs(w: Workload, composition: str, seed: int = None) -> dict:
     """make_inputs plus post_weights, with the weights a composition leaves
-    out set to None."""
+    out set to None, and its exact_mask flag."""
     x = make_inputs(w, seed)
     x.update(post_weights(w, seed))
-    for name, used in zip(("w_kq", "w_head", "w_kq_post", "w_head_post"),
-                          COMPOSITIONS[composition]):
-        if not used:
+    comp = COMPOSITIONS[composition]
+    for name in WEIGHT_NAMES:
+        if not comp.get(name):
             x[name] = None
+    x["exact_mask"] = bool(comp.get("exact_mask"))
     return x
 
 

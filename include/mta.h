@@ -212,21 +212,31 @@ MTA_API mta_status mta_forward_noalloc(const mta_shape *shape, const void *q, co
 /* One composition of the module ("Multi-Token Attention -- Paper Graph",
  * "Putting Everything Together: The Full MTA Module").  The steps run in
  * this fixed order, each bracketed one only when its weights are given:
- *   S1+S2, [S3 with w_kq], S4, S5, [S6 with w_head],
+ *   S1+S2, [S3 with w_kq], [L1: head mix of the logits with w_head_pre],
+ *   S4, S5, [S6 with w_head],
  *   [P1: conv of the probabilities with w_kq_post, zero where j > i],
  *   [P2: Eq. (7) head mix with w_head_post], S7..S9
  * P1 is the post-softmax variant of "Key-Query Convolution":
  * A1 -> Mask_0(Conv2d_theta(A1)), with the index ranges and zero padding of
- * S3.  The pages' default is {w_kq, w_head}; the repeated MTA convolution
- * ("repeat this operation") is all four; "both post-softmax" is
- * {w_kq_post, w_head_post}.  Both key-query kernels are [H][c_q][c_k] and
- * both head mixes [H/c_h][c_h][c_h], laid out as w_kq and w_head above;
+ * S3.  L1 is the pre-softmax version of "Head Mixing Convolution": the
+ * logits of a group's heads are mixed, on the keys j <= i, before S4; S3
+ * then L1 is the separable case of the 3-D convolution of "Putting
+ * Everything Together" ("both pre-softmax").  exact_mask != 0 replaces S2's
+ * Mask_0 for S3 by the indicator of Eq. (4): the tap (i', j') of output
+ * (i, j) adds theta q_{i-i'} k_{j-j'} / sqrt(d) whenever key j - j' <= i
+ * (Mask_0 keeps it only for j - j' <= i - i').  The pages' default is
+ * {w_kq, w_head}; the repeated MTA convolution ("repeat this operation") is
+ * {w_kq, w_head, w_kq_post, w_head_post}; "both post-softmax" is
+ * {w_kq_post, w_head_post}.  Both key-query kernels are [H][c_q][c_k] and the
+ * three head mixes [H/c_h][c_h][c_h], laid out as w_kq and w_head above;
  * pointers are device memory, 16-byte aligned, NULL for a step left out. */
 typedef struct {
     const float *w_kq;         /* S3 before the softmax, or NULL */
     const float *w_head;       /* S6 right after the softmax, or NULL */
     const float *w_kq_post;    /* P1 on the probabilities, or NULL */
     const float *w_head_post;  /* P2 after P1, or NULL */
+    const float *w_head_pre;   /* L1 on the logits, or NULL */
+    int exact_mask;            /* nonzero: S3 under Eq. (4)'s indicator */
 } mta_composition;
 
 /* Bytes of device workspace mta_forward_composed needs (0 on an invalid

@@ -150,6 +150,12 @@ def test_composed_launch_sequences_and_workspace(L):
                              "k_pv_groupnorm"],
         (None, None, None, None): ["k_logits", "k_softmax_mix", "k_pv_groupnorm"],
         (a, None, a, None): ["k_logits", "k_conv", "k_softmax_mix", "k_conv", "k_pv_groupnorm"],
+        # the pre-softmax head mix of the logits and the exact indicator of Eq. (4)
+        (a, None, None, None, a, 0): ["k_logits", "k_conv", "k_head_mix", "k_softmax_mix",
+                                      "k_pv_groupnorm"],
+        (a, a, a, a, a, 1): ["k_logits", "k_conv", "k_head_mix", "k_softmax_mix", "k_conv",
+                             "k_head_mix", "k_pv_groupnorm"],
+        (a, a, None, None, None, 1): ["k_logits", "k_conv", "k_softmax_mix", "k_pv_groupnorm"],
     }
     for ptrs, names in seqs.items():
         comp = C(*ptrs)
@@ -160,6 +166,8 @@ def test_composed_launch_sequences_and_workspace(L):
     default = C(a, a, None, None)
     assert mta.mta_composed_kernel_names(fused, default) == \
         [mta.mta_kernel_name(fused, i) for i in range(mta.mta_kernel_count(fused))]
+    # the default weights with the exact indicator leave the fused path
+    assert "k_mta_fused" not in mta.mta_composed_kernel_names(fused, C(a, a, None, None, None, 1))
     assert L.mta_composed_workspace_size(ctypes.byref(fused), ctypes.byref(default)) == \
         mta.mta_workspace_size(fused)
     assert L.mta_composed_workspace_size(ctypes.byref(fused), None) == 0
@@ -183,6 +191,7 @@ def test_composed_argument_checks(L):
     assert call(s, rep, gw=z) == -1
     assert call(s, rep, q=z) == -1
     assert call(s, C(1 << 20, 1 << 20, (1 << 20) + 8, None)) == -3
+    assert call(s, C(1 << 20, None, None, None, (1 << 20) + 4, 0)) == -3
     assert call(s, rep, gate=ctypes.c_void_p((1 << 20) + 2)) == -3
     assert call(s, rep, nbytes=need - 1) == -4
     assert call(s, rep, ws=z) == -1

@@ -1,5 +1,7 @@
 """Parity of the compositions of "Putting Everything Together: The Full MTA
-Module" (and the post-softmax variant of "Key-Query Convolution") on the GPU,
+Module" (with the post-softmax variant of "Key-Query Convolution", the
+pre-softmax head mix of "Head Mixing Convolution" and the exact indicator of
+Eq. (4)) on the GPU,
 called through mta_forward_composed, against the fp64 oracle's composed
 forward on the same inputs.
 
@@ -34,7 +36,7 @@ def to_device(x, io):
     dt = torch.bfloat16 if io == "bf16" else torch.float32
     dev = torch.device("cuda", 0)
     d = {n: torch.from_numpy(np.ascontiguousarray(x[n])).to(dev).to(dt) for n in ("q", "k", "v")}
-    for n in WEIGHTS + ("gn_weight", "gn_bias"):
+    for n in WEIGHTS + ("w_head_pre", "gn_weight", "gn_bias"):
         d[n] = None if x[n] is None else torch.from_numpy(np.ascontiguousarray(x[n])).to(dev)
     return d
 
@@ -43,7 +45,8 @@ def run(d, x, gate=None, events=None):
     out = mta.mta_forward_composed(d["q"], d["k"], d["v"], *(d[n] for n in WEIGHTS),
                                    gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
                                    depth_scale=x["depth_scale"], gate=gate,
-                                   gn_eps=x["gn_eps"], events=events)
+                                   gn_eps=x["gn_eps"], events=events, w_head_pre=d["w_head_pre"],
+                                   exact_mask=x["exact_mask"])
     mta.mta_sync_status()
     return out.float().cpu().numpy().astype(np.float64)
 
@@ -51,7 +54,8 @@ def run(d, x, gate=None, events=None):
 def oracle_full(x, gate=None):
     return oracle.forward_composed(x["q"], x["k"], x["v"], *(x[n] for n in WEIGHTS),
                                    x["gn_weight"], x["gn_bias"], x["depth_scale"],
-                                   gn_eps=x["gn_eps"], gate=gate)
+                                   gn_eps=x["gn_eps"], gate=gate, w_head_pre=x["w_head_pre"],
+                                   exact_mask=x["exact_mask"])
 
 
 @pytest.mark.parametrize("comp", sorted(COMPOSITIONS))
@@ -76,7 +80,8 @@ RAGGED = [
 ]
 
 
-@pytest.mark.parametrize("comp", ["repeat", "post_kq", "both_post"])
+@pytest.mark.parametrize("comp", ["repeat", "post_kq", "both_post", "exact_both_pre",
+                                  "exact_repeat"])
 @pytest.mark.parametrize("shape", RAGGED, ids=[str(s) for s in RAGGED])
 def test_ragged_shapes_elementwise(shape, comp):
     B, H, T, d, c_q, c_k, c_h, io = shape
@@ -99,6 +104,25 @@ def test_strong_post_kernels_and_gate():
     gate = np.array([-2.0, -0.5, 0.75, 3.0], dtype=np.float32)
     got = run(d, x, gate=torch.from_numpy(gate).cuda())
     assert_close(got, oracle_full(x, gate=gate), w.io, "strong gated")
+
+
+@pytest.mark.parametrize("comp", ["exact_both_pre", "exact_repeat"])
+def test_strong_kernels_exact_mask_and_logit_mix(comp):
+    """Kernels far from the identity in fp32, where the exact indicator of
+    Eq. (4) and the logit mix move the output far beyond the tolerance: the
+    GPU must match the oracle with them, and the oracle without the exact
+    mask must be far off (so that the test tells the two maskings apart)."""
+    w = Workload("strong_exact", 2, 4, 160, 64, 6, 11, 2, "f32", seed=33)
+    x = composed_inputs(w, comp)
+    rng = np.random.default_rng(34)
+    x["w_kq"] = (0.4 * rng.standard_normal(x["w_kq"].shape)).astype(np.float32)
+    if x["w_head_pre"] is not None:
+        x["w_head_pre"] = rng.standard_normal(x["w_head_pre"].shape).astype(np.float32)
+    got = run(to_device(x, w.io), x)
+    ref = oracle_full(x)
+    assert_close(got, ref, w.io, "strong " + comp)
+    two_pass = oracle_full(dict(x, exact_mask=False))
+    assert np.abs(two_pass - ref).max() > 100 * 1e-4
 
 
 def test_default_composition_is_mta_forward():
@@ -129,7 +153,7 @@ def test_traced_launches_follow_the_chain():
     assert_close(got, oracle_full(x), w.io, "traced")
 
 
-@pytest.mark.parametrize("comp", ["repeat", "both_post"])
+@pytest.mark.parametrize("comp", ["repeat", "both_post", "exact_both_pre"])
 def test_full_size_sampled_rows(comp):
     """The T = 4096 workload (two [B,H,T,T] fp32 maps, 4.3 GB) on rows
     sampled per batch entry, including tile edges and both ends."""
@@ -144,5 +168,6 @@ def test_full_size_sampled_rows(comp):
         rows = sample_rows(w.T, rng, n=6)
         ref = oracle.rows_composed(x["q"], x["k"], x["v"], *(x[n] for n in WEIGHTS),
                                    x["gn_weight"], x["gn_bias"], x["depth_scale"], b, rows,
-                                   gn_eps=x["gn_eps"])
+                                   gn_eps=x["gn_eps"], w_head_pre=x["w_head_pre"],
+                                   exact_mask=x["exact_mask"])
         assert_close(got[b, rows], ref, w.io, "longctx_4k %s b=%d" % (comp, b))

@@ -9,6 +9,7 @@ import subprocess
 import sys
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -81,20 +82,22 @@ def test_reference_arm_times_a_composition():
     assert d["config"]["composition"] == "repeat" and d["value"] > 0
 
 
-def test_oracle_units_are_slices_of_the_composed_forward():
+@pytest.mark.parametrize("name", ["repeat", "exact_both_pre"])
+def test_oracle_units_are_slices_of_the_composed_forward(name):
     # The CPU-baseline sample cuts (batch, head-group) units out of the
     # workload, post-softmax weights included; each unit's oracle output
     # is the matching slice of the whole problem's.
     import oracle
     from convolved_logit_attention_b200.workloads import COMPOSITIONS, composed_inputs
     w = WORKLOADS["tiny_f32"]
-    x = composed_inputs(w, "repeat")
-    flops = w.composition_flops(COMPOSITIONS["repeat"])
+    x = composed_inputs(w, name)
+    flops = w.composition_flops(COMPOSITIONS[name])
     units, f = bench.oracle_sample(w, x, 2, flops)
     assert f == 2 * flops // (w.B * w.G)
     full = oracle.forward_composed(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["w_kq_post"],
-                                   x["w_head_post"], x["gn_weight"], x["gn_bias"], w.depth_scale)
+                                   x["w_head_post"], x["gn_weight"], x["gn_bias"], w.depth_scale,
+                                   w_head_pre=x["w_head_pre"], exact_mask=x["exact_mask"])
     for g, u in enumerate(units):
-        part = oracle.forward_composed(*u[:7], u[7], u[8], w.depth_scale)
+        part = bench.run_oracle_unit(u, w)
         cs = slice(g * w.c_h * w.d, (g + 1) * w.c_h * w.d)
         np.testing.assert_array_equal(part[0], full[0, :, cs])
