@@ -25,7 +25,8 @@ class _Shape(ctypes.Structure):
 class _Composition(ctypes.Structure):
     _fields_ = [("w_kq", ctypes.c_void_p), ("w_head_pre", ctypes.c_void_p),
                 ("w_head", ctypes.c_void_p), ("w_kq_post", ctypes.c_void_p),
-                ("w_head_post", ctypes.c_void_p), ("exact_mask", ctypes.c_int)]
+                ("w_head_post", ctypes.c_void_p), ("exact_mask", ctypes.c_int),
+                ("w_kq_3d", ctypes.c_void_p)]
 
 
 _lib = None
@@ -178,22 +179,28 @@ def stages(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, b=0, gn_eps=1
     return {"C": C, "P": P, "A": A, "O": O, "out": out}
 
 
-def _composed(q, ws, exact_mask, gn_eps):
+def _composed(q, ws, exact_mask, gn_eps, w3=None):
     """Shape and C struct of a composition.  ws = (w_kq, w_head_pre, w_head,
-    w_kq_post, w_head_post), float64 arrays or None: (c_q, c_k) from the
-    key-query kernels (both [H, c_q, c_k] when both are given), c_h from the
-    head mixes (1 when there is none)."""
+    w_kq_post, w_head_post), float64 arrays or None, and w3 the 3-D kernel
+    [H/c_h, c_h, c_h, c_q, c_k] or None: (c_q, c_k) from the key-query
+    kernels (all alike), c_h from the head mixes or the 3-D kernel (1 when
+    there is none)."""
     B, H, T, d = q.shape
     kq = [w for w in (ws[0], ws[3]) if w is not None]
     hm = [w for w in (ws[1], ws[2], ws[4]) if w is not None]
-    c_q, c_k = kq[0].shape[1:] if kq else (1, 1)
-    c_h = hm[0].shape[-1] if hm else 1
+    if w3 is not None:
+        c_h, c_q, c_k = w3.shape[2:]
+    else:
+        c_q, c_k = kq[0].shape[1:] if kq else (1, 1)
+        c_h = hm[0].shape[-1] if hm else 1
     for w in kq:
         assert w.shape == (H, c_q, c_k), w.shape
     for w in hm:
         assert w.shape == (H // c_h, c_h, c_h), w.shape
+    if w3 is not None:
+        assert w3.shape == (H // c_h, c_h, c_h, c_q, c_k), w3.shape
     comp = _Composition(*[None if w is None else w.ctypes.data for w in ws],
-                        int(bool(exact_mask)))
+                        int(bool(exact_mask)), None if w3 is None else w3.ctypes.data)
     return _shape(B, H, T, d, c_q, c_k, c_h, gn_eps), comp
 
 
@@ -204,17 +211,19 @@ def _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post):
 
 def forward_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
                      depth_scale, gn_eps=1e-5, nthreads=0, gate=None, w_head_pre=None,
-                     exact_mask=False):
+                     exact_mask=False, w_kq_3d=None):
     """out[B, T, H*d] of a composition of "Putting Everything Together": the
     steps Mask_0, [key-query conv w_kq], [head mix of the logits
     w_head_pre], Mask_-inf, softmax, [head mix w_head], [key-query conv
     w_kq_post on the probabilities, Mask_0], [head mix w_head_post], A V,
     GroupNorm, scale; a bracketed step whose weights are None is left out.
     exact_mask: the w_kq conv uses Eq. (4)'s indicator instead of Mask_0.
-    gate as in forward."""
+    w_kq_3d [H/c_h, c_h, c_h, c_q, c_k]: the 3-D conv over (query, key,
+    head) in place of w_kq.  gate as in forward."""
     q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
     ws = _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post)
-    s, comp = _composed(q, ws, exact_mask, gn_eps)
+    w3 = None if w_kq_3d is None else _f64(w_kq_3d)
+    s, comp = _composed(q, ws, exact_mask, gn_eps, w3)
     g = None if gate is None else _f64(gate)
     out = np.empty((s.B, s.T, s.H * s.d), dtype=np.float64)
     rc = _load().mta_oracle_forward_composed(ctypes.byref(s), _ptr(q), _ptr(k), _ptr(v),
@@ -228,11 +237,12 @@ def forward_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, g
 
 def rows_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
                   depth_scale, b, row_idx, gn_eps=1e-5, nthreads=0, gate=None,
-                  w_head_pre=None, exact_mask=False):
+                  w_head_pre=None, exact_mask=False, w_kq_3d=None):
     """out[b, row_idx, :] of forward_composed, one row at a time."""
     q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
     ws = _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post)
-    s, comp = _composed(q, ws, exact_mask, gn_eps)
+    w3 = None if w_kq_3d is None else _f64(w_kq_3d)
+    s, comp = _composed(q, ws, exact_mask, gn_eps, w3)
     g = None if gate is None else _f64(gate)
     idx = np.ascontiguousarray(np.asarray(row_idx, dtype=np.int32))
     out = np.empty((idx.size, s.H * s.d), dtype=np.float64)
@@ -248,14 +258,15 @@ def rows_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_b
 
 def stages_composed(q, k, v, w_kq, w_head, w_kq_post, w_head_post, gn_weight, gn_bias,
                     depth_scale, b=0, gn_eps=1e-5, gate=None, w_head_pre=None,
-                    exact_mask=False):
+                    exact_mask=False, w_kq_3d=None):
     """Intermediates of forward_composed for batch entry b (small T only):
     C [H,T,T] softmax input (after both masks and the logit mix), P [H,T,T]
     softmax, A1 [H,T,T] after the first head mix, A [H,T,T] the attention
     that meets V, O [H,T,d] pre-normalisation head outputs, out [T, H*d]."""
     q, k, v, gw, gb = map(_f64, (q, k, v, gn_weight, gn_bias))
     ws = _weights(w_kq, w_head_pre, w_head, w_kq_post, w_head_post)
-    s, comp = _composed(q, ws, exact_mask, gn_eps)
+    w3 = None if w_kq_3d is None else _f64(w_kq_3d)
+    s, comp = _composed(q, ws, exact_mask, gn_eps, w3)
     g = None if gate is None else _f64(gate)
     H, T, d = s.H, s.T, s.d
     C, P, A1, A = (np.empty((H, T, T)) for _ in range(4))

@@ -40,6 +40,10 @@
  *          separable case of the 3-D convolution over (query, key, head).
  *   [HMPRE] same page, "Head Mixing Convolution", pre-softmax version: the
  *          logits of a group's heads are mixed, A^h_new = sum_h' w A^h'.
+ *   [CONV3D] same page, "Putting Everything Together", "Both pre-softmax
+ *          (3D convolution view)": one kernel over (query, key, head) per
+ *          group, C^h[i][j] = sum_{h' in group} sum_{i',j'}
+ *          theta3[h][h'][i'][j'] A0^{h'}[i-i'][j-j'].
  *   [EXACT] same page, Eq. (4): the tap (i', j') of output (i, j) adds
  *          theta q_{i-i'} k_{j-j'}^T / sqrt(d) whenever key j - j' <= i (the
  *          indicator 1_{i >= j-j'}), which Eq. (5)'s two-pass masking
@@ -82,6 +86,7 @@ typedef struct {
     const double *w_kq;        /* key-query kernel before the softmax, or NULL */
     const double *w_head_pre;  /* head mix of the logits before the softmax, or NULL */
     int exact;                 /* [EXACT] masking of the first conv instead of [KQ5] */
+    const double *w_kq_3d;     /* [CONV3D] kernel in place of w_kq, or NULL */
     const double *w_head;      /* head mix right after the softmax, or NULL */
     const double *w_kq_post;   /* key-query kernel on the probabilities, or NULL */
     const double *w_head_post; /* head mix after w_kq_post, or NULL */
@@ -233,6 +238,7 @@ typedef struct {
     double *ring1;  /* [c_h][c_q][T] first-stage attention rows A1, the same ring */
     double *C;      /* [c_h][T] softmax inputs before the logit mix */
     double *Cm;     /* [c_h][T] after the logit mix [HMPRE] */
+    double *Ct;     /* [T] one input head's conv under [CONV3D] */
     double *P;      /* [c_h][T] softmax rows of the group's heads */
     double *A1;     /* [c_h][T] first-stage rows (after the first head mix) */
     double *A2;     /* [c_h][T] after the post-softmax key-query conv */
@@ -250,6 +256,7 @@ static int alloc_unit(const mta_oracle_shape *s, unit_buffers *u)
     u->ring1 = (double *)calloc(hq * T, sizeof(double));
     u->C = (double *)malloc(hT * sizeof(double));
     u->Cm = (double *)malloc(hT * sizeof(double));
+    u->Ct = (double *)malloc(T * sizeof(double));
     u->P = (double *)malloc(hT * sizeof(double));
     u->A1 = (double *)malloc(hT * sizeof(double));
     u->A2 = (double *)malloc(hT * sizeof(double));
@@ -258,13 +265,13 @@ static int alloc_unit(const mta_oracle_shape *s, unit_buffers *u)
     u->zero = (double *)calloc(T, sizeof(double));
     u->rows0 = (double **)malloc(hq * sizeof(double *));
     u->rows1 = (double **)malloc(hq * sizeof(double *));
-    return u->ring0 && u->ring1 && u->C && u->Cm && u->P && u->A1 && u->A2 && u->A3 && u->O &&
+    return u->ring0 && u->ring1 && u->C && u->Cm && u->Ct && u->P && u->A1 && u->A2 && u->A3 && u->O &&
            u->zero && u->rows0 && u->rows1;
 }
 
 static void free_unit(unit_buffers *u)
 {
-    free(u->ring0); free(u->ring1); free(u->C); free(u->Cm); free(u->P); free(u->A1); free(u->A2);
+    free(u->ring0); free(u->ring1); free(u->C); free(u->Cm); free(u->Ct); free(u->P); free(u->A1); free(u->A2);
     free(u->A3); free(u->O); free(u->zero); free(u->rows0); free(u->rows1);
 }
 
@@ -280,7 +287,8 @@ typedef struct {
 
 /* Query row r of group g up to the first head mix.  rows0[hh*c_q + ip] is
  * A0[r - ip] of head g*c_h + hh.  [KQ5] per head: the key-query conv with
- * w_kq when given (else A0[r] itself) and Mask_-inf; [HMPRE] with
+ * w_kq, or the [CONV3D] kernel over the group's heads, when given (else
+ * A0[r] itself) and Mask_-inf; [HMPRE] with
  * w_head_pre when given; softmax; then [HM7] with w_head when given.
  * Leaves the group's rows in u->A1. */
 static void first_stage(const mta_oracle_shape *s, const mta_oracle_args *a, int g, int r,
@@ -291,7 +299,14 @@ static void first_stage(const mta_oracle_shape *s, const mta_oracle_args *a, int
         int h = g * c_h + hh;
         double *const *rows = rows0 + (size_t)hh * c_q;
         double *C = u->C + (size_t)hh * T;
-        if (a->w_kq)
+        if (a->w_kq_3d) {
+            for (int j = 0; j < T; ++j) C[j] = (j <= r) ? 0.0 : -INFINITY;
+            for (int hi = 0; hi < c_h; ++hi) {      /* every input head of the group */
+                const double *th3 = a->w_kq_3d + ((size_t)h * c_h + hi) * c_q * c_k;
+                conv2d_row(s, th3, r, rows0 + (size_t)hi * c_q, a->exact, -INFINITY, u->Ct);
+                for (int j = 0; j <= r && j < T; ++j) C[j] += u->Ct[j];
+            }
+        } else if (a->w_kq)
             conv2d_row(s, a->w_kq + (size_t)h * c_q * c_k, r, rows, a->exact, -INFINITY, C);
         else
             for (int j = 0; j < T; ++j) C[j] = (j <= r) ? rows[0][j] : -INFINITY;
@@ -512,6 +527,8 @@ typedef struct {
     const double *w_kq_post;   /* [H][c_q][c_k] [POST] conv of the probabilities */
     const double *w_head_post; /* [H/c_h][c_h][c_h] [HM7] mix after w_kq_post */
     int exact_mask;            /* nonzero: [EXACT] masking of the w_kq conv */
+    const double *w_kq_3d;     /* [H/c_h][c_h][c_h][c_q][c_k] [CONV3D] kernel, in place
+                                  of w_kq (giving both is an error) */
 } mta_oracle_composition;
 
 static mta_oracle_args composed_args(const double *q, const double *k, const double *v,
@@ -525,6 +542,7 @@ static mta_oracle_args composed_args(const double *q, const double *k, const dou
     a.exact = c->exact_mask != 0;
     a.w_kq_post = c->w_kq_post;
     a.w_head_post = c->w_head_post;
+    a.w_kq_3d = c->w_kq_3d;
     return a;
 }
 
@@ -557,7 +575,7 @@ int mta_oracle_forward_composed(const mta_oracle_shape *s, const double *q, cons
                                 double depth_scale, const double *gate, double *out,
                                 int nthreads)
 {
-    if (!c) return -1;
+    if (!c || (c->w_kq && c->w_kq_3d)) return -1;
     mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return forward_args(s, &a, out, nthreads);
 }
@@ -590,7 +608,7 @@ int mta_oracle_rows_composed(const mta_oracle_shape *s, const double *q, const d
                              double depth_scale, const double *gate, int b,
                              const int *rows_idx, int nrows, double *out_rows, int nthreads)
 {
-    if (!c) return -1;
+    if (!c || (c->w_kq && c->w_kq_3d)) return -1;
     mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return rows_args(s, &a, b, rows_idx, nrows, out_rows, nthreads);
 }
@@ -623,7 +641,7 @@ int mta_oracle_stages_composed(const mta_oracle_shape *s, const double *q, const
                                double depth_scale, const double *gate, int b, double *C,
                                double *P, double *A1, double *A, double *O, double *out)
 {
-    if (!c) return -1;
+    if (!c || (c->w_kq && c->w_kq_3d)) return -1;
     mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return stages_args(s, &a, b, C, P, A1, A, O, out);
 }

@@ -399,3 +399,99 @@ def test_pre_softmax_rows_and_forward_agree(name):
     for b in range(shape[0]):
         r = call_pre(oracle.rows_composed, q, k, v, ws, exact, gw, gb, 0.8, b=b, row_idx=idx)
         np.testing.assert_allclose(r, out[b, idx], rtol=0, atol=1e-13)
+
+
+def conv3d_brute_force(q, k, v, th3, w, gw, gb, depth, exact=False, eps=1e-5):
+    """ "Both pre-softmax (3D convolution view)": C^h = sum over the group's
+    input heads h' of the 2-D conv (scipy, or the indicator form of Eq. (4))
+    of head h''s logits with theta3[h][h'], then Mask_-inf, softmax, the
+    post-softmax mix w (or none), A V, GroupNorm."""
+    B, H, T, d = q.shape
+    G, c_h = th3.shape[:2]
+    causal = np.tril(np.ones((T, T), dtype=bool))
+    Afull = np.einsum("bhie,bhje->bhij", q, k) / np.sqrt(d)
+    A0 = np.where(causal, Afull, 0.0)
+    C = np.zeros_like(Afull)
+    for g in range(G):
+        for ho in range(c_h):
+            for hi in range(c_h):
+                src = slice(g * c_h + hi, g * c_h + hi + 1)
+                kern = th3[g, ho, hi][None]
+                part = indicator_conv(Afull[:, src], kern) if exact else true_conv2d(A0[:, src], kern)
+                C[:, g * c_h + ho] += part[:, 0]
+    C = np.where(causal, C, -np.inf)
+    P = scipy.special.softmax(C, axis=-1)
+    A = mix(P, w) if w is not None else P
+    O = A @ v
+    Y = F.group_norm(torch.as_tensor(O).permute(0, 2, 1, 3).reshape(B * T, H * d), H,
+                     torch.as_tensor(gw), torch.as_tensor(gb), eps).numpy().reshape(B, T, H * d)
+    return {"C": C, "P": P, "A": A, "O": O, "out": depth * Y}
+
+
+@pytest.mark.parametrize("exact", [False, True])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_conv3d_matches_brute_force(shape, exact):
+    rng = np.random.default_rng(zlib.crc32(repr((shape, exact, "3d")).encode()))
+    B, H, T, d, c_q, c_k, c_h = shape
+    q, k, v, _, w, gw, gb = rand_inputs(rng, *shape)
+    th3 = 0.3 * rng.standard_normal((H // c_h, c_h, c_h, c_q, c_k))
+    use_w = w if shape[1] != 3 else None       # with and without the post-softmax mix
+    ref = conv3d_brute_force(q, k, v, th3, use_w, gw, gb, 0.7, exact=exact)
+    out = oracle.forward_composed(q, k, v, None, use_w, None, None, gw, gb, 0.7, w_kq_3d=th3,
+                                  exact_mask=exact)
+    np.testing.assert_allclose(out, ref["out"], rtol=0, atol=1e-11)
+    st = oracle.stages_composed(q, k, v, None, use_w, None, None, gw, gb, 0.7, b=0, w_kq_3d=th3,
+                                exact_mask=exact)
+    live = np.isfinite(ref["C"][0])
+    assert np.array_equal(live, np.isfinite(st["C"]))
+    np.testing.assert_allclose(st["C"][live], ref["C"][0][live], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(st["O"], ref["O"][0], rtol=0, atol=1e-11)
+
+
+def test_conv3d_single_cross_head_tap():
+    # A 3-D kernel whose one non-zero tap is theta3[out 0][in 1][i'][j'] = 1:
+    # head 0's logits are head 1's masked logits shifted by (i', j') (Mask_0
+    # zeros, not -inf, where that pair is not causal), and head 1's live
+    # logits are all zero, so its attention is uniform over j <= i.
+    rng = np.random.default_rng(50)
+    H, T, d, c_q, c_k = 2, 12, 5, 3, 5
+    q, k, v = (rng.standard_normal((1, H, T, d)) for _ in range(3))
+    gw, gb = np.ones(H * d), np.zeros(H * d)
+    for ip, jj in ((0, 2), (2, 0), (1, 4)):
+        jp = jj - c_k // 2
+        th3 = np.zeros((1, 2, 2, c_q, c_k)); th3[0, 0, 1, ip, jj] = 1.0
+        st = oracle.stages_composed(q, k, v, None, None, None, None, gw, gb, 1.0, w_kq_3d=th3)
+        for i in range(T):
+            for j in range(i + 1):
+                r, c = i - ip, j - jp
+                want = float(q[0, 1, r] @ k[0, 1, c]) / np.sqrt(d) if (0 <= r and 0 <= c <= r) \
+                    else 0.0
+                assert abs(st["C"][0, i, j] - want) < 1e-12, (ip, jp, i, j)
+                assert st["C"][1, i, j] == 0.0
+            np.testing.assert_allclose(st["P"][1, i, : i + 1], 1.0 / (i + 1), rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("exact", [False, True])
+def test_separable_conv3d_is_conv_then_logit_mix(exact):
+    # theta3[h][h'] = w_pre[h][h'] theta_{h'} makes the 3-D conv the key-query
+    # conv followed by the pre-softmax head mix (the factorisation of the
+    # 3-D view); a block-diagonal theta3 is the plain key-query conv.
+    rng = np.random.default_rng(51)
+    shape = (2, 4, 21, 8, 4, 5, 2)
+    B, H, T, d, c_q, c_k, c_h = shape
+    q, k, v, th, w, gw, gb = rand_inputs(rng, *shape)
+    w_pre = rng.standard_normal(w.shape)
+    G = H // c_h
+    th3 = np.einsum("goi,gicd->goicd", w_pre, th.reshape(G, c_h, c_q, c_k))
+    a = oracle.forward_composed(q, k, v, None, w, None, None, gw, gb, 0.8, w_kq_3d=th3,
+                                exact_mask=exact)
+    b = oracle.forward_composed(q, k, v, th, w, None, None, gw, gb, 0.8, w_head_pre=w_pre,
+                                exact_mask=exact)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    diag = np.einsum("oi,gicd->goicd", np.eye(c_h), th.reshape(G, c_h, c_q, c_k))
+    c = oracle.forward_composed(q, k, v, None, w, None, None, gw, gb, 0.8, w_kq_3d=diag,
+                                exact_mask=exact)
+    e = oracle.forward_composed(q, k, v, th, w, None, None, gw, gb, 0.8, exact_mask=exact)
+    np.testing.assert_allclose(c, e, rtol=0, atol=1e-13)
+    with pytest.raises(RuntimeError):
+        oracle.forward_composed(q, k, v, th, w, None, None, gw, gb, 0.8, w_kq_3d=th3)

@@ -60,6 +60,11 @@ MUTATIONS = [
      "if (exact && c > i - ip) continue;"),
     ("exact rows without the keys past the query", "const int last = a->exact ? r + s->c_q - 1 : r;",
      "const int last = a->exact ? r + s->c_q - 2 : r;"),
+    # the 3-D convolution over (query, key, head)
+    ("3-D conv reads the output head's own logits", "rows0 + (size_t)hi * c_q, a->exact",
+     "rows0 + (size_t)hh * c_q, a->exact"),
+    ("3-D kernel indexed [in][out]", "a->w_kq_3d + ((size_t)h * c_h + hi)",
+     "a->w_kq_3d + (((size_t)g * c_h + hi) * c_h + hh)"),
 ]
 
 PIN_CHECKS = [
@@ -83,6 +88,8 @@ PIN_CHECKS = [
     lambda: cpins.test_exact_indicator_single_tap_closed_form(3, 5),
     cpins.test_logit_mix_is_softmax_of_mixed_logits,
     lambda: cpins.test_pre_softmax_rows_and_forward_agree("exact_everything"),
+    lambda: [cpins.test_conv3d_matches_brute_force(cpins.SHAPES[1], e) for e in (False, True)],
+    cpins.test_conv3d_single_cross_head_tap,
 ]
 
 
