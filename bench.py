@@ -181,15 +181,15 @@ WEIGHTS = ("w_kq", "w_head", "w_kq_post", "w_head_post")   # positional order of
 
 def compose_kw(args, d):
     """Keyword arguments of mta_forward_composed beyond the four positional
-    weights: the logit mix and the exact-mask flag of the composition."""
-    return {"w_head_pre": d.get("w_head_pre"),
+    weights: the logit mix, the 3-D kernel and the exact-mask flag."""
+    return {"w_head_pre": d.get("w_head_pre"), "w_kq_3d": d.get("w_kq_3d"),
             "exact_mask": bool(COMPOSITIONS[args.compose].get("exact_mask"))}
 
 
 def device_inputs(x, io, device):
     dt = torch.bfloat16 if io == "bf16" else torch.float32
     d = {n: torch.from_numpy(x[n]).to(device).to(dt) for n in ("q", "k", "v")}
-    for n in WEIGHTS + ("w_head_pre", "gn_weight", "gn_bias"):
+    for n in WEIGHTS + ("w_head_pre", "w_kq_3d", "gn_weight", "gn_bias"):
         d[n] = torch.from_numpy(x[n]).to(device) if x.get(n) is not None else None
     return d
 
@@ -199,14 +199,26 @@ def step_flops(args, w):
         else w.algorithmic_flops()
 
 
-def kernel_units(name, w):
+def conv_heads_per_launch(comp):
+    """Input heads per k_conv launch, averaged over a composition's k_conv
+    launches: c_h for the 3-D kernel, 1 for every 2-D one."""
+    if not comp:
+        return 1.0
+    per = [comp["c_h"]] if comp.get("w_kq_3d") else ([1] if comp.get("w_kq") else [])
+    per += [1] if comp.get("w_kq_post") else []
+    return sum(per) / len(per) if per else 1.0
+
+
+def kernel_units(name, w, comp=None):
     """(bound, algorithmic amount per launch, unit) for each kernel the
-    library launches on workload w.  L = T(T+1)/2 live logits per (b, h)."""
+    library launches on workload w (comp: the composition's steps, with
+    c_h, when one is timed).  L = T(T+1)/2 live logits per (b, h)."""
     logits = w.B * w.H * w.live_logits()
     io_bytes = 2 if w.io == "bf16" else 4
+    conv = logits * 2 * w.c_q * w.c_k * conv_heads_per_launch(comp)
     table = {
         "k_logits": ("alu", logits * 2 * w.d, "FLOP"),
-        "k_conv": ("alu", logits * 2 * w.c_q * w.c_k, "FLOP"),
+        "k_conv": ("alu", conv, "FLOP"),
         "k_softmax_mix": ("hbm", logits * 8, "B"),            # read C, write A_new (fp32)
         "k_head_mix": ("hbm", logits * 8, "B"),               # read and write one fp32 map
         "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
@@ -243,8 +255,8 @@ def load_traffic():
     return out
 
 
-def roofline(name, w, avg_ms, peaks, peak_src):
-    bound, amount, unit = kernel_units(name, w)
+def roofline(name, w, avg_ms, peaks, peak_src, comp=None):
+    bound, amount, unit = kernel_units(name, w, comp)
     secs = avg_ms / 1e3
     traffic = load_traffic().get(name)
     tr_bytes = None
@@ -271,7 +283,7 @@ def time_mta(args, w, d, world, device):
     if args.compose:
         kw = compose_kw(args, d)
         shape = mta.composed_shape(d["q"], *(d[n] for n in WEIGHTS), gn_eps=w.gn_eps,
-                                   w_head_pre=kw["w_head_pre"])
+                                   w_head_pre=kw["w_head_pre"], w_kq_3d=kw["w_kq_3d"])
         comp = mta.composition(*(d[n] for n in WEIGHTS), **kw)
         names = mta.mta_composed_kernel_names(shape, comp)
         nk = len(names)
@@ -370,7 +382,8 @@ def time_e2e(args, w, x, device):
     first input copy of the timed steps to the end of their last output copy."""
     import convolved_logit_attention_b200 as mta
     dt = torch.bfloat16 if w.io == "bf16" else torch.float32
-    names = tuple(n for n in ("q", "k", "v") + WEIGHTS + ("w_head_pre", "gn_weight", "gn_bias")
+    names = tuple(n for n in ("q", "k", "v") + WEIGHTS + ("w_head_pre", "w_kq_3d", "gn_weight",
+                                                         "gn_bias")
                   if x.get(n) is not None)
     host = {n: torch.from_numpy(x[n]).to(dt).pin_memory() for n in ("q", "k", "v")}
     for n in names[3:]:
@@ -382,7 +395,8 @@ def time_e2e(args, w, x, device):
     if args.compose:
         wts = [dev[0].get(n) for n in WEIGHTS]
         kw = compose_kw(args, dev[0])
-        shape = mta.composed_shape(dev[0]["q"], *wts, gn_eps=w.gn_eps, w_head_pre=kw["w_head_pre"])
+        shape = mta.composed_shape(dev[0]["q"], *wts, gn_eps=w.gn_eps, w_head_pre=kw["w_head_pre"],
+                                   w_kq_3d=kw["w_kq_3d"])
         ws_bytes = mta.lib().mta_composed_workspace_size(
             ctypes.byref(shape), ctypes.byref(mta.composition(*wts, **kw)))
     else:
@@ -457,6 +471,7 @@ def oracle_sample(w, x, n_units, flops_per_step):
                       "v": x["v"][b:b + 1, hs], "w_kq": part("w_kq", hs),
                       "w_head_pre": part("w_head_pre", gs), "w_head": part("w_head", gs),
                       "w_kq_post": part("w_kq_post", hs), "w_head_post": part("w_head_post", gs),
+                      "w_kq_3d": part("w_kq_3d", gs),
                       "gn_weight": x["gn_weight"][cs], "gn_bias": x["gn_bias"][cs],
                       "exact_mask": bool(x.get("exact_mask"))})
     flops = len(units) * flops_per_step // (w.B * w.G)
@@ -466,14 +481,16 @@ def oracle_sample(w, x, n_units, flops_per_step):
 def run_oracle_unit(u, w, nthreads=1):
     import oracle
     default = (u["w_kq"] is not None and u["w_head"] is not None and u["w_head_pre"] is None
-               and u["w_kq_post"] is None and u["w_head_post"] is None and not u["exact_mask"])
+               and u["w_kq_post"] is None and u["w_head_post"] is None and not u["exact_mask"]
+               and u["w_kq_3d"] is None)
     if default:
         return oracle.forward(u["q"], u["k"], u["v"], u["w_kq"], u["w_head"], u["gn_weight"],
                               u["gn_bias"], w.depth_scale, gn_eps=w.gn_eps, nthreads=nthreads)
     return oracle.forward_composed(u["q"], u["k"], u["v"], u["w_kq"], u["w_head"], u["w_kq_post"],
                                    u["w_head_post"], u["gn_weight"], u["gn_bias"], w.depth_scale,
                                    gn_eps=w.gn_eps, nthreads=nthreads,
-                                   w_head_pre=u["w_head_pre"], exact_mask=u["exact_mask"])
+                                   w_head_pre=u["w_head_pre"], exact_mask=u["exact_mask"],
+                                   w_kq_3d=u["w_kq_3d"])
 
 
 def run_oracle_units(units, w, nthreads):
@@ -554,7 +571,8 @@ def mta_arm(args, w, world, rank, local):
     kernels = dict(res["per_kernel_ms"])   # average ms per launch, traced pass
     # the dominant kernel by device time per step (a name may launch twice)
     dom = max(kernels, key=lambda n: kernels[n] * res["names"].count(n))
-    rl = roofline(dom, w, kernels[dom], peaks, peak_src)
+    comp = dict(COMPOSITIONS[args.compose], c_h=w.c_h) if args.compose else None
+    rl = roofline(dom, w, kernels[dom], peaks, peak_src, comp)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -569,7 +587,7 @@ def mta_arm(args, w, world, rank, local):
             "roofline": {k: rl[k] for k in ("bound", "achieved", "peak", "unit", "frac",
                                              "traffic")},
             "roofline_detail": rl,
-            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src),
+            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src, comp),
                              launches_per_step=res["names"].count(n))
                         for n in dict.fromkeys(res["names"])],
             "gpu_launches": res["launches"], "clocks": res["clocks"]}

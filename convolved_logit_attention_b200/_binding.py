@@ -44,7 +44,8 @@ class MtaShape(ctypes.Structure):
 class MtaComposition(ctypes.Structure):
     _fields_ = [("w_kq", ctypes.c_void_p), ("w_head", ctypes.c_void_p),
                 ("w_kq_post", ctypes.c_void_p), ("w_head_post", ctypes.c_void_p),
-                ("w_head_pre", ctypes.c_void_p), ("exact_mask", ctypes.c_int)]
+                ("w_head_pre", ctypes.c_void_p), ("exact_mask", ctypes.c_int),
+                ("w_kq_3d", ctypes.c_void_p)]
 
 
 class MtaError(RuntimeError):
@@ -307,22 +308,31 @@ def mta_sync_status(stream=None, device=None):
 
 
 def composition(w_kq=None, w_head=None, w_kq_post=None, w_head_post=None, w_head_pre=None,
-                exact_mask=False) -> MtaComposition:
+                exact_mask=False, w_kq_3d=None) -> MtaComposition:
     """The C struct of a composition; the tensors must outlive its use."""
     ptrs = [t.data_ptr() if t is not None else None
             for t in (w_kq, w_head, w_kq_post, w_head_post, w_head_pre)]
-    return MtaComposition(*ptrs, int(bool(exact_mask)))
+    return MtaComposition(*ptrs, int(bool(exact_mask)),
+                          w_kq_3d.data_ptr() if w_kq_3d is not None else None)
 
 
 def composed_shape(q, w_kq=None, w_head=None, w_kq_post=None, w_head_post=None,
-                   gn_eps=1e-5, w_head_pre=None) -> MtaShape:
+                   gn_eps=1e-5, w_head_pre=None, w_kq_3d=None) -> MtaShape:
     """Shape of a composition: (c_q, c_k) from the key-query kernels (equal
-    when both are given), c_h from the head mixes (1 when there is none)."""
+    when both are given), c_h from the head mixes or the 3-D kernel (1 when
+    there is none)."""
     B, H, T, d = q.shape
     kq = [w for w in (w_kq, w_kq_post) if w is not None]
     hm = [w for w in (w_head_pre, w_head, w_head_post) if w is not None]
-    c_q, c_k = tuple(kq[0].shape[1:]) if kq else (1, 1)
-    c_h = hm[0].shape[-1] if hm else 1
+    if w_kq_3d is not None:
+        if w_kq_3d.dim() != 5:
+            raise ValueError("w_kq_3d must be [H/c_h, c_h, c_h, c_q, c_k]")
+        c_h, c_q, c_k = tuple(w_kq_3d.shape[2:])
+        if tuple(w_kq_3d.shape) != (H // c_h, c_h, c_h, c_q, c_k) or H % c_h:
+            raise ValueError("w_kq_3d must be [H/c_h, c_h, c_h, c_q, c_k]")
+    else:
+        c_q, c_k = tuple(kq[0].shape[1:]) if kq else (1, 1)
+        c_h = hm[0].shape[-1] if hm else 1
     for w in kq:
         if w.dim() != 3 or tuple(w.shape) != (H, c_q, c_k):
             raise ValueError("key-query kernels must both be [H, c_q, c_k]")
@@ -341,13 +351,13 @@ def mta_composed_kernel_names(shape: MtaShape, comp: MtaComposition):
 def mta_forward_composed(q, k, v, w_kq=None, w_head=None, w_kq_post=None, w_head_post=None,
                          gn_weight=None, gn_bias=None, depth_scale=1.0, gate=None, out=None,
                          workspace=None, stream=None, gn_eps=1e-5, events=None,
-                         w_head_pre=None, exact_mask=False):
+                         w_head_pre=None, exact_mask=False, w_kq_3d=None):
     """Forward of one composition of the module (see mta_composition in
     include/mta.h): weights left as None are steps left out.  gate (float32
     [H]) replaces the depth scale by sigmoid(gate[h]).  With events (a list
     of torch.cuda.Event, two per launch) the traced entry records them
     around the launches.  Returns out [B, T, H*d]."""
-    ws_ = [w_kq, w_head, w_kq_post, w_head_post, w_head_pre]
+    ws_ = [w_kq, w_head, w_kq_post, w_head_post, w_head_pre, w_kq_3d]
     if q.device.type != "cuda":
         raise ValueError("inputs must be CUDA tensors")
     for name, t in (("k", k), ("v", v)):
@@ -365,8 +375,8 @@ def mta_forward_composed(q, k, v, w_kq=None, w_head=None, w_kq_post=None, w_head
         raise ValueError("gn_weight and gn_bias must have H*d elements")
     if gate is not None and gate.shape != (H,):
         raise ValueError("gate must be [H]")
-    shape = composed_shape(q, *ws_[:4], gn_eps=gn_eps, w_head_pre=w_head_pre)
-    comp = composition(*ws_, exact_mask=exact_mask)
+    shape = composed_shape(q, *ws_[:4], gn_eps=gn_eps, w_head_pre=w_head_pre, w_kq_3d=w_kq_3d)
+    comp = composition(*ws_[:5], exact_mask=exact_mask, w_kq_3d=w_kq_3d)
     if out is None:
         out = torch.empty((B, T, H * d), dtype=q.dtype, device=q.device)
     elif (out.shape != (B, T, H * d) or out.dtype != q.dtype or out.device != q.device

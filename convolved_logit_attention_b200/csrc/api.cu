@@ -142,7 +142,7 @@ namespace {
 bool is_default_composition(const mta_composition *c)
 {
     return c->w_kq && c->w_head && !c->w_kq_post && !c->w_head_post && !c->w_head_pre &&
-           !c->exact_mask;
+           !c->exact_mask && !c->w_kq_3d;
 }
 
 mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const void *v,
@@ -150,7 +150,7 @@ mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const
                          float depth_scale, const float *gate, void *out, void *workspace,
                          size_t workspace_bytes, void *stream, void *const *events, int n_events)
 {
-    if (!c) return MTA_ERR_INVALID_ARG;
+    if (!c || (c->w_kq && c->w_kq_3d)) return MTA_ERR_INVALID_ARG;
     if (gate && ((uintptr_t)gate & 3u) != 0) return MTA_ERR_ALIGNMENT;
     if (is_default_composition(c))
         return forward_impl(0, s, q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias, depth_scale,
@@ -162,14 +162,16 @@ mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const
         if (!p) return MTA_ERR_INVALID_ARG;
     for (const void *p : need)
         if (!aligned(p, 16)) return MTA_ERR_ALIGNMENT;
-    const void *opt[] = {c->w_kq, c->w_head, c->w_kq_post, c->w_head_post, c->w_head_pre};
+    const void *opt[] = {c->w_kq, c->w_head, c->w_kq_post, c->w_head_post, c->w_head_pre,
+                         c->w_kq_3d};
     for (const void *p : opt)
         if (p && !aligned(p, 16)) return MTA_ERR_ALIGNMENT;
     if (n_events < 0 || (n_events > 0 && !events)) return MTA_ERR_INVALID_ARG;
     rc = check_workspace(workspace, workspace_bytes, mta::unfused_workspace_bytes(*s));
     if (rc != MTA_OK) return rc;
     mta::ForwardArgs a{q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias, depth_scale, out, gate,
-                       c->w_kq_post, c->w_head_post, c->w_head_pre, c->exact_mask != 0};
+                       c->w_kq_post, c->w_head_post, c->w_head_pre, c->exact_mask != 0,
+                       c->w_kq_3d};
     mta::Trace tr;
     tr.events = events;
     tr.n = n_events;
@@ -185,6 +187,7 @@ mta::ForwardArgs chain_args(const mta_composition *c)
     a.w_head_post = c->w_head_post;
     a.w_head_pre = c->w_head_pre;
     a.exact_mask = c->exact_mask != 0;
+    a.w_kq_3d = c->w_kq_3d;
     return a;
 }
 

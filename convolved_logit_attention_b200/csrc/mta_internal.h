@@ -24,6 +24,8 @@ struct ForwardArgs {
     // exact indicator of Eq. (4) for that conv instead of Mask_0.
     const float *w_head_pre = nullptr;
     int exact_mask = 0;
+    // The 3-D kernel [H/c_h][c_h][c_h][c_q][c_k] in place of w_kq, or null.
+    const float *w_kq_3d = nullptr;
 };
 
 // Optional CUDA events recorded around the kernel launches of one call.

@@ -124,7 +124,10 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
 // and of the zero padding.  With kExact (the exact indicator of Eq. (4))
 // the halo keeps src[r][c] for c <= r + band, and each output row i zeroes
 // the keys c > i of the segments it reads: a tap (i', j') then adds
-// src[i-i'][j-j'] exactly when j - j' <= i.  Thread (warp w, lane l) owns output row l and
+// src[i-i'][j-j'] exactly when j - j' <= i.  With nin > 1 (the 3-D
+// convolution of "Putting Everything Together", nin = c_h) output head h
+// sums the convs of the nin heads of its group, with the kernel
+// w[(h * nin + hi)][c_q][c_k] for input head hi, one halo after another.  Thread (warp w, lane l) owns output row l and
 // the 16 columns 16w .. 16w+15: per query tap i' it loads the row segment
 // those columns reach (16 + c_k - 1 values) and the tap row theta[i'][*]
 // with 16-byte shared loads into registers and applies the c_k key taps from
@@ -132,11 +135,12 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
 // the FMA count.  Halo rows are kConvStride floats apart, 4 (mod 32) banks,
 // so the 16-byte loads of 8 consecutive rows hit distinct banks.  The taps
 // accumulate in the order i' then j' for every output.
-template <int CK, bool kExact>
-__global__ void __launch_bounds__(256)
+template <int CK, bool kExact, bool kMulti>
+__global__ void __launch_bounds__(256, kExact || kMulti ? 4 : 1)
 k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__restrict__ w_kq,
-       int T, int H, int c_q, int band)
+       int T, int H, int c_q, int band, int nin_arg)
 {
+    const int nin = kMulti ? nin_arg : 1;         // a compile-time 1 for the 2-D kernels
     constexpr int NC = kConvCols / 8;             // output columns per thread
     constexpr int NV = (CK + NC - 1 + 3) / 4;     // float4 loads per row segment
     constexpr int CKP = (CK + 3) / 4 * 4;         // padded tap row
@@ -147,54 +151,61 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
     if (j0 > i0 + kConvRows - 1) return;          // tile entirely above the diagonal
     const size_t bh = blockIdx.z;
     const int h = (int)(bh % H);
+    const size_t b = bh / H;
     __shared__ __align__(16) float tile[(kConvRows + kMaxCq - 1) * kConvStride];
     static_assert(kMaxCk <= 16, "tap rows are padded to 16 floats");
     __shared__ __align__(16) float th[kMaxCq * 16];
     const int tid = threadIdx.x;
     const int rows = kConvRows + c_q - 1;
-    const float *mb = src + bh * (size_t)T * T;
-    for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
-        const int rr = idx / kLoadCols, cc = idx % kLoadCols;
-        const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
-        tile[rr * kConvStride + cc] =
-            (r >= 0 && r < T && c >= 0 && c < T && c <= r + band) ? mb[(size_t)r * T + c] : 0.f;
-    }
-    for (int idx = tid; idx < c_q * CKP; idx += 256) {
-        const int ip = idx / CKP, jj = idx % CKP;
-        th[idx] = jj < CK ? w_kq[((size_t)h * c_q + ip) * CK + jj] : 0.f;
-    }
-    __syncthreads();
     const int ro = tid % 32;                      // output row within the tile
     const int c0 = (tid / 32) * NC;               // first of the thread's output columns
     float acc[NC];
 #pragma unroll
     for (int u = 0; u < NC; ++u) acc[u] = 0.f;
-    for (int ip = 0; ip < c_q; ++ip) {
-        const float4 *seg4 =
-            reinterpret_cast<const float4 *>(&tile[(ro + c_q - 1 - ip) * kConvStride + c0]);
-        float seg[4 * NV];
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const float4 t = seg4[v];
-            seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
+    for (int hi = 0; hi < nin; ++hi) {
+        const int hin = (h / nin) * nin + hi;     // input head (h itself when nin = 1)
+        const float *mb = src + (b * H + hin) * (size_t)T * T;
+        const float *wk = w_kq + ((size_t)h * nin + hi) * c_q * CK;
+        if (hi > 0) __syncthreads();              // every thread is done with the last halo
+        for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
+            const int rr = idx / kLoadCols, cc = idx % kLoadCols;
+            const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
+            tile[rr * kConvStride + cc] =
+                (r >= 0 && r < T && c >= 0 && c < T && c <= r + band) ? mb[(size_t)r * T + c]
+                                                                      : 0.f;
         }
-        if (kExact) {                             // the indicator: keys past query i read 0
-            const int kfirst = j0 - L + c0;       // key of seg[0]
-#pragma unroll
-            for (int v = 0; v < 4 * NV; ++v)
-                if (kfirst + v > i0 + ro) seg[v] = 0.f;
+        for (int idx = tid; idx < c_q * CKP; idx += 256) {
+            const int ip = idx / CKP, jj = idx % CKP;
+            th[idx] = jj < CK ? wk[(size_t)ip * CK + jj] : 0.f;
         }
-        const float4 *tr4 = reinterpret_cast<const float4 *>(&th[ip * CKP]);
-        float tr[CKP];
+        __syncthreads();
+        for (int ip = 0; ip < c_q; ++ip) {
+            const float4 *seg4 =
+                reinterpret_cast<const float4 *>(&tile[(ro + c_q - 1 - ip) * kConvStride + c0]);
+            float seg[4 * NV];
 #pragma unroll
-        for (int v = 0; v < CKP / 4; ++v) {
-            const float4 t = tr4[v];
-            tr[4 * v] = t.x; tr[4 * v + 1] = t.y; tr[4 * v + 2] = t.z; tr[4 * v + 3] = t.w;
+            for (int v = 0; v < NV; ++v) {
+                const float4 t = seg4[v];
+                seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
+            }
+            if (kExact) {                         // the indicator: keys past query i read 0
+                const int kfirst = j0 - L + c0;   // key of seg[0]
+#pragma unroll
+                for (int v = 0; v < 4 * NV; ++v)
+                    if (kfirst + v > i0 + ro) seg[v] = 0.f;
+            }
+            const float4 *tr4 = reinterpret_cast<const float4 *>(&th[ip * CKP]);
+            float tr[CKP];
+#pragma unroll
+            for (int v = 0; v < CKP / 4; ++v) {
+                const float4 t = tr4[v];
+                tr[4 * v] = t.x; tr[4 * v + 1] = t.y; tr[4 * v + 2] = t.z; tr[4 * v + 3] = t.w;
+            }
+#pragma unroll
+            for (int jj = 0; jj < CK; ++jj)
+#pragma unroll
+                for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[CK - 1 - jj + u], acc[u]);
         }
-#pragma unroll
-        for (int jj = 0; jj < CK; ++jj)
-#pragma unroll
-            for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[CK - 1 - jj + u], acc[u]);
     }
     const int i = i0 + ro;
     if (i >= T) return;
@@ -499,16 +510,24 @@ void launch_logits(const mta_shape &s, const void *q, const void *k, float *map0
 }
 
 void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq, int band,
-                 cudaStream_t st)
+                 int nin, cudaStream_t st)
 {
     dim3 g2((s.T + kConvCols - 1) / kConvCols, (s.T + kConvRows - 1) / kConvRows, s.B * s.H);
     switch (s.c_k) {
 #define MTA_CONV_CASE(n) \
         case n:                                                                          \
-            if (band > 0)                                                                \
-                k_conv<n, true><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q, band);  \
+            if (band > 0 && nin > 1)                                                     \
+                k_conv<n, true, true><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q,   \
+                                                          band, nin);                    \
+            else if (band > 0)                                                           \
+                k_conv<n, true, false><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q,  \
+                                                           band, 1);                     \
+            else if (nin > 1)                                                            \
+                k_conv<n, false, true><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q,  \
+                                                           0, nin);                      \
             else                                                                         \
-                k_conv<n, false><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q, 0);    \
+                k_conv<n, false, false><<<g2, 256, 0, st>>>(src, dst, w_kq, s.T, s.H, s.c_q, \
+                                                            0, 1);                       \
             break;
         MTA_CONV_CASE(1) MTA_CONV_CASE(2) MTA_CONV_CASE(3) MTA_CONV_CASE(4) MTA_CONV_CASE(5)
         MTA_CONV_CASE(6) MTA_CONV_CASE(7) MTA_CONV_CASE(8) MTA_CONV_CASE(9) MTA_CONV_CASE(10)
@@ -551,7 +570,7 @@ int unfused_chain(const ForwardArgs &a, const char **names)
 {
     int n = 0;
     names[n++] = "k_logits";
-    if (a.w_kq) names[n++] = "k_conv";
+    if (a.w_kq || a.w_kq_3d) names[n++] = "k_conv";
     if (a.w_head_pre) names[n++] = "k_head_mix";
     names[n++] = "k_softmax_mix";
     if (a.w_kq_post) names[n++] = "k_conv";
@@ -568,15 +587,16 @@ mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cu
                           const Trace &tr)
 {
     float *maps[2] = {(float *)ws, (float *)ws + bh_tt(s)};
-    const int band = (a.exact_mask && a.w_kq) ? s.c_q - 1 : 0;
+    const float *w_first = a.w_kq_3d ? a.w_kq_3d : a.w_kq;   // at most one is given
+    const int band = (a.exact_mask && w_first) ? s.c_q - 1 : 0;
     int cur = 0, launch = 0;
     mta_status rc = MTA_OK;
     tr.before(launch, st);
     logits(s, a.q, a.k, maps[0], band, st);
     tr.after(launch++, st);
-    if (a.w_kq) {
+    if (w_first) {
         tr.before(launch, st);
-        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq, band, st);
+        launch_conv(s, maps[cur], maps[cur ^ 1], w_first, band, a.w_kq_3d ? s.c_h : 1, st);
         tr.after(launch++, st);
         cur ^= 1;
     }
@@ -594,7 +614,7 @@ mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     cur ^= 1;
     if (a.w_kq_post) {
         tr.before(launch, st);
-        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq_post, 0, st);
+        launch_conv(s, maps[cur], maps[cur ^ 1], a.w_kq_post, 0, 1, st);
         tr.after(launch++, st);
         cur ^= 1;
     }
@@ -618,7 +638,7 @@ mta_status launch_debug_attention(const mta_shape &s, const void *q, const void 
     float *map0 = (float *)ws;
     float *map1 = map0 + bh_tt(s);
     logits(s, q, k, map0, 0, st);
-    launch_conv(s, map0, map1, w_kq, 0, st);
+    launch_conv(s, map0, map1, w_kq, 0, 1, st);
     mta_status rc = softmax_mix(s, map1, attn, w_head, stage == 0 ? 1 : 2, st);
     if (rc != MTA_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;

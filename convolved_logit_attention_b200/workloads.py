@@ -36,9 +36,11 @@ Recipes:
                   replaced by q_t + N(0, 0.1^2).
   w_kq_post,      the second key-query kernel and head mix of the
   w_head_post,    compositions of "Putting Everything Together: The Full MTA
-  w_head_pre      Module" and the pre-softmax head mix of the logits, drawn
-                  like w_kq and w_head from their own stream (seed + 7919), so
-                  that the default inputs stay unchanged.
+  w_head_pre,     Module", the pre-softmax head mix of the logits and the 3-D
+  w_kq_3d         kernel (identity on each head's own centre tap plus
+                  N(0, 0.05^2) everywhere), drawn like w_kq and w_head from
+                  their own stream (seed + 7919), so that the default inputs
+                  stay unchanged.
 """
 from dataclasses import dataclass, replace
 
@@ -82,15 +84,16 @@ class Workload:
 
     def composition_flops(self, comp: dict) -> int:
         """algorithmic_flops for a composition (an entry of COMPOSITIONS):
-        every key-query conv costs c_q c_k MACs per live logit and every
-        head mix c_h."""
+        every key-query conv costs c_q c_k MACs per live logit (the 3-D conv
+        c_h c_q c_k) and every head mix c_h."""
         n_kq = sum(bool(comp.get(n)) for n in ("w_kq", "w_kq_post"))
+        n_kq += self.c_h * bool(comp.get("w_kq_3d"))
         n_mix = sum(bool(comp.get(n)) for n in ("w_head_pre", "w_head", "w_head_post"))
         per_logit = 4 * self.d + 2 * n_kq * self.c_q * self.c_k + 2 * n_mix * self.c_h
         return self.B * self.H * self.live_logits() * per_logit
 
 
-WEIGHT_NAMES = ("w_kq", "w_head_pre", "w_head", "w_kq_post", "w_head_post")
+WEIGHT_NAMES = ("w_kq", "w_head_pre", "w_head", "w_kq_post", "w_head_post", "w_kq_3d")
 
 # The steps of each composition: the weights it has (the others are None)
 # and whether its first key-query conv uses the exact indicator of Eq. (4).
@@ -107,6 +110,8 @@ COMPOSITIONS = {
     "exact": dict(w_kq=1, w_head=1, exact_mask=1),
     "exact_both_pre": dict(w_kq=1, w_head_pre=1, exact_mask=1),
     "exact_repeat": dict(w_kq=1, w_head=1, w_kq_post=1, w_head_post=1, exact_mask=1),
+    "conv3d": dict(w_kq_3d=1),             # one 3-D kernel over (query, key, head)
+    "conv3d_exact_mix": dict(w_kq_3d=1, w_head=1, exact_mask=1),
 }
 
 
@@ -186,8 +191,13 @@ def post_weights(w: Workload, seed: int = None) -> dict:
         np.float32(0.05) * rng.standard_normal((w.G, w.c_h, w.c_h), dtype=np.float32)
     w_head_pre = np.eye(w.c_h, dtype=np.float32)[None] + \
         np.float32(0.05) * rng.standard_normal((w.G, w.c_h, w.c_h), dtype=np.float32)
+    # the 3-D kernel: identity (theta3[h][h][0][centre] = 1) plus N(0, 0.05^2)
+    w_kq_3d = np.float32(0.05) * rng.standard_normal((w.G, w.c_h, w.c_h, w.c_q, w.c_k),
+                                                     dtype=np.float32)
+    for hh in range(w.c_h):
+        w_kq_3d[:, hh, hh, 0, w.c_k // 2] += np.float32(1.0)
     return {"w_kq_post": w_kq_post, "w_head_post": w_head_post.astype(np.float32),
-            "w_head_pre": w_head_pre.astype(np.float32)}
+            "w_head_pre": w_head_pre.astype(np.float32), "w_kq_3d": w_kq_3d}
 
 
 def composed_inputs(w: Workload, composition: str, seed: int = None) -> dict:

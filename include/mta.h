@@ -229,7 +229,12 @@ MTA_API mta_status mta_forward_noalloc(const mta_shape *shape, const void *q, co
  * {w_kq, w_head, w_kq_post, w_head_post}; "both post-softmax" is
  * {w_kq_post, w_head_post}.  Both key-query kernels are [H][c_q][c_k] and the
  * three head mixes [H/c_h][c_h][c_h], laid out as w_kq and w_head above;
- * pointers are device memory, 16-byte aligned, NULL for a step left out. */
+ * pointers are device memory, 16-byte aligned, NULL for a step left out.
+ * w_kq_3d [H/c_h][c_h][c_h][c_q][c_k] is the general 3-D kernel of "Both
+ * pre-softmax (3D convolution view)": S3 becomes C^h = sum over the input
+ * heads h' of h's group of the 2-D conv of A0^{h'} with
+ * w_kq_3d[group][h][h'] (tap layout as w_kq), under either masking.  Giving
+ * both w_kq and w_kq_3d is MTA_ERR_INVALID_ARG. */
 typedef struct {
     const float *w_kq;         /* S3 before the softmax, or NULL */
     const float *w_head;       /* S6 right after the softmax, or NULL */
@@ -237,6 +242,7 @@ typedef struct {
     const float *w_head_post;  /* P2 after P1, or NULL */
     const float *w_head_pre;   /* L1 on the logits, or NULL */
     int exact_mask;            /* nonzero: S3 under Eq. (4)'s indicator */
+    const float *w_kq_3d;      /* the 3-D kernel in place of w_kq, or NULL (below) */
 } mta_composition;
 
 /* Bytes of device workspace mta_forward_composed needs (0 on an invalid

@@ -156,6 +156,9 @@ def test_composed_launch_sequences_and_workspace(L):
         (a, a, a, a, a, 1): ["k_logits", "k_conv", "k_head_mix", "k_softmax_mix", "k_conv",
                              "k_head_mix", "k_pv_groupnorm"],
         (a, a, None, None, None, 1): ["k_logits", "k_conv", "k_softmax_mix", "k_pv_groupnorm"],
+        # the 3-D kernel in place of the key-query kernel
+        (None, a, None, None, None, 0, a): ["k_logits", "k_conv", "k_softmax_mix",
+                                            "k_pv_groupnorm"],
     }
     for ptrs, names in seqs.items():
         comp = C(*ptrs)
@@ -192,6 +195,8 @@ def test_composed_argument_checks(L):
     assert call(s, rep, q=z) == -1
     assert call(s, C(1 << 20, 1 << 20, (1 << 20) + 8, None)) == -3
     assert call(s, C(1 << 20, None, None, None, (1 << 20) + 4, 0)) == -3
+    assert call(s, C(None, None, None, None, None, 0, (1 << 20) + 4)) == -3
+    assert call(s, C(1 << 20, None, None, None, None, 0, 1 << 20)) == -1   # w_kq and w_kq_3d
     assert call(s, rep, gate=ctypes.c_void_p((1 << 20) + 2)) == -3
     assert call(s, rep, nbytes=need - 1) == -4
     assert call(s, rep, ws=z) == -1

@@ -36,7 +36,7 @@ def to_device(x, io):
     dt = torch.bfloat16 if io == "bf16" else torch.float32
     dev = torch.device("cuda", 0)
     d = {n: torch.from_numpy(np.ascontiguousarray(x[n])).to(dev).to(dt) for n in ("q", "k", "v")}
-    for n in WEIGHTS + ("w_head_pre", "gn_weight", "gn_bias"):
+    for n in WEIGHTS + ("w_head_pre", "w_kq_3d", "gn_weight", "gn_bias"):
         d[n] = None if x[n] is None else torch.from_numpy(np.ascontiguousarray(x[n])).to(dev)
     return d
 
@@ -46,7 +46,7 @@ def run(d, x, gate=None, events=None):
                                    gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
                                    depth_scale=x["depth_scale"], gate=gate,
                                    gn_eps=x["gn_eps"], events=events, w_head_pre=d["w_head_pre"],
-                                   exact_mask=x["exact_mask"])
+                                   exact_mask=x["exact_mask"], w_kq_3d=d["w_kq_3d"])
     mta.mta_sync_status()
     return out.float().cpu().numpy().astype(np.float64)
 
@@ -55,7 +55,7 @@ def oracle_full(x, gate=None):
     return oracle.forward_composed(x["q"], x["k"], x["v"], *(x[n] for n in WEIGHTS),
                                    x["gn_weight"], x["gn_bias"], x["depth_scale"],
                                    gn_eps=x["gn_eps"], gate=gate, w_head_pre=x["w_head_pre"],
-                                   exact_mask=x["exact_mask"])
+                                   exact_mask=x["exact_mask"], w_kq_3d=x["w_kq_3d"])
 
 
 @pytest.mark.parametrize("comp", sorted(COMPOSITIONS))
@@ -81,7 +81,7 @@ RAGGED = [
 
 
 @pytest.mark.parametrize("comp", ["repeat", "post_kq", "both_post", "exact_both_pre",
-                                  "exact_repeat"])
+                                  "exact_repeat", "conv3d_exact_mix"])
 @pytest.mark.parametrize("shape", RAGGED, ids=[str(s) for s in RAGGED])
 def test_ragged_shapes_elementwise(shape, comp):
     B, H, T, d, c_q, c_k, c_h, io = shape
@@ -125,6 +125,17 @@ def test_strong_kernels_exact_mask_and_logit_mix(comp):
     assert np.abs(two_pass - ref).max() > 100 * 1e-4
 
 
+def test_strong_conv3d_kernel():
+    """A 3-D kernel far from the identity, cross-head taps included, in
+    fp32 with the exact mask and without."""
+    w = Workload("strong_3d", 2, 4, 150, 32, 4, 7, 2, "f32", seed=35)
+    rng = np.random.default_rng(36)
+    for comp in ("conv3d", "conv3d_exact_mix"):
+        x = composed_inputs(w, comp)
+        x["w_kq_3d"] = (0.4 * rng.standard_normal(x["w_kq_3d"].shape)).astype(np.float32)
+        assert_close(run(to_device(x, w.io), x), oracle_full(x), w.io, "strong " + comp)
+
+
 def test_default_composition_is_mta_forward():
     """The default composition takes mta_forward's own path: same bits."""
     w = WORKLOADS["toy_letters"]
@@ -153,7 +164,7 @@ def test_traced_launches_follow_the_chain():
     assert_close(got, oracle_full(x), w.io, "traced")
 
 
-@pytest.mark.parametrize("comp", ["repeat", "both_post", "exact_both_pre"])
+@pytest.mark.parametrize("comp", ["repeat", "both_post", "exact_both_pre", "conv3d"])
 def test_full_size_sampled_rows(comp):
     """The T = 4096 workload (two [B,H,T,T] fp32 maps, 4.3 GB) on rows
     sampled per batch entry, including tile edges and both ends."""
@@ -169,5 +180,5 @@ def test_full_size_sampled_rows(comp):
         ref = oracle.rows_composed(x["q"], x["k"], x["v"], *(x[n] for n in WEIGHTS),
                                    x["gn_weight"], x["gn_bias"], x["depth_scale"], b, rows,
                                    gn_eps=x["gn_eps"], w_head_pre=x["w_head_pre"],
-                                   exact_mask=x["exact_mask"])
+                                   exact_mask=x["exact_mask"], w_kq_3d=x["w_kq_3d"])
         assert_close(got[b, rows], ref, w.io, "longctx_4k %s b=%d" % (comp, b))

@@ -82,7 +82,7 @@ def test_reference_arm_times_a_composition():
     assert d["config"]["composition"] == "repeat" and d["value"] > 0
 
 
-@pytest.mark.parametrize("name", ["repeat", "exact_both_pre"])
+@pytest.mark.parametrize("name", ["repeat", "exact_both_pre", "conv3d_exact_mix"])
 def test_oracle_units_are_slices_of_the_composed_forward(name):
     # The CPU-baseline sample cuts (batch, head-group) units out of the
     # workload, post-softmax weights included; each unit's oracle output
@@ -96,7 +96,8 @@ def test_oracle_units_are_slices_of_the_composed_forward(name):
     assert f == 2 * flops // (w.B * w.G)
     full = oracle.forward_composed(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["w_kq_post"],
                                    x["w_head_post"], x["gn_weight"], x["gn_bias"], w.depth_scale,
-                                   w_head_pre=x["w_head_pre"], exact_mask=x["exact_mask"])
+                                   w_head_pre=x["w_head_pre"], exact_mask=x["exact_mask"],
+                                   w_kq_3d=x["w_kq_3d"])
     for g, u in enumerate(units):
         part = bench.run_oracle_unit(u, w)
         cs = slice(g * w.c_h * w.d, (g + 1) * w.c_h * w.d)
