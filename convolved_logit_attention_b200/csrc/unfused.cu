@@ -136,7 +136,7 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
 // so the 16-byte loads of 8 consecutive rows hit distinct banks.  The taps
 // accumulate in the order i' then j' for every output.
 template <int CK, bool kExact, bool kMulti>
-__global__ void __launch_bounds__(256, kExact || kMulti ? 4 : 1)
+__global__ void __launch_bounds__(256, kExact || kMulti ? 4 : 5)
 k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__restrict__ w_kq,
        int T, int H, int c_q, int band, int nin_arg)
 {
@@ -151,7 +151,7 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
     if (j0 > i0 + kConvRows - 1) return;          // tile entirely above the diagonal
     const size_t bh = blockIdx.z;
     const int h = (int)(bh % H);
-    const size_t b = bh / H;
+    const size_t b = kMulti ? bh / H : 0;
     __shared__ __align__(16) float tile[(kConvRows + kMaxCq - 1) * kConvStride];
     static_assert(kMaxCk <= 16, "tap rows are padded to 16 floats");
     __shared__ __align__(16) float th[kMaxCq * 16];
@@ -163,9 +163,9 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
 #pragma unroll
     for (int u = 0; u < NC; ++u) acc[u] = 0.f;
     for (int hi = 0; hi < nin; ++hi) {
-        const int hin = (h / nin) * nin + hi;     // input head (h itself when nin = 1)
-        const float *mb = src + (b * H + hin) * (size_t)T * T;
-        const float *wk = w_kq + ((size_t)h * nin + hi) * c_q * CK;
+        // input head and kernel block (h's own for the 2-D kernels)
+        const float *mb = src + (kMulti ? b * H + (h / nin) * nin + hi : bh) * (size_t)T * T;
+        const float *wk = w_kq + (kMulti ? (size_t)h * nin + hi : (size_t)h) * c_q * CK;
         if (hi > 0) __syncthreads();              // every thread is done with the last halo
         for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
             const int rr = idx / kLoadCols, cc = idx % kLoadCols;
