@@ -206,3 +206,29 @@ def test_composed_argument_checks(L):
     fused = shape(B=2, H=16, T=4096, d=128, c_q=6, c_k=11, c_h=2)
     fneed = mta.mta_workspace_size(fused)
     assert call(fused, C(1 << 20, 1 << 20, None, None), nbytes=fneed - 1) == -4
+
+
+def test_ctypes_structs_match_the_c_header_layout(tmp_path):
+    # The binding's ctypes mirrors of mta_shape and mta_composition must have
+    # the header's field offsets and sizes; a C program built against
+    # include/mta.h prints them.
+    import subprocess
+    fields = {"mta_shape": [f[0] for f in _binding.MtaShape._fields_],
+              "mta_composition": [f[0] for f in _binding.MtaComposition._fields_]}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "mta.h"', 'int main(void) {']
+    for st, names in fields.items():
+        lines.append('printf("%s size %%zu\\n", sizeof(%s));' % (st, st))
+        for n in names:
+            lines.append('printf("%s %s %%zu\\n", offsetof(%s, %s));' % (st, n, st, n))
+    lines.append('return 0; }')
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for st, cls in (("mta_shape", _binding.MtaShape), ("mta_composition", _binding.MtaComposition)):
+        assert got[(st, "size")] == ctypes.sizeof(cls), st
+        for n in fields[st]:
+            assert got[(st, n)] == getattr(cls, n).offset, (st, n)
