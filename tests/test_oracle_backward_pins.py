@@ -87,3 +87,57 @@ def test_gradients_are_causal():
         for name in ("q", "k", "v"):
             assert np.all(g[name][:, :, t + 1:] == 0.0), (name, t)
             assert np.abs(g[name][:, :, : t + 1]).max() > 0.0
+
+
+# (w_kq, w_kq_3d, w_head_pre, w_head, w_kq_post, w_head_post, exact_mask)
+COMPOSED = {
+    "repeat": (1, 0, 0, 1, 1, 1, 0),
+    "exact_both_pre": (1, 0, 1, 0, 0, 0, 1),
+    "conv3d_exact_mix": (0, 1, 0, 1, 0, 0, 1),
+}
+
+
+def composed_inputs_of(shape, use, seed):
+    rng = np.random.default_rng(seed)
+    q, k, v, th, w, gw, gb = rand_inputs(rng, *shape)
+    B, H, T, d, c_q, c_k, c_h = shape
+    th3 = 0.3 * rng.standard_normal((H // c_h, c_h, c_h, c_q, c_k))
+    extra = dict(w_kq=th, w_kq_3d=th3, w_head_pre=rng.standard_normal(w.shape), w_head=w,
+                 w_kq_post=0.5 * rng.standard_normal(th.shape),
+                 w_head_post=rng.standard_normal(w.shape))
+    x = dict(q=q, k=k, v=v, gn_weight=gw, gn_bias=gb)
+    for name, u in zip(("w_kq", "w_kq_3d", "w_head_pre", "w_head", "w_kq_post", "w_head_post"),
+                       use[:6]):
+        x[name] = extra[name] if u else None
+    return x, bool(use[6]), rng
+
+
+def c_forward(x, exact, depth=0.7):
+    return oracle.forward_composed(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["w_kq_post"],
+                                   x["w_head_post"], x["gn_weight"], x["gn_bias"], depth,
+                                   w_head_pre=x["w_head_pre"], exact_mask=exact,
+                                   w_kq_3d=x["w_kq_3d"])
+
+
+@pytest.mark.parametrize("name", sorted(COMPOSED))
+def test_composed_restatement_and_gradients(name):
+    # The torch restatement of each composition equals the C oracle's
+    # composed forward, and its autograd gradients equal central finite
+    # differences of that C forward along random directions.
+    shape = (1, 4, 10, 4, 3, 5, 2)
+    x, exact, rng = composed_inputs_of(shape, COMPOSED[name], 64)
+    ref = c_forward(x, exact)
+    ts = {n: None if x.get(n) is None else torch.as_tensor(x[n]) for n in backward.COMPOSED_NAMES}
+    np.testing.assert_allclose(backward.forward_composed(ts, 0.7, exact).numpy(), ref, rtol=0,
+                               atol=1e-12)
+    dout = rng.standard_normal(ref.shape)
+    g = backward.gradients_composed(x, dout, 0.7, exact)
+    h = 1e-5
+    for n, grad in g.items():
+        delta = rng.standard_normal(x[n].shape)
+        plus, minus = dict(x), dict(x)
+        plus[n] = x[n] + h * delta
+        minus[n] = x[n] - h * delta
+        fd = float(np.sum((c_forward(plus, exact) - c_forward(minus, exact)) * dout)) / (2 * h)
+        an = float(np.sum(grad * delta))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, n, fd, an)
