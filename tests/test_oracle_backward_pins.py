@@ -8,6 +8,8 @@ the C oracle's forward along random directions, which shares no code with
 autograd; the gradients of the affine parameters have closed forms; and
 gradients respect causality.
 """
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -141,3 +143,43 @@ def test_composed_restatement_and_gradients(name):
         fd = float(np.sum((c_forward(plus, exact) - c_forward(minus, exact)) * dout)) / (2 * h)
         an = float(np.sum(grad * delta))
         assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, n, fd, an)
+
+
+# Planted mistakes in the torch restatement; some pin above must catch each.
+BACKWARD_MUTATIONS = [
+    ("key shift sign", "C = C + w_kq[:, ip, jj].view(1, H, 1, 1) * _shift(A0, ip, jp)",
+     "C = C + w_kq[:, ip, jj].view(1, H, 1, 1) * _shift(A0, ip, -jp)"),
+    ("mix transposed", 'A = torch.einsum("goi,bgitj->bgotj", w_head,',
+     'A = torch.einsum("gio,bgitj->bgotj", w_head,'),
+    ("unbiased variance", "var = ((O - mean) ** 2).mean(dim=-1, keepdim=True)\n    xhat",
+     "var = ((O - mean) ** 2).sum(dim=-1, keepdim=True) / (d - 1)\n    xhat"),
+    ("exact indicator against the shifted query",
+     "S = torch.where(J - jp <= I, S, torch.zeros((), dtype=X.dtype))",
+     "S = torch.where(J - jp <= I - ip, S, torch.zeros((), dtype=X.dtype))"),
+    ("post conv not masked", 'A = torch.where(causal, _conv(A, t["w_kq_post"], False), zero)',
+     'A = _conv(A, t["w_kq_post"], False)'),
+]
+
+
+@pytest.mark.parametrize("name,before,after", BACKWARD_MUTATIONS,
+                         ids=[m[0] for m in BACKWARD_MUTATIONS])
+def test_backward_pins_catch_planted_mistakes(monkeypatch, tmp_path, name, before, after):
+    import importlib.util
+    src = open(backward.__file__).read()
+    assert src.count(before) == 1, before
+    path = tmp_path / "mutant_backward.py"
+    path.write_text(src.replace(before, after))
+    spec = importlib.util.spec_from_file_location("mutant_backward", str(path))
+    mutant = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mutant)
+    monkeypatch.setattr(sys.modules[__name__], "backward", mutant)
+    checks = [lambda: test_torch_restatement_equals_the_c_oracle(SHAPES[1]),
+              lambda: test_gradients_match_finite_differences_of_the_c_oracle(SHAPES[1])]
+    checks += [lambda n=n: test_composed_restatement_and_gradients(n) for n in sorted(COMPOSED)]
+    caught = 0
+    for check in checks:
+        try:
+            check()
+        except AssertionError:
+            caught += 1
+    assert caught, "no pin caught: " + name
