@@ -314,7 +314,8 @@ mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stream)
 mta_status mta_sync_status(void *stream)
 {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MTA_ERR_CUDA;
-    const unsigned int err = mta::fused_take_error();
+    const unsigned int err = mta::fused_take_error((cudaStream_t)stream);
+    if (err == ~0u) return MTA_ERR_CUDA;
     if (err & 1u) return MTA_ERR_DEVICE_TIMEOUT;
     if (err & 2u) return MTA_ERR_RANGE;
     return MTA_OK;

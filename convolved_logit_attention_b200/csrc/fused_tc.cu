@@ -1178,6 +1178,7 @@ const char *const kFusedNames[4] = {"k_fold_keys", "k_fold_aux", "k_mta_fused", 
 struct SideStream {
     cudaStream_t s = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    unsigned long long ctx = 0;    // context the handles belong to
 };
 std::mutex g_side_lock;
 
@@ -1186,13 +1187,20 @@ mta_status side_stream(SideStream *out)
     constexpr int kMaxDevices = 64;
     static SideStream tab[kMaxDevices];
     int dev = 0;
+    unsigned long long ctx = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTA_ERR_CUDA;
+    if (!current_context_id(&ctx)) return MTA_ERR_CUDA;
     SideStream &ss = tab[dev];
-    if (!ss.s) {
-        if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess ||
-            cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess)
+    // handles made in a context that has since been destroyed (a device
+    // reset) are dead: make new ones in the current context
+    if (!ss.s || ss.ctx != ctx) {
+        SideStream fresh;
+        if (cudaEventCreateWithFlags(&fresh.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&fresh.s, cudaStreamNonBlocking) != cudaSuccess)
             return MTA_ERR_CUDA;
+        fresh.ctx = ctx;
+        ss = fresh;
     }
     *out = ss;
     return MTA_OK;
@@ -1381,28 +1389,45 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[MTA_NOALLOC_SCR
 mta_status noalloc_scratch(void **ptr)
 {
     constexpr int kMaxDevices = 64;
-    static void *addr[kMaxDevices] = {};
+    struct Entry {
+        void *addr;
+        unsigned long long ctx;
+    };
+    static Entry tab[kMaxDevices] = {};
     static std::mutex lock;
     int dev = 0;
+    unsigned long long ctx = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTA_ERR_CUDA;
+    if (!current_context_id(&ctx)) return MTA_ERR_CUDA;
     std::lock_guard<std::mutex> guard(lock);
-    if (!addr[dev]) {
+    // the address belongs to the context the module was loaded in: look it up
+    // again after the device's context was destroyed and re-created
+    if (!tab[dev].addr || tab[dev].ctx != ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MTA_ERR_CUDA;
-        addr[dev] = p;
+        tab[dev].addr = p;
+        tab[dev].ctx = ctx;
     }
-    *ptr = addr[dev];
+    *ptr = tab[dev].addr;
     return MTA_OK;
 }
 
-unsigned int fused_take_error()
+// Read and clear of the error word in one atomic step on the caller's
+// stream, so that a flag raised between a read and a separate clear is not
+// lost; the value goes through a second device word to the host.
+__device__ unsigned int g_fused_error_taken;
+
+__global__ void k_take_error() { g_fused_error_taken = atomicExch(&g_fused_error, 0u); }
+
+unsigned int fused_take_error(cudaStream_t st)
 {
+    k_take_error<<<1, 1, 0, st>>>();
     unsigned int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_fused_error, sizeof(v)) != cudaSuccess) return 0;
-    if (v) {
-        unsigned int z = 0;
-        cudaMemcpyToSymbol(g_fused_error, &z, sizeof(z));
-    }
+    if (cudaGetLastError() != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&v, g_fused_error_taken, sizeof(v), 0, cudaMemcpyDeviceToHost,
+                                  st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return ~0u;
     return v;
 }
 

@@ -66,10 +66,12 @@ const char *fused_kernel_name(const mta_shape &s, int index);
 mta_status launch_fused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                         const Trace &tr);
 // Device address of the static scratch mta_forward_noalloc works in (looked
-// up once per device, with that device current).
+// up once per device and context, with that device current).
 mta_status noalloc_scratch(void **ptr);
 mta_status launch_selftest_wait_timeout(long long budget_cycles, cudaStream_t st);
-// Reads and clears the fused kernels' device error word on the current device.
-unsigned int fused_take_error();
+// Reads and clears, in one atomic step on stream `st`, the fused kernels'
+// device error word of the current device (one word per device, shared by
+// every stream), then synchronises `st`; ~0u when a CUDA call failed.
+unsigned int fused_take_error(cudaStream_t st);
 
 }  // namespace mta

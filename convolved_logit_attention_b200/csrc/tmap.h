@@ -59,4 +59,38 @@ inline bool make_tmap_f16(CUtensorMap *map, const void *base, int rank, const ui
     return make_tmap_16b(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, rank, dims, strides_bytes, box);
 }
 
+// Unique id of the calling thread's current CUDA context (driver API,
+// through the entry point).  Ids are never reused within a process, so a
+// cached handle or device address tagged with one is recognised as stale
+// once its context has been destroyed and another created in its place.
+inline bool current_context_id(unsigned long long *id)
+{
+    using GetCurrentFn = CUresult (*)(CUcontext *);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+            qa != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+            qb != cudaDriverEntryPointSuccess)
+            return false;
+        get_current = (GetCurrentFn)a;
+        get_id = (GetIdFn)b;
+    }
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return false;
+    if (!ctx) {
+        // no context bound to this thread yet: cudaSetDevice makes the
+        // device's primary context current (CUDA 12 initialises it there)
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess ||
+            get_current(&ctx) != CUDA_SUCCESS || !ctx)
+            return false;
+    }
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 }  // namespace mta

@@ -200,6 +200,9 @@ MTA_API mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stre
  *     Nothing is enqueued in either case.
  *   - The first call on a device looks up the scratch's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept per device and context: after the device's context
+ *     is destroyed (cudaDeviceReset) the next call looks it up again, so make
+ *     that call outside stream capture as well.
  *   - All calls on a device share the one scratch area and leave their data
  *     in it.  Every byte a call reads there it has written first, so stale
  *     contents do no harm, but calls whose work overlaps on the GPU (other
@@ -285,7 +288,11 @@ MTA_API const char *mta_composed_kernel_name(const mta_shape *shape, const mta_c
 /* Synchronises `stream`, then reports (and clears) the device error flags:
  * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
  * the fused path met a value outside fp16 range, MTA_ERR_CUDA if the
- * synchronisation itself failed, MTA_OK otherwise. */
+ * synchronisation itself failed, MTA_OK otherwise.  The flags are one word per
+ * device, shared by every stream and caller of the library on that device:
+ * the word is read and cleared in one atomic step (a small kernel on
+ * `stream`), so no raised flag is lost, but a call reports flags raised by
+ * any work on the device since the previous report. */
 MTA_API mta_status mta_sync_status(void *stream);
 
 #ifdef __cplusplus
