@@ -201,8 +201,15 @@ def mta_kernel_name(shape: MtaShape, index: int, unfused: bool = False) -> str:
     return r.decode() if r is not None else None
 
 
+def _after(check, stream, device):
+    """With check, synchronise the call's stream and raise MtaError on a
+    device-side flag (MTA_ERR_RANGE, MTA_ERR_DEVICE_TIMEOUT)."""
+    if check:
+        mta_sync_status(stream, device)
+
+
 def _forward(fn_name, size_fn, q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale,
-             out, workspace, stream, gn_eps, traced=None):
+             out, workspace, stream, gn_eps, traced=None, check=False):
     _check_inputs(q, k, v, w_kq, w_head, gn_weight, gn_bias)
     B, H, T, d = q.shape
     if out is None:
@@ -222,20 +229,27 @@ def _forward(fn_name, size_fn, q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_
         handles = (ctypes.c_void_p * max(len(events), 1))(*[e.cuda_event for e in events])
         status = lib().mta_forward_traced(int(unfused), *args, handles, len(events))
     _check(fn_name, status)
+    _after(check, stream, q.device)
     return out
 
 
 def mta_forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out=None,
-                workspace=None, stream=None, gn_eps=1e-5):
-    """MTA forward on the path mta_forward_path() names; returns out [B, T, H*d]."""
+                workspace=None, stream=None, gn_eps=1e-5, check=False):
+    """MTA forward on the path mta_forward_path() names; returns out [B, T, H*d].
+
+    The call is asynchronous.  Device-side conditions (a bounded wait that
+    ran out, a value outside the range of the fused path's fp16 operands)
+    are only seen at a synchronisation: with check=True the call synchronises
+    its stream and raises MtaError for them; otherwise call mta_sync_status()."""
     return _forward("mta_forward", mta_workspace_size, q, k, v, w_kq, w_head, gn_weight,
-                    gn_bias, depth_scale, out, workspace, stream, gn_eps)
+                    gn_bias, depth_scale, out, workspace, stream, gn_eps, check=check)
 
 
 def mta_forward_gated(q, k, v, w_kq, w_head, gn_weight, gn_bias, gate, out=None,
-                      workspace=None, stream=None, gn_eps=1e-5):
+                      workspace=None, stream=None, gn_eps=1e-5, check=False):
     """MTA forward with the sigmoid-gated output: head h of GroupNorm times
-    sigmoid(gate[h]) (gate: float32 [H] on the device); returns out [B, T, H*d]."""
+    sigmoid(gate[h]) (gate: float32 [H] on the device); returns out [B, T, H*d].
+    check as for mta_forward."""
     _check_inputs(q, k, v, w_kq, w_head, gn_weight, gn_bias)
     B, H, T, d = q.shape
     if gate.dtype != torch.float32 or gate.shape != (H,) or gate.device != q.device \
@@ -253,14 +267,17 @@ def mta_forward_gated(q, k, v, w_kq, w_head, gn_weight, gn_bias, gate, out=None,
                                      _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                      _stream_ptr(stream, q.device))
     _check("mta_forward_gated", status)
+    _after(check, stream, q.device)
     return out
 
 
 def mta_forward_unfused(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out=None,
-                        workspace=None, stream=None, gn_eps=1e-5):
-    """MTA forward with materialised T x T maps (fp32 arithmetic)."""
+                        workspace=None, stream=None, gn_eps=1e-5, check=False):
+    """MTA forward with materialised T x T maps (fp32 arithmetic); check as
+    for mta_forward."""
     return _forward("mta_forward_unfused", mta_unfused_workspace_size, q, k, v, w_kq, w_head,
-                    gn_weight, gn_bias, depth_scale, out, workspace, stream, gn_eps)
+                    gn_weight, gn_bias, depth_scale, out, workspace, stream, gn_eps,
+                    check=check)
 
 
 def mta_forward_traced(unfused, events, q, k, v, w_kq, w_head, gn_weight, gn_bias,
@@ -301,7 +318,10 @@ def mta_selftest_wait_timeout(budget_cycles=1 << 20, stream=None, device=None):
 
 
 def mta_sync_status(stream=None, device=None):
-    """Synchronises the stream and raises MtaError on a device-side timeout."""
+    """Synchronises the stream and raises MtaError for a device-side flag
+    (MTA_ERR_DEVICE_TIMEOUT, MTA_ERR_RANGE).  The flags are one word per
+    device: this reports what any work on the device raised since the last
+    report."""
     if device is None:
         device = torch.device("cuda", torch.cuda.current_device())
     _check("mta_sync_status", lib().mta_sync_status(_stream_ptr(stream, device)))
@@ -351,12 +371,12 @@ def mta_composed_kernel_names(shape: MtaShape, comp: MtaComposition):
 def mta_forward_composed(q, k, v, w_kq=None, w_head=None, w_kq_post=None, w_head_post=None,
                          gn_weight=None, gn_bias=None, depth_scale=1.0, gate=None, out=None,
                          workspace=None, stream=None, gn_eps=1e-5, events=None,
-                         w_head_pre=None, exact_mask=False, w_kq_3d=None):
+                         w_head_pre=None, exact_mask=False, w_kq_3d=None, check=False):
     """Forward of one composition of the module (see mta_composition in
     include/mta.h): weights left as None are steps left out.  gate (float32
     [H]) replaces the depth scale by sigmoid(gate[h]).  With events (a list
     of torch.cuda.Event, two per launch) the traced entry records them
-    around the launches.  Returns out [B, T, H*d]."""
+    around the launches.  check as for mta_forward.  Returns out [B, T, H*d]."""
     ws_ = [w_kq, w_head, w_kq_post, w_head_post, w_head_pre, w_kq_3d]
     if q.device.type != "cuda":
         raise ValueError("inputs must be CUDA tensors")
@@ -396,4 +416,5 @@ def mta_forward_composed(q, k, v, w_kq=None, w_head=None, w_kq_post=None, w_head
         handles = (ctypes.c_void_p * max(len(events), 1))(*[e.cuda_event for e in events])
         _check("mta_forward_composed_traced",
                lib().mta_forward_composed_traced(*args, handles, len(events)))
+    _after(check, stream, q.device)
     return out

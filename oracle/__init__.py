@@ -53,6 +53,8 @@ def _configure(lib):
     lib.mta_oracle_stages_composed.argtypes = [sp, dp, dp, dp, cp, dp, dp, ctypes.c_double, dp,
                                                ctypes.c_int, dp, dp, dp, dp, dp, dp]
     lib.mta_oracle_max_threads.argtypes = []
+    lib.mta_oracle_set_row_chunk.argtypes = [ctypes.c_int]
+    lib.mta_oracle_set_row_chunk.restype = None
     for f in (lib.mta_oracle_forward, lib.mta_oracle_rows, lib.mta_oracle_stages,
               lib.mta_oracle_forward_gated, lib.mta_oracle_rows_gated,
               lib.mta_oracle_forward_composed, lib.mta_oracle_rows_composed,
@@ -109,6 +111,12 @@ def _unpack(q, w_kq, w_head):
 
 def max_threads() -> int:
     return int(_load().mta_oracle_max_threads())
+
+
+def set_row_chunk(rows: int) -> None:
+    """Rows per task of the full forward (0: chosen from the thread count).
+    The split never changes a value; the tests use this to show it."""
+    _load().mta_oracle_set_row_chunk(int(rows))
 
 
 def forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gn_eps=1e-5,

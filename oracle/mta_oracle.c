@@ -400,10 +400,19 @@ static int args_ok(const mta_oracle_shape *s, const mta_oracle_args *a)
     return shape_ok(s) && a->q && a->k && a->v && a->gn_weight && a->gn_bias;
 }
 
-/* Full forward: out[B][T][H*d].  Units (b, g) are independent and spread over
- * threads; inside a unit the query rows run in order, keeping the last c_q
- * masked logit rows and first-stage rows of each head in rings.  Returns 0
- * on success. */
+/* Rows per task of the full forward: 0 picks a size from the thread count;
+ * a positive value forces it (the tests use that to show that the split does
+ * not change a single bit). */
+static int g_row_chunk = 0;
+
+/* Full forward: out[B][T][H*d].  Units (b, g) are independent; inside a unit
+ * the query rows run in order, keeping the last c_q masked logit rows and
+ * first-stage rows of each head in rings.  When there are fewer units than
+ * threads, each unit's rows are also split into chunks run as separate
+ * tasks: a chunk first recomputes the 2 (c_q - 1) rows before it, which
+ * refills both rings with exactly the values the unsplit loop would hold
+ * (every masked logit row is computed on its own from q and k), and writes
+ * output only from its first row on.  Returns 0 on success. */
 static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, double *out,
                         int nthreads)
 {
@@ -412,17 +421,35 @@ static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, do
     const int G = s->H / s->c_h;
     const int units = s->B * G;
     const size_t HD = (size_t)s->H * s->d;
-    int failed = 0;
+    int threads = 1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
+    threads = omp_get_max_threads();
+#endif
+    int chunk = s->T;
+    if (g_row_chunk > 0)
+        chunk = g_row_chunk;
+    else if (units < 4 * threads) {
+        const int per_unit = (4 * threads + units - 1) / units;
+        chunk = (s->T + per_unit - 1) / per_unit;
+        if (chunk < 256) chunk = 256;
+    }
+    const int nchunks = (s->T + chunk - 1) / chunk;
+    const int warm = 2 * (s->c_q - 1);
+    int failed = 0;
+#ifdef _OPENMP
 #pragma omp parallel for schedule(dynamic, 1) reduction(|:failed)
 #endif
-    for (int un = 0; un < units; ++un) {
-        int b = un / G, g = un % G;
+    for (int task = 0; task < units * nchunks; ++task) {
+        /* later chunks cost more (causal rows grow): start with them */
+        const int un = task % units, ch = nchunks - 1 - task / units;
+        const int b = un / G, g = un % G;
+        const int first = ch * chunk;
+        const int last = first + chunk < s->T ? first + chunk : s->T;
         unit_buffers u;
         if (!alloc_unit(s, &u)) { failed |= 1; free_unit(&u); continue; }
         const size_t T = (size_t)s->T;
-        for (int i = 0; i < s->T; ++i) {
+        for (int i = first - warm > 0 ? first - warm : 0; i < last; ++i) {
             /* the new rows i take the ring slots of rows i - c_q */
             const size_t slot = (size_t)(i % s->c_q);
             for (int hh = 0; hh < s->c_h; ++hh)
@@ -433,6 +460,7 @@ static int forward_args(const mta_oracle_shape *s, const mta_oracle_args *pa, do
             for (int hh = 0; hh < s->c_h; ++hh)
                 memcpy(u.ring1 + ((size_t)hh * s->c_q + slot) * T, u.A1 + (size_t)hh * T,
                        T * sizeof(double));
+            if (i < first) continue;   /* warm-up row: rings only */
             point_rows(s, u.ring1, i, u.zero, u.rows1);
             second_stage(s, &a, b, g, i, &u, u.rows1, out + ((size_t)b * s->T + i) * HD, NULL);
         }
@@ -645,6 +673,9 @@ int mta_oracle_stages_composed(const mta_oracle_shape *s, const double *q, const
     mta_oracle_args a = composed_args(q, k, v, c, gn_weight, gn_bias, depth_scale, gate);
     return stages_args(s, &a, b, C, P, A1, A, O, out);
 }
+
+/* Rows per task of the full forward (0: chosen from the thread count). */
+void mta_oracle_set_row_chunk(int rows) { g_row_chunk = rows > 0 ? rows : 0; }
 
 int mta_oracle_max_threads(void)
 {

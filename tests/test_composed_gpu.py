@@ -18,7 +18,8 @@ import oracle
 import convolved_logit_attention_b200 as mta
 from convolved_logit_attention_b200.workloads import (COMPOSITIONS, WORKLOADS, Workload,
                                                       composed_inputs)
-from tests.test_parity_gpu import assert_close, sample_rows
+from tests.test_parity_gpu import assert_close
+from tests.test_parity_full_gpu import assert_every_element
 
 pytestmark = pytest.mark.gpu
 
@@ -165,20 +166,17 @@ def test_traced_launches_follow_the_chain():
 
 
 @pytest.mark.parametrize("comp", ["repeat", "both_post", "exact_both_pre", "conv3d"])
-def test_full_size_sampled_rows(comp):
-    """The T = 4096 workload (two [B,H,T,T] fp32 maps, 4.3 GB) on rows
-    sampled per batch entry, including tile edges and both ends."""
+def test_full_size_every_element(comp):
+    """The T = 4096 workload (two [B,H,T,T] fp32 maps, 4.3 GB), every element
+    against the oracle's full forward of the same composition."""
     w = WORKLOADS["longctx_4k"]
     x = composed_inputs(w, comp)
     d = to_device(x, w.io)
     got = run(d, x)
     del d
     torch.cuda.empty_cache()
-    rng = np.random.default_rng(13)
-    for b in range(w.B):
-        rows = sample_rows(w.T, rng, n=6)
-        ref = oracle.rows_composed(x["q"], x["k"], x["v"], *(x[n] for n in WEIGHTS),
-                                   x["gn_weight"], x["gn_bias"], x["depth_scale"], b, rows,
-                                   gn_eps=x["gn_eps"], w_head_pre=x["w_head_pre"],
-                                   exact_mask=x["exact_mask"], w_kq_3d=x["w_kq_3d"])
-        assert_close(got[b, rows], ref, w.io, "longctx_4k %s b=%d" % (comp, b))
+    ref = oracle.forward_composed(x["q"], x["k"], x["v"], *(x[n] for n in WEIGHTS),
+                                  x["gn_weight"], x["gn_bias"], x["depth_scale"],
+                                  gn_eps=x["gn_eps"], w_head_pre=x["w_head_pre"],
+                                  exact_mask=x["exact_mask"], w_kq_3d=x["w_kq_3d"])
+    assert_every_element(got, ref, w.H, w.d, "longctx_4k " + comp)

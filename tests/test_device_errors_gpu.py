@@ -50,3 +50,24 @@ def test_values_beyond_fp16_range_are_reported():
         mta.mta_sync_status()
     assert exc.value.status == -7
     mta.mta_sync_status()   # cleared
+
+
+def test_check_flag_raises_at_the_call():
+    # check=True synchronises the call's stream and raises what the device
+    # flagged, so a torch caller does not get non-finite output silently
+    w = Workload("range_check", 1, 2, 130, 64, 6, 11, 2, "bf16", seed=3)
+    x = make_inputs(w)
+    dev = torch.device("cuda", 0)
+    d = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v")}
+    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
+        d[n] = torch.from_numpy(x[n]).to(dev)
+    mta.mta_sync_status()
+    out = mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                          d["gn_bias"], x["depth_scale"], check=True)
+    assert torch.isfinite(out.float()).all()
+    d["k"][0, 0, 40, 5] = 2.0e5
+    with pytest.raises(mta.MtaError) as exc:
+        mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                        d["gn_bias"], x["depth_scale"], check=True)
+    assert exc.value.status == -7
+    mta.mta_sync_status()   # cleared

@@ -320,3 +320,27 @@ def test_workload_flop_count_uses_pages_mac_count():
     w = WORKLOADS["longctx_4k"]
     per_logit = w.algorithmic_flops() // (w.B * w.H * w.live_logits())
     assert per_logit == 4 * w.d + 2 * 66 + 2 * w.c_h
+
+
+@pytest.mark.parametrize("chunk", [1, 5, 7, 16])
+def test_row_chunks_change_no_bit(chunk):
+    """The full forward split into row chunks (each warming its rings up on
+    the rows before it) gives the same bits as the unsplit loop, for the
+    default module and for a composition with a post-softmax conv, whose
+    second ring needs the longest warm-up."""
+    rng = np.random.default_rng(31)
+    B, H, T, d, c_q, c_k, c_h = 1, 4, 37, 8, 6, 11, 2
+    q, k, v, th, w, gw, gb = rand_inputs(rng, B, H, T, d, c_q, c_k, c_h)
+    th2 = 0.3 * rng.standard_normal(th.shape)
+    w2 = rng.standard_normal(w.shape)
+    try:
+        oracle.set_row_chunk(T)
+        ref = oracle.forward(q, k, v, th, w, gw, gb, 0.8)
+        ref_c = oracle.forward_composed(q, k, v, th, w, th2, w2, gw, gb, 0.8)
+        oracle.set_row_chunk(chunk)
+        got = oracle.forward(q, k, v, th, w, gw, gb, 0.8)
+        got_c = oracle.forward_composed(q, k, v, th, w, th2, w2, gw, gb, 0.8)
+    finally:
+        oracle.set_row_chunk(0)
+    assert np.array_equal(got, ref)
+    assert np.array_equal(got_c, ref_c)
