@@ -68,6 +68,9 @@ def parse_args(argv=None):
                         "instead of mta_forward")
     p.add_argument("--compose", choices=sorted(COMPOSITIONS), default=None,
                    help="time mta_forward_composed on this composition of the module")
+    p.add_argument("--backward", action="store_true",
+                   help="time mta_backward (gradients of the default composition for a seeded "
+                        "upstream gradient) instead of the forward")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -222,13 +225,20 @@ def kernel_units(name, w, comp=None):
         "k_softmax_mix": ("hbm", logits * 8, "B"),            # read C, write A_new (fp32)
         "k_head_mix": ("hbm", logits * 8, "B"),               # read and write one fp32 map
         "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
-        # read k, write the c_q folded-key copies (fp16)
-        "k_fold_keys": ("hbm", w.B * w.H * w.T * w.d * 2 * (1 + w.c_q), "B"),
-        # read q and k, write the permuted q (fp16) and the 16-entry correction rows
-        "k_fold_aux": ("hbm", w.B * w.H * w.T * (w.d * 2 * 3 + 64), "B"),
+        # the prologue: read k, write the c_q folded-key copies (fp16); read q
+        # and k, write the permuted q (fp16) and the 16-entry correction rows
+        "k_fold": ("hbm", w.B * w.H * w.T * (w.d * 2 * (1 + w.c_q) + w.d * 2 * 3 + 64), "B"),
         "k_mta_fused": ("tensor", w.algorithmic_flops(), "FLOP"),
         # read the fp16 partial outputs (c_h per output head), write out
         "k_mix_groupnorm": ("hbm", w.B * w.T * w.H * w.d * (2 * w.c_h + io_bytes), "B"),
+        # backward: causal products of a map with a [T, d] operand, 2d FLOP per live logit
+        "k_causal_mm": ("alu", logits * 2 * w.d, "FLOP"),
+        # read O and dout, write dO (fp32)
+        "k_gn_bwd": ("hbm", w.B * w.H * w.T * w.d * (4 + io_bytes + 4), "B"),
+        # read dA and P twice, write dC (fp32 maps)
+        "k_mix_softmax_bwd": ("hbm", logits * 20, "B"),
+        "k_conv_adj": ("alu", logits * 2 * w.c_q * w.c_k, "FLOP"),
+        "k_dtheta": ("alu", logits * 2 * w.c_q * w.c_k, "FLOP"),
     }
     return table.get(name, ("unknown", 0, "FLOP"))
 
@@ -370,6 +380,97 @@ def time_mta(args, w, d, world, device):
         per_kernel[name] /= names.count(name)
     return {"total_ms": total_ms, "per_kernel_ms": per_kernel, "names": names,
             "launches": nk * args.steps, "clocks": sampler.summary(), "path": path}
+
+
+def backward_flops(w):
+    """Algorithmic FLOPs of the gradients (the forward's recompute excluded):
+    per live logit dA = dO V^T and dV = A^T dO (2d each), the mix backward
+    and the dw sums (c_h MACs each), the adjoint convolution and the kernel
+    gradient (c_q c_k MACs each), dQ and dK (2d each): twice the forward's
+    4d + 2 c_q c_k + 2 c_h."""
+    return 2 * w.algorithmic_flops()
+
+
+def time_backward(args, w, x, d, world, device):
+    """K timed mta_backward calls (L2 flushed before each), then a traced
+    pass for the per-kernel breakdown."""
+    import convolved_logit_attention_b200 as mta
+    dt = torch.bfloat16 if w.io == "bf16" else torch.float32
+    rng = np.random.default_rng(w.seed + 1000)
+    dout = torch.from_numpy(rng.standard_normal((w.B, w.T, w.H * w.d)).astype(np.float32))
+    dout = dout.to(device).to(dt)
+    shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"], w.gn_eps)
+    names = mta.mta_backward_kernel_names(shape)
+    ws = torch.empty(mta.mta_backward_workspace_size(shape), dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(events=None):
+        mta.mta_backward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                         d["gn_bias"], w.depth_scale, dout, workspace=ws, stream=stream,
+                         gn_eps=w.gn_eps, events=events)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    mta.mta_sync_status(stream, device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with sampler:
+        for s in range(args.steps):
+            flush.zero_()
+            ev[s][0].record(stream)
+            step()
+            ev[s][1].record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world)
+    mta.mta_sync_status(stream, device)
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    n_tr = min(args.steps, 3)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
+           for _ in range(n_tr)]
+    for s in range(n_tr):
+        flush.zero_()
+        step(kev[s])
+    torch.cuda.synchronize(device)
+    per_kernel = {}
+    for i, name in enumerate(names):
+        per_kernel[name] = per_kernel.get(name, 0.0) + sum(
+            kev[s][2 * i].elapsed_time(kev[s][2 * i + 1]) for s in range(n_tr)) / n_tr
+    for name in per_kernel:
+        per_kernel[name] /= names.count(name)
+    return {"total_ms": total_ms, "per_kernel_ms": per_kernel, "names": names,
+            "launches": len(names) * args.steps, "clocks": sampler.summary()}
+
+
+def backward_line(args, w, x, d, world, rank, device):
+    peaks, peak_src = load_peaks()
+    res = time_backward(args, w, x, d, world, device)
+    total_ms = dist_max(res["total_ms"], world, device)
+    flops = backward_flops(w)
+    value = replica_tflops(world, flops, args.steps, total_ms)
+    kernels = res["per_kernel_ms"]
+    dom = max(kernels, key=lambda n: kernels[n] * res["names"].count(n))
+    rl = roofline(dom, w, kernels[dom], peaks, peak_src)
+    line = {"metric": "MTA bwd TFLOP/s at T=4096 (gradient FLOPs, 2x the forward's; the "
+                      "forward recompute excluded)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": dict(workload_config(w, "materialised backward"), **{"pass": "backward"}),
+            "tokens_per_s": world * w.tokens() * args.steps / (total_ms / 1e3),
+            "peaks": dict(peaks, source=peak_src),
+            "roofline": {k: rl[k] for k in ("bound", "achieved", "peak", "unit", "frac",
+                                             "traffic")},
+            "kernels": [dict(roofline(n, w, kernels[n], peaks, peak_src),
+                             launches_per_step=res["names"].count(n))
+                        for n in dict.fromkeys(res["names"])],
+            "gpu_launches": res["launches"], "clocks": res["clocks"]}
+    return line if rank == 0 else None
 
 
 def time_e2e(args, w, x, device):
@@ -559,6 +660,8 @@ def mta_arm(args, w, world, rank, local):
     x = (composed_inputs(w, args.compose, seed=w.seed + rank) if args.compose
          else make_inputs(w, seed=w.seed + rank))
     d = device_inputs(x, w.io, device)
+    if args.backward:
+        return backward_line(args, w, x, d, world, rank, device)
     peaks, peak_src = load_peaks()
     res = time_mta(args, w, d, world, device)
     bad = [r for r in res["clocks"]["reasons"] if r in BAD_REASONS]

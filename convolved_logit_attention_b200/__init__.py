@@ -13,7 +13,8 @@ from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
                        mta_forward_unfused, mta_kernel_count, mta_kernel_name,
                        mta_selftest_wait_timeout,
                        mta_status_string, mta_sync_status, mta_unfused_workspace_size,
-                       mta_version, mta_workspace_size, shape_of)
+                       mta_version, mta_workspace_size, shape_of, GRAD_NAMES, mta_backward,
+                       mta_backward_kernel_names, mta_backward_workspace_size)
 
 __all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC",
            "MTA_PATH_MATERIALISED", "MtaComposition", "MtaError", "MtaShape", "lib",
@@ -23,4 +24,5 @@ __all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC",
            "mta_forward_unfused", "mta_kernel_count", "mta_kernel_name",
            "mta_selftest_wait_timeout",
            "mta_status_string", "mta_sync_status", "mta_unfused_workspace_size", "mta_version",
-           "mta_workspace_size", "shape_of"]
+           "mta_workspace_size", "shape_of", "GRAD_NAMES", "mta_backward",
+           "mta_backward_kernel_names", "mta_backward_workspace_size"]

@@ -27,7 +27,9 @@ EXPORTS = ("mta_version", "mta_status_string", "mta_forward_path", "mta_workspac
            "mta_debug_attention", "mta_kernel_count", "mta_kernel_name", "mta_forward_traced",
            "mta_selftest_wait_timeout", "mta_forward_noalloc", "mta_sync_status",
            "mta_forward_gated", "mta_composed_workspace_size", "mta_forward_composed",
-           "mta_forward_composed_traced", "mta_composed_kernel_count", "mta_composed_kernel_name")
+           "mta_forward_composed_traced", "mta_composed_kernel_count", "mta_composed_kernel_name",
+           "mta_backward", "mta_backward_traced", "mta_backward_workspace_size",
+           "mta_backward_kernel_count", "mta_backward_kernel_name")
 
 
 class MtaShape(ctypes.Structure):
@@ -105,6 +107,17 @@ def lib():
         L.mta_composed_kernel_count.restype = ctypes.c_int
         L.mta_composed_kernel_name.argtypes = [sp, cp, ctypes.c_int]
         L.mta_composed_kernel_name.restype = ctypes.c_char_p
+        bwd = [sp, vp, vp, vp, fp, fp, fp, fp, ctypes.c_float, fp, vp] + [fp] * 8 + \
+            [vp, ctypes.c_size_t, vp]
+        L.mta_backward.argtypes, L.mta_backward.restype = bwd, ctypes.c_int
+        L.mta_backward_traced.argtypes = bwd + [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+        L.mta_backward_traced.restype = ctypes.c_int
+        L.mta_backward_workspace_size.argtypes = [sp]
+        L.mta_backward_workspace_size.restype = ctypes.c_size_t
+        L.mta_backward_kernel_count.argtypes = [sp]
+        L.mta_backward_kernel_count.restype = ctypes.c_int
+        L.mta_backward_kernel_name.argtypes = [sp, ctypes.c_int]
+        L.mta_backward_kernel_name.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -418,3 +431,55 @@ def mta_forward_composed(q, k, v, w_kq=None, w_head=None, w_kq_post=None, w_head
                lib().mta_forward_composed_traced(*args, handles, len(events)))
     _after(check, stream, q.device)
     return out
+
+
+GRAD_NAMES = ("q", "k", "v", "w_kq", "w_head", "gn_weight", "gn_bias")
+
+
+def mta_backward_workspace_size(shape: MtaShape) -> int:
+    return lib().mta_backward_workspace_size(ctypes.byref(shape))
+
+
+def mta_backward_kernel_names(shape: MtaShape):
+    n = lib().mta_backward_kernel_count(ctypes.byref(shape))
+    return [lib().mta_backward_kernel_name(ctypes.byref(shape), i).decode() for i in range(n)]
+
+
+def mta_backward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, dout, gate=None,
+                 workspace=None, stream=None, gn_eps=1e-5, events=None, check=False):
+    """Gradients of the forward (mta_forward, or mta_forward_gated with gate)
+    for the upstream gradient dout [B, T, H*d] (q's dtype): a dict of float32
+    tensors keyed by the input names (GRAD_NAMES, plus "gate" with a gate).
+    With events (torch.cuda.Event, two per launch) the traced entry records
+    them around its launches."""
+    _check_inputs(q, k, v, w_kq, w_head, gn_weight, gn_bias)
+    B, H, T, d = q.shape
+    if (dout.shape != (B, T, H * d) or dout.dtype != q.dtype or dout.device != q.device
+            or not dout.is_contiguous()):
+        raise ValueError("dout must be a contiguous [B, T, H*d] tensor like q")
+    if gate is not None and (gate.dtype != torch.float32 or gate.shape != (H,)
+                             or gate.device != q.device or not gate.is_contiguous()):
+        raise ValueError("gate must be a contiguous float32 [H] tensor on q's device")
+    shape = shape_of(q, w_kq, w_head, gn_eps)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"q": torch.empty(q.shape, **f32), "k": torch.empty(q.shape, **f32),
+         "v": torch.empty(q.shape, **f32), "w_kq": torch.empty(w_kq.shape, **f32),
+         "w_head": torch.empty(w_head.shape, **f32), "gn_weight": torch.empty(H * d, **f32),
+         "gn_bias": torch.empty(H * d, **f32)}
+    if gate is not None:
+        g["gate"] = torch.empty(H, **f32)
+    ws = _workspace(mta_backward_workspace_size(shape), q.device, workspace)
+    args = [ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(w_kq), _ptr(w_head),
+            _ptr(gn_weight), _ptr(gn_bias), float(depth_scale), _ptr(gate), _ptr(dout)]
+    args += [_ptr(g[n]) for n in GRAD_NAMES] + [_ptr(g.get("gate"))]
+    args += [_ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream, q.device)]
+    if events is None:
+        _check("mta_backward", lib().mta_backward(*args))
+    else:
+        for e in events:
+            if not e.cuda_event:
+                e.record()
+        handles = (ctypes.c_void_p * max(len(events), 1))(*[e.cuda_event for e in events])
+        _check("mta_backward_traced", lib().mta_backward_traced(*args, handles, len(events)))
+    _after(check, stream, q.device)
+    return g

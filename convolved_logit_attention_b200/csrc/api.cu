@@ -65,7 +65,7 @@ const char *mta_status_string(mta_status st)
         case MTA_ERR_WORKSPACE: return "workspace too small";
         case MTA_ERR_CUDA: return "CUDA runtime error";
         case MTA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
-        case MTA_ERR_RANGE: return "value outside the fp16 range of the fused path";
+        case MTA_ERR_RANGE: return "non-finite input on the fused path";
     }
     return "unknown status";
 }
@@ -95,7 +95,7 @@ mta_status forward_impl(int unfused, const mta_shape *s, const void *q, const vo
                         const void *v, const float *w_kq, const float *w_head,
                         const float *gn_weight, const float *gn_bias, float depth_scale,
                         const float *gate, void *out, void *workspace, size_t workspace_bytes,
-                        void *stream, void *const *events, int n_events)
+                        void *stream, void *const *events, int n_events, int exact_mask = 0)
 {
     mta_status rc = check_shape(s);
     if (rc == MTA_OK) rc = check_tensors(q, k, v, w_kq, w_head, gn_weight, gn_bias, out);
@@ -106,6 +106,7 @@ mta_status forward_impl(int unfused, const mta_shape *s, const void *q, const vo
     rc = check_workspace(workspace, workspace_bytes, need);
     if (rc != MTA_OK) return rc;
     mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out, gate};
+    a.exact_mask = exact_mask;
     mta::Trace tr;
     tr.events = events;
     tr.n = n_events;
@@ -139,10 +140,12 @@ mta_status mta_forward_gated(const mta_shape *s, const void *q, const void *k, c
 
 namespace {
 
+// The pages' default composition {w_kq, w_head}, under either masking of the
+// first convolution: mta_forward's path (fused where mta_forward_path says so).
 bool is_default_composition(const mta_composition *c)
 {
     return c->w_kq && c->w_head && !c->w_kq_post && !c->w_head_post && !c->w_head_pre &&
-           !c->exact_mask && !c->w_kq_3d;
+           !c->w_kq_3d;
 }
 
 mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const void *v,
@@ -154,7 +157,8 @@ mta_status composed_impl(const mta_shape *s, const void *q, const void *k, const
     if (gate && ((uintptr_t)gate & 3u) != 0) return MTA_ERR_ALIGNMENT;
     if (is_default_composition(c))
         return forward_impl(0, s, q, k, v, c->w_kq, c->w_head, gn_weight, gn_bias, depth_scale,
-                            gate, out, workspace, workspace_bytes, stream, events, n_events);
+                            gate, out, workspace, workspace_bytes, stream, events, n_events,
+                            c->exact_mask != 0);
     mta_status rc = check_shape(s);
     if (rc != MTA_OK) return rc;
     const void *need[] = {q, k, v, gn_weight, gn_bias, out};
@@ -303,6 +307,64 @@ mta_status mta_debug_attention(const mta_shape *s, const void *q, const void *k,
     if (rc != MTA_OK) return rc;
     return mta::launch_debug_attention(*s, q, k, w_kq, w_head, attn, stage, workspace,
                                        (cudaStream_t)stream);
+}
+
+size_t mta_backward_workspace_size(const mta_shape *s)
+{
+    if (check_shape(s) != MTA_OK) return 0;
+    return mta::backward_workspace_bytes(*s);
+}
+
+int mta_backward_kernel_count(const mta_shape *s)
+{
+    return check_shape(s) == MTA_OK ? mta::kBackwardKernels : 0;
+}
+
+const char *mta_backward_kernel_name(const mta_shape *s, int index)
+{
+    if (check_shape(s) != MTA_OK || index < 0 || index >= mta::kBackwardKernels) return nullptr;
+    return mta::kBackwardKernelNames[index];
+}
+
+mta_status mta_backward_traced(const mta_shape *s, const void *q, const void *k, const void *v,
+                               const float *w_kq, const float *w_head, const float *gn_weight,
+                               const float *gn_bias, float depth_scale, const float *gate,
+                               const void *dout, float *dq, float *dk, float *dv, float *dw_kq,
+                               float *dw_head, float *dgn_weight, float *dgn_bias, float *dgate,
+                               void *workspace, size_t workspace_bytes, void *stream,
+                               void *const *events, int n_events)
+{
+    mta_status rc = check_shape(s);
+    if (rc == MTA_OK) rc = check_tensors(q, k, v, w_kq, w_head, gn_weight, gn_bias, dout);
+    if (rc != MTA_OK) return rc;
+    const void *grads[] = {dq, dk, dv, dw_kq, dw_head, dgn_weight, dgn_bias};
+    for (const void *p : grads)
+        if (!p) return MTA_ERR_INVALID_ARG;
+    for (const void *p : grads)
+        if (!aligned(p, 16)) return MTA_ERR_ALIGNMENT;
+    if ((gate == nullptr) != (dgate == nullptr)) return MTA_ERR_INVALID_ARG;
+    if (gate && (!aligned(gate, 4) || !aligned(dgate, 4))) return MTA_ERR_ALIGNMENT;
+    if (n_events < 0 || (n_events > 0 && !events)) return MTA_ERR_INVALID_ARG;
+    rc = check_workspace(workspace, workspace_bytes, mta::backward_workspace_bytes(*s));
+    if (rc != MTA_OK) return rc;
+    mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, nullptr, gate};
+    mta::BackwardArgs g{dout, dq, dk, dv, dw_kq, dw_head, dgn_weight, dgn_bias, dgate};
+    mta::Trace tr;
+    tr.events = events;
+    tr.n = n_events;
+    return mta::launch_backward(*s, a, g, workspace, (cudaStream_t)stream, tr);
+}
+
+mta_status mta_backward(const mta_shape *s, const void *q, const void *k, const void *v,
+                        const float *w_kq, const float *w_head, const float *gn_weight,
+                        const float *gn_bias, float depth_scale, const float *gate,
+                        const void *dout, float *dq, float *dk, float *dv, float *dw_kq,
+                        float *dw_head, float *dgn_weight, float *dgn_bias, float *dgate,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    return mta_backward_traced(s, q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gate,
+                               dout, dq, dk, dv, dw_kq, dw_head, dgn_weight, dgn_bias, dgate,
+                               workspace, workspace_bytes, stream, nullptr, 0);
 }
 
 mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stream)

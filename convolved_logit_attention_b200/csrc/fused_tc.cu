@@ -11,16 +11,19 @@
 // floor(c_k/2) diagonals of the main one, and a per-row correction table
 // subtracts them there.
 //
-// Four kernels:
-//   k_fold_keys      per (b, h, 128-key block): Kf^{(i')} for every i' (fp16,
-//                    scaled by log2(e)/sqrt(d) so that the softmax runs on
-//                    exp2).  fp16 carries three more mantissa bits than bf16
-//                    for the folded logits; values outside its range raise an
-//                    error.
-//   k_fold_aux       per (b, h, 128-row block): the query rows of the block
-//                    (fp16) in the permuted order the main kernel's shifted
-//                    operand needs, and the correction table corr[i][e] for
-//                    key j = i - e.
+// Three kernels, launched back to back on the caller's stream (the last two
+// with programmatic dependent launch, so each is scheduled while its
+// predecessor drains):
+//   k_fold           the prologue, CTAs in two roles:
+//                    - per (b, h, 128-key block): Kf^{(i')} for every i' (fp16,
+//                      scaled by log2(e)/sqrt(d) so that the softmax runs on
+//                      exp2).  fp16 carries three more mantissa bits than bf16
+//                      for the folded logits; values outside its range raise an
+//                      error.
+//                    - per (b, h, 64-row half block): the query rows (fp16) in
+//                      the permuted order the main kernel's shifted operand
+//                      needs, and the correction table corr[i][e] for key
+//                      j = i - e.
 //   k_mta_fused      per (b, source head h', 128 query rows): for every key
 //                    tile, S = sum_{i'} Q_{shift i'} Kf^{(i')T} on tcgen05
 //                    (TMEM accumulator), correction + causal mask + online
@@ -75,7 +78,7 @@ __host__ __device__ inline int d_m(int c_q, int c_k) { return c_q - 1 + c_k / 2;
 constexpr int kProRows = 128;     // rows (keys and queries) per prologue CTA
 constexpr int kProQLo = 7;        // query rows before the block whose future logits are needed
 constexpr int kAuxRows = 64;      // query rows per aux prologue CTA
-constexpr int kAuxThreads = 160;  // aux prologue: one future-logit work item per thread
+constexpr int kProThreads = 256;  // threads of a prologue CTA (either role)
 
 // Packed fp32 pairs (Blackwell's f32x2 arithmetic): one instruction does two
 // fp32 FMAs, each rounded once, exactly as fmaf would.
@@ -127,6 +130,52 @@ __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Largest |x| over rows [r_lo, r_hi) (clipped to [0, T)) of one head's bf16
+// [T][D] rows, reduced over the CTA (blockDim.x a multiple of 32, at most
+// 256): every thread gets the result.  A non-finite element anywhere makes
+// the result +inf.  `red` is 8 floats of shared memory.
+template <int D>
+__device__ float rows_absmax(const __nv_bfloat16 *__restrict__ head, int r_lo, int r_hi, int T,
+                             float *red)
+{
+    const int lo = r_lo > 0 ? r_lo : 0, hi = r_hi < T ? r_hi : T;
+    float m = 0.f;
+    bool finite = true;
+    for (int idx = threadIdx.x; idx < (hi - lo) * (D / 8); idx += blockDim.x) {
+        const uint4 v = *(const uint4 *)(head + (size_t)(lo + idx / (D / 8)) * D + 8 * (idx % (D / 8)));
+        const __nv_bfloat162 *p = (const __nv_bfloat162 *)&v;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float2 f = __bfloat1622float2(p[u]);
+            finite &= fabsf(f.x) <= 3.0e38f && fabsf(f.y) <= 3.0e38f;   // false for NaN too
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+    if (!finite) m = INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __syncthreads();                           // red may still be read by an earlier use
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = m;
+    __syncthreads();
+    float r = red[0];
+    for (int w = 1; w < (int)blockDim.x / 32; ++w) r = fmaxf(r, red[w]);
+    return r;
+}
+
+// The power-of-two exponent e >= 0 of a block's fp16 operand scale: the
+// smallest e with bound * 2^-e <= 2^14, a quarter of the fp16 range, so that
+// sums of the block's products stay far from overflow.  Blocks whose bound is
+// already below it keep e = 0 (the usual case: the fused path then computes
+// exactly as without scaling).  Returns -1 for a non-finite bound.
+__device__ __forceinline__ int range_exponent(float bound)
+{
+    if (bound <= 16384.f) return 0;
+    if (!(bound <= 3.0e38f)) return -1;
+    int e = 0;
+    frexpf(bound / 16384.f, &e);               // bound / 2^14 <= 2^e
+    return e;
+}
+
 // Folded keys: one CTA per (128-key block, b*H + h), 256 threads; thread =
 // one column pair x a run of RPG consecutive keys, in windows of SUB keys.
 // Kf^{(i')}_j = sum_jj ths[i'][jj] k_{j + RT - jj}, with the taps zero-padded
@@ -134,9 +183,11 @@ __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a
 // real kernel, so every tap index is a compile-time constant.  The two
 // columns of a pair share every tap: one packed f32x2 FMA per tap.
 template <int D, int CK>
-__global__ void __launch_bounds__(256, 3)
-k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
-            __half *__restrict__ kf, int T, int Tp, int H, int c_q, int c_k, float scale)
+__device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bfloat16 *__restrict__ k,
+                                                const float *__restrict__ w_kq,
+                                                __half *__restrict__ kf, int *__restrict__ kexp,
+                                                int T, int Tp, int H, int nqb, int c_q, int c_k,
+                                                float scale)
 {
     constexpr int EP = D / 2;                  // column pairs
     constexpr int RG = 256 / EP;               // key runs per block
@@ -145,7 +196,7 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
     constexpr int SUB = 16;
     constexpr int WS = SUB + CK - 1;           // window rows
     __shared__ float ths[8 * CK];              // zero-padded taps times the logit scale
-    const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
+    const int h = bh % H;
     const int j0 = blk * kProRows;
     const int tid = threadIdx.x;
     const int R = c_k / 2, shift = RT - R;     // real tap jj sits at padded index jj + shift
@@ -154,7 +205,30 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
         ths[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] * scale
                                                      : 0.f;
     }
+    // Range of the block's folded keys: |Kf^{(i')}_j| <= max |k| over the
+    // window rows times max_{i'} sum_{j'} |theta'|.  Beyond 2^14 the taps are
+    // scaled by 2^-e (exactly), and the main kernel multiplies the logits of
+    // this key block back by 2^e.
+    __shared__ float red[8];
+    __shared__ int s_e;
+    const float mk = rows_absmax<D>(k + (size_t)bh * T * D, j0 - LT, j0 + kProRows + RT, T, red);
+    if (tid == 0) {
+        float tb = 0.f;
+        for (int ip = 0; ip < c_q; ++ip) {
+            float a = 0.f;
+            for (int jj = 0; jj < CK; ++jj) a += fabsf(ths[ip * CK + jj]);
+            tb = fmaxf(tb, a);
+        }
+        int e = range_exponent(mk * tb);
+        if (e < 0) { atomicOr(&g_fused_error, kErrRange); e = 0; }
+        s_e = e;
+        kexp[(size_t)bh * nqb + blk] = e;
+    }
     __syncthreads();
+    if (s_e != 0) {
+        for (int idx = tid; idx < 8 * CK; idx += 256) ths[idx] = ldexpf(ths[idx], -s_e);
+        __syncthreads();
+    }
     const int ep = tid % EP, rg = tid / EP;
     const __nv_bfloat16 *kh = k + (size_t)bh * T * D + 2 * ep;
     __half2 amax = __floats2half2_rn(0.f, 0.f);   // largest |Kf| this thread wrote, per column
@@ -188,7 +262,8 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
             }
         }
     }
-    // a folded key beyond the fp16 range became infinite (NaN inputs stay NaN)
+    // a folded key beyond the fp16 range became infinite: only non-finite
+    // inputs get here after the scaling above (NaN inputs stay NaN)
     const float2 am = __half22float2(amax);
     if (am.x > 65504.f || am.y > 65504.f) atomicOr(&g_fused_error, kErrRange);
 }
@@ -200,26 +275,32 @@ k_fold_keys(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ w_kq,
 //      [1, D_m], for r in [j0 - 7, j0 + 64), from shared-memory copies of
 //      the rows involved.
 //  (d) corr[i][e] = sum over taps (i', j') with delta = i' - j' - e >= 1 and
-//      r = i - i' >= 0 of theta[i'][j'] F[r][delta].
+//      r = i - i' >= 0 of theta[i'][j'] F[r][delta]: the terms of keys past
+//      the tap's own query row r, which Mask_0 of Eq. (5) removes.  With
+//      `exact` (the indicator of Eq. (4), which keeps a tap whenever its key
+//      is not past the output's query i) only the terms with delta > i',
+//      that is key r + delta > i, are removed.
 template <int D>
-__global__ void __launch_bounds__(kAuxThreads, 4)
-k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-           const float *__restrict__ w_kq, __half *__restrict__ qp, float *__restrict__ corr, int T,
-           int Tp, int H, int c_q, int c_k, float scale)
+__device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloat16 *__restrict__ q,
+                                               const __nv_bfloat16 *__restrict__ k,
+                                               const float *__restrict__ w_kq,
+                                               __half *__restrict__ qp, float *__restrict__ corr,
+                                               int *__restrict__ qexp, int T, int Tp, int H,
+                                               int nqb, int c_q, int c_k, float scale, int exact)
 {
     constexpr int QR = kProQLo + kAuxRows;
     constexpr int TW = 16;                     // tap row stride (c_k <= 15)
     __shared__ float th[8 * TW];
     __shared__ float fs[QR * kCorrW];
     extern __shared__ __align__(16) __nv_bfloat16 qk_sm[];   // section (c) row copies
-    const int blk = blockIdx.x, bh = blockIdx.y, h = bh % H;
+    const int h = bh % H;
     const int j0 = blk * kAuxRows;
     // the 128-row query block whose permuted rows this CTA writes one half of
     const int qblk = j0 / kProRows, half = (j0 % kProRows) / kAuxRows;
     const int tid = threadIdx.x;
     const size_t head_off = (size_t)bh * T * D;
     const int R = c_k / 2;
-    for (int idx = tid; idx < 8 * TW; idx += kAuxThreads) {
+    for (int idx = tid; idx < 8 * TW; idx += kProThreads) {
         const int ip = idx / TW, jj = idx % TW;
         th[idx] = (ip < c_q && jj < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jj] : 0.f;
     }
@@ -235,7 +316,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     constexpr int CPR = D / 8;                 // 16-byte chunks per row
     __nv_bfloat16 *qsm = qk_sm;                // [QRP][RS]
     __nv_bfloat16 *ksm = qk_sm + QRP * RS;     // [KRP][RS]
-    for (int idx = tid; idx < (QRP + KRP) * CPR; idx += kAuxThreads) {
+    for (int idx = tid; idx < (QRP + KRP) * CPR; idx += kProThreads) {
         const int row = idx / CPR, c8 = idx % CPR;
         const bool isq = row < QRP;
         const int lr = isq ? row : row - QRP;
@@ -246,6 +327,20 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
     tc::cp_async_wait_all();
     __syncthreads();
+    // Range of the 128-row block's permuted queries (rows i0 - c_q + 1 ..
+    // i0 + 127, the same for both halves' CTAs): beyond 2^14 they are scaled
+    // by 2^-e before the fp16 rounding, and the main kernel multiplies this
+    // block's logits back by 2^e.
+    __shared__ float red[8];
+    int eq;
+    {
+        const int i0 = qblk * kProRows;
+        const float mq = rows_absmax<D>(q + head_off, i0 - (c_q - 1), i0 + kProRows, T, red);
+        eq = range_exponent(mq);
+        if (eq < 0) { if (tid == 0) atomicOr(&g_fused_error, kErrRange); eq = 0; }
+        if (tid == 0 && half == 0) qexp[(size_t)bh * nqb + qblk] = eq;
+    }
+    const float qsc = ldexpf(1.f, -eq);       // exact: a power of two
     // (b) permuted query rows of the 128-row block jb0 = j0 - 64*half: atom a,
     //     row s <- q_{jb0-(c_q-1)+a+16s}; this CTA writes rows s in
     //     [4*half, 4*half+4), which lie in its copy [j0-7, j0+64) since
@@ -254,7 +349,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
         const int NA = q_atoms(c_q);
         __half *dst = qp + ((size_t)bh * (Tp / kBM) + qblk) * (size_t)NA * 8 * D;
         bool range_ok = true;
-        for (int idx = tid; idx < NA * 4 * CPR; idx += kAuxThreads) {
+        for (int idx = tid; idx < NA * 4 * CPR; idx += kProThreads) {
             const int rowh = idx / CPR, c8 = idx % CPR;
             const int a = rowh / 4, sr = rowh % 4;                // atom, row within this half
             const int row = 8 * a + 4 * half + sr;                // row of the block's atom layout
@@ -265,7 +360,9 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
             __half2 *hp = (__half2 *)&outv;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float2 f = __bfloat1622float2(bp[u]);
+                float2 f = __bfloat1622float2(bp[u]);
+                f.x *= qsc;
+                f.y *= qsc;
                 range_ok &= fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
                 hp[u] = __floats2half2_rn(f.x, f.y);
             }
@@ -318,7 +415,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     __syncthreads();
     // taps indexed by s = e + delta: ts[i'][s] = theta[i'][i' + R - s]
     __shared__ float ts[8 * 32];
-    for (int idx = tid; idx < 8 * 32; idx += kAuxThreads) {
+    for (int idx = tid; idx < 8 * 32; idx += kProThreads) {
         const int ip = idx / 32, jj = ip + R - idx % 32;
         ts[idx] = (ip < c_q && jj >= 0 && jj < c_k) ? th[ip * TW + jj] : 0.f;
     }
@@ -342,7 +439,7 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
             for (int x = 1; x < EH + kCorrW - 1; ++x) t[x] = trow[x];
 #pragma unroll
             for (int dl = 1; dl <= kCorrW - 2; ++dl) {
-                const float f = frow[dl - 1];
+                const float f = dl > exact * ip ? frow[dl - 1] : 0.f;
                 const unsigned long long ff = f2_pack(f, f);
 #pragma unroll
                 for (int p = 0; p < EH / 2; ++p)
@@ -358,12 +455,48 @@ k_fold_aux(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict_
     }
 }
 
-// Dynamic shared memory of the aux prologue: bf16 copies of 80 query rows
-// and 96 key rows (71 and 84 used, the rest zero), each padded by 8 elements.
+// Dynamic shared memory of the aux role: bf16 copies of 80 query rows and
+// 96 key rows (71 and 84 used, the rest zero), each padded by 8 elements.
 size_t prologue_smem_bytes(int D)
 {
     const int QRP = (kProQLo + kAuxRows + 15) / 16 * 16;
     return (size_t)(QRP + QRP + 16) * (D + 8) * sizeof(__nv_bfloat16);
+}
+
+__device__ __forceinline__ void launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void wait_prerequisites()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// The whole prologue as one launch of 3 * nqb * BH CTAs in two roles: CTA
+// 3u + 1 folds the keys of 128-key block u (u = b*H*nqb + ...), CTAs 3u and
+// 3u + 2 build the permuted queries and correction rows of the two 64-row
+// halves of the same 128-row block.  The fold is bound by FP32 issue and the
+// rest by load latency, so interleaving them puts both kinds of CTA on every
+// SM and each hides the other; it also keeps the q and k rows of a block in
+// L2 for the three CTAs that read them.  The dependent main kernel may be
+// scheduled as soon as every CTA of this grid has started.
+template <int D, int CK>
+__global__ void __launch_bounds__(kProThreads, 3)
+k_fold(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+       const float *__restrict__ w_kq, __half *__restrict__ kf, __half *__restrict__ qp,
+       float *__restrict__ corr, int *__restrict__ sexp, int T, int Tp, int H, int nqb, int c_q,
+       int c_k, float scale, int exact)
+{
+    launch_dependents();
+    const int u = blockIdx.x / 3, role = blockIdx.x % 3;
+    const int bh = u / nqb, blk = u % nqb;
+    if (role == 1)
+        fold_keys_block<D, CK>(blk, bh, k, w_kq, kf, sexp + (size_t)gridDim.x / 3, T, Tp, H, nqb,
+                               c_q, c_k, scale);
+    else
+        fold_aux_block<D>(2 * blk + role / 2, bh, q, k, w_kq, qp, corr, sexp, T, Tp, H, nqb, c_q,
+                          c_k, scale, exact);
 }
 
 // ------------------------------------------------------------ main kernel
@@ -520,8 +653,8 @@ template <int D, int CH, bool PAIR>
 __global__ void __launch_bounds__(224, 1)
 k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
             const __grid_constant__ CUtensorMap mapV, const float *__restrict__ corr,
-            const float *__restrict__ w_head, __half *__restrict__ part, int T, int Tp, int H,
-            int c_q, int nqb, int nbh)
+            const int *__restrict__ sexp, const float *__restrict__ w_head,
+            __half *__restrict__ part, int T, int Tp, int H, int c_q, int nqb, int nbh)
 {
     using C = FusedCfg<D, CH, PAIR>;
     static_assert(C::kStages <= kGateQ - kGateStage0, "one gate barrier id per ring slot");
@@ -579,6 +712,9 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     if constexpr (PAIR) tc::cluster_sync();   // the peer's barriers exist before any remote use
     tc::tc_fence_after();
     const uint32_t tm = *tmem_slot;
+    // everything above overlaps the prologue's tail; its outputs (Kf, the
+    // permuted queries, the correction rows) are read only after this
+    wait_prerequisites();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -654,27 +790,6 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 advance();
                 return true;
             };
-            // L2 prefetch of key tile u of an item, so that the ring loads
-            // find it in L2
-            auto prefetch = [&](const WorkItem &it, int u) {
-                if (u >= it.ntiles) return;
-                for (int ip = 0; ip < c_q; ++ip)
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tc::tma_prefetch_3d(&mapK, 64 * c, u * kBN + (PAIR ? (int)rank * C::kKfRows : 0),
-                                            it.bh * c_q + ip);
-                for (int vs = 0; vs < C::kVSlots; ++vs) {
-                    const int z0 = it.b * H + it.g * CH + it.hh0 + vs * C::kVHeads;
-                    if (PAIR && C::kVHeads == 2) {
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tc::tma_prefetch_3d(&mapV, 64 * c, u * kBN, z0 + (int)rank);
-                    } else if (PAIR) {
-                        tc::tma_prefetch_3d(&mapV, 64 * (int)rank, u * kBN, z0);
-                    } else {
-                        for (int j = 0; j < C::kVHeads; ++j) tc::tma_prefetch_3d(&mapV, 0, u * kBN, z0 + j);
-                    }
-                }
-            };
-            constexpr int kPrefetch = 2;     // key tiles prefetched ahead
             // slot order = the issuer's: per item, Kf(t) then V(t-1) for each
             // tile, and the item's last V right after its last Kf
             WorkItem it, nx;
@@ -684,15 +799,13 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 for (int t = 0; t < it.ntiles && ok; ++t) {
                     for (int m = 0; m < kf_slots && ok; ++m) ok = load_kf(it, t, m);
                     if (ok && t == 0) ok = load_q(it);
-                    // prefetch: the item's tiles kPrefetch ahead, then the next
-                    // item's Q block and first tiles
-                    for (int u = (t == 0 ? 1 : t + kPrefetch); u <= t + kPrefetch; ++u) prefetch(it, u);
-                    if (have_next && t == it.ntiles - 1) {
+                    // the next item's Q block into L2 while this item's last
+                    // tile runs.  (Prefetching key tiles ahead as well was
+                    // measured slower: the prefetches compete with the ring's
+                    // own loads.)
+                    if (have_next && t == it.ntiles - 1)
                         for (int c = 0; c < C::kChunks; ++c)
                             tc::tma_prefetch_3d(&mapQ, 64 * c, nx.qb * NA * 8, nx.bh);
-                        prefetch(nx, 0);
-                        prefetch(nx, 1);
-                    }
                     for (int vs = 0; vs < C::kVSlots && ok && t > 0; ++vs) ok = load_v(it, t - 1, vs);
                 }
                 for (int vs = 0; vs < C::kVSlots && ok; ++vs) ok = load_v(it, it.ntiles - 1, vs);
@@ -889,8 +1002,13 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
             }
             const bool have_next = item(k + 1, nx);
             float m_run = -INFINITY, l = 0.f;
+            // range exponents of this CTA's query block and of each key tile
+            // (zero unless the prologue scaled a block's fp16 operands down)
+            const int eq = sexp[(size_t)it.bh * nqb + qb];
+            const int *ekp = sexp + (size_t)BH * nqb + (size_t)it.bh * nqb;
             for (int t = 0; t < it.ntiles; ++t, ++gt) {
                 const int sb = gt & 1;
+                const int escale = eq + ekp[t];
                 ok = __all_sync(0xffffffffu, wait_role<PAIR>(&s_full[sb], (gt >> 1) & 1, abort_flag));
                 if (!ok) break;
                 tc::tc_fence_after();
@@ -908,6 +1026,11 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
 #pragma unroll
                 for (int j = 0; j < kBN / 32; ++j) tc::tmem_ld32f(lane_base + sb * kBN + 32 * j, s + 32 * j);
                 tc::tmem_ld_wait();
+                if (escale != 0) {      // undo the blocks' operand scaling (exact)
+                    const float f = ldexpf(1.f, escale);
+#pragma unroll
+                    for (int c = 0; c < kBN; ++c) s[c] *= f;
+                }
                 // Band tiles (this block's diagonal tile and the one before it):
                 // for key j0 + c the diagonal offset is e = i_row - j0 - c; keys
                 // with e < 0 are in the future (-inf), and the Mask_0 correction
@@ -1060,6 +1183,8 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
     }
     tc::tc_fence_before();
     __syncthreads();
+    // this CTA's work is done: the GroupNorm kernel may be scheduled
+    launch_dependents();
     // in a pair, the leader's MMAs touch both CTAs' TMEM and shared memory
     if constexpr (PAIR) tc::cluster_sync();
     if (warp == 1) {
@@ -1083,69 +1208,82 @@ __global__ void k_selftest_wait_timeout(long long budget)
 
 // ------------------------------------------------------------ mix + GroupNorm
 
-__device__ __forceinline__ float warp_sum(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
+// Thread = 8 consecutive channels e0..e0+7 of one (b, t, h); the d/8 threads
+// of a head are consecutive lanes of one warp (16 at d = 128, 8 at d = 64).
+// O^h = sum_{h'} part[b][t][h][h'] (fp16 partials, one 16-byte load per
+// source head, summed in fp32), then GroupNorm over the head's d values
+// (mean and biased variance by shuffles within the lane group), affine, and
+// the head's scale: the depth scale, or sigmoid(g_h) ("Group Normalization
+// with Sigmoid Gating").  One 16-byte bf16 store per thread.
+constexpr int kMixThreads = 256;
 
-// One CTA per (query row i, batch b); warp w handles heads w, w+4, ...:
-// O^h = sum_{h'} part[b][i][h][h'] (fp16 partials, summed in fp32), then
-// GroupNorm over the head's d values (mean and biased variance by warp
-// shuffles), affine, and the head's scale: the depth scale, or sigmoid(g_h)
-// ("Group Normalization with Sigmoid Gating").
 template <int D, int CH>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kMixThreads)
 k_mix_groupnorm(const __half *__restrict__ part, const float *__restrict__ gn_weight,
                 const float *__restrict__ gn_bias, float depth_scale,
                 const float *__restrict__ gate, float eps, __nv_bfloat16 *__restrict__ out,
-                int T, int H)
+                int T, int H, long long units)
 {
-    const int i = blockIdx.x, b = blockIdx.y;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    constexpr int PER = D / 64;                // column pairs per lane
-    for (int h = warp; h < H; h += 4) {
-        const __half2 *src = (const __half2 *)(part + (((size_t)b * T + i) * H + h) * (size_t)(CH * D));
-        float2 o[PER];
+    constexpr int G = D / 8;                   // threads per (b, t, h)
+    const long long u0 = (long long)blockIdx.x * (kMixThreads / G) + threadIdx.x / G;
+    const bool live = u0 < units;              // the grid's last warp may be partly past the end:
+    const long long u = live ? u0 : units - 1; // its lanes recompute a valid unit, store nothing
+    const int e0 = 8 * (threadIdx.x % G);
+    wait_prerequisites();                      // the partial outputs are complete
+    const int h = (int)(u % H);
+    const long long bt = u / H;                // b * T + t
+    const uint4 *src = (const uint4 *)(part + (bt * H + h) * (long long)(CH * D) + e0);
+    uint4 raw[CH];
 #pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            float2 acc = make_float2(0.f, 0.f);
+    for (int hs = 0; hs < CH; ++hs) raw[hs] = src[hs * (D / 8)];
+    float o[8];
 #pragma unroll
-            for (int hs = 0; hs < CH; ++hs) {
-                const float2 f = __half22float2(src[hs * (D / 2) + lane + 32 * u]);
-                acc.x += f.x;
-                acc.y += f.y;
-            }
-            o[u] = acc;
-        }
-        float sum = 0.f;
+    for (int x = 0; x < 8; ++x) o[x] = 0.f;
 #pragma unroll
-        for (int u = 0; u < PER; ++u) sum += o[u].x + o[u].y;
-        const float mean = warp_sum(sum) / D;
-        float sq = 0.f;
+    for (int hs = 0; hs < CH; ++hs) {
+        const __half2 *hp = (const __half2 *)&raw[hs];
 #pragma unroll
-        for (int u = 0; u < PER; ++u)
-            sq += (o[u].x - mean) * (o[u].x - mean) + (o[u].y - mean) * (o[u].y - mean);
-        const float inv = 1.f / sqrtf(warp_sum(sq) / D + eps);
-        // the head's output scale: sigmoid(g_h), or the depth scale
-        const float scale = gate ? 1.f / (1.f + expf(-gate[h])) : depth_scale;
-        __nv_bfloat162 *dst = (__nv_bfloat162 *)(out + ((size_t)b * T + i) * ((size_t)H * D) + (size_t)h * D);
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int e = 2 * (lane + 32 * u), ch = h * D + e;
-            dst[lane + 32 * u] = __floats2bfloat162_rn(
-                scale * ((o[u].x - mean) * inv * gn_weight[ch] + gn_bias[ch]),
-                scale * ((o[u].y - mean) * inv * gn_weight[ch + 1] + gn_bias[ch + 1]));
+        for (int x = 0; x < 4; ++x) {
+            const float2 f = __half22float2(hp[x]);
+            o[2 * x] += f.x;
+            o[2 * x + 1] += f.y;
         }
     }
+    float sum = 0.f;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) sum += o[x];
+#pragma unroll
+    for (int m = G / 2; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+    const float mean = sum / D;
+    float sq = 0.f;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) sq += (o[x] - mean) * (o[x] - mean);
+#pragma unroll
+    for (int m = G / 2; m > 0; m >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, m);
+    const float inv = 1.f / sqrtf(sq / D + eps);
+    // the head's output scale: sigmoid(g_h), or the depth scale
+    const float scale = gate ? 1.f / (1.f + expf(-gate[h])) : depth_scale;
+    const float4 *gw = (const float4 *)(gn_weight + h * D + e0);
+    const float4 *gb = (const float4 *)(gn_bias + h * D + e0);
+    const float4 w0 = gw[0], w1 = gw[1], b0 = gb[0], b1 = gb[1];
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    uint4 res;
+    uint32_t *rp = (uint32_t *)&res;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        const float y0 = scale * ((o[2 * x] - mean) * inv * wv[2 * x] + bv[2 * x]);
+        const float y1 = scale * ((o[2 * x + 1] - mean) * inv * wv[2 * x + 1] + bv[2 * x + 1]);
+        rp[x] = pack_bf16(y0, y1);
+    }
+    if (live) *(uint4 *)(out + bt * ((long long)H * D) + (long long)h * D + e0) = res;
 }
 
 // ------------------------------------------------------------ host side
 
 struct FusedLayout {
     int Tp, nqb, NA;
-    size_t off_kf, off_qp, off_corr, off_part, total;
+    size_t off_kf, off_qp, off_corr, off_part, off_exp, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1162,49 +1300,13 @@ FusedLayout fused_layout(const mta_shape &s)
     L.off_qp = off;   off += align256(BH * L.nqb * L.NA * 8 * s.d * 2);
     L.off_corr = off; off += align256(BH * L.Tp * kCorrW * 4);
     L.off_part = off; off += align256((size_t)s.B * s.T * s.H * s.c_h * s.d * 2);
+    L.off_exp = off;  off += align256(2 * BH * L.nqb * sizeof(int));   // query, then key blocks
     L.total = off;
     return L;
 }
 
-const char *const kFusedNames[4] = {"k_fold_keys", "k_fold_aux", "k_mta_fused", "k_mix_groupnorm"};
-
-// The two prologue kernels are independent and bound by different units
-// (FMA issue vs load latency), so k_fold_aux runs on a side stream of the
-// library while k_fold_keys runs on the caller's stream; the caller's stream
-// forks to the side stream and joins back before the main kernel.  One side
-// stream and event pair per device; the fork/join sequence is enqueued under
-// a lock so that concurrent callers cannot interleave their event records.
-// The pattern is also legal under stream capture.
-struct SideStream {
-    cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-    unsigned long long ctx = 0;    // context the handles belong to
-};
-std::mutex g_side_lock;
-
-mta_status side_stream(SideStream *out)
-{
-    constexpr int kMaxDevices = 64;
-    static SideStream tab[kMaxDevices];
-    int dev = 0;
-    unsigned long long ctx = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MTA_ERR_CUDA;
-    if (!current_context_id(&ctx)) return MTA_ERR_CUDA;
-    SideStream &ss = tab[dev];
-    // handles made in a context that has since been destroyed (a device
-    // reset) are dead: make new ones in the current context
-    if (!ss.s || ss.ctx != ctx) {
-        SideStream fresh;
-        if (cudaEventCreateWithFlags(&fresh.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming) != cudaSuccess ||
-            cudaStreamCreateWithFlags(&fresh.s, cudaStreamNonBlocking) != cudaSuccess)
-            return MTA_ERR_CUDA;
-        fresh.ctx = ctx;
-        ss = fresh;
-    }
-    *out = ss;
-    return MTA_OK;
-}
+constexpr int kFusedKernels = 3;
+const char *const kFusedNames[kFusedKernels] = {"k_fold", "k_mta_fused", "k_mix_groupnorm"};
 
 // Clusters of the main kernel that fit on the device at once (one CTA per SM
 // at this shared-memory size), cached per kernel instantiation and device.
@@ -1253,6 +1355,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     __half *qp = (__half *)(w + L.off_qp);
     float *corr = (float *)(w + L.off_corr);
     __half *part = (__half *)(w + L.off_part);
+    int *sexp = (int *)(w + L.off_exp);
     const uint64_t BH = (uint64_t)s.B * s.H;
     CUtensorMap mQ, mK, mV;
     {
@@ -1274,37 +1377,28 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         if (!make_tmap_bf16(&mV, a.v, 3, dims, strides, box)) return MTA_ERR_CUDA;
     }
     auto main_kernel = k_mta_fused<D, CH, PAIR>;
-    auto fold_keys = s.c_k == 11 ? k_fold_keys<D, 11>
-                   : s.c_k == 3  ? k_fold_keys<D, 3>
-                                 : k_fold_keys<D, 15>;
-    const int aux_smem = (int)prologue_smem_bytes(D);
+    auto fold = s.c_k == 11 ? k_fold<D, 11> : s.c_k == 3 ? k_fold<D, 3> : k_fold<D, 15>;
+    const int pro_smem = (int)prologue_smem_bytes(D);
     if (cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(k_fold_aux<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, aux_smem) !=
+        cudaFuncSetAttribute(fold, cudaFuncAttributeMaxDynamicSharedMemorySize, pro_smem) !=
             cudaSuccess)
         return MTA_ERR_CUDA;
     const float scale = kLog2e / sqrtf((float)D);
-    {
-        std::lock_guard<std::mutex> guard(g_side_lock);
-        SideStream side;
-        if (side_stream(&side) != MTA_OK) return MTA_ERR_CUDA;
-        if (cudaEventRecord(side.fork, st) != cudaSuccess ||
-            cudaStreamWaitEvent(side.s, side.fork, 0) != cudaSuccess)
-            return MTA_ERR_CUDA;
-        tr.before(1, side.s);
-        k_fold_aux<D><<<dim3(L.Tp / kAuxRows, (unsigned)BH), kAuxThreads, aux_smem, side.s>>>(
-            (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, qp, corr, s.T, L.Tp, s.H,
-            s.c_q, s.c_k, scale);
-        tr.after(1, side.s);
-        tr.before(0, st);
-        fold_keys<<<dim3(L.nqb, (unsigned)BH), 256, 0, st>>>((const __nv_bfloat16 *)a.k, a.w_kq, kf,
-                                                             s.T, L.Tp, s.H, s.c_q, s.c_k, scale);
-        tr.after(0, st);
-        if (cudaEventRecord(side.join, side.s) != cudaSuccess ||
-            cudaStreamWaitEvent(st, side.join, 0) != cudaSuccess)
-            return MTA_ERR_CUDA;
-    }
-    tr.before(2, st);
+    tr.before(0, st);
+    fold<<<dim3((unsigned)(3 * L.nqb * BH)), kProThreads, pro_smem, st>>>(
+        (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, kf, qp, corr, sexp, s.T, L.Tp,
+        s.H, L.nqb, s.c_q, s.c_k, scale, a.exact_mask ? 1 : 0);
+    tr.after(0, st);
+    // The main kernel and the GroupNorm kernel are launched with programmatic
+    // stream serialisation: each may be scheduled while its predecessor still
+    // runs (the predecessor's CTAs signal it), does its set-up, and waits in
+    // griddepcontrol.wait until the predecessor has completed and its writes
+    // are visible.
+    cudaLaunchAttribute pdl;
+    pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl.val.programmaticStreamSerializationAllowed = 1;
+    tr.before(1, st);
     {
         // persistent: as many clusters as can be resident at once, each
         // walking its share of the work items
@@ -1312,29 +1406,42 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         cfg.blockDim = dim3(224, 1, 1);
         cfg.dynamicSmemBytes = C::kSmemBytes;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = PAIR ? 2 : 1;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1] = pdl;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         const int n_items = (int)BH * (PAIR ? L.nqb / 2 : L.nqb) * C::kSplits;
         int resident = 0;
         if (max_resident_clusters<D, CH>(cfg, &resident) != MTA_OK)
             return MTA_ERR_CUDA;
         const int ncl = resident < n_items ? resident : n_items;
         cfg.gridDim = dim3((unsigned)(ncl * (PAIR ? 2 : 1)), 1, 1);
-        if (cudaLaunchKernelEx(&cfg, main_kernel, mQ, mK, mV, (const float *)corr, a.w_head, part,
+        if (cudaLaunchKernelEx(&cfg, main_kernel, mQ, mK, mV, (const float *)corr,
+                               (const int *)sexp, a.w_head, part,
                                s.T, L.Tp, s.H, s.c_q, L.nqb, (int)BH) != cudaSuccess)
             return MTA_ERR_CUDA;
     }
+    tr.after(1, st);
+    tr.before(2, st);
+    {
+        const long long units = (long long)s.B * s.T * s.H;     // (b, t, h)
+        const int per_cta = kMixThreads / (D / 8);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((units + per_cta - 1) / per_cta), 1, 1);
+        cfg.blockDim = dim3(kMixThreads, 1, 1);
+        cfg.stream = st;
+        cfg.attrs = &pdl;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, k_mix_groupnorm<D, CH>, (const __half *)part, a.gn_weight,
+                               a.gn_bias, a.depth_scale, a.gate, s.gn_eps,
+                               (__nv_bfloat16 *)a.out, s.T, s.H, units) != cudaSuccess)
+            return MTA_ERR_CUDA;
+    }
     tr.after(2, st);
-    tr.before(3, st);
-    k_mix_groupnorm<D, CH><<<dim3(s.T, s.B), 128, 0, st>>>(part, a.gn_weight, a.gn_bias,
-                                                         a.depth_scale, a.gate, s.gn_eps,
-                                                         (__nv_bfloat16 *)a.out, s.T, s.H);
-    tr.after(3, st);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
@@ -1352,11 +1459,11 @@ bool fused_supported(const mta_shape &s)
 
 size_t fused_workspace_bytes(const mta_shape &s) { return fused_layout(s).total; }
 
-int fused_kernel_count(const mta_shape &) { return 4; }
+int fused_kernel_count(const mta_shape &) { return kFusedKernels; }
 
 const char *fused_kernel_name(const mta_shape &, int index)
 {
-    return (index >= 0 && index < 4) ? kFusedNames[index] : nullptr;
+    return (index >= 0 && index < kFusedKernels) ? kFusedNames[index] : nullptr;
 }
 
 mta_status launch_fused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,

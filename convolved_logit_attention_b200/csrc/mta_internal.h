@@ -45,6 +45,24 @@ inline size_t bh_tt(const mta_shape &s) {
 }
 
 // Materialised chain (unfused.cu).
+// Launchers of its kernels, also used by the backward pass (backward.cu):
+//  logits        map[bh][i][j] = q_i . k_j / sqrt(d) for j <= i + band, 0 above
+//  logits_f32_io map[bh][i][j] = scale * a_i . b_j for j <= i (a fp32 [B*H][T][d],
+//                b of the I/O type)
+//  launch_conv   the Eq. (4) key-query convolution of src into dst (j <= i)
+//  softmax_mix   softmax rows of map1 and the Eq. (7) head mix (w_head null:
+//                the identity) into dst
+//  head_mix      Eq. (7) without a softmax
+void logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
+            cudaStream_t st);
+void logits_f32_io(const mta_shape &s, const float *a, const void *b, float scale, float *map,
+                   cudaStream_t st);
+void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq, int band,
+                 int nin, cudaStream_t st);
+mta_status softmax_mix(const mta_shape &s, const float *map1, float *dst, const float *w_head,
+                       int mode, cudaStream_t st);
+mta_status head_mix(const mta_shape &s, const float *src, float *dst, const float *w_head,
+                    cudaStream_t st);
 size_t unfused_workspace_bytes(const mta_shape &s);
 constexpr int kUnfusedKernels = 4;
 extern const char *const kUnfusedKernelNames[kUnfusedKernels];
@@ -57,6 +75,22 @@ mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cu
 mta_status launch_debug_attention(const mta_shape &s, const void *q, const void *k,
                                   const float *w_kq, const float *w_head, float *attn, int stage,
                                   void *ws, cudaStream_t st);
+
+// Backward pass (backward.cu): gradients of the default composition, on
+// materialised maps in fp32.  Output pointers are device memory, fp32.
+struct BackwardArgs {
+    const void *dout;          // [B][T][H*d], I/O type
+    float *dq, *dk, *dv;       // [B][H][T][d]
+    float *dw_kq;              // [H][c_q][c_k]
+    float *dw_head;            // [H/c_h][c_h][c_h]
+    float *dgn_weight, *dgn_bias;   // [H*d]
+    float *dgate;              // [H], with a gate only
+};
+constexpr int kBackwardKernels = 14;
+extern const char *const kBackwardKernelNames[kBackwardKernels];
+size_t backward_workspace_bytes(const mta_shape &s);
+mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const BackwardArgs &g,
+                           void *ws, cudaStream_t st, const Trace &tr);
 
 // Fused tcgen05 path (fused_tc.cu).
 bool fused_supported(const mta_shape &s);

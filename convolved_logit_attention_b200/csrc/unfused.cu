@@ -48,9 +48,9 @@ constexpr int kMaxD = 128;
 // columns with tx, so that its operands for one contraction index are four
 // 16-byte shared loads (eight lanes of a warp read 128 contiguous bytes) for
 // 64 FMAs.  Chunks of 16 contraction indices are staged transposed.
-template <typename TIO>
+template <typename TQ, typename TK>
 __global__ void __launch_bounds__(256)
-k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict__ map0,
+k_logits(const TQ *__restrict__ q, const TK *__restrict__ k, float *__restrict__ map0,
          int T, int d, float scale, int band)
 {
     const int ct = blockIdx.x, rt = blockIdx.y;
@@ -66,8 +66,8 @@ k_logits(const TIO *__restrict__ q, const TIO *__restrict__ k, float *__restrict
     for (int u = 0; u < 8; ++u)
 #pragma unroll
         for (int w = 0; w < 8; ++w) acc[u][w] = 0.f;
-    const TIO *qb = q + bh * (size_t)T * d;
-    const TIO *kb = k + bh * (size_t)T * d;
+    const TQ *qb = q + bh * (size_t)T * d;
+    const TK *kb = k + bh * (size_t)T * d;
     for (int e0 = 0; e0 < d; e0 += kLogitDk) {
         for (int idx = tid; idx < kLogitTile * kLogitDk; idx += 256) {
             const int r = idx / kLogitDk, e = idx % kLogitDk;
@@ -455,6 +455,10 @@ k_pv_groupnorm(const float *__restrict__ amap, const TIO *__restrict__ v,
     }
 }
 
+}  // namespace
+
+// Launchers of the chain's kernels, shared with the backward pass
+// (backward.cu) through mta_internal.h.
 template <int CH>
 void launch_softmax_mix(const mta_shape &s, const float *map1, float *dst, const float *w_head,
                         int mode, cudaStream_t st)
@@ -499,14 +503,14 @@ mta_status head_mix(const mta_shape &s, const float *src, float *dst, const floa
     return MTA_OK;
 }
 
-template <typename TIO>
-void launch_logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
-                   cudaStream_t st)
+template <typename TQ, typename TK>
+void launch_logits(const mta_shape &s, const void *q, const void *k, float *map0, float scale,
+                   int band, cudaStream_t st)
 {
     const int nt = (s.T + kLogitTile - 1) / kLogitTile;
     dim3 g1(nt, nt, s.B * s.H);
-    k_logits<TIO><<<g1, 256, 0, st>>>((const TIO *)q, (const TIO *)k, map0, s.T, s.d,
-                                      1.0f / sqrtf((float)s.d), band);
+    k_logits<TQ, TK><<<g1, 256, 0, st>>>((const TQ *)q, (const TK *)k, map0, s.T, s.d, scale,
+                                         band);
 }
 
 void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq, int band,
@@ -540,11 +544,23 @@ void launch_conv(const mta_shape &s, const float *src, float *dst, const float *
 void logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
             cudaStream_t st)
 {
+    const float scale = 1.0f / sqrtf((float)s.d);
     if (s.io == MTA_BF16)
-        launch_logits<__nv_bfloat16>(s, q, k, map0, band, st);
+        launch_logits<__nv_bfloat16, __nv_bfloat16>(s, q, k, map0, scale, band, st);
     else
-        launch_logits<float>(s, q, k, map0, band, st);
+        launch_logits<float, float>(s, q, k, map0, scale, band, st);
 }
+
+void logits_f32_io(const mta_shape &s, const float *a, const void *b, float scale, float *map,
+                   cudaStream_t st)
+{
+    if (s.io == MTA_BF16)
+        launch_logits<float, __nv_bfloat16>(s, a, b, map, scale, 0, st);
+    else
+        launch_logits<float, float>(s, a, b, map, scale, 0, st);
+}
+
+namespace {
 
 void pv_groupnorm(const mta_shape &s, const float *amap, const ForwardArgs &a, cudaStream_t st)
 {

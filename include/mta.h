@@ -68,7 +68,7 @@ typedef enum {
     MTA_ERR_WORKSPACE = -4,      /* workspace smaller than the *_workspace_size query */
     MTA_ERR_CUDA = -5,           /* a CUDA runtime call failed */
     MTA_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
-    MTA_ERR_RANGE = -7           /* the fused path met q or folded-key values beyond fp16 range */
+    MTA_ERR_RANGE = -7           /* the fused path met a non-finite q, k or folded key */
 } mta_status;
 
 typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
@@ -112,9 +112,16 @@ MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
 
 /* The MTA forward S1..S9 above, out = depth_scale * GN(...), written to out.
  * The fused path computes the folded logits on tensor cores with fp16
- * operands (q and the folded keys, |x| <= 65504, else the call's next
- * mta_sync_status() reports MTA_ERR_RANGE) and P V with bf16 operands, both
- * with fp32 accumulation; the materialised path computes in fp32.
+ * operands (q and the folded keys) and P V with bf16 operands, both with fp32
+ * accumulation; the materialised path computes in fp32.  Any finite bf16
+ * input is in the fused path's domain: a 128-row block of queries or of
+ * folded keys whose magnitude bound exceeds 2^14 is scaled by a power of two
+ * before the fp16 rounding and its logits scaled back exactly.  Values more
+ * than 2^28 times smaller than their block's largest then fall into fp16's
+ * subnormal range, with an absolute error up to 2^(e-25) for the block's
+ * scale 2^e (for one query of 2e6 among N(0,1) values, e = 7: 4e-6).  A
+ * non-finite q or k makes the call's next mta_sync_status() report
+ * MTA_ERR_RANGE.
  * The workspace is scratch owned by the caller for the duration of the
  * enqueued work; its contents on entry are ignored. */
 MTA_API mta_status mta_forward(const mta_shape *shape, const void *q, const void *k, const void *v,
@@ -250,13 +257,17 @@ typedef struct {
 
 /* Bytes of device workspace mta_forward_composed needs (0 on an invalid
  * shape or a NULL composition): mta_workspace_size() for the default
- * composition, two fp32 [B][H][T][T] maps for every other one. */
+ * composition (either masking), two fp32 [B][H][T][T] maps for every other
+ * one. */
 MTA_API size_t mta_composed_workspace_size(const mta_shape *shape, const mta_composition *comp);
 
 /* The forward of the composition *comp, written to out.  The default
- * composition takes mta_forward's path (fused where mta_forward_path says
- * so); every other composition runs on the materialised chain, in fp32, with
- * P1 as a second conv launch and P2 as a mix-only launch.  gate is NULL for
+ * composition {w_kq, w_head} takes mta_forward's path (fused where
+ * mta_forward_path says so), under either masking: with exact_mask the fused
+ * kernels change only which taps the Mask_0 correction table subtracts
+ * (those whose key lies past the output's query instead of past the tap's
+ * own query).  Every other composition runs on the materialised chain, in
+ * fp32, with P1 as a second conv launch and P2 as a mix-only launch.  gate is NULL for
  * out = depth_scale * GN(...), or a device array of H floats (4-byte
  * aligned) for the sigmoid gate of mta_forward_gated, depth_scale then
  * ignored.  A NULL comp is MTA_ERR_INVALID_ARG; every other argument and the
@@ -285,9 +296,51 @@ MTA_API int mta_composed_kernel_count(const mta_shape *shape, const mta_composit
 MTA_API const char *mta_composed_kernel_name(const mta_shape *shape, const mta_composition *comp,
                                              int index);
 
+/* Backward pass ("Multi-Token Attention -- Paper Graph", section 3.4, the
+ * forward S1..S9 above; the pages report training cost, Table 9, but give no
+ * gradients, so these are the forward's own by the chain rule).  Given
+ * dout = dL/d(out) [B][T][H*d] (dtype shape->io), writes the gradient of L
+ * with respect to every input, all fp32, caller-owned device memory:
+ *   dq, dk, dv           [B][H][T][d]
+ *   dw_kq                [H][c_q][c_k]       (layout of w_kq)
+ *   dw_head              [H/c_h][c_h][c_h]   (layout of w_head)
+ *   dgn_weight, dgn_bias [H*d]
+ *   dgate                [H], only with gate != NULL (out = GN(...) * sigmoid(g),
+ *                        as mta_forward_gated; depth_scale is then ignored);
+ *                        NULL exactly when gate is NULL, else MTA_ERR_INVALID_ARG.
+ * Every output is overwritten (not accumulated into).  The forward maps are
+ * recomputed in the workspace (mta_backward_workspace_size: three fp32
+ * [B][H][T][T] maps plus O and partial sums), and every step runs in fp32 on
+ * the materialised chain; the parameter gradients are sums of per-block
+ * partials in a fixed order, so repeated calls give identical bits.  Pointers
+ * 16-byte aligned (gate and dgate 4-byte), the workspace 256-byte aligned;
+ * argument errors as for mta_forward, nothing enqueued on an error. */
+MTA_API size_t mta_backward_workspace_size(const mta_shape *shape);
+MTA_API mta_status mta_backward(const mta_shape *shape, const void *q, const void *k,
+                                const void *v, const float *w_kq, const float *w_head,
+                                const float *gn_weight, const float *gn_bias, float depth_scale,
+                                const float *gate, const void *dout, float *dq, float *dk,
+                                float *dv, float *dw_kq, float *dw_head, float *dgn_weight,
+                                float *dgn_bias, float *dgate, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/* mta_backward that records caller-created events around its launches, as
+ * mta_forward_traced does; the launches are those mta_backward_kernel_name
+ * lists (the last entry covers the final reductions). */
+MTA_API mta_status mta_backward_traced(const mta_shape *shape, const void *q, const void *k,
+                                       const void *v, const float *w_kq, const float *w_head,
+                                       const float *gn_weight, const float *gn_bias,
+                                       float depth_scale, const float *gate, const void *dout,
+                                       float *dq, float *dk, float *dv, float *dw_kq,
+                                       float *dw_head, float *dgn_weight, float *dgn_bias,
+                                       float *dgate, void *workspace, size_t workspace_bytes,
+                                       void *stream, void *const *events, int n_events);
+MTA_API int mta_backward_kernel_count(const mta_shape *shape);
+MTA_API const char *mta_backward_kernel_name(const mta_shape *shape, int index);
+
 /* Synchronises `stream`, then reports (and clears) the device error flags:
  * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
- * the fused path met a value outside fp16 range, MTA_ERR_CUDA if the
+ * the fused path met a non-finite input, MTA_ERR_CUDA if the
  * synchronisation itself failed, MTA_OK otherwise.  The flags are one word per
  * device, shared by every stream and caller of the library on that device:
  * the word is read and cleared in one atomic step (a small kernel on

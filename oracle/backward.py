@@ -1,5 +1,6 @@
 """fp64 gradients of the Multi-Token Attention forward (the pages' default
-composition), for a future backward pass.
+composition, with the depth scale or the sigmoid gate), the reference of the
+CUDA backward pass.
 
 TEST INFRASTRUCTURE ONLY: like the rest of this package, only the test suite
 may call it; the CUDA library never imports it.
@@ -39,10 +40,19 @@ def _shift(X, a, b):
     return torch.nn.functional.pad(X, (b, -b, a, -a))
 
 
-def forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gn_eps=1e-5):
+def _out_scale(depth_scale, gate, H):
+    """The per-head output scale: the depth scale ("Article Overview",
+    section 2), or sigmoid(g_h) with a gate ("Group Normalization with
+    Sigmoid Gating"); shaped to broadcast over [B, H, T, d]."""
+    if gate is None:
+        return depth_scale
+    return torch.sigmoid(gate).view(1, H, 1, 1)
+
+
+def forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gn_eps=1e-5, gate=None):
     """out [B, T, H*d] from float64 torch tensors (the layouts of the C
     oracle: q, k, v [B,H,T,d]; w_kq [H,c_q,c_k]; w_head [H/c_h,c_h,c_h];
-    gn_weight, gn_bias [H*d])."""
+    gn_weight, gn_bias [H*d]; gate [H] or None)."""
     B, H, T, d = q.shape
     _, c_q, c_k = w_kq.shape
     c_h = w_head.shape[-1]
@@ -63,19 +73,90 @@ def forward(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, gn_eps=1e-5)
     var = ((O - mean) ** 2).mean(dim=-1, keepdim=True)
     xhat = (O - mean) / torch.sqrt(var + gn_eps)
     y = xhat * gn_weight.view(H, 1, d) + gn_bias.view(H, 1, d)
-    return depth_scale * y.permute(0, 2, 1, 3).reshape(B, T, H * d)
+    y = _out_scale(depth_scale, gate, H) * y
+    return y.permute(0, 2, 1, 3).reshape(B, T, H * d)
 
 
-def gradients(inputs, dout, depth_scale, gn_eps=1e-5):
-    """The gradient of sum(out * dout) with respect to every input: a dict
-    name -> float64 array of the input's shape, for inputs a dict of arrays
-    keyed by NAMES and dout [B, T, H*d]."""
+def _leaves(inputs, gate):
     ts = {n: torch.tensor(np.asarray(inputs[n], dtype=np.float64), requires_grad=True)
           for n in NAMES}
-    out = forward(*(ts[n] for n in NAMES), depth_scale, gn_eps)
-    grads = torch.autograd.grad(out, [ts[n] for n in NAMES],
+    if gate is not None:
+        ts["gate"] = torch.tensor(np.asarray(gate, dtype=np.float64), requires_grad=True)
+    return ts
+
+
+def gradients(inputs, dout, depth_scale, gn_eps=1e-5, gate=None):
+    """The gradient of sum(out * dout) with respect to every input: a dict
+    name -> float64 array of the input's shape, for inputs a dict of arrays
+    keyed by NAMES and dout [B, T, H*d].  With gate [H] (the sigmoid gate in
+    place of the depth scale) the dict also holds "gate"."""
+    ts = _leaves(inputs, gate)
+    out = forward(*(ts[n] for n in NAMES), depth_scale, gn_eps, gate=ts.get("gate"))
+    names = list(ts)
+    grads = torch.autograd.grad(out, [ts[n] for n in names],
                                 grad_outputs=torch.as_tensor(np.asarray(dout, np.float64)))
-    return {n: g.numpy() for n, g in zip(NAMES, grads)}
+    return {n: g.numpy() for n, g in zip(names, grads)}
+
+
+def forward_rows(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, rows, gn_eps=1e-5,
+                 gate=None):
+    """out[:, rows, :] ([B, len(rows), H*d]) of the same forward, computed
+    from only what those rows depend on: for query row i, the masked logit
+    rows i - c_q + 1 .. i over the keys 0 .. i (Mask_0 zeroes every key past
+    its own row, and Eq. (4)'s taps reach keys j - j' <= i + floor(c_k/2)
+    only through such zeros), the Eq. (4) convolution at the keys j <= i,
+    softmax, Eq. (7) mix, A V over the keys j <= i and the GroupNorm.  The
+    gradient of sum(out[:, rows] * dout_rows) through it is the full
+    forward's gradient for an upstream gradient that is zero off `rows`."""
+    B, H, T, d = q.shape
+    _, c_q, c_k = w_kq.shape
+    c_h = w_head.shape[-1]
+    G = H // c_h
+    R = c_k // 2
+    outs = []
+    for i in rows:
+        n = i + 1                                          # keys 0 .. i
+        r_idx = [i - ip for ip in range(c_q)]              # logit rows i - i'
+        A0 = []
+        for r in r_idx:
+            if r < 0:
+                A0.append(torch.zeros(B, H, n, dtype=q.dtype))
+                continue
+            row = (q[:, :, r, :].unsqueeze(-2) @ k[:, :, :n, :].transpose(-1, -2)).squeeze(-2)
+            row = row / math.sqrt(d)
+            keep = torch.arange(n) <= r                    # Mask_0
+            A0.append(torch.where(keep, row, torch.zeros((), dtype=q.dtype)))
+        C = torch.zeros(B, H, n, dtype=q.dtype)
+        for ip in range(c_q):
+            for jj in range(c_k):
+                jp = jj - R                                # C[j] += theta A0[i-ip][j-jp]
+                src = A0[ip]
+                if jp >= 0:
+                    shifted = torch.nn.functional.pad(src, (jp, 0))[..., :n]
+                else:
+                    shifted = torch.nn.functional.pad(src, (0, -jp))[..., -jp:]
+                C = C + w_kq[:, ip, jj].view(1, H, 1) * shifted
+        P = torch.softmax(C, dim=-1)                       # keys j <= i only
+        A = torch.einsum("goi,bgij->bgoj", w_head, P.reshape(B, G, c_h, n)).reshape(B, H, n)
+        O = (A.unsqueeze(-2) @ v[:, :, :n, :]).squeeze(-2)  # [B, H, d]
+        mean = O.mean(dim=-1, keepdim=True)
+        var = ((O - mean) ** 2).mean(dim=-1, keepdim=True)
+        y = (O - mean) / torch.sqrt(var + gn_eps) * gn_weight.view(H, d) + gn_bias.view(H, d)
+        scale = depth_scale if gate is None else torch.sigmoid(gate).view(1, H, 1)
+        outs.append((scale * y).reshape(B, H * d))
+    return torch.stack(outs, dim=1)
+
+
+def gradients_rows(inputs, rows, dout_rows, depth_scale, gn_eps=1e-5, gate=None):
+    """gradients() for an upstream gradient that is zero except at the query
+    rows `rows`, where it is dout_rows [B, len(rows), H*d]; computed through
+    forward_rows, so that large T stays cheap."""
+    ts = _leaves(inputs, gate)
+    out = forward_rows(*(ts[n] for n in NAMES), depth_scale, rows, gn_eps, gate=ts.get("gate"))
+    names = list(ts)
+    grads = torch.autograd.grad(out, [ts[n] for n in names],
+                                grad_outputs=torch.as_tensor(np.asarray(dout_rows, np.float64)))
+    return {n: g.numpy() for n, g in zip(names, grads)}
 
 
 # Every composition of "Putting Everything Together: The Full MTA Module":

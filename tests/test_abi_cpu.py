@@ -126,9 +126,11 @@ def test_unfused_workspace_is_two_fp32_maps(L):
 def test_forward_path_selection(L, kw, path):
     s = shape(**kw)
     assert mta.mta_forward_path(s) == path
-    assert mta.mta_kernel_count(s) == 4      # fold keys, fold aux, main, mix+GN; or the 4 materialised kernels
     names = [mta.mta_kernel_name(s, i) for i in range(mta.mta_kernel_count(s))]
-    assert ("k_mta_fused" in names) == (path == 0)
+    if path == 0:   # prologue, main kernel, mix + GroupNorm
+        assert names == ["k_fold", "k_mta_fused", "k_mix_groupnorm"]
+    else:           # the four materialised kernels
+        assert names == ["k_logits", "k_conv", "k_softmax_mix", "k_pv_groupnorm"]
 
 
 def test_selftest_rejects_bad_budget(L):
@@ -169,8 +171,10 @@ def test_composed_launch_sequences_and_workspace(L):
     default = C(a, a, None, None)
     assert mta.mta_composed_kernel_names(fused, default) == \
         [mta.mta_kernel_name(fused, i) for i in range(mta.mta_kernel_count(fused))]
-    # the default weights with the exact indicator leave the fused path
-    assert "k_mta_fused" not in mta.mta_composed_kernel_names(fused, C(a, a, None, None, None, 1))
+    # the default weights under the exact indicator of Eq. (4) stay on the
+    # fused path (only the prologue's correction table changes)
+    assert mta.mta_composed_kernel_names(fused, C(a, a, None, None, None, 1)) == \
+        ["k_fold", "k_mta_fused", "k_mix_groupnorm"]
     assert L.mta_composed_workspace_size(ctypes.byref(fused), ctypes.byref(default)) == \
         mta.mta_workspace_size(fused)
     assert L.mta_composed_workspace_size(ctypes.byref(fused), None) == 0

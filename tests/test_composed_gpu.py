@@ -165,7 +165,7 @@ def test_traced_launches_follow_the_chain():
     assert_close(got, oracle_full(x), w.io, "traced")
 
 
-@pytest.mark.parametrize("comp", ["repeat", "both_post", "exact_both_pre", "conv3d"])
+@pytest.mark.parametrize("comp", ["exact", "repeat", "both_post", "exact_both_pre", "conv3d"])
 def test_full_size_every_element(comp):
     """The T = 4096 workload (two [B,H,T,T] fp32 maps, 4.3 GB), every element
     against the oracle's full forward of the same composition."""

@@ -32,10 +32,8 @@ def test_expired_wait_is_reported_and_context_survives():
     assert torch.isfinite(out.float()).all()
 
 
-def test_values_beyond_fp16_range_are_reported():
-    # bf16 holds 1e5, fp16 does not: the fused path's folded operands would
-    # overflow, which the prologue reports instead of producing infinities.
-    w = Workload("range", 1, 2, 130, 64, 6, 11, 2, "bf16", seed=2)
+def _range_case(seed):
+    w = Workload("range", 1, 2, 130, 64, 6, 11, 2, "bf16", seed=seed)
     x = make_inputs(w)
     dev = torch.device("cuda", 0)
     d = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v")}
@@ -43,7 +41,38 @@ def test_values_beyond_fp16_range_are_reported():
         d[n] = torch.from_numpy(x[n]).to(dev)
     shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"])
     assert mta.mta_forward_path(shape) == mta.MTA_PATH_FUSED_TC
-    d["q"][0, 1, 17, 3] = 1.0e5
+    return x, d
+
+
+@pytest.mark.parametrize("which,value", [("q", 1.0e5), ("k", 1.0e6), ("q", -2.0e6)])
+def test_values_beyond_fp16_range_match_the_oracle(which, value):
+    # bf16 holds these, fp16 does not: the prologue scales the query block (or
+    # the folded-key block) that holds them by a power of two, and the main
+    # kernel multiplies those tiles' logits back, so the fused path computes
+    # them instead of overflowing.
+    import oracle
+    x, d = _range_case(2)
+    x[which] = x[which].copy()
+    x[which][0, 1, 17, 3] = value           # exactly representable in bf16
+    d[which][0, 1, 17, 3] = value
+    mta.mta_sync_status()
+    out = mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                          d["gn_bias"], x["depth_scale"], check=True)
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = oracle.forward(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                         x["gn_bias"], x["depth_scale"])
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref)
+    assert err.max() <= 2e-2 and np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 5e-3, \
+        (err.max(), np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+def test_non_finite_input_is_reported():
+    # an infinite query: the prologue cannot scale it into fp16 and raises the
+    # range flag, which mta_sync_status reports (and clears)
+    x, d = _range_case(3)
+    d["q"][0, 1, 17, 3] = float("inf")
+    mta.mta_sync_status()
     mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
                     d["gn_bias"], x["depth_scale"])
     with pytest.raises(mta.MtaError) as exc:
@@ -55,17 +84,12 @@ def test_values_beyond_fp16_range_are_reported():
 def test_check_flag_raises_at_the_call():
     # check=True synchronises the call's stream and raises what the device
     # flagged, so a torch caller does not get non-finite output silently
-    w = Workload("range_check", 1, 2, 130, 64, 6, 11, 2, "bf16", seed=3)
-    x = make_inputs(w)
-    dev = torch.device("cuda", 0)
-    d = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v")}
-    for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
-        d[n] = torch.from_numpy(x[n]).to(dev)
+    x, d = _range_case(4)
     mta.mta_sync_status()
     out = mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
                           d["gn_bias"], x["depth_scale"], check=True)
     assert torch.isfinite(out.float()).all()
-    d["k"][0, 0, 40, 5] = 2.0e5
+    d["k"][0, 0, 40, 5] = float("nan")
     with pytest.raises(mta.MtaError) as exc:
         mta.mta_forward(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
                         d["gn_bias"], x["depth_scale"], check=True)

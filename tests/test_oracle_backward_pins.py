@@ -91,6 +91,84 @@ def test_gradients_are_causal():
             assert np.abs(g[name][:, :, : t + 1]).max() > 0.0
 
 
+GATE = np.array([-1.5, 0.25, 2.0, -0.5])
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_gated_restatement_and_gate_gradient(shape):
+    # "Group Normalization with Sigmoid Gating": the torch restatement with a
+    # gate equals the C oracle's gated forward, and every gradient (the
+    # gate's included) equals central finite differences of that C forward.
+    x, rng = inputs_of(shape, 65)
+    H = shape[1]
+    gate = GATE[:H].copy()
+    c_fwd = lambda xx, gg: oracle.forward(*(xx[n] for n in backward.NAMES), 0.0, gate=gg)
+    ref = c_fwd(x, gate)
+    got = backward.forward(*(torch.as_tensor(x[n]) for n in backward.NAMES), 0.0,
+                           gate=torch.as_tensor(gate)).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    dout = rng.standard_normal(ref.shape)
+    g = backward.gradients(x, dout, 0.0, gate=gate)
+    assert set(g) == set(backward.NAMES) | {"gate"}
+    h = 1e-5
+    for name in list(backward.NAMES) + ["gate"]:
+        base = gate if name == "gate" else x[name]
+        delta = rng.standard_normal(base.shape)
+        if name == "gate":
+            fp, fm = c_fwd(x, gate + h * delta), c_fwd(x, gate - h * delta)
+        else:
+            plus, minus = dict(x), dict(x)
+            plus[name] = x[name] + h * delta
+            minus[name] = x[name] - h * delta
+            fp, fm = c_fwd(plus, gate), c_fwd(minus, gate)
+        fd = float(np.sum((fp - fm) * dout)) / (2 * h)
+        an = float(np.sum(g[name] * delta))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+ROW_SHAPES = [
+    # B, H, T, d, c_q, c_k, c_h
+    (2, 4, 23, 6, 6, 11, 2),
+    (1, 4, 19, 5, 3, 4, 4),      # even c_k
+    (1, 3, 17, 4, 8, 15, 1),
+]
+
+
+@pytest.mark.parametrize("shape", ROW_SHAPES)
+def test_row_restricted_forward_equals_the_c_oracle_rows(shape):
+    # forward_rows recomputes only what the chosen rows depend on; it must
+    # give the C oracle's rows (computed there one row at a time from scratch),
+    # with and without the gate.
+    x, _ = inputs_of(shape, 66)
+    B, H, T = shape[:3]
+    rows = [0, 1, 2, 7, T // 2, T - 2, T - 1]
+    ts = [torch.as_tensor(x[n]) for n in backward.NAMES]
+    got = backward.forward_rows(*ts, 0.7, rows).numpy()
+    gate = GATE[:H].copy()
+    got_g = backward.forward_rows(*ts, 0.0, rows, gate=torch.as_tensor(gate)).numpy()
+    for b in range(B):
+        ref = oracle.rows(*(x[n] for n in backward.NAMES), 0.7, b, rows)
+        np.testing.assert_allclose(got[b], ref, rtol=0, atol=1e-12)
+        ref_g = oracle.rows(*(x[n] for n in backward.NAMES), 0.0, b, rows, gate=gate)
+        np.testing.assert_allclose(got_g[b], ref_g, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("shape", ROW_SHAPES)
+def test_row_restricted_gradients_equal_full_gradients(shape):
+    # An upstream gradient that vanishes off a few rows: the gradients through
+    # forward_rows equal those of the full restatement (which the finite
+    # difference pins above tie to the C oracle).
+    x, rng = inputs_of(shape, 67)
+    B, H, T, d = shape[:4]
+    rows = [1, 5, T - 1]
+    dout = np.zeros((B, T, H * d))
+    dout[:, rows] = rng.standard_normal((B, len(rows), H * d))
+    full = backward.gradients(x, dout, 0.7)
+    part = backward.gradients_rows(x, rows, dout[:, rows], 0.7)
+    for n in backward.NAMES:
+        np.testing.assert_allclose(part[n], full[n], rtol=0, atol=1e-11, err_msg=n)
+
+
 # (w_kq, w_kq_3d, w_head_pre, w_head, w_kq_post, w_head_post, exact_mask)
 COMPOSED = {
     "repeat": (1, 0, 0, 1, 1, 1, 0),
@@ -158,6 +236,15 @@ BACKWARD_MUTATIONS = [
      "S = torch.where(J - jp <= I - ip, S, torch.zeros((), dtype=X.dtype))"),
     ("post conv not masked", 'A = torch.where(causal, _conv(A, t["w_kq_post"], False), zero)',
      'A = _conv(A, t["w_kq_post"], False)'),
+    ("gate not squashed", "return torch.sigmoid(gate).view(1, H, 1, 1)",
+     "return gate.view(1, H, 1, 1)"),
+    ("row restatement: key shift sign", "jp = jj - R                                # C[j]",
+     "jp = R - jj                                # C[j]"),
+    ("row restatement: no Mask_0", "keep = torch.arange(n) <= r                    # Mask_0",
+     "keep = torch.arange(n) <= i                    # Mask_0"),
+    ("row restatement: gate ignored",
+     "scale = depth_scale if gate is None else torch.sigmoid(gate).view(1, H, 1)",
+     "scale = depth_scale"),
 ]
 
 
@@ -174,7 +261,9 @@ def test_backward_pins_catch_planted_mistakes(monkeypatch, tmp_path, name, befor
     spec.loader.exec_module(mutant)
     monkeypatch.setattr(sys.modules[__name__], "backward", mutant)
     checks = [lambda: test_torch_restatement_equals_the_c_oracle(SHAPES[1]),
-              lambda: test_gradients_match_finite_differences_of_the_c_oracle(SHAPES[1])]
+              lambda: test_gradients_match_finite_differences_of_the_c_oracle(SHAPES[1]),
+              lambda: test_gated_restatement_and_gate_gradient(SHAPES[1]),
+              lambda: test_row_restricted_forward_equals_the_c_oracle_rows(ROW_SHAPES[0])]
     checks += [lambda n=n: test_composed_restatement_and_gradients(n) for n in sorted(COMPOSED)]
     caught = 0
     for check in checks:
