@@ -5,7 +5,7 @@ include/mta.h); this package is its Python binding, with the same function
 names as the C entry points, plus the seeded synthetic workloads used by the
 tests and the benchmark (``convolved_logit_attention_b200.workloads``).
 """
-from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
+from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC, MTA_PATH_FUSED_F32,
                        MTA_PATH_MATERIALISED, MtaComposition, MtaError, MtaShape, lib,
                        make_shape, composed_shape, composition, mta_composed_kernel_names,
                        mta_debug_attention, mta_forward_composed, mta_forward, mta_forward_gated, mta_forward_path,
@@ -16,7 +16,7 @@ from ._binding import (EXPORTS, LIB_PATH, MTA_BF16, MTA_F32, MTA_PATH_FUSED_TC,
                        mta_version, mta_workspace_size, shape_of, GRAD_NAMES, mta_backward,
                        mta_backward_kernel_names, mta_backward_workspace_size)
 
-__all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC",
+__all__ = ["EXPORTS", "LIB_PATH", "MTA_BF16", "MTA_F32", "MTA_PATH_FUSED_TC", "MTA_PATH_FUSED_F32",
            "MTA_PATH_MATERIALISED", "MtaComposition", "MtaError", "MtaShape", "lib",
            "make_shape", "composed_shape", "composition", "mta_composed_kernel_names",
            "mta_debug_attention", "mta_forward_composed", "mta_forward", "mta_forward_gated", "mta_forward_path",

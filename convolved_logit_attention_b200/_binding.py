@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmta.so")
 
 MTA_F32, MTA_BF16 = 0, 1
-MTA_PATH_FUSED_TC, MTA_PATH_MATERIALISED = 0, 1
+MTA_PATH_FUSED_TC, MTA_PATH_MATERIALISED, MTA_PATH_FUSED_F32 = 0, 1, 2
 STATUS = {0: "MTA_OK", -1: "MTA_ERR_INVALID_ARG", -2: "MTA_ERR_UNSUPPORTED",
           -3: "MTA_ERR_ALIGNMENT", -4: "MTA_ERR_WORKSPACE", -5: "MTA_ERR_CUDA",
           -6: "MTA_ERR_DEVICE_TIMEOUT", -7: "MTA_ERR_RANGE"}

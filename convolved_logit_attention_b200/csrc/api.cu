@@ -70,17 +70,39 @@ const char *mta_status_string(mta_status st)
     return "unknown status";
 }
 
+namespace {
+
+// The path of a forward call: the fused kernels for the shapes they take
+// (the fp32 one has no exact-mask variant), else the materialised chain.
+mta_path path_of(const mta_shape &s, int unfused, int exact)
+{
+    if (unfused) return MTA_PATH_MATERIALISED;
+    if (mta::fused_supported(s)) return MTA_PATH_FUSED_TC;
+    if (!exact && mta::fused_f32_supported(s)) return MTA_PATH_FUSED_F32;
+    return MTA_PATH_MATERIALISED;
+}
+
+size_t path_workspace(const mta_shape &s, mta_path p)
+{
+    switch (p) {
+        case MTA_PATH_FUSED_TC: return mta::fused_workspace_bytes(s);
+        case MTA_PATH_FUSED_F32: return 0;
+        default: return mta::unfused_workspace_bytes(s);
+    }
+}
+
+}  // namespace
+
 mta_path mta_forward_path(const mta_shape *s)
 {
     if (check_shape(s) != MTA_OK) return MTA_PATH_MATERIALISED;
-    return mta::fused_supported(*s) ? MTA_PATH_FUSED_TC : MTA_PATH_MATERIALISED;
+    return path_of(*s, 0, 0);
 }
 
 size_t mta_workspace_size(const mta_shape *s)
 {
     if (check_shape(s) != MTA_OK) return 0;
-    return mta::fused_supported(*s) ? mta::fused_workspace_bytes(*s)
-                                    : mta::unfused_workspace_bytes(*s);
+    return path_workspace(*s, path_of(*s, 0, 0));
 }
 
 size_t mta_unfused_workspace_size(const mta_shape *s)
@@ -101,9 +123,8 @@ mta_status forward_impl(int unfused, const mta_shape *s, const void *q, const vo
     if (rc == MTA_OK) rc = check_tensors(q, k, v, w_kq, w_head, gn_weight, gn_bias, out);
     if (rc != MTA_OK) return rc;
     if (n_events < 0 || (n_events > 0 && !events)) return MTA_ERR_INVALID_ARG;
-    const bool fused = !unfused && mta::fused_supported(*s);
-    const size_t need = fused ? mta::fused_workspace_bytes(*s) : mta::unfused_workspace_bytes(*s);
-    rc = check_workspace(workspace, workspace_bytes, need);
+    const mta_path path = path_of(*s, unfused, exact_mask);
+    rc = check_workspace(workspace, workspace_bytes, path_workspace(*s, path));
     if (rc != MTA_OK) return rc;
     mta::ForwardArgs a{q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out, gate};
     a.exact_mask = exact_mask;
@@ -111,8 +132,11 @@ mta_status forward_impl(int unfused, const mta_shape *s, const void *q, const vo
     tr.events = events;
     tr.n = n_events;
     cudaStream_t st = (cudaStream_t)stream;
-    return fused ? mta::launch_fused(*s, a, workspace, st, tr)
-                 : mta::launch_unfused(*s, a, workspace, st, tr);
+    switch (path) {
+        case MTA_PATH_FUSED_TC: return mta::launch_fused(*s, a, workspace, st, tr);
+        case MTA_PATH_FUSED_F32: return mta::launch_fused_f32(*s, a, st, tr);
+        default: return mta::launch_unfused(*s, a, workspace, st, tr);
+    }
 }
 
 }  // namespace
@@ -200,7 +224,8 @@ mta::ForwardArgs chain_args(const mta_composition *c)
 size_t mta_composed_workspace_size(const mta_shape *s, const mta_composition *c)
 {
     if (!c || check_shape(s) != MTA_OK) return 0;
-    return is_default_composition(c) ? mta_workspace_size(s) : mta::unfused_workspace_bytes(*s);
+    return is_default_composition(c) ? path_workspace(*s, path_of(*s, 0, c->exact_mask))
+                                     : mta::unfused_workspace_bytes(*s);
 }
 
 mta_status mta_forward_composed(const mta_shape *s, const void *q, const void *k, const void *v,
@@ -226,7 +251,9 @@ mta_status mta_forward_composed_traced(const mta_shape *s, const void *q, const 
 int mta_composed_kernel_count(const mta_shape *s, const mta_composition *c)
 {
     if (!c || check_shape(s) != MTA_OK) return 0;
-    if (is_default_composition(c)) return mta_kernel_count(s, 0);
+    if (is_default_composition(c) && !c->exact_mask) return mta_kernel_count(s, 0);
+    if (is_default_composition(c) && path_of(*s, 0, 1) == MTA_PATH_FUSED_TC)
+        return mta::fused_kernel_count(*s);
     const char *names[mta::kMaxChainKernels];
     return mta::unfused_chain(chain_args(c), names);
 }
@@ -234,7 +261,9 @@ int mta_composed_kernel_count(const mta_shape *s, const mta_composition *c)
 const char *mta_composed_kernel_name(const mta_shape *s, const mta_composition *c, int index)
 {
     if (!c || check_shape(s) != MTA_OK || index < 0) return nullptr;
-    if (is_default_composition(c)) return mta_kernel_name(s, 0, index);
+    if (is_default_composition(c) && !c->exact_mask) return mta_kernel_name(s, 0, index);
+    if (is_default_composition(c) && path_of(*s, 0, 1) == MTA_PATH_FUSED_TC)
+        return mta::fused_kernel_name(*s, index);
     const char *names[mta::kMaxChainKernels];
     const int n = mta::unfused_chain(chain_args(c), names);
     return index < n ? names[index] : nullptr;
@@ -278,16 +307,22 @@ mta_status mta_forward_noalloc(const mta_shape *s, const void *q, const void *k,
 int mta_kernel_count(const mta_shape *s, int unfused)
 {
     if (check_shape(s) != MTA_OK) return 0;
-    if (!unfused && mta::fused_supported(*s)) return mta::fused_kernel_count(*s);
-    return mta::kUnfusedKernels;
+    switch (path_of(*s, unfused, 0)) {
+        case MTA_PATH_FUSED_TC: return mta::fused_kernel_count(*s);
+        case MTA_PATH_FUSED_F32: return 1;
+        default: return mta::kUnfusedKernels;
+    }
 }
 
 const char *mta_kernel_name(const mta_shape *s, int unfused, int index)
 {
     if (check_shape(s) != MTA_OK || index < 0 || index >= mta_kernel_count(s, unfused))
         return nullptr;
-    if (!unfused && mta::fused_supported(*s)) return mta::fused_kernel_name(*s, index);
-    return mta::kUnfusedKernelNames[index];
+    switch (path_of(*s, unfused, 0)) {
+        case MTA_PATH_FUSED_TC: return mta::fused_kernel_name(*s, index);
+        case MTA_PATH_FUSED_F32: return "k_mta_fused_f32";
+        default: return mta::kUnfusedKernelNames[index];
+    }
 }
 
 mta_status mta_debug_attention(const mta_shape *s, const void *q, const void *k,

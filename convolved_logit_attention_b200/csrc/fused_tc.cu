@@ -130,28 +130,10 @@ __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Largest |x| over rows [r_lo, r_hi) (clipped to [0, T)) of one head's bf16
-// [T][D] rows, reduced over the CTA (blockDim.x a multiple of 32, at most
-// 256): every thread gets the result.  A non-finite element anywhere makes
-// the result +inf.  `red` is 8 floats of shared memory.
-template <int D>
-__device__ float rows_absmax(const __nv_bfloat16 *__restrict__ head, int r_lo, int r_hi, int T,
-                             float *red)
+// Largest value of m over the CTA (blockDim.x a multiple of 32, at most
+// 256); every thread gets the result.  `red` is 8 floats of shared memory.
+__device__ float block_max(float m, float *red)
 {
-    const int lo = r_lo > 0 ? r_lo : 0, hi = r_hi < T ? r_hi : T;
-    float m = 0.f;
-    bool finite = true;
-    for (int idx = threadIdx.x; idx < (hi - lo) * (D / 8); idx += blockDim.x) {
-        const uint4 v = *(const uint4 *)(head + (size_t)(lo + idx / (D / 8)) * D + 8 * (idx % (D / 8)));
-        const __nv_bfloat162 *p = (const __nv_bfloat162 *)&v;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float2 f = __bfloat1622float2(p[u]);
-            finite &= fabsf(f.x) <= 3.0e38f && fabsf(f.y) <= 3.0e38f;   // false for NaN too
-            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
-    }
-    if (!finite) m = INFINITY;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     __syncthreads();                           // red may still be read by an earlier use
@@ -162,32 +144,40 @@ __device__ float rows_absmax(const __nv_bfloat16 *__restrict__ head, int r_lo, i
     return r;
 }
 
-// The power-of-two exponent e >= 0 of a block's fp16 operand scale: the
-// smallest e with bound * 2^-e <= 2^14, a quarter of the fp16 range, so that
-// sums of the block's products stay far from overflow.  Blocks whose bound is
-// already below it keep e = 0 (the usual case: the fused path then computes
-// exactly as without scaling).  Returns -1 for a non-finite bound.
-__device__ __forceinline__ int range_exponent(float bound)
+// |x| of both halves of a bf16 pair, folded into a running max; a NaN or
+// infinite element makes the max +inf.
+__device__ __forceinline__ float absmax_bf2(float m, uint32_t v)
 {
-    if (bound <= 16384.f) return 0;
-    if (!(bound <= 3.0e38f)) return -1;
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+    const float ax = fabsf(f.x), ay = fabsf(f.y);
+    return (ax <= 3.0e38f && ay <= 3.0e38f) ? fmaxf(m, fmaxf(ax, ay)) : INFINITY;  // NaN: false
+}
+
+// The power-of-two exponent e >= 0 of a block's fp16 operand scale, from the
+// largest |value| of the block: 0 when it fits fp16 (the usual case: the
+// block is then computed exactly as without scaling), else the smallest e
+// with max * 2^-e <= 2^15.  -1 for a non-finite max.
+__device__ __forceinline__ int range_exponent(float mx)
+{
+    if (mx <= 65504.f) return 0;
+    if (!(mx <= 3.0e38f)) return -1;
     int e = 0;
-    frexpf(bound / 16384.f, &e);               // bound / 2^14 <= 2^e
+    frexpf(mx / 32768.f, &e);                  // mx / 2^15 <= 2^e
     return e;
 }
 
-// Folded keys: one CTA per (128-key block, b*H + h), 256 threads; thread =
-// one column pair x a run of RPG consecutive keys, in windows of SUB keys.
-// Kf^{(i')}_j = sum_jj ths[i'][jj] k_{j + RT - jj}, with the taps zero-padded
-// to CK (CK = c_k for the common sizes, 15 otherwise) and centred like the
-// real kernel, so every tap index is a compile-time constant.  The two
-// columns of a pair share every tap: one packed f32x2 FMA per tap.
+// Folded keys of one 128-key block with the taps in ths (the logit scale,
+// and a range scale if any, included): thread = one column pair x a run of
+// RPG consecutive keys, in windows of SUB keys.  Kf^{(i')}_j =
+// sum_jj ths[i'][jj] k_{j + RT - jj}, with the taps zero-padded to CK (CK =
+// c_k for the common sizes, 15 otherwise) and centred like the real kernel,
+// so every tap index is a compile-time constant.  The two columns of a pair
+// share every tap: one packed f32x2 FMA per tap.  Returns the largest |Kf|
+// this thread wrote (after the fp16 rounding: +inf where a value overflowed).
 template <int D, int CK>
-__device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bfloat16 *__restrict__ k,
-                                                const float *__restrict__ w_kq,
-                                                __half *__restrict__ kf, int *__restrict__ kexp,
-                                                int T, int Tp, int H, int nqb, int c_q, int c_k,
-                                                float scale)
+__device__ __forceinline__ float fold_keys_run(int blk, int bh, const __nv_bfloat16 *__restrict__ k,
+                                               const float *ths, __half *__restrict__ kf, int T,
+                                               int Tp, int c_q)
 {
     constexpr int EP = D / 2;                  // column pairs
     constexpr int RG = 256 / EP;               // key runs per block
@@ -195,43 +185,10 @@ __device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bflo
     constexpr int RT = CK / 2, LT = CK - 1 - RT;
     constexpr int SUB = 16;
     constexpr int WS = SUB + CK - 1;           // window rows
-    __shared__ float ths[8 * CK];              // zero-padded taps times the logit scale
-    const int h = bh % H;
     const int j0 = blk * kProRows;
-    const int tid = threadIdx.x;
-    const int R = c_k / 2, shift = RT - R;     // real tap jj sits at padded index jj + shift
-    for (int idx = tid; idx < 8 * CK; idx += 256) {
-        const int ip = idx / CK, jp = idx % CK - shift;
-        ths[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] * scale
-                                                     : 0.f;
-    }
-    // Range of the block's folded keys: |Kf^{(i')}_j| <= max |k| over the
-    // window rows times max_{i'} sum_{j'} |theta'|.  Beyond 2^14 the taps are
-    // scaled by 2^-e (exactly), and the main kernel multiplies the logits of
-    // this key block back by 2^e.
-    __shared__ float red[8];
-    __shared__ int s_e;
-    const float mk = rows_absmax<D>(k + (size_t)bh * T * D, j0 - LT, j0 + kProRows + RT, T, red);
-    if (tid == 0) {
-        float tb = 0.f;
-        for (int ip = 0; ip < c_q; ++ip) {
-            float a = 0.f;
-            for (int jj = 0; jj < CK; ++jj) a += fabsf(ths[ip * CK + jj]);
-            tb = fmaxf(tb, a);
-        }
-        int e = range_exponent(mk * tb);
-        if (e < 0) { atomicOr(&g_fused_error, kErrRange); e = 0; }
-        s_e = e;
-        kexp[(size_t)bh * nqb + blk] = e;
-    }
-    __syncthreads();
-    if (s_e != 0) {
-        for (int idx = tid; idx < 8 * CK; idx += 256) ths[idx] = ldexpf(ths[idx], -s_e);
-        __syncthreads();
-    }
-    const int ep = tid % EP, rg = tid / EP;
+    const int ep = threadIdx.x % EP, rg = threadIdx.x / EP;
     const __nv_bfloat16 *kh = k + (size_t)bh * T * D + 2 * ep;
-    __half2 amax = __floats2half2_rn(0.f, 0.f);   // largest |Kf| this thread wrote, per column
+    __half2 amax = __floats2half2_rn(0.f, 0.f);
 #pragma unroll 1
     for (int sub = 0; sub < RPG / SUB; ++sub) {
         const int jr0 = j0 + rg * RPG + sub * SUB;     // first key of the window
@@ -262,10 +219,75 @@ __device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bflo
             }
         }
     }
-    // a folded key beyond the fp16 range became infinite: only non-finite
-    // inputs get here after the scaling above (NaN inputs stay NaN)
     const float2 am = __half22float2(amax);
-    if (am.x > 65504.f || am.y > 65504.f) atomicOr(&g_fused_error, kErrRange);
+    return fmaxf(am.x, am.y);
+}
+
+// Largest |x| over rows [r_lo, r_hi) (clipped to [0, T)) of one head's bf16
+// [T][D] rows, over the CTA (every thread gets it; +inf for a non-finite
+// element).  `red` is 8 floats of shared memory.
+template <int D>
+__device__ float rows_absmax(const __nv_bfloat16 *__restrict__ head, int r_lo, int r_hi, int T,
+                             float *red)
+{
+    const int lo = r_lo > 0 ? r_lo : 0, hi = r_hi < T ? r_hi : T;
+    float m = 0.f;
+    for (int idx = threadIdx.x; idx < (hi - lo) * (D / 8); idx += blockDim.x) {
+        const uint4 v = *(const uint4 *)(head + (size_t)(lo + idx / (D / 8)) * D + 8 * (idx % (D / 8)));
+        m = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(m, v.x), v.y), v.z), v.w);
+    }
+    return block_max(m, red);
+}
+
+// Folded keys: one CTA per (128-key block, b*H + h), 256 threads.  The
+// block is written as computed, and an fp16 overflow shows up as +inf in the
+// largest |Kf| written.  Such a block (a bf16 input of order 1e4 or more) is
+// computed a second time with the taps scaled by 2^-e, exactly, e chosen from
+// the bound max |k| over the window times max_{i'} sum_{j'} |tap|; the main
+// kernel multiplies the logits of this key block back by 2^e.
+template <int D, int CK>
+__device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bfloat16 *__restrict__ k,
+                                                const float *__restrict__ w_kq,
+                                                __half *__restrict__ kf, int *__restrict__ kexp,
+                                                int T, int Tp, int H, int nqb, int c_q, int c_k,
+                                                float scale)
+{
+    constexpr int RT = CK / 2;
+    __shared__ float ths[8 * CK];              // zero-padded taps times the logit scale
+    __shared__ float red[8];
+    const int h = bh % H;
+    const int tid = threadIdx.x;
+    const int R = c_k / 2, shift = RT - R;     // real tap jj sits at padded index jj + shift
+    for (int idx = tid; idx < 8 * CK; idx += 256) {
+        const int ip = idx / CK, jp = idx % CK - shift;
+        ths[idx] = (ip < c_q && jp >= 0 && jp < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jp] * scale
+                                                     : 0.f;
+    }
+    __syncthreads();
+    const float amax = fold_keys_run<D, CK>(blk, bh, k, ths, kf, T, Tp, c_q);
+    int e = 0;
+    if (block_max(amax, red) > 65504.f) {      // the same in every thread; rare
+        constexpr int LT = CK - 1 - RT;
+        const int j0 = blk * kProRows;
+        const float mk = rows_absmax<D>(k + (size_t)bh * T * D, j0 - LT, j0 + kProRows + RT, T, red);
+        float tb = 0.f;
+        for (int ip = 0; ip < c_q; ++ip) {
+            float a = 0.f;
+            for (int jj = 0; jj < CK; ++jj) a += fabsf(ths[ip * CK + jj]);
+            tb = fmaxf(tb, a);
+        }
+        e = range_exponent(mk * tb);
+        if (e < 0) {                           // non-finite input: report it
+            if (tid == 0) atomicOr(&g_fused_error, kErrRange);
+            e = 0;
+        } else {
+            __syncthreads();                   // every thread has read the taps
+            for (int idx = tid; idx < 8 * CK; idx += 256) ths[idx] = ldexpf(ths[idx], -e);
+            __syncthreads();
+            fold_keys_run<D, CK>(blk, bh, k, ths, kf, T, Tp, c_q);
+        }
+    }
+    if (tid == 0) kexp[(size_t)bh * nqb + blk] = e;
 }
 
 // The rest of the prologue: one CTA per (64-row block, b*H + h), 160
@@ -325,21 +347,45 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
         const __nv_bfloat16 *src = (isq ? q : k) + head_off + (size_t)(in ? g : 0) * D + 8 * c8;
         tc::cp_async16((isq ? qsm : ksm) + lr * RS + 8 * c8, src, in);
     }
+    // Range of the 128-row block's permuted queries: both halves' CTAs take
+    // the largest |q| over the rows [i0 - 7, i0 + 128), their own 71 rows from
+    // the copy and the other half's 64 rows loaded here, while the copy is in
+    // flight.  A block beyond the fp16 range is scaled by 2^-e before the
+    // rounding, and the main kernel multiplies its logits back by 2^e.
+    const int i0 = qblk * kProRows;
+    constexpr int NL = 64 * CPR / kProThreads;
+    static_assert(64 * CPR % kProThreads == 0, "other-half rows per thread");
+    float mq = 0.f;
+    {
+        const int ro = half == 0 ? i0 + kAuxRows : i0 - kProQLo;   // the other half's rows
+#pragma unroll
+        for (int u = 0; u < NL; ++u) {
+            const int idx = tid + u * kProThreads;
+            const int row = ro + idx / CPR, c8 = idx % CPR;
+            if (row >= 0 && row < T) {
+                const uint4 v = *(const uint4 *)(q + head_off + (size_t)row * D + 8 * c8);
+                mq = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(mq, v.x), v.y), v.z), v.w);
+            }
+        }
+    }
     tc::cp_async_wait_all();
     __syncthreads();
-    // Range of the 128-row block's permuted queries (rows i0 - c_q + 1 ..
-    // i0 + 127, the same for both halves' CTAs): beyond 2^14 they are scaled
-    // by 2^-e before the fp16 rounding, and the main kernel multiplies this
-    // block's logits back by 2^e.
-    __shared__ float red[8];
-    int eq;
-    {
-        const int i0 = qblk * kProRows;
-        const float mq = rows_absmax<D>(q + head_off, i0 - (c_q - 1), i0 + kProRows, T, red);
-        eq = range_exponent(mq);
-        if (eq < 0) { if (tid == 0) atomicOr(&g_fused_error, kErrRange); eq = 0; }
-        if (tid == 0 && half == 0) qexp[(size_t)bh * nqb + qblk] = eq;
+    for (int idx = tid; idx < QR * CPR; idx += kProThreads) {
+        const uint4 v = *(const uint4 *)(qsm + (idx / CPR) * RS + 8 * (idx % CPR));
+        mq = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(mq, v.x), v.y), v.z), v.w);
     }
+    // a non-finite key among this CTA's copied rows (they cover every key of
+    // the head over the grid) is reported here: the fold cannot tell a NaN
+    bool kfin = true;
+    for (int idx = tid; idx < KR * CPR; idx += kProThreads) {
+        const uint4 v = *(const uint4 *)(ksm + (idx / CPR) * RS + 8 * (idx % CPR));
+        kfin &= absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(0.f, v.x), v.y), v.z), v.w) <= 3.0e38f;
+    }
+    if (!kfin) atomicOr(&g_fused_error, kErrRange);
+    __shared__ float red[8];
+    int eq = range_exponent(block_max(mq, red));
+    if (eq < 0) { if (tid == 0) atomicOr(&g_fused_error, kErrRange); eq = 0; }
+    if (tid == 0 && half == 0) qexp[(size_t)bh * nqb + qblk] = eq;
     const float qsc = ldexpf(1.f, -eq);       // exact: a power of two
     // (b) permuted query rows of the 128-row block jb0 = j0 - 64*half: atom a,
     //     row s <- q_{jb0-(c_q-1)+a+16s}; this CTA writes rows s in

@@ -92,6 +92,11 @@ size_t backward_workspace_bytes(const mta_shape &s);
 mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const BackwardArgs &g,
                            void *ws, cudaStream_t st, const Trace &tr);
 
+// Fused fp32 path (fused_f32.cu): fp32 I/O, CUDA cores, no workspace.
+bool fused_f32_supported(const mta_shape &s);
+mta_status launch_fused_f32(const mta_shape &s, const ForwardArgs &a, cudaStream_t st,
+                            const Trace &tr);
+
 // Fused tcgen05 path (fused_tc.cu).
 bool fused_supported(const mta_shape &s);
 size_t fused_workspace_bytes(const mta_shape &s);

@@ -88,8 +88,12 @@ typedef struct {
 
 /* Which device path mta_forward takes for a shape. */
 typedef enum {
-    MTA_PATH_FUSED_TC = 0,       /* fused tcgen05 kernel: no T x T map in HBM */
-    MTA_PATH_MATERIALISED = 1    /* the S1..S9 chain of mta_forward_unfused */
+    MTA_PATH_FUSED_TC = 0,       /* bf16 I/O, d in {64, 128}: fused tcgen05 kernels, no T x T
+                                    map in HBM */
+    MTA_PATH_MATERIALISED = 1,   /* the S1..S9 chain of mta_forward_unfused */
+    MTA_PATH_FUSED_F32 = 2       /* fp32 I/O with c_h * d <= 256: one fused kernel on CUDA
+                                    cores (fp32 arithmetic), no T x T map in HBM, no
+                                    workspace */
 } mta_path;
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */

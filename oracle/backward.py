@@ -36,7 +36,10 @@ NAMES = ("q", "k", "v", "w_kq", "w_head", "gn_weight", "gn_bias")
 
 def _shift(X, a, b):
     """Y[..., i, j] = X[..., i - a, j - b], zero where i - a or j - b falls
-    outside the map (negative padding crops)."""
+    outside the map (negative padding crops); a shift by the map's whole
+    height or width or more leaves only zeros."""
+    if abs(a) >= X.shape[-2] or abs(b) >= X.shape[-1]:
+        return torch.zeros_like(X)
     return torch.nn.functional.pad(X, (b, -b, a, -a))
 
 

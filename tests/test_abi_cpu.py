@@ -120,8 +120,9 @@ def test_unfused_workspace_is_two_fp32_maps(L):
     (dict(B=1, H=16, T=16384, d=128, c_q=6, c_k=11, c_h=4), 0),    # split output heads
     (dict(B=1, H=16, T=256, d=128, c_q=6, c_k=11, c_h=8), 1),      # c_h * d > 512
     (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2), 1),        # d not 64 or 128
-    (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2, io="f32"), 1),
-    (dict(B=1, H=4, T=128, d=128, c_q=6, c_k=11, c_h=2, io="f32"), 1),
+    (dict(B=1, H=4, T=128, d=32, c_q=6, c_k=11, c_h=2, io="f32"), 2),    # the fp32 workload
+    (dict(B=1, H=4, T=128, d=128, c_q=6, c_k=11, c_h=2, io="f32"), 2),
+    (dict(B=1, H=8, T=128, d=128, c_q=6, c_k=11, c_h=4, io="f32"), 1),   # c_h * d > 256
 ])
 def test_forward_path_selection(L, kw, path):
     s = shape(**kw)
@@ -129,6 +130,9 @@ def test_forward_path_selection(L, kw, path):
     names = [mta.mta_kernel_name(s, i) for i in range(mta.mta_kernel_count(s))]
     if path == 0:   # prologue, main kernel, mix + GroupNorm
         assert names == ["k_fold", "k_mta_fused", "k_mix_groupnorm"]
+    elif path == 2:  # one fused fp32 kernel, no workspace
+        assert names == ["k_mta_fused_f32"]
+        assert mta.mta_workspace_size(s) == 0
     else:           # the four materialised kernels
         assert names == ["k_logits", "k_conv", "k_softmax_mix", "k_pv_groupnorm"]
 

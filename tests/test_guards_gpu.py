@@ -34,6 +34,12 @@ SHAPES = [
     (1, 8, 255, 64, 3, 5, 8),
     (1, 2, 513, 128, 2, 3, 1),
 ]
+# fp32 I/O: the fused CUDA-core kernel (path 2) and, past c_h * d = 256, the chain
+SHAPES_F32 = [
+    (1, 4, 128, 32, 6, 11, 2),
+    (2, 2, 77, 64, 4, 15, 2),
+    (1, 2, 1, 128, 8, 15, 2),
+]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -43,11 +49,12 @@ def _built():
     assert torch.cuda.is_available()
 
 
-def _inputs(shape, seed):
+def _inputs(shape, seed, io="bf16"):
     B, H, T, d, c_q, c_k, c_h = shape
-    x = make_inputs(Workload("guards", B, H, T, d, c_q, c_k, c_h, "bf16", seed=seed))
+    x = make_inputs(Workload("guards", B, H, T, d, c_q, c_k, c_h, io, seed=seed))
     dev = torch.device("cuda", 0)
-    t = {n: torch.from_numpy(x[n]).to(dev).to(torch.bfloat16) for n in ("q", "k", "v")}
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    t = {n: torch.from_numpy(x[n]).to(dev).to(dt) for n in ("q", "k", "v")}
     for n in ("w_kq", "w_head", "gn_weight", "gn_bias"):
         t[n] = torch.from_numpy(x[n]).to(dev)
     return x, t
@@ -95,3 +102,25 @@ def test_stores_stay_inside_out_and_workspace(shape, unfused):
     out = out_body.view(torch.bfloat16).float()
     assert torch.isfinite(out).all()
     assert not bool((out_body.view(torch.int16) == np.int16(-23131)).any())
+
+
+@pytest.mark.parametrize("shape", SHAPES_F32, ids=[str(s) for s in SHAPES_F32])
+def test_fp32_fused_stores_stay_inside_out(shape):
+    B, H, T, d, c_q, c_k, c_h = shape
+    x, t = _inputs(shape, seed=sum(shape) + 1, io="f32")
+    mshape = mta.make_shape(B, H, T, d, c_q, c_k, c_h, "f32", x["gn_eps"])
+    assert mta.mta_forward_path(mshape) == mta.MTA_PATH_FUSED_F32
+    assert mta.mta_workspace_size(mshape) == 0
+    out_bytes = B * T * H * d * 4
+    out_buf, out_body = _guarded(out_bytes)
+    L = mta.lib()
+    p = lambda a: ctypes.c_void_p(a.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = L.mta_forward(ctypes.byref(mshape), p(t["q"]), p(t["k"]), p(t["v"]), p(t["w_kq"]),
+                       p(t["w_head"]), p(t["gn_weight"]), p(t["gn_bias"]),
+                       ctypes.c_float(x["depth_scale"]), p(out_body), None, ctypes.c_size_t(0),
+                       stream)
+    assert rc == 0
+    mta.mta_sync_status()
+    assert _guards_intact(out_buf, out_bytes), "a store landed outside out"
+    assert torch.isfinite(out_body.view(torch.float32)).all()

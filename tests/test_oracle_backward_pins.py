@@ -40,6 +40,19 @@ def test_torch_restatement_equals_the_c_oracle(shape):
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("shape", [(1, 2, 1, 4, 6, 11, 2), (2, 2, 2, 3, 8, 15, 1),
+                                   (1, 4, 3, 4, 4, 3, 4)])
+def test_shorter_than_the_kernel(shape):
+    # T below c_q or c_k: every shift past the map reads zeros, as in the C
+    # oracle; the restatement and its gradients stay defined
+    x, rng = inputs_of(shape, 68)
+    ref = oracle.forward(*(x[n] for n in backward.NAMES), 0.7)
+    got = backward.forward(*(torch.as_tensor(x[n]) for n in backward.NAMES), 0.7).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    g = backward.gradients(x, rng.standard_normal(ref.shape), 0.7)
+    assert all(np.isfinite(v).all() for v in g.values())
+
+
 @pytest.mark.parametrize("shape", SHAPES)
 def test_gradients_match_finite_differences_of_the_c_oracle(shape):
     # <grad_X, delta> = (f(X + h delta) - f(X - h delta)) . dout / (2 h),

@@ -67,6 +67,14 @@ def oracle_full(x):
 FNS = {"forward": mta.mta_forward, "unfused": mta.mta_forward_unfused}
 
 
+def test_each_small_workload_takes_a_fused_path():
+    # the fp32 workload on the fused CUDA-core kernel, the bf16 one on tcgen05
+    for name, path in (("tiny_f32", mta.MTA_PATH_FUSED_F32), ("toy_letters", mta.MTA_PATH_FUSED_TC)):
+        w = WORKLOADS[name]
+        s = mta.make_shape(w.B, w.H, w.T, w.d, w.c_q, w.c_k, w.c_h, w.io)
+        assert mta.mta_forward_path(s) == path, name
+
+
 @pytest.mark.parametrize("fn", sorted(FNS))
 @pytest.mark.parametrize("name", ["tiny_f32", "toy_letters"])
 def test_small_workloads_elementwise(name, fn):
