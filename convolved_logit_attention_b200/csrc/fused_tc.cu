@@ -374,14 +374,6 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
         const uint4 v = *(const uint4 *)(qsm + (idx / CPR) * RS + 8 * (idx % CPR));
         mq = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(mq, v.x), v.y), v.z), v.w);
     }
-    // a non-finite key among this CTA's copied rows (they cover every key of
-    // the head over the grid) is reported here: the fold cannot tell a NaN
-    bool kfin = true;
-    for (int idx = tid; idx < KR * CPR; idx += kProThreads) {
-        const uint4 v = *(const uint4 *)(ksm + (idx / CPR) * RS + 8 * (idx % CPR));
-        kfin &= absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(0.f, v.x), v.y), v.z), v.w) <= 3.0e38f;
-    }
-    if (!kfin) atomicOr(&g_fused_error, kErrRange);
     __shared__ float red[8];
     int eq = range_exponent(block_max(mq, red));
     if (eq < 0) { if (tid == 0) atomicOr(&g_fused_error, kErrRange); eq = 0; }
@@ -1316,12 +1308,18 @@ k_mix_groupnorm(const __half *__restrict__ part, const float *__restrict__ gn_we
     const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     uint4 res;
     uint32_t *rp = (uint32_t *)&res;
+    bool finite = true;
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
         const float y0 = scale * ((o[2 * x] - mean) * inv * wv[2 * x] + bv[2 * x]);
         const float y1 = scale * ((o[2 * x + 1] - mean) * inv * wv[2 * x + 1] + bv[2 * x + 1]);
+        finite &= fabsf(y0) <= 3.0e38f && fabsf(y1) <= 3.0e38f;   // false for NaN too
         rp[x] = pack_bf16(y0, y1);
     }
+    // an output that is not finite can only come from a non-finite q, k or v
+    // (or one the fp16 operands could not hold): report it
+    if (__any_sync(0xffffffffu, live && !finite) && threadIdx.x % 32 == 0)
+        atomicOr(&g_fused_error, kErrRange);
     if (live) *(uint4 *)(out + bt * ((long long)H * D) + (long long)h * D + e0) = res;
 }
 

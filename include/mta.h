@@ -68,7 +68,8 @@ typedef enum {
     MTA_ERR_WORKSPACE = -4,      /* workspace smaller than the *_workspace_size query */
     MTA_ERR_CUDA = -5,           /* a CUDA runtime call failed */
     MTA_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
-    MTA_ERR_RANGE = -7           /* the fused path met a non-finite q, k or folded key */
+    MTA_ERR_RANGE = -7           /* the fused path met a non-finite input or produced a
+                                    non-finite output */
 } mta_status;
 
 typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
@@ -124,8 +125,8 @@ MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
  * than 2^28 times smaller than their block's largest then fall into fp16's
  * subnormal range, with an absolute error up to 2^(e-25) for the block's
  * scale 2^e (for one query of 2e6 among N(0,1) values, e = 7: 4e-6).  A
- * non-finite q or k makes the call's next mta_sync_status() report
- * MTA_ERR_RANGE.
+ * non-finite q, k or v (anything that makes an output non-finite) makes the
+ * call's next mta_sync_status() report MTA_ERR_RANGE.
  * The workspace is scratch owned by the caller for the duration of the
  * enqueued work; its contents on entry are ignored. */
 MTA_API mta_status mta_forward(const mta_shape *shape, const void *q, const void *k, const void *v,

@@ -5,10 +5,15 @@ The backward computes every step in fp32 on the materialised chain, from the
 same rounded inputs and upstream gradient the oracle widens to fp64.  Its
 error is fp32 rounding accumulated over sums of up to T * c_q * c_k terms,
 relative to the size of the gradient, so each gradient is held to
-    max-abs <= 2e-4 * max|ref|   and   rel-L2 <= 1e-4,
+    max-abs <= 2e-4 * S   and   rel-L2 <= 1e-4,
 about two orders of magnitude above what fp32 summation of these lengths
 gives on random data, and far below what a wrong index, sign or mask would
-leave (those move whole rows or taps by O(1) relative error).
+leave (those move whole rows or taps by O(1) relative error).  S is the
+gradient's own largest |entry|, but at least 1% of the largest entry of any
+gradient of the case: a gradient whose exact value cancels to almost zero
+(dw_head at T = 1 is exactly 0, because GroupNorm's backward projects dO off
+V) keeps the fp32 rounding of the terms that cancel, whose size is that of
+the case's other gradients.  Such a gradient is held to the max-abs bound.
 """
 import zlib
 
@@ -58,23 +63,27 @@ def _gpu_grads(d, x):
     return {n: t.cpu().numpy().astype(np.float64) for n, t in g.items()}
 
 
+FLOOR = 1e-2      # of the case's largest gradient entry (see the module docstring)
+
+
 def assert_grads_close(got, ref, what):
     assert set(got) == set(ref), (sorted(got), sorted(ref))
+    case_max = max(float(np.abs(r).max()) for r in ref.values())
     for n in ref:
         a, r = got[n], ref[n]
         assert a.shape == r.shape, (what, n, a.shape, r.shape)
         assert np.isfinite(a).all(), "%s d%s: non-finite" % (what, n)
-        scale = float(np.abs(r).max())
-        if scale == 0.0:
-            assert np.abs(a).max() == 0.0, "%s d%s: expected zeros" % (what, n)
-            continue
+        own = float(np.abs(r).max())
+        scale = max(own, FLOOR * case_max)
         err = np.abs(a - r)
         rel_max = float(err.max()) / scale
-        rel_l2 = float(np.linalg.norm(a - r) / np.linalg.norm(r))
         idx = np.unravel_index(int(err.argmax()), err.shape)
-        assert rel_max <= TOL_REL_MAX and rel_l2 <= TOL_REL_L2, \
-            "%s d%s: max-abs/max|ref| %.3g rel-L2 %.3g (worst at %s)" % (what, n, rel_max,
-                                                                         rel_l2, idx)
+        assert rel_max <= TOL_REL_MAX, \
+            "%s d%s: max-abs/S %.3g (worst at %s; max|ref| %.3g, S %.3g)" % (
+                what, n, rel_max, idx, own, scale)
+        if own >= FLOOR * case_max:
+            rel_l2 = float(np.linalg.norm(a - r) / np.linalg.norm(r))
+            assert rel_l2 <= TOL_REL_L2, "%s d%s: rel-L2 %.3g" % (what, n, rel_l2)
 
 
 def _case(w, seed_dout, gate=None, x=None):
