@@ -65,7 +65,7 @@ const char *mta_status_string(mta_status st)
         case MTA_ERR_WORKSPACE: return "workspace too small";
         case MTA_ERR_CUDA: return "CUDA runtime error";
         case MTA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
-        case MTA_ERR_RANGE: return "non-finite input on the fused path";
+        case MTA_ERR_RANGE: return "input outside the fused path's accuracy domain (beyond fp16 or non-finite)";
     }
     return "unknown status";
 }

@@ -277,8 +277,10 @@ __device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bflo
             tb = fmaxf(tb, a);
         }
         e = range_exponent(mk * tb);
-        if (e < 0) {                           // non-finite input: report it
-            if (tid == 0) atomicOr(&g_fused_error, kErrRange);
+        // reported either way: a non-finite input, or a block beyond fp16 that
+        // stays finite but whose logits near the diagonal lose accuracy
+        if (tid == 0) atomicOr(&g_fused_error, kErrRange);
+        if (e < 0) {
             e = 0;
         } else {
             __syncthreads();                   // every thread has read the taps
@@ -288,6 +290,37 @@ __device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bflo
         }
     }
     if (tid == 0) kexp[(size_t)bh * nqb + blk] = e;
+}
+
+// The terms of four correction entries e = E0 .. E0+3 of one row: for every
+// query tap i' < c_q and padded key tap jj, thp[i'][jj] times the future logit
+// F[i - i'][delta] (frow0 is row i's F row; row i - i' lies i' rows of
+// stride fstride before it), delta = i' + RT - jj - e.  Every index is static
+// after unrolling, so terms outside 1 <= delta <= 14 are never emitted.
+template <int CK, int E0>
+__device__ __forceinline__ void corr_terms(float (&acc)[4], const float *frow0, int fstride,
+                                           const float *thp, int c_q, int exact)
+{
+    constexpr int RT = CK / 2;
+#pragma unroll
+    for (int ip = 0; ip < 8; ++ip) {
+        if (ip < c_q) {
+            const float *frow = frow0 - ip * fstride;
+#pragma unroll
+            for (int jj = 0; jj < CK; ++jj) {
+                if (ip + RT - jj - E0 < 1) continue;          // every delta of this tap < 1
+                const float t = thp[ip * CK + jj];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int delta = ip + RT - jj - (E0 + e);
+                    if (delta >= 1 && delta <= kCorrW - 2) {
+                        const float f = (exact && delta <= ip) ? 0.f : frow[delta - 1];
+                        acc[e] = fmaf(t, f, acc[e]);
+                    }
+                }
+            }
+        }
+    }
 }
 
 // The rest of the prologue: one CTA per (64-row block, b*H + h), 160
@@ -302,7 +335,7 @@ __device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bflo
 //      `exact` (the indicator of Eq. (4), which keeps a tap whenever its key
 //      is not past the output's query i) only the terms with delta > i',
 //      that is key r + delta > i, are removed.
-template <int D>
+template <int D, int CK>
 __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloat16 *__restrict__ q,
                                                const __nv_bfloat16 *__restrict__ k,
                                                const float *__restrict__ w_kq,
@@ -311,9 +344,10 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
                                                int nqb, int c_q, int c_k, float scale, int exact)
 {
     constexpr int QR = kProQLo + kAuxRows;
-    constexpr int TW = 16;                     // tap row stride (c_k <= 15)
-    __shared__ float th[8 * TW];
-    __shared__ float fs[QR * kCorrW];
+    constexpr int RT = CK / 2;                 // the taps' padded centre
+    constexpr int kFs = kCorrW + 1;            // F row stride: rows of a warp hit distinct banks
+    __shared__ float thp[8 * CK];              // taps zero-padded to CK and centred at RT
+    __shared__ float fs[QR * kFs];
     extern __shared__ __align__(16) __nv_bfloat16 qk_sm[];   // section (c) row copies
     const int h = bh % H;
     const int j0 = blk * kAuxRows;
@@ -321,12 +355,11 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
     const int qblk = j0 / kProRows, half = (j0 % kProRows) / kAuxRows;
     const int tid = threadIdx.x;
     const size_t head_off = (size_t)bh * T * D;
-    const int R = c_k / 2;
-    for (int idx = tid; idx < 8 * TW; idx += kProThreads) {
-        const int ip = idx / TW, jj = idx % TW;
-        th[idx] = (ip < c_q && jj < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jj] : 0.f;
+    const int shift = RT - c_k / 2;            // real tap jj sits at padded index jj + shift
+    for (int idx = tid; idx < 8 * CK; idx += kProThreads) {
+        const int ip = idx / CK, jj = idx % CK - shift;
+        thp[idx] = (ip < c_q && jj >= 0 && jj < c_k) ? w_kq[((size_t)h * c_q + ip) * c_k + jj] : 0.f;
     }
-    __syncthreads();
     // Row copies in shared memory, all in flight at once (cp.async): q rows
     // [j0-7, j0+64) and k rows [j0-6, j0+78), zero outside [0, T); rows are
     // padded by 16 bytes so that threads on different rows hit different banks,
@@ -376,7 +409,8 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
     }
     __shared__ float red[8];
     int eq = range_exponent(block_max(mq, red));
-    if (eq < 0) { if (tid == 0) atomicOr(&g_fused_error, kErrRange); eq = 0; }
+    if (eq != 0 && tid == 0 && half == 0) atomicOr(&g_fused_error, kErrRange);   // see the fold
+    if (eq < 0) eq = 0;
     if (tid == 0 && half == 0) qexp[(size_t)bh * nqb + qblk] = eq;
     const float qsc = ldexpf(1.f, -eq);       // exact: a power of two
     // (b) permuted query rows of the 128-row block jb0 = j0 - 64*half: atom a,
@@ -444,52 +478,32 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
                     const int dl = kr - rr + 1;
                     if (rr < QR && dl >= 1 && dl <= kCorrW - 2) {
                         const int r = j0 - kProQLo + rr;
-                        fs[rr * kCorrW + dl - 1] =
+                        fs[rr * kFs + dl - 1] =
                             (r >= 0 && dl <= Dm && r + dl < T) ? acc[j][x] * scale : 0.f;
                     }
                 }
         }
     }
     __syncthreads();
-    // taps indexed by s = e + delta: ts[i'][s] = theta[i'][i' + R - s]
-    __shared__ float ts[8 * 32];
-    for (int idx = tid; idx < 8 * 32; idx += kProThreads) {
-        const int ip = idx / 32, jj = ip + R - idx % 32;
-        ts[idx] = (ip < c_q && jj >= 0 && jj < c_k) ? th[ip * TW + jj] : 0.f;
-    }
-    __syncthreads();
-    // (d) correction table: thread = one row i and 8 of its 16 entries e.
-    //     corr[i][e] = sum_{i'} sum_{delta} ts[i'][e + delta] F[i - i'][delta];
-    //     taps with delta < 1 or jj outside [0, c_k) are zero in ts, F rows
-    //     before the sequence are zero, so e >= D_m comes out zero too.
-    if (tid < 2 * kAuxRows) {
-        constexpr int EH = kCorrW / 2;
-        const int ir = tid >> 1, e0 = (tid & 1) * EH, i = j0 + ir;
-        // entries e, e+1 share F[.][delta]: one packed f32x2 FMA for both
-        unsigned long long acc[EH / 2];
-#pragma unroll
-        for (int p = 0; p < EH / 2; ++p) acc[p] = 0ull;
-        for (int ip = 0; ip < c_q; ++ip) {
-            const float *frow = fs + (ir + kProQLo - ip) * kCorrW;   // F row i - i'
-            const float *trow = ts + ip * 32 + e0;
-            float t[EH + kCorrW - 1];
-#pragma unroll
-            for (int x = 1; x < EH + kCorrW - 1; ++x) t[x] = trow[x];
-#pragma unroll
-            for (int dl = 1; dl <= kCorrW - 2; ++dl) {
-                const float f = dl > exact * ip ? frow[dl - 1] : 0.f;
-                const unsigned long long ff = f2_pack(f, f);
-#pragma unroll
-                for (int p = 0; p < EH / 2; ++p)
-                    acc[p] = f2_fma(f2_pack(t[2 * p + dl], t[2 * p + 1 + dl]), ff, acc[p]);
-            }
+    // (d) correction rows: thread = one row i (tid % 64) and the 4 entries
+    //     e = 4g .. 4g+3, g = tid / 64 (the same in a whole warp):
+    //     corr[i][e] = sum over taps (i', jj) of thp[i'][jj] F[i - i'][delta],
+    //     delta = i' + RT - jj - e.  With the taps padded and centred at RT
+    //     every delta is a compile-time constant, so only the terms with
+    //     1 <= delta <= 14 are emitted (F is zero past D_m and before the
+    //     sequence; padded taps are zero).  Under the exact mask the terms
+    //     with delta <= i' are dropped.
+    {
+        const int ir = tid % kAuxRows, g = tid / kAuxRows;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        switch (g) {
+            case 0: corr_terms<CK, 0>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
+            case 1: corr_terms<CK, 4>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
+            case 2: corr_terms<CK, 8>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
+            default: corr_terms<CK, 12>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
         }
-        float4 *dst = (float4 *)(corr + ((size_t)bh * Tp + i) * kCorrW + e0);
-#pragma unroll
-        for (int u = 0; u < EH / 4; ++u) {
-            const float2 lo = f2_unpack(acc[2 * u]), hi = f2_unpack(acc[2 * u + 1]);
-            dst[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
-        }
+        *(float4 *)(corr + ((size_t)bh * Tp + j0 + ir) * kCorrW + 4 * g) =
+            make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
 }
 
@@ -533,8 +547,8 @@ k_fold(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
         fold_keys_block<D, CK>(blk, bh, k, w_kq, kf, sexp + (size_t)gridDim.x / 3, T, Tp, H, nqb,
                                c_q, c_k, scale);
     else
-        fold_aux_block<D>(2 * blk + role / 2, bh, q, k, w_kq, qp, corr, sexp, T, Tp, H, nqb, c_q,
-                          c_k, scale, exact);
+        fold_aux_block<D, CK>(2 * blk + role / 2, bh, q, k, w_kq, qp, corr, sexp, T, Tp, H, nqb,
+                              c_q, c_k, scale, exact);
 }
 
 // ------------------------------------------------------------ main kernel

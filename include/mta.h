@@ -68,8 +68,8 @@ typedef enum {
     MTA_ERR_WORKSPACE = -4,      /* workspace smaller than the *_workspace_size query */
     MTA_ERR_CUDA = -5,           /* a CUDA runtime call failed */
     MTA_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait expired */
-    MTA_ERR_RANGE = -7           /* the fused path met a non-finite input or produced a
-                                    non-finite output */
+    MTA_ERR_RANGE = -7           /* the fused path met inputs outside its accuracy domain
+                                    (beyond fp16, or non-finite): see mta_forward */
 } mta_status;
 
 typedef enum { MTA_F32 = 0, MTA_BF16 = 1 } mta_dtype;
@@ -118,15 +118,18 @@ MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
 /* The MTA forward S1..S9 above, out = depth_scale * GN(...), written to out.
  * The fused path computes the folded logits on tensor cores with fp16
  * operands (q and the folded keys) and P V with bf16 operands, both with fp32
- * accumulation; the materialised path computes in fp32.  Any finite bf16
- * input is in the fused path's domain: a 128-row block of queries or of
- * folded keys whose magnitude bound exceeds 2^14 is scaled by a power of two
- * before the fp16 rounding and its logits scaled back exactly.  Values more
- * than 2^28 times smaller than their block's largest then fall into fp16's
- * subnormal range, with an absolute error up to 2^(e-25) for the block's
- * scale 2^e (for one query of 2e6 among N(0,1) values, e = 7: 4e-6).  A
- * non-finite q, k or v (anything that makes an output non-finite) makes the
- * call's next mta_sync_status() report MTA_ERR_RANGE.
+ * accumulation; the materialised path computes in fp32.  The fused path
+ * subtracts, on the tiles next to the diagonal, the future terms that Mask_0
+ * removes; those terms were computed with fp16 operands, so the logits there
+ * carry an absolute error of about 2^-11 |theta| |q| |k| / sqrt(d) per future
+ * term (negligible for activations of order 10, ruinous for order 1e4).  A
+ * 128-row block of queries or of folded keys beyond the fp16 range is scaled
+ * by a power of two before the rounding and its logits scaled back exactly,
+ * so the output stays finite, and the call's next mta_sync_status() reports
+ * MTA_ERR_RANGE: such inputs are outside the fused path's accuracy domain and
+ * mta_forward_unfused (fp32 throughout) is the path for them.  A non-finite
+ * q, k or v, or anything that makes an output non-finite, is reported the
+ * same way.
  * The workspace is scratch owned by the caller for the duration of the
  * enqueued work; its contents on entry are ignored. */
 MTA_API mta_status mta_forward(const mta_shape *shape, const void *q, const void *k, const void *v,
@@ -345,7 +348,7 @@ MTA_API const char *mta_backward_kernel_name(const mta_shape *shape, int index);
 
 /* Synchronises `stream`, then reports (and clears) the device error flags:
  * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
- * the fused path met a non-finite input, MTA_ERR_CUDA if the
+ * the fused path met inputs beyond fp16 or non-finite ones, MTA_ERR_CUDA if the
  * synchronisation itself failed, MTA_OK otherwise.  The flags are one word per
  * device, shared by every stream and caller of the library on that device:
  * the word is read and cleared in one atomic step (a small kernel on
