@@ -225,6 +225,9 @@ def kernel_units(name, w, comp=None):
         "k_softmax_mix": ("hbm", logits * 8, "B"),            # read C, write A_new (fp32)
         "k_head_mix": ("hbm", logits * 8, "B"),               # read and write one fp32 map
         "k_pv_groupnorm": ("alu", logits * 2 * w.d, "FLOP"),
+        # tensor-core forms: write (read) the fp32 map, read q and k (v, write out)
+        "k_logits_tc": ("hbm", logits * 4 + w.B * w.H * w.T * w.d * 2 * io_bytes, "B"),
+        "k_pv_groupnorm_tc": ("hbm", logits * 4 + w.B * w.H * w.T * w.d * 2 * io_bytes, "B"),
         # the prologue: read k, write the c_q folded-key copies (fp16); read q
         # and k, write the permuted q (fp16) and the 16-entry correction rows
         "k_fold": ("hbm", w.B * w.H * w.T * (w.d * 2 * (1 + w.c_q) + w.d * 2 * 3 + 64), "B"),

@@ -286,8 +286,8 @@ def mta_forward_gated(q, k, v, w_kq, w_head, gn_weight, gn_bias, gate, out=None,
 
 def mta_forward_unfused(q, k, v, w_kq, w_head, gn_weight, gn_bias, depth_scale, out=None,
                         workspace=None, stream=None, gn_eps=1e-5, check=False):
-    """MTA forward with materialised T x T maps (fp32 arithmetic); check as
-    for mta_forward."""
+    """MTA forward with materialised fp32 T x T maps (tensor-core Q K^T and A V
+    for bf16 I/O at d = 64 or 128); check as for mta_forward."""
     return _forward("mta_forward_unfused", mta_unfused_workspace_size, q, k, v, w_kq, w_head,
                     gn_weight, gn_bias, depth_scale, out, workspace, stream, gn_eps,
                     check=check)

@@ -255,7 +255,7 @@ int mta_composed_kernel_count(const mta_shape *s, const mta_composition *c)
     if (is_default_composition(c) && path_of(*s, 0, 1) == MTA_PATH_FUSED_TC)
         return mta::fused_kernel_count(*s);
     const char *names[mta::kMaxChainKernels];
-    return mta::unfused_chain(chain_args(c), names);
+    return mta::unfused_chain(*s, chain_args(c), names);
 }
 
 const char *mta_composed_kernel_name(const mta_shape *s, const mta_composition *c, int index)
@@ -265,7 +265,7 @@ const char *mta_composed_kernel_name(const mta_shape *s, const mta_composition *
     if (is_default_composition(c) && path_of(*s, 0, 1) == MTA_PATH_FUSED_TC)
         return mta::fused_kernel_name(*s, index);
     const char *names[mta::kMaxChainKernels];
-    const int n = mta::unfused_chain(chain_args(c), names);
+    const int n = mta::unfused_chain(*s, chain_args(c), names);
     return index < n ? names[index] : nullptr;
 }
 
@@ -321,7 +321,7 @@ const char *mta_kernel_name(const mta_shape *s, int unfused, int index)
     switch (path_of(*s, unfused, 0)) {
         case MTA_PATH_FUSED_TC: return mta::fused_kernel_name(*s, index);
         case MTA_PATH_FUSED_F32: return "k_mta_fused_f32";
-        default: return mta::kUnfusedKernelNames[index];
+        default: return mta::unfused_kernel_name(*s, index);
     }
 }
 
@@ -358,7 +358,7 @@ int mta_backward_kernel_count(const mta_shape *s)
 const char *mta_backward_kernel_name(const mta_shape *s, int index)
 {
     if (check_shape(s) != MTA_OK || index < 0 || index >= mta::kBackwardKernels) return nullptr;
-    return mta::kBackwardKernelNames[index];
+    return mta::backward_kernel_name(*s, index);
 }
 
 mta_status mta_backward_traced(const mta_shape *s, const void *q, const void *k, const void *v,
@@ -411,8 +411,10 @@ mta_status mta_selftest_wait_timeout(long long budget_cycles, void *stream)
 mta_status mta_sync_status(void *stream)
 {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MTA_ERR_CUDA;
-    const unsigned int err = mta::fused_take_error((cudaStream_t)stream);
-    if (err == ~0u) return MTA_ERR_CUDA;
+    const unsigned int fused = mta::fused_take_error((cudaStream_t)stream);
+    const unsigned int chain = mta::chain_take_error((cudaStream_t)stream);
+    if (fused == ~0u || chain == ~0u) return MTA_ERR_CUDA;
+    const unsigned int err = fused | chain;
     if (err & 1u) return MTA_ERR_DEVICE_TIMEOUT;
     if (err & 2u) return MTA_ERR_RANGE;
     return MTA_OK;

@@ -590,10 +590,16 @@ void reduce(const float *part, float *out, int n_outer, int n_mid, int n_inner, 
 
 }  // namespace
 
-const char *const kBackwardKernelNames[kBackwardKernels] = {
-    "k_logits", "k_conv", "k_softmax_mix", "k_head_mix", "k_causal_mm", "k_gn_bwd",
-    "k_causal_mm", "k_logits", "k_mix_softmax_bwd", "k_conv_adj", "k_dtheta", "k_causal_mm",
-    "k_causal_mm", "k_reduce"};
+const char *backward_kernel_name(const mta_shape &s, int index)
+{
+    static const char *const names[kBackwardKernels] = {
+        "k_logits", "k_conv", "k_softmax_mix", "k_head_mix", "k_causal_mm", "k_gn_bwd",
+        "k_causal_mm", "k_logits", "k_mix_softmax_bwd", "k_conv_adj", "k_dtheta", "k_causal_mm",
+        "k_causal_mm", "k_reduce"};
+    if (index < 0 || index >= kBackwardKernels) return nullptr;
+    // the recomputed logits take the chain's kernel for the shape
+    return index == 0 ? unfused_kernel_name(s, 0) : names[index];
+}
 
 size_t backward_workspace_bytes(const mta_shape &s) { return bwd_layout(s).total; }
 
@@ -610,7 +616,8 @@ mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const Backw
     mta_status rc = MTA_OK;
     int n = 0;
     // forward recompute
-    tr.before(n, st); logits(s, a.q, a.k, m1, 0, st); tr.after(n++, st);
+    tr.before(n, st); rc = logits(s, a.q, a.k, m1, 0, st); tr.after(n++, st);
+    if (rc != MTA_OK) return rc;
     tr.before(n, st); launch_conv(s, m1, m2, a.w_kq, 0, 1, st); tr.after(n++, st);
     tr.before(n, st); rc = softmax_mix(s, m2, m3, nullptr, 0, st); tr.after(n++, st);
     if (rc != MTA_OK) return rc;

@@ -53,8 +53,8 @@ inline size_t bh_tt(const mta_shape &s) {
 //  softmax_mix   softmax rows of map1 and the Eq. (7) head mix (w_head null:
 //                the identity) into dst
 //  head_mix      Eq. (7) without a softmax
-void logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
-            cudaStream_t st);
+mta_status logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
+                  cudaStream_t st);
 void logits_f32_io(const mta_shape &s, const float *a, const void *b, float scale, float *map,
                    cudaStream_t st);
 void launch_conv(const mta_shape &s, const float *src, float *dst, const float *w_kq, int band,
@@ -65,11 +65,25 @@ mta_status head_mix(const mta_shape &s, const float *src, float *dst, const floa
                     cudaStream_t st);
 size_t unfused_workspace_bytes(const mta_shape &s);
 constexpr int kUnfusedKernels = 4;
-extern const char *const kUnfusedKernelNames[kUnfusedKernels];
+// Kernel names of the default chain for shape s (tensor-core logits and
+// A V for bf16 I/O at d = 64 or 128, CUDA-core fp32 otherwise).
+const char *unfused_kernel_name(const mta_shape &s, int index);
 // Launch sequence of launch_unfused for the steps a names (at most
 // kMaxChainKernels); fills names[] in launch order and returns the count.
 constexpr int kMaxChainKernels = 7;
-int unfused_chain(const ForwardArgs &a, const char **names);
+int unfused_chain(const mta_shape &s, const ForwardArgs &a, const char **names);
+// Tensor-core kernels of the chain (unfused_tc.cu), bf16 I/O with d = 64 or
+// 128 (chain_tc_supported): logits_tc as `logits`, pv_groupnorm_tc the
+// A V + GroupNorm + output-scale step into a.out.
+bool chain_tc_supported(const mta_shape &s);
+mta_status logits_tc(const mta_shape &s, const void *q, const void *k, float *map0, int band,
+                     cudaStream_t st);
+mta_status pv_groupnorm_tc(const mta_shape &s, const float *amap, const ForwardArgs &a,
+                           cudaStream_t st);
+// Reads and clears, in one atomic step on stream `st`, the device error word
+// of these kernels (bit 0: a bounded wait expired), then synchronises `st`;
+// ~0u when a CUDA call failed.
+unsigned int chain_take_error(cudaStream_t st);
 mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cudaStream_t st,
                           const Trace &tr);
 mta_status launch_debug_attention(const mta_shape &s, const void *q, const void *k,
@@ -87,7 +101,7 @@ struct BackwardArgs {
     float *dgate;              // [H], with a gate only
 };
 constexpr int kBackwardKernels = 14;
-extern const char *const kBackwardKernelNames[kBackwardKernels];
+const char *backward_kernel_name(const mta_shape &s, int index);
 size_t backward_workspace_bytes(const mta_shape &s);
 mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const BackwardArgs &g,
                            void *ws, cudaStream_t st, const Trace &tr);

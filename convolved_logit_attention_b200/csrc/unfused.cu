@@ -1,7 +1,9 @@
 // Materialised MTA forward: the T x T maps of one call live in the workspace.
 //
 // One kernel per group of steps of "Multi-Token Attention -- Paper Graph",
-// section 3.4, all arithmetic in fp32 on CUDA cores:
+// section 3.4, all arithmetic in fp32 on CUDA cores (for bf16 I/O at d = 64
+// or 128, k_logits and k_pv_groupnorm give way to the tcgen05 kernels of
+// unfused_tc.cu):
 //   k_logits        S1 + S2   A0 = Mask_0(Q K^T / sqrt(d))      -> map0
 //   k_conv          S3 (+S4)  C = Conv2d_theta(A0), Eq. (4)/(5) -> map1
 //   k_softmax_mix   S5 + S6   softmax rows, post-softmax head mix (Eq. (7))
@@ -541,14 +543,16 @@ void launch_conv(const mta_shape &s, const float *src, float *dst, const float *
     }
 }
 
-void logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
-            cudaStream_t st)
+mta_status logits(const mta_shape &s, const void *q, const void *k, float *map0, int band,
+                  cudaStream_t st)
 {
+    if (chain_tc_supported(s)) return logits_tc(s, q, k, map0, band, st);
     const float scale = 1.0f / sqrtf((float)s.d);
     if (s.io == MTA_BF16)
         launch_logits<__nv_bfloat16, __nv_bfloat16>(s, q, k, map0, scale, band, st);
     else
         launch_logits<float, float>(s, q, k, map0, scale, band, st);
+    return MTA_OK;
 }
 
 void logits_f32_io(const mta_shape &s, const float *a, const void *b, float scale, float *map,
@@ -562,8 +566,10 @@ void logits_f32_io(const mta_shape &s, const float *a, const void *b, float scal
 
 namespace {
 
-void pv_groupnorm(const mta_shape &s, const float *amap, const ForwardArgs &a, cudaStream_t st)
+mta_status pv_groupnorm(const mta_shape &s, const float *amap, const ForwardArgs &a,
+                        cudaStream_t st)
 {
+    if (chain_tc_supported(s)) return pv_groupnorm_tc(s, amap, a, st);
     dim3 g4((s.T + kPvRows - 1) / kPvRows, s.B * s.H);
     if (s.io == MTA_BF16)
         k_pv_groupnorm<__nv_bfloat16><<<g4, 256, 0, st>>>(
@@ -573,25 +579,33 @@ void pv_groupnorm(const mta_shape &s, const float *amap, const ForwardArgs &a, c
         k_pv_groupnorm<float><<<g4, 256, 0, st>>>(amap, (const float *)a.v, a.gn_weight,
                                                   a.gn_bias, a.depth_scale, a.gate, s.gn_eps,
                                                   (float *)a.out, s.T, s.H, s.d);
+    return MTA_OK;
 }
 
 }  // namespace
 
-const char *const kUnfusedKernelNames[kUnfusedKernels] = {"k_logits", "k_conv",
-                                                         "k_softmax_mix", "k_pv_groupnorm"};
+const char *unfused_kernel_name(const mta_shape &s, int index)
+{
+    static const char *const fp32[kUnfusedKernels] = {"k_logits", "k_conv", "k_softmax_mix",
+                                                      "k_pv_groupnorm"};
+    static const char *const tc[kUnfusedKernels] = {"k_logits_tc", "k_conv", "k_softmax_mix",
+                                                    "k_pv_groupnorm_tc"};
+    if (index < 0 || index >= kUnfusedKernels) return nullptr;
+    return chain_tc_supported(s) ? tc[index] : fp32[index];
+}
 
 size_t unfused_workspace_bytes(const mta_shape &s) { return 2 * bh_tt(s) * sizeof(float); }
 
-int unfused_chain(const ForwardArgs &a, const char **names)
+int unfused_chain(const mta_shape &s, const ForwardArgs &a, const char **names)
 {
     int n = 0;
-    names[n++] = "k_logits";
+    names[n++] = unfused_kernel_name(s, 0);
     if (a.w_kq || a.w_kq_3d) names[n++] = "k_conv";
     if (a.w_head_pre) names[n++] = "k_head_mix";
     names[n++] = "k_softmax_mix";
     if (a.w_kq_post) names[n++] = "k_conv";
     if (a.w_head_post) names[n++] = "k_head_mix";
-    names[n++] = "k_pv_groupnorm";
+    names[n++] = unfused_kernel_name(s, 3);
     return n;
 }
 
@@ -608,8 +622,9 @@ mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     int cur = 0, launch = 0;
     mta_status rc = MTA_OK;
     tr.before(launch, st);
-    logits(s, a.q, a.k, maps[0], band, st);
+    rc = logits(s, a.q, a.k, maps[0], band, st);
     tr.after(launch++, st);
+    if (rc != MTA_OK) return rc;
     if (w_first) {
         tr.before(launch, st);
         launch_conv(s, maps[cur], maps[cur ^ 1], w_first, band, a.w_kq_3d ? s.c_h : 1, st);
@@ -642,8 +657,9 @@ mta_status launch_unfused(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         cur ^= 1;
     }
     tr.before(launch, st);
-    pv_groupnorm(s, maps[cur], a, st);
+    rc = pv_groupnorm(s, maps[cur], a, st);
     tr.after(launch, st);
+    if (rc != MTA_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
 
@@ -653,9 +669,10 @@ mta_status launch_debug_attention(const mta_shape &s, const void *q, const void 
 {
     float *map0 = (float *)ws;
     float *map1 = map0 + bh_tt(s);
-    logits(s, q, k, map0, 0, st);
+    mta_status rc = logits(s, q, k, map0, 0, st);
+    if (rc != MTA_OK) return rc;
     launch_conv(s, map0, map1, w_kq, 0, 1, st);
-    mta_status rc = softmax_mix(s, map1, attn, w_head, stage == 0 ? 1 : 2, st);
+    rc = softmax_mix(s, map1, attn, w_head, stage == 0 ? 1 : 2, st);
     if (rc != MTA_OK) return rc;
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }

@@ -118,7 +118,10 @@ MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
 /* The MTA forward S1..S9 above, out = depth_scale * GN(...), written to out.
  * The fused path computes the folded logits on tensor cores with fp16
  * operands (q and the folded keys) and P V with bf16 operands, both with fp32
- * accumulation; the materialised path computes in fp32.  The fused path
+ * accumulation.  The materialised path keeps fp32 maps; for bf16 I/O at
+ * d = 64 or 128 its Q K^T runs on tensor cores from the bf16 inputs (exact
+ * products, fp32 accumulation) and its A V with the attention weights rounded
+ * to bf16, otherwise both are fp32 CUDA-core products.  The fused path
  * subtracts, on the tiles next to the diagonal, the future terms that Mask_0
  * removes; those terms were computed with fp16 operands, so the logits there
  * carry an absolute error of about 2^-11 |theta| |q| |k| / sqrt(d) per future
@@ -127,7 +130,8 @@ MTA_API size_t mta_unfused_workspace_size(const mta_shape *shape);
  * by a power of two before the rounding and its logits scaled back exactly,
  * so the output stays finite, and the call's next mta_sync_status() reports
  * MTA_ERR_RANGE: such inputs are outside the fused path's accuracy domain and
- * mta_forward_unfused (fp32 throughout) is the path for them.  A non-finite
+ * mta_forward_unfused (fp32 logits, and bf16 operands, which have the fp32
+ * exponent range) is the path for them.  A non-finite
  * q, k or v, or anything that makes an output non-finite, is reported the
  * same way.
  * The workspace is scratch owned by the caller for the duration of the
@@ -349,11 +353,12 @@ MTA_API const char *mta_backward_kernel_name(const mta_shape *shape, int index);
 /* Synchronises `stream`, then reports (and clears) the device error flags:
  * MTA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait expired, MTA_ERR_RANGE if
  * the fused path met inputs beyond fp16 or non-finite ones, MTA_ERR_CUDA if the
- * synchronisation itself failed, MTA_OK otherwise.  The flags are one word per
- * device, shared by every stream and caller of the library on that device:
- * the word is read and cleared in one atomic step (a small kernel on
- * `stream`), so no raised flag is lost, but a call reports flags raised by
- * any work on the device since the previous report. */
+ * synchronisation itself failed, MTA_OK otherwise.  The flags are two words
+ * per device (one for the fused kernels, one for the materialised chain's
+ * tensor-core kernels), shared by every stream and caller of the library on
+ * that device: each word is read and cleared in one atomic step (a small
+ * kernel on `stream`), so no raised flag is lost, but a call reports flags
+ * raised by any work on the device since the previous report. */
 MTA_API mta_status mta_sync_status(void *stream);
 
 #ifdef __cplusplus

@@ -133,8 +133,21 @@ def test_forward_path_selection(L, kw, path):
     elif path == 2:  # one fused fp32 kernel, no workspace
         assert names == ["k_mta_fused_f32"]
         assert mta.mta_workspace_size(s) == 0
-    else:           # the four materialised kernels
-        assert names == ["k_logits", "k_conv", "k_softmax_mix", "k_pv_groupnorm"]
+    else:           # the four materialised kernels; bf16 at d = 64 or 128 takes the
+        # tensor-core logits and A V kernels
+        tc = kw.get("io", "bf16") == "bf16" and kw["d"] in (64, 128)
+        assert names == (["k_logits_tc", "k_conv", "k_softmax_mix", "k_pv_groupnorm_tc"] if tc
+                         else ["k_logits", "k_conv", "k_softmax_mix", "k_pv_groupnorm"])
+
+
+def test_backward_launch_names_follow_the_chain(L):
+    # the recomputed logits take the chain's kernel; dA = dO V^T (fp32 dO)
+    # always runs on CUDA cores
+    for kw, first in ((dict(d=128), "k_logits_tc"), (dict(d=32), "k_logits"),
+                      (dict(d=64, io="f32"), "k_logits")):
+        names = mta.mta_backward_kernel_names(shape(**kw))
+        assert len(names) == 14 and names[0] == first and names[7] == "k_logits"
+        assert names.count("k_causal_mm") == 4
 
 
 def test_selftest_rejects_bad_budget(L):
@@ -183,6 +196,12 @@ def test_composed_launch_sequences_and_workspace(L):
         mta.mta_workspace_size(fused)
     assert L.mta_composed_workspace_size(ctypes.byref(fused), None) == 0
     assert L.mta_composed_kernel_name(ctypes.byref(s), ctypes.byref(C(a, a, a, a)), 6) is None
+    # bf16 at d = 64: the same chain with the tensor-core logits and A V kernels
+    s64 = shape(d=64)
+    assert mta.mta_composed_kernel_names(s64, C(a, a, a, a)) == \
+        ["k_logits_tc", "k_conv", "k_softmax_mix", "k_conv", "k_head_mix", "k_pv_groupnorm_tc"]
+    assert mta.mta_composed_kernel_names(shape(d=64, io="f32"), C(a, a, a, a)) == \
+        ["k_logits", "k_conv", "k_softmax_mix", "k_conv", "k_head_mix", "k_pv_groupnorm"]
 
 
 def test_composed_argument_checks(L):

@@ -92,3 +92,24 @@ def test_gated_output_full_size_every_element():
     ref = oracle.forward(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
                          x["gn_bias"], 0.0, gn_eps=x["gn_eps"], gate=gate)
     assert_every_element(got, ref, w.H, w.d, "longctx_4k gated")
+
+
+def test_materialised_path_full_size_every_element():
+    """The materialised chain (mta_forward_unfused) on the T = 4096 workload,
+    every element: its logits and A V run as tcgen05 tiles for bf16 I/O,
+    with the fp32 maps of the chain in between."""
+    w = WORKLOADS["longctx_4k"]
+    x = make_inputs(w)
+    d = _device(x)
+    shape = mta.shape_of(d["q"], d["w_kq"], d["w_head"], x["gn_eps"])
+    names = [mta.mta_kernel_name(shape, i, unfused=1) for i in range(4)]
+    assert names == ["k_logits_tc", "k_conv", "k_softmax_mix", "k_pv_groupnorm_tc"]
+    out = mta.mta_forward_unfused(d["q"], d["k"], d["v"], d["w_kq"], d["w_head"], d["gn_weight"],
+                                  d["gn_bias"], x["depth_scale"], gn_eps=x["gn_eps"])
+    mta.mta_sync_status()
+    got = out.float().cpu().numpy().astype(np.float64)
+    del d, out
+    torch.cuda.empty_cache()
+    ref = oracle.forward(x["q"], x["k"], x["v"], x["w_kq"], x["w_head"], x["gn_weight"],
+                         x["gn_bias"], x["depth_scale"], gn_eps=x["gn_eps"])
+    assert_every_element(got, ref, w.H, w.d, "longctx_4k materialised")

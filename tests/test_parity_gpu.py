@@ -99,6 +99,8 @@ RAGGED = [
     (1, 2, 511, 64, 4, 15, 2, "bf16"),
     (2, 4, 384, 128, 6, 11, 4, "bf16"),     # output heads split over two work items
     (1, 8, 200, 64, 3, 5, 8, "bf16"),
+    (1, 2, 1, 128, 6, 11, 2, "bf16"),       # one token on the tensor-core chain
+    (1, 2, 3, 64, 4, 15, 2, "bf16"),        # rows shorter than a 16-byte store
 ]
 
 
