@@ -236,6 +236,9 @@ def kernel_units(name, w, comp=None):
         "k_mix_groupnorm": ("hbm", w.B * w.T * w.H * w.d * (2 * w.c_h + io_bytes), "B"),
         # backward: causal products of a map with a [T, d] operand, 2d FLOP per live logit
         "k_causal_mm": ("alu", logits * 2 * w.d, "FLOP"),
+        # the same products and dA = dO V^T as 3xTF32 MMAs: read (or write) the
+        # fp32 map, read the [T, d] operand, write (or read) an fp32 [T, d] array
+        "k_mm_tf32": ("hbm", logits * 4 + w.B * w.H * w.T * w.d * (4 + 4), "B"),
         # read O and dout, write dO (fp32)
         "k_gn_bwd": ("hbm", w.B * w.H * w.T * w.d * (4 + io_bytes + 4), "B"),
         # read dA and P twice, write dC (fp32 maps)

@@ -571,9 +571,10 @@ void conv_adj_and_dtheta(const mta_shape &s, const float *dc, const float *a0, f
 }
 
 template <bool kTrans>
-void causal_mm(const mta_shape &s, const float *map, const void *x, bool x_io, float *out,
-               float scale, cudaStream_t st)
+mta_status causal_mm(const mta_shape &s, const float *map, const void *x, bool x_io, float *out,
+                     float scale, cudaStream_t st)
 {
+    if (mm_tf32_supported(s)) return causal_mm_tf32(s, kTrans, map, x, x_io, out, scale, st);
     dim3 g((s.T + kMmRows - 1) / kMmRows, s.B * s.H);
     if (x_io && s.io == MTA_BF16)
         k_causal_mm<__nv_bfloat16, kTrans><<<g, 256, 0, st>>>(map, (const __nv_bfloat16 *)x, out,
@@ -581,6 +582,7 @@ void causal_mm(const mta_shape &s, const float *map, const void *x, bool x_io, f
     else
         k_causal_mm<float, kTrans><<<g, 256, 0, st>>>(map, (const float *)x, out, s.T, s.d,
                                                       scale);
+    return MTA_OK;
 }
 
 void reduce(const float *part, float *out, int n_outer, int n_mid, int n_inner, cudaStream_t st)
@@ -597,8 +599,13 @@ const char *backward_kernel_name(const mta_shape &s, int index)
         "k_causal_mm", "k_logits", "k_mix_softmax_bwd", "k_conv_adj", "k_dtheta", "k_causal_mm",
         "k_causal_mm", "k_reduce"};
     if (index < 0 || index >= kBackwardKernels) return nullptr;
-    // the recomputed logits take the chain's kernel for the shape
-    return index == 0 ? unfused_kernel_name(s, 0) : names[index];
+    // the recomputed logits take the chain's kernel for the shape; at d = 64
+    // or 128 the fp32 products (A V, dV, dA, dQ, dK) run as 3xTF32 MMAs
+    if (index == 0) return unfused_kernel_name(s, 0);
+    if (mm_tf32_supported(s) && (index == 4 || index == 6 || index == 7 || index == 11 ||
+                                 index == 12))
+        return "k_mm_tf32";
+    return names[index];
 }
 
 size_t backward_workspace_bytes(const mta_shape &s) { return bwd_layout(s).total; }
@@ -623,7 +630,8 @@ mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const Backw
     if (rc != MTA_OK) return rc;
     tr.before(n, st); rc = head_mix(s, m3, m2, a.w_head, st); tr.after(n++, st);
     if (rc != MTA_OK) return rc;
-    tr.before(n, st); causal_mm<false>(s, m2, a.v, true, od, 1.f, st); tr.after(n++, st);
+    tr.before(n, st); rc = causal_mm<false>(s, m2, a.v, true, od, 1.f, st); tr.after(n++, st);
+    if (rc != MTA_OK) return rc;
     // GroupNorm and output scale
     tr.before(n, st);
     {
@@ -639,8 +647,13 @@ mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const Backw
     }
     tr.after(n++, st);
     // dV = A^T dO, then dA = dO V^T over the A map
-    tr.before(n, st); causal_mm<true>(s, m2, od, false, g.dv, 1.f, st); tr.after(n++, st);
-    tr.before(n, st); logits_f32_io(s, od, a.v, 1.f, m2, st); tr.after(n++, st);
+    tr.before(n, st); rc = causal_mm<true>(s, m2, od, false, g.dv, 1.f, st); tr.after(n++, st);
+    if (rc != MTA_OK) return rc;
+    tr.before(n, st);
+    if (mm_tf32_supported(s)) rc = logits_f32_tf32(s, od, a.v, 1.f, m2, st);
+    else logits_f32_io(s, od, a.v, 1.f, m2, st);
+    tr.after(n++, st);
+    if (rc != MTA_OK) return rc;
     // head mix and softmax: dA -> dC in M2, dw partials
     tr.before(n, st); rc = mix_softmax_bwd(s, m2, m3, a.w_head, pw, st); tr.after(n++, st);
     if (rc != MTA_OK) return rc;
@@ -648,8 +661,10 @@ mta_status launch_backward(const mta_shape &s, const ForwardArgs &a, const Backw
     conv_adj_and_dtheta(s, m2, m1, m3, pth, a.w_kq, st, tr, n);
     n += 2;
     // dQ = dA^ K / sqrt d, dK = dA^T Q / sqrt d
-    tr.before(n, st); causal_mm<false>(s, m3, a.k, true, g.dq, rsd, st); tr.after(n++, st);
-    tr.before(n, st); causal_mm<true>(s, m3, a.q, true, g.dk, rsd, st); tr.after(n++, st);
+    tr.before(n, st); rc = causal_mm<false>(s, m3, a.k, true, g.dq, rsd, st); tr.after(n++, st);
+    if (rc != MTA_OK) return rc;
+    tr.before(n, st); rc = causal_mm<true>(s, m3, a.q, true, g.dk, rsd, st); tr.after(n++, st);
+    if (rc != MTA_OK) return rc;
     // the parameter gradients
     tr.before(n, st);
     const int G = s.H / s.c_h;

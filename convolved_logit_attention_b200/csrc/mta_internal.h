@@ -80,6 +80,19 @@ mta_status logits_tc(const mta_shape &s, const void *q, const void *k, float *ma
                      cudaStream_t st);
 mta_status pv_groupnorm_tc(const mta_shape &s, const float *amap, const ForwardArgs &a,
                            cudaStream_t st);
+// fp32 products of the backward pass on tensor cores (3xTF32, the accuracy of
+// an fp32 dot product), for d = 64 or 128 (mm_tf32_supported):
+//  causal_mm_tf32  out[bh][r][:] = scale * sum over c of M[r][c] X[c][:], with
+//                  trans false: M = map rows, c <= r; trans true: M = map^T,
+//                  c >= r.  X is [B*H][T][d], of the I/O type when x_io, else
+//                  fp32; out fp32 [B*H][T][d]
+//  logits_f32_tf32 map[bh][i][j] = scale * a_i . b_j for j <= i, 0 above (a fp32
+//                  [B*H][T][d], b of the I/O type)
+bool mm_tf32_supported(const mta_shape &s);
+mta_status causal_mm_tf32(const mta_shape &s, bool trans, const float *map, const void *x,
+                          bool x_io, float *out, float scale, cudaStream_t st);
+mta_status logits_f32_tf32(const mta_shape &s, const float *a, const void *b, float scale,
+                           float *map, cudaStream_t st);
 // Reads and clears, in one atomic step on stream `st`, the device error word
 // of these kernels (bit 0: a bounded wait expired), then synchronises `st`;
 // ~0u when a CUDA call failed.

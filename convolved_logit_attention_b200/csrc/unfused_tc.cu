@@ -360,6 +360,366 @@ k_pv_groupnorm_tc(const float *__restrict__ amap, const __grid_constant__ CUtens
     }
 }
 
+// ----------------------------------------------------------------------------
+// fp32 products on tensor cores (3xTF32) for the backward pass.
+//
+// A TF32 operand keeps sign, exponent and the top 10 mantissa bits of an fp32
+// word.  With x_hi = x with its low 13 mantissa bits cleared (exact in TF32)
+// and x_lo = x - x_hi (exact in fp32, at most 2^-10 |x|),
+//   A B = A_hi B_hi + A_lo B_hi + A_hi B_lo + A_lo B_lo,
+// and the last term (at most 2^-20 |A B| per product) is dropped; x_lo itself
+// enters the MMA with a further relative error of 2^-10 at most, so every
+// product carries about 2^-20 relative error before the fp32 accumulation:
+// the accuracy of an fp32 dot product, at tensor-core rate (three TF32 MMAs
+// per K step, two when the X operand is bf16, whose x_lo is 0).
+//
+// k_mm_tf32<MODE, D, TX>, one 128-row block of output per CTA, 256 threads,
+// contraction in chunks of 32 (one 128-byte swizzled row of fp32):
+//   MODE 0: out[r][e] = scale * sum_{j <= r} map[r][j] X[j][e]     (O = A V, dQ)
+//   MODE 1: out[r][e] = scale * sum_{i >= r} map[i][r] X[i][e]     (dV = A^T dO, dK)
+//   MODE 2: map[i][j] = scale * sum_e A[i][e] X[j][e] for j <= i, 0 above,
+//           one 128 x 128 tile of the causal triangle               (dA = dO V^T)
+// Every thread converts its share of each chunk (hi and lo tiles, K-major,
+// in the MMA's 128-byte-swizzled layout, transposed where the source runs
+// along the tile's rows) from registers loaded two chunks ahead; thread 0
+// issues the chunk's MMAs once all threads have arrived and commits to the
+// stage's barrier, which frees the stage two chunks later.
+constexpr int kMmKc = 32;             // contraction indices per chunk
+constexpr int kMmStages = 2;
+
+__device__ __forceinline__ float tf32_hi(float x)
+{
+    return __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+}
+
+// Byte offset of fp32 element (row, k) of a K-major 128-byte-swizzled tile
+// whose rows hold 32 elements (tile base 1024-byte aligned).
+__device__ __forceinline__ uint32_t sw128_f32(uint32_t row, uint32_t k)
+{
+    return row * 128u + ((((k >> 2) ^ (row & 7u)) & 7u) << 4) + ((k & 3u) << 2);
+}
+
+// Transposed loads (a source that runs along the tile's rows, read for 32
+// contraction indices): slot = warp + 8u and lane give contraction index
+// tq_k and row quad tq_q (rows 4 tq_q .. +3).  A warp reads 16 source rows x
+// 32 bytes (whole sectors), and each of its four scalar stores per quad hits
+// 32 distinct banks of the K-major swizzled tile.
+__device__ __forceinline__ int tq_k(int slot, int lane) { return 16 * (slot & 1) + (lane & 15); }
+__device__ __forceinline__ int tq_q(int slot, int lane) { return 2 * (slot >> 1) + (lane >> 4); }
+
+__device__ __forceinline__ void store_split4(uint8_t *hi, uint8_t *lo, uint32_t off, float4 v)
+{
+    const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+    *reinterpret_cast<float4 *>(hi + off) = h;
+    *reinterpret_cast<float4 *>(lo + off) = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+}
+
+__device__ __forceinline__ void store_split1(uint8_t *hi, uint8_t *lo, uint32_t off, float v)
+{
+    const float h = tf32_hi(v);
+    *reinterpret_cast<float *>(hi + off) = h;
+    *reinterpret_cast<float *>(lo + off) = v - h;
+}
+
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p)
+{
+    const uint2 t = *reinterpret_cast<const uint2 *>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&t.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&t.y);
+    return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+}
+
+template <int MODE, int D, typename TX>
+struct MmCfg {
+    static constexpr bool kXlo = sizeof(TX) == 4;               // an fp32 X operand has a lo part
+    static constexpr int N = MODE == 2 ? kTile : D;             // accumulator columns
+    static constexpr int kATile = kTile * kMmKc * 4;            // 16 KB
+    static constexpr int kBTile = N * kMmKc * 4;
+    static constexpr int kStage = 2 * kATile + (kXlo ? 2 : 1) * kBTile;
+    static constexpr int kSmem = kMmStages * kStage + 1024;
+    static constexpr int kBU = N * kMmKc / 4 / kPvThreads;     // X float4 groups per thread
+};
+
+template <int MODE, int D, typename TX>
+__global__ void __launch_bounds__(kPvThreads, 2)
+k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__restrict__ out, int T,
+          float scale)
+{
+    using C = MmCfg<MODE, D, TX>;
+    unsigned int *err = &g_chain_error;
+    int r0, j0 = 0, c_begin, c_end;
+    const int bh = MODE == 2 ? blockIdx.z : blockIdx.y;
+    if (MODE == 2) {
+        r0 = blockIdx.y * kTile;
+        j0 = blockIdx.x * kTile;
+        if (j0 > r0 + kTile - 1) return;                         // the tile lies above the diagonal
+        c_begin = 0;
+        c_end = D;
+    } else {
+        // longest contraction first: MODE 0 grows with the row block, MODE 1 shrinks
+        const int blk = MODE == 0 ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+        r0 = blk * kTile;
+        c_begin = MODE == 0 ? 0 : r0;
+        c_end = MODE == 0 ? min(T, r0 + kTile) : T;
+    }
+    const int nch = (c_end - c_begin + kMmKc - 1) / kMmKc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t a_full[kMmStages], mma_done[kMmStages];
+    __shared__ uint32_t tslot;
+    __shared__ int abort_flag;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    if (tid == 0) {
+        for (int s = 0; s < kMmStages; ++s) {
+            tc::mbar_init(&a_full[s], kPvThreads);
+            tc::mbar_init(&mma_done[s], 1);
+        }
+        abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 0) { tc::tmem_alloc(&tslot, C::N); tc::tmem_relinquish(); }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = tslot;
+    const size_t TT = (size_t)T * T;
+    const float *amap = asrc + (size_t)bh * (MODE == 2 ? (size_t)T * D : TT);
+    const TX *xb = x + (size_t)bh * T * D;
+    const bool vec = (T & 3) == 0;
+    // A operand, four groups of 4 per thread; X operand, C::kBU groups of 4
+    struct Regs { float4 a[4], x[C::kBU]; };
+    Regs set0, set1;                 // chunks n (even) and n + 1 (odd), loaded two chunks ahead
+    auto load_chunk = [&](int n, Regs &R) {
+        const int c0 = c_begin + n * kMmKc;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int f = tid + kPvThreads * u;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (MODE == 0) {                 // row r0 + (f >> 3), keys c0 + 4 (f & 7) .. +3
+                const int i = r0 + (f >> 3), j = c0 + 4 * (f & 7);
+                if (i < T && j <= i) {
+                    const float *p = amap + (size_t)i * T + j;
+                    if (vec && j + 3 <= i) v = ld4(p);
+                    else {
+                        v.x = p[0];
+                        if (j + 1 <= i) v.y = p[1];
+                        if (j + 2 <= i) v.z = p[2];
+                        if (j + 3 <= i) v.w = p[3];
+                    }
+                }
+            } else if (MODE == 1) {          // query c0 + tq_k, keys r0 + 4 tq_q .. +3
+                const int slot = warp + 8 * u;
+                const int i = c0 + tq_k(slot, lane), j = r0 + 4 * tq_q(slot, lane);
+                if (i < T && j <= i) {
+                    const float *p = amap + (size_t)i * T + j;
+                    if (vec && j + 3 <= i) v = ld4(p);
+                    else {
+                        v.x = p[0];
+                        if (j + 1 <= i && j + 1 < T) v.y = p[1];
+                        if (j + 2 <= i && j + 2 < T) v.z = p[2];
+                        if (j + 3 <= i && j + 3 < T) v.w = p[3];
+                    }
+                }
+            } else {                         // row r0 + (f >> 3), channels c0 + 4 (f & 7) .. +3
+                const int i = r0 + (f >> 3);
+                if (i < T) v = ld4(amap + (size_t)i * D + c0 + 4 * (f & 7));
+            }
+            R.a[u] = v;
+        }
+#pragma unroll
+        for (int u = 0; u < C::kBU; ++u) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (MODE == 2) {                 // key j0 + (f >> 3), channels c0 + 4 (f & 7) .. +3
+                const int f = tid + kPvThreads * u, j = j0 + (f >> 3);
+                if (j < T) v = ld4(xb + (size_t)j * D + c0 + 4 * (f & 7));
+            } else {                         // index c0 + tq_k, channels 4 tq_q .. +3
+                const int slot = warp + 8 * u, c = c0 + tq_k(slot, lane);
+                if (c < T) v = ld4(xb + (size_t)c * D + 4 * tq_q(slot, lane));
+            }
+            R.x[u] = v;
+        }
+    };
+    auto store_chunk = [&](uint8_t *st, const Regs &R) {
+        uint8_t *ahi = st, *alo = st + C::kATile;
+        uint8_t *bhi = st + 2 * C::kATile, *blo = bhi + C::kBTile;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int f = tid + kPvThreads * u;
+            if (MODE == 1) {                 // transposed: rows 4 tq_q + q, column tq_k
+                const int slot = warp + 8 * u, kk = tq_k(slot, lane), rr = 4 * tq_q(slot, lane);
+                store_split1(ahi, alo, sw128_f32(rr, kk), R.a[u].x);
+                store_split1(ahi, alo, sw128_f32(rr + 1, kk), R.a[u].y);
+                store_split1(ahi, alo, sw128_f32(rr + 2, kk), R.a[u].z);
+                store_split1(ahi, alo, sw128_f32(rr + 3, kk), R.a[u].w);
+            } else {
+                store_split4(ahi, alo, sw128_f32(f >> 3, 4 * (f & 7)), R.a[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < C::kBU; ++u) {
+            const float4 v = R.x[u];
+            if (MODE == 2) {
+                const int f = tid + kPvThreads * u;
+                const uint32_t off = sw128_f32(f >> 3, 4 * (f & 7));
+                if (C::kXlo) store_split4(bhi, blo, off, v);
+                else *reinterpret_cast<float4 *>(bhi + off) = v;    // bf16 values are exact in TF32
+            } else {                         // transposed: rows (channels) 4 tq_q + q, column tq_k
+                const int slot = warp + 8 * u, kk = tq_k(slot, lane), e = 4 * tq_q(slot, lane);
+                const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t off = sw128_f32(e + q, kk);
+                    if (C::kXlo) store_split1(bhi, blo, off, w[q]);
+                    else *reinterpret_cast<float *>(bhi + off) = w[q];
+                }
+            }
+        }
+    };
+    const uint32_t idesc = tc::idesc_tf32(kTile, C::N, false, false);
+    int committed = 0;
+    bool ok = true;
+    // one chunk: wait for its stage, convert from the registers, refill them
+    // with chunk n + 2, and (thread 0) issue the MMAs once everyone arrived
+    auto step = [&](int n, Regs &R) -> bool {
+        const int s = n % kMmStages;
+        const uint32_t use = (uint32_t)(n / kMmStages);
+        uint8_t *st = base + s * C::kStage;
+        if (n >= kMmStages && !wait_or_abort(&mma_done[s], (use - 1) & 1, &abort_flag, err))
+            return false;
+        store_chunk(st, R);
+        if (n + 2 < nch) load_chunk(n + 2, R);
+        tc::fence_async_shared();
+        tc::mbar_arrive(&a_full[s]);
+        if (tid == 0) {
+            if (!wait_or_abort(&a_full[s], use & 1, &abort_flag, err)) return false;
+            tc::tc_fence_after();
+            const uint64_t dah = tc::sdesc_sw128(tc::smem_u32(st), 16, 1024);
+            const uint64_t dal = tc::sdesc_sw128(tc::smem_u32(st + C::kATile), 16, 1024);
+            const uint64_t dbh = tc::sdesc_sw128(tc::smem_u32(st + 2 * C::kATile), 16, 1024);
+            const uint64_t dbl = tc::sdesc_sw128(tc::smem_u32(st + 2 * C::kATile + C::kBTile), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kMmKc / 8; ++kk) {       // K = 8 per MMA: 32 bytes of a row
+                const uint64_t o = (uint64_t)((kk * 32) >> 4);
+                tc::mma_tf32(tm, dah + o, dbh + o, idesc, (n | kk) ? 1u : 0u);
+                tc::mma_tf32(tm, dal + o, dbh + o, idesc, 1u);
+                if (C::kXlo) tc::mma_tf32(tm, dah + o, dbl + o, idesc, 1u);
+            }
+            tc::mma_commit(&mma_done[s]);
+            ++committed;
+        }
+        return true;
+    };
+    load_chunk(0, set0);
+    if (nch > 1) load_chunk(1, set1);
+    for (int n = 0; n < nch && ok; n += 2) {
+        ok = step(n, set0);
+        if (ok && n + 1 < nch) ok = step(n + 1, set1);
+    }
+    const int last = nch - 1;
+    ok = ok && wait_or_abort(&mma_done[last % kMmStages], (uint32_t)(last / kMmStages) & 1,
+                             &abort_flag, err);
+    if (tid == 0 && !ok && committed > 0)   // after an abort: the MMAs in flight finish first
+        tc::mbar_wait(&mma_done[(committed - 1) % kMmStages],
+                      (uint32_t)((committed - 1) / kMmStages) & 1, kBudget);
+    if (warp < 4 && __all_sync(0xffffffffu, ok)) {
+        tc::tc_fence_after();
+        const int i = r0 + 32 * warp + lane;
+        const uint32_t row = tm + ((uint32_t)(32 * warp) << 16);
+        if (MODE != 2) {
+            float *dst = out + ((size_t)bh * T + i) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                tc::tmem_ld32f(row + 32 * c, v);
+                tc::tmem_ld_wait();
+                if (i < T) {
+#pragma unroll
+                    for (int m = 0; m < 8; ++m)
+                        *reinterpret_cast<float4 *>(dst + 32 * c + 4 * m) =
+                            make_float4(v[4 * m] * scale, v[4 * m + 1] * scale, v[4 * m + 2] * scale,
+                                        v[4 * m + 3] * scale);
+                }
+            }
+        } else {
+            // the map tile, through a per-warp staging tile (stage 0 is free:
+            // every MMA has completed) so that stores cover whole row segments
+            float *stage = (float *)base + warp * 32 * kStageStride;
+            float *srow = stage + lane * kStageStride;
+            float *mb = out + (size_t)bh * TT;
+#pragma unroll 1
+            for (int jc = 0; jc < kTile / 32; ++jc) {
+                float v[32];
+                tc::tmem_ld32f(row + 32 * jc, v);
+                tc::tmem_ld_wait();
+                const int jb = j0 + 32 * jc;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] = (jb + c <= i) ? v[c] * scale : 0.f;
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    *reinterpret_cast<float4 *>(srow + 4 * m) =
+                        make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+                __syncwarp();
+                if (vec) {
+#pragma unroll
+                    for (int rho = 0; rho < 8; ++rho) {
+                        const int rr = 4 * rho + (lane >> 3);
+                        const int ii = r0 + 32 * warp + rr, jj = jb + 4 * (lane & 7);
+                        const float4 t = *reinterpret_cast<const float4 *>(stage + rr * kStageStride +
+                                                                           4 * (lane & 7));
+                        if (ii < T && jj < T) *reinterpret_cast<float4 *>(mb + (size_t)ii * T + jj) = t;
+                    }
+                } else {
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const int ii = r0 + 32 * warp + rr, jj = jb + lane;
+                        if (ii < T && jj < T) mb[(size_t)ii * T + jj] = stage[rr * kStageStride + lane];
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tm, C::N);
+    }
+}
+
+template <int MODE, int D, typename TX>
+mta_status launch_mm_tf32_t(const mta_shape &s, const float *a, const void *xv, float *out,
+                            float scale, cudaStream_t st)
+{
+    using C = MmCfg<MODE, D, TX>;
+    auto kern = k_mm_tf32<MODE, D, TX>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+        cudaSuccess)
+        return MTA_ERR_CUDA;
+    const int nb = (s.T + kTile - 1) / kTile;
+    const unsigned BH = (unsigned)(s.B * s.H);
+    const dim3 grid = MODE == 2 ? dim3(nb, nb, BH) : dim3(nb, BH);
+    kern<<<grid, kPvThreads, C::kSmem, st>>>(a, (const TX *)xv, out, s.T, scale);
+    return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
+}
+
+template <int MODE, typename TX>
+mta_status launch_mm_tf32_d(const mta_shape &s, const float *a, const void *xv, float *out,
+                            float scale, cudaStream_t st)
+{
+    return s.d == 128 ? launch_mm_tf32_t<MODE, 128, TX>(s, a, xv, out, scale, st)
+                      : launch_mm_tf32_t<MODE, 64, TX>(s, a, xv, out, scale, st);
+}
+
+template <int MODE>
+mta_status launch_mm_tf32(const mta_shape &s, const float *a, const void *xv, bool x_io,
+                          float *out, float scale, cudaStream_t st)
+{
+    if (x_io && s.io == MTA_BF16)
+        return launch_mm_tf32_d<MODE, __nv_bfloat16>(s, a, xv, out, scale, st);
+    return launch_mm_tf32_d<MODE, float>(s, a, xv, out, scale, st);
+}
+
 template <int D>
 mta_status launch_logits_tc_t(const mta_shape &s, const void *q, const void *k, float *map0,
                               int band, cudaStream_t st)
@@ -422,6 +782,21 @@ unsigned int chain_take_error(cudaStream_t st)
         cudaStreamSynchronize(st) != cudaSuccess)
         return ~0u;
     return v;
+}
+
+bool mm_tf32_supported(const mta_shape &s) { return s.d == 64 || s.d == 128; }
+
+mta_status causal_mm_tf32(const mta_shape &s, bool trans, const float *map, const void *x,
+                          bool x_io, float *out, float scale, cudaStream_t st)
+{
+    return trans ? launch_mm_tf32<1>(s, map, x, x_io, out, scale, st)
+                 : launch_mm_tf32<0>(s, map, x, x_io, out, scale, st);
+}
+
+mta_status logits_f32_tf32(const mta_shape &s, const float *a, const void *b, float scale,
+                           float *map, cudaStream_t st)
+{
+    return launch_mm_tf32<2>(s, a, b, true, map, scale, st);
 }
 
 bool chain_tc_supported(const mta_shape &s)

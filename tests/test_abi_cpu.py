@@ -141,13 +141,17 @@ def test_forward_path_selection(L, kw, path):
 
 
 def test_backward_launch_names_follow_the_chain(L):
-    # the recomputed logits take the chain's kernel; dA = dO V^T (fp32 dO)
-    # always runs on CUDA cores
-    for kw, first in ((dict(d=128), "k_logits_tc"), (dict(d=32), "k_logits"),
-                      (dict(d=64, io="f32"), "k_logits")):
+    # the recomputed logits take the chain's kernel; at d = 64 or 128 the fp32
+    # products (A V, dV, dA = dO V^T, dQ, dK) are 3xTF32 tensor-core launches
+    for kw, first, tf32 in ((dict(d=128), "k_logits_tc", True), (dict(d=32), "k_logits", False),
+                            (dict(d=64, io="f32"), "k_logits", True)):
         names = mta.mta_backward_kernel_names(shape(**kw))
-        assert len(names) == 14 and names[0] == first and names[7] == "k_logits"
-        assert names.count("k_causal_mm") == 4
+        assert len(names) == 14 and names[0] == first
+        if tf32:
+            assert [names[i] for i in (4, 6, 7, 11, 12)] == ["k_mm_tf32"] * 5
+            assert "k_causal_mm" not in names
+        else:
+            assert names[7] == "k_logits" and names.count("k_causal_mm") == 4
 
 
 def test_selftest_rejects_bad_budget(L):
