@@ -54,6 +54,7 @@ def assert_every_element(got, ref, H, d, what):
         b, t, c // d, c % d, t % 128, bad_rows)
     assert maxabs <= TOL_BF16_MAXABS and rel <= TOL_BF16_RELL2, \
         "%s: max-abs %.3g rel-L2 %.3g, %s" % (what, maxabs, rel, where)
+    print("%s: max-abs %.4g rel-L2 %.4g over %d elements" % (what, maxabs, rel, got.size))
     return maxabs, rel
 
 
