@@ -391,9 +391,16 @@ k_conv_adj(const float *__restrict__ src, float *__restrict__ dst, const float *
     if (r >= T) return;
     float *row = dst + bh * (size_t)T * T + (size_t)r * T;
 #pragma unroll
-    for (int u = 0; u < NC; ++u) {
-        const int c = c0 + cl + u;
-        if (c <= r && c < T) row[c] = acc[u];
+    for (int g = 0; g < NC / 4; ++g) {
+        const int cb = c0 + cl + 4 * g;
+        if ((T & 3) == 0 && cb + 3 <= r) {       // 16-byte stores where the row segment is whole
+            *reinterpret_cast<float4 *>(row + cb) =
+                make_float4(acc[4 * g], acc[4 * g + 1], acc[4 * g + 2], acc[4 * g + 3]);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (cb + u <= r && cb + u < T) row[cb + u] = acc[4 * g + u];
+        }
     }
 }
 
@@ -444,9 +451,16 @@ k_dtheta(const float *__restrict__ dc, const float *__restrict__ a0, float *__re
     {
         const float *grow = dc + bh * (size_t)T * T + (size_t)i * T;
 #pragma unroll
-        for (int u = 0; u < NC; ++u) {
-            const int j = j0 + cl + u;
-            g[u] = (i < T && j <= i) ? grow[j] : 0.f;
+        for (int q = 0; q < NC / 4; ++q) {
+            const int jb = j0 + cl + 4 * q;
+            if ((T & 3) == 0 && i < T && jb + 3 <= i) {   // 16-byte loads of whole segments
+                const float4 t = *reinterpret_cast<const float4 *>(grow + jb);
+                g[4 * q] = t.x; g[4 * q + 1] = t.y; g[4 * q + 2] = t.z; g[4 * q + 3] = t.w;
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    g[4 * q + u] = (i < T && jb + u <= i) ? grow[jb + u] : 0.f;
+            }
         }
     }
     for (int ip = 0; ip < c_q; ++ip) {
