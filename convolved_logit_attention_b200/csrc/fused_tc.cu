@@ -1131,16 +1131,29 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 need = mt > m_run + 8.f;
                 m_new = need ? mt : m_run;
                 alpha = ex2(m_run - m_new);
-                // P~ = exp2(S - m), packed to bf16 pairs
+                // P~ = exp2(S - m), packed to bf16 pairs; each half goes to TMEM
+                // (over the first kBN/2 columns of the S buffer, where PV(t) reads
+                // it as the A operand) as soon as it is ready, so the first store
+                // overlaps the second half's exponentials
 #pragma unroll
-                for (int c = 0; c < kBN; c += 2) {
+                for (int c = 0; c < kBN / 2; c += 2) {
                     const float p0 = ex2(s[c] - m_new), p1 = ex2(s[c + 1] - m_new);
                     lp[(c >> 1) & 7] += p0 + p1;
                     pk[c >> 1] = pack_bf16(p0, p1);
                 }
+                tc::tmem_st32(lane_base + sb * kBN, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+#pragma unroll
+                for (int c = kBN / 2; c < kBN; c += 2) {
+                    const float p0 = ex2(s[c] - m_new), p1 = ex2(s[c + 1] - m_new);
+                    lp[(c >> 1) & 7] += p0 + p1;
+                    pk[c >> 1] = pack_bf16(p0, p1);
+                }
+                tc::tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
                 } else {
 #pragma unroll
                     for (int x = 0; x < kBN / 2; ++x) pk[x] = 0u;
+                    tc::tmem_st32(lane_base + sb * kBN, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+                    tc::tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
                 }
                 // Every warp waits for PV(t-1) to complete before it publishes
                 // P~(t).  p_full counts arrivals from all softmax warps (of both
@@ -1170,10 +1183,7 @@ k_mta_fused(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CU
                 }
                 l = l * alpha + (((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7])));
                 m_run = m_new;
-                // P~(t) goes to TMEM over the first kBN/2 columns of its S buffer,
-                // where PV(t) reads it as the A operand
-                tc::tmem_st32(lane_base + sb * kBN, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-                tc::tmem_st32(lane_base + sb * kBN + 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + 32));
+                // P~(t) is in TMEM once the stores issued above have completed
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();

@@ -124,3 +124,44 @@ def test_fp32_fused_stores_stay_inside_out(shape):
     mta.mta_sync_status()
     assert _guards_intact(out_buf, out_bytes), "a store landed outside out"
     assert torch.isfinite(out_body.view(torch.float32)).all()
+
+
+# The backward pass: every gradient buffer and the workspace between guard
+# regions, at ragged T, both I/O types and d = 64 / 128 (the tensor-core
+# products) as well as d = 32 (the CUDA-core ones).
+BWD_SHAPES = [
+    # B, H, T, d, c_q, c_k, c_h, io
+    (1, 2, 1, 128, 6, 11, 2, "bf16"),
+    (1, 2, 129, 128, 6, 11, 2, "bf16"),
+    (2, 4, 200, 64, 4, 15, 2, "f32"),
+    (1, 4, 130, 128, 8, 15, 4, "bf16"),
+    (1, 2, 65, 32, 3, 4, 2, "bf16"),
+]
+
+
+@pytest.mark.parametrize("shape", BWD_SHAPES, ids=[str(s) for s in BWD_SHAPES])
+def test_backward_stores_stay_inside_gradients_and_workspace(shape):
+    B, H, T, d, c_q, c_k, c_h, io = shape
+    x, t = _inputs(shape[:7], seed=sum(shape[:7]) + 2, io=io)
+    dt = torch.bfloat16 if io == "bf16" else torch.float32
+    dout = torch.randn(B, T, H * d, device="cuda").to(dt)
+    mshape = mta.make_shape(B, H, T, d, c_q, c_k, c_h, io, x["gn_eps"])
+    sizes = {"q": B * H * T * d, "k": B * H * T * d, "v": B * H * T * d, "w_kq": H * c_q * c_k,
+             "w_head": (H // c_h) * c_h * c_h, "gn_weight": H * d, "gn_bias": H * d}
+    bufs = {n: _guarded(4 * m) for n, m in sizes.items()}
+    need = mta.mta_backward_workspace_size(mshape)
+    ws_buf, ws_body = _guarded(need)
+    L = mta.lib()
+    p = lambda a: ctypes.c_void_p(a.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = L.mta_backward(ctypes.byref(mshape), p(t["q"]), p(t["k"]), p(t["v"]), p(t["w_kq"]),
+                        p(t["w_head"]), p(t["gn_weight"]), p(t["gn_bias"]),
+                        ctypes.c_float(x["depth_scale"]), None, p(dout),
+                        *[p(bufs[n][1]) for n in mta.GRAD_NAMES], None, p(ws_body),
+                        ctypes.c_size_t(need), stream)
+    assert rc == 0
+    mta.mta_sync_status()
+    for n, (buf, body) in bufs.items():
+        assert _guards_intact(buf, 4 * sizes[n]), "a store landed outside d" + n
+        assert torch.isfinite(body.view(torch.float32)).all(), "d" + n + " not finite"
+    assert _guards_intact(ws_buf, need), "a store landed outside the workspace"
