@@ -379,13 +379,15 @@ k_pv_groupnorm_tc(const float *__restrict__ amap, const __grid_constant__ CUtens
 //   MODE 1: out[r][e] = scale * sum_{i >= r} map[i][r] X[i][e]     (dV = A^T dO, dK)
 //   MODE 2: map[i][j] = scale * sum_e A[i][e] X[j][e] for j <= i, 0 above,
 //           one 128 x 128 tile of the causal triangle               (dA = dO V^T)
-// Every thread converts its share of each chunk (hi and lo tiles, K-major,
-// in the MMA's 128-byte-swizzled layout, transposed where the source runs
-// along the tile's rows) from registers loaded two chunks ahead; thread 0
-// issues the chunk's MMAs once all threads have arrived and commits to the
-// stage's barrier, which frees the stage two chunks later.
+// The raw source rows of a chunk are copied with cp.async into a ring of
+// staging buffers, one chunk ahead; each copy's completion is counted on the
+// buffer's barrier (one arrival per thread).  Every thread then converts its
+// share of the chunk from shared memory into the K-major hi and lo tiles in
+// the MMA's 128-byte-swizzled layout (transposed where the source runs along
+// the tile's rows, masked to the causal triangle), and thread 0 issues the
+// chunk's MMAs once all threads have arrived; their commit frees the tiles for
+// the next chunk.  Rows of the map must be 16-byte aligned (T % 4 == 0).
 constexpr int kMmKc = 32;             // contraction indices per chunk
-constexpr int kMmStages = 2;
 
 __device__ __forceinline__ float tf32_hi(float x)
 {
@@ -399,11 +401,11 @@ __device__ __forceinline__ uint32_t sw128_f32(uint32_t row, uint32_t k)
     return row * 128u + ((((k >> 2) ^ (row & 7u)) & 7u) << 4) + ((k & 3u) << 2);
 }
 
-// Transposed loads (a source that runs along the tile's rows, read for 32
+// Transposed conversion (a source that runs along the tile's rows, read for 32
 // contraction indices): slot = warp + 8u and lane give contraction index
-// tq_k and row quad tq_q (rows 4 tq_q .. +3).  A warp reads 16 source rows x
-// 32 bytes (whole sectors), and each of its four scalar stores per quad hits
-// 32 distinct banks of the K-major swizzled tile.
+// tq_k and row quad tq_q (rows 4 tq_q .. +3).  A warp reads 16 staged rows x
+// 32 bytes and each of its four scalar stores per quad hits 32 distinct banks
+// of the K-major swizzled tile.
 __device__ __forceinline__ int tq_k(int slot, int lane) { return 16 * (slot & 1) + (lane & 15); }
 __device__ __forceinline__ int tq_q(int slot, int lane) { return 2 * (slot >> 1) + (lane >> 4); }
 
@@ -433,20 +435,41 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p)
 template <int MODE, int D, typename TX>
 struct MmCfg {
     static constexpr bool kXlo = sizeof(TX) == 4;               // an fp32 X operand has a lo part
+    static constexpr int kES = (int)sizeof(TX);
     static constexpr int N = MODE == 2 ? kTile : D;             // accumulator columns
     static constexpr int kATile = kTile * kMmKc * 4;            // 16 KB
     static constexpr int kBTile = N * kMmKc * 4;
     static constexpr int kStage = 2 * kATile + (kXlo ? 2 : 1) * kBTile;
-    static constexpr int kSmem = kMmStages * kStage + 1024;
-    static constexpr int kBU = N * kMmKc / 4 / kPvThreads;     // X float4 groups per thread
+    // staging: the A rows (MODE 1: 32 map rows of 128 keys, padded by 16 B so
+    // that transposed reads spread over the banks) and the X rows (MODE 0/1:
+    // 32 rows of D, padded; MODE 2: 128 rows of 32 channels)
+    static constexpr int kAPitch = MODE == 1 ? kTile * 4 + 16 : kMmKc * 4;       // bytes
+    static constexpr int kARows = MODE == 1 ? kMmKc : kTile;
+    static constexpr int kXPitch = MODE == 2 ? kMmKc * kES : D * kES + 16;
+    static constexpr int kXRows = MODE == 2 ? kTile : kMmKc;
+    static constexpr int kRawA = kARows * kAPitch;
+    static constexpr int kRaw = (kRawA + kXRows * kXPitch + 1023) / 1024 * 1024;
+    // one tile stage and two staging buffers: 97 KB with a bf16 X, so two CTAs
+    // share an SM and one's conversion, MMAs and stores overlap the other's
+    // (measured faster than two tile stages and three staging buffers at one
+    // CTA per SM); 130 KB, one CTA per SM, with an fp32 X
+    static constexpr int kStages = 1;
+    static constexpr int kRawStages = 2;
+    static constexpr int kSmem = kStages * kStage + kRawStages * kRaw + 1024;
+    static constexpr int kMinBlocks = kSmem <= 113 * 1024 ? 2 : 1;
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+    static constexpr int kACopies = kARows * kAPitch / 16 / kPvThreads;   // 16-B copies per thread
+    static constexpr int kXCopies = kXRows * (MODE == 2 ? kMmKc * kES : D * kES) / 16 / kPvThreads;
+    static constexpr int kBU = N * kMmKc / 4 / kPvThreads;     // X groups of 4 per thread
 };
 
 template <int MODE, int D, typename TX>
-__global__ void __launch_bounds__(kPvThreads, 2)
+__global__ void __launch_bounds__(kPvThreads, MmCfg<MODE, D, TX>::kMinBlocks)
 k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__restrict__ out, int T,
           float scale)
 {
     using C = MmCfg<MODE, D, TX>;
+    constexpr int R = C::kRawStages;
     unsigned int *err = &g_chain_error;
     int r0, j0 = 0, c_begin, c_end;
     const int bh = MODE == 2 ? blockIdx.z : blockIdx.y;
@@ -466,15 +489,17 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
     const int nch = (c_end - c_begin + kMmKc - 1) / kMmKc;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t a_full[kMmStages], mma_done[kMmStages];
+    uint8_t *raw0 = base + C::kStages * C::kStage;
+    __shared__ uint64_t a_full[C::kStages], mma_done[C::kStages], raw_full[C::kRawStages];
     __shared__ uint32_t tslot;
     __shared__ int abort_flag;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     if (tid == 0) {
-        for (int s = 0; s < kMmStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             tc::mbar_init(&a_full[s], kPvThreads);
             tc::mbar_init(&mma_done[s], 1);
         }
+        for (int s = 0; s < R; ++s) tc::mbar_init(&raw_full[s], kPvThreads);
         abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -486,86 +511,86 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
     const size_t TT = (size_t)T * T;
     const float *amap = asrc + (size_t)bh * (MODE == 2 ? (size_t)T * D : TT);
     const TX *xb = x + (size_t)bh * T * D;
-    const bool vec = (T & 3) == 0;
-    // A operand, four groups of 4 per thread; X operand, C::kBU groups of 4
-    struct Regs { float4 a[4], x[C::kBU]; };
-    Regs set0, set1;                 // chunks n (even) and n + 1 (odd), loaded two chunks ahead
-    auto load_chunk = [&](int n, Regs &R) {
+    // cp.async of chunk n into raw stage n % R (rows outside [0, T) zero-filled)
+    auto issue_copies = [&](int n) {
+        uint8_t *ra = raw0 + (n % R) * C::kRaw;
+        uint8_t *rx = ra + C::kRawA;
         const int c0 = c_begin + n * kMmKc;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < C::kACopies; ++u) {
             const int f = tid + kPvThreads * u;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (MODE == 0) {                 // row r0 + (f >> 3), keys c0 + 4 (f & 7) .. +3
+            if (MODE == 1) {                 // map row c0 + (f >> 5), keys r0 + 4 (f & 31) .. +3
+                const int i = c0 + (f >> 5), j = r0 + 4 * (f & 31);
+                const bool in = i < T && j < T;
+                tc::cp_async16(ra + (f >> 5) * C::kAPitch + 16 * (f & 31),
+                               amap + (in ? (size_t)i * T + j : 0), in);
+            } else if (MODE == 0) {          // map row r0 + (f >> 3), keys c0 + 4 (f & 7) .. +3
                 const int i = r0 + (f >> 3), j = c0 + 4 * (f & 7);
-                if (i < T && j <= i) {
-                    const float *p = amap + (size_t)i * T + j;
-                    if (vec && j + 3 <= i) v = ld4(p);
-                    else {
-                        v.x = p[0];
-                        if (j + 1 <= i) v.y = p[1];
-                        if (j + 2 <= i) v.z = p[2];
-                        if (j + 3 <= i) v.w = p[3];
-                    }
-                }
-            } else if (MODE == 1) {          // query c0 + tq_k, keys r0 + 4 tq_q .. +3
-                const int slot = warp + 8 * u;
-                const int i = c0 + tq_k(slot, lane), j = r0 + 4 * tq_q(slot, lane);
-                if (i < T && j <= i) {
-                    const float *p = amap + (size_t)i * T + j;
-                    if (vec && j + 3 <= i) v = ld4(p);
-                    else {
-                        v.x = p[0];
-                        if (j + 1 <= i && j + 1 < T) v.y = p[1];
-                        if (j + 2 <= i && j + 2 < T) v.z = p[2];
-                        if (j + 3 <= i && j + 3 < T) v.w = p[3];
-                    }
-                }
-            } else {                         // row r0 + (f >> 3), channels c0 + 4 (f & 7) .. +3
+                const bool in = i < T && j < T;
+                tc::cp_async16(ra + (f >> 3) * C::kAPitch + 16 * (f & 7),
+                               amap + (in ? (size_t)i * T + j : 0), in);
+            } else {                         // A row r0 + (f >> 3), channels c0 + 4 (f & 7) .. +3
                 const int i = r0 + (f >> 3);
-                if (i < T) v = ld4(amap + (size_t)i * D + c0 + 4 * (f & 7));
+                const bool in = i < T;
+                tc::cp_async16(ra + (f >> 3) * C::kAPitch + 16 * (f & 7),
+                               amap + (in ? (size_t)i * D + c0 + 4 * (f & 7) : 0), in);
             }
-            R.a[u] = v;
         }
+        constexpr int kRowChunks = (MODE == 2 ? kMmKc * C::kES : D * C::kES) / 16;
 #pragma unroll
-        for (int u = 0; u < C::kBU; ++u) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (MODE == 2) {                 // key j0 + (f >> 3), channels c0 + 4 (f & 7) .. +3
-                const int f = tid + kPvThreads * u, j = j0 + (f >> 3);
-                if (j < T) v = ld4(xb + (size_t)j * D + c0 + 4 * (f & 7));
-            } else {                         // index c0 + tq_k, channels 4 tq_q .. +3
-                const int slot = warp + 8 * u, c = c0 + tq_k(slot, lane);
-                if (c < T) v = ld4(xb + (size_t)c * D + 4 * tq_q(slot, lane));
-            }
-            R.x[u] = v;
+        for (int u = 0; u < C::kXCopies; ++u) {
+            const int f = tid + kPvThreads * u, row = f / kRowChunks, q = f % kRowChunks;
+            const int g = MODE == 2 ? j0 + row : c0 + row;           // source row of X
+            const bool in = g < T;
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(xb) +
+                                 (in ? (size_t)g * D * C::kES + (MODE == 2 ? (size_t)c0 * C::kES : 0) : 0) +
+                                 16 * q;
+            tc::cp_async16(rx + row * C::kXPitch + 16 * q, src, in);
         }
+        tc::cp_async_mbar_arrive(&raw_full[n % R]);
     };
-    auto store_chunk = [&](uint8_t *st, const Regs &R) {
+    // chunk n from raw stage n % R into the hi / lo tiles of stage st
+    auto convert = [&](int n, uint8_t *st) {
+        const uint8_t *ra = raw0 + (n % R) * C::kRaw;
+        const uint8_t *rx = ra + C::kRawA;
+        const int c0 = c_begin + n * kMmKc;
         uint8_t *ahi = st, *alo = st + C::kATile;
         uint8_t *bhi = st + 2 * C::kATile, *blo = bhi + C::kBTile;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int f = tid + kPvThreads * u;
-            if (MODE == 1) {                 // transposed: rows 4 tq_q + q, column tq_k
+            if (MODE == 1) {                 // transposed: rows (keys) 4 tq_q + q, column tq_k
                 const int slot = warp + 8 * u, kk = tq_k(slot, lane), rr = 4 * tq_q(slot, lane);
-                store_split1(ahi, alo, sw128_f32(rr, kk), R.a[u].x);
-                store_split1(ahi, alo, sw128_f32(rr + 1, kk), R.a[u].y);
-                store_split1(ahi, alo, sw128_f32(rr + 2, kk), R.a[u].z);
-                store_split1(ahi, alo, sw128_f32(rr + 3, kk), R.a[u].w);
+                const float4 v = *reinterpret_cast<const float4 *>(ra + kk * C::kAPitch + 4 * rr);
+                const int i = c0 + kk, j = r0 + rr;
+                const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    store_split1(ahi, alo, sw128_f32(rr + q, kk),
+                                 (i < T && j + q <= i) ? w[q] : 0.f);
             } else {
-                store_split4(ahi, alo, sw128_f32(f >> 3, 4 * (f & 7)), R.a[u]);
+                const int f = tid + kPvThreads * u, row = f >> 3, k4 = 4 * (f & 7);
+                float4 v = *reinterpret_cast<const float4 *>(ra + row * C::kAPitch + 4 * k4);
+                if (MODE == 0) {             // the causal mask (the map holds garbage above it)
+                    const int i = r0 + row, j = c0 + k4;
+                    v.x = j <= i ? v.x : 0.f;
+                    v.y = j + 1 <= i ? v.y : 0.f;
+                    v.z = j + 2 <= i ? v.z : 0.f;
+                    v.w = j + 3 <= i ? v.w : 0.f;
+                }
+                store_split4(ahi, alo, sw128_f32(row, k4), v);
             }
         }
 #pragma unroll
         for (int u = 0; u < C::kBU; ++u) {
-            const float4 v = R.x[u];
             if (MODE == 2) {
-                const int f = tid + kPvThreads * u;
-                const uint32_t off = sw128_f32(f >> 3, 4 * (f & 7));
+                const int f = tid + kPvThreads * u, row = f >> 3, k4 = 4 * (f & 7);
+                const float4 v = ld4(reinterpret_cast<const TX *>(rx + row * C::kXPitch) + k4);
+                const uint32_t off = sw128_f32(row, k4);
                 if (C::kXlo) store_split4(bhi, blo, off, v);
                 else *reinterpret_cast<float4 *>(bhi + off) = v;    // bf16 values are exact in TF32
             } else {                         // transposed: rows (channels) 4 tq_q + q, column tq_k
                 const int slot = warp + 8 * u, kk = tq_k(slot, lane), e = 4 * tq_q(slot, lane);
+                const float4 v = ld4(reinterpret_cast<const TX *>(rx + kk * C::kXPitch) + e);
                 const float w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -579,20 +604,29 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
     const uint32_t idesc = tc::idesc_tf32(kTile, C::N, false, false);
     int committed = 0;
     bool ok = true;
-    // one chunk: wait for its stage, convert from the registers, refill them
-    // with chunk n + 2, and (thread 0) issue the MMAs once everyone arrived
-    auto step = [&](int n, Regs &R) -> bool {
-        const int s = n % kMmStages;
-        const uint32_t use = (uint32_t)(n / kMmStages);
+    for (int p = 0; p < R && p < nch; ++p) issue_copies(p);
+    for (int n = 0; n < nch && ok; ++n) {
+        const int s = n % C::kStages;
+        const uint32_t use = (uint32_t)(n / C::kStages);
         uint8_t *st = base + s * C::kStage;
-        if (n >= kMmStages && !wait_or_abort(&mma_done[s], (use - 1) & 1, &abort_flag, err))
-            return false;
-        store_chunk(st, R);
-        if (n + 2 < nch) load_chunk(n + 2, R);
+        if (!wait_or_abort(&raw_full[n % R], (uint32_t)(n / R) & 1, &abort_flag, err)) {
+            ok = false;
+            break;
+        }
+        if (n >= C::kStages && !wait_or_abort(&mma_done[s], (use - 1) & 1, &abort_flag, err)) {
+            ok = false;
+            break;
+        }
+        convert(n, st);
         tc::fence_async_shared();
         tc::mbar_arrive(&a_full[s]);
+        // every thread has converted chunk n once a_full completes: its raw
+        // stage takes chunk n + R, and thread 0 issues chunk n's MMAs
+        if (!wait_or_abort(&a_full[s], use & 1, &abort_flag, err)) {
+            ok = false;
+            break;
+        }
         if (tid == 0) {
-            if (!wait_or_abort(&a_full[s], use & 1, &abort_flag, err)) return false;
             tc::tc_fence_after();
             const uint64_t dah = tc::sdesc_sw128(tc::smem_u32(st), 16, 1024);
             const uint64_t dal = tc::sdesc_sw128(tc::smem_u32(st + C::kATile), 16, 1024);
@@ -608,20 +642,15 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
             tc::mma_commit(&mma_done[s]);
             ++committed;
         }
-        return true;
-    };
-    load_chunk(0, set0);
-    if (nch > 1) load_chunk(1, set1);
-    for (int n = 0; n < nch && ok; n += 2) {
-        ok = step(n, set0);
-        if (ok && n + 1 < nch) ok = step(n + 1, set1);
+        if (n + R < nch) issue_copies(n + R);
     }
     const int last = nch - 1;
-    ok = ok && wait_or_abort(&mma_done[last % kMmStages], (uint32_t)(last / kMmStages) & 1,
+    ok = ok && wait_or_abort(&mma_done[last % C::kStages], (uint32_t)(last / C::kStages) & 1,
                              &abort_flag, err);
+    tc::cp_async_wait_all();                // no copy of this thread is still in flight
     if (tid == 0 && !ok && committed > 0)   // after an abort: the MMAs in flight finish first
-        tc::mbar_wait(&mma_done[(committed - 1) % kMmStages],
-                      (uint32_t)((committed - 1) / kMmStages) & 1, kBudget);
+        tc::mbar_wait(&mma_done[(committed - 1) % C::kStages],
+                      (uint32_t)((committed - 1) / C::kStages) & 1, kBudget);
     if (warp < 4 && __all_sync(0xffffffffu, ok)) {
         tc::tc_fence_after();
         const int i = r0 + 32 * warp + lane;
@@ -660,20 +689,13 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
                     *reinterpret_cast<float4 *>(srow + 4 * m) =
                         make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
                 __syncwarp();
-                if (vec) {
 #pragma unroll
-                    for (int rho = 0; rho < 8; ++rho) {
-                        const int rr = 4 * rho + (lane >> 3);
-                        const int ii = r0 + 32 * warp + rr, jj = jb + 4 * (lane & 7);
-                        const float4 t = *reinterpret_cast<const float4 *>(stage + rr * kStageStride +
-                                                                           4 * (lane & 7));
-                        if (ii < T && jj < T) *reinterpret_cast<float4 *>(mb + (size_t)ii * T + jj) = t;
-                    }
-                } else {
-                    for (int rr = 0; rr < 32; ++rr) {
-                        const int ii = r0 + 32 * warp + rr, jj = jb + lane;
-                        if (ii < T && jj < T) mb[(size_t)ii * T + jj] = stage[rr * kStageStride + lane];
-                    }
+                for (int rho = 0; rho < 8; ++rho) {
+                    const int rr = 4 * rho + (lane >> 3);
+                    const int ii = r0 + 32 * warp + rr, jj = jb + 4 * (lane & 7);
+                    const float4 t = *reinterpret_cast<const float4 *>(stage + rr * kStageStride +
+                                                                       4 * (lane & 7));
+                    if (ii < T && jj < T) *reinterpret_cast<float4 *>(mb + (size_t)ii * T + jj) = t;
                 }
                 __syncwarp();
             }
@@ -784,7 +806,10 @@ unsigned int chain_take_error(cudaStream_t st)
     return v;
 }
 
-bool mm_tf32_supported(const mta_shape &s) { return s.d == 64 || s.d == 128; }
+bool mm_tf32_supported(const mta_shape &s)
+{
+    return (s.d == 64 || s.d == 128) && s.T % 4 == 0;   // 16-byte map rows for cp.async
+}
 
 mta_status causal_mm_tf32(const mta_shape &s, bool trans, const float *map, const void *x,
                           bool x_io, float *out, float scale, cudaStream_t st)
