@@ -324,6 +324,41 @@ k_mix_softmax_bwd(float *__restrict__ m2, const float *__restrict__ p3,
     }
 }
 
+// Halo fill of the stencil kernels: tile[rr][cc] = src[r0 + rr][c0 + cc] for
+// rr < rows, cc < kLoadCols, zero where the row or column lies outside
+// [0, T) or the key lies past the query (c > r).  With 16-byte rows (T % 4 == 0)
+// and c0 = -LEFT (mod 4) the source is read in aligned 16-byte groups.
+template <int kLoadCols, int kStride, int LEFT>
+__device__ __forceinline__ void halo_fill(float *tile, const float *__restrict__ mb, int T,
+                                          int rows, int r0, int c0)
+{
+    if ((T & 3) == 0) {
+        constexpr int kOff = ((-LEFT) % 4 + 4) % 4;   // halo column 0 within its group
+        constexpr int NQ = (kOff + kLoadCols + 3) / 4;
+        const int cbase = c0 - kOff;
+        for (int idx = threadIdx.x; idx < rows * NQ; idx += blockDim.x) {
+            const int rr = idx / NQ, qq = idx % NQ;
+            const int r = r0 + rr, c = cbase + 4 * qq;
+            float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r >= 0 && r < T && c >= 0 && c < T && c <= r)
+                t = *reinterpret_cast<const float4 *>(mb + (size_t)r * T + c);
+            const float w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int cc = 4 * qq + e - kOff;
+                if (cc >= 0 && cc < kLoadCols) tile[rr * kStride + cc] = (c + e <= r) ? w[e] : 0.f;
+            }
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < rows * kLoadCols; idx += blockDim.x) {
+            const int rr = idx / kLoadCols, cc = idx % kLoadCols;
+            const int r = r0 + rr, c = c0 + cc;
+            tile[rr * kStride + cc] =
+                (r >= 0 && r < T && c >= 0 && c < T && c <= r) ? mb[(size_t)r * T + c] : 0.f;
+        }
+    }
+}
+
 // Adjoint of the Eq. (4) convolution with Mask_0 (the gradient of the raw
 // logits): dst[r][c] = sum_{i'<c_q} sum_{j'} theta[i'][j'] dC[r+i'][c+j'] for
 // c <= r, where dC is read as zero above the diagonal and outside [0,T)^2;
@@ -351,12 +386,7 @@ k_conv_adj(const float *__restrict__ src, float *__restrict__ dst, const float *
     const int tid = threadIdx.x;
     const int rows = kAdjRows + c_q - 1;
     const float *mb = src + bh * (size_t)T * T;
-    for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
-        const int rr = idx / kLoadCols, cc = idx % kLoadCols;
-        const int i = r0 + rr, j = c0 - R + cc;
-        tile[rr * kAdjStride + cc] =
-            (i < T && j >= 0 && j <= i) ? mb[(size_t)i * T + j] : 0.f;
-    }
+    halo_fill<kLoadCols, kAdjStride, R>(tile, mb, T, rows, r0, c0 - R);
     for (int idx = tid; idx < c_q * CKP; idx += 256) {
         const int ip = idx / CKP, jj = idx % CKP;
         th[idx] = jj < CK ? w_kq[((size_t)h * c_q + ip) * CK + jj] : 0.f;
@@ -437,12 +467,7 @@ k_dtheta(const float *__restrict__ dc, const float *__restrict__ a0, float *__re
     const int tid = threadIdx.x;
     const int rows = kAdjRows + c_q - 1;
     const float *mb = a0 + bh * (size_t)T * T;
-    for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
-        const int rr = idx / kLoadCols, cc = idx % kLoadCols;
-        const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
-        tile[rr * kAdjStride + cc] =
-            (r >= 0 && r < T && c >= 0 && c < T && c <= r) ? mb[(size_t)r * T + c] : 0.f;
-    }
+    halo_fill<kLoadCols, kAdjStride, L>(tile, mb, T, rows, i0 - (c_q - 1), j0 - L);
     __syncthreads();
     const int ro = tid % 32, cl = (tid / 32) * NC;
     const int warp = tid / 32, lane = tid % 32;

@@ -169,12 +169,34 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
         const float *mb = src + (kMulti ? b * H + (h / nin) * nin + hi : bh) * (size_t)T * T;
         const float *wk = w_kq + (kMulti ? (size_t)h * nin + hi : (size_t)h) * c_q * CK;
         if (hi > 0) __syncthreads();              // every thread is done with the last halo
-        for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
-            const int rr = idx / kLoadCols, cc = idx % kLoadCols;
-            const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
-            tile[rr * kConvStride + cc] =
-                (r >= 0 && r < T && c >= 0 && c < T && c <= r + band) ? mb[(size_t)r * T + c]
-                                                                      : 0.f;
+        if ((T & 3) == 0) {
+            // 16-byte loads of the aligned groups covering the halo columns;
+            // each element is kept where it lies in the halo and is live
+            constexpr int kOff = ((-L) % 4 + 4) % 4;   // halo column 0 within its group
+            constexpr int NQ = (kOff + kLoadCols + 3) / 4;
+            const int cbase = j0 - L - kOff;
+            for (int idx = tid; idx < rows * NQ; idx += 256) {
+                const int rr = idx / NQ, qq = idx % NQ;
+                const int r = i0 - (c_q - 1) + rr, c = cbase + 4 * qq;
+                float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (r >= 0 && r < T && c >= 0 && c < T && c <= r + band)
+                    t = *reinterpret_cast<const float4 *>(mb + (size_t)r * T + c);
+                const float w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int cc = 4 * qq + e - kOff;
+                    if (cc >= 0 && cc < kLoadCols)
+                        tile[rr * kConvStride + cc] = (c + e <= r + band) ? w[e] : 0.f;
+                }
+            }
+        } else {
+            for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
+                const int rr = idx / kLoadCols, cc = idx % kLoadCols;
+                const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
+                tile[rr * kConvStride + cc] =
+                    (r >= 0 && r < T && c >= 0 && c < T && c <= r + band) ? mb[(size_t)r * T + c]
+                                                                          : 0.f;
+            }
         }
         for (int idx = tid; idx < c_q * CKP; idx += 256) {
             const int ip = idx / CKP, jj = idx % CKP;
