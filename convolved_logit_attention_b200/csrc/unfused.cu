@@ -338,6 +338,15 @@ k_softmax_mix(const float *__restrict__ map1, float *__restrict__ dst,
 // dst^h[i][j] = sum_h' w_g[h][h'] src^h'[i][j] for j <= i.  The second head
 // mix of a repeated MTA convolution, applied to probabilities that the
 // post-softmax key-query conv has already filtered.
+constexpr float kLog2eF = 1.4426950408889634f;
+
+__device__ __forceinline__ float exp2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // The forward's S5 + S6 (mode 0) with the row held in registers, for
 // T <= 1024 * Q4 and T % 4 == 0: each thread loads its 16-byte groups of each
 // of the c_h heads' rows once (keys past i read as -inf), the c_h row maxima
@@ -394,6 +403,8 @@ k_softmax_mix_reg(const float *__restrict__ map1, float *__restrict__ dst,
         m[hh] = r;
     }
     __syncthreads();                              // red is read by every thread before reuse
+    // exp(x - m) as 2^((x - m) log2 e) with the hardware exp2 (ex2.approx, a
+    // couple of ulp): the kernel is issue-bound with a full-precision expf
 #pragma unroll
     for (int hh = 0; hh < CH; ++hh) {
         float sm = 0.f;
@@ -401,7 +412,7 @@ k_softmax_mix_reg(const float *__restrict__ map1, float *__restrict__ dst,
         for (int q = 0; q < Q4; ++q)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                v[hh][q][e] = expf(v[hh][q][e] - m[hh]);
+                v[hh][q][e] = exp2_approx((v[hh][q][e] - m[hh]) * kLog2eF);
                 sm += v[hh][q][e];
             }
         sm = warp_sum(sm);
