@@ -322,8 +322,8 @@ def time_mta(args, w, d, world, device):
 
     # The timed steps are plain public calls (mta_forward / mta_forward_unfused /
     # mta_forward_gated): events recorded between the kernels would add their
-    # own cost to the step.  A separate traced pass afterwards gives each
-    # kernel's time for the roofline.
+    # own cost to the step.  Traced steps just before and just after the timed
+    # region give each kernel's time for the roofline.
     def composed(events=None):
         mta.mta_forward_composed(d["q"], d["k"], d["v"], *(d[n] for n in WEIGHTS),
                                  gn_weight=d["gn_weight"], gn_bias=d["gn_bias"],
@@ -355,6 +355,16 @@ def time_mta(args, w, d, world, device):
         flush.zero_()
         step()
     mta.mta_sync_status(stream, device)
+    # per-kernel breakdown: traced steps bracketing the timed region, half just
+    # before it and half just after, so that their average sees the clock and
+    # power state the timed steps ran in (the gated call shares the kernels of
+    # mta_forward)
+    n_tr = min(args.steps, 10)
+    kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(n_tr)]
+    for s in range(n_tr // 2):
+        flush.zero_()
+        traced_step(kern_ev[s])
+    torch.cuda.synchronize(device)
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -370,10 +380,7 @@ def time_mta(args, w, d, world, device):
     barrier(world)
     mta.mta_sync_status(stream, device)
     total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
-    # per-kernel breakdown (the gated call shares the kernels of mta_forward)
-    n_tr = min(args.steps, 10)
-    kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk)] for _ in range(n_tr)]
-    for s in range(n_tr):
+    for s in range(n_tr // 2, n_tr):
         flush.zero_()
         traced_step(kern_ev[s])
     torch.cuda.synchronize(device)
@@ -398,8 +405,8 @@ def backward_flops(w):
 
 
 def time_backward(args, w, x, d, world, device):
-    """K timed mta_backward calls (L2 flushed before each), then a traced
-    pass for the per-kernel breakdown."""
+    """K timed mta_backward calls (L2 flushed before each), bracketed by traced
+    calls for the per-kernel breakdown."""
     import convolved_logit_attention_b200 as mta
     dt = torch.bfloat16 if w.io == "bf16" else torch.float32
     rng = np.random.default_rng(w.seed + 1000)
@@ -420,6 +427,13 @@ def time_backward(args, w, x, d, world, device):
         flush.zero_()
         step()
     mta.mta_sync_status(stream, device)
+    # traced calls bracketing the timed region (one before, the rest after)
+    n_tr = min(args.steps, 3)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
+           for _ in range(n_tr)]
+    flush.zero_()
+    step(kev[0])
+    torch.cuda.synchronize(device)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     sampler = ClockSampler(device.index if device.index is not None else 0)
@@ -435,10 +449,7 @@ def time_backward(args, w, x, d, world, device):
     barrier(world)
     mta.mta_sync_status(stream, device)
     total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    n_tr = min(args.steps, 3)
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
-           for _ in range(n_tr)]
-    for s in range(n_tr):
+    for s in range(1, n_tr):
         flush.zero_()
         step(kev[s])
     torch.cuda.synchronize(device)
