@@ -650,10 +650,16 @@ __device__ __forceinline__ bool wait_role(uint64_t *bar, uint32_t parity, volati
 }
 
 // Arrival on a barrier of the MMA-issuing CTA (rank 0 of a pair, or self).
+// Its only use publishes P~ (and a rescaled U): TMEM data whose stores the
+// arriving warp has waited for and fenced before the arrival, and which the
+// issuer reads only through MMAs it issues after an acquire wait on the
+// barrier and tcgen05.fence::after_thread_sync.  No generic-memory data rides
+// on it, so the pair form is a relaxed arrival: a release at cluster scope
+// held each softmax warp about 1500 cycles per key tile.
 template <bool PAIR>
 __device__ __forceinline__ void arrive_leader(uint64_t *bar)
 {
-    if constexpr (PAIR) tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(bar), 0));
+    if constexpr (PAIR) tc::mbar_arrive_cluster_relaxed(tc::mapa_shared(tc::smem_u32(bar), 0));
     else tc::mbar_arrive(bar);
 }
 

@@ -380,11 +380,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
     return r;
 }
 
-// Arrive on an mbarrier that may live in another CTA of the cluster, with
-// release semantics at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+// Arrive on an mbarrier that may live in another CTA of the cluster, with no
+// memory-ordering semantics of its own (relaxed, cluster scope).  It suits a
+// signal whose data are TMEM contents that the arriving thread has already
+// waited for (tcgen05.wait::st) and ordered with tcgen05.fence::before_thread_sync;
+// the release form makes the arriving warp wait about 1500 cycles on B200.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                  : "memory");
 }
 
