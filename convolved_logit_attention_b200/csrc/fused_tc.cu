@@ -144,13 +144,19 @@ __device__ float block_max(float m, float *red)
     return r;
 }
 
-// |x| of both halves of a bf16 pair, folded into a running max; a NaN or
-// infinite element makes the max +inf.
-__device__ __forceinline__ float absmax_bf2(float m, uint32_t v)
+// The largest |x| bit pattern of each bf16 half of v, folded into the two
+// halfword lanes of m (|x| orders like its bits with the sign cleared).
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t m, uint32_t v)
 {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
-    const float ax = fabsf(f.x), ay = fabsf(f.y);
-    return (ax <= 3.0e38f && ay <= 3.0e38f) ? fmaxf(m, fmaxf(ax, ay)) : INFINITY;  // NaN: false
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(v & 0x7fff7fffu));
+    return r;
+}
+// The float value of the larger lane; +inf when it is a NaN or infinity.
+__device__ __forceinline__ float bits_to_absmax(uint32_t m)
+{
+    const uint32_t top = max(m & 0xffffu, m >> 16);
+    return top >= 0x7f80u ? INFINITY : __uint_as_float(top << 16);
 }
 
 // The power-of-two exponent e >= 0 of a block's fp16 operand scale, from the
@@ -231,12 +237,12 @@ __device__ float rows_absmax(const __nv_bfloat16 *__restrict__ head, int r_lo, i
                              float *red)
 {
     const int lo = r_lo > 0 ? r_lo : 0, hi = r_hi < T ? r_hi : T;
-    float m = 0.f;
+    uint32_t mb = 0u;
     for (int idx = threadIdx.x; idx < (hi - lo) * (D / 8); idx += blockDim.x) {
         const uint4 v = *(const uint4 *)(head + (size_t)(lo + idx / (D / 8)) * D + 8 * (idx % (D / 8)));
-        m = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(m, v.x), v.y), v.z), v.w);
+        mb = absmax_bits(absmax_bits(absmax_bits(absmax_bits(mb, v.x), v.y), v.z), v.w);
     }
-    return block_max(m, red);
+    return block_max(bits_to_absmax(mb), red);
 }
 
 // Folded keys: one CTA per (128-key block, b*H + h), 256 threads.  The
@@ -297,9 +303,9 @@ __device__ __forceinline__ void fold_keys_block(int blk, int bh, const __nv_bflo
 // F[i - i'][delta] (frow0 is row i's F row; row i - i' lies i' rows of
 // stride fstride before it), delta = i' + RT - jj - e.  Every index is static
 // after unrolling, so terms outside 1 <= delta <= 14 are never emitted.
-template <int CK, int E0>
+template <int CK, int E0, bool EXACT>
 __device__ __forceinline__ void corr_terms(float (&acc)[4], const float *frow0, int fstride,
-                                           const float *thp, int c_q, int exact)
+                                           const float *thp, int c_q)
 {
     constexpr int RT = CK / 2;
 #pragma unroll
@@ -314,7 +320,7 @@ __device__ __forceinline__ void corr_terms(float (&acc)[4], const float *frow0, 
                 for (int e = 0; e < 4; ++e) {
                     const int delta = ip + RT - jj - (E0 + e);
                     if (delta >= 1 && delta <= kCorrW - 2) {
-                        const float f = (exact && delta <= ip) ? 0.f : frow[delta - 1];
+                        const float f = (EXACT && delta <= ip) ? 0.f : frow[delta - 1];
                         acc[e] = fmaf(t, f, acc[e]);
                     }
                 }
@@ -323,7 +329,7 @@ __device__ __forceinline__ void corr_terms(float (&acc)[4], const float *frow0, 
     }
 }
 
-// The rest of the prologue: one CTA per (64-row block, b*H + h), 160
+// The rest of the prologue: one CTA per (64-row block, b*H + h), 256
 // threads, three sections:
 //  (b) the block's query rows in the permuted atom order, converted to fp16.
 //  (c) future logits F[r][delta] = scale * q_r . k_{r+delta}, delta in
@@ -334,14 +340,15 @@ __device__ __forceinline__ void corr_terms(float (&acc)[4], const float *frow0, 
 //      the tap's own query row r, which Mask_0 of Eq. (5) removes.  With
 //      `exact` (the indicator of Eq. (4), which keeps a tap whenever its key
 //      is not past the output's query i) only the terms with delta > i',
-//      that is key r + delta > i, are removed.
-template <int D, int CK>
+//      that is key r + delta > i, are removed.  EXACT is that flag, a template
+//      parameter so that the common path carries no per-term select.
+template <int D, int CK, bool EXACT>
 __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloat16 *__restrict__ q,
                                                const __nv_bfloat16 *__restrict__ k,
                                                const float *__restrict__ w_kq,
                                                __half *__restrict__ qp, float *__restrict__ corr,
                                                int *__restrict__ qexp, int T, int Tp, int H,
-                                               int nqb, int c_q, int c_k, float scale, int exact)
+                                               int nqb, int c_q, int c_k, float scale)
 {
     constexpr int QR = kProQLo + kAuxRows;
     constexpr int RT = CK / 2;                 // the taps' padded centre
@@ -371,14 +378,18 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
     constexpr int CPR = D / 8;                 // 16-byte chunks per row
     __nv_bfloat16 *qsm = qk_sm;                // [QRP][RS]
     __nv_bfloat16 *ksm = qk_sm + QRP * RS;     // [KRP][RS]
-    for (int idx = tid; idx < (QRP + KRP) * CPR; idx += kProThreads) {
-        const int row = idx / CPR, c8 = idx % CPR;
-        const bool isq = row < QRP;
-        const int lr = isq ? row : row - QRP;
-        const int g = isq ? j0 - kProQLo + lr : j0 - (kProQLo - 1) + lr;
-        const bool in = (isq ? lr < QR : lr < KR) && g >= 0 && g < T;
-        const __nv_bfloat16 *src = (isq ? q : k) + head_off + (size_t)(in ? g : 0) * D + 8 * c8;
-        tc::cp_async16((isq ? qsm : ksm) + lr * RS + 8 * c8, src, in);
+    constexpr int RP = kProThreads / CPR;      // rows per pass of the CTA
+    static_assert(kProThreads % CPR == 0, "whole rows per pass");
+    const int c8 = tid % CPR;                  // the thread's 16-byte chunk of every row
+    for (int lr = tid / CPR; lr < QRP; lr += RP) {
+        const int g = j0 - kProQLo + lr;
+        const bool in = lr < QR && g >= 0 && g < T;
+        tc::cp_async16(qsm + lr * RS + 8 * c8, q + head_off + (size_t)(in ? g : 0) * D + 8 * c8, in);
+    }
+    for (int lr = tid / CPR; lr < KRP; lr += RP) {
+        const int g = j0 - (kProQLo - 1) + lr;
+        const bool in = lr < KR && g >= 0 && g < T;
+        tc::cp_async16(ksm + lr * RS + 8 * c8, k + head_off + (size_t)(in ? g : 0) * D + 8 * c8, in);
     }
     // Range of the 128-row block's permuted queries: both halves' CTAs take
     // the largest |q| over the rows [i0 - 7, i0 + 128), their own 71 rows from
@@ -388,25 +399,25 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
     const int i0 = qblk * kProRows;
     constexpr int NL = 64 * CPR / kProThreads;
     static_assert(64 * CPR % kProThreads == 0, "other-half rows per thread");
-    float mq = 0.f;
+    uint32_t mqb = 0u;
     {
         const int ro = half == 0 ? i0 + kAuxRows : i0 - kProQLo;   // the other half's rows
 #pragma unroll
         for (int u = 0; u < NL; ++u) {
-            const int idx = tid + u * kProThreads;
-            const int row = ro + idx / CPR, c8 = idx % CPR;
+            const int row = ro + tid / CPR + u * RP;
             if (row >= 0 && row < T) {
                 const uint4 v = *(const uint4 *)(q + head_off + (size_t)row * D + 8 * c8);
-                mq = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(mq, v.x), v.y), v.z), v.w);
+                mqb = absmax_bits(absmax_bits(absmax_bits(absmax_bits(mqb, v.x), v.y), v.z), v.w);
             }
         }
     }
     tc::cp_async_wait_all();
     __syncthreads();
-    for (int idx = tid; idx < QR * CPR; idx += kProThreads) {
-        const uint4 v = *(const uint4 *)(qsm + (idx / CPR) * RS + 8 * (idx % CPR));
-        mq = absmax_bf2(absmax_bf2(absmax_bf2(absmax_bf2(mq, v.x), v.y), v.z), v.w);
+    for (int lr = tid / CPR; lr < QR; lr += RP) {
+        const uint4 v = *(const uint4 *)(qsm + lr * RS + 8 * c8);
+        mqb = absmax_bits(absmax_bits(absmax_bits(absmax_bits(mqb, v.x), v.y), v.z), v.w);
     }
+    const float mq = bits_to_absmax(mqb);
     __shared__ float red[8];
     int eq = range_exponent(block_max(mq, red));
     if (eq != 0 && tid == 0 && half == 0) atomicOr(&g_fused_error, kErrRange);   // see the fold
@@ -421,8 +432,7 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
         const int NA = q_atoms(c_q);
         __half *dst = qp + ((size_t)bh * (Tp / kBM) + qblk) * (size_t)NA * 8 * D;
         bool range_ok = true;
-        for (int idx = tid; idx < NA * 4 * CPR; idx += kProThreads) {
-            const int rowh = idx / CPR, c8 = idx % CPR;
+        for (int rowh = tid / CPR; rowh < NA * 4; rowh += RP) {
             const int a = rowh / 4, sr = rowh % 4;                // atom, row within this half
             const int row = 8 * a + 4 * half + sr;                // row of the block's atom layout
             const int rq = kProQLo - (c_q - 1) + a + 16 * sr;    // copy row of q_i
@@ -430,13 +440,18 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
             const __nv_bfloat162 *bp = (const __nv_bfloat162 *)&in;
             uint4 outv;
             __half2 *hp = (__half2 *)&outv;
+            if (eq == 0) {                        // the block fits fp16 as it is
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float2 f = __bfloat1622float2(bp[u]);
-                f.x *= qsc;
-                f.y *= qsc;
-                range_ok &= fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
-                hp[u] = __floats2half2_rn(f.x, f.y);
+                for (int u = 0; u < 4; ++u) hp[u] = __float22half2_rn(__bfloat1622float2(bp[u]));
+            } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float2 f = __bfloat1622float2(bp[u]);
+                    f.x *= qsc;
+                    f.y *= qsc;
+                    range_ok &= fabsf(f.x) <= 65504.f && fabsf(f.y) <= 65504.f;
+                    hp[u] = __floats2half2_rn(f.x, f.y);
+                }
             }
             *(uint4 *)(dst + (size_t)row * D + 8 * c8) = outv;
         }
@@ -497,10 +512,10 @@ __device__ __forceinline__ void fold_aux_block(int blk, int bh, const __nv_bfloa
         const int ir = tid % kAuxRows, g = tid / kAuxRows;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         switch (g) {
-            case 0: corr_terms<CK, 0>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
-            case 1: corr_terms<CK, 4>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
-            case 2: corr_terms<CK, 8>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
-            default: corr_terms<CK, 12>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q, exact); break;
+            case 0: corr_terms<CK, 0, EXACT>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q); break;
+            case 1: corr_terms<CK, 4, EXACT>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q); break;
+            case 2: corr_terms<CK, 8, EXACT>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q); break;
+            default: corr_terms<CK, 12, EXACT>(acc, fs + (ir + kProQLo) * kFs, kFs, thp, c_q); break;
         }
         *(float4 *)(corr + ((size_t)bh * Tp + j0 + ir) * kCorrW + 4 * g) =
             make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -533,12 +548,12 @@ __device__ __forceinline__ void wait_prerequisites()
 // SM and each hides the other; it also keeps the q and k rows of a block in
 // L2 for the three CTAs that read them.  The dependent main kernel may be
 // scheduled as soon as every CTA of this grid has started.
-template <int D, int CK>
+template <int D, int CK, bool EXACT>
 __global__ void __launch_bounds__(kProThreads, 3)
 k_fold(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
        const float *__restrict__ w_kq, __half *__restrict__ kf, __half *__restrict__ qp,
        float *__restrict__ corr, int *__restrict__ sexp, int T, int Tp, int H, int nqb, int c_q,
-       int c_k, float scale, int exact)
+       int c_k, float scale)
 {
     launch_dependents();
     const int u = blockIdx.x / 3, role = blockIdx.x % 3;
@@ -547,8 +562,8 @@ k_fold(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
         fold_keys_block<D, CK>(blk, bh, k, w_kq, kf, sexp + (size_t)gridDim.x / 3, T, Tp, H, nqb,
                                c_q, c_k, scale);
     else
-        fold_aux_block<D, CK>(2 * blk + role / 2, bh, q, k, w_kq, qp, corr, sexp, T, Tp, H, nqb,
-                              c_q, c_k, scale, exact);
+        fold_aux_block<D, CK, EXACT>(2 * blk + role / 2, bh, q, k, w_kq, qp, corr, sexp, T, Tp, H,
+                                     nqb, c_q, c_k, scale);
 }
 
 // ------------------------------------------------------------ main kernel
@@ -1451,7 +1466,10 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
         if (!make_tmap_bf16(&mV, a.v, 3, dims, strides, box)) return MTA_ERR_CUDA;
     }
     auto main_kernel = k_mta_fused<D, CH, PAIR>;
-    auto fold = s.c_k == 11 ? k_fold<D, 11> : s.c_k == 3 ? k_fold<D, 3> : k_fold<D, 15>;
+    const bool ex = a.exact_mask != 0;
+    auto fold = s.c_k == 11 ? (ex ? k_fold<D, 11, true> : k_fold<D, 11, false>)
+              : s.c_k == 3  ? (ex ? k_fold<D, 3, true> : k_fold<D, 3, false>)
+                            : (ex ? k_fold<D, 15, true> : k_fold<D, 15, false>);
     const int pro_smem = (int)prologue_smem_bytes(D);
     if (cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
@@ -1462,7 +1480,7 @@ mta_status launch_fused_t(const mta_shape &s, const ForwardArgs &a, void *ws, cu
     tr.before(0, st);
     fold<<<dim3((unsigned)(3 * L.nqb * BH)), kProThreads, pro_smem, st>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, a.w_kq, kf, qp, corr, sexp, s.T, L.Tp,
-        s.H, L.nqb, s.c_q, s.c_k, scale, a.exact_mask ? 1 : 0);
+        s.H, L.nqb, s.c_q, s.c_k, scale);
     tr.after(0, st);
     // The main kernel and the GroupNorm kernel are launched with programmatic
     // stream serialisation: each may be scheduled while its predecessor still
