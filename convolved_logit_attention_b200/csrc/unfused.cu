@@ -23,6 +23,7 @@
 #include <math.h>
 
 #include "io.cuh"
+#include "tc_util.cuh"
 #include "mta_internal.h"
 
 namespace mta {
@@ -121,9 +122,13 @@ k_logits(const TQ *__restrict__ q, const TK *__restrict__ k, float *__restrict__
 
 // S3 (+S4): dst[bh][i][j] = sum_{i',j'} theta[i'][j'] src[i-i'][j-j'] for
 // j <= i (also the post-softmax conv of the probabilities).  The 32 x 128
-// output tile reads a (32 + c_q - 1)-row halo of src into shared memory;
-// reads outside [0,T) or above the diagonal (c > r) are the zeros of Mask_0
-// and of the zero padding.  With kExact (the exact indicator of Eq. (4))
+// output tile reads a (32 + c_q - 1)-row halo of src into shared memory
+// (with T a multiple of 4, as cp.async copies of the 16-byte groups that
+// hold it, so the halo starts at the group of key j0 - L and a thread's
+// segment starts kOff columns later); reads outside [0,T) or above the
+// diagonal (c > r) are the zeros of Mask_0 and of the zero padding: groups
+// outside are zero-filled by the copy, and in a tile whose halo reaches the
+// diagonal the keys past it are cleared after the copies land.  With kExact (the exact indicator of Eq. (4))
 // the halo keeps src[r][c] for c <= r + band, and each output row i zeroes
 // the keys c > i of the segments it reads: a tap (i', j') then adds
 // src[i-i'][j-j'] exactly when j - j' <= i.  With nin > 1 (the 3-D
@@ -144,11 +149,15 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
 {
     const int nin = kMulti ? nin_arg : 1;         // a compile-time 1 for the 2-D kernels
     constexpr int NC = kConvCols / 8;             // output columns per thread
-    constexpr int NV = (CK + NC - 1 + 3) / 4;     // float4 loads per row segment
     constexpr int CKP = (CK + 3) / 4 * 4;         // padded tap row
-    constexpr int kLoadCols = 7 * NC + 4 * NV;    // halo columns any thread reads
-    static_assert(kLoadCols <= kConvStride && kLoadCols >= kConvCols + CK - 1, "halo width");
     constexpr int L = (CK + 1) / 2 - 1;           // keys reached to the left
+    // With 16-byte copies the halo starts at the aligned group that holds key
+    // j0 - L: halo column x is key j0 - L - kOff + x
+    constexpr int kOff = ((-L) % 4 + 4) % 4;
+    constexpr int NV = (kOff + CK + NC - 1 + 3) / 4;   // float4 loads per row segment
+    constexpr int kLoadCols = 7 * NC + 4 * NV;    // halo columns any thread reads
+    static_assert(kLoadCols <= kConvStride && kLoadCols >= kOff + kConvCols + CK - 1, "halo width");
+    constexpr int NQ = kLoadCols / 4;             // 16-byte groups per halo row
     const int i0 = blockIdx.y * kConvRows, j0 = blockIdx.x * kConvCols;
     if (j0 > i0 + kConvRows - 1) return;          // tile entirely above the diagonal
     const size_t bh = blockIdx.z;
@@ -169,31 +178,32 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
         const float *mb = src + (kMulti ? b * H + (h / nin) * nin + hi : bh) * (size_t)T * T;
         const float *wk = w_kq + (kMulti ? (size_t)h * nin + hi : (size_t)h) * c_q * CK;
         if (hi > 0) __syncthreads();              // every thread is done with the last halo
+        const int cbase = j0 - L - kOff;          // key of halo column 0
         if ((T & 3) == 0) {
-            // 16-byte loads of the aligned groups covering the halo columns;
-            // each element is kept where it lies in the halo and is live
-            constexpr int kOff = ((-L) % 4 + 4) % 4;   // halo column 0 within its group
-            constexpr int NQ = (kOff + kLoadCols + 3) / 4;
-            const int cbase = j0 - L - kOff;
+            // cp.async copies of the 16-byte groups of the halo; a group is
+            // either inside [0, T) or outside it, and one outside (or starting
+            // past the band) is zero-filled
             for (int idx = tid; idx < rows * NQ; idx += 256) {
                 const int rr = idx / NQ, qq = idx % NQ;
                 const int r = i0 - (c_q - 1) + rr, c = cbase + 4 * qq;
-                float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r >= 0 && r < T && c >= 0 && c < T && c <= r + band)
-                    t = *reinterpret_cast<const float4 *>(mb + (size_t)r * T + c);
-                const float w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int cc = 4 * qq + e - kOff;
-                    if (cc >= 0 && cc < kLoadCols)
-                        tile[rr * kConvStride + cc] = (c + e <= r + band) ? w[e] : 0.f;
+                const bool in = r >= 0 && r < T && c >= 0 && c < T && c <= r + band;
+                tc::cp_async16(&tile[rr * kConvStride + 4 * qq], mb + (in ? (size_t)r * T + c : 0), in);
+            }
+            tc::cp_async_wait_all();
+            // keys past r + band inside a copied group must read zero (the map
+            // is not written there): only tiles whose halo reaches the band
+            if (cbase + kLoadCols - 1 > i0 - (c_q - 1) + band) {
+                __syncthreads();
+                for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
+                    const int rr = idx / kLoadCols, x = idx % kLoadCols;
+                    if (cbase + x > i0 - (c_q - 1) + rr + band) tile[rr * kConvStride + x] = 0.f;
                 }
             }
         } else {
             for (int idx = tid; idx < rows * kLoadCols; idx += 256) {
-                const int rr = idx / kLoadCols, cc = idx % kLoadCols;
-                const int r = i0 - (c_q - 1) + rr, c = j0 - L + cc;
-                tile[rr * kConvStride + cc] =
+                const int rr = idx / kLoadCols, x = idx % kLoadCols;
+                const int r = i0 - (c_q - 1) + rr, c = cbase + x;
+                tile[rr * kConvStride + x] =
                     (r >= 0 && r < T && c >= 0 && c < T && c <= r + band) ? mb[(size_t)r * T + c]
                                                                           : 0.f;
             }
@@ -213,7 +223,7 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
                 seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
             }
             if (kExact) {                         // the indicator: keys past query i read 0
-                const int kfirst = j0 - L + c0;   // key of seg[0]
+                const int kfirst = cbase + c0;    // key of seg[0]
 #pragma unroll
                 for (int v = 0; v < 4 * NV; ++v)
                     if (kfirst + v > i0 + ro) seg[v] = 0.f;
@@ -228,7 +238,7 @@ k_conv(const float *__restrict__ src, float *__restrict__ dst, const float *__re
 #pragma unroll
             for (int jj = 0; jj < CK; ++jj)
 #pragma unroll
-                for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[CK - 1 - jj + u], acc[u]);
+                for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[kOff + CK - 1 - jj + u], acc[u]);
         }
     }
     const int i = i0 + ro;
