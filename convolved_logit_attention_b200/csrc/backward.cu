@@ -32,6 +32,7 @@
 #include <stdint.h>
 
 #include "io.cuh"
+#include "tc_util.cuh"
 #include "mta_internal.h"
 
 namespace mta {
@@ -324,36 +325,43 @@ k_mix_softmax_bwd(float *__restrict__ m2, const float *__restrict__ p3,
     }
 }
 
-// Halo fill of the stencil kernels: tile[rr][cc] = src[r0 + rr][c0 + cc] for
-// rr < rows, cc < kLoadCols, zero where the row or column lies outside
-// [0, T) or the key lies past the query (c > r).  With 16-byte rows (T % 4 == 0)
-// and c0 = -LEFT (mod 4) the source is read in aligned 16-byte groups.
+// Halo fill of the stencil kernels.  The halo starts at the 16-byte group
+// that holds key c0 (kOff = -LEFT mod 4 columns before it, c0 = -LEFT
+// (mod 4)): tile[rr][x] = src[r0 + rr][c0 - kOff + x] for rr < rows,
+// x < kLoadCols, zero where the row or column lies outside [0, T) or the key
+// lies past the query (c > r).  With 16-byte rows (T % 4 == 0) every group
+// is one cp.async copy, zero-filled when it lies outside (a group is wholly
+// inside or outside [0, T)) or starts past the diagonal; in a tile whose
+// halo reaches the diagonal the keys past it are cleared once the copies have
+// landed.  The caller synchronises the CTA before reading the tile.
 template <int kLoadCols, int kStride, int LEFT>
 __device__ __forceinline__ void halo_fill(float *tile, const float *__restrict__ mb, int T,
                                           int rows, int r0, int c0)
 {
+    constexpr int kOff = ((-LEFT) % 4 + 4) % 4;
+    static_assert(kLoadCols % 4 == 0, "whole groups");
+    const int cbase = c0 - kOff;
     if ((T & 3) == 0) {
-        constexpr int kOff = ((-LEFT) % 4 + 4) % 4;   // halo column 0 within its group
-        constexpr int NQ = (kOff + kLoadCols + 3) / 4;
-        const int cbase = c0 - kOff;
+        constexpr int NQ = kLoadCols / 4;
         for (int idx = threadIdx.x; idx < rows * NQ; idx += blockDim.x) {
             const int rr = idx / NQ, qq = idx % NQ;
             const int r = r0 + rr, c = cbase + 4 * qq;
-            float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r >= 0 && r < T && c >= 0 && c < T && c <= r)
-                t = *reinterpret_cast<const float4 *>(mb + (size_t)r * T + c);
-            const float w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int cc = 4 * qq + e - kOff;
-                if (cc >= 0 && cc < kLoadCols) tile[rr * kStride + cc] = (c + e <= r) ? w[e] : 0.f;
+            const bool in = r >= 0 && r < T && c >= 0 && c < T && c <= r;
+            tc::cp_async16(&tile[rr * kStride + 4 * qq], mb + (in ? (size_t)r * T + c : 0), in);
+        }
+        tc::cp_async_wait_all();
+        if (cbase + kLoadCols - 1 > r0) {         // the halo reaches the diagonal
+            __syncthreads();
+            for (int idx = threadIdx.x; idx < rows * kLoadCols; idx += blockDim.x) {
+                const int rr = idx / kLoadCols, x = idx % kLoadCols;
+                if (cbase + x > r0 + rr) tile[rr * kStride + x] = 0.f;
             }
         }
     } else {
         for (int idx = threadIdx.x; idx < rows * kLoadCols; idx += blockDim.x) {
-            const int rr = idx / kLoadCols, cc = idx % kLoadCols;
-            const int r = r0 + rr, c = c0 + cc;
-            tile[rr * kStride + cc] =
+            const int rr = idx / kLoadCols, x = idx % kLoadCols;
+            const int r = r0 + rr, c = cbase + x;
+            tile[rr * kStride + x] =
                 (r >= 0 && r < T && c >= 0 && c < T && c <= r) ? mb[(size_t)r * T + c] : 0.f;
         }
     }
@@ -372,11 +380,12 @@ k_conv_adj(const float *__restrict__ src, float *__restrict__ dst, const float *
            int T, int H, int c_q)
 {
     constexpr int NC = kAdjCols / 8;
-    constexpr int NV = (CK + NC - 1 + 3) / 4;
+    constexpr int R = CK / 2;                     // keys reached to the left: j' >= -R
+    constexpr int kOff = ((-R) % 4 + 4) % 4;      // the halo starts kOff keys before c0 - R
+    constexpr int NV = (kOff + CK + NC - 1 + 3) / 4;
     constexpr int CKP = (CK + 3) / 4 * 4;
     constexpr int kLoadCols = 7 * NC + 4 * NV;
-    static_assert(kLoadCols <= kAdjStride && kLoadCols >= kAdjCols + CK - 1, "halo width");
-    constexpr int R = CK / 2;                     // keys reached to the left: j' >= -R
+    static_assert(kLoadCols <= kAdjStride && kLoadCols >= kOff + kAdjCols + CK - 1, "halo width");
     const int r0 = blockIdx.y * kAdjRows, c0 = blockIdx.x * kAdjCols;
     if (c0 > r0 + kAdjRows - 1) return;           // tile entirely above the diagonal
     const size_t bh = blockIdx.z;
@@ -415,7 +424,7 @@ k_conv_adj(const float *__restrict__ src, float *__restrict__ dst, const float *
 #pragma unroll
         for (int jj = 0; jj < CK; ++jj)
 #pragma unroll
-            for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[jj + u], acc[u]);
+            for (int u = 0; u < NC; ++u) acc[u] = fmaf(tr[jj], seg[kOff + jj + u], acc[u]);
     }
     const int r = r0 + ro;
     if (r >= T) return;
@@ -447,10 +456,11 @@ k_dtheta(const float *__restrict__ dc, const float *__restrict__ a0, float *__re
          int B, int T, int H, int c_q)
 {
     constexpr int NC = kAdjCols / 8;
-    constexpr int NV = (CK + NC - 1 + 3) / 4;
-    constexpr int kLoadCols = 7 * NC + 4 * NV;
-    static_assert(kLoadCols <= kAdjStride && kLoadCols >= kAdjCols + CK - 1, "halo width");
     constexpr int L = (CK + 1) / 2 - 1;           // keys reached to the left by A0 taps
+    constexpr int kOff = ((-L) % 4 + 4) % 4;      // the halo starts kOff keys before j0 - L
+    constexpr int NV = (kOff + CK + NC - 1 + 3) / 4;
+    constexpr int kLoadCols = 7 * NC + 4 * NV;
+    static_assert(kLoadCols <= kAdjStride && kLoadCols >= kOff + kAdjCols + CK - 1, "halo width");
     const int nct = gridDim.x, nrt = gridDim.y;
     const int tile_id = blockIdx.y * nct + blockIdx.x;
     const int ntiles = nct * nrt;
@@ -463,7 +473,7 @@ k_dtheta(const float *__restrict__ dc, const float *__restrict__ a0, float *__re
         return;
     }
     __shared__ __align__(16) float tile[(kAdjRows + kMaxCq - 1) * kAdjStride];
-    __shared__ float red[8][16];
+    __shared__ float red[2][8][16];           // double-buffered by query tap
     const int tid = threadIdx.x;
     const int rows = kAdjRows + c_q - 1;
     const float *mb = a0 + bh * (size_t)T * T;
@@ -497,22 +507,39 @@ k_dtheta(const float *__restrict__ dc, const float *__restrict__ a0, float *__re
             const float4 t = seg4[v];
             seg[4 * v] = t.x; seg[4 * v + 1] = t.y; seg[4 * v + 2] = t.z; seg[4 * v + 3] = t.w;
         }
-        float acc[CK];
+        float v[16];                              // the thread's partial of each key tap
 #pragma unroll
-        for (int jj = 0; jj < CK; ++jj) {
+        for (int jj = 0; jj < 16; ++jj) {
             float a = 0.f;
+            if (jj < CK) {
 #pragma unroll
-            for (int u = 0; u < NC; ++u) a = fmaf(g[u], seg[CK - 1 - jj + u], a);
-            acc[jj] = warp_sum(a);
+                for (int u = 0; u < NC; ++u) a = fmaf(g[u], seg[kOff + CK - 1 - jj + u], a);
+            }
+            v[jj] = a;
         }
-        __syncthreads();                          // red is free again
-        if (lane == 0)
+        // Sum the 16 partials over the warp in 16 shuffles: at each step a lane
+        // keeps the half of its values that its bit of the offset selects and
+        // adds its partner's copy of that half; then lanes l and l ^ 1 both
+        // hold the warp sum of tap k = (l >> 1) (a fixed order: deterministic).
 #pragma unroll
-            for (int jj = 0; jj < CK; ++jj) red[warp][jj] = acc[jj];
-        __syncthreads();
+        for (int o = 16, n = 16; o >= 2; o >>= 1, n >>= 1) {
+            const bool hi = (lane & o) != 0;
+#pragma unroll
+            for (int x = 0; x < n / 2; ++x) {
+                const float keep = hi ? v[x + n / 2] : v[x];
+                const float send = hi ? v[x] : v[x + n / 2];
+                v[x] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        const float tap = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+        const int k = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                      ((lane >> 1) & 1);
+        float (*rb)[16] = red[ip & 1];
+        if ((lane & 1) == 0) rb[warp][k] = tap;
+        __syncthreads();                          // red[ip & 1] is complete
         if (tid < CK) {
             float a = 0.f;
-            for (int w = 0; w < 8; ++w) a += red[w][tid];
+            for (int w = 0; w < 8; ++w) a += rb[w][tid];
             dst[ip * CK + tid] = a;
         }
     }
