@@ -591,12 +591,124 @@ BwdLayout bwd_layout(const mta_shape &s)
     return L;
 }
 
+// k_mix_softmax_bwd with the row held in registers (T % 4 == 0, T <= 1024 NJ):
+// thread t owns the 16-byte groups j = 4t + 1024n (n < NJ) of every head's
+// dA and P row, read once; the reductions and the dC write use those
+// registers.  Entries past the diagonal inside a group read as zero and are
+// written as zero (nothing reads the map above the diagonal).
+template <int CH, int NJ>
+__global__ void __launch_bounds__(256)
+k_mix_softmax_bwd_reg(float *__restrict__ m2, const float *__restrict__ p3,
+                      const float *__restrict__ w_head, float *__restrict__ pw, int B, int T, int H)
+{
+    const int i = blockIdx.x, bg = blockIdx.y;
+    const int G = H / CH;
+    const int b = bg / G, g = bg % G;
+    __shared__ float wsm[CH * CH];
+    __shared__ float red[8][CH * CH + CH];
+    for (int idx = threadIdx.x; idx < CH * CH; idx += 256) wsm[idx] = w_head[(size_t)g * CH * CH + idx];
+    const size_t bh0 = (size_t)b * H + (size_t)g * CH;
+    float da[NJ][CH][4], p[NJ][CH][4];
+#pragma unroll
+    for (int n = 0; n < NJ; ++n) {
+        const int j4 = 4 * threadIdx.x + 1024 * n;
+#pragma unroll
+        for (int hh = 0; hh < CH; ++hh) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), q = a;
+            if (j4 <= i) {
+                const size_t off = ((bh0 + hh) * T + i) * (size_t)T + j4;
+                a = *reinterpret_cast<const float4 *>(m2 + off);
+                q = *reinterpret_cast<const float4 *>(p3 + off);
+            }
+            const float av[4] = {a.x, a.y, a.z, a.w}, qv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool live = j4 + e <= i;
+                da[n][hh][e] = live ? av[e] : 0.f;
+                p[n][hh][e] = live ? qv[e] : 0.f;
+            }
+        }
+    }
+    __syncthreads();                              // wsm
+    float dw[CH * CH], dot[CH];
+#pragma unroll
+    for (int x = 0; x < CH * CH; ++x) dw[x] = 0.f;
+#pragma unroll
+    for (int x = 0; x < CH; ++x) dot[x] = 0.f;
+#pragma unroll
+    for (int n = 0; n < NJ; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int hi = 0; hi < CH; ++hi) {
+                float dp = 0.f;
+#pragma unroll
+                for (int ho = 0; ho < CH; ++ho) {
+                    dp = fmaf(wsm[ho * CH + hi], da[n][ho][e], dp);
+                    dw[ho * CH + hi] = fmaf(da[n][ho][e], p[n][hi][e], dw[ho * CH + hi]);
+                }
+                dot[hi] = fmaf(dp, p[n][hi][e], dot[hi]);
+            }
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+#pragma unroll
+    for (int x = 0; x < CH * CH; ++x) {
+        const float v = warp_sum(dw[x]);
+        if (lane == 0) red[warp][x] = v;
+    }
+#pragma unroll
+    for (int x = 0; x < CH; ++x) {
+        const float v = warp_sum(dot[x]);
+        if (lane == 0) red[warp][CH * CH + x] = v;
+    }
+    __syncthreads();
+    float rowdot[CH];
+#pragma unroll
+    for (int x = 0; x < CH; ++x) {
+        float a = 0.f;
+        for (int w = 0; w < 8; ++w) a += red[w][CH * CH + x];
+        rowdot[x] = a;
+    }
+    if (threadIdx.x < CH * CH) {
+        float a = 0.f;
+        for (int w = 0; w < 8; ++w) a += red[w][threadIdx.x];
+        pw[((size_t)g * B * T + (size_t)b * T + i) * (CH * CH) + threadIdx.x] = a;
+    }
+#pragma unroll
+    for (int n = 0; n < NJ; ++n) {
+        const int j4 = 4 * threadIdx.x + 1024 * n;
+        if (j4 > i) continue;
+#pragma unroll
+        for (int hi = 0; hi < CH; ++hi) {
+            float o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float dp = 0.f;
+#pragma unroll
+                for (int ho = 0; ho < CH; ++ho) dp = fmaf(wsm[ho * CH + hi], da[n][ho][e], dp);
+                o[e] = p[n][hi][e] * (dp - rowdot[hi]);
+            }
+            *reinterpret_cast<float4 *>(m2 + ((bh0 + hi) * T + i) * (size_t)T + j4) =
+                make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 template <int CH>
 void launch_mix_softmax_bwd(const mta_shape &s, float *m2, const float *p3, const float *w,
                             float *pw, cudaStream_t st)
 {
-    k_mix_softmax_bwd<CH><<<dim3(s.T, s.B * (s.H / CH)), 256, 0, st>>>(m2, p3, w, pw, s.B, s.T,
-                                                                        s.H);
+    const dim3 grid(s.T, s.B * (s.H / CH));
+    if constexpr (CH <= 2) {
+        if (s.T % 4 == 0 && s.T <= 4096) {       // the row fits the registers of one CTA
+            switch ((s.T + 1023) / 1024) {
+                case 1: k_mix_softmax_bwd_reg<CH, 1><<<grid, 256, 0, st>>>(m2, p3, w, pw, s.B, s.T, s.H); return;
+                case 2: k_mix_softmax_bwd_reg<CH, 2><<<grid, 256, 0, st>>>(m2, p3, w, pw, s.B, s.T, s.H); return;
+                case 3: k_mix_softmax_bwd_reg<CH, 3><<<grid, 256, 0, st>>>(m2, p3, w, pw, s.B, s.T, s.H); return;
+                default: k_mix_softmax_bwd_reg<CH, 4><<<grid, 256, 0, st>>>(m2, p3, w, pw, s.B, s.T, s.H); return;
+            }
+        }
+    }
+    k_mix_softmax_bwd<CH><<<grid, 256, 0, st>>>(m2, p3, w, pw, s.B, s.T, s.H);
 }
 
 mta_status mix_softmax_bwd(const mta_shape &s, float *m2, const float *p3, const float *w,
