@@ -196,8 +196,10 @@ k_pv_groupnorm_tc(const float *__restrict__ amap, const __grid_constant__ CUtens
     constexpr int kABytes = kTile * kPvKeys * 2;   // 16 KB: 128 rows x 64 keys, bf16
     constexpr int kVBytes = kPvKeys * D * 2;       // 64 keys x D, D/64 chunks of 8 KB
     constexpr int kStageBytes = kABytes + kVBytes;
-    const int i0 = blockIdx.x * kTile;
-    const int bh = blockIdx.y;
+    // the grid's slow index is the query block, longest first, so the
+    // scheduler deals out the causal rows longest-first across the heads
+    const int i0 = ((int)gridDim.y - 1 - (int)blockIdx.y) * kTile;
+    const int bh = blockIdx.x;
     const int b = bh / H, h = bh % H;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -472,7 +474,7 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
     constexpr int R = C::kRawStages;
     unsigned int *err = &g_chain_error;
     int r0, j0 = 0, c_begin, c_end;
-    const int bh = MODE == 2 ? blockIdx.z : blockIdx.y;
+    const int bh = MODE == 2 ? blockIdx.z : blockIdx.x;
     if (MODE == 2) {
         r0 = blockIdx.y * kTile;
         j0 = blockIdx.x * kTile;
@@ -480,8 +482,10 @@ k_mm_tf32(const float *__restrict__ asrc, const TX *__restrict__ x, float *__res
         c_begin = 0;
         c_end = D;
     } else {
-        // longest contraction first: MODE 0 grows with the row block, MODE 1 shrinks
-        const int blk = MODE == 0 ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+        // longest contraction first (the row block is the grid's slow index, so
+        // the order holds across the heads): MODE 0 grows with the row block,
+        // MODE 1 shrinks
+        const int blk = MODE == 0 ? (int)gridDim.y - 1 - (int)blockIdx.y : (int)blockIdx.y;
         r0 = blk * kTile;
         c_begin = MODE == 0 ? 0 : r0;
         c_end = MODE == 0 ? min(T, r0 + kTile) : T;
@@ -720,7 +724,7 @@ mta_status launch_mm_tf32_t(const mta_shape &s, const float *a, const void *xv, 
         return MTA_ERR_CUDA;
     const int nb = (s.T + kTile - 1) / kTile;
     const unsigned BH = (unsigned)(s.B * s.H);
-    const dim3 grid = MODE == 2 ? dim3(nb, nb, BH) : dim3(nb, BH);
+    const dim3 grid = MODE == 2 ? dim3(nb, nb, BH) : dim3(BH, nb);
     kern<<<grid, kPvThreads, C::kSmem, st>>>(a, (const TX *)xv, out, s.T, scale);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
 }
@@ -782,7 +786,7 @@ mta_status launch_pv_tc_t(const mta_shape &s, const float *amap, const ForwardAr
                              smem) != cudaSuccess)
         return MTA_ERR_CUDA;
     const int nb = (s.T + kTile - 1) / kTile;
-    k_pv_groupnorm_tc<D><<<dim3(nb, (unsigned)BH), kPvThreads, smem, st>>>(
+    k_pv_groupnorm_tc<D><<<dim3((unsigned)BH, nb), kPvThreads, smem, st>>>(
         amap, mV, a.gn_weight, a.gn_bias, a.depth_scale, a.gate, s.gn_eps,
         (__nv_bfloat16 *)a.out, s.T, s.H);
     return cudaGetLastError() == cudaSuccess ? MTA_OK : MTA_ERR_CUDA;
